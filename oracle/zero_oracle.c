@@ -1,0 +1,427 @@
+/*
+ * zero_oracle.c -- TEST INFRASTRUCTURE, not product code.
+ *
+ * Plain, slow, single-threaded CPU oracle for the ZeRO partitioned
+ * mixed-precision step. Only tests/, __graft_entry__.smoke() and bench.py's
+ * CPU-baseline / reference legs may load it; the CUDA library never does.
+ * Built with gcc -O2 -ffp-contract=off -fno-fast-math, so every float
+ * operation below is one IEEE binary32 operation rounded to nearest-even
+ * (x86-64 evaluates float expressions in float, FLT_EVAL_METHOD == 0) and no
+ * multiply-add is fused.
+ *
+ * Page references are given as [page] + bullet; the page keys are listed in
+ * zero_oracle.h.
+ */
+#include "zero_oracle.h"
+
+#include <math.h>
+#include <stdlib.h>
+#include <string.h>
+
+/* ======================================================================= */
+/* Half formats.                                                           */
+/*                                                                         */
+/* [inferensys-instr] mixed-precision bullets: parameters and gradients are */
+/* held in FP16 or BF16 and gradients are upcast to FP32 for the update;    */
+/* [inferensys-legal] "FP16 Master Weights" bullet: an FP32 master copy is  */
+/* kept. Both formats are decoded and encoded here from their definitions   */
+/* (sign, biased exponent, stored significand), value by value, with        */
+/* round-to-nearest-even, gradual underflow, and overflow to infinity.      */
+/* ======================================================================= */
+
+typedef struct {
+    int mant_bits; /* stored significand bits */
+    int exp_bits;
+    int bias;
+    int emin; /* smallest normal exponent (unbiased) */
+    int emax; /* largest normal exponent (unbiased) */
+} half_format;
+
+static const half_format FMT_FP16 = {10, 5, 15, -14, 15};
+static const half_format FMT_BF16 = {7, 8, 127, -126, 127};
+
+static const half_format* fmt_of(int32_t dtype) {
+    return dtype == ORACLE_FP16 ? &FMT_FP16 : &FMT_BF16;
+}
+
+float oracle_half_to_float(uint16_t h, int32_t dtype) {
+    const half_format* f = fmt_of(dtype);
+    int sign = (h >> 15) & 1;
+    int emask = (1 << f->exp_bits) - 1;
+    int e = (h >> f->mant_bits) & emask;
+    int frac = h & ((1 << f->mant_bits) - 1);
+    double val;
+    if (e == emask) {
+        if (frac != 0) return NAN;
+        val = INFINITY;
+    } else if (e == 0) {
+        /* subnormal: frac * 2^(emin - mant_bits) */
+        val = ldexp((double)frac, f->emin - f->mant_bits);
+    } else {
+        /* normal: (2^mant_bits + frac) * 2^(e - bias - mant_bits) */
+        val = ldexp((double)((1 << f->mant_bits) + frac), e - f->bias - f->mant_bits);
+    }
+    return (float)(sign ? -val : val); /* exact: every half value is a float */
+}
+
+uint16_t oracle_float_to_half(float x, int32_t dtype) {
+    const half_format* f = fmt_of(dtype);
+    uint16_t sign = signbit(x) ? (uint16_t)0x8000 : (uint16_t)0;
+    uint16_t exp_all = (uint16_t)(((1 << f->exp_bits) - 1) << f->mant_bits);
+    if (isnan(x)) /* quiet NaN: exponent all ones, top significand bit set */
+        return (uint16_t)(sign | exp_all | (1u << (f->mant_bits - 1)));
+    if (isinf(x)) return (uint16_t)(sign | exp_all);
+    double a = fabs((double)x);
+    if (a == 0.0) return sign;
+    int e2;
+    frexp(a, &e2);      /* a = fr * 2^e2, fr in [0.5, 1) */
+    int E = e2 - 1;     /* a in [2^E, 2^(E+1)) */
+    if (E < f->emin) E = f->emin; /* subnormal range shares the emin quantum */
+    double q = ldexp(1.0, E - f->mant_bits); /* spacing of the format at E */
+    double n = nearbyint(a / q); /* a / q is exact (power-of-two divisor); ties to even */
+    double one = ldexp(1.0, f->mant_bits);  /* 2^mant_bits */
+    if (n >= 2.0 * one) { /* rounding carried into the next binade */
+        n = n / 2.0;
+        E += 1;
+    }
+    if (E > f->emax) return (uint16_t)(sign | exp_all); /* overflow to infinity */
+    if (n < one) /* subnormal (only at E == emin): exponent field 0 */
+        return (uint16_t)(sign | (uint16_t)n);
+    return (uint16_t)(sign | (uint16_t)((E + f->bias) << f->mant_bits) |
+                      (uint16_t)(n - one));
+}
+
+void oracle_half_to_float_n(const uint16_t* h, float* out, int64_t n, int32_t dtype) {
+    for (int64_t i = 0; i < n; i++) out[i] = oracle_half_to_float(h[i], dtype);
+}
+
+void oracle_float_to_half_n(const float* x, uint16_t* out, int64_t n, int32_t dtype) {
+    for (int64_t i = 0; i < n; i++) out[i] = oracle_float_to_half(x[i], dtype);
+}
+
+/* ======================================================================= */
+/* Flat-buffer layout.                                                     */
+/*                                                                         */
+/* [inferensys-instr] ZeRO-1/2/3 mechanism bullets: each process owns and   */
+/* updates one partition. [inferensys-legal] "Bandwidth Optimization"       */
+/* bullet: small parameter groups are fused into larger transfers.          */
+/* [inferensys-legal] ZeRO-3 "All-Gather on Demand": a layer's parameters   */
+/* are gathered before that layer runs.                                     */
+/* Readings (the pages give no layout): tensors are laid out back to back in */
+/* list order, each starting at a multiple of `align` elements; L is the end */
+/* of the last tensor; the shard length S is the smallest multiple of 8 that */
+/* is at least ceil(L / R); T = R * S; rank r owns [r*S, (r+1)*S).           */
+/* Buckets are formed greedily over the tensors in reverse list order (the   */
+/* order gradients become ready): a tensor joins the open bucket while the   */
+/* bucket's raw element count stays <= bucket_elems, a tensor larger than    */
+/* that is a bucket of its own, and no tensor is ever split. A bucket's flat */
+/* range runs from its first tensor's offset to the next tensor's offset, so */
+/* alignment padding belongs to the bucket in front of it; the bucket that   */
+/* holds the last tensor also owns the tail padding [L, T). bucket_elems <=0 */
+/* means one bucket. Layers are given per tensor by non-decreasing ids that  */
+/* start at 0 and step by 0 or 1; layer l spans from its first tensor's      */
+/* offset to the next layer's first offset, and the last layer ends at L.    */
+/* ======================================================================= */
+
+static int64_t round_up(int64_t x, int64_t m) { return ((x + m - 1) / m) * m; }
+
+int32_t oracle_layout(const int64_t* numels, int64_t n, int32_t R, int32_t align,
+                      int64_t bucket_elems, const int32_t* layer_ids,
+                      int64_t* offsets, int64_t* sizes_out,
+                      int64_t* tensor_bucket, int64_t* bucket_lo, int64_t* bucket_hi,
+                      int64_t* layer_lo, int64_t* layer_hi) {
+    if (n < 1 || R < 1 || align < 1) return 1;
+    int64_t P = 0, cursor = 0;
+    for (int64_t k = 0; k < n; k++) {
+        if (numels[k] < 1) return 1;
+        offsets[k] = round_up(cursor, align);
+        cursor = offsets[k] + numels[k];
+        P += numels[k];
+    }
+    int64_t L = cursor;
+    int64_t S = round_up((L + R - 1) / R, 8);
+    int64_t T = (int64_t)R * S;
+
+    /* buckets: walk tensors from last to first */
+    int64_t nb = 0;
+    int64_t k = n - 1;
+    while (k >= 0) {
+        int64_t hi_k = k; /* highest tensor of this bucket */
+        int64_t total = numels[k];
+        int64_t lo_k = k;
+        if (bucket_elems > 0) {
+            while (lo_k - 1 >= 0 && total + numels[lo_k - 1] <= bucket_elems) {
+                lo_k -= 1;
+                total += numels[lo_k];
+            }
+        } else {
+            lo_k = 0;
+        }
+        bucket_lo[nb] = offsets[lo_k];
+        bucket_hi[nb] = (hi_k == n - 1) ? T : offsets[hi_k + 1];
+        for (int64_t j = lo_k; j <= hi_k; j++) tensor_bucket[j] = nb;
+        nb += 1;
+        k = lo_k - 1;
+    }
+    /* the first tensor sits at offset 0, so the buckets cover [0, T) */
+
+    /* layers */
+    int64_t nl = 0;
+    if (layer_ids == NULL) {
+        for (int64_t j = 0; j < n; j++) {
+            layer_lo[j] = offsets[j];
+            layer_hi[j] = (j + 1 < n) ? offsets[j + 1] : L;
+        }
+        nl = n;
+    } else {
+        if (layer_ids[0] != 0) return 1;
+        for (int64_t j = 1; j < n; j++) {
+            int32_t d = layer_ids[j] - layer_ids[j - 1];
+            if (d != 0 && d != 1) return 1;
+        }
+        for (int64_t j = 0; j < n; j++) {
+            if (j == 0 || layer_ids[j] != layer_ids[j - 1]) {
+                if (nl > 0) layer_hi[nl - 1] = offsets[j];
+                layer_lo[nl] = offsets[j];
+                nl += 1;
+            }
+        }
+        layer_hi[nl - 1] = L;
+    }
+
+    sizes_out[0] = P;
+    sizes_out[1] = L;
+    sizes_out[2] = S;
+    sizes_out[3] = T;
+    sizes_out[4] = nb;
+    sizes_out[5] = nl;
+    return 0;
+}
+
+/* ======================================================================= */
+/* Loss-scale state machine.                                               */
+/*                                                                         */
+/* [inferensys-legal] "Dynamic Loss Scaling" bullet and [inferensys-instr]  */
+/* "Loss Scaling" bullet: gradients are scaled up before backward, scaled   */
+/* down before the update, and the factor adjusts itself.                   */
+/* [inferensys-legal] "BFloat16 Compatibility": bf16 needs no loss scaling. */
+/* Readings: only DYNAMIC mode skips; an overflowing step leaves the model  */
+/* state and the step count alone, halves the scale (floor min_scale) and   */
+/* clears the clean-step counter; a clean step counts, and after            */
+/* growth_interval clean steps in a row the scale doubles and the counter   */
+/* clears. NONE and STATIC report the flag and never skip.                  */
+/* ======================================================================= */
+
+int32_t oracle_fsm_update(oracle_fsm* st, int32_t overflow) {
+    int32_t skip = 0;
+    st->last_overflow = overflow ? 1 : 0;
+    if (st->mode == ORACLE_SCALE_DYNAMIC) {
+        if (overflow) {
+            float s = st->scale * st->backoff_factor;
+            st->scale = (s < st->min_scale) ? st->min_scale : s;
+            st->good = 0;
+            skip = 1;
+        } else {
+            st->t += 1;
+            st->good += 1;
+            if (st->good >= st->growth_interval) {
+                st->scale = st->scale * st->growth_factor;
+                st->good = 0;
+            }
+        }
+    } else {
+        st->t += 1;
+    }
+    st->last_skipped = skip;
+    return skip;
+}
+
+/* ======================================================================= */
+/* Gradient reduction.                                                     */
+/*                                                                         */
+/* [inferensys-instr] "Baseline (DP)": one all-reduce after backward        */
+/* averages the gradients; ZeRO-2 "Communication": a reduce-scatter does    */
+/* the same averaging and leaves each partition on its owner.              */
+/* Reading: the R replicas are summed in fp32 in rank order 0..R-1 starting */
+/* from replica 0; the division by R is folded into the unscale multiply.   */
+/* ======================================================================= */
+
+int32_t oracle_allreduce_sum(int64_t P, int32_t R, int32_t dtype,
+                             const uint16_t* grads, float* acc) {
+    int32_t overflow = 0;
+    for (int64_t e = 0; e < P; e++) {
+        float s = oracle_half_to_float(grads[e], dtype);
+        for (int32_t r = 1; r < R; r++)
+            s = s + oracle_half_to_float(grads[(int64_t)r * P + e], dtype);
+        acc[e] = s;
+        if (!isfinite(s)) overflow = 1;
+    }
+    return overflow;
+}
+
+/* ======================================================================= */
+/* AdamW on the fp32 master copy, then the cast to the half parameter.     */
+/*                                                                         */
+/* [inferensys-genomic] memory breakdown: fp32 master weights, momentum and */
+/* variance (12 bytes per parameter) next to fp16 parameters and gradients; */
+/* [inferensys-instr] "Precision Management": the update runs in FP32 on    */
+/* upcast gradients and the weights are cast back to half for the next      */
+/* forward pass.                                                           */
+/* Reading (the pages print no Adam formula): Adam with Kingma-Ba bias      */
+/* correction and decoupled weight decay applied first, eps added after the */
+/* bias-corrected square root:                                             */
+/*   g = acc * inv,   inv = 1 / (R * scale)                                 */
+/*   p = p * (1 - lr*wd)                                                    */
+/*   m = b1*m + (1-b1)*g                                                    */
+/*   v = b2*v + (1-b2)*(g*g)                                                */
+/*   p = p - (lr / (1 - b1^t)) * (m / (sqrt(v) / sqrt(1 - b2^t) + eps))      */
+/*   param = half(p)                                                        */
+/* Scalar coefficients are formed in double and rounded once to float;      */
+/* every per-element operation is one rounded float operation.              */
+/* ======================================================================= */
+
+typedef struct {
+    float inv, dec, b1f, omb1, b2f, omb2, epsf, ss, bc2s;
+} adamw_coeffs;
+
+static adamw_coeffs make_coeffs(const oracle_adamw* hp, int32_t R, float scale, int64_t t) {
+    adamw_coeffs c;
+    c.inv = (float)(1.0 / ((double)R * (double)scale));
+    c.dec = (float)(1.0 - hp->lr * hp->weight_decay);
+    c.b1f = (float)hp->beta1;
+    c.omb1 = (float)(1.0 - hp->beta1);
+    c.b2f = (float)hp->beta2;
+    c.omb2 = (float)(1.0 - hp->beta2);
+    c.epsf = (float)hp->eps;
+    c.ss = (float)(hp->lr / (1.0 - pow(hp->beta1, (double)t)));
+    c.bc2s = (float)sqrt(1.0 - pow(hp->beta2, (double)t));
+    return c;
+}
+
+static void adamw_element(const adamw_coeffs* c, float acc, float* p, float* m, float* v,
+                          uint16_t* param, int32_t dtype) {
+    float g = acc * c->inv;
+    float pp = *p * c->dec;
+    float mm = c->b1f * *m + c->omb1 * g;
+    float vv = c->b2f * *v + c->omb2 * (g * g);
+    float den = sqrtf(vv) / c->bc2s + c->epsf;
+    pp = pp - c->ss * (mm / den);
+    *p = pp;
+    *m = mm;
+    *v = vv;
+    *param = oracle_float_to_half(pp, dtype);
+}
+
+static float effective_scale(const oracle_fsm* st) {
+    return st->mode == ORACLE_SCALE_NONE ? 1.0f : st->scale;
+}
+
+int32_t oracle_step(int64_t P, int32_t R, int32_t dtype, const uint16_t* grads,
+                    float* master, float* m, float* v, uint16_t* param,
+                    const oracle_adamw* hp, oracle_fsm* st) {
+    float* acc = (float*)malloc(sizeof(float) * (size_t)(P > 0 ? P : 1));
+    if (!acc) return -1;
+    int32_t overflow = oracle_allreduce_sum(P, R, dtype, grads, acc);
+    float scale = effective_scale(st);
+    adamw_coeffs c = make_coeffs(hp, R, scale, st->t + 1);
+
+    double nrm = 0.0;
+    for (int64_t e = 0; e < P; e++) {
+        float g = acc[e] * c.inv;
+        nrm += (double)g * (double)g;
+    }
+
+    int32_t skip = (st->mode == ORACLE_SCALE_DYNAMIC) && overflow;
+    if (!skip) {
+        for (int64_t e = 0; e < P; e++)
+            adamw_element(&c, acc[e], &master[e], &m[e], &v[e], &param[e], dtype);
+    }
+    oracle_fsm_update(st, overflow);
+    st->grad_norm_sq = nrm;
+    free(acc);
+    return skip;
+}
+
+/* ======================================================================= */
+/* The same step, partitioned.                                             */
+/*                                                                         */
+/* [mbrenndoerfer] introduction: every replica holds the same state and     */
+/* applies the same update, so partitioning removes redundancy without      */
+/* changing the result. [inferensys-instr] ZeRO-2: a reduce-scatter leaves  */
+/* each owner with its partition's reduced gradients, each owner updates    */
+/* only its partition; ZeRO-3 / ZeRO-1: the updated half parameters are     */
+/* all-gathered.                                                           */
+/* ======================================================================= */
+
+int32_t oracle_step_sharded(int64_t S, int32_t R, int32_t dtype, const uint16_t* grads,
+                            float* master, float* m, float* v, uint16_t* param,
+                            uint16_t* gathered, const oracle_adamw* hp, oracle_fsm* st) {
+    int64_t T = (int64_t)R * S;
+    float* acc = (float*)malloc(sizeof(float) * (size_t)(T > 0 ? T : 1));
+    if (!acc) return -1;
+
+    /* reduce-scatter: owner o receives the sum over ranks of [o*S, (o+1)*S) */
+    int32_t overflow = 0;
+    for (int32_t o = 0; o < R; o++) {
+        float* acc_o = acc + (int64_t)o * S;
+        int32_t flag_o = 0;
+        for (int64_t j = 0; j < S; j++) {
+            int64_t i = (int64_t)o * S + j;
+            float s = oracle_half_to_float(grads[i], dtype);
+            for (int32_t r = 1; r < R; r++)
+                s = s + oracle_half_to_float(grads[(int64_t)r * T + i], dtype);
+            acc_o[j] = s;
+            if (!isfinite(s)) flag_o = 1;
+        }
+        overflow |= flag_o; /* all-reduce (OR) of the owners' flags */
+    }
+
+    float scale = effective_scale(st);
+    adamw_coeffs c = make_coeffs(hp, R, scale, st->t + 1);
+    double nrm = 0.0;
+    for (int32_t o = 0; o < R; o++)
+        for (int64_t j = 0; j < S; j++) {
+            float g = acc[(int64_t)o * S + j] * c.inv;
+            nrm += (double)g * (double)g;
+        }
+
+    int32_t skip = (st->mode == ORACLE_SCALE_DYNAMIC) && overflow;
+    if (!skip) {
+        for (int32_t o = 0; o < R; o++) /* each owner updates its own shard */
+            for (int64_t j = 0; j < S; j++) {
+                int64_t i = (int64_t)o * S + j;
+                adamw_element(&c, acc[i], &master[i], &m[i], &v[i], &param[i], dtype);
+            }
+    }
+    /* all-gather of the half parameters */
+    for (int32_t o = 0; o < R; o++)
+        for (int64_t j = 0; j < S; j++) gathered[(int64_t)o * S + j] = param[(int64_t)o * S + j];
+
+    oracle_fsm_update(st, overflow);
+    st->grad_norm_sq = nrm;
+    free(acc);
+    return skip;
+}
+
+/* ======================================================================= */
+/* Model-state memory per rank.                                            */
+/*                                                                         */
+/* [inferensys-genomic] memory breakdown: 2 bytes of fp16 parameters, 2 of  */
+/* fp16 gradients and 12 of fp32 optimizer state (master, momentum,         */
+/* variance) per parameter. Stage bullets on every inferensys page: ZeRO-1  */
+/* shards the optimizer state, ZeRO-2 also the gradients, ZeRO-3 also the   */
+/* parameters.                                                             */
+/* ======================================================================= */
+
+double oracle_model_state_bytes(int32_t stage, double psi, double N) {
+    const double param_b = 2.0, grad_b = 2.0, optim_b = 12.0;
+    switch (stage) {
+        case 0: return (param_b + grad_b + optim_b) * psi;
+        case 1: return (param_b + grad_b) * psi + optim_b * psi / N;
+        case 2: return param_b * psi + (grad_b + optim_b) * psi / N;
+        case 3: return (param_b + grad_b + optim_b) * psi / N;
+        default: return -1.0;
+    }
+}
+
+double oracle_fp32_weight_bytes(double psi) { return 4.0 * psi; }
