@@ -1,0 +1,467 @@
+#!/usr/bin/env python
+"""Benchmark of the ZeRO data-parallel hot path on B200.
+
+One step = one pass of the whole path over one batch of synthetic
+gradients: the fused reduce-scatter + unscale + overflow check + AdamW +
+cast kernel over every shard (ping-pong state under dynamic loss scaling),
+the device-side loss-scale update, and the ZeRO-3 gather of every layer into
+a contiguous buffer. The partition plan is built once, before timing.
+
+Default workload: GPT-2-small-shaped parameter list (124,439,808 params,
+148 tensors), R=8 simulated ranks, fp16 gradients, dynamic loss scaling from
+2^16. Inputs (about 5.7 GB touched per step) are resident in HBM and larger
+than the 126 MB L2.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+With N > 1 (under torch.distributed.run) every rank runs its own independent
+replica of the workload (weak scaling, no collective on the data path); the
+time is the maximum over ranks. `--impl reference` times the CPU oracle on
+host cores on a bounded sample of the same workload.
+"""
+import argparse
+import datetime
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "params updated/sec per ZeRO step and achieved HBM GB/s vs B200 peak, 1 GPU"
+FALLBACK_HBM_GBS = 6650.0
+
+
+def parse_args(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.splitlines()[1])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="gpt2s")
+    ap.add_argument("--path", choices=["auto", "pingpong", "inplace", "twopass"], default="auto")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    return ap.parse_args(argv)
+
+
+# ---- distributed plumbing ---------------------------------------------------
+
+def dist_init():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import torch.distributed as dist
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=300))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(local)
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def aggregate(ms_local, units_local, world):
+    """Max of the per-rank times and sum of the per-rank units (whole job)."""
+    if world == 1:
+        return ms_local, units_local
+    import torch.distributed as dist
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([ms_local], dtype=torch.float64, device=dev)
+    u = torch.tensor([units_local], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    dist.all_reduce(u, op=dist.ReduceOp.SUM)
+    return float(t.item()), float(u.item())
+
+
+# ---- clocks -----------------------------------------------------------------
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons during a region."""
+
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index):
+        self.dev = device_index
+        self.proc = None
+        self.file = None
+
+    def start(self):
+        try:
+            self.file = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
+                 "-i", str(self.dev), "-lms", "100"], stdout=self.file, stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.file.flush()
+        rows = []
+        with open(self.file.name) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) == 9:
+                    rows.append(parts)
+        os.unlink(self.file.name)
+        if not rows:
+            return None
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({n for r in rows for n, v in zip(names, r[5:9]) if v == "Active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons, "samples": len(rows)}
+
+
+# ---- peaks and profile-derived traffic --------------------------------------
+
+def hbm_peak():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    except (OSError, KeyError, ValueError):
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def kernels_sha():
+    p = os.path.join(ROOT, "zero_partitioned_mixed_reduce_b200", "csrc", "kernels.cu")
+    with open(p, "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:16]
+
+
+def profiled_traffic(kernel, workload):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken
+    on the current kernel source; else None."""
+    p = os.path.join(ROOT, "profiles", "traffic.txt")
+    if not os.path.exists(p):
+        return None
+    sha = kernels_sha()
+    for line in open(p):
+        t = line.split()
+        if len(t) >= 4 and not line.startswith("#") and t[0] == kernel and t[1] == workload \
+                and t[2] == sha:
+            return float(t[3])
+    return None
+
+
+# ---- the workload -------------------------------------------------------------
+
+class Bench:
+    def __init__(self, name, path):
+        import zero_partitioned_mixed_reduce_b200 as Z
+        from zero_partitioned_mixed_reduce_b200 import synth
+        self.Z, self.synth = Z, synth
+        self.wl = wl = synth.workload(name)
+        self.R, self.dtype = wl["R"], wl["dtype"]
+        if path == "auto":
+            path = "pingpong" if wl["mode"] == synth.DYNAMIC else "inplace"
+        self.path = path
+        self.plan = Z.Plan(wl["numels"], wl["layer_ids"], wl["R"], wl["dtype"], 8,
+                           wl["bucket_elems"])
+        self.P, self.T, self.S, self.L = self.plan.P, self.plan.T, self.plan.S, self.plan.L
+        sets = 2 if path == "pingpong" else 1
+        self.state = Z.ShardedState(self.plan, sets=sets, with_acc=(path == "twopass"))
+        half = Z.state.HALF[wl["dtype"]]
+        # initial fp32 master ~N(0, 0.02) and its half copy, tensor by tensor
+        for k, (n, off) in enumerate(zip(wl["numels"], self.plan.offsets)):
+            x = synth.tensor_master(n, wl["index"], k, "cuda")
+            for kset in range(sets):
+                self._write(self.state.master[kset], off, x)
+                self._write(self.state.param[kset], off, x.to(half))
+        # one batch of gradients at the initial loss scale, padding zero
+        scale = wl["init_scale"] if wl["mode"] != synth.NONE else 1.0
+        self.grads = []
+        for r in range(self.R):
+            g = torch.zeros(self.T, dtype=half, device="cuda")
+            for k, (n, off) in enumerate(zip(wl["numels"], self.plan.offsets)):
+                g[off:off + n] = synth.tensor_grads(n, wl["dist"], wl["sigma"], scale,
+                                                    wl["dtype"], wl["index"], 1, r, k, "cuda")
+            self.grads.append(g)
+        self.ctx = Z.zero_ctx_create(self.plan.handle, wl["mode"], wl["init_scale"],
+                                     wl["interval"])
+        self.max_layer = max(hi - lo for lo, hi in self.plan.layers)
+        self.layer_buf = torch.empty(self.max_layer, dtype=half, device="cuda")
+        torch.cuda.synchronize()
+
+    def _write(self, shards, off, values):
+        n, pos, S = values.numel(), 0, self.S
+        while pos < n:
+            r, j = divmod(off + pos, S)
+            k = min(n - pos, S - j)
+            shards[r][j:j + k].copy_(values[pos:pos + k])
+            pos += k
+
+    def launches_per_step(self):
+        n = 1 + len(self.plan.layers)
+        if self.path == "twopass":
+            n += len(self.plan.buckets)
+        return n
+
+    def step_bytes(self):
+        """Algorithmic HBM bytes of one step (and of its dominant kernel)."""
+        R, T = self.R, self.T
+        if self.path == "twopass":
+            main = (2 * R + 4) * T + 30 * T
+        else:
+            main = (2 * R + 26) * T
+        return main + 4 * self.L, main
+
+    def step(self, stream, ev=None):
+        Z = self.Z
+        hp = self.wl["hp"]
+        if ev is not None:
+            ev[0].record(stream)
+        if self.path == "twopass":
+            for b in range(len(self.plan.buckets)):
+                Z.zero_reduce_scatter_bucket(self.ctx, b, self.grads, self.state.acc, stream)
+            Z.zero_step(self.ctx, hp, self.state.handle, None, stream)
+        else:
+            Z.zero_step(self.ctx, hp, self.state.handle, self.grads, stream)
+        if ev is not None:
+            ev[1].record(stream)
+        for l, (lo, hi) in enumerate(self.plan.layers):
+            Z.zero_gather_layer(self.ctx, l, self.state.handle, self.layer_buf, stream)
+
+    def loss_scale(self, stream):
+        return self.Z.zero_loss_scale(self.ctx, stream=stream)
+
+    def close(self):
+        self.Z.zero_ctx_destroy(self.ctx)
+
+
+def run_ours(args, world, rank, local):
+    if not torch.cuda.is_available():
+        print(json.dumps({"error": "no CUDA device: the benchmark has no CPU fallback"}))
+        sys.exit(1)
+    b = Bench(args.workload, args.path)
+    stream = torch.cuda.current_stream()
+    for _ in range(args.warmup):
+        b.step(stream)
+    torch.cuda.synchronize()
+    f0 = b.loss_scale(stream)
+    assert f0["last_overflow"] == 0, "warm-up steps must be clean"
+
+    K = args.steps
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(K)]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(local)
+    clocks.start()
+    barrier(world)
+    torch.cuda.synchronize()
+    start.record(stream)
+    for i in range(K):
+        b.step(stream, evs[i])
+    end.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    clk = clocks.stop()
+    ms_local = start.elapsed_time(end)
+    kern_ms = [e0.elapsed_time(e1) for e0, e1 in evs]
+    f1 = b.loss_scale(stream)
+    assert f1["last_overflow"] == 0 and f1["t"] == f0["t"] + K
+    ms, units = aggregate(ms_local, float(b.P) * K, world)
+
+    step_bytes, main_bytes = b.step_bytes()
+    peak, peak_src = hbm_peak()
+    kavg = statistics.mean(kern_ms)
+    achieved = main_bytes / (kavg * 1e-3) / 1e9
+    kernel_name = {"pingpong": "fused_step_kernel", "inplace": "fused_step_kernel",
+                   "twopass": "reduce_scatter+step_from_acc"}[b.path]
+    traffic = profiled_traffic(kernel_name, args.workload)
+    out = {
+        "metric": METRIC,
+        "value": units / (ms * 1e-3),
+        "unit": "params/s",
+        "n_gpus": world,
+        "steps": K,
+        "warmup": args.warmup,
+        "ms_per_step": ms / K,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "f32",
+        "data": "synthetic",
+        "hbm_gbs": step_bytes * K * world / (ms * 1e-3) / 1e9,
+        "hbm_frac_of_peak": step_bytes * K / (ms * 1e-3) / 1e9 / peak,
+        "config": {
+            "workload": f"{args.workload}: {len(b.wl['numels'])} tensors, P={b.P}, R={b.R} "
+                        f"simulated ranks, {'fp16' if b.dtype else 'bf16'} grads, "
+                        f"loss scale mode {b.wl['mode']}",
+            "R": b.R, "P": b.P, "T": b.T, "S": b.S, "n_layers": len(b.plan.layers),
+            "path": {"pingpong": "fused reduce-scatter+AdamW, ping-pong state",
+                     "inplace": "fused reduce-scatter+AdamW, in place",
+                     "twopass": "bucketed reduce-scatter, then AdamW from fp32 accumulators"}[b.path]
+                    + " + device loss-scale update + ZeRO-3 gather of every layer",
+            "bytes_per_step": step_bytes,
+            "l2": f"inputs larger than L2 ({step_bytes / 1e9:.1f} GB touched per step, L2 126 MB)",
+            "parallelism": "1 GPU" if world == 1 else f"{world} independent replicas",
+        },
+        "roofline": {"bound": "hbm", "kernel": kernel_name, "achieved": achieved, "peak": peak,
+                     "peak_source": f"{peak_src} hbm_gbs", "unit": "GB/s", "frac": achieved / peak,
+                     "traffic": traffic, "algorithmic_bytes_per_launch": main_bytes,
+                     "avg_launch_ms": kavg},
+        "clocks": clk,
+        "gpu_launches": K * b.launches_per_step(),
+    }
+    if not args.no_e2e:
+        out["e2e"] = e2e(b, args, stream, world)
+    b.close()
+    del b
+    torch.cuda.empty_cache()
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        out["cpu_baseline"] = cpu_baseline(args.workload)
+    if rank == 0:
+        print(json.dumps(out), flush=True)
+
+
+def e2e(b, args, stream, world):
+    """The same metric through the C ABI with host buffers: every step copies
+    its R gradient replicas from pinned host memory and reads the step's
+    result (the loss-scale state: overflow, skip, scale, grad norm) back."""
+    host = [g.cpu().pin_memory() for g in b.grads]
+    K = max(3, min(args.steps, 10))
+    for _ in range(2):
+        for r in range(b.R):
+            b.grads[r].copy_(host[r], non_blocking=True)
+        b.step(stream)
+        b.loss_scale(stream)
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    torch.cuda.synchronize()
+    start.record(stream)
+    for _ in range(K):
+        for r in range(b.R):
+            b.grads[r].copy_(host[r], non_blocking=True)
+        b.step(stream)
+        b.loss_scale(stream)  # synchronizes the stream: the result is on the host
+    end.record(stream)
+    torch.cuda.synchronize()
+    ms, units = aggregate(start.elapsed_time(end), float(b.P) * K, world)
+    return {"value": units / (ms * 1e-3), "unit": "params/s",
+            "h2d_bytes_per_step": sum(h.numel() * h.element_size() for h in host),
+            "d2h_bytes_per_step": 40, "steps": K}
+
+
+# ---- the CPU oracle as a baseline ----------------------------------------------
+
+def oracle_sample(name, target_s=10.0, max_elems=1 << 26):
+    """Time the oracle's step on a prefix sample of the workload, sized for
+    about target_s seconds. Returns (params/s, sample elements, seconds)."""
+    import oracle as O
+    from zero_partitioned_mixed_reduce_b200 import synth
+    wl = synth.workload(name)
+    R, dtype = wl["R"], wl["dtype"]
+    scale = wl["init_scale"] if wl["mode"] != synth.NONE else 1.0
+
+    def inputs(n):
+        numels, left = [], n
+        for k in wl["numels"]:
+            if left <= 0:
+                break
+            numels.append(min(k, left))
+            left -= numels[-1]
+        x = torch.cat([synth.tensor_master(c, wl["index"], k, "cpu") for k, c in enumerate(numels)])
+        g = np.stack([torch.cat([synth.tensor_grads(c, wl["dist"], wl["sigma"], scale, dtype,
+                                                    wl["index"], 1, r, k, "cpu")
+                                 for k, c in enumerate(numels)]).view(torch.int16).numpy()
+                      .view(np.uint16) for r in range(R)])
+        return O.State(x.numpy(), dtype), g
+
+    hp = O.AdamW(**{k: wl["hp"][k] for k in ("lr", "beta1", "beta2", "eps", "weight_decay")})
+    n = 1 << 18
+    st, g = inputs(n)
+    fsm = O.make_fsm(wl["mode"], scale=scale, interval=wl["interval"])
+    t = time.perf_counter()
+    O.step(st, g, hp, fsm)
+    rate = n / (time.perf_counter() - t)
+    n = int(min(max_elems, max(n, rate * target_s)))
+    st, g = inputs(n)
+    fsm = O.make_fsm(wl["mode"], scale=scale, interval=wl["interval"])
+    t = time.perf_counter()
+    O.step(st, g, hp, fsm)
+    dt = time.perf_counter() - t
+    return n / dt, n, dt, (st, g, hp, fsm)
+
+
+def cpu_baseline(name):
+    rate, n, dt, _ = oracle_sample(name)
+    return {"value": rate, "unit": "params/s", "cores": 1, "kind": "oracle",
+            "sample": f"one step of the first {n} params of {name} (all R replicas), "
+                      f"{dt:.1f} s single-threaded"}
+
+
+def run_reference(args, world, rank):
+    """The oracle on host cores: each step a bounded prefix sample."""
+    if rank != 0:
+        return
+    import oracle as O
+    rate, n, dt, (st, g, hp, fsm) = oracle_sample(args.workload, target_s=1.0,
+                                                  max_elems=1 << 22)
+    for _ in range(args.warmup):
+        O.step(st, g, hp, fsm)
+    t = time.perf_counter()
+    for _ in range(args.steps):
+        O.step(st, g, hp, fsm)
+    sec = time.perf_counter() - t
+    value = n * args.steps / sec
+    from zero_partitioned_mixed_reduce_b200 import synth
+    wl = synth.workload(args.workload)
+    out = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "params/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": sec * 1e3 / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "config": {"workload": f"{args.workload}: {len(wl['numels'])} tensors, "
+                               f"P={sum(wl['numels'])}, R={wl['R']} simulated ranks",
+                   "sample_params_per_step": n},
+        "cpu_baseline": {"value": value, "unit": "params/s", "cores": 1, "kind": "oracle",
+                         "sample": f"each step the first {n} params of {args.workload}"},
+        "e2e": {"value": value, "unit": "params/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(out), flush=True)
+
+
+def main(argv=None):
+    args = parse_args(argv)
+    world, rank, local = dist_init()
+    try:
+        if args.impl == "reference":
+            run_reference(args, world, rank)
+        else:
+            run_ours(args, world, rank, local)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,316 @@
+/*
+ * zero_b200.h -- C ABI of libzero_b200.so: the data-parallel hot path of ZeRO
+ * (partitioned mixed-precision AdamW over a flat, sharded model state) on one
+ * NVIDIA B200 (sm_100a). R data-parallel ranks are simulated as R gradient
+ * buffers and R state shards in the HBM of one GPU.
+ *
+ * Sources are four web pages titled "ZeRO Optimization":
+ *   [legal]    inferensys glossary, domain-specific legal pre-training
+ *   [instr]    inferensys glossary, instruction-tuning methodologies
+ *   [intro]    mbrenndoerfer, "ZeRO Optimization: Optimizer, Gradient, and
+ *              Parameter Partitioning", introduction
+ *   [genomic]  inferensys glossary, genomic MLOps
+ * Each entry point cites the passage that defines its operation.
+ *
+ * Conventions for every call:
+ *  - Every call returns a zero_status; nothing throws across the ABI. On an
+ *    error, zero_last_error() gives a message for the calling thread.
+ *  - Device pointers are owned by the caller (for example allocated by
+ *    PyTorch) and must stay valid until the work enqueued on the stream has
+ *    finished. Half buffers (gradients, parameters, gather output) must be
+ *    16-byte aligned; fp32 buffers (master, m, v, accumulators) must be
+ *    32-byte aligned. A misaligned pointer returns ZERO_ERR_ALIGN and
+ *    nothing is launched.
+ *  - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *    stream). Every GPU call is asynchronous on that stream, except where a
+ *    call says it synchronizes. A CUDA error raised by earlier asynchronous
+ *    work surfaces as ZERO_ERR_CUDA on a later call or on zero_sync.
+ *  - A context is bound to the CUDA device that was current when it was
+ *    created; calls with another device current return ZERO_ERR_INVALID_ARG.
+ *  - The library owns only the plan (host memory) and the context's small
+ *    device scratch (loss-scale state, overflow flag, per-block norm
+ *    partials, bias-correction power table).
+ */
+#ifndef ZERO_B200_H
+#define ZERO_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define ZERO_MAX_RANKS 64
+
+typedef enum {
+    ZERO_OK = 0,
+    ZERO_ERR_INVALID_ARG = 1, /* a bad argument value (null, out-of-range config, ...) */
+    ZERO_ERR_ALIGN = 2,       /* a device pointer violates the alignment rule above */
+    ZERO_ERR_CUDA = 3,        /* a CUDA runtime error (launch, async fault, no device) */
+    ZERO_ERR_OOM = 4,         /* host or device allocation failed */
+    ZERO_ERR_RANGE = 5,       /* a bucket / layer / tensor index or a size out of range */
+    ZERO_ERR_TIMEOUT = 6,     /* reserved: a bounded device wait gave up */
+    ZERO_ERR_STATE = 7        /* the call does not fit the context's state */
+} zero_status;
+
+typedef enum { ZERO_BF16 = 0, ZERO_FP16 = 1 } zero_dtype;
+
+typedef enum {
+    ZERO_SCALE_NONE = 0,    /* no loss scaling (bf16; [legal] "BFloat16 Compatibility") */
+    ZERO_SCALE_STATIC = 1,  /* fixed scale, never skips */
+    ZERO_SCALE_DYNAMIC = 2  /* skip + back off on overflow, grow after clean steps */
+} zero_scale_mode;
+
+typedef struct zero_plan_s zero_plan_t;
+typedef struct zero_ctx_s zero_ctx_t;
+
+/* ------------------------------------------------------------------------ */
+/* Partition plan (host only; no GPU needed).                               */
+/* ------------------------------------------------------------------------ */
+
+typedef struct {
+    int32_t R;            /* simulated data-parallel ranks, 1..ZERO_MAX_RANKS */
+    int32_t dtype;        /* zero_dtype of gradients and parameters */
+    int32_t tensor_align; /* each tensor starts at a multiple of this many
+                             elements, 1..4096 (8 = 16 bytes of half) */
+    int32_t reserved;     /* must be 0 */
+    int64_t bucket_elems; /* reduce-scatter bucket capacity in raw elements;
+                             <= 0 means one bucket for the whole model */
+} zero_plan_config;
+
+typedef struct {
+    int64_t P;         /* raw parameter count (sum of numels) */
+    int64_t L;         /* flat length: end of the last tensor */
+    int64_t S;         /* shard length, a multiple of 8 */
+    int64_t T;         /* padded total R*S */
+    int64_t n_tensors, n_buckets, n_layers;
+    int32_t R, dtype, tensor_align, reserved;
+} zero_plan_info;
+
+/*
+ * zero_plan -- lay n parameter tensors into one flat buffer cut into R equal
+ * shards, and group them into reduce-scatter buckets and gather layers.
+ *
+ * Defines: [instr] ZeRO-1/2/3 "Mechanism" bullets (each data-parallel
+ * process owns and updates one partition of optimizer state, gradients and
+ * parameters); [legal] "Bandwidth Optimization" bullet (small parameter
+ * groups are fused to cope with irregular transformer tensor sizes);
+ * [legal] ZeRO-3 "All-Gather on Demand" bullet (parameters are gathered per
+ * layer before the layer runs).
+ *
+ * Layout: tensors are placed back to back in list order, tensor k at the
+ * smallest multiple of tensor_align at or after the end of tensor k-1
+ * (tensor 0 at 0); L is the end of the last tensor; S is the smallest
+ * multiple of 8 that is >= ceil(L/R); T = R*S; rank r owns flat range
+ * [r*S, (r+1)*S). Padding elements carry zero gradients and stay zero.
+ * Buckets: greedy over tensors in reverse list order (the order gradients
+ * become ready); a tensor joins the open bucket while the bucket's raw
+ * element count stays <= bucket_elems; a larger tensor forms its own bucket;
+ * tensors are never split. Bucket 0 holds the last tensor. A bucket's flat
+ * range runs from its first tensor's offset to the next tensor's offset (the
+ * bucket holding the last tensor ends at T), so the buckets partition
+ * [0, T). Layers: layer_ids[k] gives tensor k's layer; ids start at 0 and
+ * step by 0 or +1; layer l spans its first tensor's offset up to the next
+ * layer's first offset, and the last layer ends at L. layer_ids == NULL makes
+ * every tensor its own layer.
+ *
+ * numels: n counts (each >= 1), host memory, read during the call only.
+ * Errors: ZERO_ERR_INVALID_ARG for n < 1, a count < 1, R or tensor_align out
+ * of range, a bad dtype or layer id sequence; ZERO_ERR_RANGE if T/8 does not
+ * fit in 31 bits; ZERO_ERR_OOM. On success *out owns a plan that the caller
+ * frees with zero_plan_destroy.
+ */
+zero_status zero_plan(const int64_t* numels, const int32_t* layer_ids, int64_t n,
+                      const zero_plan_config* cfg, zero_plan_t** out);
+void zero_plan_destroy(zero_plan_t* plan);
+
+zero_status zero_plan_get_info(const zero_plan_t* plan, zero_plan_info* info);
+/* Tensor k: flat offset, numel, owning bucket and layer (any output may be NULL). */
+zero_status zero_plan_tensor(const zero_plan_t* plan, int64_t k, int64_t* offset, int64_t* numel,
+                             int64_t* bucket, int64_t* layer);
+/* Bucket b's flat range [lo, hi). */
+zero_status zero_plan_bucket(const zero_plan_t* plan, int64_t b, int64_t* lo, int64_t* hi);
+/* Layer l's flat range [lo, hi). */
+zero_status zero_plan_layer(const zero_plan_t* plan, int64_t l, int64_t* lo, int64_t* hi);
+
+/*
+ * zero_plan_memory -- model-state bytes one rank holds under this plan at a
+ * given ZeRO stage (0 = plain data parallel, 1, 2, 3), counting 2 bytes of
+ * half parameters, 2 of half gradients and 12 of fp32 master + momentum +
+ * variance per element of the padded layout: stage 0: 16T; stage 1:
+ * 4T + 12S; stage 2: 2T + 14S; stage 3: 16S.
+ * Defines: [genomic] memory-breakdown bullets (2 + 2 + 12 bytes per
+ * parameter) and the stage bullets of [legal] and [genomic] (ZeRO-1 shards
+ * the optimizer state, ZeRO-2 adds gradients, ZeRO-3 adds parameters).
+ * Errors: ZERO_ERR_INVALID_ARG for another stage or a NULL output.
+ */
+zero_status zero_plan_memory(const zero_plan_t* plan, int32_t stage, int64_t* bytes_per_rank);
+
+/* ------------------------------------------------------------------------ */
+/* Context: device scratch and the loss-scale state.                        */
+/* ------------------------------------------------------------------------ */
+
+typedef struct {
+    int32_t mode;            /* zero_scale_mode */
+    float init_scale;        /* starting scale (STATIC, DYNAMIC); > 0, power of two advised */
+    int64_t growth_interval; /* DYNAMIC: clean steps in a row before growth, >= 1 */
+    float growth_factor;     /* DYNAMIC: multiplier on growth, > 1 (2) */
+    float backoff_factor;    /* DYNAMIC: multiplier on overflow, in (0, 1) (0.5) */
+    float min_scale;         /* DYNAMIC: floor of the scale, > 0 (1) */
+    int32_t reserved;        /* must be 0 */
+} zero_loss_scale_config;
+
+/*
+ * zero_ctx_create -- bind a context to the current CUDA device and allocate
+ * its device scratch. The plan's layout is copied; the plan may be destroyed
+ * afterwards. Defines the loss-scale state of [legal] "Dynamic Loss
+ * Scaling" and [instr] "Loss Scaling": the scale starts at init_scale (1 in
+ * NONE mode), the step count t at 0.
+ * Errors: ZERO_ERR_INVALID_ARG (bad config), ZERO_ERR_CUDA (no device),
+ * ZERO_ERR_OOM. Free with zero_ctx_destroy (which synchronizes the device).
+ */
+zero_status zero_ctx_create(const zero_plan_t* plan, const zero_loss_scale_config* cfg,
+                            zero_ctx_t** out);
+zero_status zero_ctx_destroy(zero_ctx_t* ctx);
+
+/* ------------------------------------------------------------------------ */
+/* The step.                                                                */
+/* ------------------------------------------------------------------------ */
+
+typedef struct {
+    double lr, beta1, beta2, eps, weight_decay;
+} zero_adamw;
+
+/*
+ * Sharded model state. Each array holds R device pointers (host memory, read
+ * during the call only); entry r points at rank r's shard of S elements.
+ * master/m/v are fp32, param is the plan's half dtype. Set 0 is required;
+ * set 1 (all four arrays non-NULL, or all NULL) enables ping-pong steps:
+ * the fused step then reads set `cur` and writes set 1-cur, and flips `cur`
+ * only if the step is applied, so a skipped step costs no extra traffic.
+ * acc holds R fp32 accumulators of S elements for the two-pass path (may be
+ * NULL for the fused path and for gathers).
+ */
+typedef struct {
+    float* const* master[2];
+    float* const* m[2];
+    float* const* v[2];
+    void* const* param[2];
+    float* const* acc;
+} zero_state;
+
+/*
+ * zero_reduce_scatter_bucket -- sum the R gradient replicas of one bucket
+ * into the owning ranks' fp32 accumulators:
+ *   acc[o][i - o*S] = ((f32(g_0[i]) + f32(g_1[i])) + ...) + f32(g_{R-1}[i])
+ * for every flat index i of the bucket, o = i / S; the overflow flag of the
+ * current step is OR-ed with "some sum is inf or NaN". Accumulators are
+ * overwritten, not added to. bucket = -1 reduces the whole range [0, T) in
+ * one launch.
+ * Defines: [legal] "Reduce-Scatter" bullet and [instr] ZeRO-2
+ * "Communication" bullet (a reduce-scatter aggregates and averages the
+ * gradients and leaves each partition on its owner, replacing DP's
+ * all-reduce); the division by R is folded into the step's unscale.
+ * grads: R device pointers to full replicas of T half elements in the plan's
+ * flat layout (zero in padding). acc: R device pointers, S fp32 each.
+ * Errors: ZERO_ERR_RANGE (bucket), ZERO_ERR_INVALID_ARG, ZERO_ERR_ALIGN,
+ * ZERO_ERR_CUDA.
+ */
+zero_status zero_reduce_scatter_bucket(zero_ctx_t* ctx, int64_t bucket, const void* const* grads,
+                                       float* const* acc, void* stream);
+
+/*
+ * zero_step -- one optimizer step on every shard, then the loss-scale update.
+ *
+ * With g = acc * (1 / (R * scale)) the unscaled, averaged gradient (scale = 1
+ * in NONE mode), t the step count after this step, and every operation one
+ * rounded fp32 operation without fused multiply-add:
+ *   p = p * (1 - lr*wd)
+ *   m = b1*m + (1-b1)*g
+ *   v = b2*v + (1-b2)*(g*g)
+ *   p = p - (lr / (1 - b1^t)) * (m / (sqrt(v) / sqrt(1 - b2^t) + eps))
+ *   param = round-to-nearest-even half(p)
+ * Scalar coefficients are formed in double and rounded once to float. The
+ * step is skipped (state untouched, t unchanged) only in DYNAMIC mode when
+ * the step's overflow flag is set. The loss-scale update then runs on the
+ * device without a host round trip: DYNAMIC overflow -> scale = max(scale *
+ * backoff, min_scale), clean count 0; DYNAMIC clean -> t += 1, count += 1,
+ * and at growth_interval the scale grows and the count clears; NONE/STATIC
+ * -> t += 1. The squared L2 norm of g is recorded (diagnostic).
+ *
+ * Defines: [instr] ZeRO-1 "Mechanism" (each process updates only its
+ * partition of the Adam state), [genomic] memory breakdown (fp32 master,
+ * momentum and variance), [instr] "Precision Management" (fp32 update on
+ * upcast gradients, weights cast back to half), [legal] "Dynamic Loss
+ * Scaling" and [instr] "Loss Scaling" (unscale before the update; the scale
+ * adjusts itself). The Adam formula itself is not printed on the pages; the
+ * one above is bias-corrected Adam with decoupled weight decay.
+ *
+ * grads == NULL: two-pass path; g comes from the accumulators written by
+ * zero_reduce_scatter_bucket for this step (state->acc), the step is done in
+ * place on set cur. grads != NULL: fused path; the R replicas are reduced,
+ * checked, and applied in one pass with no accumulator: in place when the
+ * state has one set (NONE or STATIC mode only, since an in-place fused step
+ * cannot be undone), ping-pong when it has two.
+ * Errors: ZERO_ERR_INVALID_ARG (a NULL pointer, DYNAMIC fused in place,
+ * bad hyper-parameters), ZERO_ERR_ALIGN, ZERO_ERR_STATE (one state set
+ * given after ping-pong steps), ZERO_ERR_CUDA, ZERO_ERR_OOM.
+ */
+zero_status zero_step(zero_ctx_t* ctx, const zero_adamw* hp, const zero_state* state,
+                      const void* const* grads, void* stream);
+
+/*
+ * zero_gather_layer -- assemble one layer's half parameters from the R
+ * shards of the current set into a contiguous buffer:
+ *   out[j] = param[cur][o][lo + j - o*S],  o = (lo + j) / S,  0 <= j < hi - lo.
+ * Defines: [legal] ZeRO-3 "All-Gather on Demand" and [instr] ZeRO-3 forward /
+ * backward bullets (a layer's parameters are all-gathered just before use
+ * and released afterwards; the backward pass gathers again); [genomic]
+ * "Bucketed All-Gather".
+ * out: device buffer of (hi - lo) half elements, 16-byte aligned; the
+ * caller owns and releases it.
+ * Errors: ZERO_ERR_RANGE (layer), ZERO_ERR_INVALID_ARG, ZERO_ERR_ALIGN,
+ * ZERO_ERR_STATE, ZERO_ERR_CUDA.
+ */
+zero_status zero_gather_layer(zero_ctx_t* ctx, int64_t layer, const zero_state* state, void* out,
+                              void* stream);
+
+typedef struct {
+    float scale;           /* current loss scale */
+    int32_t cur;           /* state set holding the current model (0 or 1) */
+    int64_t good;          /* clean steps since the last scale change */
+    int64_t t;             /* applied optimizer steps */
+    int32_t last_overflow; /* the last step saw an inf/NaN gradient sum */
+    int32_t last_skipped;  /* the last step was skipped */
+    double grad_norm_sq;   /* squared L2 norm of the last step's unscaled, averaged gradient */
+} zero_loss_scale_state;
+
+#define ZERO_LOSS_SCALE_GET 0
+#define ZERO_LOSS_SCALE_SET 1
+
+/*
+ * zero_loss_scale -- read (GET) or overwrite (SET) the device-resident
+ * loss-scale state; SET is how a run resumes from a checkpoint. Both
+ * synchronize `stream` (GET reads the state after all work queued on it).
+ * Defines: the state of [legal] "Dynamic Loss Scaling".
+ * Errors: ZERO_ERR_INVALID_ARG (op, NULL, cur not 0/1, scale <= 0, t < 0),
+ * ZERO_ERR_CUDA.
+ */
+zero_status zero_loss_scale(zero_ctx_t* ctx, zero_loss_scale_state* inout, int32_t op,
+                            void* stream);
+
+/* zero_sync -- synchronize `stream` and report any pending CUDA error. */
+zero_status zero_sync(zero_ctx_t* ctx, void* stream);
+
+/* Copy the calling thread's last error message into buf (NUL-terminated,
+ * truncated to n bytes); returns the message's full length. */
+size_t zero_last_error(char* buf, size_t n);
+
+/* Library version string (static storage). */
+const char* zero_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif

@@ -1,0 +1,199 @@
+"""Helpers for the GPU parity tests: guard-banded device buffers, seeded
+inputs shared by both sides, and comparison against the oracle.
+
+Every device buffer handed to the library is a view into a larger
+allocation whose guard bands (GUARD elements on each side) hold a canary
+pattern; `check_guards` verifies after every launch that no kernel wrote
+outside its buffer.
+"""
+import numpy as np
+import torch
+
+import oracle as O
+import zero_partitioned_mixed_reduce_b200 as Z
+from zero_partitioned_mixed_reduce_b200 import synth
+
+GUARD = 64  # elements; keeps 32-byte alignment for fp32 and 16-byte for half
+CANARY_F32 = 0x7FBADBAD  # a NaN pattern no kernel writes
+CANARY_U16 = 0x7DAD
+
+HALF = {0: torch.bfloat16, 1: torch.float16}
+
+
+class Guarded:
+    """Buffers of n elements with canary guard bands."""
+
+    def __init__(self):
+        self.allocs = []
+
+    def f32(self, n):
+        base = torch.empty(n + 2 * GUARD, dtype=torch.int32, device="cuda")
+        base.fill_(CANARY_F32)
+        self.allocs.append((base, "f32"))
+        return base[GUARD:GUARD + n].view(torch.float32)
+
+    def half(self, n, dtype):
+        base = torch.empty(n + 2 * GUARD, dtype=torch.int16, device="cuda")
+        base.fill_(np.int16(np.uint16(CANARY_U16).view(np.int16)))
+        self.allocs.append((base, "u16"))
+        return base[GUARD:GUARD + n].view(HALF[dtype])
+
+    def check(self):
+        torch.cuda.synchronize()
+        for base, kind in self.allocs:
+            head, tail = base[:GUARD], base[-GUARD:]
+            if kind == "f32":
+                ok = bool((head == CANARY_F32).all()) and bool((tail == CANARY_F32).all())
+            else:
+                c = int(np.uint16(CANARY_U16).view(np.int16))
+                ok = bool((head == c).all()) and bool((tail == c).all())
+            assert ok, "a kernel wrote into a guard band"
+
+
+def u16(t: torch.Tensor) -> np.ndarray:
+    return t.detach().contiguous().view(torch.int16).cpu().numpy().view(np.uint16)
+
+
+def f32bits(a: np.ndarray) -> np.ndarray:
+    return np.ascontiguousarray(a, np.float32).view(np.uint32)
+
+
+class Case:
+    """One parity case: a tensor list, R, dtype, alignment, loss-scale mode and
+    path ("inplace", "pingpong", "twopass"), run for a few steps on the GPU
+    and in the oracle on the same bytes."""
+
+    def __init__(self, numels, R, dtype, align=8, mode=O.SCALE_NONE, init_scale=1.0, interval=1000,
+                 path="pingpong", bucket_elems=0, layer_ids=None, sigma=1e-2, seed=5, hp=None):
+        self.wl = synth.custom_workload(numels, R, dtype, mode, init_scale, interval, sigma,
+                                        layer_ids=layer_ids, bucket_elems=bucket_elems, index=seed)
+        self.R, self.dtype, self.mode, self.path = R, dtype, mode, path
+        self.hp = hp or self.wl["hp"]
+        self.lay = O.Layout(numels, R, align, bucket_elems, layer_ids)
+        self.plan = Z.Plan(numels, layer_ids, R, dtype, align, bucket_elems)
+        self.idx = self.lay.flat_index()
+        S, T = self.plan.S, self.plan.T
+        self.g = Guarded()
+        sets = 2 if path == "pingpong" else 1
+        self.sets = sets
+        self.master = [[self.g.f32(S) for _ in range(R)] for _ in range(sets)]
+        self.m = [[self.g.f32(S) for _ in range(R)] for _ in range(sets)]
+        self.v = [[self.g.f32(S) for _ in range(R)] for _ in range(sets)]
+        self.param = [[self.g.half(S, dtype) for _ in range(R)] for _ in range(sets)]
+        self.acc = [self.g.f32(S) for _ in range(R)] if path == "twopass" else None
+        self.grads = [self.g.half(T, dtype) for _ in range(R)]
+        self.handle = Z.StateHandle(
+            [dict(master=self.master[k], m=self.m[k], v=self.v[k], param=self.param[k])
+             for k in range(sets)], self.acc)
+        # initial state: fp32 master ~N(0, 0.02), half param = torch cast of it
+        x = synth.flat_master(self.wl, "cpu")
+        p0 = x.to(HALF[dtype])
+        self.ostate = O.State(x.numpy(), dtype, u16(p0))
+        mpad = self.plan.pack(x, fill=0.0)
+        ppad = self.plan.pack(p0, fill=0)
+        for k in range(sets):
+            for r in range(R):
+                sl = slice(r * S, (r + 1) * S)
+                self.master[k][r].copy_(mpad[sl])
+                self.param[k][r].copy_(ppad[sl])
+                self.m[k][r].zero_()
+                self.v[k][r].zero_()
+        self.ofsm = O.make_fsm(mode, scale=init_scale if mode != O.SCALE_NONE else 1.0,
+                               interval=interval)
+        self.ctx = Z.zero_ctx_create(self.plan.handle, mode, init_scale, interval)
+        self.step_no = 0
+
+    def close(self):
+        if self.ctx:
+            Z.zero_ctx_destroy(self.ctx)
+            self.ctx = None
+
+    def make_grads(self, inject=None):
+        """Seeded replicas at the current loss scale; returns (R, P) uint16."""
+        scale = self.ofsm.scale if self.mode != O.SCALE_NONE else 1.0
+        rows = [synth.flat_grads(self.wl, self.step_no, r, scale, "cpu") for r in range(self.R)]
+        g = np.stack([u16(t) for t in rows])
+        if inject:
+            for (r, e, bits) in inject:
+                g[r, e] = bits
+        return g
+
+    def step(self, inject=None):
+        self.step_no += 1
+        g = self.make_grads(inject)
+        # GPU inputs: padded replicas (padding zero)
+        for r in range(self.R):
+            gp = np.zeros(self.plan.T, np.uint16)
+            gp[self.idx] = g[r]
+            self.grads[r].view(torch.int16).copy_(torch.from_numpy(gp.view(np.int16)))
+        if self.path == "twopass":
+            for b in range(len(self.plan.buckets)):
+                Z.zero_reduce_scatter_bucket(self.ctx, b, self.grads, self.acc)
+            Z.zero_step(self.ctx, self.hp, self.handle, None)
+        else:
+            Z.zero_step(self.ctx, self.hp, self.handle, self.grads)
+        skipped = O.step(self.ostate, g, O.AdamW(**{k: self.hp[k] for k in
+                                                    ("lr", "beta1", "beta2", "eps",
+                                                     "weight_decay")}), self.ofsm)
+        self.g.check()
+        return skipped
+
+    def gpu_fsm(self):
+        return Z.zero_loss_scale(self.ctx)
+
+    def gpu_state(self):
+        cur = self.gpu_fsm()["cur"]
+        k = cur if self.sets == 2 else 0
+        idx = self.idx
+        cat = lambda bufs: torch.cat([b for b in bufs]).cpu()
+        master = cat(self.master[k]).numpy()[idx]
+        m = cat(self.m[k]).numpy()[idx]
+        v = cat(self.v[k]).numpy()[idx]
+        param = u16(torch.cat(self.param[k]))[idx]
+        pads = np.ones(self.plan.T, bool)
+        pads[idx] = False
+        return dict(master=master, m=m, v=v, param=param, cur=cur,
+                    pad_master=cat(self.master[k]).numpy()[pads],
+                    pad_param=u16(torch.cat(self.param[k]))[pads])
+
+    def compare(self, exact=True):
+        """Assert parity with the oracle after the last step."""
+        f = self.gpu_fsm()
+        o = self.ofsm
+        assert (f["t"], f["good"], f["last_overflow"], f["last_skipped"]) == \
+               (o.t, o.good, o.last_overflow, o.last_skipped), (f, o.t, o.good)
+        assert np.float32(f["scale"]) == np.float32(o.scale)
+        if np.isfinite(o.grad_norm_sq):
+            assert abs(f["grad_norm_sq"] - o.grad_norm_sq) <= 1e-9 * abs(o.grad_norm_sq) + 1e-300
+        else:
+            assert not np.isfinite(f["grad_norm_sq"])
+        s = self.gpu_state()
+        st = self.ostate
+        for name in ("master", "m", "v"):
+            a, b = s[name], getattr(st, name)
+            fin = np.isfinite(b)
+            assert np.array_equal(np.isfinite(a), fin), name
+            rel = np.abs(a[fin].astype(np.float64) - b[fin]) / np.maximum(np.abs(b[fin]), 1e-30)
+            assert rel.size == 0 or rel.max() <= 1e-5, (name, rel.max())
+            if exact:
+                assert np.array_equal(f32bits(a[fin]), f32bits(b[fin])), \
+                    (name, int(np.sum(f32bits(a[fin]) != f32bits(b[fin]))))
+        pa, pb = s["param"].astype(np.int32), st.param.astype(np.int32)
+        nan_b = half_is_nan(st.param, self.dtype)
+        assert np.array_equal(half_is_nan(s["param"], self.dtype), nan_b)
+        # within 1 ulp: same sign and adjacent encodings
+        d = np.abs(pa[~nan_b] - pb[~nan_b])
+        assert d.size == 0 or d.max() <= 1
+        if exact:
+            assert np.array_equal(pa[~nan_b], pb[~nan_b])
+        # padding stays zero
+        assert np.all(s["pad_master"] == 0) and np.all(s["pad_param"] == 0)
+        return s
+
+
+def half_is_nan(h: np.ndarray, dtype: int) -> np.ndarray:
+    """NaN encodings: all-ones exponent with a non-zero significand."""
+    h = h.astype(np.uint32)
+    if dtype == O.FP16:
+        return ((h & 0x7C00) == 0x7C00) & ((h & 0x03FF) != 0)
+    return ((h & 0x7F80) == 0x7F80) & ((h & 0x007F) != 0)

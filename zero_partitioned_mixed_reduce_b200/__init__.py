@@ -1,0 +1,15 @@
+"""ZeRO data-parallel hot path for B200 (sm_100a): partitioned mixed-precision
+AdamW over a flat sharded state, R data-parallel ranks simulated on one GPU.
+
+The compute is in libzero_b200.so (hand-written CUDA, C ABI in
+include/zero_b200.h); this package binds it with ctypes and uses PyTorch
+only for device memory and streams.
+"""
+from ._capi import (  # noqa: F401
+    ZERO_BF16, ZERO_FP16, ZERO_LOSS_SCALE_GET, ZERO_LOSS_SCALE_SET, ZERO_MAX_RANKS,
+    ZERO_SCALE_DYNAMIC, ZERO_SCALE_NONE, ZERO_SCALE_STATIC, LIB_PATH, StateHandle, ZeroError,
+    zero_adamw, zero_ctx_create, zero_ctx_destroy, zero_gather_layer, zero_last_error,
+    zero_loss_scale, zero_plan, zero_plan_bucket, zero_plan_destroy, zero_plan_get_info,
+    zero_plan_layer, zero_plan_memory, zero_plan_tensor, zero_reduce_scatter_bucket, zero_step,
+    zero_sync, zero_version)
+from .state import Plan, ShardedState  # noqa: F401

@@ -1,0 +1,266 @@
+"""ctypes binding of libzero_b200.so (include/zero_b200.h).
+
+Argument marshalling only: every step of the hot path runs in the library's
+CUDA kernels. The functions carry the C names; on a non-OK status they raise
+ZeroError with the library's message. Device buffers can be passed as
+integers or as any object with a ``data_ptr()`` method (torch tensors).
+If the shared library is missing this module raises ImportError: there is
+no fallback.
+"""
+import ctypes as C
+import os
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libzero_b200.so")
+
+ZERO_MAX_RANKS = 64
+ZERO_OK, ZERO_ERR_INVALID_ARG, ZERO_ERR_ALIGN, ZERO_ERR_CUDA = 0, 1, 2, 3
+ZERO_ERR_OOM, ZERO_ERR_RANGE, ZERO_ERR_TIMEOUT, ZERO_ERR_STATE = 4, 5, 6, 7
+ZERO_BF16, ZERO_FP16 = 0, 1
+ZERO_SCALE_NONE, ZERO_SCALE_STATIC, ZERO_SCALE_DYNAMIC = 0, 1, 2
+ZERO_LOSS_SCALE_GET, ZERO_LOSS_SCALE_SET = 0, 1
+
+STATUS_NAMES = {0: "ZERO_OK", 1: "ZERO_ERR_INVALID_ARG", 2: "ZERO_ERR_ALIGN", 3: "ZERO_ERR_CUDA",
+                4: "ZERO_ERR_OOM", 5: "ZERO_ERR_RANGE", 6: "ZERO_ERR_TIMEOUT", 7: "ZERO_ERR_STATE"}
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(
+        f"{LIB_PATH} is missing: build it with `python -m zero_partitioned_mixed_reduce_b200.build` "
+        "(nvcc, sm_100a). There is no CPU fallback.")
+
+
+class ZeroError(RuntimeError):
+    def __init__(self, status, message):
+        super().__init__(f"{STATUS_NAMES.get(status, status)}: {message}")
+        self.status = status
+
+
+class zero_plan_config(C.Structure):
+    _fields_ = [("R", C.c_int32), ("dtype", C.c_int32), ("tensor_align", C.c_int32),
+                ("reserved", C.c_int32), ("bucket_elems", C.c_int64)]
+
+
+class zero_plan_info(C.Structure):
+    _fields_ = [("P", C.c_int64), ("L", C.c_int64), ("S", C.c_int64), ("T", C.c_int64),
+                ("n_tensors", C.c_int64), ("n_buckets", C.c_int64), ("n_layers", C.c_int64),
+                ("R", C.c_int32), ("dtype", C.c_int32), ("tensor_align", C.c_int32),
+                ("reserved", C.c_int32)]
+
+
+class zero_loss_scale_config(C.Structure):
+    _fields_ = [("mode", C.c_int32), ("init_scale", C.c_float), ("growth_interval", C.c_int64),
+                ("growth_factor", C.c_float), ("backoff_factor", C.c_float),
+                ("min_scale", C.c_float), ("reserved", C.c_int32)]
+
+
+class zero_adamw(C.Structure):
+    _fields_ = [("lr", C.c_double), ("beta1", C.c_double), ("beta2", C.c_double),
+                ("eps", C.c_double), ("weight_decay", C.c_double)]
+
+
+_PP = C.POINTER(C.c_void_p)
+
+
+class zero_state(C.Structure):
+    _fields_ = [("master", _PP * 2), ("m", _PP * 2), ("v", _PP * 2), ("param", _PP * 2),
+                ("acc", _PP)]
+
+
+class zero_loss_scale_state(C.Structure):
+    _fields_ = [("scale", C.c_float), ("cur", C.c_int32), ("good", C.c_int64), ("t", C.c_int64),
+                ("last_overflow", C.c_int32), ("last_skipped", C.c_int32),
+                ("grad_norm_sq", C.c_double)]
+
+
+_lib = C.CDLL(LIB_PATH)
+_P = C.c_void_p
+_S = C.c_int32  # zero_status
+
+
+def _sig(name, restype, argtypes):
+    f = getattr(_lib, name)
+    f.restype = restype
+    f.argtypes = argtypes
+    return f
+
+
+_sig("zero_plan", _S, [_P, _P, C.c_int64, C.POINTER(zero_plan_config), C.POINTER(_P)])
+_sig("zero_plan_destroy", None, [_P])
+_sig("zero_plan_get_info", _S, [_P, C.POINTER(zero_plan_info)])
+_sig("zero_plan_tensor", _S, [_P, C.c_int64, C.POINTER(C.c_int64), C.POINTER(C.c_int64),
+                              C.POINTER(C.c_int64), C.POINTER(C.c_int64)])
+_sig("zero_plan_bucket", _S, [_P, C.c_int64, C.POINTER(C.c_int64), C.POINTER(C.c_int64)])
+_sig("zero_plan_layer", _S, [_P, C.c_int64, C.POINTER(C.c_int64), C.POINTER(C.c_int64)])
+_sig("zero_plan_memory", _S, [_P, C.c_int32, C.POINTER(C.c_int64)])
+_sig("zero_ctx_create", _S, [_P, C.POINTER(zero_loss_scale_config), C.POINTER(_P)])
+_sig("zero_ctx_destroy", _S, [_P])
+_sig("zero_reduce_scatter_bucket", _S, [_P, C.c_int64, _PP, _PP, _P])
+_sig("zero_step", _S, [_P, C.POINTER(zero_adamw), C.POINTER(zero_state), _PP, _P])
+_sig("zero_gather_layer", _S, [_P, C.c_int64, C.POINTER(zero_state), _P, _P])
+_sig("zero_loss_scale", _S, [_P, C.POINTER(zero_loss_scale_state), C.c_int32, _P])
+_sig("zero_sync", _S, [_P, _P])
+_sig("zero_last_error", C.c_size_t, [C.c_char_p, C.c_size_t])
+_sig("zero_version", C.c_char_p, [])
+
+
+def _check(status):
+    if status != ZERO_OK:
+        buf = C.create_string_buffer(1024)
+        _lib.zero_last_error(buf, 1024)
+        raise ZeroError(status, buf.value.decode(errors="replace"))
+
+
+def _addr(x):
+    if x is None:
+        return None
+    if isinstance(x, int):
+        return x
+    return int(x.data_ptr())
+
+
+def _ptr_array(xs):
+    """R device pointers -> C array (kept alive by the caller)."""
+    if xs is None:
+        return None
+    arr = (C.c_void_p * len(xs))(*[_addr(x) for x in xs])
+    return C.cast(arr, _PP), arr
+
+
+def _stream(s):
+    if s is None:
+        return None
+    if isinstance(s, int):
+        return s
+    return int(s.cuda_stream)  # torch.cuda.Stream
+
+
+# ---- plan ------------------------------------------------------------------
+
+def zero_plan(numels, layer_ids=None, R=1, dtype=ZERO_BF16, tensor_align=8, bucket_elems=0):
+    """Returns an opaque plan handle (int). Free with zero_plan_destroy."""
+    n = len(numels)
+    nb = (C.c_int64 * max(n, 1))(*[int(x) for x in numels])
+    lid = None
+    if layer_ids is not None:
+        lid = (C.c_int32 * max(n, 1))(*[int(x) for x in layer_ids])
+    cfg = zero_plan_config(R, dtype, tensor_align, 0, bucket_elems)
+    out = C.c_void_p()
+    _check(_lib.zero_plan(nb, lid, n, C.byref(cfg), C.byref(out)))
+    return out.value
+
+
+def zero_plan_destroy(plan):
+    _lib.zero_plan_destroy(plan)
+
+
+def zero_plan_get_info(plan):
+    info = zero_plan_info()
+    _check(_lib.zero_plan_get_info(plan, C.byref(info)))
+    return {k: getattr(info, k) for k, _ in zero_plan_info._fields_ if k != "reserved"}
+
+
+def zero_plan_tensor(plan, k):
+    off, num, b, l = C.c_int64(), C.c_int64(), C.c_int64(), C.c_int64()
+    _check(_lib.zero_plan_tensor(plan, k, C.byref(off), C.byref(num), C.byref(b), C.byref(l)))
+    return off.value, num.value, b.value, l.value
+
+
+def zero_plan_bucket(plan, b):
+    lo, hi = C.c_int64(), C.c_int64()
+    _check(_lib.zero_plan_bucket(plan, b, C.byref(lo), C.byref(hi)))
+    return lo.value, hi.value
+
+
+def zero_plan_layer(plan, l):
+    lo, hi = C.c_int64(), C.c_int64()
+    _check(_lib.zero_plan_layer(plan, l, C.byref(lo), C.byref(hi)))
+    return lo.value, hi.value
+
+
+def zero_plan_memory(plan, stage):
+    b = C.c_int64()
+    _check(_lib.zero_plan_memory(plan, stage, C.byref(b)))
+    return b.value
+
+
+# ---- context ---------------------------------------------------------------
+
+def zero_ctx_create(plan, mode=ZERO_SCALE_NONE, init_scale=1.0, growth_interval=1000,
+                    growth_factor=2.0, backoff_factor=0.5, min_scale=1.0):
+    cfg = zero_loss_scale_config(mode, init_scale, growth_interval, growth_factor,
+                                 backoff_factor, min_scale, 0)
+    out = C.c_void_p()
+    _check(_lib.zero_ctx_create(plan, C.byref(cfg), C.byref(out)))
+    return out.value
+
+
+def zero_ctx_destroy(ctx):
+    _check(_lib.zero_ctx_destroy(ctx))
+
+
+class StateHandle:
+    """A zero_state built from R-long lists of device buffers per field.
+
+    sets: list of one or two dicts with keys master, m, v, param; acc: list or
+    None. Keeps the pointer arrays alive as long as the handle lives."""
+
+    def __init__(self, sets, acc=None):
+        self._keep = []
+        self.c = zero_state()
+        for k, d in enumerate(sets):
+            for field in ("master", "m", "v", "param"):
+                p, arr = _ptr_array(d[field])
+                self._keep.append(arr)
+                getattr(self.c, field)[k] = p
+        if acc is not None:
+            p, arr = _ptr_array(acc)
+            self._keep.append(arr)
+            self.c.acc = p
+
+
+def zero_reduce_scatter_bucket(ctx, bucket, grads, acc, stream=None):
+    g, ga = _ptr_array(grads)
+    a, aa = _ptr_array(acc)
+    _check(_lib.zero_reduce_scatter_bucket(ctx, bucket, g, a, _stream(stream)))
+
+
+def zero_step(ctx, hp, state: StateHandle, grads=None, stream=None):
+    """hp: zero_adamw or a dict with lr, beta1, beta2, eps, weight_decay."""
+    if isinstance(hp, dict):
+        hp = zero_adamw(hp["lr"], hp["beta1"], hp["beta2"], hp["eps"], hp["weight_decay"])
+    g = None
+    if grads is not None:
+        g, ga = _ptr_array(grads)
+    _check(_lib.zero_step(ctx, C.byref(hp), C.byref(state.c), g, _stream(stream)))
+
+
+def zero_gather_layer(ctx, layer, state: StateHandle, out, stream=None):
+    _check(_lib.zero_gather_layer(ctx, layer, C.byref(state.c), _addr(out), _stream(stream)))
+
+
+def zero_loss_scale(ctx, op=ZERO_LOSS_SCALE_GET, state=None, stream=None):
+    """GET returns a dict; SET takes a dict (or zero_loss_scale_state)."""
+    st = zero_loss_scale_state()
+    if op == ZERO_LOSS_SCALE_SET:
+        if isinstance(state, dict):
+            for k, _ in zero_loss_scale_state._fields_:
+                if k in state:
+                    setattr(st, k, state[k])
+        else:
+            st = state
+    _check(_lib.zero_loss_scale(ctx, C.byref(st), op, _stream(stream)))
+    return {k: getattr(st, k) for k, _ in zero_loss_scale_state._fields_}
+
+
+def zero_sync(ctx, stream=None):
+    _check(_lib.zero_sync(ctx, _stream(stream)))
+
+
+def zero_last_error():
+    buf = C.create_string_buffer(1024)
+    _lib.zero_last_error(buf, 1024)
+    return buf.value.decode(errors="replace")
+
+
+def zero_version():
+    return _lib.zero_version().decode()

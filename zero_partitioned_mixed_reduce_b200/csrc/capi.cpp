@@ -1,0 +1,413 @@
+// C ABI of libzero_b200.so: context lifecycle, argument validation, kernel
+// launches and the loss-scale state. See include/zero_b200.h for the
+// contract of every call.
+#include <cmath>
+#include <cstring>
+#include <new>
+#include <string>
+#include <vector>
+
+#include "internal.h"
+
+namespace {
+
+thread_local std::string g_last_error;
+
+}  // namespace
+
+zero_status zb_fail(zero_status code, const std::string& msg) {
+    g_last_error = msg;
+    return code;
+}
+
+struct zero_ctx_s {
+    int device = 0;
+    int32_t R = 0, dtype = 0;
+    int64_t S = 0, T = 0;
+    std::vector<int64_t> bucket_lo, bucket_hi, layer_lo, layer_hi;
+    zero_loss_scale_config cfg{};
+    zb::DevState* st = nullptr;   // device
+    double* partials = nullptr;   // device, grid_cap entries
+    int grid_cap = 0;
+    double2* powtab = nullptr;    // device, powtab_len entries
+    int64_t powtab_len = 0;
+    double pow_b1 = NAN, pow_b2 = NAN;
+    int64_t t_bound = 0;          // upper bound of the device step count
+    bool two_sets = false;        // a ping-pong step has run (or cur was set to 1)
+};
+
+namespace {
+
+zero_status cuda_fail(const char* where, cudaError_t e) {
+    return zb_fail(ZERO_ERR_CUDA, std::string(where) + ": " + cudaGetErrorName(e) + ": " +
+                                      cudaGetErrorString(e));
+}
+
+zero_status check_device(const zero_ctx_t* ctx, const char* where) {
+    int dev = -1;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(where, e);
+    if (dev != ctx->device)
+        return zb_fail(ZERO_ERR_INVALID_ARG, std::string(where) + ": context belongs to device " +
+                                                 std::to_string(ctx->device) +
+                                                 " but device " + std::to_string(dev) +
+                                                 " is current");
+    // surface errors of earlier asynchronous work
+    e = cudaPeekAtLastError();
+    if (e != cudaSuccess) {
+        cudaGetLastError();
+        return cuda_fail(where, e);
+    }
+    return ZERO_OK;
+}
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+template <typename Ptr>
+zero_status check_ranks(Ptr const* arr, int R, uintptr_t align, const char* where,
+                        const char* what) {
+    if (!arr) return zb_fail(ZERO_ERR_INVALID_ARG, std::string(where) + ": " + what + " is NULL");
+    for (int r = 0; r < R; ++r) {
+        if (!arr[r])
+            return zb_fail(ZERO_ERR_INVALID_ARG, std::string(where) + ": " + what + "[" +
+                                                     std::to_string(r) + "] is NULL");
+        if (!aligned(arr[r], align))
+            return zb_fail(ZERO_ERR_ALIGN, std::string(where) + ": " + what + "[" +
+                                               std::to_string(r) + "] is not " +
+                                               std::to_string(align) + "-byte aligned");
+    }
+    return ZERO_OK;
+}
+
+// Validate the state sets; returns the number of sets (1 or 2) in *sets.
+zero_status check_state(const zero_ctx_t* ctx, const zero_state* st, const char* where, int* sets,
+                        bool params_only) {
+    if (!st) return zb_fail(ZERO_ERR_INVALID_ARG, std::string(where) + ": state is NULL");
+    const int R = ctx->R;
+    zero_status s;
+    const bool set1_any = st->master[1] || st->m[1] || st->v[1] || st->param[1];
+    const bool set1_all = st->master[1] && st->m[1] && st->v[1] && st->param[1];
+    if (params_only) {
+        if ((s = check_ranks(st->param[0], R, 16, where, "param[0]")) != ZERO_OK) return s;
+        if (st->param[1] && (s = check_ranks(st->param[1], R, 16, where, "param[1]")) != ZERO_OK)
+            return s;
+        *sets = st->param[1] ? 2 : 1;
+        return ZERO_OK;
+    }
+    if (set1_any && !set1_all)
+        return zb_fail(ZERO_ERR_INVALID_ARG,
+                       std::string(where) + ": state set 1 must be given completely or not at all");
+    for (int k = 0; k < (set1_all ? 2 : 1); ++k) {
+        if ((s = check_ranks(st->master[k], R, 32, where, k ? "master[1]" : "master[0]")) != ZERO_OK) return s;
+        if ((s = check_ranks(st->m[k], R, 32, where, k ? "m[1]" : "m[0]")) != ZERO_OK) return s;
+        if ((s = check_ranks(st->v[k], R, 32, where, k ? "v[1]" : "v[0]")) != ZERO_OK) return s;
+        if ((s = check_ranks(st->param[k], R, 16, where, k ? "param[1]" : "param[0]")) != ZERO_OK) return s;
+    }
+    *sets = set1_all ? 2 : 1;
+    return ZERO_OK;
+}
+
+void fill_state_ptrs(const zero_ctx_t* ctx, const zero_state* st, int sets, zb::RankPtrs* p) {
+    for (int r = 0; r < ctx->R; ++r)
+        for (int k = 0; k < 2; ++k) {
+            const int from = (k < sets) ? k : 0;  // one set: both slots alias set 0
+            p->master[k][r] = st->master[from] ? st->master[from][r] : nullptr;
+            p->m[k][r] = st->m[from] ? st->m[from][r] : nullptr;
+            p->v[k][r] = st->v[from] ? st->v[from][r] : nullptr;
+            p->param[k][r] = st->param[from] ? st->param[from][r] : nullptr;
+        }
+}
+
+// Host-built table of (beta1^t, beta2^t), t = 0..len-1, computed with the C
+// library's pow in double; the device forms the bias corrections from it.
+zero_status ensure_powtab(zero_ctx_t* ctx, double b1, double b2, int64_t need_t, cudaStream_t s) {
+    if (ctx->powtab && ctx->pow_b1 == b1 && ctx->pow_b2 == b2 && need_t < ctx->powtab_len)
+        return ZERO_OK;
+    int64_t len = 1024;
+    while (len <= need_t) len *= 2;
+    std::vector<double2> host(static_cast<size_t>(len));
+    for (int64_t t = 0; t < len; ++t)
+        host[t] = make_double2(std::pow(b1, static_cast<double>(t)), std::pow(b2, static_cast<double>(t)));
+    // kernels already queued may still read the old table
+    cudaError_t e = cudaStreamSynchronize(s);
+    if (e != cudaSuccess) return cuda_fail("zero_step: power table", e);
+    if (ctx->powtab) cudaFree(ctx->powtab);
+    ctx->powtab = nullptr;
+    ctx->powtab_len = 0;
+    e = cudaMalloc(&ctx->powtab, sizeof(double2) * static_cast<size_t>(len));
+    if (e != cudaSuccess) {
+        cudaGetLastError();
+        return zb_fail(ZERO_ERR_OOM, "zero_step: cannot allocate the power table");
+    }
+    e = cudaMemcpy(ctx->powtab, host.data(), sizeof(double2) * host.size(), cudaMemcpyHostToDevice);
+    if (e != cudaSuccess) return cuda_fail("zero_step: power table upload", e);
+    ctx->powtab_len = len;
+    ctx->pow_b1 = b1;
+    ctx->pow_b2 = b2;
+    return ZERO_OK;
+}
+
+}  // namespace
+
+extern "C" zero_status zero_ctx_create(const zero_plan_t* plan, const zero_loss_scale_config* cfg,
+                                       zero_ctx_t** out) {
+    if (!out) return zb_fail(ZERO_ERR_INVALID_ARG, "zero_ctx_create: out is NULL");
+    *out = nullptr;
+    if (!plan || !cfg) return zb_fail(ZERO_ERR_INVALID_ARG, "zero_ctx_create: NULL plan or cfg");
+    if (cfg->mode < ZERO_SCALE_NONE || cfg->mode > ZERO_SCALE_DYNAMIC)
+        return zb_fail(ZERO_ERR_INVALID_ARG, "zero_ctx_create: bad loss-scale mode");
+    if (cfg->mode != ZERO_SCALE_NONE && !(cfg->init_scale > 0.0f && std::isfinite(cfg->init_scale)))
+        return zb_fail(ZERO_ERR_INVALID_ARG, "zero_ctx_create: init_scale must be finite and > 0");
+    if (cfg->mode == ZERO_SCALE_DYNAMIC) {
+        if (cfg->growth_interval < 1)
+            return zb_fail(ZERO_ERR_INVALID_ARG, "zero_ctx_create: growth_interval must be >= 1");
+        if (!(cfg->growth_factor > 1.0f) || !(cfg->backoff_factor > 0.0f && cfg->backoff_factor < 1.0f) ||
+            !(cfg->min_scale > 0.0f))
+            return zb_fail(ZERO_ERR_INVALID_ARG,
+                           "zero_ctx_create: need growth_factor > 1, 0 < backoff_factor < 1, min_scale > 0");
+    }
+    if (cfg->reserved != 0) return zb_fail(ZERO_ERR_INVALID_ARG, "zero_ctx_create: reserved must be 0");
+
+    zero_ctx_t* ctx = new (std::nothrow) zero_ctx_t();
+    if (!ctx) return zb_fail(ZERO_ERR_OOM, "zero_ctx_create: out of host memory");
+    cudaError_t e = cudaGetDevice(&ctx->device);
+    if (e != cudaSuccess) {
+        delete ctx;
+        cudaGetLastError();
+        return cuda_fail("zero_ctx_create", e);
+    }
+    ctx->R = plan->R;
+    ctx->dtype = plan->dtype;
+    ctx->S = plan->S;
+    ctx->T = plan->T;
+    ctx->bucket_lo = plan->bucket_lo;
+    ctx->bucket_hi = plan->bucket_hi;
+    ctx->layer_lo = plan->layer_lo;
+    ctx->layer_hi = plan->layer_hi;
+    ctx->cfg = *cfg;
+    ctx->grid_cap = zb::step_grid_cap(ctx->device);
+
+    e = cudaMalloc(&ctx->st, sizeof(zb::DevState));
+    if (e == cudaSuccess) e = cudaMalloc(&ctx->partials, sizeof(double) * ctx->grid_cap);
+    if (e != cudaSuccess) {
+        cudaGetLastError();
+        if (ctx->st) cudaFree(ctx->st);
+        delete ctx;
+        return zb_fail(ZERO_ERR_OOM, "zero_ctx_create: cannot allocate device scratch");
+    }
+    zb::DevState init{};
+    init.scale = cfg->mode == ZERO_SCALE_NONE ? 1.0f : cfg->init_scale;
+    e = cudaMemcpy(ctx->st, &init, sizeof(init), cudaMemcpyHostToDevice);
+    if (e == cudaSuccess) e = cudaMemset(ctx->partials, 0, sizeof(double) * ctx->grid_cap);
+    if (e != cudaSuccess) {
+        cudaFree(ctx->st);
+        cudaFree(ctx->partials);
+        delete ctx;
+        return cuda_fail("zero_ctx_create", e);
+    }
+    *out = ctx;
+    return ZERO_OK;
+}
+
+extern "C" zero_status zero_ctx_destroy(zero_ctx_t* ctx) {
+    if (!ctx) return ZERO_OK;
+    int prev = -1;
+    cudaGetDevice(&prev);
+    cudaSetDevice(ctx->device);
+    cudaError_t e = cudaDeviceSynchronize();
+    cudaFree(ctx->st);
+    cudaFree(ctx->partials);
+    if (ctx->powtab) cudaFree(ctx->powtab);
+    if (prev >= 0) cudaSetDevice(prev);
+    delete ctx;
+    if (e != cudaSuccess) return cuda_fail("zero_ctx_destroy", e);
+    return ZERO_OK;
+}
+
+extern "C" zero_status zero_reduce_scatter_bucket(zero_ctx_t* ctx, int64_t bucket,
+                                                  const void* const* grads, float* const* acc,
+                                                  void* stream) {
+    const char* where = "zero_reduce_scatter_bucket";
+    if (!ctx) return zb_fail(ZERO_ERR_INVALID_ARG, "zero_reduce_scatter_bucket: ctx is NULL");
+    zero_status s = check_device(ctx, where);
+    if (s != ZERO_OK) return s;
+    int64_t lo, hi;
+    if (bucket == -1) {
+        lo = 0;
+        hi = ctx->T;
+    } else if (bucket < 0 || bucket >= static_cast<int64_t>(ctx->bucket_lo.size())) {
+        return zb_fail(ZERO_ERR_RANGE, "zero_reduce_scatter_bucket: bucket index out of range");
+    } else {
+        lo = ctx->bucket_lo[bucket];
+        hi = ctx->bucket_hi[bucket];
+    }
+    if ((s = check_ranks(grads, ctx->R, 16, where, "grads")) != ZERO_OK) return s;
+    if ((s = check_ranks(acc, ctx->R, 32, where, "acc")) != ZERO_OK) return s;
+    zb::RankPtrs p;
+    for (int r = 0; r < ctx->R; ++r) {
+        p.g[r] = grads[r];
+        p.acc[r] = acc[r];
+    }
+    cudaError_t e = zb::launch_reduce_scatter(ctx->R, ctx->dtype, ctx->S, lo, hi, ctx->st, p,
+                                              static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(where, e);
+    return ZERO_OK;
+}
+
+extern "C" zero_status zero_step(zero_ctx_t* ctx, const zero_adamw* hp, const zero_state* state,
+                                 const void* const* grads, void* stream) {
+    const char* where = "zero_step";
+    if (!ctx || !hp) return zb_fail(ZERO_ERR_INVALID_ARG, "zero_step: NULL ctx or hyper-parameters");
+    zero_status s = check_device(ctx, where);
+    if (s != ZERO_OK) return s;
+    if (!(hp->lr >= 0.0) || !(hp->beta1 >= 0.0 && hp->beta1 < 1.0) ||
+        !(hp->beta2 >= 0.0 && hp->beta2 < 1.0) || !(hp->eps > 0.0) || !(hp->weight_decay >= 0.0) ||
+        !std::isfinite(hp->lr) || !std::isfinite(hp->weight_decay))
+        return zb_fail(ZERO_ERR_INVALID_ARG,
+                       "zero_step: need lr >= 0, 0 <= beta < 1, eps > 0, weight_decay >= 0");
+    int sets = 1;
+    if ((s = check_state(ctx, state, where, &sets, false)) != ZERO_OK) return s;
+    const bool fused = grads != nullptr;
+    if (fused) {
+        if ((s = check_ranks(grads, ctx->R, 16, where, "grads")) != ZERO_OK) return s;
+        if (sets == 1 && ctx->cfg.mode == ZERO_SCALE_DYNAMIC)
+            return zb_fail(ZERO_ERR_INVALID_ARG,
+                           "zero_step: a fused step with dynamic loss scaling needs state set 1 "
+                           "(ping-pong) so that a skipped step can be undone; or use the two-pass path");
+    } else {
+        if ((s = check_ranks(state->acc, ctx->R, 32, where, "acc")) != ZERO_OK) return s;
+    }
+    if (sets == 1 && ctx->two_sets)
+        return zb_fail(ZERO_ERR_STATE,
+                       "zero_step: the current model may live in state set 1; pass both sets");
+
+    cudaStream_t cs = static_cast<cudaStream_t>(stream);
+    if ((s = ensure_powtab(ctx, hp->beta1, hp->beta2, ctx->t_bound + 1, cs)) != ZERO_OK) return s;
+
+    zb::StepParams sp;
+    sp.R = ctx->R;
+    sp.dtype = ctx->dtype;
+    sp.mode = ctx->cfg.mode;
+    sp.pingpong = (fused && sets == 2) ? 1 : 0;
+    sp.S8 = static_cast<uint32_t>(ctx->S / 8);
+    sp.T8 = static_cast<uint32_t>(ctx->T / 8);
+    sp.dec = static_cast<float>(1.0 - hp->lr * hp->weight_decay);
+    sp.b1f = static_cast<float>(hp->beta1);
+    sp.omb1 = static_cast<float>(1.0 - hp->beta1);
+    sp.b2f = static_cast<float>(hp->beta2);
+    sp.omb2 = static_cast<float>(1.0 - hp->beta2);
+    sp.epsf = static_cast<float>(hp->eps);
+    sp.lr = hp->lr;
+    sp.interval = ctx->cfg.growth_interval;
+    sp.growth = ctx->cfg.growth_factor;
+    sp.backoff = ctx->cfg.backoff_factor;
+    sp.min_scale = ctx->cfg.min_scale;
+    sp.st = ctx->st;
+    sp.partials = ctx->partials;
+    sp.powtab = ctx->powtab;
+    sp.powtab_len = ctx->powtab_len;
+    sp.grid_cap = ctx->grid_cap;
+
+    zb::RankPtrs p;
+    fill_state_ptrs(ctx, state, sets, &p);
+    for (int r = 0; r < ctx->R; ++r) {
+        p.g[r] = fused ? grads[r] : nullptr;
+        p.acc[r] = fused ? nullptr : state->acc[r];
+    }
+    cudaError_t e = fused ? zb::launch_fused_step(sp, p, cs) : zb::launch_step_from_acc(sp, p, cs);
+    if (e != cudaSuccess) return cuda_fail(where, e);
+    ctx->t_bound += 1;
+    if (sp.pingpong) ctx->two_sets = true;
+    return ZERO_OK;
+}
+
+extern "C" zero_status zero_gather_layer(zero_ctx_t* ctx, int64_t layer, const zero_state* state,
+                                         void* out, void* stream) {
+    const char* where = "zero_gather_layer";
+    if (!ctx) return zb_fail(ZERO_ERR_INVALID_ARG, "zero_gather_layer: ctx is NULL");
+    zero_status s = check_device(ctx, where);
+    if (s != ZERO_OK) return s;
+    if (layer < 0 || layer >= static_cast<int64_t>(ctx->layer_lo.size()))
+        return zb_fail(ZERO_ERR_RANGE, "zero_gather_layer: layer index out of range");
+    if (!out) return zb_fail(ZERO_ERR_INVALID_ARG, "zero_gather_layer: out is NULL");
+    if (!aligned(out, 16)) return zb_fail(ZERO_ERR_ALIGN, "zero_gather_layer: out is not 16-byte aligned");
+    int sets = 1;
+    if ((s = check_state(ctx, state, where, &sets, true)) != ZERO_OK) return s;
+    if (sets == 1 && ctx->two_sets)
+        return zb_fail(ZERO_ERR_STATE,
+                       "zero_gather_layer: the current parameters may live in set 1; pass param[1]");
+    zb::RankPtrs p;
+    for (int r = 0; r < ctx->R; ++r) {
+        p.param[0][r] = state->param[0][r];
+        p.param[1][r] = sets == 2 ? state->param[1][r] : state->param[0][r];
+    }
+    cudaError_t e = zb::launch_gather(ctx->R, ctx->S, ctx->layer_lo[layer], ctx->layer_hi[layer],
+                                      ctx->st, p, out, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(where, e);
+    return ZERO_OK;
+}
+
+extern "C" zero_status zero_loss_scale(zero_ctx_t* ctx, zero_loss_scale_state* inout, int32_t op,
+                                       void* stream) {
+    const char* where = "zero_loss_scale";
+    if (!ctx || !inout) return zb_fail(ZERO_ERR_INVALID_ARG, "zero_loss_scale: NULL argument");
+    zero_status s = check_device(ctx, where);
+    if (s != ZERO_OK) return s;
+    cudaStream_t cs = static_cast<cudaStream_t>(stream);
+    zb::DevState d{};
+    if (op == ZERO_LOSS_SCALE_GET) {
+        cudaError_t e = cudaMemcpyAsync(&d, ctx->st, sizeof(d), cudaMemcpyDeviceToHost, cs);
+        if (e == cudaSuccess) e = cudaStreamSynchronize(cs);
+        if (e != cudaSuccess) return cuda_fail(where, e);
+        if (d.err != 0)
+            return zb_fail(ZERO_ERR_STATE, "zero_loss_scale: device reported an inconsistent step "
+                                           "counter (power table behind t)");
+        inout->scale = d.scale;
+        inout->cur = d.cur;
+        inout->good = d.good;
+        inout->t = d.t;
+        inout->last_overflow = d.last_overflow;
+        inout->last_skipped = d.last_skipped;
+        inout->grad_norm_sq = d.grad_norm_sq;
+        ctx->t_bound = d.t;
+        return ZERO_OK;
+    }
+    if (op != ZERO_LOSS_SCALE_SET)
+        return zb_fail(ZERO_ERR_INVALID_ARG, "zero_loss_scale: op must be GET or SET");
+    if ((inout->cur != 0 && inout->cur != 1) || !(inout->scale > 0.0f) ||
+        !std::isfinite(inout->scale) || inout->t < 0 || inout->good < 0)
+        return zb_fail(ZERO_ERR_INVALID_ARG,
+                       "zero_loss_scale: need cur in {0,1}, finite scale > 0, t >= 0, good >= 0");
+    d.scale = ctx->cfg.mode == ZERO_SCALE_NONE ? 1.0f : inout->scale;
+    d.cur = inout->cur;
+    d.good = inout->good;
+    d.t = inout->t;
+    d.last_overflow = inout->last_overflow;
+    d.last_skipped = inout->last_skipped;
+    d.grad_norm_sq = inout->grad_norm_sq;
+    cudaError_t e = cudaMemcpyAsync(ctx->st, &d, sizeof(d), cudaMemcpyHostToDevice, cs);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(cs);
+    if (e != cudaSuccess) return cuda_fail(where, e);
+    ctx->t_bound = inout->t;
+    if (inout->cur == 1) ctx->two_sets = true;
+    return ZERO_OK;
+}
+
+extern "C" zero_status zero_sync(zero_ctx_t* ctx, void* stream) {
+    if (!ctx) return zb_fail(ZERO_ERR_INVALID_ARG, "zero_sync: ctx is NULL");
+    cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+    if (e == cudaSuccess) e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail("zero_sync", e);
+    return ZERO_OK;
+}
+
+extern "C" size_t zero_last_error(char* buf, size_t n) {
+    if (buf && n > 0) {
+        const size_t k = g_last_error.size() < n - 1 ? g_last_error.size() : n - 1;
+        std::memcpy(buf, g_last_error.data(), k);
+        buf[k] = '\0';
+    }
+    return g_last_error.size();
+}
+
+extern "C" const char* zero_version(void) { return "zero_b200 0.1.0 (sm_100a)"; }

@@ -1,0 +1,80 @@
+// Internal declarations shared by the host C++ (plan, C ABI) and the CUDA
+// kernels of libzero_b200.so. Not installed; the public ABI is
+// include/zero_b200.h.
+#pragma once
+
+#include <cstdint>
+#include <string>
+#include <vector>
+
+#include <cuda_runtime.h>
+
+#include "zero_b200.h"
+
+struct zero_plan_s {
+    int32_t R = 0, dtype = 0, align = 0;
+    int64_t bucket_elems = 0;
+    int64_t P = 0, L = 0, S = 0, T = 0;
+    std::vector<int64_t> numel, offset, tensor_bucket, tensor_layer;
+    std::vector<int64_t> bucket_lo, bucket_hi;
+    std::vector<int64_t> layer_lo, layer_hi;
+};
+
+namespace zb {
+
+// Device-resident loss-scale / step state. One per context, in the
+// context's device scratch. Written by the last block of every step kernel.
+struct alignas(64) DevState {
+    float scale;
+    int32_t cur;
+    int64_t good;
+    int64_t t;
+    int32_t last_overflow;
+    int32_t last_skipped;
+    double grad_norm_sq;
+    uint32_t flag;  // OR of "some reduced gradient is inf/NaN" for the step in progress
+    uint32_t done;  // blocks of the running step kernel that have finished
+    int32_t err;    // device-side consistency error (0 = none)
+    int32_t pad;
+};
+
+// Everything a step kernel needs besides the rank pointers. Filled on the host.
+struct StepParams {
+    int32_t R = 0, dtype = 0, mode = 0, pingpong = 0;
+    uint32_t S8 = 0, T8 = 0;  // shard and total length in 8-element vectors
+    float dec = 0, b1f = 0, omb1 = 0, b2f = 0, omb2 = 0, epsf = 0;
+    double lr = 0;
+    int64_t interval = 1;
+    float growth = 2, backoff = 0.5f, min_scale = 1;
+    DevState* st = nullptr;
+    double* partials = nullptr;
+    const double2* powtab = nullptr;  // powtab[t] = (beta1^t, beta2^t)
+    int64_t powtab_len = 0;
+    int grid_cap = 0;  // capacity of `partials`
+};
+
+// Rank pointer tables, sized for the largest R.
+struct RankPtrs {
+    const void* g[ZERO_MAX_RANKS];
+    float* acc[ZERO_MAX_RANKS];
+    float* master[2][ZERO_MAX_RANKS];
+    float* m[2][ZERO_MAX_RANKS];
+    float* v[2][ZERO_MAX_RANKS];
+    void* param[2][ZERO_MAX_RANKS];
+};
+
+// Kernel launchers (kernels.cu). Each returns the launch's cudaError_t.
+cudaError_t launch_fused_step(const StepParams& sp, const RankPtrs& p, cudaStream_t s);
+cudaError_t launch_step_from_acc(const StepParams& sp, const RankPtrs& p, cudaStream_t s);
+cudaError_t launch_reduce_scatter(int32_t R, int32_t dtype, int64_t S, int64_t lo, int64_t hi,
+                                  DevState* st, const RankPtrs& p, cudaStream_t s);
+cudaError_t launch_gather(int32_t R, int64_t S, int64_t lo, int64_t hi, const DevState* st,
+                          const RankPtrs& p, void* out, cudaStream_t s);
+
+// Grid the step kernels use for a given problem (for sizing `partials`).
+int step_grid_cap(int device);
+
+}  // namespace zb
+
+// Set the calling thread's last error message; returns `code`.
+zero_status zb_fail(zero_status code, const std::string& msg);

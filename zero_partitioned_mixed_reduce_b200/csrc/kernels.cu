@@ -1,0 +1,721 @@
+// CUDA kernels of the ZeRO data-parallel hot path for B200 (sm_100a).
+//
+// The path is bound by HBM bandwidth: about 20 floating-point operations per
+// parameter against 2R + 26 bytes moved (fused step), so there is no
+// contraction to put on tensor cores. Every kernel streams 8-element vectors
+// (16 bytes of half, 32 bytes of fp32 moved with one 256-bit access) through
+// a persistent grid of a few blocks per SM, keeps many loads in flight per
+// thread, and reduces flags and norms with warp shuffles and one shared-memory
+// pass per block. Global decisions (overflow, skip, loss-scale update) are
+// taken by the last block of the step kernel to finish, found with an atomic
+// counter, so no block ever waits on another and no extra launch is needed.
+//
+// Arithmetic matches include/zero_b200.h exactly: one IEEE fp32 operation per
+// step via __f*_rn intrinsics (the file is also built with --fmad=false),
+// IEEE division and square root, round-to-nearest-even casts to half that
+// keep subnormals and overflow to infinity.
+//
+// Pages (all titled "ZeRO Optimization"): inferensys legal pre-training and
+// instruction-tuning glossaries for the reduce-scatter, ZeRO-1/2/3 mechanism,
+// mixed-precision and loss-scaling bullets; inferensys genomic glossary for
+// the 2 + 2 + 12 bytes-per-parameter state.
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+
+#include <cfloat>
+#include <cstdint>
+#include <mutex>
+
+#include "internal.h"
+
+namespace zb {
+
+constexpr int kThreads = 256;
+constexpr int kWarps = kThreads / 32;
+
+// ---------------------------------------------------------------------------
+// Memory access helpers.
+// ---------------------------------------------------------------------------
+
+struct F8 {
+    float x[8];
+};
+
+// Gradients are read exactly once per step and never written by the step:
+// read-only path, no L1 allocation.
+__device__ __forceinline__ uint4 ld_grad(const uint4* p) {
+    uint4 r;
+    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+                 : "l"(p));
+    return r;
+}
+
+__device__ __forceinline__ uint16_t ld_grad1(const uint16_t* p) {
+    uint16_t r;
+    asm volatile("ld.global.nc.L1::no_allocate.u16 %0, [%1];" : "=h"(r) : "l"(p));
+    return r;
+}
+
+// 8 fp32 values with one 256-bit access (sm_100); p is 32-byte aligned.
+__device__ __forceinline__ F8 ld_f8(const float* p) {
+    F8 r;
+    asm volatile("ld.global.L1::no_allocate.v8.f32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+                 : "=f"(r.x[0]), "=f"(r.x[1]), "=f"(r.x[2]), "=f"(r.x[3]), "=f"(r.x[4]),
+                   "=f"(r.x[5]), "=f"(r.x[6]), "=f"(r.x[7])
+                 : "l"(p));
+    return r;
+}
+
+__device__ __forceinline__ void st_f8(float* p, const F8& v) {
+    asm volatile("st.global.v8.f32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"l"(p), "f"(v.x[0]),
+                 "f"(v.x[1]), "f"(v.x[2]), "f"(v.x[3]), "f"(v.x[4]), "f"(v.x[5]), "f"(v.x[6]),
+                 "f"(v.x[7])
+                 : "memory");
+}
+
+__device__ __forceinline__ void st_u4(void* p, const uint4& v) {
+    asm volatile("st.global.v4.u32 [%0], {%1,%2,%3,%4};" ::"l"(p), "r"(v.x), "r"(v.y), "r"(v.z),
+                 "r"(v.w)
+                 : "memory");
+}
+
+// ---------------------------------------------------------------------------
+// Half formats: two values per 32-bit word, element 0 in the low half.
+// ---------------------------------------------------------------------------
+
+struct Bf16 {
+    static __device__ __forceinline__ float2 unpack(uint32_t w) {
+        // a bf16 is the top half of the fp32 with the same value
+        return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
+    }
+    static __device__ __forceinline__ float one(uint16_t h) {
+        return __uint_as_float(static_cast<uint32_t>(h) << 16);
+    }
+    static __device__ __forceinline__ uint32_t pack(float lo, float hi) {
+        __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+        uint32_t w;
+        memcpy(&w, &h, 4);
+        return w;
+    }
+};
+
+struct Fp16 {
+    static __device__ __forceinline__ float2 unpack(uint32_t w) {
+        __half2 h;
+        memcpy(&h, &w, 4);
+        return __half22float2(h);
+    }
+    static __device__ __forceinline__ float one(uint16_t h) {
+        return __half2float(__ushort_as_half(h));
+    }
+    static __device__ __forceinline__ uint32_t pack(float lo, float hi) {
+        __half2 h = __floats2half2_rn(lo, hi);
+        uint32_t w;
+        memcpy(&w, &h, 4);
+        return w;
+    }
+};
+
+template <typename H>
+__device__ __forceinline__ void unpack8(const uint4& q, float* f) {
+    float2 a = H::unpack(q.x), b = H::unpack(q.y), c = H::unpack(q.z), d = H::unpack(q.w);
+    f[0] = a.x; f[1] = a.y; f[2] = b.x; f[3] = b.y;
+    f[4] = c.x; f[5] = c.y; f[6] = d.x; f[7] = d.y;
+}
+
+template <typename H>
+__device__ __forceinline__ void add8(const uint4& q, float* f) {
+    float g[8];
+    unpack8<H>(q, g);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) f[e] = __fadd_rn(f[e], g[e]);
+}
+
+template <typename H>
+__device__ __forceinline__ uint4 pack8(const float* f) {
+    return make_uint4(H::pack(f[0], f[1]), H::pack(f[2], f[3]), H::pack(f[4], f[5]),
+                      H::pack(f[6], f[7]));
+}
+
+__device__ __forceinline__ bool nonfinite(float x) { return !(fabsf(x) <= FLT_MAX); }
+
+// ---------------------------------------------------------------------------
+// AdamW on one element. Every line is one rounded fp32 operation.
+// ---------------------------------------------------------------------------
+
+struct Coef {
+    float inv, dec, b1f, omb1, b2f, omb2, epsf, ss, bc2s;
+};
+
+__device__ __forceinline__ float adamw1(const Coef& c, float acc, float& p, float& m, float& v) {
+    const float g = __fmul_rn(acc, c.inv);
+    float pp = __fmul_rn(p, c.dec);
+    const float mm = __fadd_rn(__fmul_rn(c.b1f, m), __fmul_rn(c.omb1, g));
+    const float vv = __fadd_rn(__fmul_rn(c.b2f, v), __fmul_rn(c.omb2, __fmul_rn(g, g)));
+    const float den = __fadd_rn(__fdiv_rn(__fsqrt_rn(vv), c.bc2s), c.epsf);
+    pp = __fsub_rn(pp, __fmul_rn(c.ss, __fdiv_rn(mm, den)));
+    p = pp;
+    m = mm;
+    v = vv;
+    return g;
+}
+
+// Per-step coefficients. scale and t live on the device (the loss-scale
+// state machine may skip steps without the host knowing), so the parts that
+// depend on them are formed here, in double, with the same IEEE operations
+// the host would use; beta^t comes from the host-built power table.
+__device__ __forceinline__ Coef make_coef(const StepParams& sp, int R, float scale, int64_t t1) {
+    Coef c;
+    const double dscale = sp.mode == ZERO_SCALE_NONE ? 1.0 : static_cast<double>(scale);
+    c.inv = __double2float_rn(__ddiv_rn(1.0, __dmul_rn(static_cast<double>(R), dscale)));
+    c.dec = sp.dec;
+    c.b1f = sp.b1f;
+    c.omb1 = sp.omb1;
+    c.b2f = sp.b2f;
+    c.omb2 = sp.omb2;
+    c.epsf = sp.epsf;
+    const double2 pw = sp.powtab[t1 < sp.powtab_len ? t1 : sp.powtab_len - 1];
+    c.ss = __double2float_rn(__ddiv_rn(sp.lr, __dsub_rn(1.0, pw.x)));
+    c.bc2s = __double2float_rn(__dsqrt_rn(__dsub_rn(1.0, pw.y)));
+    return c;
+}
+
+struct Prologue {
+    Coef c;
+    int src, dst, skip;
+};
+
+// Thread 0 of each block reads the device state once; the block shares it.
+__device__ __forceinline__ void read_prologue(const StepParams& sp, int R, Prologue* out,
+                                              bool skip_on_flag) {
+    if (threadIdx.x == 0) {
+        const volatile DevState* st = sp.st;
+        const float scale = st->scale;
+        const int64_t t1 = st->t + 1;
+        const int cur = st->cur;
+        if (t1 >= sp.powtab_len) sp.st->err = 1;  // host keeps the table ahead of t
+        out->c = make_coef(sp, R, scale, t1);
+        out->src = cur;
+        out->dst = sp.pingpong ? (cur ^ 1) : cur;
+        out->skip = skip_on_flag && sp.mode == ZERO_SCALE_DYNAMIC && st->flag != 0u;
+    }
+    __syncthreads();
+}
+
+// ---------------------------------------------------------------------------
+// Block reductions and the end-of-step decision.
+// ---------------------------------------------------------------------------
+
+__device__ __forceinline__ double warp_sum(double x) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
+    return x;
+}
+
+// Deterministic for a fixed grid: fixed per-thread order, fixed tree.
+__device__ double block_sum(double x, double* smem) {
+    x = warp_sum(x);
+    const int w = threadIdx.x >> 5, l = threadIdx.x & 31;
+    __syncthreads();
+    if (l == 0) smem[w] = x;
+    __syncthreads();
+    double r = 0.0;
+    if (w == 0) {
+        r = l < kWarps ? smem[l] : 0.0;
+        r = warp_sum(r);
+    }
+    return r;  // valid in thread 0
+}
+
+// Loss-scale state machine; one thread. Same rules as the header states.
+__device__ void fsm_update(const StepParams& sp, DevState* st, double norm) {
+    const uint32_t ovf = *reinterpret_cast<volatile uint32_t*>(&st->flag);
+    int skipped = 0;
+    if (sp.mode == ZERO_SCALE_DYNAMIC) {
+        if (ovf) {
+            const float s = __fmul_rn(st->scale, sp.backoff);
+            st->scale = (s < sp.min_scale) ? sp.min_scale : s;
+            st->good = 0;
+            skipped = 1;
+        } else {
+            st->t = st->t + 1;
+            st->good = st->good + 1;
+            if (st->good >= sp.interval) {
+                st->scale = __fmul_rn(st->scale, sp.growth);
+                st->good = 0;
+            }
+            if (sp.pingpong) st->cur ^= 1;
+        }
+    } else {
+        st->t = st->t + 1;
+        if (sp.pingpong) st->cur ^= 1;
+    }
+    st->last_overflow = ovf ? 1 : 0;
+    st->last_skipped = skipped;
+    st->grad_norm_sq = norm;
+    st->flag = 0u;
+    st->done = 0u;
+    __threadfence();
+}
+
+// Every block publishes its norm partial and flag; the last block to finish
+// sums the partials in block order and runs the state machine.
+__device__ void step_epilogue(const StepParams& sp, double nrm, bool bad) {
+    __shared__ double red[kWarps];
+    __shared__ int last;
+    const double bn = block_sum(nrm, red);
+    const int any_bad = __syncthreads_or(bad ? 1 : 0);
+    if (threadIdx.x == 0) {
+        sp.partials[blockIdx.x] = bn;
+        if (any_bad) atomicOr(&sp.st->flag, 1u);
+        __threadfence();
+        const unsigned prev = atomicAdd(&sp.st->done, 1u);
+        last = (prev == gridDim.x - 1);
+    }
+    __syncthreads();
+    if (!last) return;
+    __threadfence();
+    double x = 0.0;
+    for (unsigned i = threadIdx.x; i < gridDim.x; i += kThreads)
+        x += *reinterpret_cast<volatile double*>(&sp.partials[i]);
+    const double total = block_sum(x, red);
+    if (threadIdx.x == 0) fsm_update(sp, sp.st, total);
+}
+
+// Owner of a flat vector index, tracked incrementally along a grid-stride loop.
+struct OwnerCursor {
+    uint32_t o, base, S8;
+    __device__ __forceinline__ OwnerCursor(uint32_t v, uint32_t s8) : S8(s8) {
+        o = v / s8;
+        base = o * s8;
+    }
+    __device__ __forceinline__ void seek(uint32_t v) {
+        while (v - base >= S8) {
+            base += S8;
+            ++o;
+        }
+    }
+};
+
+// ---------------------------------------------------------------------------
+// Fused reduce-scatter + unscale + overflow check + AdamW + cast.
+// One pass: read R gradient vectors and master/m/v, write master/m/v/param.
+// ---------------------------------------------------------------------------
+
+template <int CAP>
+struct FusedArgs {
+    StepParams sp;
+    const uint4* g[CAP];
+    float* master[2][CAP];
+    float* m[2][CAP];
+    float* v[2][CAP];
+    uint4* param[2][CAP];
+};
+
+template <typename H, int RC>
+__global__ void __launch_bounds__(kThreads)
+    fused_step_kernel(const __grid_constant__ FusedArgs<RC == 0 ? ZERO_MAX_RANKS : RC> a) {
+    const StepParams& sp = a.sp;
+    const int R = RC > 0 ? RC : sp.R;
+    __shared__ Prologue pro;
+    read_prologue(sp, R, &pro, false);
+    const Coef c = pro.c;
+    const int src = pro.src, dst = pro.dst;
+
+    double nrm = 0.0;
+    bool bad = false;
+    const uint32_t stride = gridDim.x * kThreads;
+    uint32_t vi = blockIdx.x * kThreads + threadIdx.x;
+    OwnerCursor oc(vi, sp.S8);
+    for (; vi < sp.T8; vi += stride) {
+        oc.seek(vi);
+        const uint32_t o = oc.o;
+        const size_t j8 = static_cast<size_t>(vi - oc.base) * 8;
+        float acc[8];
+        F8 p, m, v;
+        if constexpr (RC > 0) {
+            uint4 gv[RC];
+#pragma unroll
+            for (int r = 0; r < RC; ++r) gv[r] = ld_grad(a.g[r] + vi);
+            p = ld_f8(a.master[src][o] + j8);
+            m = ld_f8(a.m[src][o] + j8);
+            v = ld_f8(a.v[src][o] + j8);
+            unpack8<H>(gv[0], acc);
+#pragma unroll
+            for (int r = 1; r < RC; ++r) add8<H>(gv[r], acc);
+        } else {
+            uint4 g0 = ld_grad(a.g[0] + vi);
+            p = ld_f8(a.master[src][o] + j8);
+            m = ld_f8(a.m[src][o] + j8);
+            v = ld_f8(a.v[src][o] + j8);
+            unpack8<H>(g0, acc);
+#pragma unroll 4
+            for (int r = 1; r < R; ++r) add8<H>(ld_grad(a.g[r] + vi), acc);
+        }
+        float out[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+            bad |= nonfinite(acc[e]);
+            const float g = adamw1(c, acc[e], p.x[e], m.x[e], v.x[e]);
+            const double gd = static_cast<double>(g);
+            nrm = fma(gd, gd, nrm);
+            out[e] = p.x[e];
+        }
+        st_f8(a.master[dst][o] + j8, p);
+        st_f8(a.m[dst][o] + j8, m);
+        st_f8(a.v[dst][o] + j8, v);
+        st_u4(a.param[dst][o] + (j8 >> 3), pack8<H>(out));
+    }
+    step_epilogue(sp, nrm, bad);
+}
+
+// ---------------------------------------------------------------------------
+// Two-pass step: AdamW from the fp32 accumulators written by the
+// reduce-scatter kernel. In place on set cur; skipped (state untouched) in
+// DYNAMIC mode when the reduce-scatter raised the overflow flag. The norm is
+// always formed from the accumulators.
+// ---------------------------------------------------------------------------
+
+struct AccArgs {
+    StepParams sp;
+    const float* acc[ZERO_MAX_RANKS];
+    float* master[2][ZERO_MAX_RANKS];
+    float* m[2][ZERO_MAX_RANKS];
+    float* v[2][ZERO_MAX_RANKS];
+    uint4* param[2][ZERO_MAX_RANKS];
+};
+
+template <typename H>
+__global__ void __launch_bounds__(kThreads) step_from_acc_kernel(const __grid_constant__ AccArgs a) {
+    const StepParams& sp = a.sp;
+    __shared__ Prologue pro;
+    read_prologue(sp, sp.R, &pro, true);
+    const Coef c = pro.c;
+    const int cur = pro.src;
+    const bool skip = pro.skip != 0;
+
+    double nrm = 0.0;
+    const uint32_t stride = gridDim.x * kThreads;
+    uint32_t vi = blockIdx.x * kThreads + threadIdx.x;
+    OwnerCursor oc(vi, sp.S8);
+    for (; vi < sp.T8; vi += stride) {
+        oc.seek(vi);
+        const uint32_t o = oc.o;
+        const size_t j8 = static_cast<size_t>(vi - oc.base) * 8;
+        const F8 acc = ld_f8(a.acc[o] + j8);
+        if (skip) {
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                const double gd = static_cast<double>(__fmul_rn(acc.x[e], c.inv));
+                nrm = fma(gd, gd, nrm);
+            }
+            continue;
+        }
+        F8 p = ld_f8(a.master[cur][o] + j8);
+        F8 m = ld_f8(a.m[cur][o] + j8);
+        F8 v = ld_f8(a.v[cur][o] + j8);
+        float out[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+            const float g = adamw1(c, acc.x[e], p.x[e], m.x[e], v.x[e]);
+            const double gd = static_cast<double>(g);
+            nrm = fma(gd, gd, nrm);
+            out[e] = p.x[e];
+        }
+        st_f8(a.master[cur][o] + j8, p);
+        st_f8(a.m[cur][o] + j8, m);
+        st_f8(a.v[cur][o] + j8, v);
+        st_u4(a.param[cur][o] + (j8 >> 3), pack8<H>(out));
+    }
+    step_epilogue(sp, nrm, false);
+}
+
+// ---------------------------------------------------------------------------
+// Bucketed reduce-scatter into the owners' fp32 accumulators.
+// Flat range [lo, hi): an unaligned head and tail are done element by
+// element, the aligned body with 8-element vectors (S is a multiple of 8, so
+// an aligned vector never straddles two shards).
+// ---------------------------------------------------------------------------
+
+template <int CAP>
+struct RsArgs {
+    int64_t lo, hi, S;
+    uint32_t S8, v0, v1;   // aligned body in vectors: [v0, v1)
+    int64_t head_end, tail_begin;
+    int32_t R;
+    DevState* st;
+    const uint4* g[CAP];
+    float* acc[CAP];
+};
+
+template <typename H, int RC>
+__global__ void __launch_bounds__(kThreads)
+    reduce_scatter_kernel(const __grid_constant__ RsArgs<RC == 0 ? ZERO_MAX_RANKS : RC> a) {
+    const int R = RC > 0 ? RC : a.R;
+    bool bad = false;
+    const uint32_t stride = gridDim.x * kThreads;
+    const uint32_t tid = blockIdx.x * kThreads + threadIdx.x;
+    uint32_t vi = a.v0 + tid;
+    OwnerCursor oc(vi, a.S8);
+    for (; vi < a.v1; vi += stride) {
+        oc.seek(vi);
+        float acc[8];
+        if constexpr (RC > 0) {
+            uint4 gv[RC];
+#pragma unroll
+            for (int r = 0; r < RC; ++r) gv[r] = ld_grad(a.g[r] + vi);
+            unpack8<H>(gv[0], acc);
+#pragma unroll
+            for (int r = 1; r < RC; ++r) add8<H>(gv[r], acc);
+        } else {
+            unpack8<H>(ld_grad(a.g[0] + vi), acc);
+#pragma unroll 4
+            for (int r = 1; r < R; ++r) add8<H>(ld_grad(a.g[r] + vi), acc);
+        }
+        F8 out;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+            bad |= nonfinite(acc[e]);
+            out.x[e] = acc[e];
+        }
+        st_f8(a.acc[oc.o] + static_cast<size_t>(vi - oc.base) * 8, out);
+    }
+    // unaligned edges, element by element
+    const int64_t nhead = a.head_end - a.lo;
+    const int64_t ntail = a.hi - a.tail_begin;
+    if (tid < nhead + ntail) {
+        const int64_t i = tid < nhead ? a.lo + tid : a.tail_begin + (tid - nhead);
+        const int64_t o = i / a.S;
+        float s = H::one(ld_grad1(reinterpret_cast<const uint16_t*>(a.g[0]) + i));
+        for (int r = 1; r < R; ++r)
+            s = __fadd_rn(s, H::one(ld_grad1(reinterpret_cast<const uint16_t*>(a.g[r]) + i)));
+        bad |= nonfinite(s);
+        a.acc[o][i - o * a.S] = s;
+    }
+    if (__syncthreads_or(bad ? 1 : 0) && threadIdx.x == 0) atomicOr(&a.st->flag, 1u);
+}
+
+// ---------------------------------------------------------------------------
+// ZeRO-3 layer gather from the current parameter set.
+// ---------------------------------------------------------------------------
+
+struct GatherArgs {
+    int64_t lo, n, S;  // flat start, element count, shard length
+    uint32_t S8;
+    int32_t aligned;   // lo % 8 == 0
+    const DevState* st;
+    const uint16_t* param[2][ZERO_MAX_RANKS];
+    uint16_t* out;
+};
+
+__global__ void __launch_bounds__(kThreads) gather_kernel(const __grid_constant__ GatherArgs a) {
+    __shared__ int s_cur;
+    if (threadIdx.x == 0) s_cur = reinterpret_cast<const volatile DevState*>(a.st)->cur;
+    __syncthreads();
+    const int cur = s_cur;
+    const uint32_t stride = gridDim.x * kThreads;
+    const uint32_t tid = blockIdx.x * kThreads + threadIdx.x;
+    int64_t done = 0;
+    if (a.aligned) {
+        const uint32_t n8 = static_cast<uint32_t>(a.n / 8);
+        const uint32_t vlo = static_cast<uint32_t>(a.lo / 8);
+        uint32_t vj = tid;
+        OwnerCursor oc(vlo + vj, a.S8);
+        for (; vj < n8; vj += stride) {
+            const uint32_t vi = vlo + vj;
+            oc.seek(vi);
+            const uint4 q = ld_grad(reinterpret_cast<const uint4*>(a.param[cur][oc.o]) + (vi - oc.base));
+            st_u4(a.out + static_cast<size_t>(vj) * 8, q);
+        }
+        done = static_cast<int64_t>(n8) * 8;
+    }
+    for (int64_t j = done + tid; j < a.n; j += stride) {
+        const int64_t i = a.lo + j;
+        const int64_t o = i / a.S;
+        a.out[j] = ld_grad1(a.param[cur][o] + (i - o * a.S));
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Launchers.
+// ---------------------------------------------------------------------------
+
+namespace {
+
+struct DeviceInfo {
+    int sms = 0;
+};
+
+DeviceInfo& device_info(int dev) {
+    static DeviceInfo infos[64];
+    static std::once_flag flags[64];
+    std::call_once(flags[dev & 63], [&] {
+        cudaDeviceGetAttribute(&infos[dev & 63].sms, cudaDevAttrMultiProcessorCount, dev);
+    });
+    return infos[dev & 63];
+}
+
+int current_sms() {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    return device_info(dev).sms;
+}
+
+template <typename K>
+int blocks_per_sm(K kernel) {
+    int n = 0;
+    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kernel, kThreads, 0);
+    return n > 0 ? n : 1;
+}
+
+uint32_t grid_for(uint64_t work_items, int per_sm, int cap) {
+    const uint64_t need = (work_items + kThreads - 1) / kThreads;
+    uint64_t g = static_cast<uint64_t>(current_sms()) * static_cast<uint64_t>(per_sm);
+    if (g > need) g = need;
+    if (cap > 0 && g > static_cast<uint64_t>(cap)) g = cap;
+    return static_cast<uint32_t>(g > 0 ? g : 1);
+}
+
+template <typename H, int RC>
+cudaError_t fused_t(const StepParams& sp, const RankPtrs& p, cudaStream_t s) {
+    constexpr int CAP = RC == 0 ? ZERO_MAX_RANKS : RC;
+    FusedArgs<CAP> a;
+    a.sp = sp;
+    for (int r = 0; r < sp.R; ++r) {
+        a.g[r] = static_cast<const uint4*>(p.g[r]);
+        for (int k = 0; k < 2; ++k) {
+            a.master[k][r] = p.master[k][r];
+            a.m[k][r] = p.m[k][r];
+            a.v[k][r] = p.v[k][r];
+            a.param[k][r] = static_cast<uint4*>(p.param[k][r]);
+        }
+    }
+    static const int per_sm = blocks_per_sm(fused_step_kernel<H, RC>);
+    const uint32_t grid = grid_for(sp.T8, per_sm, sp.grid_cap);
+    fused_step_kernel<H, RC><<<grid, kThreads, 0, s>>>(a);
+    return cudaGetLastError();
+}
+
+template <typename H>
+cudaError_t fused_dispatch(const StepParams& sp, const RankPtrs& p, cudaStream_t s) {
+    switch (sp.R) {
+        case 1: return fused_t<H, 1>(sp, p, s);
+        case 2: return fused_t<H, 2>(sp, p, s);
+        case 4: return fused_t<H, 4>(sp, p, s);
+        case 8: return fused_t<H, 8>(sp, p, s);
+        case 16: return fused_t<H, 16>(sp, p, s);
+        default: return fused_t<H, 0>(sp, p, s);
+    }
+}
+
+template <typename H, int RC>
+cudaError_t rs_t(int32_t R, int64_t S, int64_t lo, int64_t hi, DevState* st, const RankPtrs& p,
+                 cudaStream_t s) {
+    constexpr int CAP = RC == 0 ? ZERO_MAX_RANKS : RC;
+    RsArgs<CAP> a;
+    a.lo = lo;
+    a.hi = hi;
+    a.S = S;
+    a.S8 = static_cast<uint32_t>(S / 8);
+    a.R = R;
+    a.st = st;
+    // aligned body [ceil8(lo), floor8(hi)), if non-empty
+    const int64_t vlo = (lo + 7) / 8, vhi = hi / 8;
+    if (vlo < vhi) {
+        a.v0 = static_cast<uint32_t>(vlo);
+        a.v1 = static_cast<uint32_t>(vhi);
+        a.head_end = vlo * 8;
+        a.tail_begin = vhi * 8;
+    } else {
+        a.v0 = a.v1 = 0;
+        a.head_end = hi;  // everything is "head"
+        a.tail_begin = hi;
+    }
+    for (int r = 0; r < R; ++r) {
+        a.g[r] = static_cast<const uint4*>(p.g[r]);
+        a.acc[r] = p.acc[r];
+    }
+    static const int per_sm = blocks_per_sm(reduce_scatter_kernel<H, RC>);
+    const uint64_t items = static_cast<uint64_t>(a.v1 - a.v0);
+    const uint64_t edges = static_cast<uint64_t>((a.head_end - lo) + (hi - a.tail_begin));
+    const uint32_t grid = grid_for(items > edges ? items : edges, per_sm, 0);
+    reduce_scatter_kernel<H, RC><<<grid, kThreads, 0, s>>>(a);
+    return cudaGetLastError();
+}
+
+template <typename H>
+cudaError_t rs_dispatch(int32_t R, int64_t S, int64_t lo, int64_t hi, DevState* st,
+                        const RankPtrs& p, cudaStream_t s) {
+    switch (R) {
+        case 1: return rs_t<H, 1>(R, S, lo, hi, st, p, s);
+        case 2: return rs_t<H, 2>(R, S, lo, hi, st, p, s);
+        case 4: return rs_t<H, 4>(R, S, lo, hi, st, p, s);
+        case 8: return rs_t<H, 8>(R, S, lo, hi, st, p, s);
+        case 16: return rs_t<H, 16>(R, S, lo, hi, st, p, s);
+        default: return rs_t<H, 0>(R, S, lo, hi, st, p, s);
+    }
+}
+
+template <typename H>
+cudaError_t acc_t(const StepParams& sp, const RankPtrs& p, cudaStream_t s) {
+    AccArgs a;
+    a.sp = sp;
+    for (int r = 0; r < sp.R; ++r) {
+        a.acc[r] = p.acc[r];
+        for (int k = 0; k < 2; ++k) {
+            a.master[k][r] = p.master[k][r];
+            a.m[k][r] = p.m[k][r];
+            a.v[k][r] = p.v[k][r];
+            a.param[k][r] = static_cast<uint4*>(p.param[k][r]);
+        }
+    }
+    static const int per_sm = blocks_per_sm(step_from_acc_kernel<H>);
+    const uint32_t grid = grid_for(sp.T8, per_sm, sp.grid_cap);
+    step_from_acc_kernel<H><<<grid, kThreads, 0, s>>>(a);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_fused_step(const StepParams& sp, const RankPtrs& p, cudaStream_t s) {
+    return sp.dtype == ZERO_FP16 ? fused_dispatch<Fp16>(sp, p, s) : fused_dispatch<Bf16>(sp, p, s);
+}
+
+cudaError_t launch_step_from_acc(const StepParams& sp, const RankPtrs& p, cudaStream_t s) {
+    return sp.dtype == ZERO_FP16 ? acc_t<Fp16>(sp, p, s) : acc_t<Bf16>(sp, p, s);
+}
+
+cudaError_t launch_reduce_scatter(int32_t R, int32_t dtype, int64_t S, int64_t lo, int64_t hi,
+                                  DevState* st, const RankPtrs& p, cudaStream_t s) {
+    return dtype == ZERO_FP16 ? rs_dispatch<Fp16>(R, S, lo, hi, st, p, s)
+                              : rs_dispatch<Bf16>(R, S, lo, hi, st, p, s);
+}
+
+cudaError_t launch_gather(int32_t R, int64_t S, int64_t lo, int64_t hi, const DevState* st,
+                          const RankPtrs& p, void* out, cudaStream_t s) {
+    GatherArgs a;
+    a.lo = lo;
+    a.n = hi - lo;
+    a.S = S;
+    a.S8 = static_cast<uint32_t>(S / 8);
+    a.aligned = (lo % 8) == 0;
+    a.st = st;
+    for (int r = 0; r < R; ++r)
+        for (int k = 0; k < 2; ++k) a.param[k][r] = static_cast<const uint16_t*>(p.param[k][r]);
+    a.out = static_cast<uint16_t*>(out);
+    if (a.n <= 0) return cudaSuccess;
+    static const int per_sm = blocks_per_sm(gather_kernel);
+    const uint64_t items = a.aligned ? static_cast<uint64_t>(a.n / 8) : static_cast<uint64_t>(a.n);
+    const uint32_t grid = grid_for(items > 0 ? items : 1, per_sm, 0);
+    gather_kernel<<<grid, kThreads, 0, s>>>(a);
+    return cudaGetLastError();
+}
+
+int step_grid_cap(int device) {
+    // at most 8 blocks of 256 threads fit on an SM
+    return device_info(device).sms * 8;
+}
+
+}  // namespace zb
