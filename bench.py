@@ -25,9 +25,7 @@ import hashlib
 import json
 import os
 import statistics
-import subprocess
 import sys
-import tempfile
 import time
 
 import numpy as np
@@ -44,13 +42,15 @@ FALLBACK_HBM_GBS = 6650.0
 def parse_args(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.splitlines()[1])
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=100)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="gpt2s")
     ap.add_argument("--path", choices=["auto", "pingpong", "inplace", "twopass"], default="auto")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--first-tensors", type=int, default=0,
+                    help="use only the first N tensors of the workload (small profiling cases)")
     return ap.parse_args(argv)
 
 
@@ -93,50 +93,65 @@ def aggregate(ms_local, units_local, world):
 # ---- clocks -----------------------------------------------------------------
 
 class ClockSampler:
-    """nvidia-smi samples of SM clock and throttle reasons during a region."""
+    """SM clock and clock-event (throttle) reasons sampled through NVML from a
+    background thread every ~2 ms while the timed region runs."""
 
-    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown"}
 
     def __init__(self, device_index):
         self.dev = device_index
-        self.proc = None
-        self.file = None
+        self.samples = []
+        self.thread = None
+        self.stop_flag = False
+        self.nvml = None
+
+    def _handle(self):
+        import pynvml as N
+        N.nvmlInit()
+        self.nvml = N
+        try:
+            uuid = str(torch.cuda.get_device_properties(self.dev).uuid)
+            return N.nvmlDeviceGetHandleByUUID("GPU-" + uuid)
+        except Exception:
+            return N.nvmlDeviceGetHandleByIndex(self.dev)
+
+    def _run(self, h):
+        N = self.nvml
+        get_reasons = getattr(N, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+            N.nvmlDeviceGetCurrentClocksThrottleReasons
+        while not self.stop_flag:
+            try:
+                sm = N.nvmlDeviceGetClockInfo(h, N.NVML_CLOCK_SM)
+                rs = get_reasons(h)
+                self.samples.append((sm, rs))
+            except Exception:
+                pass
+            time.sleep(0.002)
 
     def start(self):
+        import threading
         try:
-            self.file = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
-                 "-i", str(self.dev), "-lms", "100"], stdout=self.file, stderr=subprocess.DEVNULL)
-        except (OSError, FileNotFoundError):
-            self.proc = None
+            h = self._handle()
+            self.max_mhz = self.nvml.nvmlDeviceGetMaxClockInfo(h, self.nvml.NVML_CLOCK_SM)
+        except Exception:
+            self.thread = None
+            return
+        self.thread = threading.Thread(target=self._run, args=(h,), daemon=True)
+        self.thread.start()
 
     def stop(self):
-        if self.proc is None:
+        if self.thread is None:
             return None
-        self.proc.terminate()
-        try:
-            self.proc.wait(timeout=5)
-        except subprocess.TimeoutExpired:
-            self.proc.kill()
-        self.file.flush()
-        rows = []
-        with open(self.file.name) as f:
-            for line in f:
-                parts = [p.strip() for p in line.split(",")]
-                if len(parts) == 9:
-                    rows.append(parts)
-        os.unlink(self.file.name)
-        if not rows:
+        self.stop_flag = True
+        self.thread.join(timeout=5)
+        if not self.samples:
             return None
-        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
-        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({n for r in rows for n, v in zip(names, r[5:9]) if v == "Active"})
-        return {"sm_mhz": statistics.median(sm) if sm else None,
-                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons, "samples": len(rows)}
+        sm = [s for s, _ in self.samples]
+        reasons = sorted({name for _, rs in self.samples for bit, name in self.REASONS.items()
+                          if rs & bit})
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": self.max_mhz, "reasons": reasons,
+                "samples": len(sm), "source": "nvml"}
 
 
 # ---- peaks and profile-derived traffic --------------------------------------
@@ -150,9 +165,12 @@ def hbm_peak():
 
 
 def kernels_sha():
-    p = os.path.join(ROOT, "zero_partitioned_mixed_reduce_b200", "csrc", "kernels.cu")
-    with open(p, "rb") as f:
-        return hashlib.sha256(f.read()).hexdigest()[:16]
+    """Hash of the step kernels' source (kernels.cu and its device header)."""
+    h = hashlib.sha256()
+    for name in ("kernels.cu", "device_common.cuh"):
+        with open(os.path.join(ROOT, "zero_partitioned_mixed_reduce_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
 
 
 def profiled_traffic(kernel, workload):
@@ -173,11 +191,14 @@ def profiled_traffic(kernel, workload):
 # ---- the workload -------------------------------------------------------------
 
 class Bench:
-    def __init__(self, name, path):
+    def __init__(self, name, path, first_tensors=0):
         import zero_partitioned_mixed_reduce_b200 as Z
         from zero_partitioned_mixed_reduce_b200 import synth
         self.Z, self.synth = Z, synth
         self.wl = wl = synth.workload(name)
+        if first_tensors:
+            wl["numels"] = wl["numels"][:first_tensors]
+            wl["layer_ids"] = wl["layer_ids"][:first_tensors] if wl["layer_ids"] else None
         self.R, self.dtype = wl["R"], wl["dtype"]
         if path == "auto":
             path = "pingpong" if wl["mode"] == synth.DYNAMIC else "inplace"
@@ -259,7 +280,7 @@ def run_ours(args, world, rank, local):
     if not torch.cuda.is_available():
         print(json.dumps({"error": "no CUDA device: the benchmark has no CPU fallback"}))
         sys.exit(1)
-    b = Bench(args.workload, args.path)
+    b = Bench(args.workload, args.path, args.first_tensors)
     stream = torch.cuda.current_stream()
     for _ in range(args.warmup):
         b.step(stream)
@@ -311,7 +332,9 @@ def run_ours(args, world, rank, local):
         "hbm_gbs": step_bytes * K * world / (ms * 1e-3) / 1e9,
         "hbm_frac_of_peak": step_bytes * K / (ms * 1e-3) / 1e9 / peak,
         "config": {
-            "workload": f"{args.workload}: {len(b.wl['numels'])} tensors, P={b.P}, R={b.R} "
+            "workload": f"{args.workload}"
+                        f"{f' (first {args.first_tensors} tensors)' if args.first_tensors else ''}"
+                        f": {len(b.wl['numels'])} tensors, P={b.P}, R={b.R} "
                         f"simulated ranks, {'fp16' if b.dtype else 'bf16'} grads, "
                         f"loss scale mode {b.wl['mode']}",
             "R": b.R, "P": b.P, "T": b.T, "S": b.S, "n_layers": len(b.plan.layers),

@@ -29,7 +29,7 @@ CPP_SOURCES = ["plan.cpp", "capi.cpp"]
 
 
 def _sources():
-    return ([os.path.join(CSRC, s) for s in CU_SOURCES + CPP_SOURCES + ["internal.h"]]
+    return ([os.path.join(CSRC, s) for s in CU_SOURCES + CPP_SOURCES + ["internal.h", "device_common.cuh"]]
             + [os.path.join(INCLUDE, "zero_b200.h")])
 
 
