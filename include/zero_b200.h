@@ -300,6 +300,46 @@ typedef struct {
 zero_status zero_loss_scale(zero_ctx_t* ctx, zero_loss_scale_state* inout, int32_t op,
                             void* stream);
 
+/*
+ * zero_step_noalloc -- the two-pass step (reduce-scatter of all R replicas
+ * into fp32 accumulators, then the AdamW step above, in place on one state
+ * set) for callers that cannot allocate device memory: processes whose GPU
+ * memory is owned by another allocator that has already reserved it, and
+ * loops that may not call cudaMalloc or cudaFree because those calls
+ * synchronize the device or can fail mid-run. This call allocates nothing
+ * and needs no context: its scratch (the accumulators, the per-block norm
+ * partials and a control word) lives in one static device array of
+ * 16 MiB + 32 KiB + 256 B that every GPU loading this library holds until
+ * the process exits. The pages have no counterpart to this entry point; it
+ * is a deployment variant of zero_reduce_scatter_bucket(-1) + zero_step
+ * (grads == NULL) and gives the same results.
+ *
+ * plan: the layout (host only); its padded length T must be at most
+ * ZERO_NOALLOC_MAX_ELEMS, else ZERO_ERR_RANGE. cfg: loss-scale mode and
+ * rules as for zero_ctx_create. inout: HOST memory; the loss-scale state
+ * before the step (cur must be 0), overwritten with the state after it.
+ * grads: R device pointers to full half replicas of T elements; master, m, v
+ * (fp32, 32-byte aligned) and param (half, 16-byte aligned): R device
+ * pointers to the shards of S elements, updated in place.
+ *
+ * Set-up: the first call on each device (with that device current) looks up
+ * the device address of the static scratch; make that first call before any
+ * stream capture begins. Every call shares the same scratch and leaves the
+ * last call's contents in it (the control word is cleared at the start of
+ * each call). Calls whose work overlaps on the GPU -- two streams, two host
+ * threads, or two devices' calls racing on one device -- race on the
+ * scratch and give wrong results; serialize them. The call synchronizes
+ * `stream` before it returns (it reads the overflow flag and the norm back
+ * to update `inout`).
+ * Errors: ZERO_ERR_RANGE (model too large), ZERO_ERR_INVALID_ARG,
+ * ZERO_ERR_ALIGN, ZERO_ERR_CUDA.
+ */
+#define ZERO_NOALLOC_MAX_ELEMS 4194304
+zero_status zero_step_noalloc(const zero_plan_t* plan, const zero_loss_scale_config* cfg,
+                              zero_loss_scale_state* inout, const zero_adamw* hp,
+                              const void* const* grads, float* const* master, float* const* m,
+                              float* const* v, void* const* param, void* stream);
+
 /* zero_sync -- synchronize `stream` and report any pending CUDA error. */
 zero_status zero_sync(zero_ctx_t* ctx, void* stream);
 

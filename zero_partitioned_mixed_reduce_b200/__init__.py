@@ -11,5 +11,5 @@ from ._capi import (  # noqa: F401
     zero_adamw, zero_ctx_create, zero_ctx_destroy, zero_gather_layer, zero_last_error,
     zero_loss_scale, zero_plan, zero_plan_bucket, zero_plan_destroy, zero_plan_get_info,
     zero_plan_layer, zero_plan_memory, zero_plan_tensor, zero_reduce_scatter_bucket, zero_step,
-    zero_sync, zero_version)
+    zero_step_noalloc, ZERO_NOALLOC_MAX_ELEMS, zero_sync, zero_version)
 from .state import Plan, ShardedState  # noqa: F401

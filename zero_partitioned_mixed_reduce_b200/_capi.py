@@ -98,6 +98,9 @@ _sig("zero_reduce_scatter_bucket", _S, [_P, C.c_int64, _PP, _PP, _P])
 _sig("zero_step", _S, [_P, C.POINTER(zero_adamw), C.POINTER(zero_state), _PP, _P])
 _sig("zero_gather_layer", _S, [_P, C.c_int64, C.POINTER(zero_state), _P, _P])
 _sig("zero_loss_scale", _S, [_P, C.POINTER(zero_loss_scale_state), C.c_int32, _P])
+_sig("zero_step_noalloc", _S, [_P, C.POINTER(zero_loss_scale_config),
+                               C.POINTER(zero_loss_scale_state), C.POINTER(zero_adamw), _PP, _PP,
+                               _PP, _PP, _PP, _P])
 _sig("zero_sync", _S, [_P, _P])
 _sig("zero_last_error", C.c_size_t, [C.c_char_p, C.c_size_t])
 _sig("zero_version", C.c_char_p, [])
@@ -249,6 +252,31 @@ def zero_loss_scale(ctx, op=ZERO_LOSS_SCALE_GET, state=None, stream=None):
         else:
             st = state
     _check(_lib.zero_loss_scale(ctx, C.byref(st), op, _stream(stream)))
+    return {k: getattr(st, k) for k, _ in zero_loss_scale_state._fields_}
+
+
+ZERO_NOALLOC_MAX_ELEMS = 4194304
+
+
+def zero_step_noalloc(plan, cfg, state, hp, grads, master, m, v, param, stream=None):
+    """The two-pass step without any device allocation (see the header).
+
+    cfg: dict with mode, growth_interval, growth_factor, backoff_factor,
+    min_scale (init_scale is ignored: the scale comes from `state`). state:
+    dict with scale, cur (0), good, t (and optionally the last_* fields).
+    Returns the loss-scale state after the step. Synchronizes `stream`."""
+    c = zero_loss_scale_config(cfg.get("mode", ZERO_SCALE_NONE), 1.0,
+                               cfg.get("growth_interval", 1000), cfg.get("growth_factor", 2.0),
+                               cfg.get("backoff_factor", 0.5), cfg.get("min_scale", 1.0), 0)
+    st = zero_loss_scale_state()
+    for k, _ in zero_loss_scale_state._fields_:
+        if k in state:
+            setattr(st, k, state[k])
+    if isinstance(hp, dict):
+        hp = zero_adamw(hp["lr"], hp["beta1"], hp["beta2"], hp["eps"], hp["weight_decay"])
+    arrays = [_ptr_array(x) for x in (grads, master, m, v, param)]
+    _check(_lib.zero_step_noalloc(plan, C.byref(c), C.byref(st), C.byref(hp),
+                                  *[a[0] for a in arrays], _stream(stream)))
     return {k: getattr(st, k) for k, _ in zero_loss_scale_state._fields_}
 
 

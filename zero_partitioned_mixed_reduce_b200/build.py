@@ -24,7 +24,7 @@ NVCC_FLAGS = ["-O3", "-std=c++17", *ARCH, "-lineinfo", "--fmad=false", "-Xptxas"
 CXX_FLAGS = ["-O2", "-std=c++17", "-fPIC", "-Wall", "-Wextra", "-I", INCLUDE, "-I", CSRC,
              "-I", os.path.join(CUDA_HOME, "include")]
 
-CU_SOURCES = ["kernels.cu"]
+CU_SOURCES = ["kernels.cu", "noalloc.cu"]
 CPP_SOURCES = ["plan.cpp", "capi.cpp"]
 
 
