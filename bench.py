@@ -49,6 +49,9 @@ def parse_args(argv=None):
     ap.add_argument("--path", choices=["auto", "pingpong", "inplace", "twopass"], default="auto")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--gather-bucket", type=int, default=32 << 20,
+                    help="gather consecutive layers in one launch up to this many elements "
+                         "(0: one launch per layer)")
     ap.add_argument("--first-tensors", type=int, default=0,
                     help="use only the first N tensors of the workload (small profiling cases)")
     return ap.parse_args(argv)
@@ -191,7 +194,7 @@ def profiled_traffic(kernel, workload):
 # ---- the workload -------------------------------------------------------------
 
 class Bench:
-    def __init__(self, name, path, first_tensors=0):
+    def __init__(self, name, path, first_tensors=0, gather_bucket=32 << 20):
         import zero_partitioned_mixed_reduce_b200 as Z
         from zero_partitioned_mixed_reduce_b200 import synth
         self.Z, self.synth = Z, synth
@@ -227,7 +230,26 @@ class Bench:
         self.ctx = Z.zero_ctx_create(self.plan.handle, wl["mode"], wl["init_scale"],
                                      wl["interval"])
         self.max_layer = max(hi - lo for lo, hi in self.plan.layers)
-        self.layer_buf = torch.empty(self.max_layer, dtype=half, device="cuda")
+        # gather buckets: consecutive layers up to gather_bucket elements (a larger
+        # layer alone), at most 64 per launch; each layer lands in its own
+        # 16-byte-aligned slice of one reusable bucket buffer
+        self.gather_buckets = []
+        if gather_bucket > 0:
+            first, size, offs = 0, 0, []
+            for l, (lo, hi) in enumerate(self.plan.layers):
+                n = hi - lo
+                if offs and (size + n > gather_bucket or len(offs) == Z.ZERO_GATHER_MAX_LAYERS):
+                    self.gather_buckets.append((first, offs, size))
+                    first, size, offs = l, 0, []
+                offs.append(size)
+                size += (n + 7) // 8 * 8
+            self.gather_buckets.append((first, offs, size))
+            cap = max(b[2] for b in self.gather_buckets)
+        else:
+            cap = self.max_layer
+        self.layer_buf = torch.empty(cap, dtype=half, device="cuda")
+        base = self.layer_buf.data_ptr()
+        self.gather_outs = [[base + 2 * o for o in offs] for _, offs, _ in self.gather_buckets]
         torch.cuda.synchronize()
 
     def _write(self, shards, off, values):
@@ -239,7 +261,7 @@ class Bench:
             pos += k
 
     def launches_per_step(self):
-        n = 1 + len(self.plan.layers)
+        n = 1 + (len(self.gather_buckets) if self.gather_buckets else len(self.plan.layers))
         if self.path == "twopass":
             n += len(self.plan.buckets)
         return n
@@ -266,8 +288,12 @@ class Bench:
             Z.zero_step(self.ctx, hp, self.state.handle, self.grads, stream)
         if ev is not None:
             ev[1].record(stream)
-        for l, (lo, hi) in enumerate(self.plan.layers):
-            Z.zero_gather_layer(self.ctx, l, self.state.handle, self.layer_buf, stream)
+        if self.gather_buckets:
+            for (first, _, _), outs in zip(self.gather_buckets, self.gather_outs):
+                Z.zero_gather_layers(self.ctx, first, outs, self.state.handle, stream)
+        else:
+            for l in range(len(self.plan.layers)):
+                Z.zero_gather_layer(self.ctx, l, self.state.handle, self.layer_buf, stream)
 
     def loss_scale(self, stream):
         return self.Z.zero_loss_scale(self.ctx, stream=stream)
@@ -280,7 +306,7 @@ def run_ours(args, world, rank, local):
     if not torch.cuda.is_available():
         print(json.dumps({"error": "no CUDA device: the benchmark has no CPU fallback"}))
         sys.exit(1)
-    b = Bench(args.workload, args.path, args.first_tensors)
+    b = Bench(args.workload, args.path, args.first_tensors, args.gather_bucket)
     stream = torch.cuda.current_stream()
     for _ in range(args.warmup):
         b.step(stream)
@@ -342,6 +368,9 @@ def run_ours(args, world, rank, local):
                      "inplace": "fused reduce-scatter+AdamW, in place",
                      "twopass": "bucketed reduce-scatter, then AdamW from fp32 accumulators"}[b.path]
                     + " + device loss-scale update + ZeRO-3 gather of every layer",
+            "gather": (f"{len(b.gather_buckets)} bucketed launches of consecutive layers "
+                       f"(<= {args.gather_bucket} elements each)" if b.gather_buckets
+                       else f"{len(b.plan.layers)} per-layer launches"),
             "bytes_per_step": step_bytes,
             "l2": f"inputs larger than L2 ({step_bytes / 1e9:.1f} GB touched per step, L2 126 MB)",
             "parallelism": "1 GPU" if world == 1 else f"{world} independent replicas",

@@ -276,6 +276,24 @@ zero_status zero_step(zero_ctx_t* ctx, const zero_adamw* hp, const zero_state* s
 zero_status zero_gather_layer(zero_ctx_t* ctx, int64_t layer, const zero_state* state, void* out,
                               void* stream);
 
+/*
+ * zero_gather_layers -- gather `count` consecutive layers in one launch:
+ * layer first+i into outs[i], for 0 <= i < count, with exactly the result of
+ * count calls of zero_gather_layer.
+ * Defines: [genomic] "Bucketed All-Gather" bullet (parameter shards are
+ * grouped into buckets and a whole bucket is all-gathered at once, ahead of
+ * the layers that use it) and [legal] ZeRO-3 "Prefetching Scheduler"
+ * (upcoming layers are fetched ahead of use).
+ * count: 1..ZERO_GATHER_MAX_LAYERS. outs: count device pointers (host
+ * array, read during the call), each 16-byte aligned and holding its layer's
+ * (hi - lo) half elements; caller-owned.
+ * Errors: ZERO_ERR_RANGE (first/count), ZERO_ERR_INVALID_ARG, ZERO_ERR_ALIGN,
+ * ZERO_ERR_STATE, ZERO_ERR_CUDA.
+ */
+#define ZERO_GATHER_MAX_LAYERS 64
+zero_status zero_gather_layers(zero_ctx_t* ctx, int64_t first, int64_t count,
+                               const zero_state* state, void* const* outs, void* stream);
+
 typedef struct {
     float scale;           /* current loss scale */
     int32_t cur;           /* state set holding the current model (0 or 1) */

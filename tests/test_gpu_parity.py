@@ -158,6 +158,38 @@ def test_gather_layers(align, path):
         c.close()
 
 
+@pytest.mark.parametrize("align", [1, 8])
+@pytest.mark.parametrize("R", [1, 3, 8])
+def test_bucketed_gather_matches_oracle_and_single_gathers(align, R):
+    numels = [3001, 17, 8, 2048, 5, 700, 1, 9000, 64, 3]
+    layer_ids = [0, 0, 1, 1, 2, 2, 3, 4, 5, 5]
+    c = Case(numels, R, O.FP16, align, O.SCALE_DYNAMIC, 64.0, path="pingpong", layer_ids=layer_ids)
+    try:
+        for _ in range(2):
+            c.step()
+        c.compare()
+        flat = np.zeros(c.plan.T, np.uint16)
+        flat[c.idx] = c.ostate.param
+        L = c.lay.layers
+        for first, count in ((0, len(L)), (1, 3), (4, 2), (5, 1), (2, 1)):
+            outs = [torch.full((L[l][1] - L[l][0] + 8,), -1, dtype=torch.int16, device="cuda")
+                    for l in range(first, first + count)]
+            Z.zero_gather_layers(c.ctx, first, outs, c.handle)
+            for i, l in enumerate(range(first, first + count)):
+                lo, hi = L[l]
+                got = u16(outs[i])
+                assert np.array_equal(got[:hi - lo], flat[lo:hi]), (first, count, l)
+                assert np.all(got[hi - lo:] == 0xFFFF)
+                single = torch.empty(hi - lo, dtype=torch.int16, device="cuda")
+                Z.zero_gather_layer(c.ctx, l, c.handle, single)
+                assert np.array_equal(u16(single), got[:hi - lo])
+        with pytest.raises(Z.ZeroError) as e:
+            Z.zero_gather_layers(c.ctx, 4, [outs[0]] * 3, c.handle)
+        assert e.value.status == 5
+    finally:
+        c.close()
+
+
 def test_deterministic_bit_for_bit():
     runs = []
     for _ in range(2):

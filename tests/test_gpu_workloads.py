@@ -189,6 +189,17 @@ def run(name, path, gather=False, steps=None):
                     out = torch.empty(hi - lo, dtype=HALF[w.dtype], device="cuda")
                     Z.zero_gather_layer(w.ctx, l, w.state.handle, out)
                     assert torch.equal(out.view(torch.int16), flat[lo:hi].view(torch.int16)), l
+                # the same layers gathered in buckets of up to 64 layers per launch
+                nl = len(w.plan.layers)
+                for first in range(0, nl, 64):
+                    ls = range(first, min(nl, first + 64))
+                    outs = [torch.empty(w.plan.layers[l][1] - w.plan.layers[l][0],
+                                        dtype=HALF[w.dtype], device="cuda") for l in ls]
+                    Z.zero_gather_layers(w.ctx, first, outs, w.state.handle)
+                    for o, l in zip(outs, ls):
+                        lo, hi = w.plan.layers[l]
+                        assert torch.equal(o.view(torch.int16), flat[lo:hi].view(torch.int16)), l
+                    del outs
                 del flat
         return w.ofsm
     finally:

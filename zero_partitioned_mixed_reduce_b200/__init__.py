@@ -8,7 +8,8 @@ only for device memory and streams.
 from ._capi import (  # noqa: F401
     ZERO_BF16, ZERO_FP16, ZERO_LOSS_SCALE_GET, ZERO_LOSS_SCALE_SET, ZERO_MAX_RANKS,
     ZERO_SCALE_DYNAMIC, ZERO_SCALE_NONE, ZERO_SCALE_STATIC, LIB_PATH, StateHandle, ZeroError,
-    zero_adamw, zero_ctx_create, zero_ctx_destroy, zero_gather_layer, zero_last_error,
+    zero_adamw, zero_ctx_create, zero_ctx_destroy, zero_gather_layer, zero_gather_layers,
+    ZERO_GATHER_MAX_LAYERS, zero_last_error,
     zero_loss_scale, zero_plan, zero_plan_bucket, zero_plan_destroy, zero_plan_get_info,
     zero_plan_layer, zero_plan_memory, zero_plan_tensor, zero_reduce_scatter_bucket, zero_step,
     zero_step_noalloc, ZERO_NOALLOC_MAX_ELEMS, zero_sync, zero_version)

@@ -97,6 +97,7 @@ _sig("zero_ctx_destroy", _S, [_P])
 _sig("zero_reduce_scatter_bucket", _S, [_P, C.c_int64, _PP, _PP, _P])
 _sig("zero_step", _S, [_P, C.POINTER(zero_adamw), C.POINTER(zero_state), _PP, _P])
 _sig("zero_gather_layer", _S, [_P, C.c_int64, C.POINTER(zero_state), _P, _P])
+_sig("zero_gather_layers", _S, [_P, C.c_int64, C.c_int64, C.POINTER(zero_state), _PP, _P])
 _sig("zero_loss_scale", _S, [_P, C.POINTER(zero_loss_scale_state), C.c_int32, _P])
 _sig("zero_step_noalloc", _S, [_P, C.POINTER(zero_loss_scale_config),
                                C.POINTER(zero_loss_scale_state), C.POINTER(zero_adamw), _PP, _PP,
@@ -239,6 +240,15 @@ def zero_step(ctx, hp, state: StateHandle, grads=None, stream=None):
 
 def zero_gather_layer(ctx, layer, state: StateHandle, out, stream=None):
     _check(_lib.zero_gather_layer(ctx, layer, C.byref(state.c), _addr(out), _stream(stream)))
+
+
+ZERO_GATHER_MAX_LAYERS = 64
+
+
+def zero_gather_layers(ctx, first, outs, state: StateHandle, stream=None):
+    """Gather layers first .. first+len(outs)-1, layer first+i into outs[i]."""
+    o, oa = _ptr_array(outs)
+    _check(_lib.zero_gather_layers(ctx, first, len(outs), C.byref(state.c), o, _stream(stream)))
 
 
 def zero_loss_scale(ctx, op=ZERO_LOSS_SCALE_GET, state=None, stream=None):

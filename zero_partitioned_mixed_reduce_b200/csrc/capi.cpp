@@ -347,6 +347,42 @@ extern "C" zero_status zero_gather_layer(zero_ctx_t* ctx, int64_t layer, const z
     return ZERO_OK;
 }
 
+extern "C" zero_status zero_gather_layers(zero_ctx_t* ctx, int64_t first, int64_t count,
+                                          const zero_state* state, void* const* outs,
+                                          void* stream) {
+    const char* where = "zero_gather_layers";
+    if (!ctx) return zb_fail(ZERO_ERR_INVALID_ARG, "zero_gather_layers: ctx is NULL");
+    zero_status s = check_device(ctx, where);
+    if (s != ZERO_OK) return s;
+    const int64_t nl = static_cast<int64_t>(ctx->layer_lo.size());
+    if (count < 1 || count > ZERO_GATHER_MAX_LAYERS || first < 0 || first >= nl || count > nl - first)
+        return zb_fail(ZERO_ERR_RANGE, "zero_gather_layers: need 0 <= first, 1 <= count <= 64 and "
+                                       "first + count <= n_layers");
+    if (!outs) return zb_fail(ZERO_ERR_INVALID_ARG, "zero_gather_layers: outs is NULL");
+    for (int64_t i = 0; i < count; ++i) {
+        if (!outs[i])
+            return zb_fail(ZERO_ERR_INVALID_ARG, "zero_gather_layers: outs[" + std::to_string(i) + "] is NULL");
+        if (!aligned(outs[i], 16))
+            return zb_fail(ZERO_ERR_ALIGN, "zero_gather_layers: outs[" + std::to_string(i) +
+                                               "] is not 16-byte aligned");
+    }
+    int sets = 1;
+    if ((s = check_state(ctx, state, where, &sets, true)) != ZERO_OK) return s;
+    if (sets == 1 && ctx->two_sets)
+        return zb_fail(ZERO_ERR_STATE,
+                       "zero_gather_layers: the current parameters may live in set 1; pass param[1]");
+    zb::RankPtrs p;
+    for (int r = 0; r < ctx->R; ++r) {
+        p.param[0][r] = state->param[0][r];
+        p.param[1][r] = sets == 2 ? state->param[1][r] : state->param[0][r];
+    }
+    cudaError_t e = zb::launch_gather_many(ctx->R, ctx->S, static_cast<int>(count),
+                                           ctx->layer_lo.data() + first, ctx->layer_hi.data() + first,
+                                           ctx->st, p, outs, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(where, e);
+    return ZERO_OK;
+}
+
 extern "C" zero_status zero_loss_scale(zero_ctx_t* ctx, zero_loss_scale_state* inout, int32_t op,
                                        void* stream) {
     const char* where = "zero_loss_scale";

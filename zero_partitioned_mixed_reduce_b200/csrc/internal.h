@@ -71,6 +71,10 @@ cudaError_t launch_reduce_scatter(int32_t R, int32_t dtype, int64_t S, int64_t l
 cudaError_t launch_gather(int32_t R, int64_t S, int64_t lo, int64_t hi, const DevState* st,
                           const RankPtrs& p, void* out, cudaStream_t s);
 
+cudaError_t launch_gather_many(int32_t R, int64_t S, int nl, const int64_t* lo, const int64_t* hi,
+                               const DevState* st, const RankPtrs& p, void* const* outs,
+                               cudaStream_t s);
+
 // Grid the step kernels use for a given problem (for sizing `partials`).
 int step_grid_cap(int device);
 

@@ -328,43 +328,85 @@ __global__ void __launch_bounds__(kThreads)
 }
 
 // ---------------------------------------------------------------------------
-// ZeRO-3 layer gather from the current parameter set.
+// ZeRO-3 gather of one or more consecutive layers from the current parameter
+// set, in one launch. The layers' ranges are cut into 8-element slots
+// numbered across the bucket; a thread's slots, and so the flat positions it
+// reads, only grow, so layer and owner are tracked incrementally. Slots of a
+// layer whose start is 8-aligned move as one 16-byte vector, several per
+// thread in flight; partial and unaligned slots go element by element.
 // ---------------------------------------------------------------------------
 
-struct GatherArgs {
-    int64_t lo, n, S;  // flat start, element count, shard length
+struct GatherManyArgs {
+    int32_t nl;
+    int64_t S;
     uint32_t S8;
-    int32_t aligned;   // lo % 8 == 0
+    uint32_t total_slots;
     const DevState* st;
     const uint16_t* param[2][ZERO_MAX_RANKS];
-    uint16_t* out;
+    int64_t lo[ZERO_GATHER_MAX_LAYERS];
+    int64_t n[ZERO_GATHER_MAX_LAYERS];
+    uint16_t* out[ZERO_GATHER_MAX_LAYERS];
+    uint32_t slot0[ZERO_GATHER_MAX_LAYERS + 1];  // first slot of each layer; slot0[nl] = total
+    int32_t aligned[ZERO_GATHER_MAX_LAYERS];
 };
 
-__global__ void __launch_bounds__(kThreads) gather_kernel(const __grid_constant__ GatherArgs a) {
+constexpr int kGatherUnroll = 4;
+
+__global__ void __launch_bounds__(kThreads) gather_many_kernel(const __grid_constant__ GatherManyArgs a) {
     __shared__ int s_cur;
     if (threadIdx.x == 0) s_cur = reinterpret_cast<const volatile DevState*>(a.st)->cur;
     __syncthreads();
     const int cur = s_cur;
     const uint32_t stride = gridDim.x * kThreads;
-    const uint32_t tid = blockIdx.x * kThreads + threadIdx.x;
-    int64_t done = 0;
-    if (a.aligned) {
-        const uint32_t n8 = static_cast<uint32_t>(a.n / 8);
-        const uint32_t vlo = static_cast<uint32_t>(a.lo / 8);
-        uint32_t vj = tid;
-        OwnerCursor oc(vlo + vj, a.S8);
-        for (; vj < n8; vj += stride) {
-            const uint32_t vi = vlo + vj;
-            oc.seek(vi);
-            const uint4 q = ld_grad(reinterpret_cast<const uint4*>(a.param[cur][oc.o]) + (vi - oc.base));
-            st_u4(a.out + static_cast<size_t>(vj) * 8, q);
+    uint32_t s = blockIdx.x * kThreads + threadIdx.x;
+    if (s >= a.total_slots) return;
+    // the current layer's values live in registers; they are reloaded only
+    // when the thread's slot crosses into the next layer
+    int l = 0;
+    while (s >= a.slot0[l + 1]) ++l;
+    uint32_t first = a.slot0[l], end = a.slot0[l + 1];
+    int64_t lo = a.lo[l], n = a.n[l];
+    uint16_t* out = a.out[l];
+    bool al = a.aligned[l] != 0;
+    OwnerCursor oc(static_cast<uint32_t>(lo / 8), a.S8);
+    for (; s < a.total_slots; s += kGatherUnroll * stride) {
+        // pass 1: issue the loads of up to kGatherUnroll whole aligned slots
+        // (partial or unaligned slots are copied element by element here)
+        uint4 q[kGatherUnroll];
+        uint16_t* dst[kGatherUnroll];
+#pragma unroll
+        for (int u = 0; u < kGatherUnroll; ++u) {
+            dst[u] = nullptr;
+            const uint32_t su = s + u * stride;
+            if (su >= a.total_slots) continue;
+            if (su >= end) {
+                do ++l; while (su >= a.slot0[l + 1]);
+                first = a.slot0[l];
+                end = a.slot0[l + 1];
+                lo = a.lo[l];
+                n = a.n[l];
+                out = a.out[l];
+                al = a.aligned[l] != 0;
+            }
+            const int64_t e0 = static_cast<int64_t>(su - first) * 8;  // first element in the layer
+            if (al && e0 + 8 <= n) {
+                const uint32_t vi = static_cast<uint32_t>((lo + e0) >> 3);
+                oc.seek(vi);
+                q[u] = ld_grad(reinterpret_cast<const uint4*>(a.param[cur][oc.o]) + (vi - oc.base));
+                dst[u] = out + e0;
+            } else {
+                const int64_t e1 = e0 + 8 < n ? e0 + 8 : n;
+                for (int64_t e = e0; e < e1; ++e) {
+                    const int64_t i = lo + e;
+                    const int64_t o = i / a.S;
+                    out[e] = ld_grad1(a.param[cur][o] + (i - o * a.S));
+                }
+            }
         }
-        done = static_cast<int64_t>(n8) * 8;
-    }
-    for (int64_t j = done + tid; j < a.n; j += stride) {
-        const int64_t i = a.lo + j;
-        const int64_t o = i / a.S;
-        a.out[j] = ld_grad1(a.param[cur][o] + (i - o * a.S));
+        // pass 2: the stores
+#pragma unroll
+        for (int u = 0; u < kGatherUnroll; ++u)
+            if (dst[u]) st_u4(dst[u], q[u]);
     }
 }
 
@@ -523,24 +565,38 @@ cudaError_t launch_reduce_scatter(int32_t R, int32_t dtype, int64_t S, int64_t l
                               : rs_dispatch<Bf16>(R, S, lo, hi, st, p, s);
 }
 
-cudaError_t launch_gather(int32_t R, int64_t S, int64_t lo, int64_t hi, const DevState* st,
-                          const RankPtrs& p, void* out, cudaStream_t s) {
-    GatherArgs a;
-    a.lo = lo;
-    a.n = hi - lo;
+cudaError_t launch_gather_many(int32_t R, int64_t S, int nl, const int64_t* lo, const int64_t* hi,
+                               const DevState* st, const RankPtrs& p, void* const* outs,
+                               cudaStream_t s) {
+    GatherManyArgs a;
+    a.nl = nl;
     a.S = S;
     a.S8 = static_cast<uint32_t>(S / 8);
-    a.aligned = (lo % 8) == 0;
     a.st = st;
     for (int r = 0; r < R; ++r)
         for (int k = 0; k < 2; ++k) a.param[k][r] = static_cast<const uint16_t*>(p.param[k][r]);
-    a.out = static_cast<uint16_t*>(out);
-    if (a.n <= 0) return cudaSuccess;
-    static const int per_sm = blocks_per_sm(gather_kernel);
-    const uint64_t items = a.aligned ? static_cast<uint64_t>(a.n / 8) : static_cast<uint64_t>(a.n);
-    const uint32_t grid = grid_for(items > 0 ? items : 1, per_sm, 0);
-    gather_kernel<<<grid, kThreads, 0, s>>>(a);
+    uint64_t slots = 0;
+    for (int l = 0; l < nl; ++l) {
+        a.lo[l] = lo[l];
+        a.n[l] = hi[l] - lo[l];
+        a.out[l] = static_cast<uint16_t*>(outs[l]);
+        a.aligned[l] = (lo[l] % 8) == 0;
+        a.slot0[l] = static_cast<uint32_t>(slots);
+        slots += static_cast<uint64_t>((a.n[l] + 7) / 8);
+    }
+    a.slot0[nl] = static_cast<uint32_t>(slots);
+    a.total_slots = static_cast<uint32_t>(slots);
+    if (slots == 0) return cudaSuccess;
+    static const int per_sm = blocks_per_sm(gather_many_kernel);
+    const uint32_t grid = grid_for((slots + kGatherUnroll - 1) / kGatherUnroll, per_sm, 0);
+    gather_many_kernel<<<grid, kThreads, 0, s>>>(a);
     return cudaGetLastError();
+}
+
+cudaError_t launch_gather(int32_t R, int64_t S, int64_t lo, int64_t hi, const DevState* st,
+                          const RankPtrs& p, void* out, cudaStream_t s) {
+    void* outs[1] = {out};
+    return launch_gather_many(R, S, 1, &lo, &hi, st, p, outs, s);
 }
 
 int step_grid_cap(int device) {
