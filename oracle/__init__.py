@@ -30,11 +30,17 @@ class FSM(C.Structure):
                 ("grad_norm_sq", C.c_double)]
 
 
+class StepOpts(C.Structure):
+    _fields_ = [("grad_divisor", C.c_double), ("max_grad_norm", C.c_double)]
+
+
 def lib():
     """Load (building first if needed) the oracle shared library."""
     global _lib
     if _lib is None:
-        path = _build.build()
+        # ZERO_ORACLE_LIB points the tests at another build of this oracle
+        # (used to check that the pins catch planted mistakes)
+        path = os.environ.get("ZERO_ORACLE_LIB") or _build.build()
         L = C.CDLL(path)
         P = C.c_void_p
         L.oracle_half_to_float.restype = C.c_float
@@ -56,6 +62,9 @@ def lib():
         L.oracle_step_sharded.restype = C.c_int32
         L.oracle_step_sharded.argtypes = [C.c_int64, C.c_int32, C.c_int32, P, P, P, P, P, P,
                                           C.POINTER(AdamW), C.POINTER(FSM)]
+        L.oracle_step_ex.restype = C.c_int32
+        L.oracle_step_ex.argtypes = [C.c_int64, C.c_int32, C.c_int32, C.c_int32, P, P, P, P, P,
+                                     C.POINTER(AdamW), C.POINTER(StepOpts), C.POINTER(FSM)]
         L.oracle_model_state_bytes.restype = C.c_double
         L.oracle_model_state_bytes.argtypes = [C.c_int32, C.c_double, C.c_double]
         L.oracle_fp32_weight_bytes.restype = C.c_double
@@ -163,6 +172,21 @@ def step(state: State, grads: np.ndarray, hp: AdamW, fsm: FSM) -> bool:
                            _ptr(state.v), _ptr(state.param), C.byref(hp), C.byref(fsm))
     if rc < 0:
         raise MemoryError("oracle_step")
+    return bool(rc)
+
+
+def step_ex(state: State, micro_grads: np.ndarray, hp: AdamW, fsm: FSM, grad_divisor=1.0,
+            max_grad_norm=0.0) -> bool:
+    """Step with accumulation over micro-batches and optional global-norm
+    clipping. micro_grads: (n_micro, R, P) uint16. Returns skipped."""
+    g = np.ascontiguousarray(micro_grads, dtype=np.uint16)
+    n_micro, R, P = g.shape
+    opts = StepOpts(grad_divisor, max_grad_norm)
+    rc = lib().oracle_step_ex(P, R, state.dtype, n_micro, _ptr(g), _ptr(state.master),
+                              _ptr(state.m), _ptr(state.v), _ptr(state.param), C.byref(hp),
+                              C.byref(opts), C.byref(fsm))
+    if rc < 0:
+        raise ValueError("oracle_step_ex rejected its arguments")
     return bool(rc)
 
 

@@ -343,6 +343,82 @@ int32_t oracle_step(int64_t P, int32_t R, int32_t dtype, const uint16_t* grads,
 }
 
 /* ======================================================================= */
+/* Gradient accumulation and global-norm clipping.                         */
+/*                                                                         */
+/* Not on the pages, which only say that ZeRO frees memory for larger      */
+/* effective batches ([inferensys-instr], large-batch paragraph). Readings: */
+/*  - micro-batch mu's all-reduced sum s_mu is formed as in                */
+/*    oracle_allreduce_sum; the accumulator is s_1, then acc + s_2, ...,   */
+/*    each addition one fp32 rounding, in micro-batch order;               */
+/*  - the unscale multiplies by (float)(1 / ((R * k) * scale)) with k the   */
+/*    grad divisor (k = number of micro-batches for a mean);                */
+/*  - overflow means a non-finite accumulator after the last micro-batch;  */
+/*  - clipping follows the usual global-norm rule: with ||g|| the L2 norm  */
+/*    of the unscaled gradient (squares summed in double),                  */
+/*    coef = (float) min(1, max_norm / (||g|| + 1e-6)), and the update uses */
+/*    g * coef (one fp32 rounding); the recorded norm is the one before     */
+/*    clipping.                                                             */
+/* ======================================================================= */
+
+int32_t oracle_step_ex(int64_t P, int32_t R, int32_t dtype, int32_t n_micro, const uint16_t* grads,
+                       float* master, float* m, float* v, uint16_t* param,
+                       const oracle_adamw* hp, const oracle_step_opts* opts, oracle_fsm* st) {
+    if (n_micro < 1 || opts->grad_divisor < 1.0) return -2;
+    float* acc = (float*)malloc(sizeof(float) * (size_t)(P > 0 ? P : 1));
+    float* part = (float*)malloc(sizeof(float) * (size_t)(P > 0 ? P : 1));
+    if (!acc || !part) {
+        free(acc);
+        free(part);
+        return -1;
+    }
+    oracle_allreduce_sum(P, R, dtype, grads, acc);
+    for (int32_t mu = 1; mu < n_micro; mu++) {
+        oracle_allreduce_sum(P, R, dtype, grads + (int64_t)mu * R * P, part);
+        for (int64_t e = 0; e < P; e++) acc[e] = acc[e] + part[e];
+    }
+    int32_t overflow = 0;
+    for (int64_t e = 0; e < P; e++)
+        if (!isfinite(acc[e])) overflow = 1;
+
+    float scale = effective_scale(st);
+    adamw_coeffs c = make_coeffs(hp, R, scale, st->t + 1);
+    c.inv = (float)(1.0 / (((double)R * opts->grad_divisor) * (double)scale));
+
+    double nrm = 0.0;
+    for (int64_t e = 0; e < P; e++) {
+        float g = acc[e] * c.inv;
+        nrm += (double)g * (double)g;
+    }
+    float coef = 1.0f;
+    if (opts->max_grad_norm > 0.0) {
+        double cd = opts->max_grad_norm / (sqrt(nrm) + 1e-6);
+        coef = (float)(cd < 1.0 ? cd : 1.0);
+    }
+
+    int32_t skip = (st->mode == ORACLE_SCALE_DYNAMIC) && overflow;
+    if (!skip) {
+        for (int64_t e = 0; e < P; e++) {
+            /* g = (acc * inv) * coef, then the AdamW update of adamw_element */
+            float g = (acc[e] * c.inv) * coef;
+            float pp = master[e] * c.dec;
+            float mm = c.b1f * m[e] + c.omb1 * g;
+            float vv = c.b2f * v[e] + c.omb2 * (g * g);
+            float den = sqrtf(vv) / c.bc2s + c.epsf;
+            pp = pp - c.ss * (mm / den);
+            master[e] = pp;
+            m[e] = mm;
+            v[e] = vv;
+            param[e] = oracle_float_to_half(pp, dtype);
+        }
+    }
+    oracle_fsm_update(st, overflow);
+    st->grad_norm_sq = nrm;
+    free(acc);
+    free(part);
+    return skip;
+}
+
+/* ======================================================================= */
 /* The same step, partitioned.                                             */
 /*                                                                         */
 /* [mbrenndoerfer] introduction: every replica holds the same state and     */

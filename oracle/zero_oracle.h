@@ -109,6 +109,21 @@ int32_t oracle_step_sharded(int64_t S, int32_t R, int32_t dtype, const uint16_t*
                             float* master, float* m, float* v, uint16_t* param,
                             uint16_t* gathered, const oracle_adamw* hp, oracle_fsm* st);
 
+/* One step with gradient accumulation and global-norm clipping (not on the
+ * pages; the readings are stated in zero_oracle.c). grads holds n_micro
+ * micro-batches, each R x P rank-major, in order. grad_divisor k >= 1 joins
+ * R and the loss scale in the unscale; max_grad_norm <= 0 turns clipping
+ * off. grad_norm_sq records the norm before clipping. Returns 1 when
+ * skipped. */
+typedef struct {
+    double grad_divisor;
+    double max_grad_norm;
+} oracle_step_opts;
+
+int32_t oracle_step_ex(int64_t P, int32_t R, int32_t dtype, int32_t n_micro, const uint16_t* grads,
+                       float* master, float* m, float* v, uint16_t* param,
+                       const oracle_adamw* hp, const oracle_step_opts* opts, oracle_fsm* st);
+
 /* ---- per-rank model-state memory (bytes) --------------------------------
  * stage 0 = plain data parallel, 1/2/3 = ZeRO stages; psi parameters, N
  * data-parallel ranks; 2 + 2 + 12 bytes per parameter. */
