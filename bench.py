@@ -49,6 +49,10 @@ def parse_args(argv=None):
     ap.add_argument("--path", choices=["auto", "pingpong", "inplace", "twopass"], default="auto")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--accum", type=int, default=1,
+                    help="micro-batches accumulated per step (two-pass path)")
+    ap.add_argument("--clip", type=float, default=0.0,
+                    help="global-norm clipping threshold (> 0: on; two-pass path)")
     ap.add_argument("--gather-bucket", type=int, default=32 << 20,
                     help="gather consecutive layers in one launch up to this many elements "
                          "(0: one launch per layer)")
@@ -194,7 +198,7 @@ def profiled_traffic(kernel, workload):
 # ---- the workload -------------------------------------------------------------
 
 class Bench:
-    def __init__(self, name, path, first_tensors=0, gather_bucket=32 << 20):
+    def __init__(self, name, path, first_tensors=0, gather_bucket=32 << 20, accum=1, clip=0.0):
         import zero_partitioned_mixed_reduce_b200 as Z
         from zero_partitioned_mixed_reduce_b200 import synth
         self.Z, self.synth = Z, synth
@@ -203,8 +207,14 @@ class Bench:
             wl["numels"] = wl["numels"][:first_tensors]
             wl["layer_ids"] = wl["layer_ids"][:first_tensors] if wl["layer_ids"] else None
         self.R, self.dtype = wl["R"], wl["dtype"]
+        self.accum, self.clip = accum, clip
         if path == "auto":
-            path = "pingpong" if wl["mode"] == synth.DYNAMIC else "inplace"
+            if accum > 1 or clip > 0:
+                path = "twopass"
+            else:
+                path = "pingpong" if wl["mode"] == synth.DYNAMIC else "inplace"
+        if (accum > 1 or clip > 0) and path != "twopass":
+            raise SystemExit("--accum/--clip need the two-pass path")
         self.path = path
         self.plan = Z.Plan(wl["numels"], wl["layer_ids"], wl["R"], wl["dtype"], 8,
                            wl["bucket_elems"])
@@ -263,14 +273,17 @@ class Bench:
     def launches_per_step(self):
         n = 1 + (len(self.gather_buckets) if self.gather_buckets else len(self.plan.layers))
         if self.path == "twopass":
-            n += len(self.plan.buckets)
+            n += self.accum * len(self.plan.buckets) + (1 if self.clip > 0 else 0)
         return n
 
     def step_bytes(self):
         """Algorithmic HBM bytes of one step (and of its dominant kernel)."""
         R, T = self.R, self.T
         if self.path == "twopass":
-            main = (2 * R + 4) * T + 30 * T
+            # first micro-batch writes the accumulators, later ones read-modify-write
+            main = (2 * R + 4) * T + (self.accum - 1) * (2 * R + 8) * T + 30 * T
+            if self.clip > 0:
+                main += 4 * T
         else:
             main = (2 * R + 26) * T
         return main + 4 * self.L, main
@@ -281,9 +294,13 @@ class Bench:
         if ev is not None:
             ev[0].record(stream)
         if self.path == "twopass":
-            for b in range(len(self.plan.buckets)):
-                Z.zero_reduce_scatter_bucket(self.ctx, b, self.grads, self.state.acc, stream)
-            Z.zero_step(self.ctx, hp, self.state.handle, None, stream)
+            for mu in range(self.accum):
+                flags = Z.ZERO_RS_ACCUMULATE if mu else 0
+                for b in range(len(self.plan.buckets)):
+                    Z.zero_reduce_scatter_bucket_ex(self.ctx, b, self.grads, self.state.acc, flags,
+                                                    stream)
+            Z.zero_step_ex(self.ctx, hp, self.state.handle, None, float(self.accum), self.clip,
+                           stream)
         else:
             Z.zero_step(self.ctx, hp, self.state.handle, self.grads, stream)
         if ev is not None:
@@ -306,7 +323,8 @@ def run_ours(args, world, rank, local):
     if not torch.cuda.is_available():
         print(json.dumps({"error": "no CUDA device: the benchmark has no CPU fallback"}))
         sys.exit(1)
-    b = Bench(args.workload, args.path, args.first_tensors, args.gather_bucket)
+    b = Bench(args.workload, args.path, args.first_tensors, args.gather_bucket, args.accum,
+              args.clip)
     stream = torch.cuda.current_stream()
     for _ in range(args.warmup):
         b.step(stream)
@@ -341,6 +359,8 @@ def run_ours(args, world, rank, local):
     achieved = main_bytes / (kavg * 1e-3) / 1e9
     kernel_name = {"pingpong": "fused_step_kernel", "inplace": "fused_step_kernel",
                    "twopass": "reduce_scatter+step_from_acc"}[b.path]
+    if b.path == "twopass" and (b.accum > 1 or b.clip > 0):
+        kernel_name += f" (accum {b.accum}{', clip' if b.clip > 0 else ''})"
     traffic = profiled_traffic(kernel_name, args.workload)
     out = {
         "metric": METRIC,
@@ -366,7 +386,9 @@ def run_ours(args, world, rank, local):
             "R": b.R, "P": b.P, "T": b.T, "S": b.S, "n_layers": len(b.plan.layers),
             "path": {"pingpong": "fused reduce-scatter+AdamW, ping-pong state",
                      "inplace": "fused reduce-scatter+AdamW, in place",
-                     "twopass": "bucketed reduce-scatter, then AdamW from fp32 accumulators"}[b.path]
+                     "twopass": f"bucketed reduce-scatter ({b.accum} micro-batch(es)), "
+                       f"{'global-norm clip, ' if b.clip > 0 else ''}"
+                       "then AdamW from fp32 accumulators"}[b.path]
                     + " + device loss-scale update + ZeRO-3 gather of every layer",
             "gather": (f"{len(b.gather_buckets)} bucketed launches of consecutive layers "
                        f"(<= {args.gather_bucket} elements each)" if b.gather_buckets

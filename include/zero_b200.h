@@ -221,6 +221,23 @@ zero_status zero_reduce_scatter_bucket(zero_ctx_t* ctx, int64_t bucket, const vo
                                        float* const* acc, void* stream);
 
 /*
+ * zero_reduce_scatter_bucket_ex -- zero_reduce_scatter_bucket with flags.
+ * ZERO_RS_ACCUMULATE adds the bucket's rank-order sum to the accumulators
+ * instead of overwriting them, for gradient accumulation over micro-batches:
+ *   acc[o][i - o*S] = acc[o][i - o*S] + (((f32(g_0[i]) + f32(g_1[i])) + ...) + f32(g_{R-1}[i]))
+ * The overflow flag is OR-ed with "some accumulator is inf or NaN". The
+ * first micro-batch of a step must not accumulate (it initializes).
+ * Defines: gradient accumulation is not on the pages, which only note that
+ * ZeRO frees memory for larger effective batches ([instr], large-batch
+ * paragraph); the reduce-scatter itself is [legal] "Reduce-Scatter".
+ * Errors: as zero_reduce_scatter_bucket, plus ZERO_ERR_INVALID_ARG for
+ * unknown flags.
+ */
+#define ZERO_RS_ACCUMULATE 1
+zero_status zero_reduce_scatter_bucket_ex(zero_ctx_t* ctx, int64_t bucket, const void* const* grads,
+                                          float* const* acc, int32_t flags, void* stream);
+
+/*
  * zero_step -- one optimizer step on every shard, then the loss-scale update.
  *
  * With g = acc * (1 / (R * scale)) the unscaled, averaged gradient (scale = 1
@@ -259,6 +276,31 @@ zero_status zero_reduce_scatter_bucket(zero_ctx_t* ctx, int64_t bucket, const vo
  */
 zero_status zero_step(zero_ctx_t* ctx, const zero_adamw* hp, const zero_state* state,
                       const void* const* grads, void* stream);
+
+/*
+ * zero_step_ex -- zero_step with options (opts == NULL: the defaults, i.e.
+ * exactly zero_step).
+ *  grad_divisor k (>= 1, default 1): the unscale multiplies by
+ *    (float)(1 / ((R * k) * scale)); k = the number of accumulated
+ *    micro-batches gives their mean.
+ *  max_grad_norm (> 0 turns clipping on, 0 = off): with ||g|| the L2 norm of
+ *    the unscaled gradient, c = (float) min(1, max_norm / (||g|| + 1e-6)) in
+ *    double, and the update uses g * c (one fp32 multiply). Clipping needs
+ *    the norm before any element is updated, so it runs on the two-pass path
+ *    only (grads == NULL): one extra pass reads the accumulators (4 bytes per
+ *    element). The recorded grad_norm_sq is the norm before clipping.
+ * Defines: not on the pages (clipping and accumulation are common practice
+ * around ZeRO training loops, not part of the method the pages describe).
+ * Errors: as zero_step, plus ZERO_ERR_INVALID_ARG for a divisor < 1, a
+ * negative or non-finite max norm, or clipping with grads != NULL.
+ */
+typedef struct {
+    double grad_divisor;
+    double max_grad_norm;
+    int64_t reserved[2]; /* must be 0 */
+} zero_step_opts;
+zero_status zero_step_ex(zero_ctx_t* ctx, const zero_adamw* hp, const zero_state* state,
+                         const void* const* grads, const zero_step_opts* opts, void* stream);
 
 /*
  * zero_gather_layer -- assemble one layer's half parameters from the R

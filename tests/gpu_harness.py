@@ -138,6 +138,36 @@ class Case:
         self.g.check()
         return skipped
 
+    def step_ex(self, n_micro, grad_divisor=1.0, max_grad_norm=0.0, inject=None):
+        """Two-pass step over n_micro accumulated micro-batches, optionally
+        clipped; inject: (micro, rank, element, bits) tuples."""
+        assert self.path == "twopass"
+        self.step_no += 1
+        scale = self.ofsm.scale if self.mode != O.SCALE_NONE else 1.0
+        micro = []
+        for mu in range(n_micro):
+            rows = [synth.flat_grads(self.wl, self.step_no * 100 + mu, r, scale, "cpu")
+                    for r in range(self.R)]
+            micro.append(np.stack([u16(t) for t in rows]))
+        g = np.stack(micro)
+        for (mu, r, e, bits) in inject or []:
+            g[mu, r, e] = bits
+        for mu in range(n_micro):
+            for r in range(self.R):
+                gp = np.zeros(self.plan.T, np.uint16)
+                gp[self.idx] = g[mu, r]
+                self.grads[r].view(torch.int16).copy_(torch.from_numpy(gp.view(np.int16)))
+            for b in range(len(self.plan.buckets)):
+                Z.zero_reduce_scatter_bucket_ex(self.ctx, b, self.grads, self.acc,
+                                                Z.ZERO_RS_ACCUMULATE if mu else 0)
+        Z.zero_step_ex(self.ctx, self.hp, self.handle, None, grad_divisor, max_grad_norm)
+        skipped = O.step_ex(self.ostate, g, O.AdamW(**{k: self.hp[k] for k in
+                                                       ("lr", "beta1", "beta2", "eps",
+                                                        "weight_decay")}),
+                            self.ofsm, grad_divisor, max_grad_norm)
+        self.g.check()
+        return skipped
+
     def gpu_fsm(self):
         return Z.zero_loss_scale(self.ctx)
 

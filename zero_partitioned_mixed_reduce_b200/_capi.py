@@ -19,6 +19,7 @@ ZERO_ERR_OOM, ZERO_ERR_RANGE, ZERO_ERR_TIMEOUT, ZERO_ERR_STATE = 4, 5, 6, 7
 ZERO_BF16, ZERO_FP16 = 0, 1
 ZERO_SCALE_NONE, ZERO_SCALE_STATIC, ZERO_SCALE_DYNAMIC = 0, 1, 2
 ZERO_LOSS_SCALE_GET, ZERO_LOSS_SCALE_SET = 0, 1
+ZERO_RS_ACCUMULATE = 1
 
 STATUS_NAMES = {0: "ZERO_OK", 1: "ZERO_ERR_INVALID_ARG", 2: "ZERO_ERR_ALIGN", 3: "ZERO_ERR_CUDA",
                 4: "ZERO_ERR_OOM", 5: "ZERO_ERR_RANGE", 6: "ZERO_ERR_TIMEOUT", 7: "ZERO_ERR_STATE"}
@@ -66,6 +67,11 @@ class zero_state(C.Structure):
                 ("acc", _PP)]
 
 
+class zero_step_opts(C.Structure):
+    _fields_ = [("grad_divisor", C.c_double), ("max_grad_norm", C.c_double),
+                ("reserved", C.c_int64 * 2)]
+
+
 class zero_loss_scale_state(C.Structure):
     _fields_ = [("scale", C.c_float), ("cur", C.c_int32), ("good", C.c_int64), ("t", C.c_int64),
                 ("last_overflow", C.c_int32), ("last_skipped", C.c_int32),
@@ -96,6 +102,9 @@ _sig("zero_ctx_create", _S, [_P, C.POINTER(zero_loss_scale_config), C.POINTER(_P
 _sig("zero_ctx_destroy", _S, [_P])
 _sig("zero_reduce_scatter_bucket", _S, [_P, C.c_int64, _PP, _PP, _P])
 _sig("zero_step", _S, [_P, C.POINTER(zero_adamw), C.POINTER(zero_state), _PP, _P])
+_sig("zero_reduce_scatter_bucket_ex", _S, [_P, C.c_int64, _PP, _PP, C.c_int32, _P])
+_sig("zero_step_ex", _S, [_P, C.POINTER(zero_adamw), C.POINTER(zero_state), _PP,
+                          C.POINTER(zero_step_opts), _P])
 _sig("zero_gather_layer", _S, [_P, C.c_int64, C.POINTER(zero_state), _P, _P])
 _sig("zero_gather_layers", _S, [_P, C.c_int64, C.c_int64, C.POINTER(zero_state), _PP, _P])
 _sig("zero_loss_scale", _S, [_P, C.POINTER(zero_loss_scale_state), C.c_int32, _P])
@@ -228,6 +237,13 @@ def zero_reduce_scatter_bucket(ctx, bucket, grads, acc, stream=None):
     _check(_lib.zero_reduce_scatter_bucket(ctx, bucket, g, a, _stream(stream)))
 
 
+def zero_reduce_scatter_bucket_ex(ctx, bucket, grads, acc, flags=0, stream=None):
+    """flags: ZERO_RS_ACCUMULATE adds to the accumulators."""
+    g, ga = _ptr_array(grads)
+    a, aa = _ptr_array(acc)
+    _check(_lib.zero_reduce_scatter_bucket_ex(ctx, bucket, g, a, flags, _stream(stream)))
+
+
 def zero_step(ctx, hp, state: StateHandle, grads=None, stream=None):
     """hp: zero_adamw or a dict with lr, beta1, beta2, eps, weight_decay."""
     if isinstance(hp, dict):
@@ -236,6 +252,19 @@ def zero_step(ctx, hp, state: StateHandle, grads=None, stream=None):
     if grads is not None:
         g, ga = _ptr_array(grads)
     _check(_lib.zero_step(ctx, C.byref(hp), C.byref(state.c), g, _stream(stream)))
+
+
+def zero_step_ex(ctx, hp, state: StateHandle, grads=None, grad_divisor=1.0, max_grad_norm=0.0,
+                 stream=None):
+    """zero_step with a grad divisor and global-norm clipping (two-pass only)."""
+    if isinstance(hp, dict):
+        hp = zero_adamw(hp["lr"], hp["beta1"], hp["beta2"], hp["eps"], hp["weight_decay"])
+    g = None
+    if grads is not None:
+        g, ga = _ptr_array(grads)
+    opts = zero_step_opts(grad_divisor, max_grad_norm)
+    _check(_lib.zero_step_ex(ctx, C.byref(hp), C.byref(state.c), g, C.byref(opts),
+                             _stream(stream)))
 
 
 def zero_gather_layer(ctx, layer, state: StateHandle, out, stream=None):

@@ -227,7 +227,15 @@ extern "C" zero_status zero_ctx_destroy(zero_ctx_t* ctx) {
 extern "C" zero_status zero_reduce_scatter_bucket(zero_ctx_t* ctx, int64_t bucket,
                                                   const void* const* grads, float* const* acc,
                                                   void* stream) {
+    return zero_reduce_scatter_bucket_ex(ctx, bucket, grads, acc, 0, stream);
+}
+
+extern "C" zero_status zero_reduce_scatter_bucket_ex(zero_ctx_t* ctx, int64_t bucket,
+                                                     const void* const* grads, float* const* acc,
+                                                     int32_t flags, void* stream) {
     const char* where = "zero_reduce_scatter_bucket";
+    if (flags & ~ZERO_RS_ACCUMULATE)
+        return zb_fail(ZERO_ERR_INVALID_ARG, "zero_reduce_scatter_bucket_ex: unknown flags");
     if (!ctx) return zb_fail(ZERO_ERR_INVALID_ARG, "zero_reduce_scatter_bucket: ctx is NULL");
     zero_status s = check_device(ctx, where);
     if (s != ZERO_OK) return s;
@@ -249,14 +257,31 @@ extern "C" zero_status zero_reduce_scatter_bucket(zero_ctx_t* ctx, int64_t bucke
         p.acc[r] = acc[r];
     }
     cudaError_t e = zb::launch_reduce_scatter(ctx->R, ctx->dtype, ctx->S, lo, hi, ctx->st, p,
-                                              static_cast<cudaStream_t>(stream));
+                                              static_cast<cudaStream_t>(stream),
+                                              (flags & ZERO_RS_ACCUMULATE) != 0);
     if (e != cudaSuccess) return cuda_fail(where, e);
     return ZERO_OK;
 }
 
 extern "C" zero_status zero_step(zero_ctx_t* ctx, const zero_adamw* hp, const zero_state* state,
                                  const void* const* grads, void* stream) {
+    return zero_step_ex(ctx, hp, state, grads, nullptr, stream);
+}
+
+extern "C" zero_status zero_step_ex(zero_ctx_t* ctx, const zero_adamw* hp, const zero_state* state,
+                                    const void* const* grads, const zero_step_opts* opts,
+                                    void* stream) {
     const char* where = "zero_step";
+    zero_step_opts o{1.0, 0.0, {0, 0}};
+    if (opts) o = *opts;
+    if (!(o.grad_divisor >= 1.0) || !std::isfinite(o.grad_divisor) || !(o.max_grad_norm >= 0.0) ||
+        !std::isfinite(o.max_grad_norm) || o.reserved[0] != 0 || o.reserved[1] != 0)
+        return zb_fail(ZERO_ERR_INVALID_ARG,
+                       "zero_step_ex: need grad_divisor >= 1, finite max_grad_norm >= 0, reserved 0");
+    if (o.max_grad_norm > 0.0 && grads != nullptr)
+        return zb_fail(ZERO_ERR_INVALID_ARG,
+                       "zero_step_ex: clipping needs the two-pass path (grads == NULL): the norm must "
+                       "be known before any element is updated");
     if (!ctx || !hp) return zb_fail(ZERO_ERR_INVALID_ARG, "zero_step: NULL ctx or hyper-parameters");
     zero_status s = check_device(ctx, where);
     if (s != ZERO_OK) return s;
@@ -298,6 +323,9 @@ extern "C" zero_status zero_step(zero_ctx_t* ctx, const zero_adamw* hp, const ze
     sp.omb2 = static_cast<float>(1.0 - hp->beta2);
     sp.epsf = static_cast<float>(hp->eps);
     sp.lr = hp->lr;
+    sp.divisor = o.grad_divisor;
+    sp.max_norm = o.max_grad_norm;
+    sp.clip = o.max_grad_norm > 0.0 ? 1 : 0;
     sp.interval = ctx->cfg.growth_interval;
     sp.growth = ctx->cfg.growth_factor;
     sp.backoff = ctx->cfg.backoff_factor;
@@ -314,7 +342,10 @@ extern "C" zero_status zero_step(zero_ctx_t* ctx, const zero_adamw* hp, const ze
         p.g[r] = fused ? grads[r] : nullptr;
         p.acc[r] = fused ? nullptr : state->acc[r];
     }
-    cudaError_t e = fused ? zb::launch_fused_step(sp, p, cs) : zb::launch_step_from_acc(sp, p, cs);
+    cudaError_t e = cudaSuccess;
+    if (sp.clip) e = zb::launch_clip_norm(sp, p, cs);
+    if (e == cudaSuccess)
+        e = fused ? zb::launch_fused_step(sp, p, cs) : zb::launch_step_from_acc(sp, p, cs);
     if (e != cudaSuccess) return cuda_fail(where, e);
     ctx->t_bound += 1;
     if (sp.pingpong) ctx->two_sets = true;

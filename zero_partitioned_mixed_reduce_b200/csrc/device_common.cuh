@@ -132,10 +132,15 @@ __device__ __forceinline__ bool nonfinite(float x) { return !(fabsf(x) <= FLT_MA
 
 struct Coef {
     float inv, dec, b1f, omb1, b2f, omb2, epsf, ss, bc2s;
+    float clip;  // global-norm clipping coefficient; exactly 1 when clipping is off
 };
 
+// Returns the unscaled gradient before clipping (for the norm); with CLIP the
+// update uses it times the clipping coefficient.
+template <bool CLIP = false>
 __device__ __forceinline__ float adamw1(const Coef& c, float acc, float& p, float& m, float& v) {
-    const float g = __fmul_rn(acc, c.inv);
+    const float g0 = __fmul_rn(acc, c.inv);
+    const float g = CLIP ? __fmul_rn(g0, c.clip) : g0;
     float pp = __fmul_rn(p, c.dec);
     const float mm = __fadd_rn(__fmul_rn(c.b1f, m), __fmul_rn(c.omb1, g));
     const float vv = __fadd_rn(__fmul_rn(c.b2f, v), __fmul_rn(c.omb2, __fmul_rn(g, g)));
@@ -144,7 +149,7 @@ __device__ __forceinline__ float adamw1(const Coef& c, float acc, float& p, floa
     p = pp;
     m = mm;
     v = vv;
-    return g;
+    return g0;
 }
 
 // ---------------------------------------------------------------------------

@@ -35,7 +35,7 @@ struct alignas(64) DevState {
     uint32_t flag;  // OR of "some reduced gradient is inf/NaN" for the step in progress
     uint32_t done;  // blocks of the running step kernel that have finished
     int32_t err;    // device-side consistency error (0 = none)
-    int32_t pad;
+    float clip;     // clipping coefficient of the step in progress
 };
 
 // Everything a step kernel needs besides the rank pointers. Filled on the host.
@@ -44,6 +44,9 @@ struct StepParams {
     uint32_t S8 = 0, T8 = 0;  // shard and total length in 8-element vectors
     float dec = 0, b1f = 0, omb1 = 0, b2f = 0, omb2 = 0, epsf = 0;
     double lr = 0;
+    double divisor = 1;       // grad divisor k: unscale by 1 / ((R * k) * scale)
+    double max_norm = 0;      // > 0: clipping on (two-pass path)
+    int32_t clip = 0;
     int64_t interval = 1;
     float growth = 2, backoff = 0.5f, min_scale = 1;
     DevState* st = nullptr;
@@ -67,7 +70,9 @@ struct RankPtrs {
 cudaError_t launch_fused_step(const StepParams& sp, const RankPtrs& p, cudaStream_t s);
 cudaError_t launch_step_from_acc(const StepParams& sp, const RankPtrs& p, cudaStream_t s);
 cudaError_t launch_reduce_scatter(int32_t R, int32_t dtype, int64_t S, int64_t lo, int64_t hi,
-                                  DevState* st, const RankPtrs& p, cudaStream_t s);
+                                  DevState* st, const RankPtrs& p, cudaStream_t s,
+                                  bool accumulate = false);
+cudaError_t launch_clip_norm(const StepParams& sp, const RankPtrs& p, cudaStream_t s);
 cudaError_t launch_gather(int32_t R, int64_t S, int64_t lo, int64_t hi, const DevState* st,
                           const RankPtrs& p, void* out, cudaStream_t s);
 

@@ -39,7 +39,9 @@ namespace zb {
 __device__ __forceinline__ Coef make_coef(const StepParams& sp, int R, float scale, int64_t t1) {
     Coef c;
     const double dscale = sp.mode == ZERO_SCALE_NONE ? 1.0 : static_cast<double>(scale);
-    c.inv = __double2float_rn(__ddiv_rn(1.0, __dmul_rn(static_cast<double>(R), dscale)));
+    c.inv = __double2float_rn(
+        __ddiv_rn(1.0, __dmul_rn(__dmul_rn(static_cast<double>(R), sp.divisor), dscale)));
+    c.clip = 1.0f;
     c.dec = sp.dec;
     c.b1f = sp.b1f;
     c.omb1 = sp.omb1;
@@ -70,6 +72,7 @@ __device__ __forceinline__ void read_prologue(const StepParams& sp, int R, Prolo
         out->src = cur;
         out->dst = sp.pingpong ? (cur ^ 1) : cur;
         out->skip = skip_on_flag && sp.mode == ZERO_SCALE_DYNAMIC && st->flag != 0u;
+        if (sp.clip) out->c.clip = st->clip;
     }
     __syncthreads();
 }
@@ -217,7 +220,7 @@ struct AccArgs {
     uint4* param[2][ZERO_MAX_RANKS];
 };
 
-template <typename H>
+template <typename H, bool CLIP>
 __global__ void __launch_bounds__(kThreads) step_from_acc_kernel(const __grid_constant__ AccArgs a) {
     const StepParams& sp = a.sp;
     __shared__ Prologue pro;
@@ -249,7 +252,7 @@ __global__ void __launch_bounds__(kThreads) step_from_acc_kernel(const __grid_co
         float out[8];
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
-            const float g = adamw1(c, acc.x[e], p.x[e], m.x[e], v.x[e]);
+            const float g = adamw1<CLIP>(c, acc.x[e], p.x[e], m.x[e], v.x[e]);
             const double gd = static_cast<double>(g);
             nrm = fma(gd, gd, nrm);
             out[e] = p.x[e];
@@ -260,6 +263,65 @@ __global__ void __launch_bounds__(kThreads) step_from_acc_kernel(const __grid_co
         st_u4(a.param[cur][o] + (j8 >> 3), pack8<H>(out));
     }
     step_epilogue(sp, nrm, false);
+}
+
+// ---------------------------------------------------------------------------
+// Global gradient norm for clipping, before the two-pass step: one read of
+// the accumulators. The last block to finish turns the sum of squares into
+// the clipping coefficient min(1, max_norm / (||g|| + 1e-6)) (in double) and
+// stores it in the device state for the step kernel.
+// ---------------------------------------------------------------------------
+
+struct NormArgs {
+    StepParams sp;
+    const float* acc[ZERO_MAX_RANKS];
+};
+
+__global__ void __launch_bounds__(kThreads) clip_norm_kernel(const __grid_constant__ NormArgs a) {
+    const StepParams& sp = a.sp;
+    __shared__ float s_inv;
+    __shared__ double red[kWarps];
+    __shared__ int last;
+    if (threadIdx.x == 0) {
+        const volatile DevState* st = sp.st;
+        const double dscale = sp.mode == ZERO_SCALE_NONE ? 1.0 : static_cast<double>(st->scale);
+        s_inv = __double2float_rn(
+            __ddiv_rn(1.0, __dmul_rn(__dmul_rn(static_cast<double>(sp.R), sp.divisor), dscale)));
+    }
+    __syncthreads();
+    const float inv = s_inv;
+    double nrm = 0.0;
+    const uint32_t stride = gridDim.x * kThreads;
+    uint32_t vi = blockIdx.x * kThreads + threadIdx.x;
+    OwnerCursor oc(vi, sp.S8);
+    for (; vi < sp.T8; vi += stride) {
+        oc.seek(vi);
+        const F8 acc = ld_f8(a.acc[oc.o] + static_cast<size_t>(vi - oc.base) * 8);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+            const double gd = static_cast<double>(__fmul_rn(acc.x[e], inv));
+            nrm = fma(gd, gd, nrm);
+        }
+    }
+    const double bn = block_sum(nrm, red);
+    if (threadIdx.x == 0) {
+        sp.partials[blockIdx.x] = bn;
+        __threadfence();
+        last = (atomicAdd(&sp.st->done, 1u) == gridDim.x - 1);
+    }
+    __syncthreads();
+    if (!last) return;
+    __threadfence();
+    double x = 0.0;
+    for (unsigned i = threadIdx.x; i < gridDim.x; i += kThreads)
+        x += *reinterpret_cast<volatile double*>(&sp.partials[i]);
+    const double total = block_sum(x, red);
+    if (threadIdx.x == 0) {
+        const double cd = __ddiv_rn(sp.max_norm, __dadd_rn(__dsqrt_rn(total), 1e-6));
+        sp.st->clip = __double2float_rn(cd < 1.0 ? cd : 1.0);
+        sp.st->done = 0u;
+        __threadfence();
+    }
 }
 
 // ---------------------------------------------------------------------------
@@ -280,7 +342,7 @@ struct RsArgs {
     float* acc[CAP];
 };
 
-template <typename H, int RC>
+template <typename H, int RC, bool ACCUM>
 __global__ void __launch_bounds__(kThreads)
     reduce_scatter_kernel(const __grid_constant__ RsArgs<RC == 0 ? ZERO_MAX_RANKS : RC> a) {
     const int R = RC > 0 ? RC : a.R;
@@ -304,13 +366,19 @@ __global__ void __launch_bounds__(kThreads)
 #pragma unroll 4
             for (int r = 1; r < R; ++r) add8<H>(ld_grad(a.g[r] + vi), acc);
         }
+        float* dst = a.acc[oc.o] + static_cast<size_t>(vi - oc.base) * 8;
         F8 out;
+        if constexpr (ACCUM) {
+            const F8 old = ld_f8(dst);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) acc[e] = __fadd_rn(old.x[e], acc[e]);
+        }
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
             bad |= nonfinite(acc[e]);
             out.x[e] = acc[e];
         }
-        st_f8(a.acc[oc.o] + static_cast<size_t>(vi - oc.base) * 8, out);
+        st_f8(dst, out);
     }
     // unaligned edges, element by element
     const int64_t nhead = a.head_end - a.lo;
@@ -321,8 +389,10 @@ __global__ void __launch_bounds__(kThreads)
         float s = H::one(ld_grad1(reinterpret_cast<const uint16_t*>(a.g[0]) + i));
         for (int r = 1; r < R; ++r)
             s = __fadd_rn(s, H::one(ld_grad1(reinterpret_cast<const uint16_t*>(a.g[r]) + i)));
+        float* dst = a.acc[o] + (i - o * a.S);
+        if constexpr (ACCUM) s = __fadd_rn(*dst, s);
         bad |= nonfinite(s);
-        a.acc[o][i - o * a.S] = s;
+        *dst = s;
     }
     if (__syncthreads_or(bad ? 1 : 0) && threadIdx.x == 0) atomicOr(&a.st->flag, 1u);
 }
@@ -482,7 +552,7 @@ cudaError_t fused_dispatch(const StepParams& sp, const RankPtrs& p, cudaStream_t
     }
 }
 
-template <typename H, int RC>
+template <typename H, int RC, bool ACCUM>
 cudaError_t rs_t(int32_t R, int64_t S, int64_t lo, int64_t hi, DevState* st, const RankPtrs& p,
                  cudaStream_t s) {
     constexpr int CAP = RC == 0 ? ZERO_MAX_RANKS : RC;
@@ -509,28 +579,28 @@ cudaError_t rs_t(int32_t R, int64_t S, int64_t lo, int64_t hi, DevState* st, con
         a.g[r] = static_cast<const uint4*>(p.g[r]);
         a.acc[r] = p.acc[r];
     }
-    static const int per_sm = blocks_per_sm(reduce_scatter_kernel<H, RC>);
+    static const int per_sm = blocks_per_sm(reduce_scatter_kernel<H, RC, ACCUM>);
     const uint64_t items = static_cast<uint64_t>(a.v1 - a.v0);
     const uint64_t edges = static_cast<uint64_t>((a.head_end - lo) + (hi - a.tail_begin));
     const uint32_t grid = grid_for(items > edges ? items : edges, per_sm, 0);
-    reduce_scatter_kernel<H, RC><<<grid, kThreads, 0, s>>>(a);
+    reduce_scatter_kernel<H, RC, ACCUM><<<grid, kThreads, 0, s>>>(a);
     return cudaGetLastError();
 }
 
-template <typename H>
+template <typename H, bool ACCUM>
 cudaError_t rs_dispatch(int32_t R, int64_t S, int64_t lo, int64_t hi, DevState* st,
                         const RankPtrs& p, cudaStream_t s) {
     switch (R) {
-        case 1: return rs_t<H, 1>(R, S, lo, hi, st, p, s);
-        case 2: return rs_t<H, 2>(R, S, lo, hi, st, p, s);
-        case 4: return rs_t<H, 4>(R, S, lo, hi, st, p, s);
-        case 8: return rs_t<H, 8>(R, S, lo, hi, st, p, s);
-        case 16: return rs_t<H, 16>(R, S, lo, hi, st, p, s);
-        default: return rs_t<H, 0>(R, S, lo, hi, st, p, s);
+        case 1: return rs_t<H, 1, ACCUM>(R, S, lo, hi, st, p, s);
+        case 2: return rs_t<H, 2, ACCUM>(R, S, lo, hi, st, p, s);
+        case 4: return rs_t<H, 4, ACCUM>(R, S, lo, hi, st, p, s);
+        case 8: return rs_t<H, 8, ACCUM>(R, S, lo, hi, st, p, s);
+        case 16: return rs_t<H, 16, ACCUM>(R, S, lo, hi, st, p, s);
+        default: return rs_t<H, 0, ACCUM>(R, S, lo, hi, st, p, s);
     }
 }
 
-template <typename H>
+template <typename H, bool CLIP>
 cudaError_t acc_t(const StepParams& sp, const RankPtrs& p, cudaStream_t s) {
     AccArgs a;
     a.sp = sp;
@@ -543,9 +613,9 @@ cudaError_t acc_t(const StepParams& sp, const RankPtrs& p, cudaStream_t s) {
             a.param[k][r] = static_cast<uint4*>(p.param[k][r]);
         }
     }
-    static const int per_sm = blocks_per_sm(step_from_acc_kernel<H>);
+    static const int per_sm = blocks_per_sm(step_from_acc_kernel<H, CLIP>);
     const uint32_t grid = grid_for(sp.T8, per_sm, sp.grid_cap);
-    step_from_acc_kernel<H><<<grid, kThreads, 0, s>>>(a);
+    step_from_acc_kernel<H, CLIP><<<grid, kThreads, 0, s>>>(a);
     return cudaGetLastError();
 }
 
@@ -556,13 +626,27 @@ cudaError_t launch_fused_step(const StepParams& sp, const RankPtrs& p, cudaStrea
 }
 
 cudaError_t launch_step_from_acc(const StepParams& sp, const RankPtrs& p, cudaStream_t s) {
-    return sp.dtype == ZERO_FP16 ? acc_t<Fp16>(sp, p, s) : acc_t<Bf16>(sp, p, s);
+    if (sp.clip) return sp.dtype == ZERO_FP16 ? acc_t<Fp16, true>(sp, p, s) : acc_t<Bf16, true>(sp, p, s);
+    return sp.dtype == ZERO_FP16 ? acc_t<Fp16, false>(sp, p, s) : acc_t<Bf16, false>(sp, p, s);
 }
 
 cudaError_t launch_reduce_scatter(int32_t R, int32_t dtype, int64_t S, int64_t lo, int64_t hi,
-                                  DevState* st, const RankPtrs& p, cudaStream_t s) {
-    return dtype == ZERO_FP16 ? rs_dispatch<Fp16>(R, S, lo, hi, st, p, s)
-                              : rs_dispatch<Bf16>(R, S, lo, hi, st, p, s);
+                                  DevState* st, const RankPtrs& p, cudaStream_t s, bool accumulate) {
+    if (accumulate)
+        return dtype == ZERO_FP16 ? rs_dispatch<Fp16, true>(R, S, lo, hi, st, p, s)
+                                  : rs_dispatch<Bf16, true>(R, S, lo, hi, st, p, s);
+    return dtype == ZERO_FP16 ? rs_dispatch<Fp16, false>(R, S, lo, hi, st, p, s)
+                              : rs_dispatch<Bf16, false>(R, S, lo, hi, st, p, s);
+}
+
+cudaError_t launch_clip_norm(const StepParams& sp, const RankPtrs& p, cudaStream_t s) {
+    NormArgs a;
+    a.sp = sp;
+    for (int r = 0; r < sp.R; ++r) a.acc[r] = p.acc[r];
+    static const int per_sm = blocks_per_sm(clip_norm_kernel);
+    const uint32_t grid = grid_for(sp.T8, per_sm, sp.grid_cap);
+    clip_norm_kernel<<<grid, kThreads, 0, s>>>(a);
+    return cudaGetLastError();
 }
 
 cudaError_t launch_gather_many(int32_t R, int64_t S, int nl, const int64_t* lo, const int64_t* hi,

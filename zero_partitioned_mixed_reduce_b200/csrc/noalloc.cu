@@ -222,6 +222,7 @@ extern "C" zero_status zero_step_noalloc(const zero_plan_t* plan, const zero_los
     a.c.epsf = static_cast<float>(hp->eps);
     a.c.ss = static_cast<float>(hp->lr / (1.0 - std::pow(hp->beta1, t1)));
     a.c.bc2s = static_cast<float>(std::sqrt(1.0 - std::pow(hp->beta2, t1)));
+    a.c.clip = 1.0f;
     a.dynamic = cfg->mode == ZERO_SCALE_DYNAMIC;
     a.S8 = static_cast<uint32_t>(plan->S / 8);
     a.T8 = static_cast<uint32_t>(plan->T / 8);
