@@ -426,6 +426,9 @@ extern "C" zero_status zero_loss_scale(zero_ctx_t* ctx, zero_loss_scale_state* i
         cudaError_t e = cudaMemcpyAsync(&d, ctx->st, sizeof(d), cudaMemcpyDeviceToHost, cs);
         if (e == cudaSuccess) e = cudaStreamSynchronize(cs);
         if (e != cudaSuccess) return cuda_fail(where, e);
+        if (d.err == 2)
+            return zb_fail(ZERO_ERR_TIMEOUT, "zero_loss_scale: a step kernel gave up waiting for its "
+                                             "tile copies (2 s); the step's results are incomplete");
         if (d.err != 0)
             return zb_fail(ZERO_ERR_STATE, "zero_loss_scale: device reported an inconsistent step "
                                            "counter (power table behind t)");

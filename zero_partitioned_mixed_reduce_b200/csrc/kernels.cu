@@ -205,6 +205,172 @@ __global__ void __launch_bounds__(kThreads)
 }
 
 // ---------------------------------------------------------------------------
+// The same fused step with the read streams staged through shared memory by
+// the Tensor Memory Accelerator: one thread issues 1-D bulk copies
+// (cp.async.bulk, no multicast) of a whole tile -- R gradient segments and
+// the master/m/v segments of one shard -- into a 2-stage ring completed by
+// mbarrier transaction counts, while the block computes the previous tile
+// from shared memory. Loads in flight then cost no registers. Used when R is
+// small: the per-element read (2R + 12 bytes) leaves room for 3 blocks of 256
+// threads per SM, and the register path keeps too few bytes in flight. Tiles
+// are shard-local (2048 elements, the last one of a shard shorter). Every
+// mbarrier wait gives up after 2 s of %globaltimer: the block then records
+// ZERO_ERR_TIMEOUT in the device state, waits (bounded) for its copies in
+// flight, and finishes without updating further tiles.
+// ---------------------------------------------------------------------------
+
+constexpr int kTmaTile = kThreads * 8;
+constexpr int kTmaStages = 2;
+constexpr int kErrTimeout = 2;
+
+template <int RC>
+struct TmaStage {
+    static constexpr int kGradBytes = RC * kTmaTile * 2;
+    static constexpr int kBytes = kGradBytes + 3 * kTmaTile * 4;
+    static constexpr int kSmem = kTmaStages * kBytes;
+};
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
+}
+__device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+        "l"(src), "r"(bytes), "r"(bar)
+        : "memory");
+}
+__device__ __forceinline__ uint64_t global_ns() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
+    return t;
+}
+// True once the phase of `parity` has completed; false after 2 s.
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
+    uint64_t t0 = 0;
+    for (uint32_t it = 0;; ++it) {
+        uint32_t done;
+        asm volatile(
+            "{ .reg .pred p; mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2; selp.u32 %0, 1, 0, p; }"
+            : "=r"(done)
+            : "r"(bar), "r"(parity)
+            : "memory");
+        if (done) return true;
+        if ((it & 63) == 0) {
+            const uint64_t t = global_ns();
+            if (t0 == 0)
+                t0 = t;
+            else if (t - t0 > 2000000000ull)
+                return false;
+        }
+    }
+}
+__device__ __forceinline__ uint4 lds16(const void* p) { return *reinterpret_cast<const uint4*>(p); }
+
+template <typename H, int RC>
+__global__ void __launch_bounds__(kThreads)
+    fused_step_tma_kernel(const __grid_constant__ FusedArgs<RC> a, uint32_t tiles_per_shard) {
+    using L = TmaStage<RC>;
+    extern __shared__ __align__(128) unsigned char smem[];
+    __shared__ __align__(8) uint64_t bars[kTmaStages];
+    const StepParams& sp = a.sp;
+    __shared__ Prologue pro;
+    read_prologue(sp, RC, &pro, false);
+    const Coef c = pro.c;
+    const int src = pro.src, dst = pro.dst;
+    const uint32_t S = sp.S8 * 8;
+    const uint32_t ntiles = RC * tiles_per_shard;
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kTmaStages; ++s) mbar_init(smem_u32(&bars[s]), 1);
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    __syncthreads();
+    // one thread queues tile `tile` into stage s
+    auto issue = [&](uint32_t tile, int s) {
+        const uint32_t o = tile / tiles_per_shard;
+        const uint32_t j0 = (tile - o * tiles_per_shard) * kTmaTile;
+        const uint32_t len = min(static_cast<uint32_t>(kTmaTile), S - j0);
+        unsigned char* base = smem + s * L::kBytes;
+        const uint32_t bar = smem_u32(&bars[s]);
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        mbar_expect_tx(bar, len * (RC * 2 + 12));
+#pragma unroll
+        for (int r = 0; r < RC; ++r)
+            bulk_g2s(smem_u32(base + r * kTmaTile * 2),
+                     reinterpret_cast<const uint16_t*>(a.g[r]) + static_cast<size_t>(o) * S + j0, len * 2,
+                     bar);
+        bulk_g2s(smem_u32(base + L::kGradBytes), a.master[src][o] + j0, len * 4, bar);
+        bulk_g2s(smem_u32(base + L::kGradBytes + kTmaTile * 4), a.m[src][o] + j0, len * 4, bar);
+        bulk_g2s(smem_u32(base + L::kGradBytes + 2 * kTmaTile * 4), a.v[src][o] + j0, len * 4, bar);
+    };
+    if (threadIdx.x == 0)
+        for (int s = 0; s < kTmaStages; ++s) {
+            const uint32_t tile = blockIdx.x + s * gridDim.x;
+            if (tile < ntiles) issue(tile, s);
+        }
+    double nrm = 0.0;
+    bool bad = false, failed = false;
+    int j = 0;
+    for (uint32_t tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++j) {
+        const int s = j % kTmaStages;
+        const bool ok = mbar_wait(smem_u32(&bars[s]), (j / kTmaStages) & 1);
+        if (__syncthreads_or(!ok)) {
+            failed = true;
+            break;
+        }
+        const uint32_t o = tile / tiles_per_shard;
+        const uint32_t j0 = (tile - o * tiles_per_shard) * kTmaTile;
+        const uint32_t len = min(static_cast<uint32_t>(kTmaTile), S - j0);
+        const uint32_t e0 = threadIdx.x * 8;
+        if (e0 < len) {
+            const unsigned char* base = smem + s * L::kBytes;
+            uint4 gv[RC];
+#pragma unroll
+            for (int r = 0; r < RC; ++r) gv[r] = lds16(base + r * kTmaTile * 2 + e0 * 2);
+            const float* ps = reinterpret_cast<const float*>(base + L::kGradBytes);
+            F8 p, m, v;
+            *reinterpret_cast<uint4*>(&p.x[0]) = lds16(ps + e0);
+            *reinterpret_cast<uint4*>(&p.x[4]) = lds16(ps + e0 + 4);
+            *reinterpret_cast<uint4*>(&m.x[0]) = lds16(ps + kTmaTile + e0);
+            *reinterpret_cast<uint4*>(&m.x[4]) = lds16(ps + kTmaTile + e0 + 4);
+            *reinterpret_cast<uint4*>(&v.x[0]) = lds16(ps + 2 * kTmaTile + e0);
+            *reinterpret_cast<uint4*>(&v.x[4]) = lds16(ps + 2 * kTmaTile + e0 + 4);
+            float acc[8];
+            unpack8<H>(gv[0], acc);
+#pragma unroll
+            for (int r = 1; r < RC; ++r) add8<H>(gv[r], acc);
+            float out[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                bad |= nonfinite(acc[e]);
+                const double gd = static_cast<double>(adamw1(c, acc[e], p.x[e], m.x[e], v.x[e]));
+                nrm = fma(gd, gd, nrm);
+                out[e] = p.x[e];
+            }
+            const size_t jj = static_cast<size_t>(j0) + e0;
+            st_f8(a.master[dst][o] + jj, p);
+            st_f8(a.m[dst][o] + jj, m);
+            st_f8(a.v[dst][o] + jj, v);
+            st_u4(a.param[dst][o] + (jj >> 3), pack8<H>(out));
+        }
+        __syncthreads();  // every thread is done with stage s
+        const uint32_t next = tile + kTmaStages * gridDim.x;
+        if (threadIdx.x == 0 && next < ntiles) issue(next, s);
+    }
+    if (failed) {
+        if (threadIdx.x == 0) sp.st->err = kErrTimeout;
+        for (int k = 0; k < kTmaStages; ++k)  // let copies in flight land (bounded)
+            mbar_wait(smem_u32(&bars[(j + k) % kTmaStages]), ((j + k) / kTmaStages) & 1);
+    }
+    step_epilogue(sp, nrm, bad);
+}
+
+// ---------------------------------------------------------------------------
 // Two-pass step: AdamW from the fp32 accumulators written by the
 // reduce-scatter kernel. In place on set cur; skipped (state untouched) in
 // DYNAMIC mode when the reduce-scatter raised the overflow flag. The norm is
@@ -540,11 +706,38 @@ cudaError_t fused_t(const StepParams& sp, const RankPtrs& p, cudaStream_t s) {
     return cudaGetLastError();
 }
 
+template <typename H, int RC>
+cudaError_t fused_tma_t(const StepParams& sp, const RankPtrs& p, cudaStream_t s) {
+    FusedArgs<RC> a;
+    a.sp = sp;
+    for (int r = 0; r < RC; ++r) {
+        a.g[r] = static_cast<const uint4*>(p.g[r]);
+        for (int k = 0; k < 2; ++k) {
+            a.master[k][r] = p.master[k][r];
+            a.m[k][r] = p.m[k][r];
+            a.v[k][r] = p.v[k][r];
+            a.param[k][r] = static_cast<uint4*>(p.param[k][r]);
+        }
+    }
+    constexpr int smem = TmaStage<RC>::kSmem;
+    static const int per_sm = [] {
+        cudaFuncSetAttribute(fused_step_tma_kernel<H, RC>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+        int n = 0;
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, fused_step_tma_kernel<H, RC>, kThreads, smem);
+        return n > 0 ? n : 1;
+    }();
+    const uint32_t S = sp.S8 * 8;
+    const uint32_t tiles_per_shard = (S + kTmaTile - 1) / kTmaTile;
+    const uint32_t grid = grid_for(static_cast<uint64_t>(tiles_per_shard) * RC * kThreads, per_sm, sp.grid_cap);
+    fused_step_tma_kernel<H, RC><<<grid, kThreads, smem, s>>>(a, tiles_per_shard);
+    return cudaGetLastError();
+}
+
 template <typename H>
 cudaError_t fused_dispatch(const StepParams& sp, const RankPtrs& p, cudaStream_t s) {
     switch (sp.R) {
-        case 1: return fused_t<H, 1>(sp, p, s);
-        case 2: return fused_t<H, 2>(sp, p, s);
+        case 1: return fused_tma_t<H, 1>(sp, p, s);
+        case 2: return fused_tma_t<H, 2>(sp, p, s);
         case 4: return fused_t<H, 4>(sp, p, s);
         case 8: return fused_t<H, 8>(sp, p, s);
         case 16: return fused_t<H, 16>(sp, p, s);
