@@ -56,6 +56,14 @@ def parse_args(argv=None):
     ap.add_argument("--gather-bucket", type=int, default=32 << 20,
                     help="gather consecutive layers in one launch up to this many elements "
                          "(0: one launch per layer)")
+    ap.add_argument("--overlap", action="store_true",
+                    help="measure the overlap scheduler on a synthetic training step instead")
+    ap.add_argument("--tokens", type=int, default=4096,
+                    help="tokens per synthetic GEMM in --overlap mode")
+    ap.add_argument("--bucket-elems", type=int, default=None,
+                    help="override the workload's reduce-scatter bucket size")
+    ap.add_argument("--carveout", type=int, default=0,
+                    help="SMs kept free of the synthetic GEMMs in --overlap mode")
     ap.add_argument("--first-tensors", type=int, default=0,
                     help="use only the first N tensors of the workload (small profiling cases)")
     return ap.parse_args(argv)
@@ -198,11 +206,14 @@ def profiled_traffic(kernel, workload):
 # ---- the workload -------------------------------------------------------------
 
 class Bench:
-    def __init__(self, name, path, first_tensors=0, gather_bucket=32 << 20, accum=1, clip=0.0):
+    def __init__(self, name, path, first_tensors=0, gather_bucket=32 << 20, accum=1, clip=0.0,
+                 bucket_elems=None):
         import zero_partitioned_mixed_reduce_b200 as Z
         from zero_partitioned_mixed_reduce_b200 import synth
         self.Z, self.synth = Z, synth
         self.wl = wl = synth.workload(name)
+        if bucket_elems is not None:
+            wl["bucket_elems"] = bucket_elems
         if first_tensors:
             wl["numels"] = wl["numels"][:first_tensors]
             wl["layer_ids"] = wl["layer_ids"][:first_tensors] if wl["layer_ids"] else None
@@ -491,6 +502,110 @@ def cpu_baseline(name):
                       f"{dt:.1f} s single-threaded"}
 
 
+def run_overlap(args, world, rank, local):
+    """A synthetic ZeRO-3 training step on the workload's layers: forward
+    (gather layer, one bf16 GEMM of 2 * tokens * n_layer flops on it), backward
+    (gather again, two GEMMs, report the layer's gradients), then the two-pass
+    optimizer step. Timed three ways: overlapped through the scheduler's
+    communication stream and look-ahead ring, serialized on one stream, and
+    compute only (no gathers, no reduce-scatters)."""
+    if not torch.cuda.is_available():
+        print(json.dumps({"error": "no CUDA device"}))
+        sys.exit(1)
+    b = Bench(args.workload, "twopass", args.first_tensors, 0, bucket_elems=args.bucket_elems)
+    Z = b.Z
+    stream = torch.cuda.current_stream()
+    wl, plan = b.wl, b.plan
+    d = 768 if args.workload == "gpt2s" else 2048
+    nl = len(plan.layers)
+    lids = wl["layer_ids"]
+    first_t = [lids.index(l) for l in range(nl)]
+    count_t = [lids.count(l) for l in range(nl)]
+    biggest = b.max_layer
+    nbufs, depth = 3, 1
+    bufs = [torch.empty(biggest + 8, dtype=torch.bfloat16, device="cuda") for _ in range(nbufs)]
+    by_addr = {t.data_ptr(): t for t in bufs}
+    x = torch.randn(args.tokens, d, device="cuda", dtype=torch.bfloat16)
+
+    def gemm(buf, l):
+        # [tokens x d] @ [d x N] on the gathered layer; N a multiple of 64 keeps
+        # the operand aligned for the tensor-core GEMM path
+        lo, hi = plan.layers[l]
+        n = ((hi - lo) // (d * 64)) * (d * 64)
+        w = buf[:n].view(d, n // d)
+        return x @ w
+
+    def step_overlap():
+        Z.zero_prefetch_begin(b.ctx, b.state.handle, bufs, depth, 1, stream)
+        for l in range(nl):
+            buf = by_addr[Z.zero_layer_acquire(b.ctx, l, stream)]
+            gemm(buf, l)
+            Z.zero_layer_release(b.ctx, l, stream)
+        Z.zero_prefetch_begin(b.ctx, b.state.handle, bufs, depth, -1, stream)
+        for l in reversed(range(nl)):
+            buf = by_addr[Z.zero_layer_acquire(b.ctx, l, stream)]
+            gemm(buf, l)
+            gemm(buf, l)
+            Z.zero_layer_release(b.ctx, l, stream)
+            Z.zero_grads_ready(b.ctx, first_t[l], count_t[l], b.grads, b.state.acc, 0, stream)
+        Z.zero_grads_join(b.ctx, stream)
+        Z.zero_step(b.ctx, wl["hp"], b.state.handle, None, stream)
+
+    def step_serial(comm=True):
+        buf = bufs[0]
+        for l in range(nl):
+            if comm:
+                Z.zero_gather_layer(b.ctx, l, b.state.handle, buf, stream)
+            gemm(buf, l)
+        done = 0
+        for l in reversed(range(nl)):
+            if comm:
+                Z.zero_gather_layer(b.ctx, l, b.state.handle, buf, stream)
+            gemm(buf, l)
+            gemm(buf, l)
+            # buckets complete once all their tensors (from the last one down) are done
+            lowest = first_t[l]
+            while comm and done < len(plan.buckets) and plan.buckets[done][0] >= plan.offsets[lowest]:
+                Z.zero_reduce_scatter_bucket(b.ctx, done, b.grads, b.state.acc, stream)
+                done += 1
+        Z.zero_step(b.ctx, wl["hp"], b.state.handle, None, stream)
+
+    def timed(fn, reps):
+        for _ in range(args.warmup):
+            fn()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(reps):
+            fn()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / reps
+
+    if args.carveout:
+        torch._C._set_sm_carveout_experimental(args.carveout)
+    reps = max(3, min(args.steps, 50))
+    # fill the accumulators once; the compute-only variant steps from them
+    Z.zero_reduce_scatter_bucket(b.ctx, -1, b.grads, b.state.acc, stream)
+    t_ovl = timed(step_overlap, reps)
+    t_ser = timed(step_serial, reps)
+    t_cmp = timed(lambda: step_serial(comm=False), reps)
+    hidden = (t_ser - t_ovl) / (t_ser - t_cmp) if t_ser > t_cmp else None
+    gemm_flops = 6.0 * args.tokens * sum(((hi - lo) // (d * 64)) * (d * 64) for lo, hi in plan.layers)
+    out = {"mode": "overlap", "workload": args.workload, "tokens": args.tokens,
+           "bucket_elems": wl["bucket_elems"],
+           "gemm_carveout_sms": args.carveout,
+           "gemm_tflops_in_compute_only": gemm_flops / (t_cmp * 1e-3) / 1e12,
+           "layers": nl, "buckets": len(plan.buckets), "ring": {"nbufs": nbufs, "depth": depth},
+           "ms_overlapped": t_ovl, "ms_serialized": t_ser,
+           "ms_compute_and_step_only": t_cmp,
+           "comm_ms_serialized": t_ser - t_cmp, "comm_ms_exposed_overlapped": t_ovl - t_cmp,
+           "fraction_of_comm_hidden": hidden, "steps": reps}
+    b.close()
+    if rank == 0:
+        print(json.dumps(out), flush=True)
+
+
 def run_reference(args, world, rank):
     """The oracle on host cores: each step a bounded prefix sample."""
     if rank != 0:
@@ -529,6 +644,8 @@ def main(argv=None):
     try:
         if args.impl == "reference":
             run_reference(args, world, rank)
+        elif args.overlap:
+            run_overlap(args, world, rank, local)
         else:
             run_ours(args, world, rank, local)
     finally:

@@ -400,6 +400,71 @@ zero_status zero_step_noalloc(const zero_plan_t* plan, const zero_loss_scale_con
                               const void* const* grads, float* const* master, float* const* m,
                               float* const* v, void* const* param, void* stream);
 
+/* ------------------------------------------------------------------------ */
+/* Overlap and prefetch scheduling (a communication stream owned by the     */
+/* context, created on first use with the highest stream priority).         */
+/* ------------------------------------------------------------------------ */
+
+/*
+ * zero_grads_ready -- report that tensors [first, first+count) have their
+ * gradients written in `grads` by the work queued on `stream` so far. Each
+ * bucket whose tensors have then all been reported is reduce-scattered at
+ * once (as zero_reduce_scatter_bucket_ex with `flags`) on the communication
+ * stream, ordered after that work by an event, so the reduction of early
+ * buckets overlaps the caller's next work on `stream`.
+ * Defines: [legal] "Communication Overlap" (a layer's gradient reduction
+ * starts as soon as its gradients are computed, hidden behind the backward
+ * pass) and [genomic] "Reduce-Scatter Overlap".
+ * grads / acc: as zero_reduce_scatter_bucket; they must stay the same
+ * buffers until zero_grads_join.
+ * Errors: ZERO_ERR_RANGE, ZERO_ERR_INVALID_ARG, ZERO_ERR_ALIGN,
+ * ZERO_ERR_STATE (a tensor reported twice before the join), ZERO_ERR_CUDA.
+ */
+zero_status zero_grads_ready(zero_ctx_t* ctx, int64_t first, int64_t count, const void* const* grads,
+                             float* const* acc, int32_t flags, void* stream);
+
+/*
+ * zero_grads_join -- make `stream` wait for every reduce-scatter issued by
+ * zero_grads_ready, and start a new round of reports (the next micro-batch
+ * or step). Every tensor must have been reported, else ZERO_ERR_STATE.
+ * A two-pass zero_step / zero_step_ex (grads == NULL) on `stream` follows.
+ */
+zero_status zero_grads_join(zero_ctx_t* ctx, void* stream);
+
+/*
+ * zero_prefetch_begin -- start one pass over the layers (direction +1:
+ * layer 0 first, the forward pass; -1: the last layer first, the backward
+ * pass) with look-ahead gathering: the layer at sequence position p is
+ * gathered (as zero_gather_layer, from the current parameter set) into
+ * bufs[p % nbufs] on the communication stream, up to `depth` positions
+ * ahead of the layer in use. A slot is refilled only after the layer it held
+ * has been released. All gathers of the pass come after the work queued on
+ * `stream` before this call (for example the optimizer step).
+ * Defines: [legal] ZeRO-3 "Prefetching Scheduler" (a look-ahead scheduler
+ * fetches the next parameters while the current layer computes) and
+ * [genomic] "Bucketed All-Gather" / "Prefetch Scheduling".
+ * bufs: nbufs device pointers (host array, copied), each 16-byte aligned and
+ * large enough for the largest layer; 1 <= nbufs <= 64; 0 <= depth < nbufs.
+ * state: param[0] (and param[1] for ping-pong) as for zero_gather_layer.
+ */
+zero_status zero_prefetch_begin(zero_ctx_t* ctx, const zero_state* state, void* const* bufs,
+                                int32_t nbufs, int32_t depth, int32_t direction, void* stream);
+
+/*
+ * zero_layer_acquire -- *buf receives the buffer that holds `layer`; work
+ * queued on `stream` after this call sees the gathered layer. Also queues the
+ * gathers of the next `depth` layers of the pass whose slots are free.
+ * Errors: ZERO_ERR_STATE when no pass is active or the layer's slot is still
+ * held by an unreleased layer (acquire in pass order, release after use).
+ */
+zero_status zero_layer_acquire(zero_ctx_t* ctx, int64_t layer, void** buf, void* stream);
+
+/*
+ * zero_layer_release -- the work queued on `stream` so far is done with
+ * `layer`'s buffer; its slot may be refilled after that work.
+ */
+zero_status zero_layer_release(zero_ctx_t* ctx, int64_t layer, void* stream);
+
 /* zero_sync -- synchronize `stream` and report any pending CUDA error. */
 zero_status zero_sync(zero_ctx_t* ctx, void* stream);
 

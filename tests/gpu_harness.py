@@ -168,6 +168,45 @@ class Case:
         self.g.check()
         return skipped
 
+    def step_overlap(self, n_micro=1, grad_divisor=1.0, max_grad_norm=0.0, busy=None):
+        """Two-pass step whose reduce-scatters are issued by the overlap
+        scheduler: each tensor's gradients are written on the caller's stream
+        (after `busy` work, standing in for backward) in reverse tensor order,
+        then reported ready; join; step."""
+        assert self.path == "twopass"
+        self.step_no += 1
+        scale = self.ofsm.scale if self.mode != O.SCALE_NONE else 1.0
+        micro = []
+        for mu in range(n_micro):
+            rows = [synth.flat_grads(self.wl, self.step_no * 100 + mu, r, scale, "cpu")
+                    for r in range(self.R)]
+            micro.append(np.stack([u16(t) for t in rows]))
+        g = np.stack(micro)
+        starts = np.concatenate([[0], np.cumsum(self.lay.numels)[:-1]])
+        dev = [torch.from_numpy(g[mu].view(np.int16)).cuda() for mu in range(n_micro)]
+        torch.cuda.synchronize()
+        for r in range(self.R):
+            self.grads[r].zero_()
+        for mu in range(n_micro):
+            for k in reversed(range(len(self.lay.numels))):
+                if busy is not None:
+                    busy()
+                off, n, st = int(self.lay.offsets[k]), int(self.lay.numels[k]), int(starts[k])
+                for r in range(self.R):
+                    self.grads[r].view(torch.int16)[off:off + n].copy_(dev[mu][r, st:st + n])
+                Z.zero_grads_ready(self.ctx, k, 1, self.grads, self.acc,
+                                   Z.ZERO_RS_ACCUMULATE if mu else 0,
+                                   torch.cuda.current_stream())
+            Z.zero_grads_join(self.ctx, torch.cuda.current_stream())
+        Z.zero_step_ex(self.ctx, self.hp, self.handle, None, grad_divisor, max_grad_norm,
+                       torch.cuda.current_stream())
+        skipped = O.step_ex(self.ostate, g, O.AdamW(**{k: self.hp[k] for k in
+                                                       ("lr", "beta1", "beta2", "eps",
+                                                        "weight_decay")}),
+                            self.ofsm, grad_divisor, max_grad_norm)
+        self.g.check()
+        return skipped
+
     def gpu_fsm(self):
         return Z.zero_loss_scale(self.ctx)
 

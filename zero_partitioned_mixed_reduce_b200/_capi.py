@@ -111,6 +111,11 @@ _sig("zero_loss_scale", _S, [_P, C.POINTER(zero_loss_scale_state), C.c_int32, _P
 _sig("zero_step_noalloc", _S, [_P, C.POINTER(zero_loss_scale_config),
                                C.POINTER(zero_loss_scale_state), C.POINTER(zero_adamw), _PP, _PP,
                                _PP, _PP, _PP, _P])
+_sig("zero_grads_ready", _S, [_P, C.c_int64, C.c_int64, _PP, _PP, C.c_int32, _P])
+_sig("zero_grads_join", _S, [_P, _P])
+_sig("zero_prefetch_begin", _S, [_P, C.POINTER(zero_state), _PP, C.c_int32, C.c_int32, C.c_int32, _P])
+_sig("zero_layer_acquire", _S, [_P, C.c_int64, C.POINTER(C.c_void_p), _P])
+_sig("zero_layer_release", _S, [_P, C.c_int64, _P])
 _sig("zero_sync", _S, [_P, _P])
 _sig("zero_last_error", C.c_size_t, [C.c_char_p, C.c_size_t])
 _sig("zero_version", C.c_char_p, [])
@@ -317,6 +322,33 @@ def zero_step_noalloc(plan, cfg, state, hp, grads, master, m, v, param, stream=N
     _check(_lib.zero_step_noalloc(plan, C.byref(c), C.byref(st), C.byref(hp),
                                   *[a[0] for a in arrays], _stream(stream)))
     return {k: getattr(st, k) for k, _ in zero_loss_scale_state._fields_}
+
+
+def zero_grads_ready(ctx, first, count, grads, acc, flags=0, stream=None):
+    g, ga = _ptr_array(grads)
+    a, aa = _ptr_array(acc)
+    _check(_lib.zero_grads_ready(ctx, first, count, g, a, flags, _stream(stream)))
+
+
+def zero_grads_join(ctx, stream=None):
+    _check(_lib.zero_grads_join(ctx, _stream(stream)))
+
+
+def zero_prefetch_begin(ctx, state: StateHandle, bufs, depth, direction=1, stream=None):
+    b, ba = _ptr_array(bufs)
+    _check(_lib.zero_prefetch_begin(ctx, C.byref(state.c), b, len(bufs), depth, direction,
+                                    _stream(stream)))
+
+
+def zero_layer_acquire(ctx, layer, stream=None):
+    """Returns the device address of the buffer holding `layer`."""
+    out = C.c_void_p()
+    _check(_lib.zero_layer_acquire(ctx, layer, C.byref(out), _stream(stream)))
+    return out.value
+
+
+def zero_layer_release(ctx, layer, stream=None):
+    _check(_lib.zero_layer_release(ctx, layer, _stream(stream)))
 
 
 def zero_sync(ctx, stream=None):

@@ -25,7 +25,7 @@ CXX_FLAGS = ["-O2", "-std=c++17", "-fPIC", "-Wall", "-Wextra", "-I", INCLUDE, "-
              "-I", os.path.join(CUDA_HOME, "include")]
 
 CU_SOURCES = ["kernels.cu", "noalloc.cu"]
-CPP_SOURCES = ["plan.cpp", "capi.cpp"]
+CPP_SOURCES = ["plan.cpp", "capi.cpp", "sched.cpp"]
 
 
 def _sources():

@@ -20,22 +20,6 @@ zero_status zb_fail(zero_status code, const std::string& msg) {
     return code;
 }
 
-struct zero_ctx_s {
-    int device = 0;
-    int32_t R = 0, dtype = 0;
-    int64_t S = 0, T = 0;
-    std::vector<int64_t> bucket_lo, bucket_hi, layer_lo, layer_hi;
-    zero_loss_scale_config cfg{};
-    zb::DevState* st = nullptr;   // device
-    double* partials = nullptr;   // device, grid_cap entries
-    int grid_cap = 0;
-    double2* powtab = nullptr;    // device, powtab_len entries
-    int64_t powtab_len = 0;
-    double pow_b1 = NAN, pow_b2 = NAN;
-    int64_t t_bound = 0;          // upper bound of the device step count
-    bool two_sets = false;        // a ping-pong step has run (or cur was set to 1)
-};
-
 namespace {
 
 zero_status cuda_fail(const char* where, cudaError_t e) {
@@ -121,7 +105,8 @@ void fill_state_ptrs(const zero_ctx_t* ctx, const zero_state* st, int sets, zb::
 // Host-built table of (beta1^t, beta2^t), t = 0..len-1, computed with the C
 // library's pow in double; the device forms the bias corrections from it.
 zero_status ensure_powtab(zero_ctx_t* ctx, double b1, double b2, int64_t need_t, cudaStream_t s) {
-    if (ctx->powtab && ctx->pow_b1 == b1 && ctx->pow_b2 == b2 && need_t < ctx->powtab_len)
+    if (ctx->powtab && ctx->pow_valid && ctx->pow_b1 == b1 && ctx->pow_b2 == b2 &&
+        need_t < ctx->powtab_len)
         return ZERO_OK;
     int64_t len = 1024;
     while (len <= need_t) len *= 2;
@@ -144,6 +129,7 @@ zero_status ensure_powtab(zero_ctx_t* ctx, double b1, double b2, int64_t need_t,
     ctx->powtab_len = len;
     ctx->pow_b1 = b1;
     ctx->pow_b2 = b2;
+    ctx->pow_valid = true;
     return ZERO_OK;
 }
 
@@ -184,6 +170,9 @@ extern "C" zero_status zero_ctx_create(const zero_plan_t* plan, const zero_loss_
     ctx->bucket_hi = plan->bucket_hi;
     ctx->layer_lo = plan->layer_lo;
     ctx->layer_hi = plan->layer_hi;
+    ctx->tensor_bucket = plan->tensor_bucket;
+    ctx->bucket_ntensors.assign(plan->bucket_lo.size(), 0);
+    for (int64_t b : plan->tensor_bucket) ctx->bucket_ntensors[b] += 1;
     ctx->cfg = *cfg;
     ctx->grid_cap = zb::step_grid_cap(ctx->device);
 
@@ -215,6 +204,7 @@ extern "C" zero_status zero_ctx_destroy(zero_ctx_t* ctx) {
     cudaGetDevice(&prev);
     cudaSetDevice(ctx->device);
     cudaError_t e = cudaDeviceSynchronize();
+    zb_sched_destroy(ctx);
     cudaFree(ctx->st);
     cudaFree(ctx->partials);
     if (ctx->powtab) cudaFree(ctx->powtab);

@@ -85,5 +85,31 @@ int step_grid_cap(int device);
 
 }  // namespace zb
 
+// Context: the plan's layout, the loss-scale config, the device scratch, and
+// the overlap / prefetch scheduler (sched.cpp).
+struct zero_sched;  // scheduler state, sched.cpp
+
+struct zero_ctx_s {
+    int device = 0;
+    int32_t R = 0, dtype = 0;
+    int64_t S = 0, T = 0;
+    std::vector<int64_t> bucket_lo, bucket_hi, layer_lo, layer_hi;
+    std::vector<int64_t> tensor_bucket;  // bucket of each tensor
+    std::vector<int64_t> bucket_ntensors;
+    zero_loss_scale_config cfg{};
+    zb::DevState* st = nullptr;   // device
+    double* partials = nullptr;   // device, grid_cap entries
+    int grid_cap = 0;
+    double2* powtab = nullptr;    // device, powtab_len entries
+    int64_t powtab_len = 0;
+    double pow_b1 = 0.0, pow_b2 = 0.0;
+    bool pow_valid = false;
+    int64_t t_bound = 0;          // upper bound of the device step count
+    bool two_sets = false;        // a ping-pong step has run (or cur was set to 1)
+    zero_sched* sched = nullptr;  // created on first use
+};
+
+void zb_sched_destroy(zero_ctx_t* ctx);
+
 // Set the calling thread's last error message; returns `code`.
 zero_status zb_fail(zero_status code, const std::string& msg);
