@@ -64,6 +64,8 @@ def parse_args(argv=None):
                     help="override the workload's reduce-scatter bucket size")
     ap.add_argument("--carveout", type=int, default=0,
                     help="SMs kept free of the synthetic GEMMs in --overlap mode")
+    ap.add_argument("--offload", action="store_true",
+                    help="measure ZeRO-Offload (CPU AdamW, with and without the delayed update)")
     ap.add_argument("--first-tensors", type=int, default=0,
                     help="use only the first N tensors of the workload (small profiling cases)")
     return ap.parse_args(argv)
@@ -606,6 +608,131 @@ def run_overlap(args, world, rank, local):
         print(json.dumps(out), flush=True)
 
 
+def run_offload(args, world, rank, local):
+    """ZeRO-Offload on the workload: per step the GPU runs a synthetic
+    forward/backward (bf16 GEMMs of 6 * tokens * P flops) and reduce-scatters
+    the gradients; the fp32 accumulators go to pinned host memory, the AdamW
+    step runs on CPU threads (zero_cpu_step) and the half parameters come back.
+    Timed serialized and with the one-step delayed parameter update (the CPU
+    step of step s overlapping the GPU work of step s+1)."""
+    import threading
+    if not torch.cuda.is_available():
+        print(json.dumps({"error": "no CUDA device"}))
+        sys.exit(1)
+    import zero_partitioned_mixed_reduce_b200 as Z
+    from zero_partitioned_mixed_reduce_b200 import synth
+    wl = synth.workload(args.workload)
+    if args.first_tensors:
+        wl["numels"] = wl["numels"][:args.first_tensors]
+        wl["layer_ids"] = wl["layer_ids"][:args.first_tensors]
+    plan = Z.Plan(wl["numels"], wl["layer_ids"], wl["R"], wl["dtype"], 8, wl["bucket_elems"])
+    R, S, T, P = plan.R, plan.S, plan.T, plan.P
+    half = Z.state.HALF[wl["dtype"]]
+    ctx = Z.zero_ctx_create(plan.handle, wl["mode"], wl["init_scale"], wl["interval"])
+    scale = wl["init_scale"] if wl["mode"] != synth.NONE else 1.0
+    grads = []
+    for r in range(R):
+        g = torch.zeros(T, dtype=half, device="cuda")
+        for k, (n, off) in enumerate(zip(wl["numels"], plan.offsets)):
+            g[off:off + n] = synth.tensor_grads(n, wl["dist"], wl["sigma"], scale, wl["dtype"],
+                                                wl["index"], 1, r, k, "cuda")
+        grads.append(g)
+    acc_gpu = [torch.zeros(S, device="cuda") for _ in range(R)]
+    pin = lambda t: t.pin_memory()
+    master = [pin(torch.randn(S) * 0.02) for _ in range(R)]
+    m = [pin(torch.zeros(S)) for _ in range(R)]
+    v = [pin(torch.zeros(S)) for _ in range(R)]
+    param_host = [pin(torch.zeros(S, dtype=half)) for _ in range(R)]
+    acc_host = [[pin(torch.zeros(S)) for _ in range(R)] for _ in range(2)]
+    param_gpu = [torch.zeros(S, dtype=half, device="cuda") for _ in range(R)]
+    copy = torch.cuda.Stream()
+    d = 768 if args.workload == "gpt2s" else 2048
+    x = torch.randn(args.tokens, d, device="cuda", dtype=torch.bfloat16)
+    w = torch.randn(d, 8192, device="cuda", dtype=torch.bfloat16)
+    n_gemm = max(1, int(round(6.0 * args.tokens * P / (2.0 * args.tokens * d * 8192))))
+    cfg = dict(mode=wl["mode"], growth_interval=wl["interval"])
+    ls = {"state": dict(scale=scale, cur=0, good=0, t=0), "up": None}
+    hp = wl["hp"]
+
+    def gpu_half(slot):
+        for _ in range(n_gemm):
+            x @ w
+        Z.zero_reduce_scatter_bucket(ctx, -1, grads, acc_gpu)
+        ev = torch.cuda.Event()
+        ev.record()
+        copy.wait_event(ev)
+        with torch.cuda.stream(copy):
+            for r in range(R):
+                acc_host[slot][r].copy_(acc_gpu[r], non_blocking=True)
+        done = torch.cuda.Event()
+        done.record(copy)
+        torch.cuda.current_stream().wait_event(done)
+        return done
+
+    def cpu_half(slot, done):
+        done.synchronize()
+        if ls["up"] is not None:
+            ls["up"].synchronize()  # the last upload has finished reading param_host
+        ls["state"] = Z.zero_cpu_step(plan.handle, cfg, ls["state"], hp, acc_host[slot], master, m, v,
+                                      param_host, nthreads=0)
+
+    def upload():
+        with torch.cuda.stream(copy):
+            for r in range(R):
+                param_gpu[r].copy_(param_host[r], non_blocking=True)
+        ev = torch.cuda.Event()
+        ev.record(copy)
+        ls["up"] = ev
+        torch.cuda.current_stream().wait_event(ev)  # the next forward reads the new parameters
+
+    def run(steps, delayed):
+        pending = None
+        for s in range(steps):
+            done = gpu_half(s % 2)
+            if pending is not None:
+                pending.join()
+                upload()
+            th = threading.Thread(target=cpu_half, args=(s % 2, done))
+            th.start()
+            if delayed:
+                pending = th
+            else:
+                th.join()
+                upload()
+        if pending is not None:
+            pending.join()
+            upload()
+        torch.cuda.synchronize()
+
+    def wall(fn):
+        torch.cuda.synchronize()
+        t = time.perf_counter()
+        fn()
+        torch.cuda.synchronize()
+        return time.perf_counter() - t
+
+    K = max(3, min(args.steps, 20))
+    run(args.warmup, False)
+    t_ser = wall(lambda: run(K, False)) / K
+    t_dpu = wall(lambda: run(K, True)) / K
+    # the parts alone
+    t_gpu = wall(lambda: [gpu_half(0) for _ in range(K)]) / K
+    done = gpu_half(0)
+    done.synchronize()
+    t_cpu = wall(lambda: [cpu_half(0, done) for _ in range(K)]) / K
+    t_up = wall(lambda: [upload() for _ in range(K)]) / K
+    out = {"mode": "offload", "workload": args.workload, "P": P, "R": R, "tokens": args.tokens,
+           "host_threads": os.cpu_count(), "gemm_flops_per_step": 2.0 * args.tokens * d * 8192 * n_gemm,
+           "ms_serialized": t_ser * 1e3, "ms_delayed_update": t_dpu * 1e3,
+           "ms_gpu_part": t_gpu * 1e3, "ms_cpu_adamw": t_cpu * 1e3, "ms_param_upload": t_up * 1e3,
+           "cpu_adamw_params_per_s": T / t_cpu, "cpu_adamw_host_GBps": 30.0 * T / t_cpu / 1e9,
+           "speedup_from_delayed_update": t_ser / t_dpu, "steps": K,
+           "timing": "host wall clock around synchronized loops (the CPU step is host work)"}
+    Z.zero_ctx_destroy(ctx)
+    if rank == 0:
+        print(json.dumps(out), flush=True)
+
+
 def run_reference(args, world, rank):
     """The oracle on host cores: each step a bounded prefix sample."""
     if rank != 0:
@@ -646,6 +773,8 @@ def main(argv=None):
             run_reference(args, world, rank)
         elif args.overlap:
             run_overlap(args, world, rank, local)
+        elif args.offload:
+            run_offload(args, world, rank, local)
         else:
             run_ours(args, world, rank, local)
     finally:

@@ -465,6 +465,37 @@ zero_status zero_layer_acquire(zero_ctx_t* ctx, int64_t layer, void** buf, void*
  */
 zero_status zero_layer_release(zero_ctx_t* ctx, int64_t layer, void* stream);
 
+/* ------------------------------------------------------------------------ */
+/* ZeRO-Offload: the optimizer step on CPU cores (host only, no GPU).       */
+/* ------------------------------------------------------------------------ */
+
+/*
+ * zero_cpu_step -- the optimizer step of zero_step_ex on host memory, for
+ * training with the fp32 master weights and Adam moments offloaded to CPU
+ * RAM: acc holds the R reduced fp32 gradient shards (for example copied
+ * from the GPU accumulators after zero_reduce_scatter_bucket), master / m /
+ * v are updated in place, and param receives the half parameters to copy
+ * back to the GPU. The overflow check, loss-scale state machine, grad
+ * divisor and clipping follow zero_step_ex exactly, and the element
+ * arithmetic is the same IEEE fp32 sequence, so results equal the GPU step
+ * bit for bit. inout (host) holds the loss-scale state before the step and
+ * receives it after; cur must be 0.
+ * Defines: [legal] "CPU Offload" (Adam on the CPU while the GPU runs forward
+ * and backward) and [genomic] "CPU Offload" (fp32 master weights and
+ * optimizer states in CPU RAM); [legal] / [genomic] "One-Step Delayed
+ * Parameter Update" is the caller overlapping this call with the next
+ * forward pass (it releases no lock and touches no GPU state).
+ * All pointers are HOST memory: R pointers each, S elements per shard
+ * (pinned memory makes the surrounding copies asynchronous). nthreads <= 0
+ * uses every hardware thread; the result does not depend on nthreads except
+ * for the summation order of grad_norm_sq.
+ * Errors: ZERO_ERR_INVALID_ARG.
+ */
+zero_status zero_cpu_step(const zero_plan_t* plan, const zero_loss_scale_config* cfg,
+                          zero_loss_scale_state* inout, const zero_adamw* hp, const zero_step_opts* opts,
+                          const float* const* acc, float* const* master, float* const* m, float* const* v,
+                          void* const* param, int32_t nthreads);
+
 /* zero_sync -- synchronize `stream` and report any pending CUDA error. */
 zero_status zero_sync(zero_ctx_t* ctx, void* stream);
 

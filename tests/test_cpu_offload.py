@@ -1,0 +1,154 @@
+"""zero_cpu_step (ZeRO-Offload: the optimizer step on CPU cores) against the
+oracle, bit for bit. Host only: these run without a GPU."""
+import numpy as np
+import pytest
+
+import oracle as O
+import zero_partitioned_mixed_reduce_b200 as Z
+
+HP = dict(lr=1e-3, beta1=0.9, beta2=0.999, eps=1e-8, weight_decay=0.01)
+OHP = O.AdamW(1e-3, 0.9, 0.999, 1e-8, 0.01)
+
+
+class Offload:
+    """Host shards of one plan, driven by zero_cpu_step, beside the oracle."""
+
+    def __init__(self, numels, R, dtype, align, mode, scale=256.0, interval=3, seed=0):
+        self.rng = np.random.default_rng(seed)
+        self.lay = O.Layout(numels, R, align)
+        self.plan = Z.Plan(numels, None, R, dtype, align, 0)
+        self.R, self.dtype, self.mode = R, dtype, mode
+        self.idx = self.lay.flat_index()
+        P, T, S = self.lay.P, self.lay.T, self.lay.S
+        x = self.rng.normal(0, 0.02, P).astype(np.float32)
+        self.ost = O.State(x, dtype)
+        flat = np.zeros(T, np.float32)
+        flat[self.idx] = x
+        pflat = np.zeros(T, np.uint16)
+        pflat[self.idx] = self.ost.param
+        self.master = [flat[r * S:(r + 1) * S].copy() for r in range(R)]
+        self.m = [np.zeros(S, np.float32) for _ in range(R)]
+        self.v = [np.zeros(S, np.float32) for _ in range(R)]
+        self.param = [pflat[r * S:(r + 1) * S].copy() for r in range(R)]
+        self.acc = [np.zeros(S, np.float32) for _ in range(R)]
+        self.fsm = O.make_fsm(mode, scale=scale if mode else 1.0, interval=interval)
+        self.cfg = dict(mode=mode, growth_interval=interval)
+        self.ls = dict(scale=scale if mode else 1.0, cur=0, good=0, t=0)
+
+    def step(self, n_micro=1, divisor=1.0, clip=0.0, inject=None, nthreads=0):
+        P, S = self.lay.P, self.lay.S
+        g = O.float_to_half(
+            (self.rng.normal(0, 1e-2, (n_micro, self.R, P)) * self.fsm.scale).astype(np.float32),
+            self.dtype)
+        if inject:
+            g[inject] = 0x7C00 if self.dtype == O.FP16 else 0x7F80
+        acc = None
+        for mu in range(n_micro):
+            s, _ = O.allreduce_sum(g[mu], self.dtype)
+            acc = s if acc is None else acc + s
+        flat = np.zeros(self.lay.T, np.float32)
+        flat[self.idx] = acc
+        for r in range(self.R):
+            self.acc[r][:] = flat[r * S:(r + 1) * S]
+        self.ls = Z.zero_cpu_step(self.plan.handle, self.cfg, self.ls, HP, self.acc, self.master,
+                                  self.m, self.v, self.param, divisor, clip, nthreads)
+        O.step_ex(self.ost, g, OHP, self.fsm, divisor, clip)
+
+    def compare(self):
+        cat = lambda xs: np.concatenate(xs)[self.idx]
+        for name, a, b in (("master", cat(self.master), self.ost.master), ("m", cat(self.m), self.ost.m),
+                           ("v", cat(self.v), self.ost.v)):
+            assert np.array_equal(a.view(np.uint32), b.view(np.uint32)), name
+        assert np.array_equal(cat(self.param), self.ost.param)
+        f, o = self.ls, self.fsm
+        assert (f["t"], f["good"], f["last_overflow"], f["last_skipped"]) == \
+               (o.t, o.good, o.last_overflow, o.last_skipped)
+        assert np.float32(f["scale"]) == np.float32(o.scale)
+        if np.isfinite(o.grad_norm_sq):
+            assert abs(f["grad_norm_sq"] - o.grad_norm_sq) <= 1e-9 * o.grad_norm_sq
+        else:
+            assert not np.isfinite(f["grad_norm_sq"])
+
+
+@pytest.mark.parametrize("R", [1, 2, 3, 8])
+@pytest.mark.parametrize("dtype", [O.BF16, O.FP16])
+@pytest.mark.parametrize("mode", [O.SCALE_NONE, O.SCALE_STATIC, O.SCALE_DYNAMIC])
+@pytest.mark.parametrize("align", [1, 8])
+def test_cpu_step_matches_oracle(R, dtype, mode, align):
+    rng = np.random.default_rng(R * 10 + dtype)
+    numels = rng.integers(1, 50_000, 5).tolist()
+    o = Offload(numels, R, dtype, align, mode, seed=R + 7 * mode)
+    for _ in range(3):
+        o.step()
+        o.compare()
+
+
+@pytest.mark.parametrize("n_micro,divisor,clip", [(2, 2.0, 0.0), (3, 3.0, 1e-3), (1, 1.0, 1e9)])
+def test_cpu_step_accumulation_and_clipping(n_micro, divisor, clip):
+    o = Offload([120_000, 77, 3], 4, O.BF16, 8, O.SCALE_NONE, seed=3)
+    for _ in range(3):
+        o.step(n_micro, divisor, clip)
+        o.compare()
+
+
+def test_cpu_step_skips_on_overflow_and_recovers():
+    o = Offload([30_000, 500], 2, O.FP16, 8, O.SCALE_DYNAMIC, scale=1024.0, interval=2, seed=5)
+    o.step()
+    o.compare()
+    before = [x.copy() for x in o.master]
+    o.step(inject=(0, 1, 123))
+    o.compare()
+    assert o.ls["last_skipped"] == 1 and o.ls["scale"] == 512.0
+    assert all(np.array_equal(a, b) for a, b in zip(before, o.master))
+    for _ in range(3):
+        o.step()
+        o.compare()
+
+
+def test_thread_count_does_not_change_the_state():
+    a = Offload([200_000, 1234], 4, O.FP16, 8, O.SCALE_DYNAMIC, seed=9)
+    b = Offload([200_000, 1234], 4, O.FP16, 8, O.SCALE_DYNAMIC, seed=9)
+    for _ in range(2):
+        a.step(nthreads=1)
+        b.step(nthreads=7)
+    for x, y in zip(a.master + a.m + a.v, b.master + b.m + b.v):
+        assert np.array_equal(x.view(np.uint32), y.view(np.uint32))
+    for x, y in zip(a.param, b.param):
+        assert np.array_equal(x, y)
+    assert abs(a.ls["grad_norm_sq"] - b.ls["grad_norm_sq"]) <= 1e-12 * a.ls["grad_norm_sq"]
+
+
+@pytest.mark.parametrize("dtype", [O.BF16, O.FP16])
+def test_half_encoding_over_many_bit_patterns(dtype):
+    # lr = 0 and wd = 0 leave master unchanged, so param must equal the
+    # oracle's encoding of arbitrary fp32 values, subnormal and overflowing ones included
+    rng = np.random.default_rng(12)
+    n = 1 << 21
+    bits = rng.integers(0, 1 << 32, n, dtype=np.uint64).astype(np.uint32)
+    special = np.array([0x00000001, 0x33000000, 0x33000001, 0x337FFFFF, 0x387FE000, 0x387FF000,
+                        0x38800000, 0x477FEFFF, 0x477FF000, 0x7F7FFFFF, 0x80000001, 0xB3800000,
+                        0x00800000, 0x007FFFFF, 0x7F800000, 0xFF800000], np.uint32)
+    bits[:special.size] = special
+    x = bits.view(np.float32)
+    x = np.where(np.isnan(x), np.float32(0.5), x).astype(np.float32)
+    plan = Z.Plan([n], None, 1, dtype, 8, 0)
+    master = [x.copy()]
+    param = [np.zeros(n, np.uint16)]
+    zeros = [np.zeros(n, np.float32) for _ in range(3)]
+    hp = dict(lr=0.0, beta1=0.9, beta2=0.999, eps=1e-8, weight_decay=0.0)
+    Z.zero_cpu_step(plan.handle, dict(mode=0), dict(scale=1.0, cur=0, good=0, t=0), hp, [zeros[0]],
+                    master, [zeros[1]], [zeros[2]], param)
+    assert np.array_equal(master[0].view(np.uint32), x.view(np.uint32))
+    assert np.array_equal(param[0], O.float_to_half(x, dtype))
+
+
+def test_cpu_step_argument_errors():
+    plan = Z.Plan([100], None, 2, O.BF16, 8, 0)
+    buf = [np.zeros(plan.S, np.float32) for _ in range(2)]
+    half = [np.zeros(plan.S, np.uint16) for _ in range(2)]
+    with pytest.raises(Z.ZeroError):
+        Z.zero_cpu_step(plan.handle, dict(mode=0), dict(scale=1.0, t=0), HP, buf, buf, buf, buf, half,
+                        grad_divisor=0.5)
+    with pytest.raises(Z.ZeroError):
+        Z.zero_cpu_step(plan.handle, dict(mode=0), dict(scale=1.0, t=0),
+                        dict(HP, beta1=1.0), buf, buf, buf, buf, half)

@@ -1,0 +1,145 @@
+"""ZeRO-Offload on the GPU: gradients reduce-scattered on the GPU, copied to
+pinned host memory, the optimizer step run by zero_cpu_step on CPU threads,
+and the half parameters copied back -- run serialized and with the one-step
+delayed parameter update (the CPU step of step s overlapping step s+1's GPU
+work). The optimizer sees the same gradients either way, so the host state
+and the GPU parameters must equal the oracle's bit for bit."""
+import threading
+
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+
+pytestmark = pytest.mark.gpu
+
+if torch.cuda.is_available():
+    import zero_partitioned_mixed_reduce_b200 as Z
+    from zero_partitioned_mixed_reduce_b200 import synth
+    from gpu_harness import u16
+
+HALF = {0: torch.bfloat16, 1: torch.float16}
+
+
+class OffloadRun:
+    def __init__(self, numels, R, dtype, mode, scale=512.0, interval=3):
+        self.wl = synth.custom_workload(numels, R, dtype, mode, scale, interval, sigma=1e-2, index=31)
+        self.lay = O.Layout(numels, R, 8)
+        self.plan = Z.Plan(numels, None, R, dtype, 8, 0)
+        self.R, self.dtype, self.mode = R, dtype, mode
+        S, T = self.plan.S, self.plan.T
+        self.idx = self.lay.flat_index()
+        x = synth.flat_master(self.wl, "cpu")
+        p0 = x.to(HALF[dtype])
+        self.ost = O.State(x.numpy(), dtype, u16(p0))
+        self.fsm = O.make_fsm(mode, scale=scale if mode else 1.0, interval=interval)
+        mflat = self.plan.pack(x, fill=0.0)
+        pflat = self.plan.pack(p0, fill=0)
+        pin = lambda t: t.pin_memory()
+        self.master = [pin(mflat[r * S:(r + 1) * S].clone()) for r in range(R)]
+        self.m = [pin(torch.zeros(S)) for _ in range(R)]
+        self.v = [pin(torch.zeros(S)) for _ in range(R)]
+        self.param_host = [pin(pflat[r * S:(r + 1) * S].clone()) for r in range(R)]
+        self.acc_host = [[pin(torch.zeros(S)) for _ in range(R)] for _ in range(2)]  # double buffer
+        self.param_gpu = [self.param_host[r].cuda() for r in range(R)]
+        self.acc_gpu = [torch.zeros(S, device="cuda") for _ in range(R)]
+        self.grads = [torch.zeros(T, dtype=HALF[dtype], device="cuda") for _ in range(R)]
+        self.ctx = Z.zero_ctx_create(self.plan.handle, mode, scale, interval)
+        self.cfg = dict(mode=mode, growth_interval=interval)
+        self.ls = dict(scale=scale if mode else 1.0, cur=0, good=0, t=0)
+        self.copy = torch.cuda.Stream()
+        self.step_no = 0
+        self.up_ev = None
+        self.hp = self.wl["hp"]
+        self.ohp = O.AdamW(*(self.hp[k] for k in ("lr", "beta1", "beta2", "eps", "weight_decay")))
+
+    def gpu_half(self, slot):
+        """GPU part of a step: grads, reduce-scatter, D2H of the accumulators
+        into host buffer `slot`. Returns the event marking the copy."""
+        self.step_no += 1
+        scale = self.ls_scale_for_grads
+        g = np.stack([u16(synth.flat_grads(self.wl, self.step_no, r, scale, "cpu")) for r in range(self.R)])
+        for r in range(self.R):
+            gp = np.zeros(self.plan.T, np.uint16)
+            gp[self.idx] = g[r]
+            self.grads[r].view(torch.int16).copy_(torch.from_numpy(gp.view(np.int16)))
+        Z.zero_reduce_scatter_bucket(self.ctx, -1, self.grads, self.acc_gpu)
+        ev = torch.cuda.Event()
+        ev.record()
+        self.copy.wait_event(ev)
+        with torch.cuda.stream(self.copy):
+            for r in range(self.R):
+                self.acc_host[slot][r].copy_(self.acc_gpu[r], non_blocking=True)
+        done = torch.cuda.Event()
+        done.record(self.copy)
+        # the next reduce-scatter may not overwrite the accumulators mid-copy
+        torch.cuda.current_stream().wait_event(done)
+        return g, done
+
+    def cpu_half(self, slot, done):
+        done.synchronize()
+        if self.up_ev is not None:
+            self.up_ev.synchronize()  # the last upload has finished reading param_host
+        self.ls = Z.zero_cpu_step(self.plan.handle, self.cfg, self.ls, self.hp, self.acc_host[slot],
+                                  self.master, self.m, self.v, self.param_host, nthreads=0)
+
+    def upload(self):
+        with torch.cuda.stream(self.copy):
+            for r in range(self.R):
+                self.param_gpu[r].copy_(self.param_host[r], non_blocking=True)
+        self.up_ev = torch.cuda.Event()
+        self.up_ev.record(self.copy)
+
+    def run(self, steps, delayed):
+        """With delayed=True the CPU step of step s runs in a thread while the
+        GPU half of step s+1 is issued (one-step delayed parameter update)."""
+        pending = None
+        for s in range(steps):
+            if self.mode == O.SCALE_DYNAMIC and delayed and pending is not None:
+                # the next step's backward must know the loss scale: wait for the
+                # previous decision, as the host loop of a delayed update does
+                pending[0].join()
+                self.upload()
+                pending = None
+            self.ls_scale_for_grads = self.ls["scale"] if self.mode else 1.0
+            g, done = self.gpu_half(s % 2)
+            O.step(self.ost, g, self.ohp, self.fsm)
+            if pending is not None:
+                pending[0].join()
+                self.upload()
+            th = threading.Thread(target=self.cpu_half, args=(s % 2, done))
+            th.start()
+            if delayed:
+                pending = (th,)
+            else:
+                th.join()
+                self.upload()
+        if pending is not None:
+            pending[0].join()
+            self.upload()
+        torch.cuda.synchronize()
+
+    def compare(self):
+        cat = lambda xs: torch.cat(xs).numpy()[self.idx]
+        for name, a, b in (("master", cat(self.master), self.ost.master), ("m", cat(self.m), self.ost.m),
+                           ("v", cat(self.v), self.ost.v)):
+            assert np.array_equal(a.view(np.uint32), b.view(np.uint32)), name
+        assert np.array_equal(u16(torch.cat(self.param_gpu))[self.idx], self.ost.param)
+        assert (self.ls["t"], self.ls["last_skipped"]) == (self.fsm.t, self.fsm.last_skipped)
+        assert np.float32(self.ls["scale"]) == np.float32(self.fsm.scale)
+
+    def close(self):
+        Z.zero_ctx_destroy(self.ctx)
+
+
+@pytest.mark.parametrize("delayed", [False, True])
+@pytest.mark.parametrize("R,dtype,mode", [(2, O.BF16, O.SCALE_NONE), (8, O.FP16, O.SCALE_DYNAMIC),
+                                          (3, O.FP16, O.SCALE_STATIC)])
+def test_offload_pipeline_matches_oracle(delayed, R, dtype, mode):
+    o = OffloadRun([200_001, 77, 4096, 3], R, dtype, mode)
+    try:
+        o.run(5, delayed)
+        o.compare()
+    finally:
+        o.close()

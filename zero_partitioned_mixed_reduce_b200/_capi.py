@@ -116,6 +116,9 @@ _sig("zero_grads_join", _S, [_P, _P])
 _sig("zero_prefetch_begin", _S, [_P, C.POINTER(zero_state), _PP, C.c_int32, C.c_int32, C.c_int32, _P])
 _sig("zero_layer_acquire", _S, [_P, C.c_int64, C.POINTER(C.c_void_p), _P])
 _sig("zero_layer_release", _S, [_P, C.c_int64, _P])
+_sig("zero_cpu_step", _S, [_P, C.POINTER(zero_loss_scale_config), C.POINTER(zero_loss_scale_state),
+                           C.POINTER(zero_adamw), C.POINTER(zero_step_opts), _PP, _PP, _PP, _PP, _PP,
+                           C.c_int32])
 _sig("zero_sync", _S, [_P, _P])
 _sig("zero_last_error", C.c_size_t, [C.c_char_p, C.c_size_t])
 _sig("zero_version", C.c_char_p, [])
@@ -349,6 +352,36 @@ def zero_layer_acquire(ctx, layer, stream=None):
 
 def zero_layer_release(ctx, layer, stream=None):
     _check(_lib.zero_layer_release(ctx, layer, _stream(stream)))
+
+
+def zero_cpu_step(plan, cfg, state, hp, acc, master, m, v, param, grad_divisor=1.0,
+                  max_grad_norm=0.0, nthreads=0):
+    """The optimizer step on host memory (all buffers host pointers, numpy
+    arrays or CPU tensors). cfg / state as for zero_step_noalloc; returns the
+    loss-scale state after the step."""
+    c = zero_loss_scale_config(cfg.get("mode", ZERO_SCALE_NONE), 1.0,
+                               cfg.get("growth_interval", 1000), cfg.get("growth_factor", 2.0),
+                               cfg.get("backoff_factor", 0.5), cfg.get("min_scale", 1.0), 0)
+    st = zero_loss_scale_state()
+    for k, _ in zero_loss_scale_state._fields_:
+        if k in state:
+            setattr(st, k, state[k])
+    if isinstance(hp, dict):
+        hp = zero_adamw(hp["lr"], hp["beta1"], hp["beta2"], hp["eps"], hp["weight_decay"])
+    opts = zero_step_opts(grad_divisor, max_grad_norm)
+    arrays = [_ptr_array([_host_addr(x) for x in xs]) for xs in (acc, master, m, v, param)]
+    _check(_lib.zero_cpu_step(plan, C.byref(c), C.byref(st), C.byref(hp), C.byref(opts),
+                              *[a[0] for a in arrays], nthreads))
+    return {k: getattr(st, k) for k, _ in zero_loss_scale_state._fields_}
+
+
+def _host_addr(x):
+    if isinstance(x, int):
+        return x
+    if hasattr(x, "ctypes"):  # numpy
+        assert x.flags["C_CONTIGUOUS"]
+        return x.ctypes.data
+    return int(x.data_ptr())
 
 
 def zero_sync(ctx, stream=None):

@@ -21,11 +21,13 @@ NVCC = os.path.join(CUDA_HOME, "bin", "nvcc")
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 NVCC_FLAGS = ["-O3", "-std=c++17", *ARCH, "-lineinfo", "--fmad=false", "-Xptxas", "-v",
               "-Xcompiler", "-fPIC", "-I", INCLUDE, "-I", CSRC]
-CXX_FLAGS = ["-O2", "-std=c++17", "-fPIC", "-Wall", "-Wextra", "-I", INCLUDE, "-I", CSRC,
-             "-I", os.path.join(CUDA_HOME, "include")]
+CXX_FLAGS = ["-O2", "-std=c++17", "-fPIC", "-Wall", "-Wextra", "-ffp-contract=off",
+             "-fno-fast-math", "-I", INCLUDE, "-I", CSRC, "-I", os.path.join(CUDA_HOME, "include")]
+# the host AdamW loop is vectorized (target_clones picks AVX-512 / AVX2 / baseline)
+CXX_EXTRA = {"cpu_adam.cpp": ["-O3", "-pthread"]}
 
 CU_SOURCES = ["kernels.cu", "noalloc.cu"]
-CPP_SOURCES = ["plan.cpp", "capi.cpp", "sched.cpp"]
+CPP_SOURCES = ["plan.cpp", "capi.cpp", "sched.cpp", "cpu_adam.cpp"]
 
 
 def _sources():
@@ -64,10 +66,10 @@ def build(force: bool = False) -> str:
         objs.append(o)
     for s in CPP_SOURCES:
         o = os.path.join(BUILD, s + ".o")
-        _run(["g++", *CXX_FLAGS, "-c", os.path.join(CSRC, s), "-o", o])
+        _run(["g++", *CXX_FLAGS, *CXX_EXTRA.get(s, []), "-c", os.path.join(CSRC, s), "-o", o])
         objs.append(o)
     tmp = OUT + f".tmp{os.getpid()}"
-    _run([NVCC, "-shared", *ARCH, "-cudart=static", *objs, "-o", tmp])
+    _run([NVCC, "-shared", *ARCH, "-cudart=static", *objs, "-o", tmp, "-Xcompiler", "-pthread"])
     os.replace(tmp, OUT)
     return OUT
 

@@ -1,0 +1,224 @@
+// Host-side AdamW for ZeRO-Offload: the fp32 master weights and the Adam
+// moments live in (pinned) host memory and the update runs on CPU cores, while
+// the GPU only holds the half parameters and reduces the gradients.
+//
+// Pages: inferensys legal pre-training glossary, "CPU Offload" (optimizer
+// states and gradients offloaded to CPU DRAM; Adam runs on the CPU while the
+// GPU runs forward and backward) and "One-Step Delayed Parameter Update"
+// (the CPU step overlaps the next forward pass); genomic glossary, "CPU
+// Offload" (fp32 master weights and optimizer states in CPU RAM, fp16
+// parameters and gradients on the GPU).
+//
+// The arithmetic is the step of include/zero_b200.h, one IEEE binary32
+// operation per line (this file is built with -ffp-contract=off), so results
+// equal the GPU step bit for bit. The element loop is plain scalar C++ that
+// the compiler vectorizes; gcc's target_clones builds AVX-512, AVX2 and
+// baseline versions and picks one at load time. The half encoders round to
+// nearest even on the bit pattern (keeping subnormals, overflowing to
+// infinity), because the AVX-512 bf16 conversion instruction treats
+// subnormal inputs as zero.
+#include <cmath>
+#include <cstring>
+#include <string>
+#include <thread>
+#include <vector>
+
+#include "internal.h"
+
+namespace {
+
+inline uint32_t f2u(float x) {
+    uint32_t u;
+    std::memcpy(&u, &x, 4);
+    return u;
+}
+
+// fp32 -> bf16, round to nearest even on the bits; NaN -> quiet NaN.
+inline uint16_t to_bf16(float x) {
+    const uint32_t u = f2u(x);
+    if ((u & 0x7fffffffu) > 0x7f800000u) return static_cast<uint16_t>((u >> 16) | 0x0040u);
+    const uint32_t lsb = (u >> 16) & 1u;
+    return static_cast<uint16_t>((u + 0x7fffu + lsb) >> 16);
+}
+
+// fp32 -> IEEE binary16, round to nearest even, subnormals kept, overflow to inf.
+inline uint16_t to_fp16(float x) {
+    const uint32_t u = f2u(x);
+    const uint16_t sign = static_cast<uint16_t>((u >> 16) & 0x8000u);
+    const uint32_t a = u & 0x7fffffffu;
+    if (a > 0x7f800000u) return static_cast<uint16_t>(sign | 0x7e00u);  // NaN
+    if (a >= 0x477ff000u) return static_cast<uint16_t>(sign | 0x7c00u);  // >= 65520: inf
+    if (a < 0x38800000u) {  // below 2^-14: fp16 subnormal (or zero)
+        // value = mant * 2^(e-150) with the implicit bit; the result counts 2^-24 units
+        const uint32_t e = a >> 23;
+        if (e < 102) return sign;  // below 2^-25: rounds to zero
+        const uint32_t mant = (a & 0x7fffffu) | 0x800000u;
+        const uint32_t shift = 126 - e;  // 14..24
+        const uint32_t q = mant >> shift;
+        const uint32_t rem = mant & ((1u << shift) - 1u);
+        const uint32_t half = 1u << (shift - 1);
+        const uint32_t r = q + ((rem > half || (rem == half && (q & 1u))) ? 1u : 0u);
+        return static_cast<uint16_t>(sign | r);
+    }
+    // normal: rebias the exponent (127 -> 15) and round the 13 dropped bits
+    const uint32_t v = a - 0x38000000u;  // exponent -= 112, still in fp32 bit layout
+    const uint32_t lsb = (v >> 13) & 1u;
+    return static_cast<uint16_t>(sign | ((v + 0x0fffu + lsb) >> 13));
+}
+
+struct Coeffs {
+    float inv, dec, b1f, omb1, b2f, omb2, epsf, ss, bc2s, clip;
+};
+
+template <bool FP16, bool CLIP>
+__attribute__((target_clones("avx512f", "avx2", "default"))) void update_range(
+    const Coeffs c, const float* __restrict acc, float* __restrict p, float* __restrict m,
+    float* __restrict v, uint16_t* __restrict out, int64_t n) {
+    for (int64_t i = 0; i < n; ++i) {
+        const float g0 = acc[i] * c.inv;
+        const float g = CLIP ? g0 * c.clip : g0;
+        float pp = p[i] * c.dec;
+        const float mm = c.b1f * m[i] + c.omb1 * g;
+        const float vv = c.b2f * v[i] + c.omb2 * (g * g);
+        const float den = std::sqrt(vv) / c.bc2s + c.epsf;
+        pp = pp - c.ss * (mm / den);
+        p[i] = pp;
+        m[i] = mm;
+        v[i] = vv;
+        out[i] = FP16 ? to_fp16(pp) : to_bf16(pp);
+    }
+}
+
+// Sum of (double)(acc * inv)^2 over [0, n) and whether any acc is non-finite.
+__attribute__((target_clones("avx512f", "avx2", "default"))) void scan_range(
+    const float* __restrict acc, float inv, int64_t n, double* nrm, int* bad) {
+    double s = 0.0;
+    int b = 0;
+    for (int64_t i = 0; i < n; ++i) {
+        const float a = acc[i];
+        b |= !(std::fabs(a) <= 3.4028234663852886e38f);
+        const double g = static_cast<double>(a * inv);
+        s += g * g;
+    }
+    *nrm = s;
+    *bad = b;
+}
+
+template <typename F>
+void parallel_chunks(int64_t total, int nthreads, F&& fn) {
+    if (nthreads <= 1 || total < (int64_t(1) << 16)) {
+        fn(0, 0, total);
+        return;
+    }
+    std::vector<std::thread> pool;
+    const int64_t chunk = (total + nthreads - 1) / nthreads;
+    for (int t = 0; t < nthreads; ++t) {
+        const int64_t a = t * chunk, b = std::min(total, a + chunk);
+        if (a >= b) break;
+        pool.emplace_back([&fn, t, a, b] { fn(t, a, b); });
+    }
+    for (auto& th : pool) th.join();
+}
+
+}  // namespace
+
+extern "C" zero_status zero_cpu_step(const zero_plan_t* plan, const zero_loss_scale_config* cfg,
+                                     zero_loss_scale_state* inout, const zero_adamw* hp,
+                                     const zero_step_opts* opts, const float* const* acc, float* const* master,
+                                     float* const* m, float* const* v, void* const* param, int32_t nthreads) {
+    if (!plan || !cfg || !inout || !hp || !acc || !master || !m || !v || !param)
+        return zb_fail(ZERO_ERR_INVALID_ARG, "zero_cpu_step: NULL argument");
+    zero_step_opts o{1.0, 0.0, {0, 0}};
+    if (opts) o = *opts;
+    if (!(o.grad_divisor >= 1.0) || !std::isfinite(o.grad_divisor) || !(o.max_grad_norm >= 0.0) ||
+        !std::isfinite(o.max_grad_norm))
+        return zb_fail(ZERO_ERR_INVALID_ARG, "zero_cpu_step: need grad_divisor >= 1 and finite max_grad_norm >= 0");
+    if (cfg->mode < ZERO_SCALE_NONE || cfg->mode > ZERO_SCALE_DYNAMIC)
+        return zb_fail(ZERO_ERR_INVALID_ARG, "zero_cpu_step: bad loss-scale mode");
+    if (cfg->mode == ZERO_SCALE_DYNAMIC &&
+        (cfg->growth_interval < 1 || !(cfg->growth_factor > 1.0f) ||
+         !(cfg->backoff_factor > 0.0f && cfg->backoff_factor < 1.0f) || !(cfg->min_scale > 0.0f)))
+        return zb_fail(ZERO_ERR_INVALID_ARG, "zero_cpu_step: bad dynamic loss-scale config");
+    const float scale = cfg->mode == ZERO_SCALE_NONE ? 1.0f : inout->scale;
+    if (!(scale > 0.0f) || !std::isfinite(scale) || inout->t < 0)
+        return zb_fail(ZERO_ERR_INVALID_ARG, "zero_cpu_step: need a finite scale > 0 and t >= 0");
+    if (!(hp->lr >= 0.0) || !(hp->beta1 >= 0.0 && hp->beta1 < 1.0) || !(hp->beta2 >= 0.0 && hp->beta2 < 1.0) ||
+        !(hp->eps > 0.0) || !(hp->weight_decay >= 0.0))
+        return zb_fail(ZERO_ERR_INVALID_ARG, "zero_cpu_step: bad hyper-parameters");
+    const int R = plan->R;
+    for (int r = 0; r < R; ++r)
+        if (!acc[r] || !master[r] || !m[r] || !v[r] || !param[r])
+            return zb_fail(ZERO_ERR_INVALID_ARG, "zero_cpu_step: NULL rank pointer");
+    if (nthreads < 1) nthreads = static_cast<int>(std::thread::hardware_concurrency());
+    if (nthreads < 1) nthreads = 1;
+    const int64_t S = plan->S;
+
+    Coeffs c;
+    const double t1 = static_cast<double>(inout->t + 1);
+    c.inv = static_cast<float>(1.0 / ((static_cast<double>(R) * o.grad_divisor) * static_cast<double>(scale)));
+    c.dec = static_cast<float>(1.0 - hp->lr * hp->weight_decay);
+    c.b1f = static_cast<float>(hp->beta1);
+    c.omb1 = static_cast<float>(1.0 - hp->beta1);
+    c.b2f = static_cast<float>(hp->beta2);
+    c.omb2 = static_cast<float>(1.0 - hp->beta2);
+    c.epsf = static_cast<float>(hp->eps);
+    c.ss = static_cast<float>(hp->lr / (1.0 - std::pow(hp->beta1, t1)));
+    c.bc2s = static_cast<float>(std::sqrt(1.0 - std::pow(hp->beta2, t1)));
+    c.clip = 1.0f;
+
+    // pass 1: overflow and squared norm; per-thread partials summed in thread order
+    std::vector<double> part(static_cast<size_t>(nthreads) * R, 0.0);
+    std::vector<int> bad(static_cast<size_t>(nthreads) * R, 0);
+    for (int r = 0; r < R; ++r)
+        parallel_chunks(S, nthreads, [&](int t, int64_t a, int64_t b) {
+            scan_range(acc[r] + a, c.inv, b - a, &part[r * nthreads + t], &bad[r * nthreads + t]);
+        });
+    double nrm = 0.0;
+    int overflow = 0;
+    for (size_t i = 0; i < part.size(); ++i) {
+        nrm += part[i];
+        overflow |= bad[i];
+    }
+    if (o.max_grad_norm > 0.0) {
+        const double cd = o.max_grad_norm / (std::sqrt(nrm) + 1e-6);
+        c.clip = static_cast<float>(cd < 1.0 ? cd : 1.0);
+    }
+
+    // pass 2: the update, unless dynamic loss scaling skips the step
+    const bool skip = cfg->mode == ZERO_SCALE_DYNAMIC && overflow;
+    if (!skip) {
+        const bool fp16 = plan->dtype == ZERO_FP16, clip = o.max_grad_norm > 0.0;
+        for (int r = 0; r < R; ++r)
+            parallel_chunks(S, nthreads, [&](int, int64_t a, int64_t b) {
+                uint16_t* out = static_cast<uint16_t*>(param[r]) + a;
+                if (fp16 && clip) update_range<true, true>(c, acc[r] + a, master[r] + a, m[r] + a, v[r] + a, out, b - a);
+                else if (fp16) update_range<true, false>(c, acc[r] + a, master[r] + a, m[r] + a, v[r] + a, out, b - a);
+                else if (clip) update_range<false, true>(c, acc[r] + a, master[r] + a, m[r] + a, v[r] + a, out, b - a);
+                else update_range<false, false>(c, acc[r] + a, master[r] + a, m[r] + a, v[r] + a, out, b - a);
+            });
+    }
+
+    // loss-scale state machine, the same rules as the device step
+    int skipped = 0;
+    if (cfg->mode == ZERO_SCALE_DYNAMIC) {
+        if (overflow) {
+            const float s = inout->scale * cfg->backoff_factor;
+            inout->scale = (s < cfg->min_scale) ? cfg->min_scale : s;
+            inout->good = 0;
+            skipped = 1;
+        } else {
+            inout->t += 1;
+            inout->good += 1;
+            if (inout->good >= cfg->growth_interval) {
+                inout->scale = inout->scale * cfg->growth_factor;
+                inout->good = 0;
+            }
+        }
+    } else {
+        inout->t += 1;
+    }
+    inout->last_overflow = overflow;
+    inout->last_skipped = skipped;
+    inout->grad_norm_sq = nrm;
+    return ZERO_OK;
+}
