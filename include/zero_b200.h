@@ -303,6 +303,40 @@ zero_status zero_step_ex(zero_ctx_t* ctx, const zero_adamw* hp, const zero_state
                          const void* const* grads, const zero_step_opts* opts, void* stream);
 
 /*
+ * zero_step_shard -- the fused step (grads != NULL path of zero_step) on
+ * shards [owner_lo, owner_hi) only, with the loss-scale update left to
+ * zero_step_commit: the step's last block writes partial[0] = sum of g^2 and
+ * partial[1] = 1 if some reduced gradient of these shards is inf/NaN, else 0.
+ * This is the per-rank half of a multi-GPU ZeRO step: rank o calls it with
+ * [o, o+1) and grads[r] pointing at rank r's gradient buffer (peer-mapped,
+ * read with plain loads or bulk copies without multicast); the ranks then
+ * all-reduce `partial` (sum) and each calls zero_step_commit with the
+ * result, so every rank takes the same skip and loss-scale decision. In one
+ * process, calling it for every shard and summing the partials gives exactly
+ * zero_step. Only the owned shards' state pointers are read (others may be
+ * NULL); DYNAMIC mode needs the ping-pong set, as for zero_step.
+ * Defines: [instr] ZeRO-2 "Mechanism" and "Communication" (each process
+ * reduces and updates only its own partition) and [instr] "Baseline (DP)" /
+ * ZeRO-2 (the reduce-scatter replaces the all-reduce); the overflow and norm
+ * are the small all-reduce every rank needs for the shared decision.
+ * partial: device, 2 doubles, 8-byte aligned, caller-owned.
+ * Errors: ZERO_ERR_RANGE (owner range), ZERO_ERR_INVALID_ARG, ZERO_ERR_ALIGN,
+ * ZERO_ERR_STATE, ZERO_ERR_CUDA.
+ */
+zero_status zero_step_shard(zero_ctx_t* ctx, const zero_adamw* hp, const zero_state* state,
+                            const void* const* grads, int32_t owner_lo, int32_t owner_hi,
+                            double* partial, void* stream);
+
+/*
+ * zero_step_commit -- the loss-scale update after zero_step_shard, from
+ * totals reduced over every shard: reduced[0] = sum of g^2 (recorded as
+ * grad_norm_sq), reduced[1] > 0 means overflow. Skip, backoff, growth, t and
+ * the ping-pong flip follow zero_step.
+ * reduced: device, 2 doubles, 8-byte aligned.
+ */
+zero_status zero_step_commit(zero_ctx_t* ctx, const double* reduced, void* stream);
+
+/*
  * zero_gather_layer -- assemble one layer's half parameters from the R
  * shards of the current set into a contiguous buffer:
  *   out[j] = param[cur][o][lo + j - o*S],  o = (lo + j) / S,  0 <= j < hi - lo.

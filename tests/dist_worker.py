@@ -1,0 +1,73 @@
+"""Worker for tests/test_gpu_dist.py, launched with torch.distributed.run:
+DistributedZero (one process per GPU, NCCL, symmetric memory) against the
+oracle. Prints "ok" on rank 0 when every step matched."""
+import os
+import sys
+
+import numpy as np
+import torch
+import torch.distributed as dist
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+
+import oracle as O  # noqa: E402
+import zero_partitioned_mixed_reduce_b200 as Z  # noqa: E402
+from zero_partitioned_mixed_reduce_b200 import synth  # noqa: E402
+from zero_partitioned_mixed_reduce_b200.dist import DistributedZero  # noqa: E402
+
+
+def u16(t):
+    return t.contiguous().view(torch.int16).cpu().numpy().view(np.uint16)
+
+
+def main():
+    torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", "0")))
+    dist.init_process_group("nccl")
+    rank, world = dist.get_rank(), dist.get_world_size()
+    numels, layer_ids = [70_001, 13, 4096, 999], [0, 0, 1, 1]
+    dz = DistributedZero(numels, layer_ids, Z.ZERO_FP16, Z.ZERO_SCALE_DYNAMIC, 256.0, 3)
+    wl = synth.custom_workload(numels, world, Z.ZERO_FP16, Z.ZERO_SCALE_DYNAMIC, 256.0, 3, sigma=1e-2,
+                               layer_ids=layer_ids, index=55)
+    lay = O.Layout(numels, world, 8, 0, layer_ids)
+    idx = lay.flat_index()
+    x = synth.flat_master(wl, "cpu")
+    p0 = x.to(torch.float16)
+    dz.load(dz.plan.pack(x.cuda()), dz.plan.pack(p0.cuda()))
+    ost = O.State(x.numpy(), O.FP16, u16(p0))
+    fsm = O.make_fsm(O.SCALE_DYNAMIC, scale=256.0, interval=3)
+    hp = wl["hp"]
+    ohp = O.AdamW(*(hp[k] for k in ("lr", "beta1", "beta2", "eps", "weight_decay")))
+    S = dz.plan.S
+    for step in range(1, 6):
+        g = np.stack([u16(synth.flat_grads(wl, step, r, fsm.scale, "cpu")) for r in range(world)])
+        if step == 3:
+            g[world - 1, 5] = 0x7C00
+        gp = np.zeros(dz.plan.T, np.uint16)
+        gp[idx] = g[rank]
+        dz.grads.view(torch.int16).copy_(torch.from_numpy(gp.view(np.int16)))
+        dz.step(hp)
+        O.step(ost, g, ohp, fsm)
+        f = dz.loss_scale()
+        assert (f["t"], f["last_skipped"], f["scale"]) == (fsm.t, fsm.last_skipped, fsm.scale), (step, f)
+        flat = np.zeros(dz.plan.T, np.float32)
+        flat[idx] = ost.master
+        mine = dz.current("master").cpu().numpy()
+        assert np.array_equal(mine.view(np.uint32), flat[rank * S:(rank + 1) * S].view(np.uint32)), step
+    # ZeRO-3 gather from every rank's shard
+    pflat = np.zeros(dz.plan.T, np.uint16)
+    pflat[idx] = ost.param
+    for l, (lo, hi) in enumerate(lay.layers):
+        out = torch.empty(hi - lo, dtype=torch.float16, device="cuda")
+        dz.gather_layer(l, out)
+        torch.cuda.synchronize()
+        assert np.array_equal(u16(out), pflat[lo:hi]), l
+    dz.close()
+    dist.barrier()
+    dist.destroy_process_group()
+    if rank == 0:
+        print("ok")
+
+
+if __name__ == "__main__":
+    main()

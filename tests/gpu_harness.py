@@ -207,6 +207,27 @@ class Case:
         self.g.check()
         return skipped
 
+    def step_sharded(self, splits, inject=None):
+        """The fused step done shard range by shard range (zero_step_shard),
+        the per-range totals summed as a cross-rank all-reduce would, then
+        zero_step_commit. splits: list of (owner_lo, owner_hi)."""
+        self.step_no += 1
+        g = self.make_grads(inject)
+        for r in range(self.R):
+            gp = np.zeros(self.plan.T, np.uint16)
+            gp[self.idx] = g[r]
+            self.grads[r].view(torch.int16).copy_(torch.from_numpy(gp.view(np.int16)))
+        partials = [torch.full((2,), -1.0, dtype=torch.float64, device="cuda") for _ in splits]
+        for (lo, hi), part in zip(splits, partials):
+            Z.zero_step_shard(self.ctx, self.hp, self.handle, self.grads, lo, hi, part)
+        reduced = torch.stack(partials).sum(0)
+        Z.zero_step_commit(self.ctx, reduced)
+        skipped = O.step(self.ostate, g, O.AdamW(**{k: self.hp[k] for k in
+                                                    ("lr", "beta1", "beta2", "eps",
+                                                     "weight_decay")}), self.ofsm)
+        self.g.check()
+        return skipped, [p.cpu().numpy() for p in partials]
+
     def gpu_fsm(self):
         return Z.zero_loss_scale(self.ctx)
 

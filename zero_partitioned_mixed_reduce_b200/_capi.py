@@ -119,6 +119,9 @@ _sig("zero_layer_release", _S, [_P, C.c_int64, _P])
 _sig("zero_cpu_step", _S, [_P, C.POINTER(zero_loss_scale_config), C.POINTER(zero_loss_scale_state),
                            C.POINTER(zero_adamw), C.POINTER(zero_step_opts), _PP, _PP, _PP, _PP, _PP,
                            C.c_int32])
+_sig("zero_step_shard", _S, [_P, C.POINTER(zero_adamw), C.POINTER(zero_state), _PP, C.c_int32,
+                             C.c_int32, _P, _P])
+_sig("zero_step_commit", _S, [_P, _P, _P])
 _sig("zero_sync", _S, [_P, _P])
 _sig("zero_last_error", C.c_size_t, [C.c_char_p, C.c_size_t])
 _sig("zero_version", C.c_char_p, [])
@@ -382,6 +385,20 @@ def _host_addr(x):
         assert x.flags["C_CONTIGUOUS"]
         return x.ctypes.data
     return int(x.data_ptr())
+
+
+def zero_step_shard(ctx, hp, state: StateHandle, grads, owner_lo, owner_hi, partial, stream=None):
+    """Fused step on shards [owner_lo, owner_hi); partial: device buffer of 2 float64."""
+    if isinstance(hp, dict):
+        hp = zero_adamw(hp["lr"], hp["beta1"], hp["beta2"], hp["eps"], hp["weight_decay"])
+    g, ga = _ptr_array(grads)
+    _check(_lib.zero_step_shard(ctx, C.byref(hp), C.byref(state.c), g, owner_lo, owner_hi,
+                                _addr(partial), _stream(stream)))
+
+
+def zero_step_commit(ctx, reduced, stream=None):
+    """Loss-scale update from reduced totals (device buffer of 2 float64)."""
+    _check(_lib.zero_step_commit(ctx, _addr(reduced), _stream(stream)))
 
 
 def zero_sync(ctx, stream=None):

@@ -325,6 +325,8 @@ extern "C" zero_status zero_step_ex(zero_ctx_t* ctx, const zero_adamw* hp, const
     sp.powtab = ctx->powtab;
     sp.powtab_len = ctx->powtab_len;
     sp.grid_cap = ctx->grid_cap;
+    sp.obeg = 0;
+    sp.oend = ctx->R;
 
     zb::RankPtrs p;
     fill_state_ptrs(ctx, state, sets, &p);
@@ -339,6 +341,128 @@ extern "C" zero_status zero_step_ex(zero_ctx_t* ctx, const zero_adamw* hp, const
     if (e != cudaSuccess) return cuda_fail(where, e);
     ctx->t_bound += 1;
     if (sp.pingpong) ctx->two_sets = true;
+    return ZERO_OK;
+}
+
+namespace {
+
+// Shard-range variant of check_state: only owners [lo, hi) need pointers.
+zero_status check_state_range(const zero_ctx_t* ctx, const zero_state* st, int lo, int hi,
+                              const char* where, int* sets) {
+    if (!st) return zb_fail(ZERO_ERR_INVALID_ARG, std::string(where) + ": state is NULL");
+    const bool any1 = st->master[1] || st->m[1] || st->v[1] || st->param[1];
+    const bool all1 = st->master[1] && st->m[1] && st->v[1] && st->param[1];
+    if (any1 && !all1)
+        return zb_fail(ZERO_ERR_INVALID_ARG, std::string(where) + ": state set 1 must be complete or absent");
+    for (int k = 0; k < (all1 ? 2 : 1); ++k) {
+        if (!st->master[k] || !st->m[k] || !st->v[k] || !st->param[k])
+            return zb_fail(ZERO_ERR_INVALID_ARG, std::string(where) + ": NULL state array");
+        for (int r = lo; r < hi; ++r) {
+            const void* f[3] = {st->master[k][r], st->m[k][r], st->v[k][r]};
+            for (const void* q : f) {
+                if (!q) return zb_fail(ZERO_ERR_INVALID_ARG, std::string(where) + ": NULL state pointer");
+                if (!aligned(q, 32)) return zb_fail(ZERO_ERR_ALIGN, std::string(where) + ": fp32 state misaligned");
+            }
+            if (!st->param[k][r]) return zb_fail(ZERO_ERR_INVALID_ARG, std::string(where) + ": NULL param pointer");
+            if (!aligned(st->param[k][r], 16)) return zb_fail(ZERO_ERR_ALIGN, std::string(where) + ": param misaligned");
+        }
+    }
+    *sets = all1 ? 2 : 1;
+    (void)ctx;
+    return ZERO_OK;
+}
+
+}  // namespace
+
+extern "C" zero_status zero_step_shard(zero_ctx_t* ctx, const zero_adamw* hp, const zero_state* state,
+                                       const void* const* grads, int32_t owner_lo, int32_t owner_hi,
+                                       double* partial, void* stream) {
+    const char* where = "zero_step_shard";
+    if (!ctx || !hp || !grads || !partial)
+        return zb_fail(ZERO_ERR_INVALID_ARG, "zero_step_shard: NULL ctx, hp, grads or partial");
+    zero_status s = check_device(ctx, where);
+    if (s != ZERO_OK) return s;
+    if (owner_lo < 0 || owner_lo >= owner_hi || owner_hi > ctx->R)
+        return zb_fail(ZERO_ERR_RANGE, "zero_step_shard: need 0 <= owner_lo < owner_hi <= R");
+    if (!aligned(partial, 8)) return zb_fail(ZERO_ERR_ALIGN, "zero_step_shard: partial not 8-byte aligned");
+    if (!(hp->lr >= 0.0) || !(hp->beta1 >= 0.0 && hp->beta1 < 1.0) || !(hp->beta2 >= 0.0 && hp->beta2 < 1.0) ||
+        !(hp->eps > 0.0) || !(hp->weight_decay >= 0.0))
+        return zb_fail(ZERO_ERR_INVALID_ARG, "zero_step_shard: bad hyper-parameters");
+    int sets = 1;
+    if ((s = check_state_range(ctx, state, owner_lo, owner_hi, where, &sets)) != ZERO_OK) return s;
+    for (int r = 0; r < ctx->R; ++r) {
+        if (!grads[r]) return zb_fail(ZERO_ERR_INVALID_ARG, "zero_step_shard: grads[" + std::to_string(r) + "] is NULL");
+        if (!aligned(grads[r], 16)) return zb_fail(ZERO_ERR_ALIGN, "zero_step_shard: grads misaligned");
+    }
+    if (sets == 1 && ctx->cfg.mode == ZERO_SCALE_DYNAMIC)
+        return zb_fail(ZERO_ERR_INVALID_ARG, "zero_step_shard: dynamic loss scaling needs state set 1 (ping-pong)");
+    if (sets == 1 && ctx->two_sets)
+        return zb_fail(ZERO_ERR_STATE, "zero_step_shard: the current model may live in state set 1");
+    cudaStream_t cs = static_cast<cudaStream_t>(stream);
+    if ((s = ensure_powtab(ctx, hp->beta1, hp->beta2, ctx->t_bound + 1, cs)) != ZERO_OK) return s;
+    zb::StepParams sp;
+    sp.R = ctx->R;
+    sp.dtype = ctx->dtype;
+    sp.mode = ctx->cfg.mode;
+    sp.pingpong = sets == 2 ? 1 : 0;
+    sp.S8 = static_cast<uint32_t>(ctx->S / 8);
+    sp.T8 = static_cast<uint32_t>(ctx->T / 8);
+    sp.dec = static_cast<float>(1.0 - hp->lr * hp->weight_decay);
+    sp.b1f = static_cast<float>(hp->beta1);
+    sp.omb1 = static_cast<float>(1.0 - hp->beta1);
+    sp.b2f = static_cast<float>(hp->beta2);
+    sp.omb2 = static_cast<float>(1.0 - hp->beta2);
+    sp.epsf = static_cast<float>(hp->eps);
+    sp.lr = hp->lr;
+    sp.interval = ctx->cfg.growth_interval;
+    sp.growth = ctx->cfg.growth_factor;
+    sp.backoff = ctx->cfg.backoff_factor;
+    sp.min_scale = ctx->cfg.min_scale;
+    sp.st = ctx->st;
+    sp.partials = ctx->partials;
+    sp.powtab = ctx->powtab;
+    sp.powtab_len = ctx->powtab_len;
+    sp.grid_cap = ctx->grid_cap;
+    sp.obeg = owner_lo;
+    sp.oend = owner_hi;
+    sp.partial_out = partial;
+    zb::RankPtrs p{};
+    for (int r = 0; r < ctx->R; ++r) {
+        p.g[r] = grads[r];
+        for (int k = 0; k < 2; ++k) {
+            const int from = k < sets ? k : 0;
+            const bool owned = r >= owner_lo && r < owner_hi;
+            p.master[k][r] = owned ? state->master[from][r] : nullptr;
+            p.m[k][r] = owned ? state->m[from][r] : nullptr;
+            p.v[k][r] = owned ? state->v[from][r] : nullptr;
+            p.param[k][r] = owned ? state->param[from][r] : nullptr;
+        }
+    }
+    cudaError_t e = zb::launch_fused_step(sp, p, cs);
+    if (e != cudaSuccess) return cuda_fail(where, e);
+    ctx->t_bound += 1;
+    ctx->shard_pingpong = sp.pingpong;
+    if (sp.pingpong) ctx->two_sets = true;
+    return ZERO_OK;
+}
+
+extern "C" zero_status zero_step_commit(zero_ctx_t* ctx, const double* reduced, void* stream) {
+    const char* where = "zero_step_commit";
+    if (!ctx || !reduced) return zb_fail(ZERO_ERR_INVALID_ARG, "zero_step_commit: NULL argument");
+    zero_status s = check_device(ctx, where);
+    if (s != ZERO_OK) return s;
+    if (!aligned(reduced, 8)) return zb_fail(ZERO_ERR_ALIGN, "zero_step_commit: reduced not 8-byte aligned");
+    zb::StepParams sp;
+    sp.R = ctx->R;
+    sp.mode = ctx->cfg.mode;
+    sp.pingpong = ctx->shard_pingpong;
+    sp.interval = ctx->cfg.growth_interval;
+    sp.growth = ctx->cfg.growth_factor;
+    sp.backoff = ctx->cfg.backoff_factor;
+    sp.min_scale = ctx->cfg.min_scale;
+    sp.st = ctx->st;
+    cudaError_t e = zb::launch_fsm_commit(sp, reduced, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(where, e);
     return ZERO_OK;
 }
 

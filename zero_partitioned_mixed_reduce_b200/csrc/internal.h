@@ -54,6 +54,11 @@ struct StepParams {
     const double2* powtab = nullptr;  // powtab[t] = (beta1^t, beta2^t)
     int64_t powtab_len = 0;
     int grid_cap = 0;  // capacity of `partials`
+    // fused step over shards [obeg, oend) only (default: all R)
+    int32_t obeg = 0, oend = 0;
+    // non-null: the step's last block writes {sum of g^2, overflow 0/1} here and
+    // leaves the loss-scale update to a later commit (sharded multi-rank step)
+    double* partial_out = nullptr;
 };
 
 // Rank pointer tables, sized for the largest R.
@@ -73,6 +78,8 @@ cudaError_t launch_reduce_scatter(int32_t R, int32_t dtype, int64_t S, int64_t l
                                   DevState* st, const RankPtrs& p, cudaStream_t s,
                                   bool accumulate = false);
 cudaError_t launch_clip_norm(const StepParams& sp, const RankPtrs& p, cudaStream_t s);
+// Loss-scale update from globally reduced totals {sum of g^2, overflow count}.
+cudaError_t launch_fsm_commit(const StepParams& sp, const double* reduced, cudaStream_t s);
 cudaError_t launch_gather(int32_t R, int64_t S, int64_t lo, int64_t hi, const DevState* st,
                           const RankPtrs& p, void* out, cudaStream_t s);
 
@@ -106,6 +113,7 @@ struct zero_ctx_s {
     bool pow_valid = false;
     int64_t t_bound = 0;          // upper bound of the device step count
     bool two_sets = false;        // a ping-pong step has run (or cur was set to 1)
+    int32_t shard_pingpong = 0;   // the last zero_step_shard wrote set 1-cur
     zero_sched* sched = nullptr;  // created on first use
 };
 

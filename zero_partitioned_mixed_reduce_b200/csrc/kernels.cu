@@ -78,8 +78,7 @@ __device__ __forceinline__ void read_prologue(const StepParams& sp, int R, Prolo
 }
 
 // Loss-scale state machine; one thread. Same rules as the header states.
-__device__ void fsm_update(const StepParams& sp, DevState* st, double norm) {
-    const uint32_t ovf = *reinterpret_cast<volatile uint32_t*>(&st->flag);
+__device__ void fsm_apply(const StepParams& sp, DevState* st, bool ovf, double norm) {
     int skipped = 0;
     if (sp.mode == ZERO_SCALE_DYNAMIC) {
         if (ovf) {
@@ -108,8 +107,14 @@ __device__ void fsm_update(const StepParams& sp, DevState* st, double norm) {
     __threadfence();
 }
 
+__device__ void fsm_update(const StepParams& sp, DevState* st, double norm) {
+    fsm_apply(sp, st, *reinterpret_cast<volatile uint32_t*>(&st->flag) != 0u, norm);
+}
+
 // Every block publishes its norm partial and flag; the last block to finish
-// sums the partials in block order and runs the state machine.
+// sums the partials in block order and runs the state machine -- or, for a
+// sharded step, hands its local totals to the caller for a cross-rank
+// reduction and a later commit.
 __device__ void step_epilogue(const StepParams& sp, double nrm, bool bad) {
     __shared__ double red[kWarps];
     __shared__ int last;
@@ -129,7 +134,21 @@ __device__ void step_epilogue(const StepParams& sp, double nrm, bool bad) {
     for (unsigned i = threadIdx.x; i < gridDim.x; i += kThreads)
         x += *reinterpret_cast<volatile double*>(&sp.partials[i]);
     const double total = block_sum(x, red);
-    if (threadIdx.x == 0) fsm_update(sp, sp.st, total);
+    if (threadIdx.x == 0) {
+        if (sp.partial_out) {
+            sp.partial_out[0] = total;
+            sp.partial_out[1] = *reinterpret_cast<volatile uint32_t*>(&sp.st->flag) != 0u ? 1.0 : 0.0;
+            sp.st->flag = 0u;
+            sp.st->done = 0u;
+            __threadfence();
+        } else {
+            fsm_update(sp, sp.st, total);
+        }
+    }
+}
+
+__global__ void fsm_commit_kernel(const __grid_constant__ StepParams sp, const double* reduced) {
+    if (threadIdx.x == 0 && blockIdx.x == 0) fsm_apply(sp, sp.st, reduced[1] > 0.0, reduced[0]);
 }
 
 // ---------------------------------------------------------------------------
@@ -160,9 +179,10 @@ __global__ void __launch_bounds__(kThreads)
     double nrm = 0.0;
     bool bad = false;
     const uint32_t stride = gridDim.x * kThreads;
-    uint32_t vi = blockIdx.x * kThreads + threadIdx.x;
+    const uint32_t vend = static_cast<uint32_t>(sp.oend) * sp.S8;
+    uint32_t vi = static_cast<uint32_t>(sp.obeg) * sp.S8 + blockIdx.x * kThreads + threadIdx.x;
     OwnerCursor oc(vi, sp.S8);
-    for (; vi < sp.T8; vi += stride) {
+    for (; vi < vend; vi += stride) {
         oc.seek(vi);
         const uint32_t o = oc.o;
         const size_t j8 = static_cast<size_t>(vi - oc.base) * 8;
@@ -284,7 +304,8 @@ __global__ void __launch_bounds__(kThreads)
     const Coef c = pro.c;
     const int src = pro.src, dst = pro.dst;
     const uint32_t S = sp.S8 * 8;
-    const uint32_t ntiles = RC * tiles_per_shard;
+    const uint32_t tbeg = static_cast<uint32_t>(sp.obeg) * tiles_per_shard;
+    const uint32_t ntiles = static_cast<uint32_t>(sp.oend) * tiles_per_shard;  // one past the last tile
     if (threadIdx.x == 0) {
         for (int s = 0; s < kTmaStages; ++s) mbar_init(smem_u32(&bars[s]), 1);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -310,13 +331,13 @@ __global__ void __launch_bounds__(kThreads)
     };
     if (threadIdx.x == 0)
         for (int s = 0; s < kTmaStages; ++s) {
-            const uint32_t tile = blockIdx.x + s * gridDim.x;
+            const uint32_t tile = tbeg + blockIdx.x + s * gridDim.x;
             if (tile < ntiles) issue(tile, s);
         }
     double nrm = 0.0;
     bool bad = false, failed = false;
     int j = 0;
-    for (uint32_t tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++j) {
+    for (uint32_t tile = tbeg + blockIdx.x; tile < ntiles; tile += gridDim.x, ++j) {
         const int s = j % kTmaStages;
         const bool ok = mbar_wait(smem_u32(&bars[s]), (j / kTmaStages) & 1);
         if (__syncthreads_or(!ok)) {
@@ -701,7 +722,7 @@ cudaError_t fused_t(const StepParams& sp, const RankPtrs& p, cudaStream_t s) {
         }
     }
     static const int per_sm = blocks_per_sm(fused_step_kernel<H, RC>);
-    const uint32_t grid = grid_for(sp.T8, per_sm, sp.grid_cap);
+    const uint32_t grid = grid_for(static_cast<uint64_t>(sp.oend - sp.obeg) * sp.S8, per_sm, sp.grid_cap);
     fused_step_kernel<H, RC><<<grid, kThreads, 0, s>>>(a);
     return cudaGetLastError();
 }
@@ -728,7 +749,8 @@ cudaError_t fused_tma_t(const StepParams& sp, const RankPtrs& p, cudaStream_t s)
     }();
     const uint32_t S = sp.S8 * 8;
     const uint32_t tiles_per_shard = (S + kTmaTile - 1) / kTmaTile;
-    const uint32_t grid = grid_for(static_cast<uint64_t>(tiles_per_shard) * RC * kThreads, per_sm, sp.grid_cap);
+    const uint32_t grid = grid_for(static_cast<uint64_t>(tiles_per_shard) * (sp.oend - sp.obeg) * kThreads, per_sm,
+                                   sp.grid_cap);
     fused_step_tma_kernel<H, RC><<<grid, kThreads, smem, s>>>(a, tiles_per_shard);
     return cudaGetLastError();
 }
@@ -816,6 +838,11 @@ cudaError_t acc_t(const StepParams& sp, const RankPtrs& p, cudaStream_t s) {
 
 cudaError_t launch_fused_step(const StepParams& sp, const RankPtrs& p, cudaStream_t s) {
     return sp.dtype == ZERO_FP16 ? fused_dispatch<Fp16>(sp, p, s) : fused_dispatch<Bf16>(sp, p, s);
+}
+
+cudaError_t launch_fsm_commit(const StepParams& sp, const double* reduced, cudaStream_t s) {
+    fsm_commit_kernel<<<1, 32, 0, s>>>(sp, reduced);
+    return cudaGetLastError();
 }
 
 cudaError_t launch_step_from_acc(const StepParams& sp, const RankPtrs& p, cudaStream_t s) {

@@ -1,0 +1,108 @@
+"""ZeRO across GPUs: one process per GPU, rank o owns shard o.
+
+Each rank keeps its full gradient buffer and its half parameter shard in
+symmetric memory (torch.distributed._symmetric_memory), so every rank can
+read every other rank's buffers with plain loads over NVLink. A step is:
+
+  1. a one-element all-reduce on the compute stream, so that every rank's
+     gradients are written before any rank reads them;
+  2. zero_step_shard on the rank's own shard, reading the R gradient buffers
+     through the peer pointers -- the reduce-scatter is the fused kernel's
+     own loads, summed in fp32 in rank order, so no half-precision partial
+     sum ever leaves a GPU;
+  3. an all-reduce (sum) of the two totals {sum g^2, overflow}, which also
+     orders every rank's kernel before anyone overwrites its gradients;
+  4. zero_step_commit, the same skip / loss-scale decision on every rank.
+
+ZeRO-3 layer gathers read the peers' parameter shards the same way.
+Argument marshalling only; the arithmetic runs in libzero_b200.so. The
+loads from peer memory are plain loads or bulk copies without multicast.
+"""
+import torch
+import torch.distributed as dist
+
+from . import _capi as Z
+from .state import HALF, Plan
+
+
+class DistributedZero:
+    def __init__(self, numels, layer_ids=None, dtype=Z.ZERO_BF16, mode=Z.ZERO_SCALE_NONE,
+                 init_scale=1.0, growth_interval=1000, tensor_align=8, bucket_elems=0, group=None):
+        import torch.distributed._symmetric_memory as symm
+        self.group = group or dist.group.WORLD
+        self.world = dist.get_world_size(self.group)
+        self.rank = dist.get_rank(self.group)
+        self.plan = Plan(numels, layer_ids, self.world, dtype, tensor_align, bucket_elems)
+        dev = torch.device("cuda", torch.cuda.current_device())
+        T, S, R = self.plan.T, self.plan.S, self.world
+        half = HALF[dtype]
+        self.dtype, self.mode = dtype, mode
+        # this rank's full gradient buffer, readable by every rank
+        self.grads = symm.empty(T, dtype=half, device=dev)
+        self.grads.zero_()
+        h = symm.rendezvous(self.grads, self.group.group_name)
+        self.grad_ptrs = [int(h.buffer_ptrs[r]) for r in range(R)]
+        self._handles = [h]
+        sets = 2 if mode == Z.ZERO_SCALE_DYNAMIC else 1
+        self.sets = sets
+        self.master = [torch.zeros(S, dtype=torch.float32, device=dev) for _ in range(sets)]
+        self.m = [torch.zeros(S, dtype=torch.float32, device=dev) for _ in range(sets)]
+        self.v = [torch.zeros(S, dtype=torch.float32, device=dev) for _ in range(sets)]
+        self.param = []
+        self.param_ptrs = []
+        for _ in range(sets):
+            p = symm.empty(S, dtype=half, device=dev)
+            p.zero_()
+            hp = symm.rendezvous(p, self.group.group_name)
+            self.param.append(p)
+            self.param_ptrs.append([int(hp.buffer_ptrs[r]) for r in range(R)])
+            self._handles.append(hp)
+
+        def own(x):  # pointer list with only this rank's shard filled in
+            return [x.data_ptr() if r == self.rank else None for r in range(R)]
+        self.handle = Z.StateHandle([dict(master=own(self.master[k]), m=own(self.m[k]),
+                                          v=own(self.v[k]), param=own(self.param[k]))
+                                     for k in range(sets)])
+        self.gather_handle = Z.StateHandle([dict(master=[None] * R, m=[None] * R, v=[None] * R,
+                                                 param=self.param_ptrs[k]) for k in range(sets)])
+        self.ctx = Z.zero_ctx_create(self.plan.handle, mode, init_scale, growth_interval)
+        self.partial = torch.zeros(2, dtype=torch.float64, device=dev)
+        self.token = torch.zeros(1, dtype=torch.float32, device=dev)
+
+    def load(self, master_padded, param_padded):
+        """Initialize this rank's shard from padded flat master (fp32) and param
+        (half) buffers of length T; m = v = 0."""
+        S, o = self.plan.S, self.rank
+        for k in range(self.sets):
+            self.master[k].copy_(master_padded[o * S:(o + 1) * S])
+            self.param[k].copy_(param_padded[o * S:(o + 1) * S])
+            self.m[k].zero_()
+            self.v[k].zero_()
+        torch.cuda.synchronize()
+        dist.barrier(self.group)
+
+    def step(self, hp, stream=None):
+        """One ZeRO step; the gradients of every rank must be in self.grads."""
+        dist.all_reduce(self.token, group=self.group)
+        Z.zero_step_shard(self.ctx, hp, self.handle, self.grad_ptrs, self.rank, self.rank + 1,
+                          self.partial, stream)
+        dist.all_reduce(self.partial, group=self.group)
+        Z.zero_step_commit(self.ctx, self.partial, stream)
+
+    def gather_layer(self, layer, out, stream=None):
+        """ZeRO-3 all-gather of one layer from every rank's parameter shard."""
+        Z.zero_gather_layer(self.ctx, layer, self.gather_handle, out, stream)
+
+    def loss_scale(self):
+        return Z.zero_loss_scale(self.ctx)
+
+    def current(self, field):
+        """This rank's shard of master / m / v / param in the current set."""
+        k = self.loss_scale()["cur"] if self.sets == 2 else 0
+        return getattr(self, field)[k]
+
+    def close(self):
+        if self.ctx:
+            torch.cuda.synchronize()
+            Z.zero_ctx_destroy(self.ctx)
+            self.ctx = None
