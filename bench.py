@@ -66,6 +66,8 @@ def parse_args(argv=None):
                     help="SMs kept free of the synthetic GEMMs in --overlap mode")
     ap.add_argument("--offload", action="store_true",
                     help="measure ZeRO-Offload (CPU AdamW, with and without the delayed update)")
+    ap.add_argument("--graph", action="store_true",
+                    help="capture the step and the gathers once into CUDA graphs and replay them")
     ap.add_argument("--first-tensors", type=int, default=0,
                     help="use only the first N tensors of the workload (small profiling cases)")
     return ap.parse_args(argv)
@@ -301,11 +303,10 @@ class Bench:
             main = (2 * R + 26) * T
         return main + 4 * self.L, main
 
-    def step(self, stream, ev=None):
+    def step_main(self, stream):
+        """The fused (or bucketed two-pass) step: the dominant kernel(s)."""
         Z = self.Z
         hp = self.wl["hp"]
-        if ev is not None:
-            ev[0].record(stream)
         if self.path == "twopass":
             for mu in range(self.accum):
                 flags = Z.ZERO_RS_ACCUMULATE if mu else 0
@@ -316,14 +317,44 @@ class Bench:
                            stream)
         else:
             Z.zero_step(self.ctx, hp, self.state.handle, self.grads, stream)
-        if ev is not None:
-            ev[1].record(stream)
+
+    def gather(self, stream):
+        Z = self.Z
         if self.gather_buckets:
             for (first, _, _), outs in zip(self.gather_buckets, self.gather_outs):
                 Z.zero_gather_layers(self.ctx, first, outs, self.state.handle, stream)
         else:
             for l in range(len(self.plan.layers)):
                 Z.zero_gather_layer(self.ctx, l, self.state.handle, self.layer_buf, stream)
+
+    def capture(self, stream, steps):
+        """Capture the step and the gathers into two CUDA graphs (the event
+        between them stays outside) after reserving `steps` bias corrections."""
+        hp = self.wl["hp"]
+        self.Z.zero_ctx_reserve_steps(self.ctx, steps, hp["beta1"], hp["beta2"], stream)
+        side = torch.cuda.Stream()
+        side.wait_stream(stream)
+        self.graphs = (torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph())
+        with torch.cuda.graph(self.graphs[0], stream=side):
+            self.step_main(torch.cuda.current_stream())
+        with torch.cuda.graph(self.graphs[1], stream=side):
+            self.gather(torch.cuda.current_stream())
+        stream.wait_stream(side)
+
+    def step(self, stream, ev=None):
+        graphs = getattr(self, "graphs", None)
+        if ev is not None:
+            ev[0].record(stream)
+        if graphs:
+            graphs[0].replay()
+        else:
+            self.step_main(stream)
+        if ev is not None:
+            ev[1].record(stream)
+        if graphs:
+            graphs[1].replay()
+        else:
+            self.gather(stream)
 
     def loss_scale(self, stream):
         return self.Z.zero_loss_scale(self.ctx, stream=stream)
@@ -339,6 +370,8 @@ def run_ours(args, world, rank, local):
     b = Bench(args.workload, args.path, args.first_tensors, args.gather_bucket, args.accum,
               args.clip)
     stream = torch.cuda.current_stream()
+    if args.graph:
+        b.capture(stream, args.warmup + args.steps + 1)
     for _ in range(args.warmup):
         b.step(stream)
     torch.cuda.synchronize()
@@ -409,6 +442,8 @@ def run_ours(args, world, rank, local):
             "bytes_per_step": step_bytes,
             "l2": f"inputs larger than L2 ({step_bytes / 1e9:.1f} GB touched per step, L2 126 MB)",
             "parallelism": "1 GPU" if world == 1 else f"{world} independent replicas",
+            "launch": "CUDA graph replay (step graph, event, gather graph)" if args.graph
+                      else "eager launches through the C ABI",
         },
         "roofline": {"bound": "hbm", "kernel": kernel_name, "achieved": achieved, "peak": peak,
                      "peak_source": f"{peak_src} hbm_gbs", "unit": "GB/s", "frac": achieved / peak,
@@ -419,6 +454,7 @@ def run_ours(args, world, rank, local):
     }
     if not args.no_e2e:
         out["e2e"] = e2e(b, args, stream, world)
+    b.graphs = None
     b.close()
     del b
     torch.cuda.empty_cache()

@@ -174,6 +174,25 @@ zero_status zero_ctx_create(const zero_plan_t* plan, const zero_loss_scale_confi
                             zero_ctx_t** out);
 zero_status zero_ctx_destroy(zero_ctx_t* ctx);
 
+/*
+ * zero_ctx_reserve_steps -- make the context's bias-correction table
+ * (beta1^t, beta2^t for the given betas) cover `steps` more optimizer steps
+ * than the host has issued. zero_step grows the table by itself, with a
+ * synchronous allocation and upload. A step captured into a CUDA graph and
+ * replayed advances the device step count without the host seeing it, so
+ * reserve at least the number of replays before capturing:
+ *   - a captured zero_step that would have to grow the table returns
+ *     ZERO_ERR_STATE and launches nothing;
+ *   - a replay beyond the reserve reads the table's last entry (never past
+ *     its end) and sets the device error flag, which the next
+ *     zero_loss_scale reports as ZERO_ERR_STATE.
+ * Outgrown tables stay allocated until zero_ctx_destroy, so no captured
+ * graph ever holds a freed table. `stream` is only checked for a capture in
+ * progress. Blocks the host while the table is uploaded; not capturable.
+ */
+zero_status zero_ctx_reserve_steps(zero_ctx_t* ctx, int64_t steps, double beta1, double beta2,
+                                   void* stream);
+
 /* ------------------------------------------------------------------------ */
 /* The step.                                                                */
 /* ------------------------------------------------------------------------ */

@@ -1,0 +1,159 @@
+"""The step captured once into a CUDA graph and replayed. Every decision of
+the step (overflow, skip, loss scale, which ping-pong set is current, the
+step count behind the bias corrections) lives on the device, so replaying
+one captured launch sequence must give the oracle's state bit for bit,
+skipped steps included. The bias-correction table is reserved before the
+capture; a capture that would have to grow it is refused on the host, and a
+replay that outruns it is reported, not read past."""
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+
+pytestmark = pytest.mark.gpu
+
+if torch.cuda.is_available():
+    import zero_partitioned_mixed_reduce_b200 as Z
+    from gpu_harness import Case
+
+FP16_INF = 0x7C00
+
+
+def _capture(fn):
+    """Capture fn(stream) into a CUDA graph on a side stream. The library
+    allocates nothing during a step, so no warm-up run precedes the capture."""
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s):
+        fn(torch.cuda.current_stream())
+    torch.cuda.current_stream().wait_stream(s)
+    return g
+
+
+def _write_grads(c, inject=None):
+    """Next step's gradient replicas into the captured (static) buffers; also
+    returns them for the oracle."""
+    c.step_no += 1
+    g = c.make_grads(inject)
+    for r in range(c.R):
+        gp = np.zeros(c.plan.T, np.uint16)
+        gp[c.idx] = g[r]
+        c.grads[r].view(torch.int16).copy_(torch.from_numpy(gp.view(np.int16)))
+    return g
+
+
+def _ohp(c):
+    return O.AdamW(**{k: c.hp[k] for k in ("lr", "beta1", "beta2", "eps", "weight_decay")})
+
+
+@pytest.mark.parametrize("R,dtype", [(1, O.BF16), (2, O.FP16), (8, O.FP16), (3, O.BF16)])
+def test_replayed_fused_step_matches_oracle(R, dtype):
+    mode = O.SCALE_DYNAMIC
+    c = Case([70_001, 4096, 13, 9_000], R, dtype, mode=mode, init_scale=2048.0, interval=2,
+             path="pingpong", seed=61)
+    try:
+        Z.zero_ctx_reserve_steps(c.ctx, 16, c.hp["beta1"], c.hp["beta2"])
+        graph = _capture(lambda s: Z.zero_step(c.ctx, c.hp, c.handle, c.grads, s))
+        bad = FP16_INF if dtype == O.FP16 else 0x7F80
+        # step 3 overflows: skipped, scale halves, the ping-pong set stays
+        for k in range(7):
+            inject = [(R - 1, 5, bad)] if k == 2 else None
+            g = _write_grads(c, inject)
+            graph.replay()
+            skipped = O.step(c.ostate, g, _ohp(c), c.ofsm)
+            assert skipped == (k == 2)
+            c.g.check()
+            c.compare()
+    finally:
+        c.close()
+
+
+def test_replayed_two_pass_step_with_clipping_matches_oracle():
+    c = Case([50_000, 333, 8_192], 4, O.BF16, mode=O.SCALE_NONE, path="twopass",
+             bucket_elems=20_000, seed=62)
+    try:
+        Z.zero_ctx_reserve_steps(c.ctx, 8, c.hp["beta1"], c.hp["beta2"])
+        nb = len(c.plan.buckets)
+
+        def step(s):
+            for b in range(nb):
+                Z.zero_reduce_scatter_bucket(c.ctx, b, c.grads, c.acc, s)
+            Z.zero_step_ex(c.ctx, c.hp, c.handle, None, 1.0, 1e-3, s)
+
+        graph = _capture(step)
+        for _ in range(4):
+            g = _write_grads(c)
+            graph.replay()
+            O.step_ex(c.ostate, g[None], _ohp(c), c.ofsm, 1.0, 1e-3)
+            c.g.check()
+            c.compare()
+    finally:
+        c.close()
+
+
+def test_replayed_step_and_gather_match_oracle():
+    layers = [0, 0, 1, 2, 2]
+    c = Case([10_000, 77, 30_001, 4_000, 123], 2, O.FP16, mode=O.SCALE_DYNAMIC, init_scale=512.0,
+             interval=3, path="pingpong", layer_ids=layers, seed=63)
+    try:
+        Z.zero_ctx_reserve_steps(c.ctx, 8, c.hp["beta1"], c.hp["beta2"])
+        L = c.lay.layers
+        outs = [torch.zeros(int(hi - lo), dtype=torch.int16, device="cuda") for lo, hi in L]
+
+        def step(s):
+            Z.zero_step(c.ctx, c.hp, c.handle, c.grads, s)
+            Z.zero_gather_layers(c.ctx, 0, outs, c.handle, s)
+
+        graph = _capture(step)
+        for k in range(5):
+            g = _write_grads(c, [(0, 9, FP16_INF)] if k == 1 else None)
+            graph.replay()
+            O.step(c.ostate, g, _ohp(c), c.ofsm)
+            s = c.compare()
+            # the gathered layers are the current parameters, layer by layer
+            full = np.zeros(c.plan.T, np.uint16)
+            full[c.idx] = s["param"]
+            got = np.concatenate([o.cpu().numpy().view(np.uint16) for o in outs])
+            want = np.concatenate([full[lo:hi] for lo, hi in L])
+            assert np.array_equal(got, want)
+    finally:
+        c.close()
+
+
+def test_capture_that_must_grow_the_table_is_refused():
+    c = Case([5_000], 2, O.BF16, path="pingpong", seed=64)
+    try:
+        s = torch.cuda.Stream()
+        s.wait_stream(torch.cuda.current_stream())
+        g = torch.cuda.CUDAGraph()
+        with pytest.raises(Z.ZeroError):
+            with torch.cuda.graph(g, stream=s):
+                Z.zero_step(c.ctx, c.hp, c.handle, c.grads, torch.cuda.current_stream())
+        torch.cuda.synchronize()
+        # nothing was launched: the context still steps normally afterwards
+        c.step()
+        c.compare()
+    finally:
+        c.close()
+
+
+def test_replay_beyond_the_reserve_is_reported():
+    c = Case([1_000], 1, O.BF16, path="pingpong", seed=65)
+    try:
+        Z.zero_ctx_reserve_steps(c.ctx, 4, c.hp["beta1"], c.hp["beta2"])
+        graph = _capture(lambda s: Z.zero_step(c.ctx, c.hp, c.handle, c.grads, s))
+        _write_grads(c)
+        # the smallest table holds 1024 entries; t + 1 reaches it on replay 1024
+        for _ in range(1023):
+            graph.replay()
+        torch.cuda.synchronize()
+        assert Z.zero_loss_scale(c.ctx)["t"] == 1023
+        graph.replay()
+        torch.cuda.synchronize()
+        with pytest.raises(Z.ZeroError):
+            Z.zero_loss_scale(c.ctx)
+        c.g.check()
+    finally:
+        c.close()

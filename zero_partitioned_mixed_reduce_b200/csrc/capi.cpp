@@ -108,17 +108,25 @@ zero_status ensure_powtab(zero_ctx_t* ctx, double b1, double b2, int64_t need_t,
     if (ctx->powtab && ctx->pow_valid && ctx->pow_b1 == b1 && ctx->pow_b2 == b2 &&
         need_t < ctx->powtab_len)
         return ZERO_OK;
+    // growing the table allocates and copies synchronously, which a stream capture forbids
+    cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+    if (cudaStreamIsCapturing(s, &cap) == cudaSuccess && cap != cudaStreamCaptureStatusNone)
+        return zb_fail(ZERO_ERR_STATE,
+                       "zero_step: the bias-correction table must grow, which cannot happen inside a "
+                       "stream capture; call zero_ctx_reserve_steps before capturing");
     int64_t len = 1024;
     while (len <= need_t) len *= 2;
     std::vector<double2> host(static_cast<size_t>(len));
     for (int64_t t = 0; t < len; ++t)
         host[t] = make_double2(std::pow(b1, static_cast<double>(t)), std::pow(b2, static_cast<double>(t)));
-    // kernels already queued may still read the old table
-    cudaError_t e = cudaStreamSynchronize(s);
-    if (e != cudaSuccess) return cuda_fail("zero_step: power table", e);
-    if (ctx->powtab) cudaFree(ctx->powtab);
+    // Kernels already queued, and kernels captured into CUDA graphs, hold the
+    // old table's address: keep it allocated until the context is destroyed.
+    // A replay that outruns its table reads the last entry and raises the
+    // device error flag instead of reading past the end.
+    if (ctx->powtab) ctx->powtab_retired.push_back(ctx->powtab);
     ctx->powtab = nullptr;
     ctx->powtab_len = 0;
+    cudaError_t e;
     e = cudaMalloc(&ctx->powtab, sizeof(double2) * static_cast<size_t>(len));
     if (e != cudaSuccess) {
         cudaGetLastError();
@@ -208,10 +216,21 @@ extern "C" zero_status zero_ctx_destroy(zero_ctx_t* ctx) {
     cudaFree(ctx->st);
     cudaFree(ctx->partials);
     if (ctx->powtab) cudaFree(ctx->powtab);
+    for (double2* old : ctx->powtab_retired) cudaFree(old);
     if (prev >= 0) cudaSetDevice(prev);
     delete ctx;
     if (e != cudaSuccess) return cuda_fail("zero_ctx_destroy", e);
     return ZERO_OK;
+}
+
+extern "C" zero_status zero_ctx_reserve_steps(zero_ctx_t* ctx, int64_t steps, double beta1, double beta2,
+                                              void* stream) {
+    if (!ctx) return zb_fail(ZERO_ERR_INVALID_ARG, "zero_ctx_reserve_steps: ctx is NULL");
+    zero_status s = check_device(ctx, "zero_ctx_reserve_steps");
+    if (s != ZERO_OK) return s;
+    if (steps < 0 || !(beta1 >= 0.0 && beta1 < 1.0) || !(beta2 >= 0.0 && beta2 < 1.0))
+        return zb_fail(ZERO_ERR_INVALID_ARG, "zero_ctx_reserve_steps: need steps >= 0 and 0 <= beta < 1");
+    return ensure_powtab(ctx, beta1, beta2, ctx->t_bound + 1 + steps, static_cast<cudaStream_t>(stream));
 }
 
 extern "C" zero_status zero_reduce_scatter_bucket(zero_ctx_t* ctx, int64_t bucket,

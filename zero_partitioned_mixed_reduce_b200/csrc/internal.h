@@ -108,6 +108,7 @@ struct zero_ctx_s {
     double* partials = nullptr;   // device, grid_cap entries
     int grid_cap = 0;
     double2* powtab = nullptr;    // device, powtab_len entries
+    std::vector<double2*> powtab_retired;  // outgrown tables, freed with the context
     int64_t powtab_len = 0;
     double pow_b1 = 0.0, pow_b2 = 0.0;
     bool pow_valid = false;
