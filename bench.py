@@ -66,6 +66,10 @@ def parse_args(argv=None):
                     help="SMs kept free of the synthetic GEMMs in --overlap mode")
     ap.add_argument("--offload", action="store_true",
                     help="measure ZeRO-Offload (CPU AdamW, with and without the delayed update)")
+    ap.add_argument("--rs-sweep", action="store_true",
+                    help="time the bucketed reduce-scatter against bucket size instead")
+    ap.add_argument("--rs-sizes", default="0,1000000,5000000,25000000,50000000,100000000,200000000",
+                    help="bucket sizes (elements; 0: one bucket for the whole model) for --rs-sweep")
     ap.add_argument("--graph", action="store_true",
                     help="capture the step and the gathers once into CUDA graphs and replay them")
     ap.add_argument("--first-tensors", type=int, default=0,
@@ -644,6 +648,78 @@ def run_overlap(args, world, rank, local):
         print(json.dumps(out), flush=True)
 
 
+def run_rs_sweep(args, world, rank, local):
+    """The bucketed reduce-scatter (one pass over every bucket of the plan)
+    against bucket size, on the workload's tensors: for each size a plan is
+    built (the flat layout does not depend on it), and the pass is timed
+    issued launch by launch and replayed from a CUDA graph. Reported as the
+    kernel's algorithmic (2R + 4) bytes per padded element over the pass."""
+    if not torch.cuda.is_available():
+        print(json.dumps({"error": "no CUDA device"}))
+        sys.exit(1)
+    import zero_partitioned_mixed_reduce_b200 as Z
+    from zero_partitioned_mixed_reduce_b200 import synth
+    wl = synth.workload(args.workload)
+    R, dtype = wl["R"], wl["dtype"]
+    sizes = [int(x) for x in args.rs_sizes.split(",")]
+    base = Z.Plan(wl["numels"], wl["layer_ids"], R, dtype, 8, 0)
+    T, S = base.T, base.S
+    scale = wl["init_scale"] if wl["mode"] != synth.NONE else 1.0
+    grads = [base.pack(synth.flat_grads(wl, 1, r, scale, "cuda")) for r in range(R)]
+    acc = [torch.empty(S, dtype=torch.float32, device="cuda") for _ in range(R)]
+    stream = torch.cuda.current_stream()
+    nbytes = (2 * R + 4) * T
+    peak, peak_src = hbm_peak()
+    reps = max(3, min(args.steps, 50))
+
+    def timed(fn):
+        for _ in range(args.warmup):
+            fn()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(reps):
+            fn()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / reps
+
+    rows = []
+    for size in sizes:
+        plan = Z.Plan(wl["numels"], wl["layer_ids"], R, dtype, 8, size)
+        assert plan.T == T
+        ctx = Z.zero_ctx_create(plan.handle, wl["mode"], wl["init_scale"], wl["interval"])
+        nb = len(plan.buckets)
+
+        def one_pass(s=stream):
+            for b in range(nb):
+                Z.zero_reduce_scatter_bucket(ctx, b, grads, acc, s)
+
+        t_eager = timed(one_pass)
+        side = torch.cuda.Stream()
+        side.wait_stream(stream)
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=side):
+            one_pass(torch.cuda.current_stream())
+        stream.wait_stream(side)
+        t_graph = timed(g.replay)
+        del g
+        fl = Z.zero_loss_scale(ctx)
+        Z.zero_ctx_destroy(ctx)
+        rows.append({"bucket_elems": size if size > 0 else "whole model", "buckets": nb,
+                     "ms_eager": t_eager, "ms_graph": t_graph,
+                     "gbs_eager": nbytes / (t_eager * 1e-3) / 1e9,
+                     "gbs_graph": nbytes / (t_graph * 1e-3) / 1e9,
+                     "frac_graph": nbytes / (t_graph * 1e-3) / 1e9 / peak,
+                     "overflow_flag": fl["last_overflow"]})
+    out = {"mode": "reduce_scatter_bucket_sweep", "workload": args.workload, "R": R, "T": T,
+           "P": base.P, "tensors": len(wl["numels"]), "algorithmic_bytes_per_pass": nbytes,
+           "peak": peak, "peak_source": f"{peak_src} hbm_gbs", "reps": reps,
+           "l2": f"inputs larger than L2 ({nbytes / 1e9:.1f} GB per pass)", "rows": rows}
+    if rank == 0:
+        print(json.dumps(out), flush=True)
+
+
 def run_offload(args, world, rank, local):
     """ZeRO-Offload on the workload: per step the GPU runs a synthetic
     forward/backward (bf16 GEMMs of 6 * tokens * P flops) and reduce-scatters
@@ -811,6 +887,8 @@ def main(argv=None):
             run_overlap(args, world, rank, local)
         elif args.offload:
             run_offload(args, world, rank, local)
+        elif args.rs_sweep:
+            run_rs_sweep(args, world, rank, local)
         else:
             run_ours(args, world, rank, local)
     finally:
