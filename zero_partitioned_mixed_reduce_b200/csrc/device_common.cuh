@@ -178,6 +178,17 @@ __device__ __forceinline__ double block_sum(double x, double* smem) {
 }
 
 // Owner of a flat vector index, tracked incrementally along a grid-stride loop.
+// First vector of this thread's grid-stride sequence over [v0, ...): the
+// sequence is laid on 128-byte lines of the half-precision gradients (8
+// vectors of 16 bytes) starting at or below v0, so every warp reads whole
+// lines; a thread whose first vector falls below v0 starts one stride later.
+// A start that is not on a line boundary made each warp straddle one more
+// line per gradient stream, about 15 % slower at R = 16.
+__device__ __forceinline__ uint32_t line_start(uint32_t v0, uint32_t stride) {
+    const uint32_t v = (v0 & ~7u) + blockIdx.x * blockDim.x + threadIdx.x;
+    return v < v0 ? v + stride : v;
+}
+
 struct OwnerCursor {
     uint32_t o, base, S8;
     __device__ __forceinline__ OwnerCursor(uint32_t v, uint32_t s8) : S8(s8) {

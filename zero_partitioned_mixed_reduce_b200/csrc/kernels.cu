@@ -180,7 +180,7 @@ __global__ void __launch_bounds__(kThreads)
     bool bad = false;
     const uint32_t stride = gridDim.x * kThreads;
     const uint32_t vend = static_cast<uint32_t>(sp.oend) * sp.S8;
-    uint32_t vi = static_cast<uint32_t>(sp.obeg) * sp.S8 + blockIdx.x * kThreads + threadIdx.x;
+    uint32_t vi = line_start(static_cast<uint32_t>(sp.obeg) * sp.S8, stride);
     OwnerCursor oc(vi, sp.S8);
     for (; vi < vend; vi += stride) {
         oc.seek(vi);
@@ -536,7 +536,7 @@ __global__ void __launch_bounds__(kThreads)
     bool bad = false;
     const uint32_t stride = gridDim.x * kThreads;
     const uint32_t tid = blockIdx.x * kThreads + threadIdx.x;
-    uint32_t vi = a.v0 + tid;
+    uint32_t vi = line_start(a.v0, stride);
     OwnerCursor oc(vi, a.S8);
     for (; vi < a.v1; vi += stride) {
         oc.seek(vi);
