@@ -362,6 +362,8 @@ class Bench:
             graphs[1].replay()
         else:
             self.gather(stream)
+        if ev is not None and len(ev) > 2:
+            ev[2].record(stream)
 
     def loss_scale(self, stream):
         return self.Z.zero_loss_scale(self.ctx, stream=stream)
@@ -386,8 +388,7 @@ def run_ours(args, world, rank, local):
     assert f0["last_overflow"] == 0, "warm-up steps must be clean"
 
     K = args.steps
-    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-           for _ in range(K)]
+    evs = [tuple(torch.cuda.Event(enable_timing=True) for _ in range(3)) for _ in range(K)]
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     clocks = ClockSampler(local)
     clocks.start()
@@ -401,7 +402,8 @@ def run_ours(args, world, rank, local):
     barrier(world)
     clk = clocks.stop()
     ms_local = start.elapsed_time(end)
-    kern_ms = [e0.elapsed_time(e1) for e0, e1 in evs]
+    kern_ms = [e0.elapsed_time(e1) for e0, e1, _ in evs]
+    gather_ms = statistics.mean(e1.elapsed_time(e2) for _, e1, e2 in evs)
     f1 = b.loss_scale(stream)
     assert f1["last_overflow"] == 0 and f1["t"] == f0["t"] + K
     ms, units = aggregate(ms_local, float(b.P) * K, world)
@@ -456,6 +458,9 @@ def run_ours(args, world, rank, local):
                      "peak_source": f"{peak_src} hbm_gbs", "unit": "GB/s", "frac": achieved / peak,
                      "traffic": traffic, "algorithmic_bytes_per_launch": main_bytes,
                      "avg_launch_ms": kavg},
+        "gather": {"avg_ms_per_step": gather_ms, "elements": b.L,
+                   "gbs": 4.0 * b.L / (gather_ms * 1e-3) / 1e9,
+                   "launches_per_step": len(b.gather_buckets) or len(b.plan.layers)},
         "clocks": clk,
         "gpu_launches": K * b.launches_per_step(),
     }
