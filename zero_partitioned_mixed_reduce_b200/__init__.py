@@ -6,6 +6,8 @@ include/zero_b200.h); this package binds it with ctypes and uses PyTorch
 only for device memory and streams.
 """
 from ._capi import (  # noqa: F401
+    ZERO_OK, ZERO_ERR_INVALID_ARG, ZERO_ERR_ALIGN, ZERO_ERR_CUDA, ZERO_ERR_OOM, ZERO_ERR_RANGE,
+    ZERO_ERR_TIMEOUT, ZERO_ERR_STATE, STATUS_NAMES,
     ZERO_BF16, ZERO_FP16, ZERO_LOSS_SCALE_GET, ZERO_LOSS_SCALE_SET, ZERO_MAX_RANKS,
     ZERO_SCALE_DYNAMIC, ZERO_SCALE_NONE, ZERO_SCALE_STATIC, LIB_PATH, StateHandle, ZeroError,
     zero_adamw, zero_ctx_create, zero_ctx_destroy, zero_gather_layer, zero_gather_layers,
