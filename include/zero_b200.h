@@ -50,7 +50,7 @@ typedef enum {
     ZERO_ERR_CUDA = 3,        /* a CUDA runtime error (launch, async fault, no device) */
     ZERO_ERR_OOM = 4,         /* host or device allocation failed */
     ZERO_ERR_RANGE = 5,       /* a bucket / layer / tensor index or a size out of range */
-    ZERO_ERR_TIMEOUT = 6,     /* reserved: a bounded device wait gave up */
+    ZERO_ERR_TIMEOUT = 6,     /* a bounded device wait gave up; the step was abandoned */
     ZERO_ERR_STATE = 7        /* the call does not fit the context's state */
 } zero_status;
 
@@ -192,6 +192,19 @@ zero_status zero_ctx_destroy(zero_ctx_t* ctx);
  */
 zero_status zero_ctx_reserve_steps(zero_ctx_t* ctx, int64_t steps, double beta1, double beta2,
                                    void* stream);
+
+/*
+ * zero_test_drop_tile -- test support for the error path of the staged
+ * fused step (R <= 2): the next zero_step / zero_step_shard with gradients
+ * issues no copy for tile `tile` (tiles are 2048-element pieces of the
+ * shards, numbered shard after shard), so the block that waits for it gives
+ * up after its 2 s limit, as it would if a copy never arrived. The step is
+ * then abandoned and reported as ZERO_ERR_TIMEOUT (see zero_loss_scale);
+ * nothing faults and the context stays usable. One-shot; no effect on the
+ * register kernel (R >= 4). Not part of the method; the pages have no
+ * counterpart. Errors: ZERO_ERR_INVALID_ARG.
+ */
+zero_status zero_test_drop_tile(zero_ctx_t* ctx, int64_t tile);
 
 /* ------------------------------------------------------------------------ */
 /* The step.                                                                */
@@ -407,8 +420,15 @@ typedef struct {
  * loss-scale state; SET is how a run resumes from a checkpoint. Both
  * synchronize `stream` (GET reads the state after all work queued on it).
  * Defines: the state of [legal] "Dynamic Loss Scaling".
+ * A step during which the device raised an error is abandoned: t, scale,
+ * good and cur keep their values from before it, so with ping-pong state
+ * the current set still holds the model from before the step (an in-place
+ * step may have updated part of its set). GET then returns
+ * ZERO_ERR_TIMEOUT (a step kernel's bounded wait for its tile copies ran
+ * out) or ZERO_ERR_STATE (the bias-correction table was behind t) until a
+ * SET, which clears the error.
  * Errors: ZERO_ERR_INVALID_ARG (op, NULL, cur not 0/1, scale <= 0, t < 0),
- * ZERO_ERR_CUDA.
+ * ZERO_ERR_TIMEOUT, ZERO_ERR_STATE, ZERO_ERR_CUDA.
  */
 zero_status zero_loss_scale(zero_ctx_t* ctx, zero_loss_scale_state* inout, int32_t op,
                             void* stream);

@@ -101,6 +101,7 @@ _sig("zero_plan_memory", _S, [_P, C.c_int32, C.POINTER(C.c_int64)])
 _sig("zero_ctx_create", _S, [_P, C.POINTER(zero_loss_scale_config), C.POINTER(_P)])
 _sig("zero_ctx_destroy", _S, [_P])
 _sig("zero_ctx_reserve_steps", _S, [_P, C.c_int64, C.c_double, C.c_double, _P])
+_sig("zero_test_drop_tile", _S, [_P, C.c_int64])
 _sig("zero_reduce_scatter_bucket", _S, [_P, C.c_int64, _PP, _PP, _P])
 _sig("zero_step", _S, [_P, C.POINTER(zero_adamw), C.POINTER(zero_state), _PP, _P])
 _sig("zero_reduce_scatter_bucket_ex", _S, [_P, C.c_int64, _PP, _PP, C.c_int32, _P])
@@ -225,6 +226,10 @@ def zero_ctx_destroy(ctx):
 
 def zero_ctx_reserve_steps(ctx, steps, beta1=0.9, beta2=0.999, stream=None):
     _check(_lib.zero_ctx_reserve_steps(ctx, steps, beta1, beta2, _stream(stream)))
+
+
+def zero_test_drop_tile(ctx, tile):
+    _check(_lib.zero_test_drop_tile(ctx, tile))
 
 
 class StateHandle:

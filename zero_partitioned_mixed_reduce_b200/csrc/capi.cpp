@@ -233,6 +233,14 @@ extern "C" zero_status zero_ctx_reserve_steps(zero_ctx_t* ctx, int64_t steps, do
     return ensure_powtab(ctx, beta1, beta2, ctx->t_bound + 1 + steps, static_cast<cudaStream_t>(stream));
 }
 
+extern "C" zero_status zero_test_drop_tile(zero_ctx_t* ctx, int64_t tile) {
+    if (!ctx) return zb_fail(ZERO_ERR_INVALID_ARG, "zero_test_drop_tile: ctx is NULL");
+    if (tile < 0 || tile >= 0xffffffffLL)
+        return zb_fail(ZERO_ERR_INVALID_ARG, "zero_test_drop_tile: need 0 <= tile < 2^32 - 1");
+    ctx->drop_tile = static_cast<uint32_t>(tile);
+    return ZERO_OK;
+}
+
 extern "C" zero_status zero_reduce_scatter_bucket(zero_ctx_t* ctx, int64_t bucket,
                                                   const void* const* grads, float* const* acc,
                                                   void* stream) {
@@ -346,6 +354,7 @@ extern "C" zero_status zero_step_ex(zero_ctx_t* ctx, const zero_adamw* hp, const
     sp.grid_cap = ctx->grid_cap;
     sp.obeg = 0;
     sp.oend = ctx->R;
+    if (fused) sp.drop_tile = ctx->drop_tile;
 
     zb::RankPtrs p;
     fill_state_ptrs(ctx, state, sets, &p);
@@ -359,6 +368,7 @@ extern "C" zero_status zero_step_ex(zero_ctx_t* ctx, const zero_adamw* hp, const
         e = fused ? zb::launch_fused_step(sp, p, cs) : zb::launch_step_from_acc(sp, p, cs);
     if (e != cudaSuccess) return cuda_fail(where, e);
     ctx->t_bound += 1;
+    if (fused) ctx->drop_tile = 0xffffffffu;
     if (sp.pingpong) ctx->two_sets = true;
     return ZERO_OK;
 }
@@ -445,6 +455,7 @@ extern "C" zero_status zero_step_shard(zero_ctx_t* ctx, const zero_adamw* hp, co
     sp.obeg = owner_lo;
     sp.oend = owner_hi;
     sp.partial_out = partial;
+    sp.drop_tile = ctx->drop_tile;
     zb::RankPtrs p{};
     for (int r = 0; r < ctx->R; ++r) {
         p.g[r] = grads[r];
@@ -460,6 +471,7 @@ extern "C" zero_status zero_step_shard(zero_ctx_t* ctx, const zero_adamw* hp, co
     cudaError_t e = zb::launch_fused_step(sp, p, cs);
     if (e != cudaSuccess) return cuda_fail(where, e);
     ctx->t_bound += 1;
+    ctx->drop_tile = 0xffffffffu;
     ctx->shard_pingpong = sp.pingpong;
     if (sp.pingpong) ctx->two_sets = true;
     return ZERO_OK;

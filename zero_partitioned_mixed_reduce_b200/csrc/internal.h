@@ -59,6 +59,9 @@ struct StepParams {
     // non-null: the step's last block writes {sum of g^2, overflow 0/1} here and
     // leaves the loss-scale update to a later commit (sharded multi-rank step)
     double* partial_out = nullptr;
+    // test support (zero_test_drop_tile): the staged kernel issues no copy
+    // for this tile, so the block waiting for it gives up after its limit
+    uint32_t drop_tile = 0xffffffffu;
 };
 
 // Rank pointer tables, sized for the largest R.
@@ -107,6 +110,7 @@ struct zero_ctx_s {
     zb::DevState* st = nullptr;   // device
     double* partials = nullptr;   // device, grid_cap entries
     int grid_cap = 0;
+    uint32_t drop_tile = 0xffffffffu;  // one-shot, for the next fused step
     double2* powtab = nullptr;    // device, powtab_len entries
     std::vector<double2*> powtab_retired;  // outgrown tables, freed with the context
     int64_t powtab_len = 0;

@@ -77,10 +77,16 @@ __device__ __forceinline__ void read_prologue(const StepParams& sp, int R, Prolo
     __syncthreads();
 }
 
-// Loss-scale state machine; one thread. Same rules as the header states.
+// Loss-scale state machine; one thread. Same rules as the header states. A
+// step during which some block raised the device error flag (a bounded wait
+// that gave up, a power table behind t) is abandoned: t, the scale, the
+// clean-step count and cur keep their values, so with ping-pong state the
+// current model is the one from before the step.
 __device__ void fsm_apply(const StepParams& sp, DevState* st, bool ovf, double norm) {
     int skipped = 0;
-    if (sp.mode == ZERO_SCALE_DYNAMIC) {
+    if (*reinterpret_cast<volatile int32_t*>(&st->err) != 0) {
+        skipped = 1;
+    } else if (sp.mode == ZERO_SCALE_DYNAMIC) {
         if (ovf) {
             const float s = __fmul_rn(st->scale, sp.backoff);
             st->scale = (s < sp.min_scale) ? sp.min_scale : s;
@@ -318,6 +324,7 @@ __global__ void __launch_bounds__(kThreads)
         const uint32_t len = min(static_cast<uint32_t>(kTmaTile), S - j0);
         unsigned char* base = smem + s * L::kBytes;
         const uint32_t bar = smem_u32(&bars[s]);
+        if (tile == sp.drop_tile) return;  // test support: this tile's wait must run out
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
         mbar_expect_tx(bar, len * (RC * 2 + 12));
 #pragma unroll
