@@ -271,3 +271,35 @@ def test_argument_errors():
             Z.zero_loss_scale(c.ctx, Z.ZERO_LOSS_SCALE_SET, dict(scale=-1.0, cur=0, t=0, good=0))
     finally:
         c.close()
+
+
+@pytest.mark.parametrize("R", [5, 7, 32, 64])
+@pytest.mark.parametrize("path,mode", [("inplace", O.SCALE_NONE), ("pingpong", O.SCALE_DYNAMIC),
+                                       ("twopass", O.SCALE_STATIC)])
+def test_many_ranks_match_oracle(R, path, mode):
+    # the runtime-R kernels, up to the ABI's maximum of 64 ranks, where most
+    # shards are short and several are pure padding
+    numels = tensor_list(R * 7 + len(path), big=(R == 7))
+    init = 1024.0 if mode != O.SCALE_NONE else 1.0
+    c = Case(numels, R, O.FP16, 8, mode, init_scale=init, interval=2, path=path, bucket_elems=2000)
+    try:
+        for _ in range(3):
+            c.step()
+            c.compare()
+    finally:
+        c.close()
+
+
+@pytest.mark.parametrize("R", [1, 2, 8, 64])
+@pytest.mark.parametrize("path", ["inplace", "pingpong", "twopass"])
+def test_single_parameter_model(R, path):
+    # P = 1: one real element, the rest of every shard is padding
+    mode = O.SCALE_DYNAMIC if path == "pingpong" else O.SCALE_NONE
+    c = Case([1], R, O.BF16, 8, mode, init_scale=8.0, interval=2, path=path)
+    try:
+        for _ in range(3):
+            c.step()
+            c.compare()
+        assert c.plan.T == 8 * R
+    finally:
+        c.close()
