@@ -46,7 +46,10 @@ def parse_args(argv=None):
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="gpt2s")
-    ap.add_argument("--path", choices=["auto", "pingpong", "inplace", "twopass"], default="auto")
+    ap.add_argument("--path", choices=["auto", "pingpong", "inplace", "twopass", "twopass_pingpong"],
+                    default="auto",
+                    help="fused step (ping-pong or in-place state) or the two-pass path "
+                         "(in-place or ping-pong state)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--accum", type=int, default=1,
@@ -235,14 +238,17 @@ class Bench:
                 # (the writes never alias the lines being read); it doubles the
                 # fp32 state, which every workload here fits
                 path = "pingpong"
-        if (accum > 1 or clip > 0) and path != "twopass":
+        self.twopass = path.startswith("twopass")
+        if (accum > 1 or clip > 0) and not self.twopass:
             raise SystemExit("--accum/--clip need the two-pass path")
         self.path = path
         self.plan = Z.Plan(wl["numels"], wl["layer_ids"], wl["R"], wl["dtype"], 8,
                            wl["bucket_elems"])
         self.P, self.T, self.S, self.L = self.plan.P, self.plan.T, self.plan.S, self.plan.L
-        sets = 2 if path == "pingpong" else 1
-        self.state = Z.ShardedState(self.plan, sets=sets, with_acc=(path == "twopass"))
+        # the two-pass step measured the same in place as ping-pong, so it
+        # keeps one state set
+        sets = 2 if path in ("pingpong", "twopass_pingpong") else 1
+        self.state = Z.ShardedState(self.plan, sets=sets, with_acc=self.twopass)
         half = Z.state.HALF[wl["dtype"]]
         # initial fp32 master ~N(0, 0.02) and its half copy, tensor by tensor
         for k, (n, off) in enumerate(zip(wl["numels"], self.plan.offsets)):
@@ -294,14 +300,14 @@ class Bench:
 
     def launches_per_step(self):
         n = 1 + (len(self.gather_buckets) if self.gather_buckets else len(self.plan.layers))
-        if self.path == "twopass":
+        if self.twopass:
             n += self.accum * len(self.plan.buckets) + (1 if self.clip > 0 else 0)
         return n
 
     def step_bytes(self):
         """Algorithmic HBM bytes of one step (and of its dominant kernel)."""
         R, T = self.R, self.T
-        if self.path == "twopass":
+        if self.twopass:
             # first micro-batch writes the accumulators, later ones read-modify-write
             main = (2 * R + 4) * T + (self.accum - 1) * (2 * R + 8) * T + 30 * T
             if self.clip > 0:
@@ -314,7 +320,7 @@ class Bench:
         """The fused (or bucketed two-pass) step: the dominant kernel(s)."""
         Z = self.Z
         hp = self.wl["hp"]
-        if self.path == "twopass":
+        if self.twopass:
             for mu in range(self.accum):
                 flags = Z.ZERO_RS_ACCUMULATE if mu else 0
                 for b in range(len(self.plan.buckets)):
@@ -380,7 +386,7 @@ def run_ours(args, world, rank, local):
               args.clip)
     stream = torch.cuda.current_stream()
     if args.graph:
-        b.capture(stream, args.warmup + args.steps + 1)
+        b.capture(stream, args.warmup + args.steps + 16)  # + the e2e leg's steps
     for _ in range(args.warmup):
         b.step(stream)
     torch.cuda.synchronize()
@@ -412,9 +418,8 @@ def run_ours(args, world, rank, local):
     peak, peak_src = hbm_peak()
     kavg = statistics.mean(kern_ms)
     achieved = main_bytes / (kavg * 1e-3) / 1e9
-    kernel_name = {"pingpong": "fused_step_kernel", "inplace": "fused_step_kernel",
-                   "twopass": "reduce_scatter+step_from_acc"}[b.path]
-    if b.path == "twopass" and (b.accum > 1 or b.clip > 0):
+    kernel_name = "reduce_scatter+step_from_acc" if b.twopass else "fused_step_kernel"
+    if b.twopass and (b.accum > 1 or b.clip > 0):
         kernel_name += f" (accum {b.accum}{', clip' if b.clip > 0 else ''})"
     traffic = profiled_traffic(kernel_name, args.workload)
     out = {
@@ -443,7 +448,10 @@ def run_ours(args, world, rank, local):
                      "inplace": "fused reduce-scatter+AdamW, in place",
                      "twopass": f"bucketed reduce-scatter ({b.accum} micro-batch(es)), "
                        f"{'global-norm clip, ' if b.clip > 0 else ''}"
-                       "then AdamW from fp32 accumulators"}[b.path]
+                       "then AdamW from fp32 accumulators, in place",
+                     "twopass_pingpong": f"bucketed reduce-scatter ({b.accum} micro-batch(es)), "
+                       f"{'global-norm clip, ' if b.clip > 0 else ''}"
+                       "then AdamW from fp32 accumulators, ping-pong state"}[b.path]
                     + " + device loss-scale update + ZeRO-3 gather of every layer",
             "gather": (f"{len(b.gather_buckets)} bucketed launches of consecutive layers "
                        f"(<= {args.gather_bucket} elements each)" if b.gather_buckets

@@ -219,8 +219,11 @@ typedef struct {
  * during the call only); entry r points at rank r's shard of S elements.
  * master/m/v are fp32, param is the plan's half dtype. Set 0 is required;
  * set 1 (all four arrays non-NULL, or all NULL) enables ping-pong steps:
- * the fused step then reads set `cur` and writes set 1-cur, and flips `cur`
- * only if the step is applied, so a skipped step costs no extra traffic.
+ * the step (fused, or from the accumulators) then reads set `cur` and
+ * writes set 1-cur, and flips `cur` only if the step is applied, so a
+ * skipped step costs no extra traffic. Ping-pong also measured faster than
+ * updating in place (writes never alias the lines being read), at the cost
+ * of a second state set.
  * acc holds R fp32 accumulators of S elements for the two-pass path (may be
  * NULL for the fused path and for gathers).
  */
@@ -298,7 +301,8 @@ zero_status zero_reduce_scatter_bucket_ex(zero_ctx_t* ctx, int64_t bucket, const
  *
  * grads == NULL: two-pass path; g comes from the accumulators written by
  * zero_reduce_scatter_bucket for this step (state->acc), the step is done in
- * place on set cur. grads != NULL: fused path; the R replicas are reduced,
+ * place on set cur when the state has one set, from set cur into set 1-cur
+ * when it has two (a skipped step writes nothing either way). grads != NULL: fused path; the R replicas are reduced,
  * checked, and applied in one pass with no accumulator: in place when the
  * state has one set (NONE or STATIC mode only, since an in-place fused step
  * cannot be undone), ping-pong when it has two.

@@ -60,8 +60,9 @@ def f32bits(a: np.ndarray) -> np.ndarray:
 
 class Case:
     """One parity case: a tensor list, R, dtype, alignment, loss-scale mode and
-    path ("inplace", "pingpong", "twopass"), run for a few steps on the GPU
-    and in the oracle on the same bytes."""
+    path ("inplace", "pingpong", "twopass", "twopass_pp": two-pass with
+    ping-pong state), run for a few steps on the GPU and in the oracle on the
+    same bytes."""
 
     def __init__(self, numels, R, dtype, align=8, mode=O.SCALE_NONE, init_scale=1.0, interval=1000,
                  path="pingpong", bucket_elems=0, layer_ids=None, sigma=1e-2, seed=5, hp=None):
@@ -74,13 +75,13 @@ class Case:
         self.idx = self.lay.flat_index()
         S, T = self.plan.S, self.plan.T
         self.g = Guarded()
-        sets = 2 if path == "pingpong" else 1
+        sets = 2 if path in ("pingpong", "twopass_pp") else 1
         self.sets = sets
         self.master = [[self.g.f32(S) for _ in range(R)] for _ in range(sets)]
         self.m = [[self.g.f32(S) for _ in range(R)] for _ in range(sets)]
         self.v = [[self.g.f32(S) for _ in range(R)] for _ in range(sets)]
         self.param = [[self.g.half(S, dtype) for _ in range(R)] for _ in range(sets)]
-        self.acc = [self.g.f32(S) for _ in range(R)] if path == "twopass" else None
+        self.acc = [self.g.f32(S) for _ in range(R)] if path.startswith("twopass") else None
         self.grads = [self.g.half(T, dtype) for _ in range(R)]
         self.handle = Z.StateHandle(
             [dict(master=self.master[k], m=self.m[k], v=self.v[k], param=self.param[k])
@@ -126,7 +127,7 @@ class Case:
             gp = np.zeros(self.plan.T, np.uint16)
             gp[self.idx] = g[r]
             self.grads[r].view(torch.int16).copy_(torch.from_numpy(gp.view(np.int16)))
-        if self.path == "twopass":
+        if self.path.startswith("twopass"):
             for b in range(len(self.plan.buckets)):
                 Z.zero_reduce_scatter_bucket(self.ctx, b, self.grads, self.acc)
             Z.zero_step(self.ctx, self.hp, self.handle, None)
@@ -141,7 +142,7 @@ class Case:
     def step_ex(self, n_micro, grad_divisor=1.0, max_grad_norm=0.0, inject=None):
         """Two-pass step over n_micro accumulated micro-batches, optionally
         clipped; inject: (micro, rank, element, bits) tuples."""
-        assert self.path == "twopass"
+        assert self.path.startswith("twopass")
         self.step_no += 1
         scale = self.ofsm.scale if self.mode != O.SCALE_NONE else 1.0
         micro = []
@@ -173,7 +174,7 @@ class Case:
         scheduler: each tensor's gradients are written on the caller's stream
         (after `busy` work, standing in for backward) in reverse tensor order,
         then reported ready; join; step."""
-        assert self.path == "twopass"
+        assert self.path.startswith("twopass")
         self.step_no += 1
         scale = self.ofsm.scale if self.mode != O.SCALE_NONE else 1.0
         micro = []

@@ -18,11 +18,12 @@ if torch.cuda.is_available():
 @pytest.mark.parametrize("dtype", [O.BF16, O.FP16])
 @pytest.mark.parametrize("n_micro,divisor", [(1, 1.0), (2, 2.0), (3, 3.0), (4, 1.0)])
 @pytest.mark.parametrize("clip", [0.0, 1e-3, 1e9])
-def test_accumulate_and_clip_match_oracle(R, dtype, n_micro, divisor, clip):
+@pytest.mark.parametrize("path", ["twopass", "twopass_pp"])
+def test_accumulate_and_clip_match_oracle(R, dtype, n_micro, divisor, clip, path):
     numels = [70_001, 13, 4096, 7, 999]
     mode = O.SCALE_DYNAMIC if dtype == O.FP16 else O.SCALE_NONE
     c = Case(numels, R, dtype, 8 if R != 3 else 1, mode, init_scale=256.0, interval=2,
-             path="twopass", bucket_elems=5000)
+             path=path, bucket_elems=5000)
     try:
         for _ in range(3):
             c.step_ex(n_micro, divisor, clip)
@@ -34,8 +35,9 @@ def test_accumulate_and_clip_match_oracle(R, dtype, n_micro, divisor, clip):
 
 
 @pytest.mark.parametrize("micro", [0, 1, 2])
-def test_overflow_in_one_micro_batch_skips(micro):
-    c = Case([5000, 33], 4, O.FP16, 8, O.SCALE_DYNAMIC, init_scale=64.0, path="twopass")
+@pytest.mark.parametrize("path", ["twopass", "twopass_pp"])
+def test_overflow_in_one_micro_batch_skips(micro, path):
+    c = Case([5000, 33], 4, O.FP16, 8, O.SCALE_DYNAMIC, init_scale=64.0, path=path)
     try:
         c.step_ex(3, 3.0, 0.5)
         c.compare()

@@ -28,7 +28,8 @@ def tensor_list(seed, big=False):
 
 
 PATHS = [("inplace", O.SCALE_NONE), ("inplace", O.SCALE_STATIC), ("pingpong", O.SCALE_NONE),
-         ("pingpong", O.SCALE_DYNAMIC), ("twopass", O.SCALE_STATIC), ("twopass", O.SCALE_DYNAMIC)]
+         ("pingpong", O.SCALE_DYNAMIC), ("twopass", O.SCALE_STATIC), ("twopass", O.SCALE_DYNAMIC),
+         ("twopass_pp", O.SCALE_NONE), ("twopass_pp", O.SCALE_DYNAMIC)]
 
 
 @pytest.mark.parametrize("R", [1, 2, 3, 4, 8, 16])
@@ -56,7 +57,7 @@ def nan_bits(dtype):
     return 0x7E00 if dtype == O.FP16 else 0x7FC0
 
 
-@pytest.mark.parametrize("path", ["pingpong", "twopass"])
+@pytest.mark.parametrize("path", ["pingpong", "twopass", "twopass_pp"])
 @pytest.mark.parametrize("dtype", [O.BF16, O.FP16])
 @pytest.mark.parametrize("where", ["first", "last", "before_pad", "after_pad"])
 @pytest.mark.parametrize("kind", ["inf", "nan"])
@@ -208,7 +209,7 @@ def test_deterministic_bit_for_bit():
         assert np.array_equal(np.asarray(a[k]).view(np.uint8), np.asarray(b[k]).view(np.uint8))
 
 
-@pytest.mark.parametrize("path", ["pingpong", "twopass"])
+@pytest.mark.parametrize("path", ["pingpong", "twopass", "twopass_pp"])
 def test_checkpoint_resume(path):
     numels = [1000, 33, 4097]
     straight = Case(numels, 4, O.FP16, 8, O.SCALE_DYNAMIC, 32.0, interval=2, path=path)

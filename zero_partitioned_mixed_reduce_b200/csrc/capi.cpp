@@ -330,7 +330,7 @@ extern "C" zero_status zero_step_ex(zero_ctx_t* ctx, const zero_adamw* hp, const
     sp.R = ctx->R;
     sp.dtype = ctx->dtype;
     sp.mode = ctx->cfg.mode;
-    sp.pingpong = (fused && sets == 2) ? 1 : 0;
+    sp.pingpong = sets == 2 ? 1 : 0;
     sp.S8 = static_cast<uint32_t>(ctx->S / 8);
     sp.T8 = static_cast<uint32_t>(ctx->T / 8);
     sp.dec = static_cast<float>(1.0 - hp->lr * hp->weight_decay);

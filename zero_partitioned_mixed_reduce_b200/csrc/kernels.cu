@@ -400,7 +400,8 @@ __global__ void __launch_bounds__(kThreads)
 
 // ---------------------------------------------------------------------------
 // Two-pass step: AdamW from the fp32 accumulators written by the
-// reduce-scatter kernel. In place on set cur; skipped (state untouched) in
+// reduce-scatter kernel. In place on set cur, or from set cur into set 1-cur
+// when both sets are given (ping-pong); skipped (no state written) in
 // DYNAMIC mode when the reduce-scatter raised the overflow flag. The norm is
 // always formed from the accumulators.
 // ---------------------------------------------------------------------------
@@ -420,7 +421,7 @@ __global__ void __launch_bounds__(kThreads) step_from_acc_kernel(const __grid_co
     __shared__ Prologue pro;
     read_prologue(sp, sp.R, &pro, true);
     const Coef c = pro.c;
-    const int cur = pro.src;
+    const int src = pro.src, dst = pro.dst;
     const bool skip = pro.skip != 0;
 
     double nrm = 0.0;
@@ -440,9 +441,9 @@ __global__ void __launch_bounds__(kThreads) step_from_acc_kernel(const __grid_co
             }
             continue;
         }
-        F8 p = ld_f8(a.master[cur][o] + j8);
-        F8 m = ld_f8(a.m[cur][o] + j8);
-        F8 v = ld_f8(a.v[cur][o] + j8);
+        F8 p = ld_f8(a.master[src][o] + j8);
+        F8 m = ld_f8(a.m[src][o] + j8);
+        F8 v = ld_f8(a.v[src][o] + j8);
         float out[8];
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
@@ -451,10 +452,10 @@ __global__ void __launch_bounds__(kThreads) step_from_acc_kernel(const __grid_co
             nrm = fma(gd, gd, nrm);
             out[e] = p.x[e];
         }
-        st_f8(a.master[cur][o] + j8, p);
-        st_f8(a.m[cur][o] + j8, m);
-        st_f8(a.v[cur][o] + j8, v);
-        st_u4(a.param[cur][o] + (j8 >> 3), pack8<H>(out));
+        st_f8(a.master[dst][o] + j8, p);
+        st_f8(a.m[dst][o] + j8, m);
+        st_f8(a.v[dst][o] + j8, v);
+        st_u4(a.param[dst][o] + (j8 >> 3), pack8<H>(out));
     }
     step_epilogue(sp, nrm, false);
 }
@@ -465,6 +466,8 @@ __global__ void __launch_bounds__(kThreads) step_from_acc_kernel(const __grid_co
 // the clipping coefficient min(1, max_norm / (||g|| + 1e-6)) (in double) and
 // stores it in the device state for the step kernel.
 // ---------------------------------------------------------------------------
+
+constexpr int kNormUnroll = 4;
 
 struct NormArgs {
     StepParams sp;
@@ -488,14 +491,27 @@ __global__ void __launch_bounds__(kThreads) clip_norm_kernel(const __grid_consta
     const uint32_t stride = gridDim.x * kThreads;
     uint32_t vi = blockIdx.x * kThreads + threadIdx.x;
     OwnerCursor oc(vi, sp.S8);
-    for (; vi < sp.T8; vi += stride) {
-        oc.seek(vi);
-        const F8 acc = ld_f8(a.acc[oc.o] + static_cast<size_t>(vi - oc.base) * 8);
+    // a short read-only pass: keep kNormUnroll vectors per thread in flight
+    for (; vi < sp.T8; vi += kNormUnroll * stride) {
+        F8 acc[kNormUnroll];
 #pragma unroll
-        for (int e = 0; e < 8; ++e) {
-            const double gd = static_cast<double>(__fmul_rn(acc.x[e], inv));
-            nrm = fma(gd, gd, nrm);
+        for (int u = 0; u < kNormUnroll; ++u) {
+            const uint32_t vu = vi + u * stride;
+            if (vu < sp.T8) {
+                oc.seek(vu);
+                acc[u] = ld_f8(a.acc[oc.o] + static_cast<size_t>(vu - oc.base) * 8);
+            } else {
+#pragma unroll
+                for (int e = 0; e < 8; ++e) acc[u].x[e] = 0.0f;
+            }
         }
+#pragma unroll
+        for (int u = 0; u < kNormUnroll; ++u)
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                const double gd = static_cast<double>(__fmul_rn(acc[u].x[e], inv));
+                nrm = fma(gd, gd, nrm);
+            }
     }
     const double bn = block_sum(nrm, red);
     if (threadIdx.x == 0) {
