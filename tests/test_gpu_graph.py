@@ -157,3 +157,45 @@ def test_replay_beyond_the_reserve_is_reported():
         c.g.check()
     finally:
         c.close()
+
+
+@pytest.mark.parametrize("mode", [O.SCALE_DYNAMIC, O.SCALE_NONE])
+def test_replayed_overlapped_step_matches_oracle(mode):
+    # the scheduler's cross-stream work (reduce-scatters on the communication
+    # stream as tensors are reported ready, then the join) captured with the
+    # gradient writes and the step into one graph
+    numels = [30_000, 77, 5_000, 12_001, 9]
+    R = 4
+    c = Case(numels, R, O.FP16, mode=mode, init_scale=256.0, interval=2, path="twopass",
+             bucket_elems=15_000, seed=66)
+    try:
+        c.step_overlap()  # first use creates the scheduler's stream and events
+        c.compare()
+        Z.zero_ctx_reserve_steps(c.ctx, 8, c.hp["beta1"], c.hp["beta2"])
+        P = c.lay.P
+        starts = np.concatenate([[0], np.cumsum(c.lay.numels)[:-1]])
+        dev = torch.zeros((R, P), dtype=torch.int16, device="cuda")
+
+        def step(s):
+            for r in range(R):
+                c.grads[r].zero_()
+            for k in reversed(range(len(numels))):
+                off, n, st = int(c.lay.offsets[k]), int(c.lay.numels[k]), int(starts[k])
+                for r in range(R):
+                    c.grads[r].view(torch.int16)[off:off + n].copy_(dev[r, st:st + n])
+                Z.zero_grads_ready(c.ctx, k, 1, c.grads, c.acc, 0, s)
+            Z.zero_grads_join(c.ctx, s)
+            Z.zero_step_ex(c.ctx, c.hp, c.handle, None, 1.0, 0.0, s)
+
+        graph = _capture(step)
+        for k in range(4):
+            c.step_no += 1
+            g = c.make_grads([(1, 40, 0x7C00)] if k == 1 else None)
+            dev.copy_(torch.from_numpy(g.view(np.int16)))
+            graph.replay()
+            skipped = O.step(c.ostate, g, _ohp(c), c.ofsm)
+            assert skipped == (k == 1 and mode == O.SCALE_DYNAMIC)
+            c.g.check()
+            c.compare()
+    finally:
+        c.close()
