@@ -216,6 +216,14 @@ def profiled_traffic(kernel, workload):
 
 # ---- the workload -------------------------------------------------------------
 
+def workload_label(name, wl, first_tensors=0):
+    """The workload as both arms name it in their `config`."""
+    part = f" (first {first_tensors} tensors)" if first_tensors else ""
+    return (f"{name}{part}: {len(wl['numels'])} tensors, P={sum(wl['numels'])}, R={wl['R']} "
+            f"simulated ranks, {'fp16' if wl['dtype'] else 'bf16'} grads, "
+            f"loss scale mode {wl['mode']}")
+
+
 class Bench:
     def __init__(self, name, path, first_tensors=0, gather_bucket=32 << 20, accum=1, clip=0.0,
                  bucket_elems=None):
@@ -438,11 +446,7 @@ def run_ours(args, world, rank, local):
         "hbm_gbs": step_bytes * K * world / (ms * 1e-3) / 1e9,
         "hbm_frac_of_peak": step_bytes * K / (ms * 1e-3) / 1e9 / peak,
         "config": {
-            "workload": f"{args.workload}"
-                        f"{f' (first {args.first_tensors} tensors)' if args.first_tensors else ''}"
-                        f": {len(b.wl['numels'])} tensors, P={b.P}, R={b.R} "
-                        f"simulated ranks, {'fp16' if b.dtype else 'bf16'} grads, "
-                        f"loss scale mode {b.wl['mode']}",
+            "workload": workload_label(args.workload, b.wl, args.first_tensors),
             "R": b.R, "P": b.P, "T": b.T, "S": b.S, "n_layers": len(b.plan.layers),
             "path": {"pingpong": "fused reduce-scatter+AdamW, ping-pong state",
                      "inplace": "fused reduce-scatter+AdamW, in place",
@@ -882,9 +886,8 @@ def run_reference(args, world, rank):
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": sec * 1e3 / args.steps, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f32", "data": "synthetic",
-        "config": {"workload": f"{args.workload}: {len(wl['numels'])} tensors, "
-                               f"P={sum(wl['numels'])}, R={wl['R']} simulated ranks",
-                   "sample_params_per_step": n},
+        "config": {"workload": workload_label(args.workload, wl), "R": wl["R"],
+                   "P": sum(wl["numels"]), "sample_params_per_step": n},
         "cpu_baseline": {"value": value, "unit": "params/s", "cores": 1, "kind": "oracle",
                          "sample": f"each step the first {n} params of {args.workload}"},
         "e2e": {"value": value, "unit": "params/s", "h2d_bytes_per_step": 0,
