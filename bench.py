@@ -55,7 +55,8 @@ def parse_args(argv=None):
     ap.add_argument("--accum", type=int, default=1,
                     help="micro-batches accumulated per step (two-pass path)")
     ap.add_argument("--clip", type=float, default=0.0,
-                    help="global-norm clipping threshold (> 0: on; two-pass path)")
+                    help="global-norm clipping threshold (> 0: on; fused path for R <= 5, "
+                         "two-pass path otherwise)")
     ap.add_argument("--gather-bucket", type=int, default=32 << 20,
                     help="gather consecutive layers in one launch up to this many elements "
                          "(0: one launch per layer)")
@@ -239,7 +240,7 @@ class Bench:
         self.R, self.dtype = wl["R"], wl["dtype"]
         self.accum, self.clip = accum, clip
         if path == "auto":
-            if accum > 1 or clip > 0:
+            if accum > 1 or (clip > 0 and wl["R"] > 5):
                 path = "twopass"
             else:
                 # ping-pong state measured 2-3 % faster than in place at R = 4 and 8
@@ -247,8 +248,8 @@ class Bench:
                 # fp32 state, which every workload here fits
                 path = "pingpong"
         self.twopass = path.startswith("twopass")
-        if (accum > 1 or clip > 0) and not self.twopass:
-            raise SystemExit("--accum/--clip need the two-pass path")
+        if accum > 1 and not self.twopass:
+            raise SystemExit("--accum needs the two-pass path")
         self.path = path
         self.plan = Z.Plan(wl["numels"], wl["layer_ids"], wl["R"], wl["dtype"], 8,
                            wl["bucket_elems"])
@@ -309,7 +310,9 @@ class Bench:
     def launches_per_step(self):
         n = 1 + (len(self.gather_buckets) if self.gather_buckets else len(self.plan.layers))
         if self.twopass:
-            n += self.accum * len(self.plan.buckets) + (1 if self.clip > 0 else 0)
+            n += self.accum * len(self.plan.buckets)
+        if self.clip > 0:
+            n += 1  # the norm pass
         return n
 
     def step_bytes(self):
@@ -322,6 +325,8 @@ class Bench:
                 main += 4 * T
         else:
             main = (2 * R + 26) * T
+            if self.clip > 0:
+                main += 2 * R * T  # the norm pass over the replicas
         return main + 4 * self.L, main
 
     def step_main(self, stream):
@@ -336,6 +341,8 @@ class Bench:
                                                     stream)
             Z.zero_step_ex(self.ctx, hp, self.state.handle, None, float(self.accum), self.clip,
                            stream)
+        elif self.clip > 0:
+            Z.zero_step_ex(self.ctx, hp, self.state.handle, self.grads, 1.0, self.clip, stream)
         else:
             Z.zero_step(self.ctx, hp, self.state.handle, self.grads, stream)
 
@@ -429,6 +436,8 @@ def run_ours(args, world, rank, local):
     kernel_name = "reduce_scatter+step_from_acc" if b.twopass else "fused_step_kernel"
     if b.twopass and (b.accum > 1 or b.clip > 0):
         kernel_name += f" (accum {b.accum}{', clip' if b.clip > 0 else ''})"
+    elif b.clip > 0:
+        kernel_name = "grad_norm+fused_step_kernel (clip)"
     traffic = profiled_traffic(kernel_name, args.workload)
     out = {
         "metric": METRIC,
@@ -448,8 +457,10 @@ def run_ours(args, world, rank, local):
         "config": {
             "workload": workload_label(args.workload, b.wl, args.first_tensors),
             "R": b.R, "P": b.P, "T": b.T, "S": b.S, "n_layers": len(b.plan.layers),
-            "path": {"pingpong": "fused reduce-scatter+AdamW, ping-pong state",
-                     "inplace": "fused reduce-scatter+AdamW, in place",
+            "path": {"pingpong": f"{'global-norm clip pass, ' if b.clip > 0 else ''}"
+                                 "fused reduce-scatter+AdamW, ping-pong state",
+                     "inplace": f"{'global-norm clip pass, ' if b.clip > 0 else ''}"
+                                "fused reduce-scatter+AdamW, in place",
                      "twopass": f"bucketed reduce-scatter ({b.accum} micro-batch(es)), "
                        f"{'global-norm clip, ' if b.clip > 0 else ''}"
                        "then AdamW from fp32 accumulators, in place",

@@ -322,13 +322,17 @@ zero_status zero_step(zero_ctx_t* ctx, const zero_adamw* hp, const zero_state* s
  *  max_grad_norm (> 0 turns clipping on, 0 = off): with ||g|| the L2 norm of
  *    the unscaled gradient, c = (float) min(1, max_norm / (||g|| + 1e-6)) in
  *    double, and the update uses g * c (one fp32 multiply). Clipping needs
- *    the norm before any element is updated, so it runs on the two-pass path
- *    only (grads == NULL): one extra pass reads the accumulators (4 bytes per
- *    element). The recorded grad_norm_sq is the norm before clipping.
+ *    the norm before any element is updated, so one read-only pass comes
+ *    first: over the accumulators on the two-pass path (4 bytes per
+ *    element), over the R replicas on the fused path (2R bytes per element;
+ *    they are summed in rank order as the step sums them). The fused path
+ *    with clipping moves 4R + 26 bytes per element against 2R + 38 for the
+ *    two-pass path, so it is the cheaper one for R <= 5. The recorded
+ *    grad_norm_sq is the norm before clipping.
  * Defines: not on the pages (clipping and accumulation are common practice
  * around ZeRO training loops, not part of the method the pages describe).
- * Errors: as zero_step, plus ZERO_ERR_INVALID_ARG for a divisor < 1, a
- * negative or non-finite max norm, or clipping with grads != NULL.
+ * Errors: as zero_step, plus ZERO_ERR_INVALID_ARG for a divisor < 1 or a
+ * negative or non-finite max norm.
  */
 typedef struct {
     double grad_divisor;

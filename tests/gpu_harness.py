@@ -169,6 +169,24 @@ class Case:
         self.g.check()
         return skipped
 
+    def step_fused_ex(self, grad_divisor=1.0, max_grad_norm=0.0, inject=None):
+        """Fused step (zero_step_ex with the replicas) with a grad divisor
+        and optional global-norm clipping; inject: (rank, element, bits)."""
+        assert self.path in ("inplace", "pingpong")
+        self.step_no += 1
+        g = self.make_grads(inject)
+        for r in range(self.R):
+            gp = np.zeros(self.plan.T, np.uint16)
+            gp[self.idx] = g[r]
+            self.grads[r].view(torch.int16).copy_(torch.from_numpy(gp.view(np.int16)))
+        Z.zero_step_ex(self.ctx, self.hp, self.handle, self.grads, grad_divisor, max_grad_norm)
+        skipped = O.step_ex(self.ostate, g[None], O.AdamW(**{k: self.hp[k] for k in
+                                                             ("lr", "beta1", "beta2", "eps",
+                                                              "weight_decay")}),
+                            self.ofsm, grad_divisor, max_grad_norm)
+        self.g.check()
+        return skipped
+
     def step_overlap(self, n_micro=1, grad_divisor=1.0, max_grad_norm=0.0, busy=None):
         """Two-pass step whose reduce-scatters are issued by the overlap
         scheduler: each tensor's gradients are written on the caller's stream

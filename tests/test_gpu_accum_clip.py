@@ -53,11 +53,11 @@ def test_overflow_in_one_micro_batch_skips(micro, path):
         c.close()
 
 
-def test_clipping_rejected_on_fused_path_and_bad_options():
+def test_bad_options():
     c = Case([100], 2, O.BF16, 8, O.SCALE_NONE, path="inplace")
     try:
         with pytest.raises(Z.ZeroError) as e:
-            Z.zero_step_ex(c.ctx, c.hp, c.handle, c.grads, 1.0, 1.0)
+            Z.zero_step_ex(c.ctx, c.hp, c.handle, c.grads, 1.0, -1.0)
         assert e.value.status == 1
         with pytest.raises(Z.ZeroError):
             Z.zero_step_ex(c.ctx, c.hp, c.handle, c.grads, 0.5, 0.0)
@@ -65,6 +65,43 @@ def test_clipping_rejected_on_fused_path_and_bad_options():
             Z.zero_reduce_scatter_bucket_ex(c.ctx, 0, c.grads, c.master[0], 4)
         # divisor on the fused path is allowed and matches the oracle
         c.step()
+        c.compare()
+    finally:
+        c.close()
+
+
+@pytest.mark.parametrize("R", [1, 2, 3, 4, 8])
+@pytest.mark.parametrize("dtype", [O.BF16, O.FP16])
+@pytest.mark.parametrize("path", ["inplace", "pingpong"])
+@pytest.mark.parametrize("clip,divisor", [(1e-3, 1.0), (1e9, 1.0), (2e-3, 2.0)])
+def test_fused_clip_matches_oracle(R, dtype, path, clip, divisor):
+    # global-norm clipping on the fused path: a norm pass over the replicas,
+    # then the fused step with the coefficient
+    mode = O.SCALE_DYNAMIC if (dtype == O.FP16 and path == "pingpong") else O.SCALE_NONE
+    c = Case([70_001, 13, 4096, 7, 999], R, dtype, 8, mode, init_scale=256.0, interval=2, path=path,
+             seed=R + 11)
+    try:
+        for _ in range(3):
+            c.step_fused_ex(divisor, clip)
+            c.compare()
+        if clip == 1e-3:
+            assert c.ofsm.grad_norm_sq > 1e-4  # the clip was active
+    finally:
+        c.close()
+
+
+def test_fused_clip_overflow_skips():
+    c = Case([20_000, 33], 2, O.FP16, 8, O.SCALE_DYNAMIC, init_scale=64.0, path="pingpong")
+    try:
+        c.step_fused_ex(1.0, 1e-2)
+        c.compare()
+        before = c.gpu_state()
+        assert c.step_fused_ex(1.0, 1e-2, inject=[(1, 17, 0x7C00)])
+        c.compare()
+        after = c.gpu_state()
+        for k in ("master", "m", "v", "param"):
+            assert np.array_equal(before[k], after[k])
+        c.step_fused_ex(1.0, 1e-2)
         c.compare()
     finally:
         c.close()

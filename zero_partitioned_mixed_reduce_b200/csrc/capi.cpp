@@ -295,10 +295,6 @@ extern "C" zero_status zero_step_ex(zero_ctx_t* ctx, const zero_adamw* hp, const
         !std::isfinite(o.max_grad_norm) || o.reserved[0] != 0 || o.reserved[1] != 0)
         return zb_fail(ZERO_ERR_INVALID_ARG,
                        "zero_step_ex: need grad_divisor >= 1, finite max_grad_norm >= 0, reserved 0");
-    if (o.max_grad_norm > 0.0 && grads != nullptr)
-        return zb_fail(ZERO_ERR_INVALID_ARG,
-                       "zero_step_ex: clipping needs the two-pass path (grads == NULL): the norm must "
-                       "be known before any element is updated");
     if (!ctx || !hp) return zb_fail(ZERO_ERR_INVALID_ARG, "zero_step: NULL ctx or hyper-parameters");
     zero_status s = check_device(ctx, where);
     if (s != ZERO_OK) return s;
@@ -363,7 +359,9 @@ extern "C" zero_status zero_step_ex(zero_ctx_t* ctx, const zero_adamw* hp, const
         p.acc[r] = fused ? nullptr : state->acc[r];
     }
     cudaError_t e = cudaSuccess;
-    if (sp.clip) e = zb::launch_clip_norm(sp, p, cs);
+    // clipping needs the global norm before any element is updated: one
+    // read-only pass over the accumulators, or over the replicas when fused
+    if (sp.clip) e = fused ? zb::launch_grad_norm(sp, p, cs) : zb::launch_clip_norm(sp, p, cs);
     if (e == cudaSuccess)
         e = fused ? zb::launch_fused_step(sp, p, cs) : zb::launch_step_from_acc(sp, p, cs);
     if (e != cudaSuccess) return cuda_fail(where, e);

@@ -177,7 +177,6 @@ __device__ __forceinline__ double block_sum(double x, double* smem) {
     return r;  // valid in thread 0
 }
 
-// Owner of a flat vector index, tracked incrementally along a grid-stride loop.
 // First vector of this thread's grid-stride sequence over [v0, ...): the
 // sequence is laid on 128-byte lines of the half-precision gradients (8
 // vectors of 16 bytes) starting at or below v0, so every warp reads whole
@@ -189,6 +188,7 @@ __device__ __forceinline__ uint32_t line_start(uint32_t v0, uint32_t stride) {
     return v < v0 ? v + stride : v;
 }
 
+// Owner of a flat vector index, tracked incrementally along a grid-stride loop.
 struct OwnerCursor {
     uint32_t o, base, S8;
     __device__ __forceinline__ OwnerCursor(uint32_t v, uint32_t s8) : S8(s8) {

@@ -80,6 +80,7 @@ cudaError_t launch_step_from_acc(const StepParams& sp, const RankPtrs& p, cudaSt
 cudaError_t launch_reduce_scatter(int32_t R, int32_t dtype, int64_t S, int64_t lo, int64_t hi,
                                   DevState* st, const RankPtrs& p, cudaStream_t s,
                                   bool accumulate = false);
+cudaError_t launch_grad_norm(const StepParams& sp, const RankPtrs& p, cudaStream_t s);
 cudaError_t launch_clip_norm(const StepParams& sp, const RankPtrs& p, cudaStream_t s);
 // Loss-scale update from globally reduced totals {sum of g^2, overflow count}.
 cudaError_t launch_fsm_commit(const StepParams& sp, const double* reduced, cudaStream_t s);

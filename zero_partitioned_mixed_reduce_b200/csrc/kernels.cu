@@ -172,7 +172,7 @@ struct FusedArgs {
     uint4* param[2][CAP];
 };
 
-template <typename H, int RC>
+template <typename H, int RC, bool CLIP>
 __global__ void __launch_bounds__(kThreads)
     fused_step_kernel(const __grid_constant__ FusedArgs<RC == 0 ? ZERO_MAX_RANKS : RC> a) {
     const StepParams& sp = a.sp;
@@ -217,7 +217,7 @@ __global__ void __launch_bounds__(kThreads)
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
             bad |= nonfinite(acc[e]);
-            const float g = adamw1(c, acc[e], p.x[e], m.x[e], v.x[e]);
+            const float g = adamw1<CLIP>(c, acc[e], p.x[e], m.x[e], v.x[e]);
             const double gd = static_cast<double>(g);
             nrm = fma(gd, gd, nrm);
             out[e] = p.x[e];
@@ -298,7 +298,7 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
 }
 __device__ __forceinline__ uint4 lds16(const void* p) { return *reinterpret_cast<const uint4*>(p); }
 
-template <typename H, int RC>
+template <typename H, int RC, bool CLIP>
 __global__ void __launch_bounds__(kThreads)
     fused_step_tma_kernel(const __grid_constant__ FusedArgs<RC> a, uint32_t tiles_per_shard) {
     using L = TmaStage<RC>;
@@ -376,7 +376,7 @@ __global__ void __launch_bounds__(kThreads)
 #pragma unroll
             for (int e = 0; e < 8; ++e) {
                 bad |= nonfinite(acc[e]);
-                const double gd = static_cast<double>(adamw1(c, acc[e], p.x[e], m.x[e], v.x[e]));
+                const double gd = static_cast<double>(adamw1<CLIP>(c, acc[e], p.x[e], m.x[e], v.x[e]));
                 nrm = fma(gd, gd, nrm);
                 out[e] = p.x[e];
             }
@@ -461,13 +461,54 @@ __global__ void __launch_bounds__(kThreads) step_from_acc_kernel(const __grid_co
 }
 
 // ---------------------------------------------------------------------------
-// Global gradient norm for clipping, before the two-pass step: one read of
-// the accumulators. The last block to finish turns the sum of squares into
-// the clipping coefficient min(1, max_norm / (||g|| + 1e-6)) (in double) and
-// stores it in the device state for the step kernel.
+// Global gradient norm for clipping, before the step: one read-only pass. The
+// two-pass path reads the accumulators (clip_norm_kernel); the fused path
+// reads the R gradient replicas and reduces them in rank order exactly as the
+// step will (grad_norm_kernel). The last block to finish turns the sum of
+// squares of the unscaled gradient into the clipping coefficient
+// min(1, max_norm / (||g|| + 1e-6)) (in double) and stores it in the device
+// state for the step kernel.
 // ---------------------------------------------------------------------------
 
 constexpr int kNormUnroll = 4;
+
+// 1 / ((R * divisor) * scale), rounded once to fp32; shared by the block.
+__device__ __forceinline__ float block_unscale(const StepParams& sp) {
+    __shared__ float s_inv;
+    if (threadIdx.x == 0) {
+        const volatile DevState* st = sp.st;
+        const double dscale = sp.mode == ZERO_SCALE_NONE ? 1.0 : static_cast<double>(st->scale);
+        s_inv = __double2float_rn(
+            __ddiv_rn(1.0, __dmul_rn(__dmul_rn(static_cast<double>(sp.R), sp.divisor), dscale)));
+    }
+    __syncthreads();
+    return s_inv;
+}
+
+// Every block publishes its partial; the last one stores the coefficient.
+__device__ void norm_to_clip(const StepParams& sp, double nrm) {
+    __shared__ double red[kWarps];
+    __shared__ int last;
+    const double bn = block_sum(nrm, red);
+    if (threadIdx.x == 0) {
+        sp.partials[blockIdx.x] = bn;
+        __threadfence();
+        last = (atomicAdd(&sp.st->done, 1u) == gridDim.x - 1);
+    }
+    __syncthreads();
+    if (!last) return;
+    __threadfence();
+    double x = 0.0;
+    for (unsigned i = threadIdx.x; i < gridDim.x; i += kThreads)
+        x += *reinterpret_cast<volatile double*>(&sp.partials[i]);
+    const double total = block_sum(x, red);
+    if (threadIdx.x == 0) {
+        const double cd = __ddiv_rn(sp.max_norm, __dadd_rn(__dsqrt_rn(total), 1e-6));
+        sp.st->clip = __double2float_rn(cd < 1.0 ? cd : 1.0);
+        sp.st->done = 0u;
+        __threadfence();
+    }
+}
 
 struct NormArgs {
     StepParams sp;
@@ -476,17 +517,7 @@ struct NormArgs {
 
 __global__ void __launch_bounds__(kThreads) clip_norm_kernel(const __grid_constant__ NormArgs a) {
     const StepParams& sp = a.sp;
-    __shared__ float s_inv;
-    __shared__ double red[kWarps];
-    __shared__ int last;
-    if (threadIdx.x == 0) {
-        const volatile DevState* st = sp.st;
-        const double dscale = sp.mode == ZERO_SCALE_NONE ? 1.0 : static_cast<double>(st->scale);
-        s_inv = __double2float_rn(
-            __ddiv_rn(1.0, __dmul_rn(__dmul_rn(static_cast<double>(sp.R), sp.divisor), dscale)));
-    }
-    __syncthreads();
-    const float inv = s_inv;
+    const float inv = block_unscale(sp);
     double nrm = 0.0;
     const uint32_t stride = gridDim.x * kThreads;
     uint32_t vi = blockIdx.x * kThreads + threadIdx.x;
@@ -513,25 +544,48 @@ __global__ void __launch_bounds__(kThreads) clip_norm_kernel(const __grid_consta
                 nrm = fma(gd, gd, nrm);
             }
     }
-    const double bn = block_sum(nrm, red);
-    if (threadIdx.x == 0) {
-        sp.partials[blockIdx.x] = bn;
-        __threadfence();
-        last = (atomicAdd(&sp.st->done, 1u) == gridDim.x - 1);
+    norm_to_clip(sp, nrm);
+}
+
+template <int CAP>
+struct GradNormArgs {
+    StepParams sp;
+    const uint4* g[CAP];
+};
+
+// The norm of the reduced gradient straight from the R half replicas (the
+// fused path has no accumulator): per 8-element vector the replicas are
+// summed in fp32 in rank order, as in the step, then unscaled and squared in
+// double. Gradients only: no state is read.
+template <typename H, int RC>
+__global__ void __launch_bounds__(kThreads)
+    grad_norm_kernel(const __grid_constant__ GradNormArgs<RC == 0 ? ZERO_MAX_RANKS : RC> a) {
+    const StepParams& sp = a.sp;
+    const int R = RC > 0 ? RC : sp.R;
+    const float inv = block_unscale(sp);
+    double nrm = 0.0;
+    const uint32_t stride = gridDim.x * kThreads;
+    for (uint32_t vi = line_start(0, stride); vi < sp.T8; vi += stride) {
+        float acc[8];
+        if constexpr (RC > 0) {
+            uint4 gv[RC];
+#pragma unroll
+            for (int r = 0; r < RC; ++r) gv[r] = ld_grad(a.g[r] + vi);
+            unpack8<H>(gv[0], acc);
+#pragma unroll
+            for (int r = 1; r < RC; ++r) add8<H>(gv[r], acc);
+        } else {
+            unpack8<H>(ld_grad(a.g[0] + vi), acc);
+#pragma unroll 4
+            for (int r = 1; r < R; ++r) add8<H>(ld_grad(a.g[r] + vi), acc);
+        }
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+            const double gd = static_cast<double>(__fmul_rn(acc[e], inv));
+            nrm = fma(gd, gd, nrm);
+        }
     }
-    __syncthreads();
-    if (!last) return;
-    __threadfence();
-    double x = 0.0;
-    for (unsigned i = threadIdx.x; i < gridDim.x; i += kThreads)
-        x += *reinterpret_cast<volatile double*>(&sp.partials[i]);
-    const double total = block_sum(x, red);
-    if (threadIdx.x == 0) {
-        const double cd = __ddiv_rn(sp.max_norm, __dadd_rn(__dsqrt_rn(total), 1e-6));
-        sp.st->clip = __double2float_rn(cd < 1.0 ? cd : 1.0);
-        sp.st->done = 0u;
-        __threadfence();
-    }
+    norm_to_clip(sp, nrm);
 }
 
 // ---------------------------------------------------------------------------
@@ -730,7 +784,7 @@ uint32_t grid_for(uint64_t work_items, int per_sm, int cap) {
     return static_cast<uint32_t>(g > 0 ? g : 1);
 }
 
-template <typename H, int RC>
+template <typename H, int RC, bool CLIP>
 cudaError_t fused_t(const StepParams& sp, const RankPtrs& p, cudaStream_t s) {
     constexpr int CAP = RC == 0 ? ZERO_MAX_RANKS : RC;
     FusedArgs<CAP> a;
@@ -744,13 +798,13 @@ cudaError_t fused_t(const StepParams& sp, const RankPtrs& p, cudaStream_t s) {
             a.param[k][r] = static_cast<uint4*>(p.param[k][r]);
         }
     }
-    static const int per_sm = blocks_per_sm(fused_step_kernel<H, RC>);
+    static const int per_sm = blocks_per_sm(fused_step_kernel<H, RC, CLIP>);
     const uint32_t grid = grid_for(static_cast<uint64_t>(sp.oend - sp.obeg) * sp.S8, per_sm, sp.grid_cap);
-    fused_step_kernel<H, RC><<<grid, kThreads, 0, s>>>(a);
+    fused_step_kernel<H, RC, CLIP><<<grid, kThreads, 0, s>>>(a);
     return cudaGetLastError();
 }
 
-template <typename H, int RC>
+template <typename H, int RC, bool CLIP>
 cudaError_t fused_tma_t(const StepParams& sp, const RankPtrs& p, cudaStream_t s) {
     FusedArgs<RC> a;
     a.sp = sp;
@@ -765,28 +819,29 @@ cudaError_t fused_tma_t(const StepParams& sp, const RankPtrs& p, cudaStream_t s)
     }
     constexpr int smem = TmaStage<RC>::kSmem;
     static const int per_sm = [] {
-        cudaFuncSetAttribute(fused_step_tma_kernel<H, RC>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+        cudaFuncSetAttribute(fused_step_tma_kernel<H, RC, CLIP>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             smem);
         int n = 0;
-        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, fused_step_tma_kernel<H, RC>, kThreads, smem);
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, fused_step_tma_kernel<H, RC, CLIP>, kThreads, smem);
         return n > 0 ? n : 1;
     }();
     const uint32_t S = sp.S8 * 8;
     const uint32_t tiles_per_shard = (S + kTmaTile - 1) / kTmaTile;
     const uint32_t grid = grid_for(static_cast<uint64_t>(tiles_per_shard) * (sp.oend - sp.obeg) * kThreads, per_sm,
                                    sp.grid_cap);
-    fused_step_tma_kernel<H, RC><<<grid, kThreads, smem, s>>>(a, tiles_per_shard);
+    fused_step_tma_kernel<H, RC, CLIP><<<grid, kThreads, smem, s>>>(a, tiles_per_shard);
     return cudaGetLastError();
 }
 
-template <typename H>
+template <typename H, bool CLIP>
 cudaError_t fused_dispatch(const StepParams& sp, const RankPtrs& p, cudaStream_t s) {
     switch (sp.R) {
-        case 1: return fused_tma_t<H, 1>(sp, p, s);
-        case 2: return fused_tma_t<H, 2>(sp, p, s);
-        case 4: return fused_t<H, 4>(sp, p, s);
-        case 8: return fused_t<H, 8>(sp, p, s);
-        case 16: return fused_t<H, 16>(sp, p, s);
-        default: return fused_t<H, 0>(sp, p, s);
+        case 1: return fused_tma_t<H, 1, CLIP>(sp, p, s);
+        case 2: return fused_tma_t<H, 2, CLIP>(sp, p, s);
+        case 4: return fused_t<H, 4, CLIP>(sp, p, s);
+        case 8: return fused_t<H, 8, CLIP>(sp, p, s);
+        case 16: return fused_t<H, 16, CLIP>(sp, p, s);
+        default: return fused_t<H, 0, CLIP>(sp, p, s);
     }
 }
 
@@ -860,7 +915,9 @@ cudaError_t acc_t(const StepParams& sp, const RankPtrs& p, cudaStream_t s) {
 }  // namespace
 
 cudaError_t launch_fused_step(const StepParams& sp, const RankPtrs& p, cudaStream_t s) {
-    return sp.dtype == ZERO_FP16 ? fused_dispatch<Fp16>(sp, p, s) : fused_dispatch<Bf16>(sp, p, s);
+    if (sp.clip)
+        return sp.dtype == ZERO_FP16 ? fused_dispatch<Fp16, true>(sp, p, s) : fused_dispatch<Bf16, true>(sp, p, s);
+    return sp.dtype == ZERO_FP16 ? fused_dispatch<Fp16, false>(sp, p, s) : fused_dispatch<Bf16, false>(sp, p, s);
 }
 
 cudaError_t launch_fsm_commit(const StepParams& sp, const double* reduced, cudaStream_t s) {
@@ -880,6 +937,35 @@ cudaError_t launch_reduce_scatter(int32_t R, int32_t dtype, int64_t S, int64_t l
                                   : rs_dispatch<Bf16, true>(R, S, lo, hi, st, p, s);
     return dtype == ZERO_FP16 ? rs_dispatch<Fp16, false>(R, S, lo, hi, st, p, s)
                               : rs_dispatch<Bf16, false>(R, S, lo, hi, st, p, s);
+}
+
+namespace {
+template <typename H, int RC>
+cudaError_t grad_norm_t(const StepParams& sp, const RankPtrs& p, cudaStream_t s) {
+    GradNormArgs<RC == 0 ? ZERO_MAX_RANKS : RC> a;
+    a.sp = sp;
+    for (int r = 0; r < sp.R; ++r) a.g[r] = static_cast<const uint4*>(p.g[r]);
+    static const int per_sm = blocks_per_sm(grad_norm_kernel<H, RC>);
+    const uint32_t grid = grid_for(sp.T8, per_sm, sp.grid_cap);
+    grad_norm_kernel<H, RC><<<grid, kThreads, 0, s>>>(a);
+    return cudaGetLastError();
+}
+
+template <typename H>
+cudaError_t grad_norm_dispatch(const StepParams& sp, const RankPtrs& p, cudaStream_t s) {
+    switch (sp.R) {
+        case 1: return grad_norm_t<H, 1>(sp, p, s);
+        case 2: return grad_norm_t<H, 2>(sp, p, s);
+        case 4: return grad_norm_t<H, 4>(sp, p, s);
+        case 8: return grad_norm_t<H, 8>(sp, p, s);
+        case 16: return grad_norm_t<H, 16>(sp, p, s);
+        default: return grad_norm_t<H, 0>(sp, p, s);
+    }
+}
+}  // namespace
+
+cudaError_t launch_grad_norm(const StepParams& sp, const RankPtrs& p, cudaStream_t s) {
+    return sp.dtype == ZERO_FP16 ? grad_norm_dispatch<Fp16>(sp, p, s) : grad_norm_dispatch<Bf16>(sp, p, s);
 }
 
 cudaError_t launch_clip_norm(const StepParams& sp, const RankPtrs& p, cudaStream_t s) {
