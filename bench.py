@@ -68,6 +68,9 @@ def parse_args(argv=None):
                     help="override the workload's reduce-scatter bucket size")
     ap.add_argument("--carveout", type=int, default=0,
                     help="SMs kept free of the synthetic GEMMs in --overlap mode")
+    ap.add_argument("--comm-sms", type=int, default=0,
+                    help="SMs the scheduler's communication kernels may fill in --overlap mode "
+                         "(0: all)")
     ap.add_argument("--offload", action="store_true",
                     help="measure ZeRO-Offload (CPU AdamW, with and without the delayed update)")
     ap.add_argument("--rs-sweep", action="store_true",
@@ -686,6 +689,7 @@ def run_overlap(args, world, rank, local):
 
     if args.carveout:
         torch._C._set_sm_carveout_experimental(args.carveout)
+    Z.zero_sched_set_comm_sms(b.ctx, args.comm_sms)
     reps = max(3, min(args.steps, 50))
     # fill the accumulators once; the compute-only variant steps from them
     Z.zero_reduce_scatter_bucket(b.ctx, -1, b.grads, b.state.acc, stream)
@@ -696,7 +700,7 @@ def run_overlap(args, world, rank, local):
     gemm_flops = 6.0 * args.tokens * sum(((hi - lo) // (d * 64)) * (d * 64) for lo, hi in plan.layers)
     out = {"mode": "overlap", "workload": args.workload, "tokens": args.tokens,
            "bucket_elems": wl["bucket_elems"],
-           "gemm_carveout_sms": args.carveout,
+           "gemm_carveout_sms": args.carveout, "comm_kernel_sms": args.comm_sms,
            "gemm_tflops_in_compute_only": gemm_flops / (t_cmp * 1e-3) / 1e12,
            "layers": nl, "buckets": len(plan.buckets), "ring": {"nbufs": nbufs, "depth": depth},
            "ms_overlapped": t_ovl, "ms_serialized": t_ser,

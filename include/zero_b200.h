@@ -487,6 +487,21 @@ zero_status zero_step_noalloc(const zero_plan_t* plan, const zero_loss_scale_con
 /* ------------------------------------------------------------------------ */
 
 /*
+ * zero_sched_set_comm_sms -- cap the kernels that the scheduler launches on
+ * its communication stream (the reduce-scatters of zero_grads_ready, the
+ * gathers of the prefetch ring) at `sms` SMs' worth of resident blocks, so
+ * that they run beside the caller's compute instead of taking every SM a
+ * finishing compute kernel frees; 0 (the default) lets them fill the GPU.
+ * Two launches always get the whole GPU, having no compute to hide behind: a
+ * step's last reduce-scatter bucket and the first gather of a prefetch pass.
+ * The kernels loop over their range with whatever grid they get, so results
+ * do not depend on the setting. Pair it with keeping as many SMs free of the
+ * compute kernels. Defines: [legal] "Communication Overlap" (the reduction
+ * runs while the backward pass continues). Errors: ZERO_ERR_INVALID_ARG.
+ */
+zero_status zero_sched_set_comm_sms(zero_ctx_t* ctx, int32_t sms);
+
+/*
  * zero_grads_ready -- report that tensors [first, first+count) have their
  * gradients written in `grads` by the work queued on `stream` so far. Each
  * bucket whose tensors have then all been reported is reduce-scattered at

@@ -17,5 +17,6 @@ from ._capi import (  # noqa: F401
     zero_reduce_scatter_bucket_ex, zero_step_ex, ZERO_RS_ACCUMULATE,
     zero_step_noalloc, ZERO_NOALLOC_MAX_ELEMS, zero_sync, zero_version, zero_grads_ready,
     zero_grads_join, zero_prefetch_begin, zero_layer_acquire, zero_layer_release, zero_cpu_step,
-    zero_step_shard, zero_step_commit, zero_ctx_reserve_steps, zero_test_drop_tile)
+    zero_step_shard, zero_step_commit, zero_ctx_reserve_steps, zero_test_drop_tile,
+    zero_sched_set_comm_sms)
 from .state import Plan, ShardedState  # noqa: F401

@@ -115,6 +115,7 @@ _sig("zero_step_noalloc", _S, [_P, C.POINTER(zero_loss_scale_config),
                                _PP, _PP, _PP, _P])
 _sig("zero_grads_ready", _S, [_P, C.c_int64, C.c_int64, _PP, _PP, C.c_int32, _P])
 _sig("zero_grads_join", _S, [_P, _P])
+_sig("zero_sched_set_comm_sms", _S, [_P, C.c_int32])
 _sig("zero_prefetch_begin", _S, [_P, C.POINTER(zero_state), _PP, C.c_int32, C.c_int32, C.c_int32, _P])
 _sig("zero_layer_acquire", _S, [_P, C.c_int64, C.POINTER(C.c_void_p), _P])
 _sig("zero_layer_release", _S, [_P, C.c_int64, _P])
@@ -226,6 +227,10 @@ def zero_ctx_destroy(ctx):
 
 def zero_ctx_reserve_steps(ctx, steps, beta1=0.9, beta2=0.999, stream=None):
     _check(_lib.zero_ctx_reserve_steps(ctx, steps, beta1, beta2, _stream(stream)))
+
+
+def zero_sched_set_comm_sms(ctx, sms):
+    _check(_lib.zero_sched_set_comm_sms(ctx, sms))
 
 
 def zero_test_drop_tile(ctx, tile):

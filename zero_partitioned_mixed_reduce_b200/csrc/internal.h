@@ -77,9 +77,12 @@ struct RankPtrs {
 // Kernel launchers (kernels.cu). Each returns the launch's cudaError_t.
 cudaError_t launch_fused_step(const StepParams& sp, const RankPtrs& p, cudaStream_t s);
 cudaError_t launch_step_from_acc(const StepParams& sp, const RankPtrs& p, cudaStream_t s);
+// max_sms > 0 caps the grid at that many SMs' worth of resident blocks (the
+// communication stream's kernels, so that they leave the rest of the GPU to
+// concurrent compute); 0 = the whole GPU.
 cudaError_t launch_reduce_scatter(int32_t R, int32_t dtype, int64_t S, int64_t lo, int64_t hi,
                                   DevState* st, const RankPtrs& p, cudaStream_t s,
-                                  bool accumulate = false);
+                                  bool accumulate = false, int max_sms = 0);
 cudaError_t launch_grad_norm(const StepParams& sp, const RankPtrs& p, cudaStream_t s);
 cudaError_t launch_clip_norm(const StepParams& sp, const RankPtrs& p, cudaStream_t s);
 // Loss-scale update from globally reduced totals {sum of g^2, overflow count}.
@@ -89,7 +92,7 @@ cudaError_t launch_gather(int32_t R, int64_t S, int64_t lo, int64_t hi, const De
 
 cudaError_t launch_gather_many(int32_t R, int64_t S, int nl, const int64_t* lo, const int64_t* hi,
                                const DevState* st, const RankPtrs& p, void* const* outs,
-                               cudaStream_t s);
+                               cudaStream_t s, int max_sms = 0);
 
 // Grid the step kernels use for a given problem (for sizing `partials`).
 int step_grid_cap(int device);

@@ -847,7 +847,7 @@ cudaError_t fused_dispatch(const StepParams& sp, const RankPtrs& p, cudaStream_t
 
 template <typename H, int RC, bool ACCUM>
 cudaError_t rs_t(int32_t R, int64_t S, int64_t lo, int64_t hi, DevState* st, const RankPtrs& p,
-                 cudaStream_t s) {
+                 cudaStream_t s, int max_sms) {
     constexpr int CAP = RC == 0 ? ZERO_MAX_RANKS : RC;
     RsArgs<CAP> a;
     a.lo = lo;
@@ -875,21 +875,21 @@ cudaError_t rs_t(int32_t R, int64_t S, int64_t lo, int64_t hi, DevState* st, con
     static const int per_sm = blocks_per_sm(reduce_scatter_kernel<H, RC, ACCUM>);
     const uint64_t items = static_cast<uint64_t>(a.v1 - a.v0);
     const uint64_t edges = static_cast<uint64_t>((a.head_end - lo) + (hi - a.tail_begin));
-    const uint32_t grid = grid_for(items > edges ? items : edges, per_sm, 0);
+    const uint32_t grid = grid_for(items > edges ? items : edges, per_sm, max_sms * per_sm);
     reduce_scatter_kernel<H, RC, ACCUM><<<grid, kThreads, 0, s>>>(a);
     return cudaGetLastError();
 }
 
 template <typename H, bool ACCUM>
 cudaError_t rs_dispatch(int32_t R, int64_t S, int64_t lo, int64_t hi, DevState* st,
-                        const RankPtrs& p, cudaStream_t s) {
+                        const RankPtrs& p, cudaStream_t s, int max_sms) {
     switch (R) {
-        case 1: return rs_t<H, 1, ACCUM>(R, S, lo, hi, st, p, s);
-        case 2: return rs_t<H, 2, ACCUM>(R, S, lo, hi, st, p, s);
-        case 4: return rs_t<H, 4, ACCUM>(R, S, lo, hi, st, p, s);
-        case 8: return rs_t<H, 8, ACCUM>(R, S, lo, hi, st, p, s);
-        case 16: return rs_t<H, 16, ACCUM>(R, S, lo, hi, st, p, s);
-        default: return rs_t<H, 0, ACCUM>(R, S, lo, hi, st, p, s);
+        case 1: return rs_t<H, 1, ACCUM>(R, S, lo, hi, st, p, s, max_sms);
+        case 2: return rs_t<H, 2, ACCUM>(R, S, lo, hi, st, p, s, max_sms);
+        case 4: return rs_t<H, 4, ACCUM>(R, S, lo, hi, st, p, s, max_sms);
+        case 8: return rs_t<H, 8, ACCUM>(R, S, lo, hi, st, p, s, max_sms);
+        case 16: return rs_t<H, 16, ACCUM>(R, S, lo, hi, st, p, s, max_sms);
+        default: return rs_t<H, 0, ACCUM>(R, S, lo, hi, st, p, s, max_sms);
     }
 }
 
@@ -931,12 +931,13 @@ cudaError_t launch_step_from_acc(const StepParams& sp, const RankPtrs& p, cudaSt
 }
 
 cudaError_t launch_reduce_scatter(int32_t R, int32_t dtype, int64_t S, int64_t lo, int64_t hi,
-                                  DevState* st, const RankPtrs& p, cudaStream_t s, bool accumulate) {
+                                  DevState* st, const RankPtrs& p, cudaStream_t s, bool accumulate,
+                                  int max_sms) {
     if (accumulate)
-        return dtype == ZERO_FP16 ? rs_dispatch<Fp16, true>(R, S, lo, hi, st, p, s)
-                                  : rs_dispatch<Bf16, true>(R, S, lo, hi, st, p, s);
-    return dtype == ZERO_FP16 ? rs_dispatch<Fp16, false>(R, S, lo, hi, st, p, s)
-                              : rs_dispatch<Bf16, false>(R, S, lo, hi, st, p, s);
+        return dtype == ZERO_FP16 ? rs_dispatch<Fp16, true>(R, S, lo, hi, st, p, s, max_sms)
+                                  : rs_dispatch<Bf16, true>(R, S, lo, hi, st, p, s, max_sms);
+    return dtype == ZERO_FP16 ? rs_dispatch<Fp16, false>(R, S, lo, hi, st, p, s, max_sms)
+                              : rs_dispatch<Bf16, false>(R, S, lo, hi, st, p, s, max_sms);
 }
 
 namespace {
@@ -980,7 +981,7 @@ cudaError_t launch_clip_norm(const StepParams& sp, const RankPtrs& p, cudaStream
 
 cudaError_t launch_gather_many(int32_t R, int64_t S, int nl, const int64_t* lo, const int64_t* hi,
                                const DevState* st, const RankPtrs& p, void* const* outs,
-                               cudaStream_t s) {
+                               cudaStream_t s, int max_sms) {
     GatherManyArgs a;
     a.nl = nl;
     a.S = S;
@@ -1001,7 +1002,7 @@ cudaError_t launch_gather_many(int32_t R, int64_t S, int nl, const int64_t* lo, 
     a.total_slots = static_cast<uint32_t>(slots);
     if (slots == 0) return cudaSuccess;
     static const int per_sm = blocks_per_sm(gather_many_kernel);
-    const uint32_t grid = grid_for((slots + kGatherUnroll - 1) / kGatherUnroll, per_sm, 0);
+    const uint32_t grid = grid_for((slots + kGatherUnroll - 1) / kGatherUnroll, per_sm, max_sms * per_sm);
     gather_many_kernel<<<grid, kThreads, 0, s>>>(a);
     return cudaGetLastError();
 }

@@ -21,6 +21,7 @@
 
 struct zero_sched {
     cudaStream_t comm = nullptr;
+    int comm_sms = 0;  // SMs the communication stream's kernels may fill (0 = all)
     // gradient readiness, per step (or micro-batch)
     std::vector<uint8_t> tensor_ready;
     std::vector<int64_t> bucket_ready;
@@ -90,6 +91,16 @@ void zb_sched_destroy(zero_ctx_t* ctx) {
     ctx->sched = nullptr;
 }
 
+extern "C" zero_status zero_sched_set_comm_sms(zero_ctx_t* ctx, int32_t sms) {
+    const char* where = "zero_sched_set_comm_sms";
+    if (!ctx) return zb_fail(ZERO_ERR_INVALID_ARG, "zero_sched_set_comm_sms: ctx is NULL");
+    if (sms < 0) return zb_fail(ZERO_ERR_INVALID_ARG, "zero_sched_set_comm_sms: need sms >= 0");
+    zero_status st = ensure_sched(ctx, where);
+    if (st != ZERO_OK) return st;
+    ctx->sched->comm_sms = sms;
+    return ZERO_OK;
+}
+
 extern "C" zero_status zero_grads_ready(zero_ctx_t* ctx, int64_t first, int64_t count,
                                         const void* const* grads, float* const* acc, int32_t flags,
                                         void* stream) {
@@ -122,12 +133,15 @@ extern "C" zero_status zero_grads_ready(zero_ctx_t* ctx, int64_t first, int64_t 
         s->tensor_ready[k] = 1;
         const int64_t b = ctx->tensor_bucket[k];
         if (++s->bucket_ready[b] != ctx->bucket_ntensors[b]) continue;
+        // the step's last bucket has no compute left to hide behind: whole GPU
+        const bool last_bucket = s->buckets_issued + 1 == static_cast<int64_t>(ctx->bucket_lo.size());
         // the whole bucket is ready: reduce-scatter it behind the caller's work
         cudaError_t e = cudaEventRecord(s->bucket_event[b], cs);
         if (e == cudaSuccess) e = cudaStreamWaitEvent(s->comm, s->bucket_event[b], 0);
         if (e == cudaSuccess)
             e = zb::launch_reduce_scatter(ctx->R, ctx->dtype, ctx->S, ctx->bucket_lo[b], ctx->bucket_hi[b],
-                                          ctx->st, p, s->comm, (flags & ZERO_RS_ACCUMULATE) != 0);
+                                          ctx->st, p, s->comm, (flags & ZERO_RS_ACCUMULATE) != 0,
+                                          last_bucket ? 0 : s->comm_sms);
         if (e != cudaSuccess) return cuda_err(where, e);
         s->buckets_issued += 1;
     }
@@ -222,8 +236,9 @@ zero_status issue_upto(zero_ctx_t* ctx, int64_t upto) {
         const int64_t layer = s->dir > 0 ? pos : nl - 1 - pos;
         void* out = s->bufs[slot];
         if (e == cudaSuccess)
+            // the pass's first gather has nothing before it to hide behind: whole GPU
             e = zb::launch_gather_many(ctx->R, ctx->S, 1, &ctx->layer_lo[layer], &ctx->layer_hi[layer], ctx->st,
-                                       s->params, &out, s->comm);
+                                       s->params, &out, s->comm, pos == 0 ? 0 : s->comm_sms);
         if (e == cudaSuccess) e = cudaEventRecord(s->slot_ready[slot], s->comm);
         if (e != cudaSuccess) return cuda_err("zero_layer_acquire", e);
         s->slot_pos[slot] = pos;
