@@ -30,12 +30,16 @@ def make_busy(n=1024, reps=4):
 
 @pytest.mark.parametrize("R,dtype", [(2, O.FP16), (4, O.BF16), (8, O.FP16)])
 @pytest.mark.parametrize("n_micro", [1, 2])
-def test_overlapped_reduce_scatter_matches_oracle(R, dtype, n_micro):
+@pytest.mark.parametrize("comm_sms", [0, 1, 5])
+def test_overlapped_reduce_scatter_matches_oracle(R, dtype, n_micro, comm_sms):
+    # comm_sms caps the grid of the communication kernels; results must not
+    # depend on it
     numels = [70_001, 13, 4096, 7, 999, 30_000, 5]
     mode = O.SCALE_DYNAMIC if dtype == O.FP16 else O.SCALE_NONE
     c = Case(numels, R, dtype, 8, mode, init_scale=256.0, interval=3, path="twopass",
              bucket_elems=20_000)
     busy = make_busy()
+    Z.zero_sched_set_comm_sms(c.ctx, comm_sms)
     try:
         for _ in range(3):
             c.step_overlap(n_micro, float(n_micro), 0.0 if R != 4 else 0.5, busy)
@@ -66,10 +70,12 @@ def test_grads_join_refuses_missing_and_repeated_reports():
 @pytest.mark.parametrize("direction", [1, -1])
 @pytest.mark.parametrize("nbufs,depth", [(1, 0), (2, 1), (3, 2), (4, 1)])
 @pytest.mark.parametrize("align", [1, 8])
-def test_prefetch_ring_delivers_every_layer(direction, nbufs, depth, align):
+@pytest.mark.parametrize("comm_sms", [0, 2])
+def test_prefetch_ring_delivers_every_layer(direction, nbufs, depth, align, comm_sms):
     numels = [3001, 17, 8, 2048, 5, 700, 1, 9000, 64, 3, 40_000, 11]
     layer_ids = [0, 0, 1, 1, 2, 2, 3, 4, 5, 5, 6, 7]
     c = Case(numels, 4, O.FP16, align, O.SCALE_DYNAMIC, 64.0, path="pingpong", layer_ids=layer_ids)
+    Z.zero_sched_set_comm_sms(c.ctx, comm_sms)
     busy = make_busy(reps=8)
     try:
         for _ in range(2):
