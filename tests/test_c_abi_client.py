@@ -1,8 +1,10 @@
-"""The C ABI used from C: tests/c_abi_client.c is compiled as strict C99
+"""The C ABI used from C. tests/c_abi_client.c is compiled as strict C99
 against include/zero_b200.h, linked against libzero_b200.so and run as a
-separate process. It calls the host-side entry points (plan, plan queries,
-memory accounting, zero_cpu_step, error reporting), and its output is
-checked against the oracle. No GPU is needed."""
+separate process: it calls the host-side entry points (plan, plan queries,
+memory accounting, zero_cpu_step, error reporting) and needs no GPU.
+tests/c_gpu_client.c (GPU tests) runs whole fused steps with buffers from
+cudaMalloc and no PyTorch in the process. Outputs are checked against the
+oracle."""
 import os
 import shutil
 import subprocess
@@ -110,3 +112,68 @@ def test_errors_from_c(client):
         assert err[k][1].startswith("zero_plan")
     version = [r for r in out if r[0] == "version"][0]
     assert "sm_100a" in " ".join(version[1:])
+
+
+@pytest.fixture(scope="module")
+def gpu_client(tmp_path_factory):
+    cuda = os.environ.get("CUDA_HOME", "/usr/local/cuda")
+    exe = str(tmp_path_factory.mktemp("cgpu") / "c_gpu_client")
+    subprocess.run(["gcc", "-std=c99", "-Wall", "-Wextra", "-Werror", "-I", os.path.join(ROOT, "include"),
+                    "-I", os.path.join(cuda, "include"), os.path.join(ROOT, "tests", "c_gpu_client.c"),
+                    "-o", exe, "-L", PKG, "-lzero_b200", "-L", os.path.join(cuda, "lib64"), "-lcudart",
+                    f"-Wl,-rpath,{PKG}", f"-Wl,-rpath,{os.path.join(cuda, 'lib64')}"], check=True)
+    return exe
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("R,dtype,mode", [(4, O.FP16, O.SCALE_DYNAMIC), (2, O.BF16, O.SCALE_NONE),
+                                          (8, O.FP16, O.SCALE_STATIC)])
+def test_gpu_step_from_c_matches_oracle(gpu_client, tmp_path, R, dtype, mode):
+    # the whole GPU step driven from C: cudaMalloc'd buffers, no PyTorch
+    rng = np.random.default_rng(R * 3 + mode)
+    numels = [3001, 17, 4096, 70_001]
+    lay = O.Layout(numels, R, 8)
+    T, P, idx = lay.T, lay.P, lay.flat_index()
+    steps, init, interval = 4, 256.0, 2
+    x = rng.normal(0, 0.02, P).astype(np.float32)
+    st = O.State(x, dtype)
+    fsm = O.make_fsm(mode, scale=init if mode != O.SCALE_NONE else 1.0, interval=interval)
+    hp = O.AdamW(1e-3, 0.9, 0.999, 1e-8, 0.01)
+    master = np.zeros(T, np.float32)
+    master[idx] = x
+    param = np.zeros(T, np.uint16)
+    param[idx] = st.param
+    blobs = [np.array([len(numels), R, dtype, mode, steps, interval], np.int64).tobytes(),
+             np.float32(init).tobytes(), np.array(numels, np.int64).tobytes(), master.tobytes(),
+             param.tobytes()]
+    for s in range(steps):
+        scale = fsm.scale if mode != O.SCALE_NONE else 1.0
+        g = O.float_to_half((rng.normal(0, 1e-2, (R, P)) * scale).astype(np.float32), dtype)
+        if s == 2:
+            g[R - 1, 11] = 0x7C00 if dtype == O.FP16 else 0x7F80
+        gp = np.zeros((R, T), np.uint16)
+        gp[:, idx] = g
+        blobs.append(gp.tobytes())
+        O.step(st, g, hp, fsm)
+    fin, fout = tmp_path / "in.bin", tmp_path / "out.bin"
+    fin.write_bytes(b"".join(blobs))
+    r = subprocess.run([gpu_client, str(fin), str(fout)], capture_output=True, text=True, timeout=300)
+    assert r.returncode == 0, r.stderr
+    raw = fout.read_bytes()
+    scale, cur = np.frombuffer(raw[:8], np.float32)[0], np.frombuffer(raw[4:8], np.int32)[0]
+    good, t = np.frombuffer(raw[8:24], np.int64)
+    last_overflow, last_skipped = np.frombuffer(raw[24:32], np.int32)
+    norm = np.frombuffer(raw[32:40], np.float64)[0]
+    assert (t, good, last_overflow, last_skipped) == (fsm.t, fsm.good, fsm.last_overflow, fsm.last_skipped)
+    assert np.float32(scale) == np.float32(fsm.scale) and cur in (0, 1)
+    assert abs(norm - fsm.grad_norm_sq) <= 1e-9 * abs(fsm.grad_norm_sq) or not np.isfinite(fsm.grad_norm_sq)
+    body = np.frombuffer(raw[40:], np.uint8)
+    f = body[:12 * T].view(np.float32).reshape(3, T)
+    got_param = body[12 * T:].view(np.uint16)
+    for k, want in enumerate((st.master, st.m, st.v)):
+        a = f[k][idx]
+        fin_ = np.isfinite(want)
+        assert np.array_equal(np.isfinite(a), fin_)
+        assert np.array_equal(a[fin_].view(np.uint32), want[fin_].view(np.uint32))
+    nan = O.half_to_float(st.param, dtype) != O.half_to_float(st.param, dtype)
+    assert np.array_equal(got_param[idx][~nan], st.param[~nan])
