@@ -368,6 +368,65 @@ zero_status zero_step_shard(zero_ctx_t* ctx, const zero_adamw* hp, const zero_st
                             double* partial, void* stream);
 
 /*
+ * zero_step_shard_ex -- zero_step_shard with the options of zero_step_ex,
+ * and the two-pass path:
+ *  - grads != NULL: the fused step over the owners' shards, as zero_step_shard;
+ *  - grads == NULL: the step from the owners' accumulators state->acc[o]
+ *    (written by zero_reduce_scatter_shard), from set cur into set 1-cur
+ *    with ping-pong state, else in place. The skip is decided only by
+ *    zero_step_commit, so DYNAMIC mode needs the ping-pong set here too.
+ *  - opts->max_grad_norm > 0: global-norm clipping. Its norm spans every
+ *    rank, so global_norm_sq (device, 1 double) must hold the cross-rank sum
+ *    of the zero_grad_norm_shard partials of this step; the coefficient
+ *    min(1, max_norm / (sqrt(global_norm_sq) + 1e-6)) is formed from it on
+ *    the device. global_norm_sq may be NULL without clipping.
+ * partial and the commit are as for zero_step_shard. Running every owner
+ * range in one process, with the partials summed, gives exactly zero_step_ex.
+ * Defines: [instr] ZeRO-2 "Mechanism"; clipping and accumulation are not on
+ * the pages (see zero_step_ex).
+ * Errors: as zero_step_shard, plus ZERO_ERR_INVALID_ARG for bad options or a
+ * missing global_norm_sq.
+ */
+zero_status zero_step_shard_ex(zero_ctx_t* ctx, const zero_adamw* hp, const zero_state* state,
+                               const void* const* grads, int32_t owner_lo, int32_t owner_hi,
+                               const zero_step_opts* opts, const double* global_norm_sq,
+                               double* partial, void* stream);
+
+/*
+ * zero_reduce_scatter_shard -- zero_reduce_scatter_bucket_ex restricted to
+ * owners [owner_lo, owner_hi): the part of bucket `bucket` (-1: every
+ * element) inside their flat range [owner_lo*S, owner_hi*S) is summed from
+ * all R replicas in rank order into acc[o] (or added to it, with
+ * ZERO_RS_ACCUMULATE), and the context's overflow flag is OR-ed as usual.
+ * This is rank o's part of a multi-GPU bucketed reduce-scatter: grads[r] is
+ * rank r's gradient buffer (peer-mapped; plain loads, no multicast) and only
+ * acc[o] for the owned ranks is touched (other entries may be NULL). A
+ * bucket with no owned element launches nothing.
+ * Defines: [legal] "Reduce-Scatter" and [instr] ZeRO-2 "Communication".
+ * Errors: ZERO_ERR_RANGE (bucket, owner range), ZERO_ERR_INVALID_ARG,
+ * ZERO_ERR_ALIGN, ZERO_ERR_CUDA.
+ */
+zero_status zero_reduce_scatter_shard(zero_ctx_t* ctx, int64_t bucket, const void* const* grads,
+                                      float* const* acc, int32_t owner_lo, int32_t owner_hi,
+                                      int32_t flags, void* stream);
+
+/*
+ * zero_grad_norm_shard -- owners [owner_lo, owner_hi)'s part of the global
+ * gradient norm for clipping: partial[0] = sum over their elements of
+ * (float)(x * inv)^2 in double, inv = (float)(1 / ((R * grad_divisor) *
+ * scale)), where x is the element's reduced gradient read either from the
+ * R replicas (grads != NULL, summed in rank order as the fused step sums
+ * them) or from the owners' accumulators (acc != NULL); partial[1] = 0.
+ * Exactly one of grads and acc is given. The ranks all-reduce partial[0]
+ * (sum) and pass it to zero_step_shard_ex as global_norm_sq.
+ * partial: device, 2 doubles, 8-byte aligned.
+ * Errors: ZERO_ERR_RANGE, ZERO_ERR_INVALID_ARG, ZERO_ERR_ALIGN, ZERO_ERR_CUDA.
+ */
+zero_status zero_grad_norm_shard(zero_ctx_t* ctx, const void* const* grads, float* const* acc,
+                                 double grad_divisor, int32_t owner_lo, int32_t owner_hi,
+                                 double* partial, void* stream);
+
+/*
  * zero_step_commit -- the loss-scale update after zero_step_shard, from
  * totals reduced over every shard: reduced[0] = sum of g^2 (recorded as
  * grad_norm_sq), reduced[1] > 0 means overflow. Skip, backoff, growth, t and

@@ -247,6 +247,60 @@ class Case:
         self.g.check()
         return skipped, [p.cpu().numpy() for p in partials]
 
+    def step_sharded_ex(self, splits, n_micro=1, grad_divisor=1.0, max_grad_norm=0.0, inject=None):
+        """The multi-rank step emulated shard range by shard range, with the
+        cross-rank sums done here: fused (path "pingpong"/"inplace") or
+        two-pass (paths "twopass*": per micro-batch and bucket,
+        zero_reduce_scatter_shard for each range), optional global-norm
+        clipping (zero_grad_norm_shard per range, summed), then
+        zero_step_shard_ex per range and one zero_step_commit.
+        inject: (micro, rank, element, bits)."""
+        self.step_no += 1
+        scale = self.ofsm.scale if self.mode != O.SCALE_NONE else 1.0
+        g = np.stack([np.stack([u16(synth.flat_grads(self.wl, self.step_no * 100 + mu, r, scale, "cpu"))
+                                for r in range(self.R)]) for mu in range(n_micro)])
+        for (mu, r, e, bits) in inject or []:
+            g[mu, r, e] = bits
+        twopass = self.path.startswith("twopass")
+        assert twopass or n_micro == 1
+        dev = lambda: torch.zeros(2, dtype=torch.float64, device="cuda")
+        for mu in range(n_micro):
+            for r in range(self.R):
+                gp = np.zeros(self.plan.T, np.uint16)
+                gp[self.idx] = g[mu, r]
+                self.grads[r].view(torch.int16).copy_(torch.from_numpy(gp.view(np.int16)))
+            if twopass:
+                for lo, hi in splits:
+                    acc = [self.acc[o] if lo <= o < hi else None for o in range(self.R)]
+                    for b in range(len(self.plan.buckets)):
+                        Z.zero_reduce_scatter_shard(self.ctx, b, self.grads, acc, lo, hi,
+                                                    Z.ZERO_RS_ACCUMULATE if mu else 0)
+        norm = None
+        if max_grad_norm > 0:
+            parts = []
+            for lo, hi in splits:
+                part = dev()
+                if twopass:
+                    acc = [self.acc[o] if lo <= o < hi else None for o in range(self.R)]
+                    Z.zero_grad_norm_shard(self.ctx, None, acc, lo, hi, part, grad_divisor)
+                else:
+                    Z.zero_grad_norm_shard(self.ctx, self.grads, None, lo, hi, part, grad_divisor)
+                parts.append(part)
+            norm = torch.stack(parts).sum(0)[:1].contiguous()  # the cross-rank all-reduce
+        partials = []
+        for lo, hi in splits:
+            part = dev()
+            Z.zero_step_shard_ex(self.ctx, self.hp, self.handle, None if twopass else self.grads, lo, hi,
+                                 part, grad_divisor, max_grad_norm, norm)
+            partials.append(part)
+        Z.zero_step_commit(self.ctx, torch.stack(partials).sum(0))
+        skipped = O.step_ex(self.ostate, g, O.AdamW(**{k: self.hp[k] for k in
+                                                       ("lr", "beta1", "beta2", "eps",
+                                                        "weight_decay")}),
+                            self.ofsm, grad_divisor, max_grad_norm)
+        self.g.check()
+        return skipped
+
     def gpu_fsm(self):
         return Z.zero_loss_scale(self.ctx)
 

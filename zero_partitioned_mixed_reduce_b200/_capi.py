@@ -125,6 +125,10 @@ _sig("zero_cpu_step", _S, [_P, C.POINTER(zero_loss_scale_config), C.POINTER(zero
 _sig("zero_step_shard", _S, [_P, C.POINTER(zero_adamw), C.POINTER(zero_state), _PP, C.c_int32,
                              C.c_int32, _P, _P])
 _sig("zero_step_commit", _S, [_P, _P, _P])
+_sig("zero_step_shard_ex", _S, [_P, C.POINTER(zero_adamw), C.POINTER(zero_state), _PP, C.c_int32,
+                                C.c_int32, C.POINTER(zero_step_opts), _P, _P, _P])
+_sig("zero_reduce_scatter_shard", _S, [_P, C.c_int64, _PP, _PP, C.c_int32, C.c_int32, C.c_int32, _P])
+_sig("zero_grad_norm_shard", _S, [_P, _PP, _PP, C.c_double, C.c_int32, C.c_int32, _P, _P])
 _sig("zero_sync", _S, [_P, _P])
 _sig("zero_last_error", C.c_size_t, [C.c_char_p, C.c_size_t])
 _sig("zero_version", C.c_char_p, [])
@@ -409,6 +413,34 @@ def zero_step_shard(ctx, hp, state: StateHandle, grads, owner_lo, owner_hi, part
     g, ga = _ptr_array(grads)
     _check(_lib.zero_step_shard(ctx, C.byref(hp), C.byref(state.c), g, owner_lo, owner_hi,
                                 _addr(partial), _stream(stream)))
+
+
+def zero_step_shard_ex(ctx, hp, state: StateHandle, grads, owner_lo, owner_hi, partial,
+                       grad_divisor=1.0, max_grad_norm=0.0, global_norm_sq=None, stream=None):
+    """Sharded step with options; grads=None steps from state's accumulators.
+    global_norm_sq: device float64 holding the cross-rank norm (clipping)."""
+    if isinstance(hp, dict):
+        hp = zero_adamw(hp["lr"], hp["beta1"], hp["beta2"], hp["eps"], hp["weight_decay"])
+    g = _ptr_array(grads)
+    opts = zero_step_opts(grad_divisor, max_grad_norm)
+    _check(_lib.zero_step_shard_ex(ctx, C.byref(hp), C.byref(state.c), g[0] if g else None, owner_lo,
+                                   owner_hi, C.byref(opts), _addr(global_norm_sq), _addr(partial),
+                                   _stream(stream)))
+
+
+def zero_reduce_scatter_shard(ctx, bucket, grads, acc, owner_lo, owner_hi, flags=0, stream=None):
+    """Bucket `bucket` (-1: all) reduce-scattered into the owners [lo, hi)'s accumulators."""
+    g, ga = _ptr_array(grads)
+    a, aa = _ptr_array(acc)
+    _check(_lib.zero_reduce_scatter_shard(ctx, bucket, g, a, owner_lo, owner_hi, flags, _stream(stream)))
+
+
+def zero_grad_norm_shard(ctx, grads, acc, owner_lo, owner_hi, partial, grad_divisor=1.0, stream=None):
+    """Owners [lo, hi)'s sum of unscaled g^2 into partial[0] (from grads or from acc)."""
+    g = _ptr_array(grads)
+    a = _ptr_array(acc)
+    _check(_lib.zero_grad_norm_shard(ctx, g[0] if g else None, a[0] if a else None, grad_divisor,
+                                     owner_lo, owner_hi, _addr(partial), _stream(stream)))
 
 
 def zero_step_commit(ctx, reduced, stream=None):

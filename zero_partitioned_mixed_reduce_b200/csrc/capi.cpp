@@ -1,6 +1,7 @@
 // C ABI of libzero_b200.so: context lifecycle, argument validation, kernel
 // launches and the loss-scale state. See include/zero_b200.h for the
 // contract of every call.
+#include <algorithm>
 #include <cmath>
 #include <cstring>
 #include <new>
@@ -401,46 +402,18 @@ zero_status check_state_range(const zero_ctx_t* ctx, const zero_state* st, int l
 
 }  // namespace
 
-extern "C" zero_status zero_step_shard(zero_ctx_t* ctx, const zero_adamw* hp, const zero_state* state,
-                                       const void* const* grads, int32_t owner_lo, int32_t owner_hi,
-                                       double* partial, void* stream) {
-    const char* where = "zero_step_shard";
-    if (!ctx || !hp || !grads || !partial)
-        return zb_fail(ZERO_ERR_INVALID_ARG, "zero_step_shard: NULL ctx, hp, grads or partial");
-    zero_status s = check_device(ctx, where);
-    if (s != ZERO_OK) return s;
-    if (owner_lo < 0 || owner_lo >= owner_hi || owner_hi > ctx->R)
-        return zb_fail(ZERO_ERR_RANGE, "zero_step_shard: need 0 <= owner_lo < owner_hi <= R");
-    if (!aligned(partial, 8)) return zb_fail(ZERO_ERR_ALIGN, "zero_step_shard: partial not 8-byte aligned");
-    if (!(hp->lr >= 0.0) || !(hp->beta1 >= 0.0 && hp->beta1 < 1.0) || !(hp->beta2 >= 0.0 && hp->beta2 < 1.0) ||
-        !(hp->eps > 0.0) || !(hp->weight_decay >= 0.0))
-        return zb_fail(ZERO_ERR_INVALID_ARG, "zero_step_shard: bad hyper-parameters");
-    int sets = 1;
-    if ((s = check_state_range(ctx, state, owner_lo, owner_hi, where, &sets)) != ZERO_OK) return s;
-    for (int r = 0; r < ctx->R; ++r) {
-        if (!grads[r]) return zb_fail(ZERO_ERR_INVALID_ARG, "zero_step_shard: grads[" + std::to_string(r) + "] is NULL");
-        if (!aligned(grads[r], 16)) return zb_fail(ZERO_ERR_ALIGN, "zero_step_shard: grads misaligned");
-    }
-    if (sets == 1 && ctx->cfg.mode == ZERO_SCALE_DYNAMIC)
-        return zb_fail(ZERO_ERR_INVALID_ARG, "zero_step_shard: dynamic loss scaling needs state set 1 (ping-pong)");
-    if (sets == 1 && ctx->two_sets)
-        return zb_fail(ZERO_ERR_STATE, "zero_step_shard: the current model may live in state set 1");
-    cudaStream_t cs = static_cast<cudaStream_t>(stream);
-    if ((s = ensure_powtab(ctx, hp->beta1, hp->beta2, ctx->t_bound + 1, cs)) != ZERO_OK) return s;
+namespace {
+
+// Parameters shared by the sharded calls (everything but the AdamW hyper-parameters).
+zb::StepParams shard_params(const zero_ctx_t* ctx, int32_t owner_lo, int32_t owner_hi, double divisor,
+                            double* partial) {
     zb::StepParams sp;
     sp.R = ctx->R;
     sp.dtype = ctx->dtype;
     sp.mode = ctx->cfg.mode;
-    sp.pingpong = sets == 2 ? 1 : 0;
     sp.S8 = static_cast<uint32_t>(ctx->S / 8);
     sp.T8 = static_cast<uint32_t>(ctx->T / 8);
-    sp.dec = static_cast<float>(1.0 - hp->lr * hp->weight_decay);
-    sp.b1f = static_cast<float>(hp->beta1);
-    sp.omb1 = static_cast<float>(1.0 - hp->beta1);
-    sp.b2f = static_cast<float>(hp->beta2);
-    sp.omb2 = static_cast<float>(1.0 - hp->beta2);
-    sp.epsf = static_cast<float>(hp->eps);
-    sp.lr = hp->lr;
+    sp.divisor = divisor;
     sp.interval = ctx->cfg.growth_interval;
     sp.growth = ctx->cfg.growth_factor;
     sp.backoff = ctx->cfg.backoff_factor;
@@ -453,26 +426,180 @@ extern "C" zero_status zero_step_shard(zero_ctx_t* ctx, const zero_adamw* hp, co
     sp.obeg = owner_lo;
     sp.oend = owner_hi;
     sp.partial_out = partial;
-    sp.drop_tile = ctx->drop_tile;
+    return sp;
+}
+
+zero_status check_owner_range(const zero_ctx_t* ctx, int32_t lo, int32_t hi, const char* where) {
+    if (lo < 0 || lo >= hi || hi > ctx->R)
+        return zb_fail(ZERO_ERR_RANGE, std::string(where) + ": need 0 <= owner_lo < owner_hi <= R");
+    return ZERO_OK;
+}
+
+zero_status check_all_grads(const zero_ctx_t* ctx, const void* const* grads, const char* where) {
+    for (int r = 0; r < ctx->R; ++r) {
+        if (!grads[r]) return zb_fail(ZERO_ERR_INVALID_ARG, std::string(where) + ": grads[" + std::to_string(r) + "] is NULL");
+        if (!aligned(grads[r], 16)) return zb_fail(ZERO_ERR_ALIGN, std::string(where) + ": grads misaligned");
+    }
+    return ZERO_OK;
+}
+
+zero_status check_owned_acc(const zero_ctx_t* ctx, float* const* acc, int32_t lo, int32_t hi, const char* where) {
+    if (!acc) return zb_fail(ZERO_ERR_INVALID_ARG, std::string(where) + ": acc is NULL");
+    for (int r = lo; r < hi; ++r) {
+        if (!acc[r]) return zb_fail(ZERO_ERR_INVALID_ARG, std::string(where) + ": acc[" + std::to_string(r) + "] is NULL");
+        if (!aligned(acc[r], 32)) return zb_fail(ZERO_ERR_ALIGN, std::string(where) + ": acc misaligned");
+    }
+    (void)ctx;
+    return ZERO_OK;
+}
+
+}  // namespace
+
+extern "C" zero_status zero_reduce_scatter_shard(zero_ctx_t* ctx, int64_t bucket, const void* const* grads,
+                                                 float* const* acc, int32_t owner_lo, int32_t owner_hi,
+                                                 int32_t flags, void* stream) {
+    const char* where = "zero_reduce_scatter_shard";
+    if (!ctx || !grads) return zb_fail(ZERO_ERR_INVALID_ARG, "zero_reduce_scatter_shard: NULL ctx or grads");
+    if (flags & ~ZERO_RS_ACCUMULATE) return zb_fail(ZERO_ERR_INVALID_ARG, "zero_reduce_scatter_shard: unknown flags");
+    zero_status s = check_device(ctx, where);
+    if (s != ZERO_OK) return s;
+    if ((s = check_owner_range(ctx, owner_lo, owner_hi, where)) != ZERO_OK) return s;
+    int64_t lo, hi;
+    if (bucket == -1) {
+        lo = 0;
+        hi = ctx->T;
+    } else if (bucket < 0 || bucket >= static_cast<int64_t>(ctx->bucket_lo.size())) {
+        return zb_fail(ZERO_ERR_RANGE, "zero_reduce_scatter_shard: bucket index out of range");
+    } else {
+        lo = ctx->bucket_lo[bucket];
+        hi = ctx->bucket_hi[bucket];
+    }
+    if ((s = check_all_grads(ctx, grads, where)) != ZERO_OK) return s;
+    if ((s = check_owned_acc(ctx, acc, owner_lo, owner_hi, where)) != ZERO_OK) return s;
+    // the bucket's part inside the owners' flat range [owner_lo * S, owner_hi * S)
+    lo = std::max<int64_t>(lo, static_cast<int64_t>(owner_lo) * ctx->S);
+    hi = std::min<int64_t>(hi, static_cast<int64_t>(owner_hi) * ctx->S);
+    if (lo >= hi) return ZERO_OK;  // no element of this bucket is owned here
     zb::RankPtrs p{};
     for (int r = 0; r < ctx->R; ++r) {
         p.g[r] = grads[r];
+        p.acc[r] = (r >= owner_lo && r < owner_hi) ? acc[r] : nullptr;
+    }
+    cudaError_t e = zb::launch_reduce_scatter(ctx->R, ctx->dtype, ctx->S, lo, hi, ctx->st, p,
+                                              static_cast<cudaStream_t>(stream), (flags & ZERO_RS_ACCUMULATE) != 0);
+    if (e != cudaSuccess) return cuda_fail(where, e);
+    return ZERO_OK;
+}
+
+extern "C" zero_status zero_grad_norm_shard(zero_ctx_t* ctx, const void* const* grads, float* const* acc,
+                                            double grad_divisor, int32_t owner_lo, int32_t owner_hi,
+                                            double* partial, void* stream) {
+    const char* where = "zero_grad_norm_shard";
+    if (!ctx || !partial) return zb_fail(ZERO_ERR_INVALID_ARG, "zero_grad_norm_shard: NULL ctx or partial");
+    if ((grads == nullptr) == (acc == nullptr))
+        return zb_fail(ZERO_ERR_INVALID_ARG, "zero_grad_norm_shard: give exactly one of grads and acc");
+    if (!(grad_divisor >= 1.0) || !std::isfinite(grad_divisor))
+        return zb_fail(ZERO_ERR_INVALID_ARG, "zero_grad_norm_shard: need a finite grad_divisor >= 1");
+    zero_status s = check_device(ctx, where);
+    if (s != ZERO_OK) return s;
+    if ((s = check_owner_range(ctx, owner_lo, owner_hi, where)) != ZERO_OK) return s;
+    if (!aligned(partial, 8)) return zb_fail(ZERO_ERR_ALIGN, "zero_grad_norm_shard: partial not 8-byte aligned");
+    if (grads && (s = check_all_grads(ctx, grads, where)) != ZERO_OK) return s;
+    if (acc && (s = check_owned_acc(ctx, acc, owner_lo, owner_hi, where)) != ZERO_OK) return s;
+    zb::StepParams sp = shard_params(ctx, owner_lo, owner_hi, grad_divisor, partial);
+    zb::RankPtrs p{};
+    for (int r = 0; r < ctx->R; ++r) {
+        p.g[r] = grads ? grads[r] : nullptr;
+        p.acc[r] = (acc && r >= owner_lo && r < owner_hi) ? acc[r] : nullptr;
+    }
+    cudaStream_t cs = static_cast<cudaStream_t>(stream);
+    cudaError_t e = grads ? zb::launch_grad_norm(sp, p, cs) : zb::launch_clip_norm(sp, p, cs);
+    if (e != cudaSuccess) return cuda_fail(where, e);
+    return ZERO_OK;
+}
+
+extern "C" zero_status zero_step_shard_ex(zero_ctx_t* ctx, const zero_adamw* hp, const zero_state* state,
+                                          const void* const* grads, int32_t owner_lo, int32_t owner_hi,
+                                          const zero_step_opts* opts, const double* global_norm_sq,
+                                          double* partial, void* stream) {
+    const char* where = "zero_step_shard";
+    if (!ctx || !hp || !partial)
+        return zb_fail(ZERO_ERR_INVALID_ARG, "zero_step_shard: NULL ctx, hp or partial");
+    zero_step_opts o{1.0, 0.0, {0, 0}};
+    if (opts) o = *opts;
+    if (!(o.grad_divisor >= 1.0) || !std::isfinite(o.grad_divisor) || !(o.max_grad_norm >= 0.0) ||
+        !std::isfinite(o.max_grad_norm) || o.reserved[0] != 0 || o.reserved[1] != 0)
+        return zb_fail(ZERO_ERR_INVALID_ARG,
+                       "zero_step_shard: need grad_divisor >= 1, finite max_grad_norm >= 0, reserved 0");
+    const bool clip = o.max_grad_norm > 0.0;
+    if (clip && !global_norm_sq)
+        return zb_fail(ZERO_ERR_INVALID_ARG,
+                       "zero_step_shard: clipping needs global_norm_sq (the cross-rank sum of the "
+                       "zero_grad_norm_shard partials)");
+    if (global_norm_sq && !aligned(global_norm_sq, 8))
+        return zb_fail(ZERO_ERR_ALIGN, "zero_step_shard: global_norm_sq not 8-byte aligned");
+    zero_status s = check_device(ctx, where);
+    if (s != ZERO_OK) return s;
+    if ((s = check_owner_range(ctx, owner_lo, owner_hi, where)) != ZERO_OK) return s;
+    if (!aligned(partial, 8)) return zb_fail(ZERO_ERR_ALIGN, "zero_step_shard: partial not 8-byte aligned");
+    if (!(hp->lr >= 0.0) || !(hp->beta1 >= 0.0 && hp->beta1 < 1.0) || !(hp->beta2 >= 0.0 && hp->beta2 < 1.0) ||
+        !(hp->eps > 0.0) || !(hp->weight_decay >= 0.0))
+        return zb_fail(ZERO_ERR_INVALID_ARG, "zero_step_shard: bad hyper-parameters");
+    int sets = 1;
+    if ((s = check_state_range(ctx, state, owner_lo, owner_hi, where, &sets)) != ZERO_OK) return s;
+    const bool fused = grads != nullptr;
+    if (fused) {
+        if ((s = check_all_grads(ctx, grads, where)) != ZERO_OK) return s;
+    } else if ((s = check_owned_acc(ctx, state->acc, owner_lo, owner_hi, where)) != ZERO_OK) {
+        return s;
+    }
+    if (sets == 1 && ctx->cfg.mode == ZERO_SCALE_DYNAMIC)
+        return zb_fail(ZERO_ERR_INVALID_ARG, "zero_step_shard: dynamic loss scaling needs state set 1 (ping-pong)");
+    if (sets == 1 && ctx->two_sets)
+        return zb_fail(ZERO_ERR_STATE, "zero_step_shard: the current model may live in state set 1");
+    cudaStream_t cs = static_cast<cudaStream_t>(stream);
+    if ((s = ensure_powtab(ctx, hp->beta1, hp->beta2, ctx->t_bound + 1, cs)) != ZERO_OK) return s;
+    zb::StepParams sp = shard_params(ctx, owner_lo, owner_hi, o.grad_divisor, partial);
+    sp.pingpong = sets == 2 ? 1 : 0;
+    sp.dec = static_cast<float>(1.0 - hp->lr * hp->weight_decay);
+    sp.b1f = static_cast<float>(hp->beta1);
+    sp.omb1 = static_cast<float>(1.0 - hp->beta1);
+    sp.b2f = static_cast<float>(hp->beta2);
+    sp.omb2 = static_cast<float>(1.0 - hp->beta2);
+    sp.epsf = static_cast<float>(hp->eps);
+    sp.lr = hp->lr;
+    sp.max_norm = o.max_grad_norm;
+    sp.clip = clip ? 1 : 0;
+    if (fused) sp.drop_tile = ctx->drop_tile;
+    zb::RankPtrs p{};
+    for (int r = 0; r < ctx->R; ++r) {
+        const bool owned = r >= owner_lo && r < owner_hi;
+        p.g[r] = fused ? grads[r] : nullptr;
+        p.acc[r] = (!fused && owned) ? state->acc[r] : nullptr;
         for (int k = 0; k < 2; ++k) {
             const int from = k < sets ? k : 0;
-            const bool owned = r >= owner_lo && r < owner_hi;
             p.master[k][r] = owned ? state->master[from][r] : nullptr;
             p.m[k][r] = owned ? state->m[from][r] : nullptr;
             p.v[k][r] = owned ? state->v[from][r] : nullptr;
             p.param[k][r] = owned ? state->param[from][r] : nullptr;
         }
     }
-    cudaError_t e = zb::launch_fused_step(sp, p, cs);
+    cudaError_t e = cudaSuccess;
+    if (clip) e = zb::launch_clip_from_norm(sp, global_norm_sq, cs);
+    if (e == cudaSuccess) e = fused ? zb::launch_fused_step(sp, p, cs) : zb::launch_step_from_acc(sp, p, cs);
     if (e != cudaSuccess) return cuda_fail(where, e);
     ctx->t_bound += 1;
-    ctx->drop_tile = 0xffffffffu;
+    if (fused) ctx->drop_tile = 0xffffffffu;
     ctx->shard_pingpong = sp.pingpong;
     if (sp.pingpong) ctx->two_sets = true;
     return ZERO_OK;
+}
+
+extern "C" zero_status zero_step_shard(zero_ctx_t* ctx, const zero_adamw* hp, const zero_state* state,
+                                       const void* const* grads, int32_t owner_lo, int32_t owner_hi,
+                                       double* partial, void* stream) {
+    if (!grads) return zb_fail(ZERO_ERR_INVALID_ARG, "zero_step_shard: grads is NULL (use zero_step_shard_ex)");
+    return zero_step_shard_ex(ctx, hp, state, grads, owner_lo, owner_hi, nullptr, nullptr, partial, stream);
 }
 
 extern "C" zero_status zero_step_commit(zero_ctx_t* ctx, const double* reduced, void* stream) {

@@ -45,7 +45,7 @@ struct StepParams {
     float dec = 0, b1f = 0, omb1 = 0, b2f = 0, omb2 = 0, epsf = 0;
     double lr = 0;
     double divisor = 1;       // grad divisor k: unscale by 1 / ((R * k) * scale)
-    double max_norm = 0;      // > 0: clipping on (two-pass path)
+    double max_norm = 0;      // > 0: clipping on
     int32_t clip = 0;
     int64_t interval = 1;
     float growth = 2, backoff = 0.5f, min_scale = 1;
@@ -54,7 +54,7 @@ struct StepParams {
     const double2* powtab = nullptr;  // powtab[t] = (beta1^t, beta2^t)
     int64_t powtab_len = 0;
     int grid_cap = 0;  // capacity of `partials`
-    // fused step over shards [obeg, oend) only (default: all R)
+    // step or norm pass over shards [obeg, oend) only (default: all R)
     int32_t obeg = 0, oend = 0;
     // non-null: the step's last block writes {sum of g^2, overflow 0/1} here and
     // leaves the loss-scale update to a later commit (sharded multi-rank step)
@@ -83,7 +83,10 @@ cudaError_t launch_step_from_acc(const StepParams& sp, const RankPtrs& p, cudaSt
 cudaError_t launch_reduce_scatter(int32_t R, int32_t dtype, int64_t S, int64_t lo, int64_t hi,
                                   DevState* st, const RankPtrs& p, cudaStream_t s,
                                   bool accumulate = false, int max_sms = 0);
+// Norm passes over owners [obeg, oend): the last block stores the clipping
+// coefficient, or, with partial_out, the range's sum of g^2 in partial_out[0].
 cudaError_t launch_grad_norm(const StepParams& sp, const RankPtrs& p, cudaStream_t s);
+cudaError_t launch_clip_from_norm(const StepParams& sp, const double* norm_sq, cudaStream_t s);
 cudaError_t launch_clip_norm(const StepParams& sp, const RankPtrs& p, cudaStream_t s);
 // Loss-scale update from globally reduced totals {sum of g^2, overflow count}.
 cudaError_t launch_fsm_commit(const StepParams& sp, const double* reduced, cudaStream_t s);

@@ -419,16 +419,19 @@ template <typename H, bool CLIP>
 __global__ void __launch_bounds__(kThreads) step_from_acc_kernel(const __grid_constant__ AccArgs a) {
     const StepParams& sp = a.sp;
     __shared__ Prologue pro;
-    read_prologue(sp, sp.R, &pro, true);
+    // a sharded step (partial_out) defers the skip to the cross-rank commit:
+    // it always writes set 1-cur, and only the commit decides whether cur flips
+    read_prologue(sp, sp.R, &pro, sp.partial_out == nullptr);
     const Coef c = pro.c;
     const int src = pro.src, dst = pro.dst;
     const bool skip = pro.skip != 0;
 
     double nrm = 0.0;
     const uint32_t stride = gridDim.x * kThreads;
-    uint32_t vi = blockIdx.x * kThreads + threadIdx.x;
+    const uint32_t vend = static_cast<uint32_t>(sp.oend) * sp.S8;
+    uint32_t vi = line_start(static_cast<uint32_t>(sp.obeg) * sp.S8, stride);
     OwnerCursor oc(vi, sp.S8);
-    for (; vi < sp.T8; vi += stride) {
+    for (; vi < vend; vi += stride) {
         oc.seek(vi);
         const uint32_t o = oc.o;
         const size_t j8 = static_cast<size_t>(vi - oc.base) * 8;
@@ -485,7 +488,14 @@ __device__ __forceinline__ float block_unscale(const StepParams& sp) {
     return s_inv;
 }
 
-// Every block publishes its partial; the last one stores the coefficient.
+// min(1, max_norm / (sqrt(norm_sq) + 1e-6)), in double, rounded once to fp32.
+__device__ __forceinline__ float clip_coefficient(double max_norm, double norm_sq) {
+    const double cd = __ddiv_rn(max_norm, __dadd_rn(__dsqrt_rn(norm_sq), 1e-6));
+    return __double2float_rn(cd < 1.0 ? cd : 1.0);
+}
+
+// Every block publishes its partial; the last one stores the coefficient, or,
+// for a shard range (partial_out), the range's sum for a cross-rank reduction.
 __device__ void norm_to_clip(const StepParams& sp, double nrm) {
     __shared__ double red[kWarps];
     __shared__ int last;
@@ -503,9 +513,22 @@ __device__ void norm_to_clip(const StepParams& sp, double nrm) {
         x += *reinterpret_cast<volatile double*>(&sp.partials[i]);
     const double total = block_sum(x, red);
     if (threadIdx.x == 0) {
-        const double cd = __ddiv_rn(sp.max_norm, __dadd_rn(__dsqrt_rn(total), 1e-6));
-        sp.st->clip = __double2float_rn(cd < 1.0 ? cd : 1.0);
+        if (sp.partial_out) {
+            // a shard range's part of the norm, for a cross-rank sum
+            sp.partial_out[0] = total;
+            sp.partial_out[1] = 0.0;
+        } else {
+            sp.st->clip = clip_coefficient(sp.max_norm, total);
+        }
         sp.st->done = 0u;
+        __threadfence();
+    }
+}
+
+// The coefficient from a norm already summed across ranks.
+__global__ void clip_from_norm_kernel(const __grid_constant__ StepParams sp, const double* norm_sq) {
+    if (threadIdx.x == 0 && blockIdx.x == 0) {
+        sp.st->clip = clip_coefficient(sp.max_norm, *norm_sq);
         __threadfence();
     }
 }
@@ -520,15 +543,16 @@ __global__ void __launch_bounds__(kThreads) clip_norm_kernel(const __grid_consta
     const float inv = block_unscale(sp);
     double nrm = 0.0;
     const uint32_t stride = gridDim.x * kThreads;
-    uint32_t vi = blockIdx.x * kThreads + threadIdx.x;
+    const uint32_t vend = static_cast<uint32_t>(sp.oend) * sp.S8;
+    uint32_t vi = line_start(static_cast<uint32_t>(sp.obeg) * sp.S8, stride);
     OwnerCursor oc(vi, sp.S8);
     // a short read-only pass: keep kNormUnroll vectors per thread in flight
-    for (; vi < sp.T8; vi += kNormUnroll * stride) {
+    for (; vi < vend; vi += kNormUnroll * stride) {
         F8 acc[kNormUnroll];
 #pragma unroll
         for (int u = 0; u < kNormUnroll; ++u) {
             const uint32_t vu = vi + u * stride;
-            if (vu < sp.T8) {
+            if (vu < vend) {
                 oc.seek(vu);
                 acc[u] = ld_f8(a.acc[oc.o] + static_cast<size_t>(vu - oc.base) * 8);
             } else {
@@ -565,7 +589,8 @@ __global__ void __launch_bounds__(kThreads)
     const float inv = block_unscale(sp);
     double nrm = 0.0;
     const uint32_t stride = gridDim.x * kThreads;
-    for (uint32_t vi = line_start(0, stride); vi < sp.T8; vi += stride) {
+    const uint32_t vend = static_cast<uint32_t>(sp.oend) * sp.S8;
+    for (uint32_t vi = line_start(static_cast<uint32_t>(sp.obeg) * sp.S8, stride); vi < vend; vi += stride) {
         float acc[8];
         if constexpr (RC > 0) {
             uint4 gv[RC];
@@ -907,7 +932,7 @@ cudaError_t acc_t(const StepParams& sp, const RankPtrs& p, cudaStream_t s) {
         }
     }
     static const int per_sm = blocks_per_sm(step_from_acc_kernel<H, CLIP>);
-    const uint32_t grid = grid_for(sp.T8, per_sm, sp.grid_cap);
+    const uint32_t grid = grid_for(static_cast<uint64_t>(sp.oend - sp.obeg) * sp.S8, per_sm, sp.grid_cap);
     step_from_acc_kernel<H, CLIP><<<grid, kThreads, 0, s>>>(a);
     return cudaGetLastError();
 }
@@ -947,7 +972,7 @@ cudaError_t grad_norm_t(const StepParams& sp, const RankPtrs& p, cudaStream_t s)
     a.sp = sp;
     for (int r = 0; r < sp.R; ++r) a.g[r] = static_cast<const uint4*>(p.g[r]);
     static const int per_sm = blocks_per_sm(grad_norm_kernel<H, RC>);
-    const uint32_t grid = grid_for(sp.T8, per_sm, sp.grid_cap);
+    const uint32_t grid = grid_for(static_cast<uint64_t>(sp.oend - sp.obeg) * sp.S8, per_sm, sp.grid_cap);
     grad_norm_kernel<H, RC><<<grid, kThreads, 0, s>>>(a);
     return cudaGetLastError();
 }
@@ -965,6 +990,11 @@ cudaError_t grad_norm_dispatch(const StepParams& sp, const RankPtrs& p, cudaStre
 }
 }  // namespace
 
+cudaError_t launch_clip_from_norm(const StepParams& sp, const double* norm_sq, cudaStream_t s) {
+    clip_from_norm_kernel<<<1, 32, 0, s>>>(sp, norm_sq);
+    return cudaGetLastError();
+}
+
 cudaError_t launch_grad_norm(const StepParams& sp, const RankPtrs& p, cudaStream_t s) {
     return sp.dtype == ZERO_FP16 ? grad_norm_dispatch<Fp16>(sp, p, s) : grad_norm_dispatch<Bf16>(sp, p, s);
 }
@@ -974,7 +1004,7 @@ cudaError_t launch_clip_norm(const StepParams& sp, const RankPtrs& p, cudaStream
     a.sp = sp;
     for (int r = 0; r < sp.R; ++r) a.acc[r] = p.acc[r];
     static const int per_sm = blocks_per_sm(clip_norm_kernel);
-    const uint32_t grid = grid_for(sp.T8, per_sm, sp.grid_cap);
+    const uint32_t grid = grid_for(static_cast<uint64_t>(sp.oend - sp.obeg) * sp.S8, per_sm, sp.grid_cap);
     clip_norm_kernel<<<grid, kThreads, 0, s>>>(a);
     return cudaGetLastError();
 }
