@@ -63,10 +63,59 @@ def main():
         torch.cuda.synchronize()
         assert np.array_equal(u16(out), pflat[lo:hi]), l
     dz.close()
+    check_accumulate_and_clip(rank, world)
     dist.barrier()
     dist.destroy_process_group()
     if rank == 0:
         print("ok")
+
+
+def check_accumulate_and_clip(rank, world):
+    """Two-pass steps over accumulated micro-batches and fused steps, with
+    global-norm clipping, against the oracle's step_ex."""
+    numels = [50_001, 77, 3000]
+    dz = DistributedZero(numels, None, Z.ZERO_BF16, Z.ZERO_SCALE_NONE, accumulate=True)
+    wl = synth.custom_workload(numels, world, Z.ZERO_BF16, Z.ZERO_SCALE_NONE, 1.0, 1000, sigma=1e-2,
+                               index=56)
+    lay = O.Layout(numels, world, 8)
+    idx = lay.flat_index()
+    x = synth.flat_master(wl, "cpu")
+    p0 = x.to(torch.bfloat16)
+    dz.load(dz.plan.pack(x.cuda()), dz.plan.pack(p0.cuda()))
+    ost = O.State(x.numpy(), O.BF16, u16(p0))
+    fsm = O.make_fsm(O.SCALE_NONE)
+    hp = wl["hp"]
+    ohp = O.AdamW(*(hp[k] for k in ("lr", "beta1", "beta2", "eps", "weight_decay")))
+    S = dz.plan.S
+
+    def write(g):
+        gp = np.zeros(dz.plan.T, np.uint16)
+        gp[idx] = g[rank]
+        dz.grads.view(torch.int16).copy_(torch.from_numpy(gp.view(np.int16)))
+
+    for step in range(1, 5):
+        clip = 1e-3 if step % 2 else 0.0
+        if step <= 2:  # two micro-batches, accumulated
+            micro = [np.stack([u16(synth.flat_grads(wl, step * 10 + mu, r, 1.0, "cpu")) for r in range(world)])
+                     for mu in range(2)]
+            for g in micro:
+                write(g)
+                dz.reduce_scatter()
+            dz.step_accumulated(hp, max_grad_norm=clip)
+            O.step_ex(ost, np.stack(micro), ohp, fsm, 2.0, clip)
+        else:  # fused
+            g = np.stack([u16(synth.flat_grads(wl, step * 10, r, 1.0, "cpu")) for r in range(world)])
+            write(g)
+            dz.step(hp, max_grad_norm=clip)
+            O.step_ex(ost, g[None], ohp, fsm, 1.0, clip)
+        f = dz.loss_scale()
+        assert f["t"] == fsm.t, (step, f)
+        assert abs(f["grad_norm_sq"] - fsm.grad_norm_sq) <= 1e-9 * fsm.grad_norm_sq, step
+        flat = np.zeros(dz.plan.T, np.float32)
+        flat[idx] = ost.master
+        mine = dz.current("master").cpu().numpy()
+        assert np.array_equal(mine.view(np.uint32), flat[rank * S:(rank + 1) * S].view(np.uint32)), step
+    dz.close()
 
 
 if __name__ == "__main__":

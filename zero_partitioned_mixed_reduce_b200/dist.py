@@ -6,13 +6,22 @@ read every other rank's buffers with plain loads over NVLink. A step is:
 
   1. a one-element all-reduce on the compute stream, so that every rank's
      gradients are written before any rank reads them;
-  2. zero_step_shard on the rank's own shard, reading the R gradient buffers
-     through the peer pointers -- the reduce-scatter is the fused kernel's
-     own loads, summed in fp32 in rank order, so no half-precision partial
-     sum ever leaves a GPU;
+  2. zero_step_shard_ex on the rank's own shard, reading the R gradient
+     buffers through the peer pointers -- the reduce-scatter is the fused
+     kernel's own loads, summed in fp32 in rank order, so no half-precision
+     partial sum ever leaves a GPU;
   3. an all-reduce (sum) of the two totals {sum g^2, overflow}, which also
      orders every rank's kernel before anyone overwrites its gradients;
   4. zero_step_commit, the same skip / loss-scale decision on every rank.
+
+With global-norm clipping, a norm pass over the rank's shard (again through
+the peer pointers) and a one-double all-reduce come before step 2.
+
+Gradient accumulation uses the two-pass form: after each micro-batch,
+reduce_scatter() sums the rank's shard of every replica into its local fp32
+accumulator (zero_reduce_scatter_shard, between two one-element
+all-reduces that order the peers' writes and reads), and
+step_accumulated() steps from it.
 
 ZeRO-3 layer gathers read the peers' parameter shards the same way.
 Argument marshalling only; the arithmetic runs in libzero_b200.so. The
@@ -27,7 +36,8 @@ from .state import HALF, Plan
 
 class DistributedZero:
     def __init__(self, numels, layer_ids=None, dtype=Z.ZERO_BF16, mode=Z.ZERO_SCALE_NONE,
-                 init_scale=1.0, growth_interval=1000, tensor_align=8, bucket_elems=0, group=None):
+                 init_scale=1.0, growth_interval=1000, tensor_align=8, bucket_elems=0, group=None,
+                 accumulate=False):
         import torch.distributed._symmetric_memory as symm
         self.group = group or dist.group.WORLD
         self.world = dist.get_world_size(self.group)
@@ -60,13 +70,18 @@ class DistributedZero:
 
         def own(x):  # pointer list with only this rank's shard filled in
             return [x.data_ptr() if r == self.rank else None for r in range(R)]
+        # the two-pass form keeps this rank's fp32 accumulator
+        self.acc = torch.zeros(S, dtype=torch.float32, device=dev) if accumulate else None
+        self.acc_list = [self.acc if r == self.rank else None for r in range(R)] if accumulate else None
         self.handle = Z.StateHandle([dict(master=own(self.master[k]), m=own(self.m[k]),
                                           v=own(self.v[k]), param=own(self.param[k]))
-                                     for k in range(sets)])
+                                     for k in range(sets)], self.acc_list)
+        self.micro = 0
         self.gather_handle = Z.StateHandle([dict(master=[None] * R, m=[None] * R, v=[None] * R,
                                                  param=self.param_ptrs[k]) for k in range(sets)])
         self.ctx = Z.zero_ctx_create(self.plan.handle, mode, init_scale, growth_interval)
         self.partial = torch.zeros(2, dtype=torch.float64, device=dev)
+        self.norm = torch.zeros(2, dtype=torch.float64, device=dev)
         self.token = torch.zeros(1, dtype=torch.float32, device=dev)
 
     def load(self, master_padded, param_padded):
@@ -81,13 +96,45 @@ class DistributedZero:
         torch.cuda.synchronize()
         dist.barrier(self.group)
 
-    def step(self, hp, stream=None):
-        """One ZeRO step; the gradients of every rank must be in self.grads."""
+    def _global_norm(self, grads, acc, divisor, stream):
+        Z.zero_grad_norm_shard(self.ctx, grads, acc, self.rank, self.rank + 1, self.norm, divisor,
+                               stream)
+        dist.all_reduce(self.norm, group=self.group)
+
+    def step(self, hp, max_grad_norm=0.0, stream=None):
+        """One fused ZeRO step; the gradients of every rank must be in
+        self.grads. max_grad_norm > 0 clips to that global norm."""
         dist.all_reduce(self.token, group=self.group)
-        Z.zero_step_shard(self.ctx, hp, self.handle, self.grad_ptrs, self.rank, self.rank + 1,
-                          self.partial, stream)
+        if max_grad_norm > 0:
+            self._global_norm(self.grad_ptrs, None, 1.0, stream)
+        Z.zero_step_shard_ex(self.ctx, hp, self.handle, self.grad_ptrs, self.rank, self.rank + 1,
+                             self.partial, 1.0, max_grad_norm, self.norm, stream)
         dist.all_reduce(self.partial, group=self.group)
         Z.zero_step_commit(self.ctx, self.partial, stream)
+
+    def reduce_scatter(self, stream=None):
+        """After a micro-batch's backward wrote self.grads on every rank: add
+        this rank's shard of the reduced gradients to its accumulator (the
+        first micro-batch of a step overwrites it)."""
+        assert self.acc is not None, "construct with accumulate=True"
+        dist.all_reduce(self.token, group=self.group)  # every replica is written
+        Z.zero_reduce_scatter_shard(self.ctx, -1, self.grad_ptrs, self.acc_list, self.rank, self.rank + 1,
+                                    Z.ZERO_RS_ACCUMULATE if self.micro else 0, stream)
+        dist.all_reduce(self.token, group=self.group)  # every peer has read this rank's replica
+        self.micro += 1
+
+    def step_accumulated(self, hp, grad_divisor=None, max_grad_norm=0.0, stream=None):
+        """The step from the accumulated micro-batches; grad_divisor defaults
+        to their count (the mean)."""
+        assert self.micro > 0, "no micro-batch was reduce-scattered"
+        k = float(self.micro) if grad_divisor is None else grad_divisor
+        if max_grad_norm > 0:
+            self._global_norm(None, self.acc_list, k, stream)
+        Z.zero_step_shard_ex(self.ctx, hp, self.handle, None, self.rank, self.rank + 1, self.partial, k,
+                             max_grad_norm, self.norm, stream)
+        dist.all_reduce(self.partial, group=self.group)
+        Z.zero_step_commit(self.ctx, self.partial, stream)
+        self.micro = 0
 
     def gather_layer(self, layer, out, stream=None):
         """ZeRO-3 all-gather of one layer from every rank's parameter shard."""
