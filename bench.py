@@ -53,7 +53,8 @@ def parse_args(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--accum", type=int, default=1,
-                    help="micro-batches accumulated per step (two-pass path)")
+                    help="micro-batches accumulated per step (the last fused into the step, or "
+                         "all reduce-scattered on the two-pass path)")
     ap.add_argument("--clip", type=float, default=0.0,
                     help="global-norm clipping threshold (> 0: on; fused path for R <= 5, "
                          "two-pass path otherwise)")
@@ -243,7 +244,9 @@ class Bench:
         self.R, self.dtype = wl["R"], wl["dtype"]
         self.accum, self.clip = accum, clip
         if path == "auto":
-            if accum > 1 or (clip > 0 and wl["R"] > 5):
+            # accumulation fuses its last micro-batch into the step unless
+            # clipping needs the full sum first
+            if (accum > 1 and clip > 0) or (clip > 0 and wl["R"] > 5):
                 path = "twopass"
             else:
                 # ping-pong state measured 2-3 % faster than in place at R = 4 and 8
@@ -251,8 +254,8 @@ class Bench:
                 # fp32 state, which every workload here fits
                 path = "pingpong"
         self.twopass = path.startswith("twopass")
-        if accum > 1 and not self.twopass:
-            raise SystemExit("--accum needs the two-pass path")
+        if accum > 1 and clip > 0 and not self.twopass:
+            raise SystemExit("--accum with --clip needs the two-pass path")
         self.path = path
         self.plan = Z.Plan(wl["numels"], wl["layer_ids"], wl["R"], wl["dtype"], 8,
                            wl["bucket_elems"])
@@ -260,7 +263,7 @@ class Bench:
         # the two-pass step measured the same in place as ping-pong, so it
         # keeps one state set
         sets = 2 if path in ("pingpong", "twopass_pingpong") else 1
-        self.state = Z.ShardedState(self.plan, sets=sets, with_acc=self.twopass)
+        self.state = Z.ShardedState(self.plan, sets=sets, with_acc=self.twopass or accum > 1)
         half = Z.state.HALF[wl["dtype"]]
         # initial fp32 master ~N(0, 0.02) and its half copy, tensor by tensor
         for k, (n, off) in enumerate(zip(wl["numels"], self.plan.offsets)):
@@ -314,6 +317,8 @@ class Bench:
         n = 1 + (len(self.gather_buckets) if self.gather_buckets else len(self.plan.layers))
         if self.twopass:
             n += self.accum * len(self.plan.buckets)
+        else:
+            n += (self.accum - 1) * len(self.plan.buckets)
         if self.clip > 0:
             n += 1  # the norm pass
         return n
@@ -326,6 +331,10 @@ class Bench:
             main = (2 * R + 4) * T + (self.accum - 1) * (2 * R + 8) * T + 30 * T
             if self.clip > 0:
                 main += 4 * T
+        elif self.accum > 1:
+            # micro-batches 1..k-1 into the accumulators, the last fused with
+            # the step (which reads the accumulators: 4 more bytes)
+            main = (2 * R + 4) * T + (self.accum - 2) * (2 * R + 8) * T + (2 * R + 30) * T
         else:
             main = (2 * R + 26) * T
             if self.clip > 0:
@@ -345,6 +354,13 @@ class Bench:
                                                     stream)
             Z.zero_step_ex(self.ctx, hp, self.state.handle, None, float(self.accum), self.clip,
                            stream)
+        elif self.accum > 1:
+            for mu in range(self.accum - 1):
+                flags = Z.ZERO_RS_ACCUMULATE if mu else 0
+                for b in range(len(self.plan.buckets)):
+                    Z.zero_reduce_scatter_bucket_ex(self.ctx, b, grads, self.state.acc, flags, stream)
+            Z.zero_step_ex(self.ctx, hp, self.state.handle, grads, float(self.accum), 0.0, stream,
+                           flags=Z.ZERO_STEP_ADD_ACC)
         elif self.clip > 0:
             Z.zero_step_ex(self.ctx, hp, self.state.handle, grads, 1.0, self.clip, stream)
         else:
@@ -443,6 +459,8 @@ def run_ours(args, world, rank, local):
         kernel_name += f" (accum {b.accum}{', clip' if b.clip > 0 else ''})"
     elif b.clip > 0:
         kernel_name = "grad_norm+fused_step_kernel (clip)"
+    elif b.accum > 1:
+        kernel_name = f"reduce_scatter+fused_step_kernel (accum {b.accum}, last micro-batch fused)"
     traffic = profiled_traffic(kernel_name, args.workload)
     out = {
         "metric": METRIC,
@@ -463,6 +481,7 @@ def run_ours(args, world, rank, local):
             "workload": workload_label(args.workload, b.wl, args.first_tensors),
             "R": b.R, "P": b.P, "T": b.T, "S": b.S, "n_layers": len(b.plan.layers),
             "path": {"pingpong": f"{'global-norm clip pass, ' if b.clip > 0 else ''}"
+                                 f"{f'{b.accum - 1} micro-batch(es) reduce-scattered, last ' if b.accum > 1 else ''}"
                                  "fused reduce-scatter+AdamW, ping-pong state",
                      "inplace": f"{'global-norm clip pass, ' if b.clip > 0 else ''}"
                                 "fused reduce-scatter+AdamW, in place",

@@ -329,15 +329,28 @@ zero_status zero_step(zero_ctx_t* ctx, const zero_adamw* hp, const zero_state* s
  *    with clipping moves 4R + 26 bytes per element against 2R + 38 for the
  *    two-pass path, so it is the cheaper one for R <= 5. The recorded
  *    grad_norm_sq is the norm before clipping.
+ *  flags & ZERO_STEP_ADD_ACC (fused path, the last micro-batch of an
+ *    accumulation): the reduced gradient is state->acc[o] plus this
+ *    micro-batch's rank-order sum of the replicas,
+ *      acc + (((f32(g_0) + f32(g_1)) + ...) + f32(g_{R-1})),
+ *    exactly what zero_reduce_scatter_bucket_ex(ZERO_RS_ACCUMULATE) followed
+ *    by the two-pass step computes, in one pass that neither writes nor
+ *    re-reads the accumulator: 2R + 30 bytes per element instead of
+ *    (2R + 8) + 30. The accumulator is read only. Not combinable with
+ *    clipping (whose norm needs the sum before the update): use the two-pass
+ *    path for that.
  * Defines: not on the pages (clipping and accumulation are common practice
  * around ZeRO training loops, not part of the method the pages describe).
- * Errors: as zero_step, plus ZERO_ERR_INVALID_ARG for a divisor < 1 or a
- * negative or non-finite max norm.
+ * Errors: as zero_step, plus ZERO_ERR_INVALID_ARG for a divisor < 1, a
+ * negative or non-finite max norm, unknown flags, or ZERO_STEP_ADD_ACC
+ * without grads, without state->acc or with clipping.
  */
+#define ZERO_STEP_ADD_ACC 1
 typedef struct {
     double grad_divisor;
     double max_grad_norm;
-    int64_t reserved[2]; /* must be 0 */
+    int64_t flags;    /* ZERO_STEP_* bits, 0 for none */
+    int64_t reserved; /* must be 0 */
 } zero_step_opts;
 zero_status zero_step_ex(zero_ctx_t* ctx, const zero_adamw* hp, const zero_state* state,
                          const void* const* grads, const zero_step_opts* opts, void* stream);
@@ -380,6 +393,8 @@ zero_status zero_step_shard(zero_ctx_t* ctx, const zero_adamw* hp, const zero_st
  *    of the zero_grad_norm_shard partials of this step; the coefficient
  *    min(1, max_norm / (sqrt(global_norm_sq) + 1e-6)) is formed from it on
  *    the device. global_norm_sq may be NULL without clipping.
+ *  - opts->flags may hold ZERO_STEP_ADD_ACC (fused path, as for
+ *    zero_step_ex): only the owners' accumulators are read.
  * partial and the commit are as for zero_step_shard. Running every owner
  * range in one process, with the partials summed, gives exactly zero_step_ex.
  * Defines: [instr] ZeRO-2 "Mechanism"; clipping and accumulation are not on

@@ -61,8 +61,9 @@ def f32bits(a: np.ndarray) -> np.ndarray:
 class Case:
     """One parity case: a tensor list, R, dtype, alignment, loss-scale mode and
     path ("inplace", "pingpong", "twopass", "twopass_pp": two-pass with
-    ping-pong state), run for a few steps on the GPU and in the oracle on the
-    same bytes."""
+    ping-pong state, "fused_acc": ping-pong state plus accumulators for the
+    fused last micro-batch), run for a few steps on the GPU and in the oracle
+    on the same bytes."""
 
     def __init__(self, numels, R, dtype, align=8, mode=O.SCALE_NONE, init_scale=1.0, interval=1000,
                  path="pingpong", bucket_elems=0, layer_ids=None, sigma=1e-2, seed=5, hp=None):
@@ -75,13 +76,14 @@ class Case:
         self.idx = self.lay.flat_index()
         S, T = self.plan.S, self.plan.T
         self.g = Guarded()
-        sets = 2 if path in ("pingpong", "twopass_pp") else 1
+        sets = 2 if path in ("pingpong", "twopass_pp", "fused_acc") else 1
         self.sets = sets
         self.master = [[self.g.f32(S) for _ in range(R)] for _ in range(sets)]
         self.m = [[self.g.f32(S) for _ in range(R)] for _ in range(sets)]
         self.v = [[self.g.f32(S) for _ in range(R)] for _ in range(sets)]
         self.param = [[self.g.half(S, dtype) for _ in range(R)] for _ in range(sets)]
-        self.acc = [self.g.f32(S) for _ in range(R)] if path.startswith("twopass") else None
+        self.acc = ([self.g.f32(S) for _ in range(R)]
+                    if path.startswith("twopass") or path == "fused_acc" else None)
         self.grads = [self.g.half(T, dtype) for _ in range(R)]
         self.handle = Z.StateHandle(
             [dict(master=self.master[k], m=self.m[k], v=self.v[k], param=self.param[k])
@@ -247,6 +249,36 @@ class Case:
         self.g.check()
         return skipped, [p.cpu().numpy() for p in partials]
 
+    def step_fused_accum(self, n_micro, grad_divisor=1.0, inject=None):
+        """Accumulation whose last micro-batch is fused into the step
+        (ZERO_STEP_ADD_ACC): micro-batches 0..n-2 reduce-scattered into the
+        accumulators, the last read straight from the replicas.
+        inject: (micro, rank, element, bits)."""
+        assert self.path == "fused_acc" and n_micro >= 2
+        self.step_no += 1
+        scale = self.ofsm.scale if self.mode != O.SCALE_NONE else 1.0
+        g = np.stack([np.stack([u16(synth.flat_grads(self.wl, self.step_no * 100 + mu, r, scale, "cpu"))
+                                for r in range(self.R)]) for mu in range(n_micro)])
+        for (mu, r, e, bits) in inject or []:
+            g[mu, r, e] = bits
+        for mu in range(n_micro):
+            for r in range(self.R):
+                gp = np.zeros(self.plan.T, np.uint16)
+                gp[self.idx] = g[mu, r]
+                self.grads[r].view(torch.int16).copy_(torch.from_numpy(gp.view(np.int16)))
+            if mu < n_micro - 1:
+                for b in range(len(self.plan.buckets)):
+                    Z.zero_reduce_scatter_bucket_ex(self.ctx, b, self.grads, self.acc,
+                                                    Z.ZERO_RS_ACCUMULATE if mu else 0)
+        Z.zero_step_ex(self.ctx, self.hp, self.handle, self.grads, grad_divisor, 0.0,
+                       flags=Z.ZERO_STEP_ADD_ACC)
+        skipped = O.step_ex(self.ostate, g, O.AdamW(**{k: self.hp[k] for k in
+                                                       ("lr", "beta1", "beta2", "eps",
+                                                        "weight_decay")}),
+                            self.ofsm, grad_divisor, 0.0)
+        self.g.check()
+        return skipped
+
     def step_sharded_ex(self, splits, n_micro=1, grad_divisor=1.0, max_grad_norm=0.0, inject=None):
         """The multi-rank step emulated shard range by shard range, with the
         cross-rank sums done here: fused (path "pingpong"/"inplace") or
@@ -262,14 +294,15 @@ class Case:
         for (mu, r, e, bits) in inject or []:
             g[mu, r, e] = bits
         twopass = self.path.startswith("twopass")
-        assert twopass or n_micro == 1
+        add_acc = self.path == "fused_acc" and n_micro > 1  # last micro-batch fused into the step
+        assert twopass or add_acc or n_micro == 1
         dev = lambda: torch.zeros(2, dtype=torch.float64, device="cuda")
         for mu in range(n_micro):
             for r in range(self.R):
                 gp = np.zeros(self.plan.T, np.uint16)
                 gp[self.idx] = g[mu, r]
                 self.grads[r].view(torch.int16).copy_(torch.from_numpy(gp.view(np.int16)))
-            if twopass:
+            if twopass or (add_acc and mu < n_micro - 1):
                 for lo, hi in splits:
                     acc = [self.acc[o] if lo <= o < hi else None for o in range(self.R)]
                     for b in range(len(self.plan.buckets)):
@@ -291,7 +324,8 @@ class Case:
         for lo, hi in splits:
             part = dev()
             Z.zero_step_shard_ex(self.ctx, self.hp, self.handle, None if twopass else self.grads, lo, hi,
-                                 part, grad_divisor, max_grad_norm, norm)
+                                 part, grad_divisor, max_grad_norm, norm,
+                                 flags=Z.ZERO_STEP_ADD_ACC if add_acc else 0)
             partials.append(part)
         Z.zero_step_commit(self.ctx, torch.stack(partials).sum(0))
         skipped = O.step_ex(self.ostate, g, O.AdamW(**{k: self.hp[k] for k in

@@ -105,3 +105,52 @@ def test_fused_clip_overflow_skips():
         c.compare()
     finally:
         c.close()
+
+
+@pytest.mark.parametrize("R", [1, 2, 3, 4, 8, 16])
+@pytest.mark.parametrize("dtype", [O.BF16, O.FP16])
+@pytest.mark.parametrize("n_micro,divisor", [(2, 2.0), (3, 3.0), (4, 1.0)])
+def test_fused_last_micro_batch_matches_oracle(R, dtype, n_micro, divisor):
+    # ZERO_STEP_ADD_ACC: the last micro-batch is summed into the step itself
+    mode = O.SCALE_DYNAMIC if dtype == O.FP16 else O.SCALE_NONE
+    c = Case([70_001, 13, 4096, 7, 999], R, dtype, 8, mode, init_scale=256.0, interval=2,
+             path="fused_acc", bucket_elems=5000, seed=R + 3 * n_micro)
+    try:
+        for _ in range(3):
+            c.step_fused_accum(n_micro, divisor)
+            c.compare()
+    finally:
+        c.close()
+
+
+@pytest.mark.parametrize("micro", [0, 2])
+def test_fused_last_micro_batch_overflow_skips(micro):
+    c = Case([20_000, 33], 4, O.FP16, 8, O.SCALE_DYNAMIC, init_scale=64.0, path="fused_acc")
+    try:
+        c.step_fused_accum(3, 3.0)
+        c.compare()
+        before = c.gpu_state()
+        assert c.step_fused_accum(3, 3.0, inject=[(micro, 1, 17, 0x7C00)])
+        c.compare()
+        after = c.gpu_state()
+        for k in ("master", "m", "v", "param"):
+            assert np.array_equal(before[k], after[k])
+    finally:
+        c.close()
+
+
+def test_add_acc_argument_errors():
+    c = Case([1000], 2, O.BF16, 8, O.SCALE_NONE, path="fused_acc")
+    try:
+        with pytest.raises(Z.ZeroError):  # with clipping
+            Z.zero_step_ex(c.ctx, c.hp, c.handle, c.grads, 1.0, 1.0, flags=Z.ZERO_STEP_ADD_ACC)
+        with pytest.raises(Z.ZeroError):  # on the two-pass path
+            Z.zero_step_ex(c.ctx, c.hp, c.handle, None, 1.0, 0.0, flags=Z.ZERO_STEP_ADD_ACC)
+        with pytest.raises(Z.ZeroError):  # unknown flag
+            Z.zero_step_ex(c.ctx, c.hp, c.handle, c.grads, 1.0, 0.0, flags=2)
+        no_acc = Z.StateHandle([dict(master=c.master[k], m=c.m[k], v=c.v[k], param=c.param[k])
+                                for k in range(2)])
+        with pytest.raises(Z.ZeroError):  # no accumulators
+            Z.zero_step_ex(c.ctx, c.hp, no_acc, c.grads, 1.0, 0.0, flags=Z.ZERO_STEP_ADD_ACC)
+    finally:
+        c.close()

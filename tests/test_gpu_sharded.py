@@ -153,3 +153,16 @@ def test_sharded_ex_argument_errors():
         assert e.value.status == Z.ZERO_ERR_INVALID_ARG
     finally:
         c.close()
+
+
+@pytest.mark.parametrize("R", [1, 2, 4, 8])
+@pytest.mark.parametrize("n_micro", [2, 3])
+def test_sharded_fused_last_micro_batch_matches_oracle(R, n_micro):
+    c = Case([70_001, 13, 4096, 7, 999], R, O.FP16, 8, O.SCALE_DYNAMIC, init_scale=256.0, interval=2,
+             path="fused_acc", bucket_elems=9000, seed=R + 60)
+    try:
+        for step in range(3):
+            c.step_sharded_ex(SPLITS[R][step % len(SPLITS[R])], n_micro, float(n_micro))
+            c.compare()
+    finally:
+        c.close()

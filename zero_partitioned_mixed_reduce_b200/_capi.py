@@ -20,6 +20,7 @@ ZERO_BF16, ZERO_FP16 = 0, 1
 ZERO_SCALE_NONE, ZERO_SCALE_STATIC, ZERO_SCALE_DYNAMIC = 0, 1, 2
 ZERO_LOSS_SCALE_GET, ZERO_LOSS_SCALE_SET = 0, 1
 ZERO_RS_ACCUMULATE = 1
+ZERO_STEP_ADD_ACC = 1
 
 STATUS_NAMES = {0: "ZERO_OK", 1: "ZERO_ERR_INVALID_ARG", 2: "ZERO_ERR_ALIGN", 3: "ZERO_ERR_CUDA",
                 4: "ZERO_ERR_OOM", 5: "ZERO_ERR_RANGE", 6: "ZERO_ERR_TIMEOUT", 7: "ZERO_ERR_STATE"}
@@ -68,8 +69,8 @@ class zero_state(C.Structure):
 
 
 class zero_step_opts(C.Structure):
-    _fields_ = [("grad_divisor", C.c_double), ("max_grad_norm", C.c_double),
-                ("reserved", C.c_int64 * 2)]
+    _fields_ = [("grad_divisor", C.c_double), ("max_grad_norm", C.c_double), ("flags", C.c_int64),
+                ("reserved", C.c_int64)]
 
 
 class zero_loss_scale_state(C.Structure):
@@ -285,14 +286,15 @@ def zero_step(ctx, hp, state: StateHandle, grads=None, stream=None):
 
 
 def zero_step_ex(ctx, hp, state: StateHandle, grads=None, grad_divisor=1.0, max_grad_norm=0.0,
-                 stream=None):
-    """zero_step with a grad divisor and global-norm clipping (two-pass only)."""
+                 stream=None, flags=0):
+    """zero_step with a grad divisor, global-norm clipping and flags
+    (ZERO_STEP_ADD_ACC: the fused step adds state's accumulators)."""
     if isinstance(hp, dict):
         hp = zero_adamw(hp["lr"], hp["beta1"], hp["beta2"], hp["eps"], hp["weight_decay"])
     g = None
     if grads is not None:
         g, ga = _ptr_array(grads)
-    opts = zero_step_opts(grad_divisor, max_grad_norm)
+    opts = zero_step_opts(grad_divisor, max_grad_norm, flags)
     _check(_lib.zero_step_ex(ctx, C.byref(hp), C.byref(state.c), g, C.byref(opts),
                              _stream(stream)))
 
@@ -416,13 +418,13 @@ def zero_step_shard(ctx, hp, state: StateHandle, grads, owner_lo, owner_hi, part
 
 
 def zero_step_shard_ex(ctx, hp, state: StateHandle, grads, owner_lo, owner_hi, partial,
-                       grad_divisor=1.0, max_grad_norm=0.0, global_norm_sq=None, stream=None):
+                       grad_divisor=1.0, max_grad_norm=0.0, global_norm_sq=None, stream=None, flags=0):
     """Sharded step with options; grads=None steps from state's accumulators.
     global_norm_sq: device float64 holding the cross-rank norm (clipping)."""
     if isinstance(hp, dict):
         hp = zero_adamw(hp["lr"], hp["beta1"], hp["beta2"], hp["eps"], hp["weight_decay"])
     g = _ptr_array(grads)
-    opts = zero_step_opts(grad_divisor, max_grad_norm)
+    opts = zero_step_opts(grad_divisor, max_grad_norm, flags)
     _check(_lib.zero_step_shard_ex(ctx, C.byref(hp), C.byref(state.c), g[0] if g else None, owner_lo,
                                    owner_hi, C.byref(opts), _addr(global_norm_sq), _addr(partial),
                                    _stream(stream)))

@@ -290,12 +290,18 @@ extern "C" zero_status zero_step_ex(zero_ctx_t* ctx, const zero_adamw* hp, const
                                     const void* const* grads, const zero_step_opts* opts,
                                     void* stream) {
     const char* where = "zero_step";
-    zero_step_opts o{1.0, 0.0, {0, 0}};
+    zero_step_opts o{1.0, 0.0, 0, 0};
     if (opts) o = *opts;
     if (!(o.grad_divisor >= 1.0) || !std::isfinite(o.grad_divisor) || !(o.max_grad_norm >= 0.0) ||
-        !std::isfinite(o.max_grad_norm) || o.reserved[0] != 0 || o.reserved[1] != 0)
+        !std::isfinite(o.max_grad_norm) || o.reserved != 0)
         return zb_fail(ZERO_ERR_INVALID_ARG,
                        "zero_step_ex: need grad_divisor >= 1, finite max_grad_norm >= 0, reserved 0");
+    if (o.flags & ~static_cast<int64_t>(ZERO_STEP_ADD_ACC))
+        return zb_fail(ZERO_ERR_INVALID_ARG, "zero_step_ex: unknown flags");
+    const bool add_acc = (o.flags & ZERO_STEP_ADD_ACC) != 0;
+    if (add_acc && (grads == nullptr || o.max_grad_norm > 0.0))
+        return zb_fail(ZERO_ERR_INVALID_ARG,
+                       "zero_step_ex: ZERO_STEP_ADD_ACC needs the fused path (grads) and no clipping");
     if (!ctx || !hp) return zb_fail(ZERO_ERR_INVALID_ARG, "zero_step: NULL ctx or hyper-parameters");
     zero_status s = check_device(ctx, where);
     if (s != ZERO_OK) return s;
@@ -307,6 +313,7 @@ extern "C" zero_status zero_step_ex(zero_ctx_t* ctx, const zero_adamw* hp, const
     int sets = 1;
     if ((s = check_state(ctx, state, where, &sets, false)) != ZERO_OK) return s;
     const bool fused = grads != nullptr;
+    if (add_acc && (s = check_ranks(state->acc, ctx->R, 32, where, "acc")) != ZERO_OK) return s;
     if (fused) {
         if ((s = check_ranks(grads, ctx->R, 16, where, "grads")) != ZERO_OK) return s;
         if (sets == 1 && ctx->cfg.mode == ZERO_SCALE_DYNAMIC)
@@ -340,6 +347,7 @@ extern "C" zero_status zero_step_ex(zero_ctx_t* ctx, const zero_adamw* hp, const
     sp.divisor = o.grad_divisor;
     sp.max_norm = o.max_grad_norm;
     sp.clip = o.max_grad_norm > 0.0 ? 1 : 0;
+    sp.add_acc = add_acc ? 1 : 0;
     sp.interval = ctx->cfg.growth_interval;
     sp.growth = ctx->cfg.growth_factor;
     sp.backoff = ctx->cfg.backoff_factor;
@@ -357,7 +365,7 @@ extern "C" zero_status zero_step_ex(zero_ctx_t* ctx, const zero_adamw* hp, const
     fill_state_ptrs(ctx, state, sets, &p);
     for (int r = 0; r < ctx->R; ++r) {
         p.g[r] = fused ? grads[r] : nullptr;
-        p.acc[r] = fused ? nullptr : state->acc[r];
+        p.acc[r] = (!fused || add_acc) ? state->acc[r] : nullptr;
     }
     cudaError_t e = cudaSuccess;
     // clipping needs the global norm before any element is updated: one
@@ -525,13 +533,19 @@ extern "C" zero_status zero_step_shard_ex(zero_ctx_t* ctx, const zero_adamw* hp,
     const char* where = "zero_step_shard";
     if (!ctx || !hp || !partial)
         return zb_fail(ZERO_ERR_INVALID_ARG, "zero_step_shard: NULL ctx, hp or partial");
-    zero_step_opts o{1.0, 0.0, {0, 0}};
+    zero_step_opts o{1.0, 0.0, 0, 0};
     if (opts) o = *opts;
     if (!(o.grad_divisor >= 1.0) || !std::isfinite(o.grad_divisor) || !(o.max_grad_norm >= 0.0) ||
-        !std::isfinite(o.max_grad_norm) || o.reserved[0] != 0 || o.reserved[1] != 0)
+        !std::isfinite(o.max_grad_norm) || o.reserved != 0)
         return zb_fail(ZERO_ERR_INVALID_ARG,
                        "zero_step_shard: need grad_divisor >= 1, finite max_grad_norm >= 0, reserved 0");
+    if (o.flags & ~static_cast<int64_t>(ZERO_STEP_ADD_ACC))
+        return zb_fail(ZERO_ERR_INVALID_ARG, "zero_step_shard: unknown flags");
+    const bool add_acc = (o.flags & ZERO_STEP_ADD_ACC) != 0;
     const bool clip = o.max_grad_norm > 0.0;
+    if (add_acc && (grads == nullptr || clip))
+        return zb_fail(ZERO_ERR_INVALID_ARG,
+                       "zero_step_shard: ZERO_STEP_ADD_ACC needs the fused path (grads) and no clipping");
     if (clip && !global_norm_sq)
         return zb_fail(ZERO_ERR_INVALID_ARG,
                        "zero_step_shard: clipping needs global_norm_sq (the cross-rank sum of the "
@@ -548,11 +562,9 @@ extern "C" zero_status zero_step_shard_ex(zero_ctx_t* ctx, const zero_adamw* hp,
     int sets = 1;
     if ((s = check_state_range(ctx, state, owner_lo, owner_hi, where, &sets)) != ZERO_OK) return s;
     const bool fused = grads != nullptr;
-    if (fused) {
-        if ((s = check_all_grads(ctx, grads, where)) != ZERO_OK) return s;
-    } else if ((s = check_owned_acc(ctx, state->acc, owner_lo, owner_hi, where)) != ZERO_OK) {
+    if (fused && (s = check_all_grads(ctx, grads, where)) != ZERO_OK) return s;
+    if ((!fused || add_acc) && (s = check_owned_acc(ctx, state->acc, owner_lo, owner_hi, where)) != ZERO_OK)
         return s;
-    }
     if (sets == 1 && ctx->cfg.mode == ZERO_SCALE_DYNAMIC)
         return zb_fail(ZERO_ERR_INVALID_ARG, "zero_step_shard: dynamic loss scaling needs state set 1 (ping-pong)");
     if (sets == 1 && ctx->two_sets)
@@ -570,12 +582,13 @@ extern "C" zero_status zero_step_shard_ex(zero_ctx_t* ctx, const zero_adamw* hp,
     sp.lr = hp->lr;
     sp.max_norm = o.max_grad_norm;
     sp.clip = clip ? 1 : 0;
+    sp.add_acc = add_acc ? 1 : 0;
     if (fused) sp.drop_tile = ctx->drop_tile;
     zb::RankPtrs p{};
     for (int r = 0; r < ctx->R; ++r) {
         const bool owned = r >= owner_lo && r < owner_hi;
         p.g[r] = fused ? grads[r] : nullptr;
-        p.acc[r] = (!fused && owned) ? state->acc[r] : nullptr;
+        p.acc[r] = ((!fused || add_acc) && owned) ? state->acc[r] : nullptr;
         for (int k = 0; k < 2; ++k) {
             const int from = k < sets ? k : 0;
             p.master[k][r] = owned ? state->master[from][r] : nullptr;

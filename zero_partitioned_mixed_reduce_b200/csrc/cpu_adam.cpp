@@ -128,11 +128,11 @@ extern "C" zero_status zero_cpu_step(const zero_plan_t* plan, const zero_loss_sc
                                      float* const* m, float* const* v, void* const* param, int32_t nthreads) {
     if (!plan || !cfg || !inout || !hp || !acc || !master || !m || !v || !param)
         return zb_fail(ZERO_ERR_INVALID_ARG, "zero_cpu_step: NULL argument");
-    zero_step_opts o{1.0, 0.0, {0, 0}};
+    zero_step_opts o{1.0, 0.0, 0, 0};
     if (opts) o = *opts;
     if (!(o.grad_divisor >= 1.0) || !std::isfinite(o.grad_divisor) || !(o.max_grad_norm >= 0.0) ||
-        !std::isfinite(o.max_grad_norm))
-        return zb_fail(ZERO_ERR_INVALID_ARG, "zero_cpu_step: need grad_divisor >= 1 and finite max_grad_norm >= 0");
+        !std::isfinite(o.max_grad_norm) || o.flags != 0 || o.reserved != 0)
+        return zb_fail(ZERO_ERR_INVALID_ARG, "zero_cpu_step: need grad_divisor >= 1, finite max_grad_norm >= 0, no flags");
     if (cfg->mode < ZERO_SCALE_NONE || cfg->mode > ZERO_SCALE_DYNAMIC)
         return zb_fail(ZERO_ERR_INVALID_ARG, "zero_cpu_step: bad loss-scale mode");
     if (cfg->mode == ZERO_SCALE_DYNAMIC &&

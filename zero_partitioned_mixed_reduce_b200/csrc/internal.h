@@ -47,6 +47,7 @@ struct StepParams {
     double divisor = 1;       // grad divisor k: unscale by 1 / ((R * k) * scale)
     double max_norm = 0;      // > 0: clipping on
     int32_t clip = 0;
+    int32_t add_acc = 0;      // fused step adds the accumulators (ZERO_STEP_ADD_ACC)
     int64_t interval = 1;
     float growth = 2, backoff = 0.5f, min_scale = 1;
     DevState* st = nullptr;

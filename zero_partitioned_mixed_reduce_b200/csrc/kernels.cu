@@ -166,13 +166,14 @@ template <int CAP>
 struct FusedArgs {
     StepParams sp;
     const uint4* g[CAP];
+    const float* acc[CAP];  // ADD_ACC variant: the owners' accumulators
     float* master[2][CAP];
     float* m[2][CAP];
     float* v[2][CAP];
     uint4* param[2][CAP];
 };
 
-template <typename H, int RC, bool CLIP>
+template <typename H, int RC, bool CLIP, bool ACC = false>
 __global__ void __launch_bounds__(kThreads)
     fused_step_kernel(const __grid_constant__ FusedArgs<RC == 0 ? ZERO_MAX_RANKS : RC> a) {
     const StepParams& sp = a.sp;
@@ -212,6 +213,12 @@ __global__ void __launch_bounds__(kThreads)
             unpack8<H>(g0, acc);
 #pragma unroll 4
             for (int r = 1; r < R; ++r) add8<H>(ld_grad(a.g[r] + vi), acc);
+        }
+        if constexpr (ACC) {
+            // the earlier micro-batches' sum, then this one's rank-order sum
+            const F8 prev = ld_f8(a.acc[o] + j8);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) acc[e] = __fadd_rn(prev.x[e], acc[e]);
         }
         float out[8];
 #pragma unroll
@@ -809,13 +816,14 @@ uint32_t grid_for(uint64_t work_items, int per_sm, int cap) {
     return static_cast<uint32_t>(g > 0 ? g : 1);
 }
 
-template <typename H, int RC, bool CLIP>
+template <typename H, int RC, bool CLIP, bool ACC = false>
 cudaError_t fused_t(const StepParams& sp, const RankPtrs& p, cudaStream_t s) {
     constexpr int CAP = RC == 0 ? ZERO_MAX_RANKS : RC;
     FusedArgs<CAP> a;
     a.sp = sp;
     for (int r = 0; r < sp.R; ++r) {
         a.g[r] = static_cast<const uint4*>(p.g[r]);
+        a.acc[r] = p.acc[r];
         for (int k = 0; k < 2; ++k) {
             a.master[k][r] = p.master[k][r];
             a.m[k][r] = p.m[k][r];
@@ -823,9 +831,9 @@ cudaError_t fused_t(const StepParams& sp, const RankPtrs& p, cudaStream_t s) {
             a.param[k][r] = static_cast<uint4*>(p.param[k][r]);
         }
     }
-    static const int per_sm = blocks_per_sm(fused_step_kernel<H, RC, CLIP>);
+    static const int per_sm = blocks_per_sm(fused_step_kernel<H, RC, CLIP, ACC>);
     const uint32_t grid = grid_for(static_cast<uint64_t>(sp.oend - sp.obeg) * sp.S8, per_sm, sp.grid_cap);
-    fused_step_kernel<H, RC, CLIP><<<grid, kThreads, 0, s>>>(a);
+    fused_step_kernel<H, RC, CLIP, ACC><<<grid, kThreads, 0, s>>>(a);
     return cudaGetLastError();
 }
 
@@ -856,6 +864,18 @@ cudaError_t fused_tma_t(const StepParams& sp, const RankPtrs& p, cudaStream_t s)
                                    sp.grid_cap);
     fused_step_tma_kernel<H, RC, CLIP><<<grid, kThreads, smem, s>>>(a, tiles_per_shard);
     return cudaGetLastError();
+}
+
+// The last micro-batch of an accumulation, fused: the register kernel at
+// every R (the staged kernel has no accumulator stream).
+template <typename H>
+cudaError_t fused_acc_dispatch(const StepParams& sp, const RankPtrs& p, cudaStream_t s) {
+    switch (sp.R) {
+        case 4: return fused_t<H, 4, false, true>(sp, p, s);
+        case 8: return fused_t<H, 8, false, true>(sp, p, s);
+        case 16: return fused_t<H, 16, false, true>(sp, p, s);
+        default: return fused_t<H, 0, false, true>(sp, p, s);
+    }
 }
 
 template <typename H, bool CLIP>
@@ -940,6 +960,8 @@ cudaError_t acc_t(const StepParams& sp, const RankPtrs& p, cudaStream_t s) {
 }  // namespace
 
 cudaError_t launch_fused_step(const StepParams& sp, const RankPtrs& p, cudaStream_t s) {
+    if (sp.add_acc)
+        return sp.dtype == ZERO_FP16 ? fused_acc_dispatch<Fp16>(sp, p, s) : fused_acc_dispatch<Bf16>(sp, p, s);
     if (sp.clip)
         return sp.dtype == ZERO_FP16 ? fused_dispatch<Fp16, true>(sp, p, s) : fused_dispatch<Bf16, true>(sp, p, s);
     return sp.dtype == ZERO_FP16 ? fused_dispatch<Fp16, false>(sp, p, s) : fused_dispatch<Bf16, false>(sp, p, s);
