@@ -93,9 +93,18 @@ def check_accumulate_and_clip(rank, world):
         gp[idx] = g[rank]
         dz.grads.view(torch.int16).copy_(torch.from_numpy(gp.view(np.int16)))
 
-    for step in range(1, 5):
+    for step in range(1, 7):
         clip = 1e-3 if step % 2 else 0.0
-        if step <= 2:  # two micro-batches, accumulated
+        if step >= 5:  # three micro-batches, the last passed to the fused step
+            micro = [np.stack([u16(synth.flat_grads(wl, step * 10 + mu, r, 1.0, "cpu")) for r in range(world)])
+                     for mu in range(3)]
+            for g in micro[:2]:
+                write(g)
+                dz.reduce_scatter()
+            write(micro[2])
+            dz.step(hp, max_grad_norm=clip)
+            O.step_ex(ost, np.stack(micro), ohp, fsm, 3.0, clip)
+        elif step <= 2:  # two micro-batches, accumulated
             micro = [np.stack([u16(synth.flat_grads(wl, step * 10 + mu, r, 1.0, "cpu")) for r in range(world)])
                      for mu in range(2)]
             for g in micro:

@@ -101,16 +101,27 @@ class DistributedZero:
                                stream)
         dist.all_reduce(self.norm, group=self.group)
 
-    def step(self, hp, max_grad_norm=0.0, stream=None):
+    def step(self, hp, max_grad_norm=0.0, grad_divisor=None, stream=None):
         """One fused ZeRO step; the gradients of every rank must be in
-        self.grads. max_grad_norm > 0 clips to that global norm."""
+        self.grads. max_grad_norm > 0 clips to that global norm. After
+        reduce_scatter() of earlier micro-batches, self.grads holds the last
+        one: it is added to the accumulator inside the fused step
+        (ZERO_STEP_ADD_ACC), or, with clipping, reduce-scattered first.
+        grad_divisor defaults to the number of micro-batches."""
+        if self.micro > 0 and max_grad_norm > 0:
+            self.reduce_scatter(stream)
+            self.step_accumulated(hp, grad_divisor, max_grad_norm, stream)
+            return
+        k = float(self.micro + 1) if grad_divisor is None else grad_divisor
+        flags = Z.ZERO_STEP_ADD_ACC if self.micro > 0 else 0
         dist.all_reduce(self.token, group=self.group)
         if max_grad_norm > 0:
-            self._global_norm(self.grad_ptrs, None, 1.0, stream)
+            self._global_norm(self.grad_ptrs, None, k, stream)
         Z.zero_step_shard_ex(self.ctx, hp, self.handle, self.grad_ptrs, self.rank, self.rank + 1,
-                             self.partial, 1.0, max_grad_norm, self.norm, stream)
+                             self.partial, k, max_grad_norm, self.norm, stream, flags=flags)
         dist.all_reduce(self.partial, group=self.group)
         Z.zero_step_commit(self.ctx, self.partial, stream)
+        self.micro = 0
 
     def reduce_scatter(self, stream=None):
         """After a micro-batch's backward wrote self.grads on every rank: add
