@@ -666,6 +666,20 @@ zero_status zero_cpu_step(const zero_plan_t* plan, const zero_loss_scale_config*
                           const float* const* acc, float* const* master, float* const* m, float* const* v,
                           void* const* param, int32_t nthreads);
 
+/*
+ * zero_debug_bounds -- what the bounds-checking debug build recorded. That
+ * build (the same sources compiled with ZERO_DEBUG_BOUNDS) checks, in every
+ * kernel, each index and pointer it derives before the access that uses it:
+ * the vector within the flat range and the shard, the owner within the
+ * range given, the owner's buffers present. A failing access is skipped
+ * (never trapped) and counted; the first one's site number (the kernel and
+ * access) and index are kept. *count receives the number of failing
+ * accesses since the last reset, or -1 in the release build, whose kernels
+ * carry no checks. reset != 0 clears the record. Synchronizes the device.
+ * Errors: ZERO_ERR_INVALID_ARG (NULL output), ZERO_ERR_CUDA.
+ */
+zero_status zero_debug_bounds(int64_t* count, int64_t* first_site, int64_t* first_index, int32_t reset);
+
 /* zero_sync -- synchronize `stream` and report any pending CUDA error. */
 zero_status zero_sync(zero_ctx_t* ctx, void* stream);
 

@@ -1,0 +1,60 @@
+"""Run a cross-section of the hot path through the bounds-checking debug
+build of the library (selected with ZERO_B200_LIB), comparing each step with
+the oracle, then print the debug build's record of skipped out-of-range
+accesses as one JSON line. Launched by tests/test_gpu_debug_bounds.py."""
+import json
+import os
+import sys
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, os.path.dirname(HERE))
+sys.path.insert(0, HERE)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+import oracle as O  # noqa: E402
+import zero_partitioned_mixed_reduce_b200 as Z  # noqa: E402
+from gpu_harness import Case  # noqa: E402
+
+
+def main():
+    assert os.environ.get("ZERO_B200_LIB"), "run with ZERO_B200_LIB pointing at the debug build"
+    count, _, _ = Z.zero_debug_bounds(reset=True)
+    assert count == 0, "expected the debug build (the release build reports -1)"
+    numels = [70_001, 13, 4096, 7, 999, 3]
+    layers = [0, 0, 1, 1, 2, 2]
+    runs = 0
+    for R in (1, 2, 3, 4, 8, 16):
+        for path, mode, dtype in (("pingpong", O.SCALE_DYNAMIC, O.FP16), ("inplace", O.SCALE_NONE, O.BF16),
+                                  ("twopass", O.SCALE_STATIC, O.FP16), ("twopass_pp", O.SCALE_DYNAMIC, O.FP16),
+                                  ("fused_acc", O.SCALE_DYNAMIC, O.FP16)):
+            c = Case(numels, R, dtype, 8 if R != 3 else 1, mode, init_scale=256.0, interval=2, path=path,
+                     bucket_elems=5000, layer_ids=layers, seed=R)
+            try:
+                if path in ("pingpong", "inplace"):
+                    c.step()
+                    c.step_fused_ex(1.0, 1e-3)  # clipping on the fused path
+                elif path == "fused_acc":
+                    c.step_fused_accum(3, 3.0)
+                else:
+                    c.step_ex(2, 2.0, 1e-3)
+                c.compare()
+                splits = [(o, o + 1) for o in range(R)]
+                if path == "fused_acc":
+                    c.step_sharded_ex(splits, 2, 2.0)
+                else:
+                    c.step_sharded_ex(splits, 1 if not path.startswith("twopass") else 2, 1.0, 1e-3)
+                c.compare()
+                outs = [torch.empty(hi - lo, dtype=torch.int16, device="cuda") for lo, hi in c.lay.layers]
+                Z.zero_gather_layers(c.ctx, 0, outs, c.handle)
+                torch.cuda.synchronize()
+                runs += 1
+            finally:
+                c.close()
+    count, site, index = Z.zero_debug_bounds()
+    print(json.dumps({"cases": runs, "count": count, "first_site": site, "first_index": index}))
+
+
+if __name__ == "__main__":
+    main()

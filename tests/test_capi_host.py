@@ -138,3 +138,13 @@ def test_no_gpu_fails_loudly():
     with pytest.raises(Z.ZeroError) as e:
         Z.zero_ctx_create(p.handle)
     assert e.value.status == _capi.ZERO_ERR_CUDA
+
+
+def test_release_build_carries_no_bounds_checks():
+    # the bounds-checking build is a separate test library; the release
+    # build reports -1 without touching a GPU
+    import os
+    import zero_partitioned_mixed_reduce_b200 as Z
+    if os.environ.get("ZERO_B200_LIB"):
+        pytest.skip("another build is loaded")
+    assert Z.zero_debug_bounds() == (-1, 0, 0)

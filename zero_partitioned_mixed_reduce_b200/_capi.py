@@ -11,7 +11,9 @@ import ctypes as C
 import os
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "libzero_b200.so")
+# ZERO_B200_LIB selects another build of the library (the bounds-checking
+# debug build in the tests); by default the in-tree release build
+LIB_PATH = os.environ.get("ZERO_B200_LIB") or os.path.join(_HERE, "libzero_b200.so")
 
 ZERO_MAX_RANKS = 64
 ZERO_OK, ZERO_ERR_INVALID_ARG, ZERO_ERR_ALIGN, ZERO_ERR_CUDA = 0, 1, 2, 3
@@ -131,6 +133,8 @@ _sig("zero_step_shard_ex", _S, [_P, C.POINTER(zero_adamw), C.POINTER(zero_state)
 _sig("zero_reduce_scatter_shard", _S, [_P, C.c_int64, _PP, _PP, C.c_int32, C.c_int32, C.c_int32, _P])
 _sig("zero_grad_norm_shard", _S, [_P, _PP, _PP, C.c_double, C.c_int32, C.c_int32, _P, _P])
 _sig("zero_sync", _S, [_P, _P])
+_sig("zero_debug_bounds", _S, [C.POINTER(C.c_int64), C.POINTER(C.c_int64), C.POINTER(C.c_int64),
+                               C.c_int32])
 _sig("zero_last_error", C.c_size_t, [C.c_char_p, C.c_size_t])
 _sig("zero_version", C.c_char_p, [])
 
@@ -448,6 +452,14 @@ def zero_grad_norm_shard(ctx, grads, acc, owner_lo, owner_hi, partial, grad_divi
 def zero_step_commit(ctx, reduced, stream=None):
     """Loss-scale update from reduced totals (device buffer of 2 float64)."""
     _check(_lib.zero_step_commit(ctx, _addr(reduced), _stream(stream)))
+
+
+def zero_debug_bounds(reset=False):
+    """(count, first_site, first_index) of the out-of-range accesses the
+    debug build's kernels skipped; count is -1 in the release build."""
+    n, site, idx = C.c_int64(), C.c_int64(), C.c_int64()
+    _check(_lib.zero_debug_bounds(C.byref(n), C.byref(site), C.byref(idx), 1 if reset else 0))
+    return n.value, site.value, idx.value
 
 
 def zero_sync(ctx, stream=None):

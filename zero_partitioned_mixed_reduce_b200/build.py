@@ -4,6 +4,11 @@ Kernels: nvcc -gencode arch=compute_100a,code=sm_100a, -O3, --fmad=false (no
 multiply-add contraction anywhere in the step), no fast-math (IEEE division
 and square root, no flush-to-zero). Host C++: g++ -O2. The CUDA runtime is
 linked statically.
+
+build(debug=True) makes libzero_b200_debug.so instead: the same sources with
+ZERO_DEBUG_BOUNDS defined, so every kernel checks the indices and pointers it
+derives before each access, skips a failing access and records it (read back
+with zero_debug_bounds). It is a test build, loaded through ZERO_B200_LIB.
 """
 import os
 import subprocess
@@ -15,6 +20,8 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 BUILD = os.path.join(ROOT, "_build")
 OUT = os.path.join(PKG, "libzero_b200.so")
+OUT_DEBUG = os.path.join(PKG, "libzero_b200_debug.so")
+BUILD_DEBUG = os.path.join(ROOT, "_build_debug")
 CUDA_HOME = os.environ.get("CUDA_HOME", "/usr/local/cuda")
 NVCC = os.path.join(CUDA_HOME, "bin", "nvcc")
 
@@ -35,10 +42,10 @@ def _sources():
             + [os.path.join(INCLUDE, "zero_b200.h")])
 
 
-def up_to_date() -> bool:
-    if not os.path.exists(OUT):
+def up_to_date(out=OUT) -> bool:
+    if not os.path.exists(out):
         return False
-    t = os.path.getmtime(OUT)
+    t = os.path.getmtime(out)
     return all(os.path.getmtime(s) <= t for s in _sources())
 
 
@@ -53,26 +60,28 @@ def _run(cmd, log=None):
     return r
 
 
-def build(force: bool = False) -> str:
+def build(force: bool = False, debug: bool = False) -> str:
     """Compile the library if it is missing or older than any source."""
-    if not force and up_to_date():
-        return OUT
-    os.makedirs(BUILD, exist_ok=True)
+    out, bdir = (OUT_DEBUG, BUILD_DEBUG) if debug else (OUT, BUILD)
+    if not force and up_to_date(out):
+        return out
+    os.makedirs(bdir, exist_ok=True)
+    extra = ["-DZERO_DEBUG_BOUNDS"] if debug else []
     objs = []
     for s in CU_SOURCES:
-        o = os.path.join(BUILD, s + ".o")
-        _run([NVCC, *NVCC_FLAGS, "-c", os.path.join(CSRC, s), "-o", o],
-             log=os.path.join(BUILD, s + ".ptxas.txt"))
+        o = os.path.join(bdir, s + ".o")
+        _run([NVCC, *NVCC_FLAGS, *extra, "-c", os.path.join(CSRC, s), "-o", o],
+             log=os.path.join(bdir, s + ".ptxas.txt"))
         objs.append(o)
     for s in CPP_SOURCES:
-        o = os.path.join(BUILD, s + ".o")
-        _run(["g++", *CXX_FLAGS, *CXX_EXTRA.get(s, []), "-c", os.path.join(CSRC, s), "-o", o])
+        o = os.path.join(bdir, s + ".o")
+        _run(["g++", *CXX_FLAGS, *extra, *CXX_EXTRA.get(s, []), "-c", os.path.join(CSRC, s), "-o", o])
         objs.append(o)
-    tmp = OUT + f".tmp{os.getpid()}"
+    tmp = out + f".tmp{os.getpid()}"
     _run([NVCC, "-shared", *ARCH, "-cudart=static", *objs, "-o", tmp, "-Xcompiler", "-pthread"])
-    os.replace(tmp, OUT)
-    return OUT
+    os.replace(tmp, out)
+    return out
 
 
 if __name__ == "__main__":
-    print(build(force="--force" in sys.argv))
+    print(build(force="--force" in sys.argv, debug="--debug" in sys.argv))

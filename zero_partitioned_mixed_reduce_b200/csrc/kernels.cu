@@ -26,11 +26,42 @@
 #include <cfloat>
 #include <cstdint>
 #include <mutex>
+#include <string>
 
 #include "device_common.cuh"
 #include "internal.h"
 
 namespace zb {
+
+// ---------------------------------------------------------------------------
+// Bounds checks of the debug build (ZERO_DEBUG_BOUNDS). ZB_IN(cond, site,
+// index) guards an access: in the debug build a false cond is counted, the
+// first failing site and index are kept, and the caller skips the access; in
+// the release build it is the constant true and cond is not evaluated.
+// Sites: 1 fused vector, 2 fused accumulator, 3 staged tile issue, 4 staged
+// tile store, 5 two-pass vector, 6 accumulator norm, 7 replica norm,
+// 8 reduce-scatter vector, 9 reduce-scatter element, 10 gather vector,
+// 11 gather element.
+// ---------------------------------------------------------------------------
+#ifdef ZERO_DEBUG_BOUNDS
+__device__ unsigned long long g_bounds_count = 0;
+__device__ unsigned long long g_bounds_first = 0;
+__device__ __noinline__ bool bounds_fail(unsigned site, unsigned long long index) {
+    atomicAdd(&g_bounds_count, 1ull);
+    atomicCAS(&g_bounds_first, 0ull, (static_cast<unsigned long long>(site) << 48) | (index & 0xffffffffffffull));
+    return false;
+}
+#define ZB_IN(cond, site, index) ((cond) ? true : ::zb::bounds_fail((site), (index)))
+#else
+#define ZB_IN(cond, site, index) true
+#endif
+
+template <typename T, int CAP>
+__device__ __forceinline__ bool ptrs_ok(T* const (&p)[CAP], int n) {
+    for (int r = 0; r < n; ++r)
+        if (!p[r]) return false;
+    return true;
+}
 
 // Per-step coefficients. scale and t live on the device (the loss-scale
 // state machine may skip steps without the host knowing), so the parts that
@@ -193,6 +224,11 @@ __global__ void __launch_bounds__(kThreads)
         oc.seek(vi);
         const uint32_t o = oc.o;
         const size_t j8 = static_cast<size_t>(vi - oc.base) * 8;
+        if (!ZB_IN(vi < sp.T8 && o >= static_cast<uint32_t>(sp.obeg) && o < static_cast<uint32_t>(sp.oend) &&
+                       vi - oc.base < sp.S8 && ptrs_ok(a.g, R) && a.master[src][o] && a.m[src][o] &&
+                       a.v[src][o] && a.master[dst][o] && a.m[dst][o] && a.v[dst][o] && a.param[dst][o],
+                   1, vi))
+            continue;
         float acc[8];
         F8 p, m, v;
         if constexpr (RC > 0) {
@@ -216,6 +252,7 @@ __global__ void __launch_bounds__(kThreads)
         }
         if constexpr (ACC) {
             // the earlier micro-batches' sum, then this one's rank-order sum
+            if (!ZB_IN(a.acc[o] != nullptr, 2, vi)) continue;
             const F8 prev = ld_f8(a.acc[o] + j8);
 #pragma unroll
             for (int e = 0; e < 8; ++e) acc[e] = __fadd_rn(prev.x[e], acc[e]);
@@ -332,6 +369,11 @@ __global__ void __launch_bounds__(kThreads)
         unsigned char* base = smem + s * L::kBytes;
         const uint32_t bar = smem_u32(&bars[s]);
         if (tile == sp.drop_tile) return;  // test support: this tile's wait must run out
+        if (!ZB_IN(o >= static_cast<uint32_t>(sp.obeg) && o < static_cast<uint32_t>(sp.oend) && j0 < S &&
+                       len % 8 == 0 && j0 + len <= S && ptrs_ok(a.g, RC) && a.master[src][o] && a.m[src][o] &&
+                       a.v[src][o],
+                   3, tile))
+            return;  // skipped: the wait for this tile runs out and the step is abandoned
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
         mbar_expect_tx(bar, len * (RC * 2 + 12));
 #pragma unroll
@@ -388,10 +430,13 @@ __global__ void __launch_bounds__(kThreads)
                 out[e] = p.x[e];
             }
             const size_t jj = static_cast<size_t>(j0) + e0;
-            st_f8(a.master[dst][o] + jj, p);
-            st_f8(a.m[dst][o] + jj, m);
-            st_f8(a.v[dst][o] + jj, v);
-            st_u4(a.param[dst][o] + (jj >> 3), pack8<H>(out));
+            // a guarded block, not a continue: every thread must reach the barrier below
+            if (ZB_IN(jj + 8 <= S && a.master[dst][o] && a.m[dst][o] && a.v[dst][o] && a.param[dst][o], 4, jj)) {
+                st_f8(a.master[dst][o] + jj, p);
+                st_f8(a.m[dst][o] + jj, m);
+                st_f8(a.v[dst][o] + jj, v);
+                st_u4(a.param[dst][o] + (jj >> 3), pack8<H>(out));
+            }
         }
         __syncthreads();  // every thread is done with stage s
         const uint32_t next = tile + kTmaStages * gridDim.x;
@@ -442,6 +487,11 @@ __global__ void __launch_bounds__(kThreads) step_from_acc_kernel(const __grid_co
         oc.seek(vi);
         const uint32_t o = oc.o;
         const size_t j8 = static_cast<size_t>(vi - oc.base) * 8;
+        if (!ZB_IN(o >= static_cast<uint32_t>(sp.obeg) && o < static_cast<uint32_t>(sp.oend) && vi - oc.base < sp.S8 &&
+                       a.acc[o] && (skip || (a.master[src][o] && a.m[src][o] && a.v[src][o] &&
+                                             a.master[dst][o] && a.m[dst][o] && a.v[dst][o] && a.param[dst][o])),
+                   5, vi))
+            continue;
         const F8 acc = ld_f8(a.acc[o] + j8);
         if (skip) {
 #pragma unroll
@@ -559,8 +609,14 @@ __global__ void __launch_bounds__(kThreads) clip_norm_kernel(const __grid_consta
 #pragma unroll
         for (int u = 0; u < kNormUnroll; ++u) {
             const uint32_t vu = vi + u * stride;
-            if (vu < vend) {
+            bool take = vu < vend;
+            if (take) {
                 oc.seek(vu);
+                take = ZB_IN(oc.o >= static_cast<uint32_t>(sp.obeg) && oc.o < static_cast<uint32_t>(sp.oend) &&
+                                 vu - oc.base < sp.S8 && a.acc[oc.o],
+                             6, vu);
+            }
+            if (take) {
                 acc[u] = ld_f8(a.acc[oc.o] + static_cast<size_t>(vu - oc.base) * 8);
             } else {
 #pragma unroll
@@ -598,6 +654,7 @@ __global__ void __launch_bounds__(kThreads)
     const uint32_t stride = gridDim.x * kThreads;
     const uint32_t vend = static_cast<uint32_t>(sp.oend) * sp.S8;
     for (uint32_t vi = line_start(static_cast<uint32_t>(sp.obeg) * sp.S8, stride); vi < vend; vi += stride) {
+        if (!ZB_IN(vi >= static_cast<uint32_t>(sp.obeg) * sp.S8 && vi < sp.T8 && ptrs_ok(a.g, R), 7, vi)) continue;
         float acc[8];
         if constexpr (RC > 0) {
             uint4 gv[RC];
@@ -649,6 +706,10 @@ __global__ void __launch_bounds__(kThreads)
     OwnerCursor oc(vi, a.S8);
     for (; vi < a.v1; vi += stride) {
         oc.seek(vi);
+        if (!ZB_IN(vi >= a.v0 && oc.o < static_cast<uint32_t>(R) && vi - oc.base < a.S8 && a.acc[oc.o] &&
+                       ptrs_ok(a.g, R),
+                   8, vi))
+            continue;
         float acc[8];
         if constexpr (RC > 0) {
             uint4 gv[RC];
@@ -682,13 +743,16 @@ __global__ void __launch_bounds__(kThreads)
     if (tid < nhead + ntail) {
         const int64_t i = tid < nhead ? a.lo + tid : a.tail_begin + (tid - nhead);
         const int64_t o = i / a.S;
-        float s = H::one(ld_grad1(reinterpret_cast<const uint16_t*>(a.g[0]) + i));
-        for (int r = 1; r < R; ++r)
-            s = __fadd_rn(s, H::one(ld_grad1(reinterpret_cast<const uint16_t*>(a.g[r]) + i)));
-        float* dst = a.acc[o] + (i - o * a.S);
-        if constexpr (ACCUM) s = __fadd_rn(*dst, s);
-        bad |= nonfinite(s);
-        *dst = s;
+        // a guarded block, not a return: every thread must reach the barrier below
+        if (ZB_IN(i >= a.lo && i < a.hi && o < R && a.acc[o] && ptrs_ok(a.g, R), 9, i)) {
+            float s = H::one(ld_grad1(reinterpret_cast<const uint16_t*>(a.g[0]) + i));
+            for (int r = 1; r < R; ++r)
+                s = __fadd_rn(s, H::one(ld_grad1(reinterpret_cast<const uint16_t*>(a.g[r]) + i)));
+            float* dst = a.acc[o] + (i - o * a.S);
+            if constexpr (ACCUM) s = __fadd_rn(*dst, s);
+            bad |= nonfinite(s);
+            *dst = s;
+        }
     }
     if (__syncthreads_or(bad ? 1 : 0) && threadIdx.x == 0) atomicOr(&a.st->flag, 1u);
 }
@@ -704,6 +768,7 @@ __global__ void __launch_bounds__(kThreads)
 
 struct GatherManyArgs {
     int32_t nl;
+    int32_t R;
     int64_t S;
     uint32_t S8;
     uint32_t total_slots;
@@ -758,6 +823,9 @@ __global__ void __launch_bounds__(kThreads) gather_many_kernel(const __grid_cons
             if (al && e0 + 8 <= n) {
                 const uint32_t vi = static_cast<uint32_t>((lo + e0) >> 3);
                 oc.seek(vi);
+                if (!ZB_IN(oc.o < static_cast<uint32_t>(a.R) && vi - oc.base < a.S8 && a.param[cur][oc.o] && out,
+                           10, vi))
+                    continue;
                 q[u] = ld_grad(reinterpret_cast<const uint4*>(a.param[cur][oc.o]) + (vi - oc.base));
                 dst[u] = out + e0;
             } else {
@@ -765,6 +833,7 @@ __global__ void __launch_bounds__(kThreads) gather_many_kernel(const __grid_cons
                 for (int64_t e = e0; e < e1; ++e) {
                     const int64_t i = lo + e;
                     const int64_t o = i / a.S;
+                    if (!ZB_IN(e >= 0 && o < a.R && i - o * a.S < a.S && a.param[cur][o] && out, 11, i)) continue;
                     out[e] = ld_grad1(a.param[cur][o] + (i - o * a.S));
                 }
             }
@@ -1036,6 +1105,7 @@ cudaError_t launch_gather_many(int32_t R, int64_t S, int nl, const int64_t* lo, 
                                cudaStream_t s, int max_sms) {
     GatherManyArgs a;
     a.nl = nl;
+    a.R = R;
     a.S = S;
     a.S8 = static_cast<uint32_t>(S / 8);
     a.st = st;
@@ -1071,3 +1141,33 @@ int step_grid_cap(int device) {
 }
 
 }  // namespace zb
+
+extern "C" zero_status zero_debug_bounds(int64_t* count, int64_t* first_site, int64_t* first_index,
+                                         int32_t reset) {
+    if (!count || !first_site || !first_index)
+        return zb_fail(ZERO_ERR_INVALID_ARG, "zero_debug_bounds: NULL output");
+#ifdef ZERO_DEBUG_BOUNDS
+    unsigned long long c = 0, f = 0;
+    cudaError_t e = cudaDeviceSynchronize();
+    if (e == cudaSuccess) e = cudaMemcpyFromSymbol(&c, zb::g_bounds_count, sizeof c);
+    if (e == cudaSuccess) e = cudaMemcpyFromSymbol(&f, zb::g_bounds_first, sizeof f);
+    if (e == cudaSuccess && reset) {
+        const unsigned long long zero = 0;
+        e = cudaMemcpyToSymbol(zb::g_bounds_count, &zero, sizeof zero);
+        if (e == cudaSuccess) e = cudaMemcpyToSymbol(zb::g_bounds_first, &zero, sizeof zero);
+    }
+    if (e != cudaSuccess) {
+        cudaGetLastError();
+        return zb_fail(ZERO_ERR_CUDA, std::string("zero_debug_bounds: ") + cudaGetErrorString(e));
+    }
+    *count = static_cast<int64_t>(c);
+    *first_site = static_cast<int64_t>(f >> 48);
+    *first_index = static_cast<int64_t>(f & 0xffffffffffffull);
+#else
+    (void)reset;
+    *count = -1;  // the release build carries no checks
+    *first_site = 0;
+    *first_index = 0;
+#endif
+    return ZERO_OK;
+}
