@@ -1,7 +1,6 @@
 """Pins for the oracle's half-format casts: torch's CPU casts are the library
 routine these must reduce to (round-to-nearest-even, gradual underflow,
 overflow to infinity)."""
-import os
 
 import numpy as np
 import pytest
