@@ -174,14 +174,14 @@ def _stream(s):
 
 def zero_plan(numels, layer_ids=None, R=1, dtype=ZERO_BF16, tensor_align=8, bucket_elems=0):
     """Returns an opaque plan handle (int). Free with zero_plan_destroy."""
+    import numpy as np
     n = len(numels)
-    nb = (C.c_int64 * max(n, 1))(*[int(x) for x in numels])
-    lid = None
-    if layer_ids is not None:
-        lid = (C.c_int32 * max(n, 1))(*[int(x) for x in layer_ids])
+    nb = np.ascontiguousarray(numels if n else [0], dtype=np.int64)
+    lid = None if layer_ids is None else np.ascontiguousarray(layer_ids if n else [0], dtype=np.int32)
     cfg = zero_plan_config(R, dtype, tensor_align, 0, bucket_elems)
     out = C.c_void_p()
-    _check(_lib.zero_plan(nb, lid, n, C.byref(cfg), C.byref(out)))
+    _check(_lib.zero_plan(nb.ctypes.data, None if lid is None else lid.ctypes.data, n, C.byref(cfg),
+                          C.byref(out)))
     return out.value
 
 
