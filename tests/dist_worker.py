@@ -74,7 +74,7 @@ def check_accumulate_and_clip(rank, world):
     """Two-pass steps over accumulated micro-batches and fused steps, with
     global-norm clipping, against the oracle's step_ex."""
     numels = [50_001, 77, 3000]
-    dz = DistributedZero(numels, None, Z.ZERO_BF16, Z.ZERO_SCALE_NONE, accumulate=True)
+    dz = DistributedZero(numels, None, Z.ZERO_BF16, Z.ZERO_SCALE_NONE, bucket_elems=20_000, accumulate=True)
     wl = synth.custom_workload(numels, world, Z.ZERO_BF16, Z.ZERO_SCALE_NONE, 1.0, 1000, sigma=1e-2,
                                index=56)
     lay = O.Layout(numels, world, 8)
@@ -124,6 +124,32 @@ def check_accumulate_and_clip(rank, world):
         flat[idx] = ost.master
         mine = dz.current("master").cpu().numpy()
         assert np.array_equal(mine.view(np.uint32), flat[rank * S:(rank + 1) * S].view(np.uint32)), step
+
+    def check_master(step):
+        flat = np.zeros(dz.plan.T, np.float32)
+        flat[idx] = ost.master
+        mine = dz.current("master").cpu().numpy()
+        assert np.array_equal(mine.view(np.uint32), flat[rank * S:(rank + 1) * S].view(np.uint32)), step
+
+    # overlapped with a backward pass: each tensor's gradients are written on
+    # the compute stream in reverse order and reported; buckets reduce-scatter
+    # on the communication stream as they complete
+    starts = np.concatenate([[0], np.cumsum(numels)[:-1]])
+    for step in range(7, 10):
+        clip = 1e-3 if step == 8 else 0.0
+        micro = [np.stack([u16(synth.flat_grads(wl, step * 10 + mu, r, 1.0, "cpu")) for r in range(world)])
+                 for mu in range(2)]
+        for mu, g in enumerate(micro):
+            dev = torch.from_numpy(g[rank].view(np.int16)).cuda()
+            for k in reversed(range(len(numels))):
+                off, n, st = int(lay.offsets[k]), numels[k], int(starts[k])
+                dz.grads.view(torch.int16)[off:off + n].copy_(dev[st:st + n])
+                dz.grads_ready(k)
+            dz.join()
+        dz.step_accumulated(hp, max_grad_norm=clip)
+        O.step_ex(ost, np.stack(micro), ohp, fsm, 2.0, clip)
+        assert dz.loss_scale()["t"] == fsm.t, step
+        check_master(step)
     dz.close()
 
 

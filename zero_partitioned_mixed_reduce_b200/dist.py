@@ -23,6 +23,16 @@ accumulator (zero_reduce_scatter_shard, between two one-element
 all-reduces that order the peers' writes and reads), and
 step_accumulated() steps from it.
 
+Overlap with backward: grads_ready(first, count) reports tensors whose
+gradients the compute stream has written. When a bucket is complete, a
+one-element all-reduce (which every rank reaches only after writing that
+bucket) and the bucket's sharded reduce-scatter are queued on a
+high-priority communication stream, so the reduction runs while backward
+continues; join() ends the micro-batch with one more all-reduce, after which
+no peer still reads this rank's gradients, and makes the compute stream wait
+for the communication stream. Every rank reports the same tensors in the
+same order, so the ranks issue the same collectives in the same order.
+
 ZeRO-3 layer gathers read the peers' parameter shards the same way.
 Argument marshalling only; the arithmetic runs in libzero_b200.so. The
 loads from peer memory are plain loads or bulk copies without multicast.
@@ -77,6 +87,7 @@ class DistributedZero:
                                           v=own(self.v[k]), param=own(self.param[k]))
                                      for k in range(sets)], self.acc_list)
         self.micro = 0
+        self.comm = None
         self.gather_handle = Z.StateHandle([dict(master=[None] * R, m=[None] * R, v=[None] * R,
                                                  param=self.param_ptrs[k]) for k in range(sets)])
         self.ctx = Z.zero_ctx_create(self.plan.handle, mode, init_scale, growth_interval)
@@ -132,6 +143,43 @@ class DistributedZero:
         Z.zero_reduce_scatter_shard(self.ctx, -1, self.grad_ptrs, self.acc_list, self.rank, self.rank + 1,
                                     Z.ZERO_RS_ACCUMULATE if self.micro else 0, stream)
         dist.all_reduce(self.token, group=self.group)  # every peer has read this rank's replica
+        self.micro += 1
+
+    def grads_ready(self, first, count=1):
+        """Tensors first .. first+count-1 of this micro-batch have their
+        gradients written in self.grads (by work on the current stream)."""
+        assert self.acc is not None, "construct with accumulate=True"
+        if self.comm is None:
+            self.comm = torch.cuda.Stream(priority=-1)
+            self.bucket_size = [0] * len(self.plan.buckets)
+            for b in self.plan.tensor_bucket:
+                self.bucket_size[b] += 1
+            self.bucket_seen = [0] * len(self.plan.buckets)
+            self.comm_token = torch.zeros(1, dtype=torch.float32, device=self.token.device)
+        compute = torch.cuda.current_stream()
+        for k in range(first, first + count):
+            b = self.plan.tensor_bucket[k]
+            self.bucket_seen[b] += 1
+            if self.bucket_seen[b] != self.bucket_size[b]:
+                continue
+            ready = torch.cuda.Event()
+            ready.record(compute)
+            with torch.cuda.stream(self.comm):
+                self.comm.wait_event(ready)
+                dist.all_reduce(self.comm_token, group=self.group)  # every rank wrote bucket b
+                Z.zero_reduce_scatter_shard(self.ctx, b, self.grad_ptrs, self.acc_list, self.rank,
+                                            self.rank + 1, Z.ZERO_RS_ACCUMULATE if self.micro else 0,
+                                            self.comm)
+
+    def join(self):
+        """End of a micro-batch's backward: every bucket must have been
+        reported. The compute stream then waits for the reductions."""
+        assert self.comm is not None and all(a == n for a, n in zip(self.bucket_seen, self.bucket_size)), \
+            "every tensor must be reported before join()"
+        with torch.cuda.stream(self.comm):
+            dist.all_reduce(self.comm_token, group=self.group)  # no peer reads this rank's grads any more
+        torch.cuda.current_stream().wait_stream(self.comm)
+        self.bucket_seen = [0] * len(self.bucket_seen)
         self.micro += 1
 
     def step_accumulated(self, hp, grad_divisor=None, max_grad_norm=0.0, stream=None):

@@ -19,15 +19,17 @@ class Plan:
         info = Z.zero_plan_get_info(self.handle)
         self.__dict__.update(info)
         self.numels = [int(n) for n in numels]
-        self.offsets = [Z.zero_plan_tensor(self.handle, k)[0] for k in range(info["n_tensors"])]
+        tensors = [Z.zero_plan_tensor(self.handle, k) for k in range(info["n_tensors"])]
+        self.offsets = [t[0] for t in tensors]
+        self.tensor_bucket = [t[2] for t in tensors]
         self.buckets = [Z.zero_plan_bucket(self.handle, b) for b in range(info["n_buckets"])]
         self.layers = [Z.zero_plan_layer(self.handle, l) for l in range(info["n_layers"])]
 
     def __del__(self):
         h = getattr(self, "handle", None)
-        if h:
-            Z.zero_plan_destroy(h)
-            self.handle = None
+        if h and Z is not None and getattr(Z, "zero_plan_destroy", None) is not None:
+            Z.zero_plan_destroy(h)  # (at interpreter exit the module may already be gone)
+        self.handle = None
 
     def pack(self, flat_unpadded, out=None, fill=0):
         """Place an unpadded concatenation of the tensors into the padded flat
