@@ -62,6 +62,21 @@ def main():
         dz.gather_layer(l, out)
         torch.cuda.synchronize()
         assert np.array_equal(u16(out), pflat[lo:hi]), l
+    # the same layers bucketed, and through the look-ahead ring
+    outs = [torch.empty(hi - lo, dtype=torch.float16, device="cuda") for lo, hi in lay.layers]
+    dz.gather_layers(0, outs)
+    torch.cuda.synchronize()
+    for l, (lo, hi) in enumerate(lay.layers):
+        assert np.array_equal(u16(outs[l]), pflat[lo:hi]), l
+    biggest = max(hi - lo for lo, hi in lay.layers)
+    bufs = [torch.empty(biggest + 8, dtype=torch.float16, device="cuda") for _ in range(2)]
+    by_addr = {b.data_ptr(): b for b in bufs}
+    dz.prefetch_begin(bufs, 1, 1)
+    for l, (lo, hi) in enumerate(lay.layers):
+        buf = by_addr[dz.layer_acquire(l)]
+        torch.cuda.synchronize()
+        assert np.array_equal(u16(buf[:hi - lo]), pflat[lo:hi]), l
+        dz.layer_release(l)
     dz.close()
     check_accumulate_and_clip(rank, world)
     dist.barrier()

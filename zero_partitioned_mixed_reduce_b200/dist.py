@@ -199,6 +199,24 @@ class DistributedZero:
         """ZeRO-3 all-gather of one layer from every rank's parameter shard."""
         Z.zero_gather_layer(self.ctx, layer, self.gather_handle, out, stream)
 
+    def gather_layers(self, first, outs, stream=None):
+        """ZeRO-3 all-gather of consecutive layers first, first+1, ... in one launch."""
+        Z.zero_gather_layers(self.ctx, first, outs, self.gather_handle, stream)
+
+    def prefetch_begin(self, bufs, depth, direction=1, stream=None):
+        """Start a pass of look-ahead ZeRO-3 gathers into the ring `bufs`
+        (the scheduler's communication stream reads every rank's shard);
+        then acquire / release each layer in order. The step that produced
+        the parameters has been committed on every rank, so their shards
+        are final."""
+        Z.zero_prefetch_begin(self.ctx, self.gather_handle, bufs, depth, direction, stream)
+
+    def layer_acquire(self, layer, stream=None):
+        return Z.zero_layer_acquire(self.ctx, layer, stream)
+
+    def layer_release(self, layer, stream=None):
+        Z.zero_layer_release(self.ctx, layer, stream)
+
     def loss_scale(self):
         return Z.zero_loss_scale(self.ctx)
 
