@@ -78,6 +78,8 @@ def parse_args(argv=None):
                     help="time the bucketed reduce-scatter against bucket size instead")
     ap.add_argument("--rs-sizes", default="0,1000000,5000000,25000000,50000000,100000000,200000000",
                     help="bucket sizes (elements; 0: one bucket for the whole model) for --rs-sweep")
+    ap.add_argument("--dist", action="store_true",
+                    help="the real multi-GPU ZeRO step over the job's GPUs (DistributedZero) instead")
     ap.add_argument("--graph", action="store_true",
                     help="capture the step and the gathers once into CUDA graphs and replay them")
     ap.add_argument("--first-tensors", type=int, default=0,
@@ -803,6 +805,110 @@ def run_rs_sweep(args, world, rank, local):
         print(json.dumps(out), flush=True)
 
 
+def run_dist(args, world, rank, local):
+    """The real multi-GPU ZeRO step (DistributedZero): the workload's tensors
+    sharded over the N GPUs of the job, each rank owning one shard and reading
+    its peers' gradient replicas over NVLink inside the fused step, then the
+    ZeRO-3 gathers of every layer from every rank's shard. Strong scaling:
+    the model is fixed, N ranks share it. Each rank writes its own replica."""
+    import socket
+    import torch.distributed as dist
+    from zero_partitioned_mixed_reduce_b200 import synth
+    from zero_partitioned_mixed_reduce_b200.dist import DistributedZero
+    if not torch.cuda.is_available():
+        print(json.dumps({"error": "no CUDA device"}))
+        sys.exit(1)
+    if not dist.is_initialized():  # one process: a group of one
+        with socket.socket() as sk:
+            sk.bind(("127.0.0.1", 0))
+            port = sk.getsockname()[1]
+        os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
+        os.environ.setdefault("MASTER_PORT", str(port))
+        dist.init_process_group("nccl", rank=0, world_size=1, timeout=datetime.timedelta(seconds=300))
+    N = dist.get_world_size()
+    wl = synth.workload(args.workload)
+    dz = DistributedZero(wl["numels"], wl["layer_ids"], wl["dtype"], wl["mode"], wl["init_scale"],
+                         wl["interval"], 8, wl["bucket_elems"])
+    plan = dz.plan
+    half = {0: torch.bfloat16, 1: torch.float16}[wl["dtype"]]
+    x = torch.cat([synth.tensor_master(n, wl["index"], k, "cuda") for k, n in enumerate(wl["numels"])])
+    dz.load(plan.pack(x), plan.pack(x.to(half)))
+    del x
+    scale = wl["init_scale"] if wl["mode"] != synth.NONE else 1.0
+    for k, (n, off) in enumerate(zip(wl["numels"], plan.offsets)):
+        dz.grads[off:off + n] = synth.tensor_grads(n, wl["dist"], wl["sigma"], scale, wl["dtype"], wl["index"],
+                                                   1, dz.rank, k, "cuda")
+    torch.cuda.synchronize()
+    # ZeRO-3 gathers of every layer, bucketed as in the single-GPU step
+    buckets, first, size, offs = [], 0, 0, []
+    for l, (lo, hi) in enumerate(plan.layers):
+        n = hi - lo
+        if offs and (size + n > args.gather_bucket or len(offs) == 64):
+            buckets.append((first, offs, size))
+            first, size, offs = l, 0, []
+        offs.append(size)
+        size += (n + 7) // 8 * 8
+    buckets.append((first, offs, size))
+    layer_buf = torch.empty(max(b[2] for b in buckets), dtype=half, device="cuda")
+    outs = [[layer_buf.data_ptr() + 2 * o for o in offs] for _, offs, _ in buckets]
+    hp = wl["hp"]
+    stream = torch.cuda.current_stream()
+
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        dz.step(hp)
+        if ev is not None:
+            ev[1].record(stream)
+        for (f, _, _), o in zip(buckets, outs):
+            dz.gather_layers(f, o)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    f0 = dz.loss_scale()
+    K = args.steps
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(local)
+    clocks.start()
+    dist.barrier()
+    torch.cuda.synchronize()
+    start.record(stream)
+    for i in range(K):
+        step(evs[i])
+    end.record(stream)
+    torch.cuda.synchronize()
+    dist.barrier()
+    clk = clocks.stop()
+    f1 = dz.loss_scale()
+    assert f1["last_overflow"] == 0 and f1["t"] == f0["t"] + K
+    ms, units = aggregate(start.elapsed_time(end), float(plan.P) * K / N, N)
+    step_ms, _ = aggregate(statistics.mean(e0.elapsed_time(e1) for e0, e1 in evs), 0.0, N)
+    S = plan.S
+    kbytes = (2 * N + 26) * S  # one rank's fused launch: N replica slices, its own state
+    peak, peak_src = hbm_peak()
+    out = {
+        "mode": "distributed", "metric": METRIC, "value": units / (ms * 1e-3), "unit": "params/s",
+        "n_gpus": N, "steps": K, "warmup": args.warmup, "ms_per_step": ms / K, "higher_is_better": True,
+        "scaling": "strong", "dtype": "f32", "data": "synthetic",
+        "config": {"workload": f"{args.workload}: {len(wl['numels'])} tensors, P={plan.P}, sharded over "
+                               f"{N} rank(s), one per GPU, {'fp16' if wl['dtype'] else 'bf16'} grads, "
+                               f"loss scale mode {wl['mode']}",
+                   "R": N, "P": plan.P, "S": S,
+                   "parallelism": f"{N} GPU(s), one shard each (DistributedZero: fused step reading the "
+                                  "peers' replicas over NVLink, NCCL for 4-16 byte all-reduces)",
+                   "gather": f"{len(buckets)} bucketed launches per step over every rank's shard"},
+        "step_ms_max_over_ranks": step_ms,
+        "per_rank_step_bytes": kbytes, "per_rank_nvlink_bytes": 2 * (N - 1) * S,
+        "per_rank_step_gbs": kbytes / (step_ms * 1e-3) / 1e9, "peak": peak,
+        "peak_source": f"{peak_src} hbm_gbs", "clocks": clk,
+    }
+    dz.close()
+    if rank == 0:
+        print(json.dumps(out), flush=True)
+
+
 def run_offload(args, world, rank, local):
     """ZeRO-Offload on the workload: per step the GPU runs a synthetic
     forward/backward (bf16 GEMMs of 6 * tokens * P flops) and reduce-scatters
@@ -971,11 +1077,13 @@ def main(argv=None):
             run_offload(args, world, rank, local)
         elif args.rs_sweep:
             run_rs_sweep(args, world, rank, local)
+        elif args.dist:
+            run_dist(args, world, rank, local)
         else:
             run_ours(args, world, rank, local)
     finally:
-        if world > 1:
-            import torch.distributed as dist
+        import torch.distributed as dist
+        if dist.is_available() and dist.is_initialized():
             dist.destroy_process_group()
 
 

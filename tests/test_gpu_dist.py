@@ -29,3 +29,18 @@ def test_distributed_zero_matches_oracle():
     r = subprocess.run(cmd, capture_output=True, text=True, env=env, cwd=ROOT)
     assert r.returncode == 0, (r.stdout[-3000:], r.stderr[-3000:])
     assert "ok" in r.stdout
+
+
+def test_bench_distributed_mode():
+    # bench.py --dist: the real multi-GPU step (at one rank here) prints one JSON line
+    import json
+    env = dict(os.environ, NCCL_NVLS_ENABLE="0")
+    cmd = ["timeout", "-k", "30", "600", sys.executable, "-m", "torch.distributed.run", "--nnodes=1",
+           "--nproc-per-node=1", "--master-addr", "127.0.0.1", "--master-port", str(free_port()),
+           os.path.join(ROOT, "bench.py"), "--dist", "--workload", "gpt2s", "--steps", "3", "--warmup", "3"]
+    r = subprocess.run(cmd, capture_output=True, text=True, env=env, cwd=ROOT)
+    assert r.returncode == 0, (r.stdout[-3000:], r.stderr[-3000:])
+    line = [ln for ln in r.stdout.splitlines() if ln.startswith("{")][-1]
+    out = json.loads(line)
+    assert out["mode"] == "distributed" and out["n_gpus"] == 1 and out["scaling"] == "strong"
+    assert out["value"] > 0 and out["config"]["R"] == 1
