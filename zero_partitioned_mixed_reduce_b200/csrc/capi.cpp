@@ -286,130 +286,6 @@ extern "C" zero_status zero_step(zero_ctx_t* ctx, const zero_adamw* hp, const ze
     return zero_step_ex(ctx, hp, state, grads, nullptr, stream);
 }
 
-extern "C" zero_status zero_step_ex(zero_ctx_t* ctx, const zero_adamw* hp, const zero_state* state,
-                                    const void* const* grads, const zero_step_opts* opts,
-                                    void* stream) {
-    const char* where = "zero_step";
-    zero_step_opts o{1.0, 0.0, 0, 0};
-    if (opts) o = *opts;
-    if (!(o.grad_divisor >= 1.0) || !std::isfinite(o.grad_divisor) || !(o.max_grad_norm >= 0.0) ||
-        !std::isfinite(o.max_grad_norm) || o.reserved != 0)
-        return zb_fail(ZERO_ERR_INVALID_ARG,
-                       "zero_step_ex: need grad_divisor >= 1, finite max_grad_norm >= 0, reserved 0");
-    if (o.flags & ~static_cast<int64_t>(ZERO_STEP_ADD_ACC))
-        return zb_fail(ZERO_ERR_INVALID_ARG, "zero_step_ex: unknown flags");
-    const bool add_acc = (o.flags & ZERO_STEP_ADD_ACC) != 0;
-    if (add_acc && (grads == nullptr || o.max_grad_norm > 0.0))
-        return zb_fail(ZERO_ERR_INVALID_ARG,
-                       "zero_step_ex: ZERO_STEP_ADD_ACC needs the fused path (grads) and no clipping");
-    if (!ctx || !hp) return zb_fail(ZERO_ERR_INVALID_ARG, "zero_step: NULL ctx or hyper-parameters");
-    zero_status s = check_device(ctx, where);
-    if (s != ZERO_OK) return s;
-    if (!(hp->lr >= 0.0) || !(hp->beta1 >= 0.0 && hp->beta1 < 1.0) ||
-        !(hp->beta2 >= 0.0 && hp->beta2 < 1.0) || !(hp->eps > 0.0) || !(hp->weight_decay >= 0.0) ||
-        !std::isfinite(hp->lr) || !std::isfinite(hp->weight_decay))
-        return zb_fail(ZERO_ERR_INVALID_ARG,
-                       "zero_step: need lr >= 0, 0 <= beta < 1, eps > 0, weight_decay >= 0");
-    int sets = 1;
-    if ((s = check_state(ctx, state, where, &sets, false)) != ZERO_OK) return s;
-    const bool fused = grads != nullptr;
-    if (add_acc && (s = check_ranks(state->acc, ctx->R, 32, where, "acc")) != ZERO_OK) return s;
-    if (fused) {
-        if ((s = check_ranks(grads, ctx->R, 16, where, "grads")) != ZERO_OK) return s;
-        if (sets == 1 && ctx->cfg.mode == ZERO_SCALE_DYNAMIC)
-            return zb_fail(ZERO_ERR_INVALID_ARG,
-                           "zero_step: a fused step with dynamic loss scaling needs state set 1 "
-                           "(ping-pong) so that a skipped step can be undone; or use the two-pass path");
-    } else {
-        if ((s = check_ranks(state->acc, ctx->R, 32, where, "acc")) != ZERO_OK) return s;
-    }
-    if (sets == 1 && ctx->two_sets)
-        return zb_fail(ZERO_ERR_STATE,
-                       "zero_step: the current model may live in state set 1; pass both sets");
-
-    cudaStream_t cs = static_cast<cudaStream_t>(stream);
-    if ((s = ensure_powtab(ctx, hp->beta1, hp->beta2, ctx->t_bound + 1, cs)) != ZERO_OK) return s;
-
-    zb::StepParams sp;
-    sp.R = ctx->R;
-    sp.dtype = ctx->dtype;
-    sp.mode = ctx->cfg.mode;
-    sp.pingpong = sets == 2 ? 1 : 0;
-    sp.S8 = static_cast<uint32_t>(ctx->S / 8);
-    sp.T8 = static_cast<uint32_t>(ctx->T / 8);
-    sp.dec = static_cast<float>(1.0 - hp->lr * hp->weight_decay);
-    sp.b1f = static_cast<float>(hp->beta1);
-    sp.omb1 = static_cast<float>(1.0 - hp->beta1);
-    sp.b2f = static_cast<float>(hp->beta2);
-    sp.omb2 = static_cast<float>(1.0 - hp->beta2);
-    sp.epsf = static_cast<float>(hp->eps);
-    sp.lr = hp->lr;
-    sp.divisor = o.grad_divisor;
-    sp.max_norm = o.max_grad_norm;
-    sp.clip = o.max_grad_norm > 0.0 ? 1 : 0;
-    sp.add_acc = add_acc ? 1 : 0;
-    sp.interval = ctx->cfg.growth_interval;
-    sp.growth = ctx->cfg.growth_factor;
-    sp.backoff = ctx->cfg.backoff_factor;
-    sp.min_scale = ctx->cfg.min_scale;
-    sp.st = ctx->st;
-    sp.partials = ctx->partials;
-    sp.powtab = ctx->powtab;
-    sp.powtab_len = ctx->powtab_len;
-    sp.grid_cap = ctx->grid_cap;
-    sp.obeg = 0;
-    sp.oend = ctx->R;
-    if (fused) sp.drop_tile = ctx->drop_tile;
-
-    zb::RankPtrs p;
-    fill_state_ptrs(ctx, state, sets, &p);
-    for (int r = 0; r < ctx->R; ++r) {
-        p.g[r] = fused ? grads[r] : nullptr;
-        p.acc[r] = (!fused || add_acc) ? state->acc[r] : nullptr;
-    }
-    cudaError_t e = cudaSuccess;
-    // clipping needs the global norm before any element is updated: one
-    // read-only pass over the accumulators, or over the replicas when fused
-    if (sp.clip) e = fused ? zb::launch_grad_norm(sp, p, cs) : zb::launch_clip_norm(sp, p, cs);
-    if (e == cudaSuccess)
-        e = fused ? zb::launch_fused_step(sp, p, cs) : zb::launch_step_from_acc(sp, p, cs);
-    if (e != cudaSuccess) return cuda_fail(where, e);
-    ctx->t_bound += 1;
-    if (fused) ctx->drop_tile = 0xffffffffu;
-    if (sp.pingpong) ctx->two_sets = true;
-    return ZERO_OK;
-}
-
-namespace {
-
-// Shard-range variant of check_state: only owners [lo, hi) need pointers.
-zero_status check_state_range(const zero_ctx_t* ctx, const zero_state* st, int lo, int hi,
-                              const char* where, int* sets) {
-    if (!st) return zb_fail(ZERO_ERR_INVALID_ARG, std::string(where) + ": state is NULL");
-    const bool any1 = st->master[1] || st->m[1] || st->v[1] || st->param[1];
-    const bool all1 = st->master[1] && st->m[1] && st->v[1] && st->param[1];
-    if (any1 && !all1)
-        return zb_fail(ZERO_ERR_INVALID_ARG, std::string(where) + ": state set 1 must be complete or absent");
-    for (int k = 0; k < (all1 ? 2 : 1); ++k) {
-        if (!st->master[k] || !st->m[k] || !st->v[k] || !st->param[k])
-            return zb_fail(ZERO_ERR_INVALID_ARG, std::string(where) + ": NULL state array");
-        for (int r = lo; r < hi; ++r) {
-            const void* f[3] = {st->master[k][r], st->m[k][r], st->v[k][r]};
-            for (const void* q : f) {
-                if (!q) return zb_fail(ZERO_ERR_INVALID_ARG, std::string(where) + ": NULL state pointer");
-                if (!aligned(q, 32)) return zb_fail(ZERO_ERR_ALIGN, std::string(where) + ": fp32 state misaligned");
-            }
-            if (!st->param[k][r]) return zb_fail(ZERO_ERR_INVALID_ARG, std::string(where) + ": NULL param pointer");
-            if (!aligned(st->param[k][r], 16)) return zb_fail(ZERO_ERR_ALIGN, std::string(where) + ": param misaligned");
-        }
-    }
-    *sets = all1 ? 2 : 1;
-    (void)ctx;
-    return ZERO_OK;
-}
-
-}  // namespace
-
 namespace {
 
 // Parameters shared by the sharded calls (everything but the AdamW hyper-parameters).
@@ -461,7 +337,135 @@ zero_status check_owned_acc(const zero_ctx_t* ctx, float* const* acc, int32_t lo
     return ZERO_OK;
 }
 
+// Options of zero_step_ex / zero_step_shard_ex, validated; *out receives them.
+zero_status check_step_opts(const zero_step_opts* opts, bool fused, const char* where, zero_step_opts* out) {
+    zero_step_opts o{1.0, 0.0, 0, 0};
+    if (opts) o = *opts;
+    if (!(o.grad_divisor >= 1.0) || !std::isfinite(o.grad_divisor) || !(o.max_grad_norm >= 0.0) ||
+        !std::isfinite(o.max_grad_norm) || o.reserved != 0)
+        return zb_fail(ZERO_ERR_INVALID_ARG,
+                       std::string(where) + ": need grad_divisor >= 1, finite max_grad_norm >= 0, reserved 0");
+    if (o.flags & ~static_cast<int64_t>(ZERO_STEP_ADD_ACC))
+        return zb_fail(ZERO_ERR_INVALID_ARG, std::string(where) + ": unknown flags");
+    if ((o.flags & ZERO_STEP_ADD_ACC) && (!fused || o.max_grad_norm > 0.0))
+        return zb_fail(ZERO_ERR_INVALID_ARG,
+                       std::string(where) + ": ZERO_STEP_ADD_ACC needs the fused path (grads) and no clipping");
+    *out = o;
+    return ZERO_OK;
+}
+
+zero_status check_hp(const zero_adamw* hp, const char* where) {
+    if (!(hp->lr >= 0.0) || !(hp->beta1 >= 0.0 && hp->beta1 < 1.0) || !(hp->beta2 >= 0.0 && hp->beta2 < 1.0) ||
+        !(hp->eps > 0.0) || !(hp->weight_decay >= 0.0) || !std::isfinite(hp->lr) ||
+        !std::isfinite(hp->weight_decay) || !std::isfinite(hp->eps))
+        return zb_fail(ZERO_ERR_INVALID_ARG,
+                       std::string(where) + ": need finite lr >= 0, 0 <= beta < 1, eps > 0, weight_decay >= 0");
+    return ZERO_OK;
+}
+
+// Everything a step launch needs, for owners [owner_lo, owner_hi).
+zb::StepParams step_params(const zero_ctx_t* ctx, const zero_adamw* hp, const zero_step_opts& o, int sets,
+                           int32_t owner_lo, int32_t owner_hi, double* partial) {
+    zb::StepParams sp = shard_params(ctx, owner_lo, owner_hi, o.grad_divisor, partial);
+    sp.pingpong = sets == 2 ? 1 : 0;
+    sp.dec = static_cast<float>(1.0 - hp->lr * hp->weight_decay);
+    sp.b1f = static_cast<float>(hp->beta1);
+    sp.omb1 = static_cast<float>(1.0 - hp->beta1);
+    sp.b2f = static_cast<float>(hp->beta2);
+    sp.omb2 = static_cast<float>(1.0 - hp->beta2);
+    sp.epsf = static_cast<float>(hp->eps);
+    sp.lr = hp->lr;
+    sp.max_norm = o.max_grad_norm;
+    sp.clip = o.max_grad_norm > 0.0 ? 1 : 0;
+    sp.add_acc = (o.flags & ZERO_STEP_ADD_ACC) ? 1 : 0;
+    return sp;
+}
+
 }  // namespace
+
+extern "C" zero_status zero_step_ex(zero_ctx_t* ctx, const zero_adamw* hp, const zero_state* state,
+                                    const void* const* grads, const zero_step_opts* opts,
+                                    void* stream) {
+    const char* where = "zero_step";
+    const bool fused = grads != nullptr;
+    zero_step_opts o;
+    zero_status s = check_step_opts(opts, fused, "zero_step_ex", &o);
+    if (s != ZERO_OK) return s;
+    const bool add_acc = (o.flags & ZERO_STEP_ADD_ACC) != 0;
+    if (!ctx || !hp) return zb_fail(ZERO_ERR_INVALID_ARG, "zero_step: NULL ctx or hyper-parameters");
+    if ((s = check_device(ctx, where)) != ZERO_OK) return s;
+    if ((s = check_hp(hp, where)) != ZERO_OK) return s;
+    int sets = 1;
+    if ((s = check_state(ctx, state, where, &sets, false)) != ZERO_OK) return s;
+    if (add_acc && (s = check_ranks(state->acc, ctx->R, 32, where, "acc")) != ZERO_OK) return s;
+    if (fused) {
+        if ((s = check_ranks(grads, ctx->R, 16, where, "grads")) != ZERO_OK) return s;
+        if (sets == 1 && ctx->cfg.mode == ZERO_SCALE_DYNAMIC)
+            return zb_fail(ZERO_ERR_INVALID_ARG,
+                           "zero_step: a fused step with dynamic loss scaling needs state set 1 "
+                           "(ping-pong) so that a skipped step can be undone; or use the two-pass path");
+    } else {
+        if ((s = check_ranks(state->acc, ctx->R, 32, where, "acc")) != ZERO_OK) return s;
+    }
+    if (sets == 1 && ctx->two_sets)
+        return zb_fail(ZERO_ERR_STATE,
+                       "zero_step: the current model may live in state set 1; pass both sets");
+
+    cudaStream_t cs = static_cast<cudaStream_t>(stream);
+    if ((s = ensure_powtab(ctx, hp->beta1, hp->beta2, ctx->t_bound + 1, cs)) != ZERO_OK) return s;
+
+    zb::StepParams sp = step_params(ctx, hp, o, sets, 0, ctx->R, nullptr);
+    if (fused) sp.drop_tile = ctx->drop_tile;
+
+    zb::RankPtrs p;
+    fill_state_ptrs(ctx, state, sets, &p);
+    for (int r = 0; r < ctx->R; ++r) {
+        p.g[r] = fused ? grads[r] : nullptr;
+        p.acc[r] = (!fused || add_acc) ? state->acc[r] : nullptr;
+    }
+    cudaError_t e = cudaSuccess;
+    // clipping needs the global norm before any element is updated: one
+    // read-only pass over the accumulators, or over the replicas when fused
+    if (sp.clip) e = fused ? zb::launch_grad_norm(sp, p, cs) : zb::launch_clip_norm(sp, p, cs);
+    if (e == cudaSuccess)
+        e = fused ? zb::launch_fused_step(sp, p, cs) : zb::launch_step_from_acc(sp, p, cs);
+    if (e != cudaSuccess) return cuda_fail(where, e);
+    ctx->t_bound += 1;
+    if (fused) ctx->drop_tile = 0xffffffffu;
+    if (sp.pingpong) ctx->two_sets = true;
+    return ZERO_OK;
+}
+
+namespace {
+
+// Shard-range variant of check_state: only owners [lo, hi) need pointers.
+zero_status check_state_range(const zero_ctx_t* ctx, const zero_state* st, int lo, int hi,
+                              const char* where, int* sets) {
+    if (!st) return zb_fail(ZERO_ERR_INVALID_ARG, std::string(where) + ": state is NULL");
+    const bool any1 = st->master[1] || st->m[1] || st->v[1] || st->param[1];
+    const bool all1 = st->master[1] && st->m[1] && st->v[1] && st->param[1];
+    if (any1 && !all1)
+        return zb_fail(ZERO_ERR_INVALID_ARG, std::string(where) + ": state set 1 must be complete or absent");
+    for (int k = 0; k < (all1 ? 2 : 1); ++k) {
+        if (!st->master[k] || !st->m[k] || !st->v[k] || !st->param[k])
+            return zb_fail(ZERO_ERR_INVALID_ARG, std::string(where) + ": NULL state array");
+        for (int r = lo; r < hi; ++r) {
+            const void* f[3] = {st->master[k][r], st->m[k][r], st->v[k][r]};
+            for (const void* q : f) {
+                if (!q) return zb_fail(ZERO_ERR_INVALID_ARG, std::string(where) + ": NULL state pointer");
+                if (!aligned(q, 32)) return zb_fail(ZERO_ERR_ALIGN, std::string(where) + ": fp32 state misaligned");
+            }
+            if (!st->param[k][r]) return zb_fail(ZERO_ERR_INVALID_ARG, std::string(where) + ": NULL param pointer");
+            if (!aligned(st->param[k][r], 16)) return zb_fail(ZERO_ERR_ALIGN, std::string(where) + ": param misaligned");
+        }
+    }
+    *sets = all1 ? 2 : 1;
+    (void)ctx;
+    return ZERO_OK;
+}
+
+}  // namespace
+
 
 extern "C" zero_status zero_reduce_scatter_shard(zero_ctx_t* ctx, int64_t bucket, const void* const* grads,
                                                  float* const* acc, int32_t owner_lo, int32_t owner_hi,
@@ -533,35 +537,24 @@ extern "C" zero_status zero_step_shard_ex(zero_ctx_t* ctx, const zero_adamw* hp,
     const char* where = "zero_step_shard";
     if (!ctx || !hp || !partial)
         return zb_fail(ZERO_ERR_INVALID_ARG, "zero_step_shard: NULL ctx, hp or partial");
-    zero_step_opts o{1.0, 0.0, 0, 0};
-    if (opts) o = *opts;
-    if (!(o.grad_divisor >= 1.0) || !std::isfinite(o.grad_divisor) || !(o.max_grad_norm >= 0.0) ||
-        !std::isfinite(o.max_grad_norm) || o.reserved != 0)
-        return zb_fail(ZERO_ERR_INVALID_ARG,
-                       "zero_step_shard: need grad_divisor >= 1, finite max_grad_norm >= 0, reserved 0");
-    if (o.flags & ~static_cast<int64_t>(ZERO_STEP_ADD_ACC))
-        return zb_fail(ZERO_ERR_INVALID_ARG, "zero_step_shard: unknown flags");
+    const bool fused = grads != nullptr;
+    zero_step_opts o;
+    zero_status s = check_step_opts(opts, fused, where, &o);
+    if (s != ZERO_OK) return s;
     const bool add_acc = (o.flags & ZERO_STEP_ADD_ACC) != 0;
     const bool clip = o.max_grad_norm > 0.0;
-    if (add_acc && (grads == nullptr || clip))
-        return zb_fail(ZERO_ERR_INVALID_ARG,
-                       "zero_step_shard: ZERO_STEP_ADD_ACC needs the fused path (grads) and no clipping");
     if (clip && !global_norm_sq)
         return zb_fail(ZERO_ERR_INVALID_ARG,
                        "zero_step_shard: clipping needs global_norm_sq (the cross-rank sum of the "
                        "zero_grad_norm_shard partials)");
     if (global_norm_sq && !aligned(global_norm_sq, 8))
         return zb_fail(ZERO_ERR_ALIGN, "zero_step_shard: global_norm_sq not 8-byte aligned");
-    zero_status s = check_device(ctx, where);
-    if (s != ZERO_OK) return s;
+    if ((s = check_device(ctx, where)) != ZERO_OK) return s;
     if ((s = check_owner_range(ctx, owner_lo, owner_hi, where)) != ZERO_OK) return s;
     if (!aligned(partial, 8)) return zb_fail(ZERO_ERR_ALIGN, "zero_step_shard: partial not 8-byte aligned");
-    if (!(hp->lr >= 0.0) || !(hp->beta1 >= 0.0 && hp->beta1 < 1.0) || !(hp->beta2 >= 0.0 && hp->beta2 < 1.0) ||
-        !(hp->eps > 0.0) || !(hp->weight_decay >= 0.0))
-        return zb_fail(ZERO_ERR_INVALID_ARG, "zero_step_shard: bad hyper-parameters");
+    if ((s = check_hp(hp, where)) != ZERO_OK) return s;
     int sets = 1;
     if ((s = check_state_range(ctx, state, owner_lo, owner_hi, where, &sets)) != ZERO_OK) return s;
-    const bool fused = grads != nullptr;
     if (fused && (s = check_all_grads(ctx, grads, where)) != ZERO_OK) return s;
     if ((!fused || add_acc) && (s = check_owned_acc(ctx, state->acc, owner_lo, owner_hi, where)) != ZERO_OK)
         return s;
@@ -571,18 +564,7 @@ extern "C" zero_status zero_step_shard_ex(zero_ctx_t* ctx, const zero_adamw* hp,
         return zb_fail(ZERO_ERR_STATE, "zero_step_shard: the current model may live in state set 1");
     cudaStream_t cs = static_cast<cudaStream_t>(stream);
     if ((s = ensure_powtab(ctx, hp->beta1, hp->beta2, ctx->t_bound + 1, cs)) != ZERO_OK) return s;
-    zb::StepParams sp = shard_params(ctx, owner_lo, owner_hi, o.grad_divisor, partial);
-    sp.pingpong = sets == 2 ? 1 : 0;
-    sp.dec = static_cast<float>(1.0 - hp->lr * hp->weight_decay);
-    sp.b1f = static_cast<float>(hp->beta1);
-    sp.omb1 = static_cast<float>(1.0 - hp->beta1);
-    sp.b2f = static_cast<float>(hp->beta2);
-    sp.omb2 = static_cast<float>(1.0 - hp->beta2);
-    sp.epsf = static_cast<float>(hp->eps);
-    sp.lr = hp->lr;
-    sp.max_norm = o.max_grad_norm;
-    sp.clip = clip ? 1 : 0;
-    sp.add_acc = add_acc ? 1 : 0;
+    zb::StepParams sp = step_params(ctx, hp, o, sets, owner_lo, owner_hi, partial);
     if (fused) sp.drop_tile = ctx->drop_tile;
     zb::RankPtrs p{};
     for (int r = 0; r < ctx->R; ++r) {
