@@ -27,6 +27,11 @@
  *    work surfaces as ZERO_ERR_CUDA on a later call or on zero_sync.
  *  - A context is bound to the CUDA device that was current when it was
  *    created; calls with another device current return ZERO_ERR_INVALID_ARG.
+ *  - Threads: a plan is read-only after zero_plan and may be shared. A
+ *    context holds host-side state (the step count bound, the scheduler's
+ *    readiness counters, the prefetch ring), so calls on one context must
+ *    not overlap in time; different contexts may be used from different
+ *    threads. zero_cpu_step uses its own worker threads and shares nothing.
  *  - The library owns only the plan (host memory) and the context's small
  *    device scratch (loss-scale state, overflow flag, per-block norm
  *    partials, bias-correction power table).
