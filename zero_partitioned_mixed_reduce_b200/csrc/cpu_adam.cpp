@@ -11,17 +11,20 @@
 //
 // The arithmetic is the step of include/zero_b200.h, one IEEE binary32
 // operation per line (this file is built with -ffp-contract=off), so results
-// equal the GPU step bit for bit. The element loop is plain scalar C++ that
-// the compiler vectorizes; gcc's target_clones builds AVX-512, AVX2 and
-// baseline versions and picks one at load time. The half encoders round to
-// nearest even on the bit pattern (keeping subnormals, overflowing to
-// infinity), because the AVX-512 bf16 conversion instruction treats
-// subnormal inputs as zero.
+// equal the GPU step bit for bit. The fp32 update is plain C++ that the
+// compiler vectorizes (IEEE division and square root vectorize exactly);
+// gcc's target_clones builds AVX-512, AVX2 and baseline versions and picks
+// one at load time. bf16 is encoded on the bit pattern, round to nearest
+// even, keeping subnormals (the AVX-512 bf16 conversion instruction treats
+// subnormal inputs as zero); fp16 uses the IEEE conversion instruction where
+// the CPU has it, with a scalar encoder of the same rounding as fallback.
 #include <cmath>
 #include <cstring>
 #include <string>
 #include <thread>
 #include <vector>
+
+#include <immintrin.h>
 
 #include "internal.h"
 
@@ -33,12 +36,17 @@ inline uint32_t f2u(float x) {
     return u;
 }
 
+// The bf16 encoder is branch-free (both cases computed, one selected) so that
+// its loop vectorizes. The fp16 encoder below is the scalar reference (the
+// fallback, the tail and the NaN fix-up of the vector conversion).
+
 // fp32 -> bf16, round to nearest even on the bits; NaN -> quiet NaN.
 inline uint16_t to_bf16(float x) {
     const uint32_t u = f2u(x);
-    if ((u & 0x7fffffffu) > 0x7f800000u) return static_cast<uint16_t>((u >> 16) | 0x0040u);
+    const bool nan = (u & 0x7fffffffu) > 0x7f800000u;
     const uint32_t lsb = (u >> 16) & 1u;
-    return static_cast<uint16_t>((u + 0x7fffu + lsb) >> 16);
+    const uint32_t rounded = (u + 0x7fffu + lsb) >> 16;
+    return static_cast<uint16_t>(nan ? ((u >> 16) | 0x0040u) : rounded);
 }
 
 // fp32 -> IEEE binary16, round to nearest even, subnormals kept, overflow to inf.
@@ -70,10 +78,12 @@ struct Coeffs {
     float inv, dec, b1f, omb1, b2f, omb2, epsf, ss, bc2s, clip;
 };
 
-template <bool FP16, bool CLIP>
-__attribute__((target_clones("avx512f", "avx2", "default"))) void update_range(
+// The fp32 AdamW update of n elements, vectorized (IEEE division and square
+// root vectorize exactly).
+template <bool CLIP>
+__attribute__((target_clones("avx512f", "avx2", "default"))) void adam_range(
     const Coeffs c, const float* __restrict acc, float* __restrict p, float* __restrict m,
-    float* __restrict v, uint16_t* __restrict out, int64_t n) {
+    float* __restrict v, int64_t n) {
     for (int64_t i = 0; i < n; ++i) {
         const float g0 = acc[i] * c.inv;
         const float g = CLIP ? g0 * c.clip : g0;
@@ -85,20 +95,105 @@ __attribute__((target_clones("avx512f", "avx2", "default"))) void update_range(
         p[i] = pp;
         m[i] = mm;
         v[i] = vv;
-        out[i] = FP16 ? to_fp16(pp) : to_bf16(pp);
+    }
+}
+
+__attribute__((target_clones("avx512f", "avx2", "default"))) void encode_bf16_range(
+    const float* __restrict p, uint16_t* __restrict out, int64_t n) {
+    for (int64_t i = 0; i < n; ++i) out[i] = to_bf16(p[i]);
+}
+
+// fp32 -> fp16 with the conversion instruction (vcvtps2ph, round to nearest
+// even: IEEE conversion, subnormal results kept, overflow to infinity, so it
+// equals to_fp16 for every non-NaN input); NaN lanes are re-encoded by
+// to_fp16, which gives the canonical quiet NaN.
+__attribute__((target("avx512f"))) void encode_fp16_avx512(const float* __restrict p, uint16_t* __restrict out,
+                                                           int64_t n) {
+    int64_t i = 0;
+    for (; i + 16 <= n; i += 16) {
+        const __m512 x = _mm512_loadu_ps(p + i);
+        const __m256i h = _mm512_cvtps_ph(x, _MM_FROUND_TO_NEAREST_INT | _MM_FROUND_NO_EXC);
+        _mm256_storeu_si256(reinterpret_cast<__m256i*>(out + i), h);
+        const __mmask16 nan = _mm512_cmp_ps_mask(x, x, _CMP_UNORD_Q);
+        if (nan)
+            for (int j = 0; j < 16; ++j)
+                if (nan & (1u << j)) out[i + j] = to_fp16(p[i + j]);
+    }
+    for (; i < n; ++i) out[i] = to_fp16(p[i]);
+}
+
+__attribute__((target("avx2,f16c"))) void encode_fp16_avx2(const float* __restrict p, uint16_t* __restrict out,
+                                                           int64_t n) {
+    int64_t i = 0;
+    for (; i + 8 <= n; i += 8) {
+        const __m256 x = _mm256_loadu_ps(p + i);
+        const __m128i h = _mm256_cvtps_ph(x, _MM_FROUND_TO_NEAREST_INT | _MM_FROUND_NO_EXC);
+        _mm_storeu_si128(reinterpret_cast<__m128i*>(out + i), h);
+        const int nan = _mm256_movemask_ps(_mm256_cmp_ps(x, x, _CMP_UNORD_Q));
+        if (nan)
+            for (int j = 0; j < 8; ++j)
+                if (nan & (1 << j)) out[i + j] = to_fp16(p[i + j]);
+    }
+    for (; i < n; ++i) out[i] = to_fp16(p[i]);
+}
+
+void encode_fp16_scalar(const float* __restrict p, uint16_t* __restrict out, int64_t n) {
+    for (int64_t i = 0; i < n; ++i) out[i] = to_fp16(p[i]);
+}
+
+using EncodeFn = void (*)(const float*, uint16_t*, int64_t);
+
+EncodeFn pick_fp16_encoder() {
+    __builtin_cpu_init();
+    if (__builtin_cpu_supports("avx512f")) return encode_fp16_avx512;
+    if (__builtin_cpu_supports("avx2") && __builtin_cpu_supports("f16c")) return encode_fp16_avx2;
+    return encode_fp16_scalar;
+}
+
+// Update then encode, block by block, so that the encode re-reads p from cache.
+template <bool FP16, bool CLIP>
+void update_range(const Coeffs c, const float* __restrict acc, float* __restrict p, float* __restrict m,
+                  float* __restrict v, uint16_t* __restrict out, int64_t n) {
+    static const EncodeFn enc16 = pick_fp16_encoder();
+    constexpr int64_t kBlock = 2048;
+    for (int64_t b = 0; b < n; b += kBlock) {
+        const int64_t k = n - b < kBlock ? n - b : kBlock;
+        adam_range<CLIP>(c, acc + b, p + b, m + b, v + b, k);
+        if (FP16)
+            enc16(p + b, out + b, k);
+        else
+            encode_bf16_range(p + b, out + b, k);
     }
 }
 
 // Sum of (double)(acc * inv)^2 over [0, n) and whether any acc is non-finite.
+// Eight running sums, one per lane of an 8-element block, then added in lane
+// order: a fixed summation order that vectorizes without reassociation.
+constexpr int kLanes = 8;
 __attribute__((target_clones("avx512f", "avx2", "default"))) void scan_range(
     const float* __restrict acc, float inv, int64_t n, double* nrm, int* bad) {
+    double lane[kLanes] = {0, 0, 0, 0, 0, 0, 0, 0};
+    int flag[kLanes] = {0, 0, 0, 0, 0, 0, 0, 0};
+    const int64_t body = n - n % kLanes;
+    for (int64_t i = 0; i < body; i += kLanes) {
+        for (int j = 0; j < kLanes; ++j) {
+            const float a = acc[i + j];
+            flag[j] |= !(std::fabs(a) <= 3.4028234663852886e38f);
+            const double g = static_cast<double>(a * inv);
+            lane[j] += g * g;
+        }
+    }
+    for (int64_t i = body; i < n; ++i) {
+        const float a = acc[i];
+        flag[0] |= !(std::fabs(a) <= 3.4028234663852886e38f);
+        const double g = static_cast<double>(a * inv);
+        lane[0] += g * g;
+    }
     double s = 0.0;
     int b = 0;
-    for (int64_t i = 0; i < n; ++i) {
-        const float a = acc[i];
-        b |= !(std::fabs(a) <= 3.4028234663852886e38f);
-        const double g = static_cast<double>(a * inv);
-        s += g * g;
+    for (int j = 0; j < kLanes; ++j) {
+        s += lane[j];
+        b |= flag[j];
     }
     *nrm = s;
     *bad = b;
