@@ -903,6 +903,11 @@ def run_dist(args, world, rank, local):
         "per_rank_step_bytes": kbytes, "per_rank_nvlink_bytes": 2 * (N - 1) * S,
         "per_rank_step_gbs": kbytes / (step_ms * 1e-3) / 1e9, "peak": peak,
         "peak_source": f"{peak_src} hbm_gbs", "clocks": clk,
+        # the slower of the HBM stream and the NVLink reads (770 GB/s per direction,
+        # the machine's measured peer copy) bounds the step
+        "roofline": {"bound": "nvlink" if 2 * (N - 1) * S / 770e9 > kbytes / (peak * 1e9) else "hbm",
+                     "target_ms": 1e3 * max(kbytes / (peak * 1e9), 2 * (N - 1) * S / 770e9),
+                     "frac": 1e3 * max(kbytes / (peak * 1e9), 2 * (N - 1) * S / 770e9) / step_ms},
     }
     dz.close()
     if rank == 0:
