@@ -199,3 +199,70 @@ def test_replayed_overlapped_step_matches_oracle(mode):
             c.compare()
     finally:
         c.close()
+
+
+def test_replayed_zero3_training_step_matches_oracle():
+    # a whole ZeRO-3 step in one graph: forward through the look-ahead gather
+    # ring, backward through it in reverse with each layer's gradients written
+    # and reported (reduce-scatters on the communication stream), the join and
+    # the step; replays must follow the oracle, and every gathered layer must
+    # equal the parameters of the step before
+    numels = [30_000, 77, 5_000, 12_001, 9, 4_096]
+    layer_ids = [0, 0, 1, 2, 2, 3]
+    R = 4
+    c = Case(numels, R, O.FP16, mode=O.SCALE_DYNAMIC, init_scale=256.0, interval=2, path="twopass_pp",
+             bucket_elems=15_000, layer_ids=layer_ids, seed=67)
+    try:
+        c.step_overlap()  # first use creates the scheduler's stream and events
+        c.compare()
+        Z.zero_ctx_reserve_steps(c.ctx, 8, c.hp["beta1"], c.hp["beta2"])
+        L = c.lay.layers
+        nl = len(L)
+        biggest = max(hi - lo for lo, hi in L)
+        ring = [torch.empty(biggest + 8, dtype=torch.int16, device="cuda") for _ in range(2)]
+        seen = [torch.empty(hi - lo, dtype=torch.int16, device="cuda") for lo, hi in L]
+        by_addr = {b.data_ptr(): b for b in ring}
+        P = c.lay.P
+        starts = np.concatenate([[0], np.cumsum(c.lay.numels)[:-1]])
+        first_t = [layer_ids.index(l) for l in range(nl)]
+        count_t = [layer_ids.count(l) for l in range(nl)]
+        dev = torch.zeros((R, P), dtype=torch.int16, device="cuda")
+
+        def step(s):
+            Z.zero_prefetch_begin(c.ctx, c.handle, ring, 1, 1, s)
+            for l in range(nl):  # forward: use (here: keep a copy of) each gathered layer
+                buf = by_addr[Z.zero_layer_acquire(c.ctx, l, s)]
+                seen[l].copy_(buf[:L[l][1] - L[l][0]])
+                Z.zero_layer_release(c.ctx, l, s)
+            for r in range(R):
+                c.grads[r].zero_()
+            Z.zero_prefetch_begin(c.ctx, c.handle, ring, 1, -1, s)
+            for l in reversed(range(nl)):  # backward: gradients of the layer's tensors
+                Z.zero_layer_acquire(c.ctx, l, s)
+                for k in range(first_t[l], first_t[l] + count_t[l]):
+                    off, n, st = int(c.lay.offsets[k]), int(c.lay.numels[k]), int(starts[k])
+                    for r in range(R):
+                        c.grads[r].view(torch.int16)[off:off + n].copy_(dev[r, st:st + n])
+                Z.zero_layer_release(c.ctx, l, s)
+                Z.zero_grads_ready(c.ctx, first_t[l], count_t[l], c.grads, c.acc, 0, s)
+            Z.zero_grads_join(c.ctx, s)
+            Z.zero_step_ex(c.ctx, c.hp, c.handle, None, 1.0, 0.0, s)
+
+        graph = _capture(step)
+        for k in range(4):
+            before = c.gpu_state()["param"]
+            c.step_no += 1
+            g = c.make_grads([(2, 100, 0x7C00)] if k == 2 else None)
+            dev.copy_(torch.from_numpy(g.view(np.int16)))
+            graph.replay()
+            torch.cuda.synchronize()
+            full = np.zeros(c.plan.T, np.uint16)
+            full[c.idx] = before
+            for l, (lo, hi) in enumerate(L):
+                assert np.array_equal(seen[l].cpu().numpy().view(np.uint16), full[lo:hi]), (k, l)
+            skipped = O.step(c.ostate, g, _ohp(c), c.ofsm)
+            assert skipped == (k == 2)
+            c.g.check()
+            c.compare()
+    finally:
+        c.close()
