@@ -31,7 +31,11 @@
  *    context holds host-side state (the step count bound, the scheduler's
  *    readiness counters, the prefetch ring), so calls on one context must
  *    not overlap in time; different contexts may be used from different
- *    threads. zero_cpu_step uses its own worker threads and shares nothing.
+ *    threads. The CPU step (zero_cpu_step, zero_cpu_scan, zero_cpu_update)
+ *    runs on a pool of worker threads that the library keeps between calls;
+ *    a call that finds the pool busy with another thread's step starts
+ *    threads of its own, so concurrent CPU steps on different buffers are
+ *    safe.
  *  - The library owns only the plan (host memory) and the context's small
  *    device scratch (loss-scale state, overflow flag, per-block norm
  *    partials, bias-correction power table).
@@ -662,8 +666,9 @@ zero_status zero_layer_release(zero_ctx_t* ctx, int64_t layer, void* stream);
  * forward pass (it releases no lock and touches no GPU state).
  * All pointers are HOST memory: R pointers each, S elements per shard
  * (pinned memory makes the surrounding copies asynchronous). nthreads <= 0
- * uses every hardware thread; the result does not depend on nthreads except
- * for the summation order of grad_norm_sq.
+ * uses every hardware thread (the calling thread is one of them); the result
+ * does not depend on nthreads except for the summation order of
+ * grad_norm_sq. Work under 65,536 elements runs on the calling thread.
  * Errors: ZERO_ERR_INVALID_ARG.
  */
 zero_status zero_cpu_step(const zero_plan_t* plan, const zero_loss_scale_config* cfg,
@@ -684,6 +689,47 @@ zero_status zero_cpu_step(const zero_plan_t* plan, const zero_loss_scale_config*
  * Errors: ZERO_ERR_INVALID_ARG (NULL output), ZERO_ERR_CUDA.
  */
 zero_status zero_debug_bounds(int64_t* count, int64_t* first_site, int64_t* first_index, int32_t reset);
+
+/*
+ * The CPU step in three calls, for callers that overlap the update with the
+ * upload of the half parameters (ZeRO-Offload with the parameters copied
+ * back range by range): zero_cpu_step equals zero_cpu_scan, then
+ * zero_cpu_update over [0, S), then zero_cpu_commit.
+ *
+ * zero_cpu_scan -- the global part of the step: reads every accumulator once
+ * and fills *out with the overflow flag, the skip decision, the squared norm
+ * and the unscale and clipping coefficients. in is the loss-scale state
+ * before the step; it is not changed. Errors: as zero_cpu_step.
+ *
+ * zero_cpu_update -- the update of elements [lo, hi) of every shard (master,
+ * m, v in place, param written), from a decision of zero_cpu_scan on the
+ * same accumulators and the same state `in`; nothing is written when the
+ * decision skips the step. Ranges may be updated in any order and from
+ * different calls; every element must be updated exactly once per step.
+ * Errors: ZERO_ERR_INVALID_ARG, ZERO_ERR_RANGE (lo, hi).
+ *
+ * zero_cpu_commit -- advances the loss-scale state after the updates:
+ * skip, backoff, growth and t as in zero_cpu_step. Errors:
+ * ZERO_ERR_INVALID_ARG.
+ */
+typedef struct {
+    double grad_norm_sq; /* sum of (float)(acc * inv)^2 over every element, in double */
+    float inv;           /* (float)(1 / ((R * grad_divisor) * scale)) */
+    float clip;          /* the clipping coefficient; 1 without clipping */
+    int32_t overflow;    /* some accumulator is inf or NaN */
+    int32_t skip;        /* DYNAMIC mode and overflow: the update writes nothing */
+    int32_t clipping;    /* clipping is on (max_grad_norm > 0) */
+    int32_t reserved;
+} zero_cpu_decision;
+zero_status zero_cpu_scan(const zero_plan_t* plan, const zero_loss_scale_config* cfg,
+                          const zero_loss_scale_state* in, const zero_step_opts* opts,
+                          const float* const* acc, int32_t nthreads, zero_cpu_decision* out);
+zero_status zero_cpu_update(const zero_plan_t* plan, const zero_loss_scale_state* in, const zero_adamw* hp,
+                            const zero_cpu_decision* decision, const float* const* acc, float* const* master,
+                            float* const* m, float* const* v, void* const* param, int64_t lo, int64_t hi,
+                            int32_t nthreads);
+zero_status zero_cpu_commit(const zero_loss_scale_config* cfg, zero_loss_scale_state* inout,
+                            const zero_cpu_decision* decision);
 
 /* zero_sync -- synchronize `stream` and report any pending CUDA error. */
 zero_status zero_sync(zero_ctx_t* ctx, void* stream);

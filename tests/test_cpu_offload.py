@@ -152,3 +152,86 @@ def test_cpu_step_argument_errors():
     with pytest.raises(Z.ZeroError):
         Z.zero_cpu_step(plan.handle, dict(mode=0), dict(scale=1.0, t=0),
                         dict(HP, beta1=1.0), buf, buf, buf, buf, half)
+
+
+@pytest.mark.parametrize("dtype", [O.BF16, O.FP16])
+@pytest.mark.parametrize("mode", [O.SCALE_NONE, O.SCALE_DYNAMIC])
+@pytest.mark.parametrize("clip", [0.0, 1e-3])
+def test_split_cpu_step_equals_cpu_step(dtype, mode, clip):
+    # scan, then the update in uneven ranges in shuffled order, then commit:
+    # the same bytes and loss-scale state as zero_cpu_step (and the oracle)
+    a = Offload([200_000, 77, 4096], 4, dtype, 8, mode, seed=21)
+    b = Offload([200_000, 77, 4096], 4, dtype, 8, mode, seed=21)
+    rng = np.random.default_rng(3)
+    for step in range(4):
+        inject = (0, 1, 123) if (step == 2 and mode == O.SCALE_DYNAMIC) else None
+        a.step(1, 1.0, clip, inject)
+        a.compare()
+        # b: the same gradients as a drew (same seed sequence), split path
+        g = O.float_to_half((b.rng.normal(0, 1e-2, (1, b.R, b.lay.P)) * b.fsm.scale).astype(np.float32), dtype)
+        if inject:
+            g[inject] = 0x7C00 if dtype == O.FP16 else 0x7F80
+        s_, _ = O.allreduce_sum(g[0], dtype)
+        flat = np.zeros(b.lay.T, np.float32)
+        flat[b.idx] = s_
+        S = b.lay.S
+        for r in range(b.R):
+            b.acc[r][:] = flat[r * S:(r + 1) * S]
+        d = Z.zero_cpu_scan(b.plan.handle, b.cfg, b.ls, b.acc, 1.0, clip)
+        cuts = np.sort(rng.choice(np.arange(1, S), 5, replace=False))
+        ranges = list(zip(np.concatenate([[0], cuts]), np.concatenate([cuts, [S]])))
+        rng.shuffle(ranges)
+        for lo, hi in ranges:
+            Z.zero_cpu_update(b.plan.handle, b.ls, HP, d, b.acc, b.master, b.m, b.v, b.param, int(lo), int(hi))
+        b.ls = Z.zero_cpu_commit(b.cfg, b.ls, d)
+        O.step_ex(b.ost, g, OHP, b.fsm, 1.0, clip)
+        b.compare()
+        for x, y in zip(a.master + a.m + a.v, b.master + b.m + b.v):
+            assert np.array_equal(x.view(np.uint32), y.view(np.uint32))
+        for x, y in zip(a.param, b.param):
+            assert np.array_equal(x, y)
+
+
+def test_cpu_update_range_errors():
+    plan = Z.Plan([100], None, 2, O.BF16, 8, 0)
+    buf = [np.zeros(plan.S, np.float32) for _ in range(2)]
+    half = [np.zeros(plan.S, np.uint16) for _ in range(2)]
+    ls = dict(scale=1.0, t=0)
+    d = Z.zero_cpu_scan(plan.handle, dict(mode=0), ls, buf)
+    with pytest.raises(Z.ZeroError) as e:
+        Z.zero_cpu_update(plan.handle, ls, HP, d, buf, buf, buf, buf, half, 0, plan.S + 1)
+    assert e.value.status == Z.ZERO_ERR_RANGE
+    with pytest.raises(Z.ZeroError):
+        Z.zero_cpu_update(plan.handle, ls, HP, d, buf, buf, buf, buf, half, 5, 4)
+
+
+def test_concurrent_cpu_steps_from_two_host_threads():
+    # the library keeps one pool of worker threads; a step that finds it busy
+    # runs on threads of its own. Both ways give the bytes of a lone step.
+    import threading
+    base = Offload([300_000, 4099], 4, O.BF16, 8, O.SCALE_DYNAMIC, seed=5)
+    base.step()
+    init = [[x.copy() for x in xs] for xs in (base.acc, base.master, base.m, base.v, base.param)]
+
+    def run(out, k):
+        acc, master, m, v, param = [[x.copy() for x in xs] for xs in init]
+        ls = dict(base.ls)
+        for _ in range(k):
+            ls = Z.zero_cpu_step(base.plan.handle, base.cfg, ls, HP, acc, master, m, v, param, 1.0, 0.0, 4)
+        out.append((master, m, v, param, ls))
+
+    lone = []
+    run(lone, 6)
+    results = [[] for _ in range(3)]
+    threads = [threading.Thread(target=run, args=(results[i], 6)) for i in range(3)]
+    for t in threads:
+        t.start()
+    for t in threads:
+        t.join()
+    for res in results:
+        (master, m, v, param, ls), = res
+        for x, y in zip(master + m + v, lone[0][0] + lone[0][1] + lone[0][2]):
+            assert np.array_equal(x.view(np.uint32), y.view(np.uint32))
+        for x, y in zip(param, lone[0][3]):
+            assert np.array_equal(x, y)
+        assert ls == lone[0][4]

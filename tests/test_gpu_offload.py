@@ -51,6 +51,7 @@ class OffloadRun:
         self.copy = torch.cuda.Stream()
         self.step_no = 0
         self.up_ev = None
+        self.pipelined = False
         self.hp = self.wl["hp"]
         self.ohp = O.AdamW(*(self.hp[k] for k in ("lr", "beta1", "beta2", "eps", "weight_decay")))
 
@@ -81,10 +82,28 @@ class OffloadRun:
         done.synchronize()
         if self.up_ev is not None:
             self.up_ev.synchronize()  # the last upload has finished reading param_host
-        self.ls = Z.zero_cpu_step(self.plan.handle, self.cfg, self.ls, self.hp, self.acc_host[slot],
-                                  self.master, self.m, self.v, self.param_host, nthreads=0)
+        if not self.pipelined:
+            self.ls = Z.zero_cpu_step(self.plan.handle, self.cfg, self.ls, self.hp, self.acc_host[slot],
+                                      self.master, self.m, self.v, self.param_host, nthreads=0)
+            return
+        # scan, then the update range by range, each range uploaded while the next updates
+        S = self.plan.S
+        dec = Z.zero_cpu_scan(self.plan.handle, self.cfg, self.ls, self.acc_host[slot])
+        for i in range(5):
+            lo, hi = S * i // 5, S * (i + 1) // 5
+            Z.zero_cpu_update(self.plan.handle, self.ls, self.hp, dec, self.acc_host[slot], self.master,
+                              self.m, self.v, self.param_host, lo, hi)
+            with torch.cuda.stream(self.copy):
+                for r in range(self.R):
+                    self.param_gpu[r][lo:hi].copy_(self.param_host[r][lo:hi], non_blocking=True)
+        self.ls = Z.zero_cpu_commit(self.cfg, self.ls, dec)
+        self.pipe_ev = torch.cuda.Event()
+        self.pipe_ev.record(self.copy)
 
     def upload(self):
+        if self.pipelined:  # the ranges are already queued
+            self.up_ev = self.pipe_ev
+            return
         with torch.cuda.stream(self.copy):
             for r in range(self.R):
                 self.param_gpu[r].copy_(self.param_host[r], non_blocking=True)
@@ -134,10 +153,12 @@ class OffloadRun:
 
 
 @pytest.mark.parametrize("delayed", [False, True])
+@pytest.mark.parametrize("pipelined", [False, True])
 @pytest.mark.parametrize("R,dtype,mode", [(2, O.BF16, O.SCALE_NONE), (8, O.FP16, O.SCALE_DYNAMIC),
                                           (3, O.FP16, O.SCALE_STATIC)])
-def test_offload_pipeline_matches_oracle(delayed, R, dtype, mode):
+def test_offload_pipeline_matches_oracle(delayed, pipelined, R, dtype, mode):
     o = OffloadRun([200_001, 77, 4096, 3], R, dtype, mode)
+    o.pipelined = pipelined
     try:
         o.run(5, delayed)
         o.compare()

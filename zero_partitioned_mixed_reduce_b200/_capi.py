@@ -81,6 +81,12 @@ class zero_loss_scale_state(C.Structure):
                 ("grad_norm_sq", C.c_double)]
 
 
+class zero_cpu_decision(C.Structure):
+    _fields_ = [("grad_norm_sq", C.c_double), ("inv", C.c_float), ("clip", C.c_float),
+                ("overflow", C.c_int32), ("skip", C.c_int32), ("clipping", C.c_int32),
+                ("reserved", C.c_int32)]
+
+
 _lib = C.CDLL(LIB_PATH)
 _P = C.c_void_p
 _S = C.c_int32  # zero_status
@@ -125,6 +131,13 @@ _sig("zero_layer_release", _S, [_P, C.c_int64, _P])
 _sig("zero_cpu_step", _S, [_P, C.POINTER(zero_loss_scale_config), C.POINTER(zero_loss_scale_state),
                            C.POINTER(zero_adamw), C.POINTER(zero_step_opts), _PP, _PP, _PP, _PP, _PP,
                            C.c_int32])
+_sig("zero_cpu_scan", _S, [_P, C.POINTER(zero_loss_scale_config), C.POINTER(zero_loss_scale_state),
+                           C.POINTER(zero_step_opts), _PP, C.c_int32, C.POINTER(zero_cpu_decision)])
+_sig("zero_cpu_update", _S, [_P, C.POINTER(zero_loss_scale_state), C.POINTER(zero_adamw),
+                             C.POINTER(zero_cpu_decision), _PP, _PP, _PP, _PP, _PP, C.c_int64, C.c_int64,
+                             C.c_int32])
+_sig("zero_cpu_commit", _S, [C.POINTER(zero_loss_scale_config), C.POINTER(zero_loss_scale_state),
+                             C.POINTER(zero_cpu_decision)])
 _sig("zero_step_shard", _S, [_P, C.POINTER(zero_adamw), C.POINTER(zero_state), _PP, C.c_int32,
                              C.c_int32, _P, _P])
 _sig("zero_step_commit", _S, [_P, _P, _P])
@@ -382,24 +395,61 @@ def zero_layer_release(ctx, layer, stream=None):
     _check(_lib.zero_layer_release(ctx, layer, _stream(stream)))
 
 
+def _cpu_cfg(cfg):
+    return zero_loss_scale_config(cfg.get("mode", ZERO_SCALE_NONE), 1.0,
+                                  cfg.get("growth_interval", 1000), cfg.get("growth_factor", 2.0),
+                                  cfg.get("backoff_factor", 0.5), cfg.get("min_scale", 1.0), 0)
+
+
+def _cpu_state(state):
+    st = zero_loss_scale_state()
+    for k, _ in zero_loss_scale_state._fields_:
+        if k in state:
+            setattr(st, k, state[k])
+    return st
+
+
+def _cpu_hp(hp):
+    if isinstance(hp, dict):
+        return zero_adamw(hp["lr"], hp["beta1"], hp["beta2"], hp["eps"], hp["weight_decay"])
+    return hp
+
+
 def zero_cpu_step(plan, cfg, state, hp, acc, master, m, v, param, grad_divisor=1.0,
                   max_grad_norm=0.0, nthreads=0):
     """The optimizer step on host memory (all buffers host pointers, numpy
     arrays or CPU tensors). cfg / state as for zero_step_noalloc; returns the
     loss-scale state after the step."""
-    c = zero_loss_scale_config(cfg.get("mode", ZERO_SCALE_NONE), 1.0,
-                               cfg.get("growth_interval", 1000), cfg.get("growth_factor", 2.0),
-                               cfg.get("backoff_factor", 0.5), cfg.get("min_scale", 1.0), 0)
-    st = zero_loss_scale_state()
-    for k, _ in zero_loss_scale_state._fields_:
-        if k in state:
-            setattr(st, k, state[k])
-    if isinstance(hp, dict):
-        hp = zero_adamw(hp["lr"], hp["beta1"], hp["beta2"], hp["eps"], hp["weight_decay"])
+    c, st, hp = _cpu_cfg(cfg), _cpu_state(state), _cpu_hp(hp)
     opts = zero_step_opts(grad_divisor, max_grad_norm)
     arrays = [_ptr_array([_host_addr(x) for x in xs]) for xs in (acc, master, m, v, param)]
     _check(_lib.zero_cpu_step(plan, C.byref(c), C.byref(st), C.byref(hp), C.byref(opts),
                               *[a[0] for a in arrays], nthreads))
+    return {k: getattr(st, k) for k, _ in zero_loss_scale_state._fields_}
+
+
+def zero_cpu_scan(plan, cfg, state, acc, grad_divisor=1.0, max_grad_norm=0.0, nthreads=0):
+    """The global part of the CPU step; returns a zero_cpu_decision."""
+    c, st = _cpu_cfg(cfg), _cpu_state(state)
+    opts = zero_step_opts(grad_divisor, max_grad_norm)
+    a = _ptr_array([_host_addr(x) for x in acc])
+    d = zero_cpu_decision()
+    _check(_lib.zero_cpu_scan(plan, C.byref(c), C.byref(st), C.byref(opts), a[0], nthreads, C.byref(d)))
+    return d
+
+
+def zero_cpu_update(plan, state, hp, decision, acc, master, m, v, param, lo, hi, nthreads=0):
+    """Update elements [lo, hi) of every shard from a zero_cpu_scan decision."""
+    st, hp = _cpu_state(state), _cpu_hp(hp)
+    arrays = [_ptr_array([_host_addr(x) for x in xs]) for xs in (acc, master, m, v, param)]
+    _check(_lib.zero_cpu_update(plan, C.byref(st), C.byref(hp), C.byref(decision),
+                                *[a[0] for a in arrays], lo, hi, nthreads))
+
+
+def zero_cpu_commit(cfg, state, decision):
+    """The loss-scale state after the step (a dict)."""
+    c, st = _cpu_cfg(cfg), _cpu_state(state)
+    _check(_lib.zero_cpu_commit(C.byref(c), C.byref(st), C.byref(decision)))
     return {k: getattr(st, k) for k, _ in zero_loss_scale_state._fields_}
 
 

@@ -18,11 +18,17 @@
 // even, keeping subnormals (the AVX-512 bf16 conversion instruction treats
 // subnormal inputs as zero); fp16 uses the IEEE conversion instruction where
 // the CPU has it, with a scalar encoder of the same rounding as fallback.
+#include <algorithm>
 #include <cmath>
+#include <condition_variable>
 #include <cstring>
+#include <functional>
+#include <mutex>
 #include <string>
 #include <thread>
 #include <vector>
+
+#include <unistd.h>
 
 #include <immintrin.h>
 
@@ -199,58 +205,216 @@ __attribute__((target_clones("avx512f", "avx2", "default"))) void scan_range(
     *bad = b;
 }
 
+// Worker threads kept between calls: a step on a small model, or an update
+// issued in several ranges, would otherwise spend a noticeable part of its
+// time starting threads. The caller's thread runs job 0 itself. One job runs
+// at a time; a call that finds the pool busy (another host thread is inside a
+// CPU step) starts its own threads instead. Workers sleep on a condition
+// variable between jobs. The pool is never destroyed (its threads simply end
+// with the process), and a forked child builds a fresh one.
+class WorkerPool {
+public:
+    static WorkerPool& get() {
+        static std::mutex mu;
+        static WorkerPool* pool = nullptr;
+        std::lock_guard<std::mutex> lk(mu);
+        if (!pool || pool->pid_ != getpid()) pool = new WorkerPool();  // a stale child copy is leaked
+        return *pool;
+    }
+
+    // fn(t) for t in [0, n), t = 0 on the calling thread; returns when all are done
+    bool try_run(int n, const std::function<void(int)>& fn) {
+        std::unique_lock<std::mutex> busy(job_mu_, std::try_to_lock);
+        if (!busy.owns_lock()) return false;
+        {
+            std::lock_guard<std::mutex> lk(mu_);
+            while (static_cast<int>(workers_.size()) < n - 1) {
+                const int id = static_cast<int>(workers_.size()) + 1;
+                workers_.emplace_back([this, id, g = gen_] { loop(id, g); });
+                workers_.back().detach();
+            }
+            job_ = &fn;
+            njob_ = n;
+            pending_ = n - 1;
+            ++gen_;
+        }
+        cv_.notify_all();
+        fn(0);
+        std::unique_lock<std::mutex> lk(mu_);
+        done_cv_.wait(lk, [this] { return pending_ == 0; });
+        job_ = nullptr;
+        return true;
+    }
+
+private:
+    WorkerPool() : pid_(getpid()) {}
+
+    // `seen` is the generation before the job that started this worker
+    void loop(int id, uint64_t seen) {
+        for (;;) {
+            const std::function<void(int)>* job;
+            {
+                std::unique_lock<std::mutex> lk(mu_);
+                cv_.wait(lk, [&] { return gen_ != seen; });
+                seen = gen_;
+                if (id >= njob_) continue;
+                job = job_;
+            }
+            (*job)(id);
+            std::lock_guard<std::mutex> lk(mu_);
+            if (--pending_ == 0) done_cv_.notify_one();
+        }
+    }
+
+    const pid_t pid_;
+    std::mutex job_mu_, mu_;
+    std::condition_variable cv_, done_cv_;
+    std::vector<std::thread> workers_;
+    const std::function<void(int)>* job_ = nullptr;
+    int njob_ = 0, pending_ = 0;
+    uint64_t gen_ = 0;
+};
+
+// fn(t) for t in [0, n) on n threads
 template <typename F>
-void parallel_chunks(int64_t total, int nthreads, F&& fn) {
-    if (nthreads <= 1 || total < (int64_t(1) << 16)) {
-        fn(0, 0, total);
+void run_parallel(int n, F&& fn) {
+    if (n <= 1) {
+        if (n == 1) fn(0);
         return;
     }
+    const std::function<void(int)> job = std::ref(fn);
+    if (WorkerPool::get().try_run(n, job)) return;
     std::vector<std::thread> pool;
-    const int64_t chunk = (total + nthreads - 1) / nthreads;
-    for (int t = 0; t < nthreads; ++t) {
-        const int64_t a = t * chunk, b = std::min(total, a + chunk);
-        if (a >= b) break;
-        pool.emplace_back([&fn, t, a, b] { fn(t, a, b); });
-    }
+    for (int t = 1; t < n; ++t) pool.emplace_back([&job, t] { job(t); });
+    job(0);
     for (auto& th : pool) th.join();
+}
+
+// Elements [lo, hi) of every one of R shards, as one index space of R*(hi-lo)
+// elements cut into nthreads equal parts: thread t calls fn(t, r, a, b) for
+// each shard piece [a, b) of its part, in shard order. One set of threads
+// serves all shards (small work runs on the calling thread).
+template <typename F>
+void parallel_shards(int R, int64_t lo, int64_t hi, int nthreads, F&& fn) {
+    const int64_t len = hi - lo, total = static_cast<int64_t>(R) * len;
+    auto part = [&](int t, int64_t q0, int64_t q1) {
+        while (q0 < q1) {
+            const int r = static_cast<int>(q0 / len);
+            const int64_t a = lo + (q0 - static_cast<int64_t>(r) * len);
+            const int64_t b = std::min(hi, a + (q1 - q0));
+            fn(t, r, a, b);
+            q0 += b - a;
+        }
+    };
+    if (len <= 0) return;
+    if (nthreads <= 1 || total < (int64_t(1) << 16)) {
+        part(0, 0, total);
+        return;
+    }
+    const int64_t chunk = (total + nthreads - 1) / nthreads;
+    const int used = static_cast<int>((total + chunk - 1) / chunk);
+    run_parallel(used, [&](int t) { part(t, t * chunk, std::min(total, (t + 1) * chunk)); });
 }
 
 }  // namespace
 
-extern "C" zero_status zero_cpu_step(const zero_plan_t* plan, const zero_loss_scale_config* cfg,
-                                     zero_loss_scale_state* inout, const zero_adamw* hp,
-                                     const zero_step_opts* opts, const float* const* acc, float* const* master,
-                                     float* const* m, float* const* v, void* const* param, int32_t nthreads) {
-    if (!plan || !cfg || !inout || !hp || !acc || !master || !m || !v || !param)
-        return zb_fail(ZERO_ERR_INVALID_ARG, "zero_cpu_step: NULL argument");
+namespace {
+
+zero_status check_cfg(const zero_loss_scale_config* cfg, const char* where) {
+    if (cfg->mode < ZERO_SCALE_NONE || cfg->mode > ZERO_SCALE_DYNAMIC)
+        return zb_fail(ZERO_ERR_INVALID_ARG, std::string(where) + ": bad loss-scale mode");
+    if (cfg->mode == ZERO_SCALE_DYNAMIC &&
+        (cfg->growth_interval < 1 || !(cfg->growth_factor > 1.0f) ||
+         !(cfg->backoff_factor > 0.0f && cfg->backoff_factor < 1.0f) || !(cfg->min_scale > 0.0f)))
+        return zb_fail(ZERO_ERR_INVALID_ARG, std::string(where) + ": bad dynamic loss-scale config");
+    return ZERO_OK;
+}
+
+int thread_count(int32_t nthreads) {
+    int n = nthreads >= 1 ? nthreads : static_cast<int>(std::thread::hardware_concurrency());
+    return n >= 1 ? n : 1;
+}
+
+}  // namespace
+
+extern "C" zero_status zero_cpu_scan(const zero_plan_t* plan, const zero_loss_scale_config* cfg,
+                                     const zero_loss_scale_state* in, const zero_step_opts* opts,
+                                     const float* const* acc, int32_t nthreads, zero_cpu_decision* out) {
+    if (!plan || !cfg || !in || !acc || !out) return zb_fail(ZERO_ERR_INVALID_ARG, "zero_cpu_scan: NULL argument");
     zero_step_opts o{1.0, 0.0, 0, 0};
     if (opts) o = *opts;
     if (!(o.grad_divisor >= 1.0) || !std::isfinite(o.grad_divisor) || !(o.max_grad_norm >= 0.0) ||
         !std::isfinite(o.max_grad_norm) || o.flags != 0 || o.reserved != 0)
-        return zb_fail(ZERO_ERR_INVALID_ARG, "zero_cpu_step: need grad_divisor >= 1, finite max_grad_norm >= 0, no flags");
-    if (cfg->mode < ZERO_SCALE_NONE || cfg->mode > ZERO_SCALE_DYNAMIC)
-        return zb_fail(ZERO_ERR_INVALID_ARG, "zero_cpu_step: bad loss-scale mode");
-    if (cfg->mode == ZERO_SCALE_DYNAMIC &&
-        (cfg->growth_interval < 1 || !(cfg->growth_factor > 1.0f) ||
-         !(cfg->backoff_factor > 0.0f && cfg->backoff_factor < 1.0f) || !(cfg->min_scale > 0.0f)))
-        return zb_fail(ZERO_ERR_INVALID_ARG, "zero_cpu_step: bad dynamic loss-scale config");
-    const float scale = cfg->mode == ZERO_SCALE_NONE ? 1.0f : inout->scale;
-    if (!(scale > 0.0f) || !std::isfinite(scale) || inout->t < 0)
+        return zb_fail(ZERO_ERR_INVALID_ARG,
+                       "zero_cpu_step: need grad_divisor >= 1, finite max_grad_norm >= 0, no flags");
+    zero_status st = check_cfg(cfg, "zero_cpu_step");
+    if (st != ZERO_OK) return st;
+    const float scale = cfg->mode == ZERO_SCALE_NONE ? 1.0f : in->scale;
+    if (!(scale > 0.0f) || !std::isfinite(scale) || in->t < 0)
         return zb_fail(ZERO_ERR_INVALID_ARG, "zero_cpu_step: need a finite scale > 0 and t >= 0");
+    const int R = plan->R;
+    for (int r = 0; r < R; ++r)
+        if (!acc[r]) return zb_fail(ZERO_ERR_INVALID_ARG, "zero_cpu_step: NULL rank pointer");
+    const int nt = thread_count(nthreads);
+    const int64_t S = plan->S;
+    const float inv =
+        static_cast<float>(1.0 / ((static_cast<double>(R) * o.grad_divisor) * static_cast<double>(scale)));
+    // overflow and squared norm; each thread sums its pieces in order, and
+    // the per-thread partials are summed in thread order
+    std::vector<double> part(static_cast<size_t>(nt), 0.0);
+    std::vector<int> bad(static_cast<size_t>(nt), 0);
+    parallel_shards(R, 0, S, nt, [&](int t, int r, int64_t a, int64_t b) {
+        double pn = 0.0;
+        int pb = 0;
+        scan_range(acc[r] + a, inv, b - a, &pn, &pb);
+        part[t] += pn;
+        bad[t] |= pb;
+    });
+    double nrm = 0.0;
+    int overflow = 0;
+    for (size_t i = 0; i < part.size(); ++i) {
+        nrm += part[i];
+        overflow |= bad[i];
+    }
+    zero_cpu_decision d;
+    d.grad_norm_sq = nrm;
+    d.inv = inv;
+    d.clip = 1.0f;
+    if (o.max_grad_norm > 0.0) {
+        const double cd = o.max_grad_norm / (std::sqrt(nrm) + 1e-6);
+        d.clip = static_cast<float>(cd < 1.0 ? cd : 1.0);
+    }
+    d.overflow = overflow;
+    d.skip = (cfg->mode == ZERO_SCALE_DYNAMIC && overflow) ? 1 : 0;
+    d.clipping = o.max_grad_norm > 0.0 ? 1 : 0;
+    d.reserved = 0;
+    *out = d;
+    return ZERO_OK;
+}
+
+extern "C" zero_status zero_cpu_update(const zero_plan_t* plan, const zero_loss_scale_state* in,
+                                       const zero_adamw* hp, const zero_cpu_decision* d,
+                                       const float* const* acc, float* const* master, float* const* m,
+                                       float* const* v, void* const* param, int64_t lo, int64_t hi,
+                                       int32_t nthreads) {
+    if (!plan || !in || !hp || !d || !acc || !master || !m || !v || !param)
+        return zb_fail(ZERO_ERR_INVALID_ARG, "zero_cpu_update: NULL argument");
     if (!(hp->lr >= 0.0) || !(hp->beta1 >= 0.0 && hp->beta1 < 1.0) || !(hp->beta2 >= 0.0 && hp->beta2 < 1.0) ||
         !(hp->eps > 0.0) || !(hp->weight_decay >= 0.0))
         return zb_fail(ZERO_ERR_INVALID_ARG, "zero_cpu_step: bad hyper-parameters");
+    const int64_t S = plan->S;
+    if (lo < 0 || lo > hi || hi > S)
+        return zb_fail(ZERO_ERR_RANGE, "zero_cpu_update: need 0 <= lo <= hi <= S");
+    if (in->t < 0) return zb_fail(ZERO_ERR_INVALID_ARG, "zero_cpu_update: need t >= 0");
     const int R = plan->R;
     for (int r = 0; r < R; ++r)
         if (!acc[r] || !master[r] || !m[r] || !v[r] || !param[r])
             return zb_fail(ZERO_ERR_INVALID_ARG, "zero_cpu_step: NULL rank pointer");
-    if (nthreads < 1) nthreads = static_cast<int>(std::thread::hardware_concurrency());
-    if (nthreads < 1) nthreads = 1;
-    const int64_t S = plan->S;
-
+    if (d->skip || lo == hi) return ZERO_OK;  // a skipped step writes nothing
+    const int nt = thread_count(nthreads);
     Coeffs c;
-    const double t1 = static_cast<double>(inout->t + 1);
-    c.inv = static_cast<float>(1.0 / ((static_cast<double>(R) * o.grad_divisor) * static_cast<double>(scale)));
+    const double t1 = static_cast<double>(in->t + 1);
+    c.inv = d->inv;
     c.dec = static_cast<float>(1.0 - hp->lr * hp->weight_decay);
     c.b1f = static_cast<float>(hp->beta1);
     c.omb1 = static_cast<float>(1.0 - hp->beta1);
@@ -259,44 +423,28 @@ extern "C" zero_status zero_cpu_step(const zero_plan_t* plan, const zero_loss_sc
     c.epsf = static_cast<float>(hp->eps);
     c.ss = static_cast<float>(hp->lr / (1.0 - std::pow(hp->beta1, t1)));
     c.bc2s = static_cast<float>(std::sqrt(1.0 - std::pow(hp->beta2, t1)));
-    c.clip = 1.0f;
+    c.clip = d->clip;
+    const bool fp16 = plan->dtype == ZERO_FP16, clip = d->clipping != 0;
+    parallel_shards(R, lo, hi, nt, [&](int, int r, int64_t a, int64_t b) {
+        const int64_t n = b - a;
+        uint16_t* out = static_cast<uint16_t*>(param[r]) + a;
+        if (fp16 && clip) update_range<true, true>(c, acc[r] + a, master[r] + a, m[r] + a, v[r] + a, out, n);
+        else if (fp16) update_range<true, false>(c, acc[r] + a, master[r] + a, m[r] + a, v[r] + a, out, n);
+        else if (clip) update_range<false, true>(c, acc[r] + a, master[r] + a, m[r] + a, v[r] + a, out, n);
+        else update_range<false, false>(c, acc[r] + a, master[r] + a, m[r] + a, v[r] + a, out, n);
+    });
+    return ZERO_OK;
+}
 
-    // pass 1: overflow and squared norm; per-thread partials summed in thread order
-    std::vector<double> part(static_cast<size_t>(nthreads) * R, 0.0);
-    std::vector<int> bad(static_cast<size_t>(nthreads) * R, 0);
-    for (int r = 0; r < R; ++r)
-        parallel_chunks(S, nthreads, [&](int t, int64_t a, int64_t b) {
-            scan_range(acc[r] + a, c.inv, b - a, &part[r * nthreads + t], &bad[r * nthreads + t]);
-        });
-    double nrm = 0.0;
-    int overflow = 0;
-    for (size_t i = 0; i < part.size(); ++i) {
-        nrm += part[i];
-        overflow |= bad[i];
-    }
-    if (o.max_grad_norm > 0.0) {
-        const double cd = o.max_grad_norm / (std::sqrt(nrm) + 1e-6);
-        c.clip = static_cast<float>(cd < 1.0 ? cd : 1.0);
-    }
-
-    // pass 2: the update, unless dynamic loss scaling skips the step
-    const bool skip = cfg->mode == ZERO_SCALE_DYNAMIC && overflow;
-    if (!skip) {
-        const bool fp16 = plan->dtype == ZERO_FP16, clip = o.max_grad_norm > 0.0;
-        for (int r = 0; r < R; ++r)
-            parallel_chunks(S, nthreads, [&](int, int64_t a, int64_t b) {
-                uint16_t* out = static_cast<uint16_t*>(param[r]) + a;
-                if (fp16 && clip) update_range<true, true>(c, acc[r] + a, master[r] + a, m[r] + a, v[r] + a, out, b - a);
-                else if (fp16) update_range<true, false>(c, acc[r] + a, master[r] + a, m[r] + a, v[r] + a, out, b - a);
-                else if (clip) update_range<false, true>(c, acc[r] + a, master[r] + a, m[r] + a, v[r] + a, out, b - a);
-                else update_range<false, false>(c, acc[r] + a, master[r] + a, m[r] + a, v[r] + a, out, b - a);
-            });
-    }
-
-    // loss-scale state machine, the same rules as the device step
+extern "C" zero_status zero_cpu_commit(const zero_loss_scale_config* cfg, zero_loss_scale_state* inout,
+                                       const zero_cpu_decision* d) {
+    if (!cfg || !inout || !d) return zb_fail(ZERO_ERR_INVALID_ARG, "zero_cpu_commit: NULL argument");
+    zero_status st = check_cfg(cfg, "zero_cpu_commit");
+    if (st != ZERO_OK) return st;
+    // the loss-scale state machine, the same rules as the device step
     int skipped = 0;
     if (cfg->mode == ZERO_SCALE_DYNAMIC) {
-        if (overflow) {
+        if (d->overflow) {
             const float s = inout->scale * cfg->backoff_factor;
             inout->scale = (s < cfg->min_scale) ? cfg->min_scale : s;
             inout->good = 0;
@@ -312,8 +460,22 @@ extern "C" zero_status zero_cpu_step(const zero_plan_t* plan, const zero_loss_sc
     } else {
         inout->t += 1;
     }
-    inout->last_overflow = overflow;
+    inout->last_overflow = d->overflow;
     inout->last_skipped = skipped;
-    inout->grad_norm_sq = nrm;
+    inout->grad_norm_sq = d->grad_norm_sq;
     return ZERO_OK;
+}
+
+extern "C" zero_status zero_cpu_step(const zero_plan_t* plan, const zero_loss_scale_config* cfg,
+                                     zero_loss_scale_state* inout, const zero_adamw* hp,
+                                     const zero_step_opts* opts, const float* const* acc, float* const* master,
+                                     float* const* m, float* const* v, void* const* param, int32_t nthreads) {
+    if (!plan || !cfg || !inout || !hp || !acc || !master || !m || !v || !param)
+        return zb_fail(ZERO_ERR_INVALID_ARG, "zero_cpu_step: NULL argument");
+    zero_cpu_decision d;
+    zero_status st = zero_cpu_scan(plan, cfg, inout, opts, acc, nthreads, &d);
+    if (st == ZERO_OK)
+        st = zero_cpu_update(plan, inout, hp, &d, acc, master, m, v, param, 0, plan->S, nthreads);
+    if (st == ZERO_OK) st = zero_cpu_commit(cfg, inout, &d);
+    return st;
 }
