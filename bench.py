@@ -56,8 +56,11 @@ def parse_args(argv=None):
                     help="micro-batches accumulated per step (the last fused into the step, or "
                          "all reduce-scattered on the two-pass path)")
     ap.add_argument("--clip", type=float, default=0.0,
-                    help="global-norm clipping threshold (> 0: on; fused path for R <= 5, "
+                    help="global-norm clipping threshold (> 0: on; fused path for R <= 4, "
                          "two-pass path otherwise)")
+    ap.add_argument("--clip-norm", choices=["rs", "pass"], default="rs",
+                    help="two-pass path with clipping: the last micro-batch's reduce-scatters take "
+                         "the norm (rs), or a separate read-only pass over the accumulators (pass)")
     ap.add_argument("--gather-bucket", type=int, default=32 << 20,
                     help="gather consecutive layers in one launch up to this many elements "
                          "(0: one launch per layer)")
@@ -233,7 +236,7 @@ def workload_label(name, wl, first_tensors=0):
 
 class Bench:
     def __init__(self, name, path, first_tensors=0, gather_bucket=32 << 20, accum=1, clip=0.0,
-                 bucket_elems=None):
+                 bucket_elems=None, clip_norm="rs"):
         import zero_partitioned_mixed_reduce_b200 as Z
         from zero_partitioned_mixed_reduce_b200 import synth
         self.Z, self.synth = Z, synth
@@ -248,7 +251,7 @@ class Bench:
         if path == "auto":
             # accumulation fuses its last micro-batch into the step unless
             # clipping needs the full sum first
-            if (accum > 1 and clip > 0) or (clip > 0 and wl["R"] > 5):
+            if (accum > 1 and clip > 0) or (clip > 0 and wl["R"] > 4):
                 path = "twopass"
             else:
                 # ping-pong state measured 2-3 % faster than in place at R = 4 and 8
@@ -256,6 +259,8 @@ class Bench:
                 # fp32 state, which every workload here fits
                 path = "pingpong"
         self.twopass = path.startswith("twopass")
+        # the two-pass clip norm from the reduce-scatters, or a separate pass
+        self.rs_norm = self.twopass and clip > 0 and clip_norm == "rs"
         if accum > 1 and clip > 0 and not self.twopass:
             raise SystemExit("--accum with --clip needs the two-pass path")
         self.path = path
@@ -284,6 +289,8 @@ class Bench:
             self.grads.append(g)
         self.ctx = Z.zero_ctx_create(self.plan.handle, wl["mode"], wl["init_scale"],
                                      wl["interval"])
+        if self.rs_norm:
+            Z.zero_ctx_set_grad_divisor(self.ctx, float(accum))
         self.max_layer = max(hi - lo for lo, hi in self.plan.layers)
         # gather buckets: consecutive layers up to gather_bucket elements (a larger
         # layer alone), at most 64 per launch; each layer lands in its own
@@ -331,8 +338,8 @@ class Bench:
         if self.twopass:
             # first micro-batch writes the accumulators, later ones read-modify-write
             main = (2 * R + 4) * T + (self.accum - 1) * (2 * R + 8) * T + 30 * T
-            if self.clip > 0:
-                main += 4 * T
+            if self.clip > 0 and not self.rs_norm:
+                main += 4 * T  # the norm pass over the accumulators
         elif self.accum > 1:
             # micro-batches 1..k-1 into the accumulators, the last fused with
             # the step (which reads the accumulators: 4 more bytes)
@@ -351,11 +358,13 @@ class Bench:
         if self.twopass:
             for mu in range(self.accum):
                 flags = Z.ZERO_RS_ACCUMULATE if mu else 0
+                if self.rs_norm and mu == self.accum - 1:
+                    flags |= Z.ZERO_RS_NORM
                 for b in range(len(self.plan.buckets)):
                     Z.zero_reduce_scatter_bucket_ex(self.ctx, b, grads, self.state.acc, flags,
                                                     stream)
             Z.zero_step_ex(self.ctx, hp, self.state.handle, None, float(self.accum), self.clip,
-                           stream)
+                           stream, flags=Z.ZERO_STEP_NORM_FROM_RS if self.rs_norm else 0)
         elif self.accum > 1:
             for mu in range(self.accum - 1):
                 flags = Z.ZERO_RS_ACCUMULATE if mu else 0
@@ -421,7 +430,7 @@ def run_ours(args, world, rank, local):
         print(json.dumps({"error": "no CUDA device: the benchmark has no CPU fallback"}))
         sys.exit(1)
     b = Bench(args.workload, args.path, args.first_tensors, args.gather_bucket, args.accum,
-              args.clip)
+              args.clip, clip_norm=args.clip_norm)
     stream = torch.cuda.current_stream()
     if args.graph:
         b.capture(stream, args.warmup + args.steps + 16)  # + the e2e leg's steps
@@ -464,6 +473,9 @@ def run_ours(args, world, rank, local):
     elif b.accum > 1:
         kernel_name = f"reduce_scatter+fused_step_kernel (accum {b.accum}, last micro-batch fused)"
     traffic = profiled_traffic(kernel_name, args.workload)
+    clip_label = ("" if b.clip <= 0 else
+                  "global-norm clip from the reduce-scatters' norm shares, " if b.rs_norm else
+                  "global-norm clip pass, ")
     out = {
         "metric": METRIC,
         "value": units / (ms * 1e-3),
@@ -488,10 +500,10 @@ def run_ours(args, world, rank, local):
                      "inplace": f"{'global-norm clip pass, ' if b.clip > 0 else ''}"
                                 "fused reduce-scatter+AdamW, in place",
                      "twopass": f"bucketed reduce-scatter ({b.accum} micro-batch(es)), "
-                       f"{'global-norm clip, ' if b.clip > 0 else ''}"
+                       f"{clip_label}"
                        "then AdamW from fp32 accumulators, in place",
                      "twopass_pingpong": f"bucketed reduce-scatter ({b.accum} micro-batch(es)), "
-                       f"{'global-norm clip, ' if b.clip > 0 else ''}"
+                       f"{clip_label}"
                        "then AdamW from fp32 accumulators, ping-pong state"}[b.path]
                     + " + device loss-scale update + ZeRO-3 gather of every layer",
             "gather": (f"{len(b.gather_buckets)} bucketed launches of consecutive layers "

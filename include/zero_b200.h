@@ -271,15 +271,38 @@ zero_status zero_reduce_scatter_bucket(zero_ctx_t* ctx, int64_t bucket, const vo
  *   acc[o][i - o*S] = acc[o][i - o*S] + (((f32(g_0[i]) + f32(g_1[i])) + ...) + f32(g_{R-1}[i]))
  * The overflow flag is OR-ed with "some accumulator is inf or NaN". The
  * first micro-batch of a step must not accumulate (it initializes).
+ * ZERO_RS_NORM also takes the call's share of the squared norm that global
+ * clipping needs, from the accumulator values it writes, as the step would
+ * form the unscaled gradient:
+ *   sum over the range of (double)((float)(acc * inv))^2,
+ *   inv = (float)(1 / ((R * d) * scale)),
+ * d the context's gradient divisor (zero_ctx_set_grad_divisor, default 1)
+ * and scale the loss scale at launch time (1 without loss scaling). The
+ * share lands in a device slot of the bucket (of the whole range for
+ * bucket -1), which a two-pass zero_step_ex with ZERO_STEP_NORM_FROM_RS
+ * sums instead of re-reading every accumulator. Give the flag to the last
+ * micro-batch's call, the one that leaves the accumulator final; a later
+ * call on the bucket without it (or a call on the whole range) makes the
+ * slot stale, and the step refuses stale or missing slots.
  * Defines: gradient accumulation is not on the pages, which only note that
  * ZeRO frees memory for larger effective batches ([instr], large-batch
  * paragraph); the reduce-scatter itself is [legal] "Reduce-Scatter".
+ * Clipping is not on the pages either.
  * Errors: as zero_reduce_scatter_bucket, plus ZERO_ERR_INVALID_ARG for
  * unknown flags.
  */
 #define ZERO_RS_ACCUMULATE 1
+#define ZERO_RS_NORM 2
 zero_status zero_reduce_scatter_bucket_ex(zero_ctx_t* ctx, int64_t bucket, const void* const* grads,
                                           float* const* acc, int32_t flags, void* stream);
+
+/*
+ * zero_ctx_set_grad_divisor -- the gradient divisor d (>= 1, finite) that
+ * later ZERO_RS_NORM reduce-scatters unscale by; the step checks that its
+ * own grad_divisor equals the one each slot was taken with. Host state
+ * only. Errors: ZERO_ERR_INVALID_ARG.
+ */
+zero_status zero_ctx_set_grad_divisor(zero_ctx_t* ctx, double grad_divisor);
 
 /*
  * zero_step -- one optimizer step on every shard, then the loss-scale update.
@@ -333,11 +356,13 @@ zero_status zero_step(zero_ctx_t* ctx, const zero_adamw* hp, const zero_state* s
  *    double, and the update uses g * c (one fp32 multiply). Clipping needs
  *    the norm before any element is updated, so one read-only pass comes
  *    first: over the accumulators on the two-pass path (4 bytes per
- *    element), over the R replicas on the fused path (2R bytes per element;
- *    they are summed in rank order as the step sums them). The fused path
- *    with clipping moves 4R + 26 bytes per element against 2R + 38 for the
- *    two-pass path, so it is the cheaper one for R <= 5. The recorded
- *    grad_norm_sq is the norm before clipping.
+ *    element; none with ZERO_STEP_NORM_FROM_RS), over the R replicas on the
+ *    fused path (2R bytes per element; they are summed in rank order as the
+ *    step sums them). The fused path with clipping moves 4R + 26 bytes per
+ *    element against 2R + 34 for the two-pass path with the reduce-scatters'
+ *    norm shares (2R + 38 with the pass), so it is the cheaper one for
+ *    R <= 3 and even at R = 4. The recorded grad_norm_sq is the norm before
+ *    clipping.
  *  flags & ZERO_STEP_ADD_ACC (fused path, the last micro-batch of an
  *    accumulation): the reduced gradient is state->acc[o] plus this
  *    micro-batch's rank-order sum of the replicas,
@@ -348,13 +373,24 @@ zero_status zero_step(zero_ctx_t* ctx, const zero_adamw* hp, const zero_state* s
  *    (2R + 8) + 30. The accumulator is read only. Not combinable with
  *    clipping (whose norm needs the sum before the update): use the two-pass
  *    path for that.
+ *  flags & ZERO_STEP_NORM_FROM_RS (two-pass path with clipping): the
+ *    global norm is the sum, in slot order, of the norm shares that this
+ *    step's ZERO_RS_NORM reduce-scatters recorded (every bucket's slot, or
+ *    the whole-range slot), instead of a read-only pass over the
+ *    accumulators: 2R + 34 bytes per element instead of 2R + 38. Refused
+ *    (ZERO_ERR_STATE) unless every slot it needs is current and was taken
+ *    with this call's grad_divisor. Every zero_step_ex marks the slots
+ *    used up.
  * Defines: not on the pages (clipping and accumulation are common practice
  * around ZeRO training loops, not part of the method the pages describe).
  * Errors: as zero_step, plus ZERO_ERR_INVALID_ARG for a divisor < 1, a
- * negative or non-finite max norm, unknown flags, or ZERO_STEP_ADD_ACC
- * without grads, without state->acc or with clipping.
+ * negative or non-finite max norm, unknown flags, ZERO_STEP_ADD_ACC
+ * without grads, without state->acc or with clipping, or
+ * ZERO_STEP_NORM_FROM_RS with grads or without clipping; ZERO_ERR_STATE for
+ * ZERO_STEP_NORM_FROM_RS without current norm slots.
  */
 #define ZERO_STEP_ADD_ACC 1
+#define ZERO_STEP_NORM_FROM_RS 2
 typedef struct {
     double grad_divisor;
     double max_grad_norm;

@@ -141,10 +141,17 @@ class Case:
         self.g.check()
         return skipped
 
-    def step_ex(self, n_micro, grad_divisor=1.0, max_grad_norm=0.0, inject=None):
+    def step_ex(self, n_micro, grad_divisor=1.0, max_grad_norm=0.0, inject=None, rs_norm=False,
+                whole=False):
         """Two-pass step over n_micro accumulated micro-batches, optionally
-        clipped; inject: (micro, rank, element, bits) tuples."""
+        clipped; inject: (micro, rank, element, bits) tuples. rs_norm: the
+        last micro-batch's reduce-scatters record the clipping norm
+        (ZERO_RS_NORM) and the step sums their shares; whole: one
+        reduce-scatter over the whole range per micro-batch."""
         assert self.path.startswith("twopass")
+        norm_flag = Z.ZERO_RS_NORM if rs_norm else 0
+        if rs_norm:
+            Z.zero_ctx_set_grad_divisor(self.ctx, grad_divisor)
         self.step_no += 1
         scale = self.ofsm.scale if self.mode != O.SCALE_NONE else 1.0
         micro = []
@@ -160,10 +167,11 @@ class Case:
                 gp = np.zeros(self.plan.T, np.uint16)
                 gp[self.idx] = g[mu, r]
                 self.grads[r].view(torch.int16).copy_(torch.from_numpy(gp.view(np.int16)))
-            for b in range(len(self.plan.buckets)):
-                Z.zero_reduce_scatter_bucket_ex(self.ctx, b, self.grads, self.acc,
-                                                Z.ZERO_RS_ACCUMULATE if mu else 0)
-        Z.zero_step_ex(self.ctx, self.hp, self.handle, None, grad_divisor, max_grad_norm)
+            flags = (Z.ZERO_RS_ACCUMULATE if mu else 0) | (norm_flag if mu == n_micro - 1 else 0)
+            for b in ([-1] if whole else range(len(self.plan.buckets))):
+                Z.zero_reduce_scatter_bucket_ex(self.ctx, b, self.grads, self.acc, flags)
+        Z.zero_step_ex(self.ctx, self.hp, self.handle, None, grad_divisor, max_grad_norm,
+                       flags=Z.ZERO_STEP_NORM_FROM_RS if rs_norm else 0)
         skipped = O.step_ex(self.ostate, g, O.AdamW(**{k: self.hp[k] for k in
                                                        ("lr", "beta1", "beta2", "eps",
                                                         "weight_decay")}),
@@ -189,12 +197,15 @@ class Case:
         self.g.check()
         return skipped
 
-    def step_overlap(self, n_micro=1, grad_divisor=1.0, max_grad_norm=0.0, busy=None):
+    def step_overlap(self, n_micro=1, grad_divisor=1.0, max_grad_norm=0.0, busy=None, rs_norm=False):
         """Two-pass step whose reduce-scatters are issued by the overlap
         scheduler: each tensor's gradients are written on the caller's stream
         (after `busy` work, standing in for backward) in reverse tensor order,
-        then reported ready; join; step."""
+        then reported ready; join; step. rs_norm: the last micro-batch's
+        reduce-scatters record the clipping norm."""
         assert self.path.startswith("twopass")
+        if rs_norm:
+            Z.zero_ctx_set_grad_divisor(self.ctx, grad_divisor)
         self.step_no += 1
         scale = self.ofsm.scale if self.mode != O.SCALE_NONE else 1.0
         micro = []
@@ -215,12 +226,13 @@ class Case:
                 off, n, st = int(self.lay.offsets[k]), int(self.lay.numels[k]), int(starts[k])
                 for r in range(self.R):
                     self.grads[r].view(torch.int16)[off:off + n].copy_(dev[mu][r, st:st + n])
-                Z.zero_grads_ready(self.ctx, k, 1, self.grads, self.acc,
-                                   Z.ZERO_RS_ACCUMULATE if mu else 0,
+                flags = (Z.ZERO_RS_ACCUMULATE if mu else 0) | \
+                    (Z.ZERO_RS_NORM if rs_norm and mu == n_micro - 1 else 0)
+                Z.zero_grads_ready(self.ctx, k, 1, self.grads, self.acc, flags,
                                    torch.cuda.current_stream())
             Z.zero_grads_join(self.ctx, torch.cuda.current_stream())
         Z.zero_step_ex(self.ctx, self.hp, self.handle, None, grad_divisor, max_grad_norm,
-                       torch.cuda.current_stream())
+                       torch.cuda.current_stream(), flags=Z.ZERO_STEP_NORM_FROM_RS if rs_norm else 0)
         skipped = O.step_ex(self.ostate, g, O.AdamW(**{k: self.hp[k] for k in
                                                        ("lr", "beta1", "beta2", "eps",
                                                         "weight_decay")}),

@@ -154,3 +154,94 @@ def test_add_acc_argument_errors():
             Z.zero_step_ex(c.ctx, c.hp, no_acc, c.grads, 1.0, 0.0, flags=Z.ZERO_STEP_ADD_ACC)
     finally:
         c.close()
+
+
+@pytest.mark.parametrize("R", [2, 3, 8, 16])
+@pytest.mark.parametrize("dtype", [O.BF16, O.FP16])
+@pytest.mark.parametrize("n_micro,divisor", [(1, 1.0), (2, 2.0), (3, 3.0)])
+@pytest.mark.parametrize("clip", [1e-3, 1e9])
+@pytest.mark.parametrize("whole", [False, True])
+def test_norm_from_reduce_scatter_matches_oracle(R, dtype, n_micro, divisor, clip, whole):
+    # the clipping norm taken by the last micro-batch's reduce-scatters
+    # (ZERO_RS_NORM) instead of a pass over the accumulators: the same bytes
+    mode = O.SCALE_DYNAMIC if dtype == O.FP16 else O.SCALE_NONE
+    c = Case([70_001, 13, 4096, 7, 999], R, dtype, 8 if R != 3 else 1, mode, init_scale=256.0,
+             interval=2, path="twopass_pp" if R != 16 else "twopass", bucket_elems=5000)
+    try:
+        for _ in range(3):
+            c.step_ex(n_micro, divisor, clip, rs_norm=True, whole=whole)
+            c.compare()
+        if clip == 1e-3:
+            assert c.ofsm.grad_norm_sq > 1e-4
+    finally:
+        c.close()
+
+
+def test_norm_from_reduce_scatter_skips_on_overflow():
+    c = Case([5000, 33], 4, O.FP16, 8, O.SCALE_DYNAMIC, init_scale=64.0, path="twopass_pp",
+             bucket_elems=1000)
+    try:
+        c.step_ex(2, 2.0, 0.5, rs_norm=True)
+        c.compare()
+        before = c.gpu_state()
+        assert c.step_ex(2, 2.0, 0.5, inject=[(1, 2, 40, 0x7C00)], rs_norm=True)
+        assert c.gpu_fsm()["last_skipped"] == 1
+        c.compare()
+        after = c.gpu_state()
+        for k in ("master", "m", "v", "param"):
+            assert np.array_equal(before[k], after[k])
+        c.step_ex(2, 2.0, 0.5, rs_norm=True)
+        c.compare()
+    finally:
+        c.close()
+
+
+def test_norm_from_reduce_scatter_refusals():
+    c = Case([3000, 17, 2048], 4, O.BF16, 8, O.SCALE_NONE, path="twopass", bucket_elems=1000)
+    nb = len(c.plan.buckets)
+    assert nb >= 3
+    norm_step = dict(flags=Z.ZERO_STEP_NORM_FROM_RS)
+    try:
+        with pytest.raises(Z.ZeroError) as e:
+            Z.zero_ctx_set_grad_divisor(c.ctx, 0.5)
+        assert e.value.status == Z.ZERO_ERR_INVALID_ARG
+        # no reduce-scatter recorded a norm share
+        with pytest.raises(Z.ZeroError) as e:
+            Z.zero_step_ex(c.ctx, c.hp, c.handle, None, 1.0, 1.0, **norm_step)
+        assert e.value.status == Z.ZERO_ERR_STATE
+        # every bucket with its share, then bucket 1 again without: stale
+        for b in range(nb):
+            Z.zero_reduce_scatter_bucket_ex(c.ctx, b, c.grads, c.acc, Z.ZERO_RS_NORM)
+        Z.zero_reduce_scatter_bucket_ex(c.ctx, 1, c.grads, c.acc, 0)
+        with pytest.raises(Z.ZeroError) as e:
+            Z.zero_step_ex(c.ctx, c.hp, c.handle, None, 1.0, 1.0, **norm_step)
+        assert e.value.status == Z.ZERO_ERR_STATE
+        # shares taken with another divisor
+        Z.zero_ctx_set_grad_divisor(c.ctx, 2.0)
+        for b in range(nb):
+            Z.zero_reduce_scatter_bucket_ex(c.ctx, b, c.grads, c.acc, Z.ZERO_RS_NORM)
+        with pytest.raises(Z.ZeroError) as e:
+            Z.zero_step_ex(c.ctx, c.hp, c.handle, None, 1.0, 1.0, **norm_step)
+        assert e.value.status == Z.ZERO_ERR_STATE
+        # a whole-range call without the flag makes every share stale
+        Z.zero_reduce_scatter_bucket_ex(c.ctx, -1, c.grads, c.acc, 0)
+        with pytest.raises(Z.ZeroError) as e:
+            Z.zero_step_ex(c.ctx, c.hp, c.handle, None, 2.0, 1.0, **norm_step)
+        assert e.value.status == Z.ZERO_ERR_STATE
+        # the flag needs the two-pass path and clipping
+        with pytest.raises(Z.ZeroError) as e:
+            Z.zero_step_ex(c.ctx, c.hp, c.handle, None, 1.0, 0.0, **norm_step)
+        assert e.value.status == Z.ZERO_ERR_INVALID_ARG
+        with pytest.raises(Z.ZeroError) as e:
+            Z.zero_step_ex(c.ctx, c.hp, c.handle, c.grads, 1.0, 1.0, **norm_step)
+        assert e.value.status == Z.ZERO_ERR_INVALID_ARG
+        # nothing above stepped: a proper step still matches the oracle
+        Z.zero_ctx_set_grad_divisor(c.ctx, 1.0)
+        c.step_ex(1, 1.0, 1e-3, rs_norm=True)
+        c.compare()
+        # a step consumes the shares
+        with pytest.raises(Z.ZeroError) as e:
+            Z.zero_step_ex(c.ctx, c.hp, c.handle, None, 1.0, 1.0, **norm_step)
+        assert e.value.status == Z.ZERO_ERR_STATE
+    finally:
+        c.close()

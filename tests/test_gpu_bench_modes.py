@@ -1,0 +1,28 @@
+"""bench.py's two-pass clipping modes run end to end and say which norm
+they used (the reduce-scatters' shares or a separate pass)."""
+import json
+import os
+import subprocess
+import sys
+
+import pytest
+
+pytestmark = pytest.mark.gpu
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.mark.parametrize("clip_norm,accum", [("rs", 1), ("rs", 3), ("pass", 3)])
+def test_two_pass_clip_bench(clip_norm, accum):
+    cmd = ["timeout", "-k", "30", "600", sys.executable, os.path.join(ROOT, "bench.py"),
+           "--path", "twopass", "--clip", "1.0", "--accum", str(accum), "--clip-norm", clip_norm,
+           "--first-tensors", "6", "--steps", "3", "--warmup", "3", "--no-e2e", "--no-cpu-baseline"]
+    r = subprocess.run(cmd, capture_output=True, text=True, cwd=ROOT)
+    assert r.returncode == 0, (r.stdout[-3000:], r.stderr[-3000:])
+    out = json.loads([ln for ln in r.stdout.splitlines() if ln.startswith("{")][-1])
+    path = out["config"]["path"]
+    if clip_norm == "rs":
+        assert "norm shares" in path
+    else:
+        assert "clip pass" in path
+    assert out["value"] > 0 and out["roofline"]["achieved"] > 0

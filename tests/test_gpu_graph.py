@@ -70,7 +70,10 @@ def test_replayed_fused_step_matches_oracle(R, dtype):
         c.close()
 
 
-def test_replayed_two_pass_step_with_clipping_matches_oracle():
+@pytest.mark.parametrize("rs_norm", [False, True])
+def test_replayed_two_pass_step_with_clipping_matches_oracle(rs_norm):
+    # rs_norm: the reduce-scatters take the clipping norm; their per-bucket
+    # counters re-arm themselves, so every replay sums fresh shares
     c = Case([50_000, 333, 8_192], 4, O.BF16, mode=O.SCALE_NONE, path="twopass",
              bucket_elems=20_000, seed=62)
     try:
@@ -79,8 +82,9 @@ def test_replayed_two_pass_step_with_clipping_matches_oracle():
 
         def step(s):
             for b in range(nb):
-                Z.zero_reduce_scatter_bucket(c.ctx, b, c.grads, c.acc, s)
-            Z.zero_step_ex(c.ctx, c.hp, c.handle, None, 1.0, 1e-3, s)
+                Z.zero_reduce_scatter_bucket_ex(c.ctx, b, c.grads, c.acc, Z.ZERO_RS_NORM if rs_norm else 0, s)
+            Z.zero_step_ex(c.ctx, c.hp, c.handle, None, 1.0, 1e-3, s,
+                           flags=Z.ZERO_STEP_NORM_FROM_RS if rs_norm else 0)
 
         graph = _capture(step)
         for _ in range(4):

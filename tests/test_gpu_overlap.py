@@ -48,6 +48,26 @@ def test_overlapped_reduce_scatter_matches_oracle(R, dtype, n_micro, comm_sms):
         c.close()
 
 
+@pytest.mark.parametrize("R,dtype", [(4, O.BF16), (8, O.FP16)])
+@pytest.mark.parametrize("n_micro", [1, 3])
+@pytest.mark.parametrize("comm_sms", [0, 2])
+def test_overlapped_reduce_scatter_with_norm_matches_oracle(R, dtype, n_micro, comm_sms):
+    # clipping whose norm the overlapped reduce-scatters take (ZERO_RS_NORM on
+    # the last micro-batch): the step reads no accumulator before updating
+    numels = [70_001, 13, 4096, 7, 999, 30_000, 5]
+    mode = O.SCALE_DYNAMIC if dtype == O.FP16 else O.SCALE_NONE
+    c = Case(numels, R, dtype, 8, mode, init_scale=256.0, interval=3, path="twopass",
+             bucket_elems=20_000)
+    busy = make_busy()
+    Z.zero_sched_set_comm_sms(c.ctx, comm_sms)
+    try:
+        for clip in (1e-3, 1e9, 2e-3):
+            c.step_overlap(n_micro, float(n_micro), clip, busy, rs_norm=True)
+            c.compare()
+    finally:
+        c.close()
+
+
 def test_grads_join_refuses_missing_and_repeated_reports():
     c = Case([100, 200, 300], 2, O.BF16, 8, O.SCALE_NONE, path="twopass", bucket_elems=250)
     try:

@@ -22,7 +22,9 @@ ZERO_BF16, ZERO_FP16 = 0, 1
 ZERO_SCALE_NONE, ZERO_SCALE_STATIC, ZERO_SCALE_DYNAMIC = 0, 1, 2
 ZERO_LOSS_SCALE_GET, ZERO_LOSS_SCALE_SET = 0, 1
 ZERO_RS_ACCUMULATE = 1
+ZERO_RS_NORM = 2
 ZERO_STEP_ADD_ACC = 1
+ZERO_STEP_NORM_FROM_RS = 2
 
 STATUS_NAMES = {0: "ZERO_OK", 1: "ZERO_ERR_INVALID_ARG", 2: "ZERO_ERR_ALIGN", 3: "ZERO_ERR_CUDA",
                 4: "ZERO_ERR_OOM", 5: "ZERO_ERR_RANGE", 6: "ZERO_ERR_TIMEOUT", 7: "ZERO_ERR_STATE"}
@@ -110,6 +112,7 @@ _sig("zero_plan_memory", _S, [_P, C.c_int32, C.POINTER(C.c_int64)])
 _sig("zero_ctx_create", _S, [_P, C.POINTER(zero_loss_scale_config), C.POINTER(_P)])
 _sig("zero_ctx_destroy", _S, [_P])
 _sig("zero_ctx_reserve_steps", _S, [_P, C.c_int64, C.c_double, C.c_double, _P])
+_sig("zero_ctx_set_grad_divisor", _S, [_P, C.c_double])
 _sig("zero_test_drop_tile", _S, [_P, C.c_int64])
 _sig("zero_reduce_scatter_bucket", _S, [_P, C.c_int64, _PP, _PP, _P])
 _sig("zero_step", _S, [_P, C.POINTER(zero_adamw), C.POINTER(zero_state), _PP, _P])
@@ -285,8 +288,14 @@ def zero_reduce_scatter_bucket(ctx, bucket, grads, acc, stream=None):
     _check(_lib.zero_reduce_scatter_bucket(ctx, bucket, g, a, _stream(stream)))
 
 
+def zero_ctx_set_grad_divisor(ctx, grad_divisor):
+    """The divisor that ZERO_RS_NORM reduce-scatters unscale by."""
+    _check(_lib.zero_ctx_set_grad_divisor(ctx, float(grad_divisor)))
+
+
 def zero_reduce_scatter_bucket_ex(ctx, bucket, grads, acc, flags=0, stream=None):
-    """flags: ZERO_RS_ACCUMULATE adds to the accumulators."""
+    """flags: ZERO_RS_ACCUMULATE adds to the accumulators; ZERO_RS_NORM also
+    records the bucket's share of the clipping norm."""
     g, ga = _ptr_array(grads)
     a, aa = _ptr_array(acc)
     _check(_lib.zero_reduce_scatter_bucket_ex(ctx, bucket, g, a, flags, _stream(stream)))
@@ -305,7 +314,8 @@ def zero_step(ctx, hp, state: StateHandle, grads=None, stream=None):
 def zero_step_ex(ctx, hp, state: StateHandle, grads=None, grad_divisor=1.0, max_grad_norm=0.0,
                  stream=None, flags=0):
     """zero_step with a grad divisor, global-norm clipping and flags
-    (ZERO_STEP_ADD_ACC: the fused step adds state's accumulators)."""
+    (ZERO_STEP_ADD_ACC: the fused step adds state's accumulators;
+    ZERO_STEP_NORM_FROM_RS: the clipping norm from the reduce-scatters' shares)."""
     if isinstance(hp, dict):
         hp = zero_adamw(hp["lr"], hp["beta1"], hp["beta2"], hp["eps"], hp["weight_decay"])
     g = None

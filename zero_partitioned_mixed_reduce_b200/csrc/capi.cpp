@@ -185,11 +185,25 @@ extern "C" zero_status zero_ctx_create(const zero_plan_t* plan, const zero_loss_
     ctx->cfg = *cfg;
     ctx->grid_cap = zb::step_grid_cap(ctx->device);
 
+    // norm-share slots: one per bucket and one for the whole range
+    const size_t slots = ctx->bucket_lo.size() + 1;
+    ctx->rs_norm_valid.assign(slots, 0);
+    ctx->rs_norm_div.assign(slots, 1.0);
+    auto free_scratch = [ctx] {
+        cudaFree(ctx->st);
+        cudaFree(ctx->partials);
+        cudaFree(ctx->rs_norm_partials);
+        cudaFree(ctx->rs_norm_done);
+        cudaFree(ctx->rs_norm);
+    };
     e = cudaMalloc(&ctx->st, sizeof(zb::DevState));
     if (e == cudaSuccess) e = cudaMalloc(&ctx->partials, sizeof(double) * ctx->grid_cap);
+    if (e == cudaSuccess) e = cudaMalloc(&ctx->rs_norm_partials, sizeof(double) * ctx->grid_cap * slots);
+    if (e == cudaSuccess) e = cudaMalloc(&ctx->rs_norm_done, sizeof(uint32_t) * slots);
+    if (e == cudaSuccess) e = cudaMalloc(&ctx->rs_norm, sizeof(double) * slots);
     if (e != cudaSuccess) {
         cudaGetLastError();
-        if (ctx->st) cudaFree(ctx->st);
+        free_scratch();
         delete ctx;
         return zb_fail(ZERO_ERR_OOM, "zero_ctx_create: cannot allocate device scratch");
     }
@@ -197,14 +211,44 @@ extern "C" zero_status zero_ctx_create(const zero_plan_t* plan, const zero_loss_
     init.scale = cfg->mode == ZERO_SCALE_NONE ? 1.0f : cfg->init_scale;
     e = cudaMemcpy(ctx->st, &init, sizeof(init), cudaMemcpyHostToDevice);
     if (e == cudaSuccess) e = cudaMemset(ctx->partials, 0, sizeof(double) * ctx->grid_cap);
+    if (e == cudaSuccess) e = cudaMemset(ctx->rs_norm_done, 0, sizeof(uint32_t) * slots);
+    if (e == cudaSuccess) e = cudaMemset(ctx->rs_norm, 0, sizeof(double) * slots);
     if (e != cudaSuccess) {
-        cudaFree(ctx->st);
-        cudaFree(ctx->partials);
+        free_scratch();
         delete ctx;
         return cuda_fail("zero_ctx_create", e);
     }
     *out = ctx;
     return ZERO_OK;
+}
+
+extern "C" zero_status zero_ctx_set_grad_divisor(zero_ctx_t* ctx, double grad_divisor) {
+    if (!ctx) return zb_fail(ZERO_ERR_INVALID_ARG, "zero_ctx_set_grad_divisor: ctx is NULL");
+    if (!(grad_divisor >= 1.0) || !std::isfinite(grad_divisor))
+        return zb_fail(ZERO_ERR_INVALID_ARG, "zero_ctx_set_grad_divisor: need a finite divisor >= 1");
+    ctx->grad_divisor = grad_divisor;
+    return ZERO_OK;
+}
+
+zb::RsNorm zb_rs_norm_note(zero_ctx_t* ctx, int64_t bucket, bool norm) {
+    const size_t whole = ctx->bucket_lo.size();
+    const size_t slot = bucket < 0 ? whole : static_cast<size_t>(bucket);
+    if (bucket < 0) {
+        // the whole range is rewritten: every per-bucket share is stale
+        std::fill(ctx->rs_norm_valid.begin(), ctx->rs_norm_valid.end(), 0);
+    } else {
+        ctx->rs_norm_valid[whole] = 0;
+    }
+    ctx->rs_norm_valid[slot] = norm ? 1 : 0;
+    zb::RsNorm n;
+    if (!norm) return n;
+    ctx->rs_norm_div[slot] = ctx->grad_divisor;
+    n.partials = ctx->rs_norm_partials + slot * static_cast<size_t>(ctx->grid_cap);
+    n.done = ctx->rs_norm_done + slot;
+    n.out = ctx->rs_norm + slot;
+    n.mode = ctx->cfg.mode;
+    n.divisor = ctx->grad_divisor;
+    return n;
 }
 
 extern "C" zero_status zero_ctx_destroy(zero_ctx_t* ctx) {
@@ -216,6 +260,9 @@ extern "C" zero_status zero_ctx_destroy(zero_ctx_t* ctx) {
     zb_sched_destroy(ctx);
     cudaFree(ctx->st);
     cudaFree(ctx->partials);
+    cudaFree(ctx->rs_norm_partials);
+    cudaFree(ctx->rs_norm_done);
+    cudaFree(ctx->rs_norm);
     if (ctx->powtab) cudaFree(ctx->powtab);
     for (double2* old : ctx->powtab_retired) cudaFree(old);
     if (prev >= 0) cudaSetDevice(prev);
@@ -252,7 +299,7 @@ extern "C" zero_status zero_reduce_scatter_bucket_ex(zero_ctx_t* ctx, int64_t bu
                                                      const void* const* grads, float* const* acc,
                                                      int32_t flags, void* stream) {
     const char* where = "zero_reduce_scatter_bucket";
-    if (flags & ~ZERO_RS_ACCUMULATE)
+    if (flags & ~(ZERO_RS_ACCUMULATE | ZERO_RS_NORM))
         return zb_fail(ZERO_ERR_INVALID_ARG, "zero_reduce_scatter_bucket_ex: unknown flags");
     if (!ctx) return zb_fail(ZERO_ERR_INVALID_ARG, "zero_reduce_scatter_bucket: ctx is NULL");
     zero_status s = check_device(ctx, where);
@@ -274,10 +321,15 @@ extern "C" zero_status zero_reduce_scatter_bucket_ex(zero_ctx_t* ctx, int64_t bu
         p.g[r] = grads[r];
         p.acc[r] = acc[r];
     }
+    const zb::RsNorm norm = zb_rs_norm_note(ctx, bucket, (flags & ZERO_RS_NORM) != 0);
     cudaError_t e = zb::launch_reduce_scatter(ctx->R, ctx->dtype, ctx->S, lo, hi, ctx->st, p,
                                               static_cast<cudaStream_t>(stream),
-                                              (flags & ZERO_RS_ACCUMULATE) != 0);
-    if (e != cudaSuccess) return cuda_fail(where, e);
+                                              (flags & ZERO_RS_ACCUMULATE) != 0, 0,
+                                              norm.partials ? &norm : nullptr);
+    if (e != cudaSuccess) {
+        ctx->rs_norm_valid[bucket < 0 ? ctx->bucket_lo.size() : static_cast<size_t>(bucket)] = 0;
+        return cuda_fail(where, e);
+    }
     return ZERO_OK;
 }
 
@@ -345,11 +397,15 @@ zero_status check_step_opts(const zero_step_opts* opts, bool fused, const char* 
         !std::isfinite(o.max_grad_norm) || o.reserved != 0)
         return zb_fail(ZERO_ERR_INVALID_ARG,
                        std::string(where) + ": need grad_divisor >= 1, finite max_grad_norm >= 0, reserved 0");
-    if (o.flags & ~static_cast<int64_t>(ZERO_STEP_ADD_ACC))
+    if (o.flags & ~static_cast<int64_t>(ZERO_STEP_ADD_ACC | ZERO_STEP_NORM_FROM_RS))
         return zb_fail(ZERO_ERR_INVALID_ARG, std::string(where) + ": unknown flags");
     if ((o.flags & ZERO_STEP_ADD_ACC) && (!fused || o.max_grad_norm > 0.0))
         return zb_fail(ZERO_ERR_INVALID_ARG,
                        std::string(where) + ": ZERO_STEP_ADD_ACC needs the fused path (grads) and no clipping");
+    if ((o.flags & ZERO_STEP_NORM_FROM_RS) && (fused || !(o.max_grad_norm > 0.0)))
+        return zb_fail(ZERO_ERR_INVALID_ARG, std::string(where) +
+                                                 ": ZERO_STEP_NORM_FROM_RS needs the two-pass path "
+                                                 "(no grads) and clipping");
     *out = o;
     return ZERO_OK;
 }
@@ -423,12 +479,39 @@ extern "C" zero_status zero_step_ex(zero_ctx_t* ctx, const zero_adamw* hp, const
         p.g[r] = fused ? grads[r] : nullptr;
         p.acc[r] = (!fused || add_acc) ? state->acc[r] : nullptr;
     }
+    // with ZERO_STEP_NORM_FROM_RS: the current norm slots, whole range or
+    // every bucket, each taken with this step's divisor
+    const size_t nb = ctx->bucket_lo.size();
+    int64_t slot_first = 0, slot_count = 0;
+    if (o.flags & ZERO_STEP_NORM_FROM_RS) {
+        auto ok = [&](size_t k) { return ctx->rs_norm_valid[k] && ctx->rs_norm_div[k] == o.grad_divisor; };
+        bool all = true;
+        for (size_t b = 0; b < nb && all; ++b) all = ok(b);
+        if (ok(nb)) {
+            slot_first = static_cast<int64_t>(nb);
+            slot_count = 1;
+        } else if (all) {
+            slot_count = static_cast<int64_t>(nb);
+        } else {
+            return zb_fail(ZERO_ERR_STATE,
+                           "zero_step: ZERO_STEP_NORM_FROM_RS, but the reduce-scatters since the last step did "
+                           "not record a current norm share of every bucket with this grad_divisor");
+        }
+    }
     cudaError_t e = cudaSuccess;
-    // clipping needs the global norm before any element is updated: one
-    // read-only pass over the accumulators, or over the replicas when fused
-    if (sp.clip) e = fused ? zb::launch_grad_norm(sp, p, cs) : zb::launch_clip_norm(sp, p, cs);
+    // clipping needs the global norm before any element is updated: the
+    // reduce-scatters' shares, or one read-only pass over the accumulators,
+    // or over the replicas when fused
+    if (sp.clip) {
+        if (slot_count > 0)
+            e = zb::launch_clip_from_rs_norm(sp, ctx->rs_norm, slot_first, slot_count, cs);
+        else
+            e = fused ? zb::launch_grad_norm(sp, p, cs) : zb::launch_clip_norm(sp, p, cs);
+    }
     if (e == cudaSuccess)
         e = fused ? zb::launch_fused_step(sp, p, cs) : zb::launch_step_from_acc(sp, p, cs);
+    // the accumulators are consumed: the next step's shares start afresh
+    std::fill(ctx->rs_norm_valid.begin(), ctx->rs_norm_valid.end(), 0);
     if (e != cudaSuccess) return cuda_fail(where, e);
     ctx->t_bound += 1;
     if (fused) ctx->drop_tile = 0xffffffffu;
@@ -491,6 +574,7 @@ extern "C" zero_status zero_reduce_scatter_shard(zero_ctx_t* ctx, int64_t bucket
     // the bucket's part inside the owners' flat range [owner_lo * S, owner_hi * S)
     lo = std::max<int64_t>(lo, static_cast<int64_t>(owner_lo) * ctx->S);
     hi = std::min<int64_t>(hi, static_cast<int64_t>(owner_hi) * ctx->S);
+    zb_rs_norm_note(ctx, bucket, false);  // the bucket's norm share (if any) is stale now
     if (lo >= hi) return ZERO_OK;  // no element of this bucket is owned here
     zb::RankPtrs p{};
     for (int r = 0; r < ctx->R; ++r) {

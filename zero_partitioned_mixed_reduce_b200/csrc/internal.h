@@ -75,6 +75,18 @@ struct RankPtrs {
     void* param[2][ZERO_MAX_RANKS];
 };
 
+// A reduce-scatter's share of the clipping norm (ZERO_RS_NORM): the launch
+// adds up sum((float)(acc * inv))^2 over the accumulator values it writes,
+// inv = 1 / ((R * divisor) * scale), one partial per block in `partials`
+// (grid capacity entries), the last block storing the total in *out.
+struct RsNorm {
+    double* partials = nullptr;
+    uint32_t* done = nullptr;
+    double* out = nullptr;
+    int32_t mode = 0;
+    double divisor = 1.0;
+};
+
 // Kernel launchers (kernels.cu). Each returns the launch's cudaError_t.
 cudaError_t launch_fused_step(const StepParams& sp, const RankPtrs& p, cudaStream_t s);
 cudaError_t launch_step_from_acc(const StepParams& sp, const RankPtrs& p, cudaStream_t s);
@@ -83,7 +95,10 @@ cudaError_t launch_step_from_acc(const StepParams& sp, const RankPtrs& p, cudaSt
 // concurrent compute); 0 = the whole GPU.
 cudaError_t launch_reduce_scatter(int32_t R, int32_t dtype, int64_t S, int64_t lo, int64_t hi,
                                   DevState* st, const RankPtrs& p, cudaStream_t s,
-                                  bool accumulate = false, int max_sms = 0);
+                                  bool accumulate = false, int max_sms = 0, const RsNorm* norm = nullptr);
+// The clipping coefficient from norm slots [first, first + count).
+cudaError_t launch_clip_from_rs_norm(const StepParams& sp, const double* slots, int64_t first, int64_t count,
+                                     cudaStream_t s);
 // Norm passes over owners [obeg, oend): the last block stores the clipping
 // coefficient, or, with partial_out, the range's sum of g^2 in partial_out[0].
 cudaError_t launch_grad_norm(const StepParams& sp, const RankPtrs& p, cudaStream_t s);
@@ -128,7 +143,21 @@ struct zero_ctx_s {
     bool two_sets = false;        // a ping-pong step has run (or cur was set to 1)
     int32_t shard_pingpong = 0;   // the last zero_step_shard wrote set 1-cur
     zero_sched* sched = nullptr;  // created on first use
+    // reduce-scatter norm shares (ZERO_RS_NORM): one slot per bucket, and
+    // slot n_buckets for a whole-range call; device partials (grid_cap per
+    // slot), counters and totals; on the host, whether each slot holds the
+    // norm of the accumulators as they now stand, and its divisor
+    double* rs_norm_partials = nullptr;
+    uint32_t* rs_norm_done = nullptr;
+    double* rs_norm = nullptr;
+    std::vector<uint8_t> rs_norm_valid;
+    std::vector<double> rs_norm_div;
+    double grad_divisor = 1.0;    // the divisor ZERO_RS_NORM unscales by
 };
+
+// Bookkeeping of a reduce-scatter of `bucket` (-1: whole range), with or
+// without its norm share; returns the launch's norm arguments (capi.cpp).
+zb::RsNorm zb_rs_norm_note(zero_ctx_t* ctx, int64_t bucket, bool norm);
 
 void zb_sched_destroy(zero_ctx_t* ctx);
 

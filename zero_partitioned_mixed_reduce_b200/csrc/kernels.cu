@@ -691,15 +691,58 @@ struct RsArgs {
     int64_t head_end, tail_begin;
     int32_t R;
     DevState* st;
+    RsNorm norm;           // norm.partials == nullptr: no norm share
     const uint4* g[CAP];
     float* acc[CAP];
 };
+
+// 1 / ((R * divisor) * scale) rounded once to fp32, as the step computes it;
+// shared by the block (every thread of the block must call it).
+__device__ __forceinline__ float block_unscale_rs(const RsNorm& n, int32_t R, const DevState* st) {
+    __shared__ float s_inv;
+    if (threadIdx.x == 0) {
+        const volatile DevState* vs = st;
+        const double dscale = n.mode == ZERO_SCALE_NONE ? 1.0 : static_cast<double>(vs->scale);
+        s_inv = __double2float_rn(
+            __ddiv_rn(1.0, __dmul_rn(__dmul_rn(static_cast<double>(R), n.divisor), dscale)));
+    }
+    __syncthreads();
+    return s_inv;
+}
+
+// The launch's share of the squared norm: every block publishes its partial,
+// the last one sums them in block order into *n.out and re-arms the counter.
+__device__ void rs_norm_finish(const RsNorm& n, double nrm) {
+    __shared__ double red[kWarps];
+    __shared__ int last;
+    const double bn = block_sum(nrm, red);
+    if (threadIdx.x == 0) {
+        n.partials[blockIdx.x] = bn;
+        __threadfence();
+        last = (atomicAdd(n.done, 1u) == gridDim.x - 1);
+    }
+    __syncthreads();
+    if (!last) return;
+    __threadfence();
+    double x = 0.0;
+    for (unsigned i = threadIdx.x; i < gridDim.x; i += kThreads)
+        x += *reinterpret_cast<volatile double*>(&n.partials[i]);
+    const double total = block_sum(x, red);
+    if (threadIdx.x == 0) {
+        *n.out = total;
+        *n.done = 0u;
+        __threadfence();
+    }
+}
 
 template <typename H, int RC, bool ACCUM>
 __global__ void __launch_bounds__(kThreads)
     reduce_scatter_kernel(const __grid_constant__ RsArgs<RC == 0 ? ZERO_MAX_RANKS : RC> a) {
     const int R = RC > 0 ? RC : a.R;
     bool bad = false;
+    const bool with_norm = a.norm.partials != nullptr;  // uniform over the grid
+    const float inv = with_norm ? block_unscale_rs(a.norm, R, a.st) : 0.0f;
+    double nrm = 0.0;
     const uint32_t stride = gridDim.x * kThreads;
     const uint32_t tid = blockIdx.x * kThreads + threadIdx.x;
     uint32_t vi = line_start(a.v0, stride);
@@ -736,6 +779,14 @@ __global__ void __launch_bounds__(kThreads)
             out.x[e] = acc[e];
         }
         st_f8(dst, out);
+        if (with_norm) {
+            // the unscaled gradient as the step will form it, squared in double
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                const double gd = static_cast<double>(__fmul_rn(acc[e], inv));
+                nrm = fma(gd, gd, nrm);
+            }
+        }
     }
     // unaligned edges, element by element
     const int64_t nhead = a.head_end - a.lo;
@@ -752,9 +803,14 @@ __global__ void __launch_bounds__(kThreads)
             if constexpr (ACCUM) s = __fadd_rn(*dst, s);
             bad |= nonfinite(s);
             *dst = s;
+            if (with_norm) {
+                const double gd = static_cast<double>(__fmul_rn(s, inv));
+                nrm = fma(gd, gd, nrm);
+            }
         }
     }
     if (__syncthreads_or(bad ? 1 : 0) && threadIdx.x == 0) atomicOr(&a.st->flag, 1u);
+    if (with_norm) rs_norm_finish(a.norm, nrm);
 }
 
 // ---------------------------------------------------------------------------
@@ -961,7 +1017,7 @@ cudaError_t fused_dispatch(const StepParams& sp, const RankPtrs& p, cudaStream_t
 
 template <typename H, int RC, bool ACCUM>
 cudaError_t rs_t(int32_t R, int64_t S, int64_t lo, int64_t hi, DevState* st, const RankPtrs& p,
-                 cudaStream_t s, int max_sms) {
+                 cudaStream_t s, int max_sms, const RsNorm* norm) {
     constexpr int CAP = RC == 0 ? ZERO_MAX_RANKS : RC;
     RsArgs<CAP> a;
     a.lo = lo;
@@ -970,6 +1026,7 @@ cudaError_t rs_t(int32_t R, int64_t S, int64_t lo, int64_t hi, DevState* st, con
     a.S8 = static_cast<uint32_t>(S / 8);
     a.R = R;
     a.st = st;
+    a.norm = norm ? *norm : RsNorm{};
     // aligned body [ceil8(lo), floor8(hi)), if non-empty
     const int64_t vlo = (lo + 7) / 8, vhi = hi / 8;
     if (vlo < vhi) {
@@ -996,14 +1053,14 @@ cudaError_t rs_t(int32_t R, int64_t S, int64_t lo, int64_t hi, DevState* st, con
 
 template <typename H, bool ACCUM>
 cudaError_t rs_dispatch(int32_t R, int64_t S, int64_t lo, int64_t hi, DevState* st,
-                        const RankPtrs& p, cudaStream_t s, int max_sms) {
+                        const RankPtrs& p, cudaStream_t s, int max_sms, const RsNorm* norm) {
     switch (R) {
-        case 1: return rs_t<H, 1, ACCUM>(R, S, lo, hi, st, p, s, max_sms);
-        case 2: return rs_t<H, 2, ACCUM>(R, S, lo, hi, st, p, s, max_sms);
-        case 4: return rs_t<H, 4, ACCUM>(R, S, lo, hi, st, p, s, max_sms);
-        case 8: return rs_t<H, 8, ACCUM>(R, S, lo, hi, st, p, s, max_sms);
-        case 16: return rs_t<H, 16, ACCUM>(R, S, lo, hi, st, p, s, max_sms);
-        default: return rs_t<H, 0, ACCUM>(R, S, lo, hi, st, p, s, max_sms);
+        case 1: return rs_t<H, 1, ACCUM>(R, S, lo, hi, st, p, s, max_sms, norm);
+        case 2: return rs_t<H, 2, ACCUM>(R, S, lo, hi, st, p, s, max_sms, norm);
+        case 4: return rs_t<H, 4, ACCUM>(R, S, lo, hi, st, p, s, max_sms, norm);
+        case 8: return rs_t<H, 8, ACCUM>(R, S, lo, hi, st, p, s, max_sms, norm);
+        case 16: return rs_t<H, 16, ACCUM>(R, S, lo, hi, st, p, s, max_sms, norm);
+        default: return rs_t<H, 0, ACCUM>(R, S, lo, hi, st, p, s, max_sms, norm);
     }
 }
 
@@ -1048,12 +1105,34 @@ cudaError_t launch_step_from_acc(const StepParams& sp, const RankPtrs& p, cudaSt
 
 cudaError_t launch_reduce_scatter(int32_t R, int32_t dtype, int64_t S, int64_t lo, int64_t hi,
                                   DevState* st, const RankPtrs& p, cudaStream_t s, bool accumulate,
-                                  int max_sms) {
+                                  int max_sms, const RsNorm* norm) {
     if (accumulate)
-        return dtype == ZERO_FP16 ? rs_dispatch<Fp16, true>(R, S, lo, hi, st, p, s, max_sms)
-                                  : rs_dispatch<Bf16, true>(R, S, lo, hi, st, p, s, max_sms);
-    return dtype == ZERO_FP16 ? rs_dispatch<Fp16, false>(R, S, lo, hi, st, p, s, max_sms)
-                              : rs_dispatch<Bf16, false>(R, S, lo, hi, st, p, s, max_sms);
+        return dtype == ZERO_FP16 ? rs_dispatch<Fp16, true>(R, S, lo, hi, st, p, s, max_sms, norm)
+                                  : rs_dispatch<Bf16, true>(R, S, lo, hi, st, p, s, max_sms, norm);
+    return dtype == ZERO_FP16 ? rs_dispatch<Fp16, false>(R, S, lo, hi, st, p, s, max_sms, norm)
+                              : rs_dispatch<Bf16, false>(R, S, lo, hi, st, p, s, max_sms, norm);
+}
+
+// The clipping coefficient from the reduce-scatters' norm shares slots
+// [first, first + count), summed in slot order (strided over the block, then
+// the block's fixed reduction tree).
+__global__ void __launch_bounds__(kThreads)
+    clip_from_rs_norm_kernel(const __grid_constant__ StepParams sp, const double* slots, int64_t first,
+                             int64_t count) {
+    __shared__ double red[kWarps];
+    double x = 0.0;
+    for (int64_t i = threadIdx.x; i < count; i += kThreads) x += slots[first + i];
+    const double total = block_sum(x, red);
+    if (threadIdx.x == 0) {
+        sp.st->clip = clip_coefficient(sp.max_norm, total);
+        __threadfence();
+    }
+}
+
+cudaError_t launch_clip_from_rs_norm(const StepParams& sp, const double* slots, int64_t first, int64_t count,
+                                     cudaStream_t s) {
+    clip_from_rs_norm_kernel<<<1, kThreads, 0, s>>>(sp, slots, first, count);
+    return cudaGetLastError();
 }
 
 namespace {

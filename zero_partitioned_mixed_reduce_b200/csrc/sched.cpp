@@ -111,7 +111,8 @@ extern "C" zero_status zero_grads_ready(zero_ctx_t* ctx, int64_t first, int64_t 
     const int64_t n = static_cast<int64_t>(ctx->tensor_bucket.size());
     if (first < 0 || count < 1 || first > n - count)
         return zb_fail(ZERO_ERR_RANGE, "zero_grads_ready: tensor range out of bounds");
-    if (flags & ~ZERO_RS_ACCUMULATE) return zb_fail(ZERO_ERR_INVALID_ARG, "zero_grads_ready: unknown flags");
+    if (flags & ~(ZERO_RS_ACCUMULATE | ZERO_RS_NORM))
+        return zb_fail(ZERO_ERR_INVALID_ARG, "zero_grads_ready: unknown flags");
     if (!grads || !acc) return zb_fail(ZERO_ERR_INVALID_ARG, "zero_grads_ready: NULL grads or acc");
     for (int r = 0; r < ctx->R; ++r) {
         if (!grads[r] || !acc[r]) return zb_fail(ZERO_ERR_INVALID_ARG, "zero_grads_ready: NULL rank pointer");
@@ -136,13 +137,17 @@ extern "C" zero_status zero_grads_ready(zero_ctx_t* ctx, int64_t first, int64_t 
         // the step's last bucket has no compute left to hide behind: whole GPU
         const bool last_bucket = s->buckets_issued + 1 == static_cast<int64_t>(ctx->bucket_lo.size());
         // the whole bucket is ready: reduce-scatter it behind the caller's work
+        const zb::RsNorm norm = zb_rs_norm_note(ctx, b, (flags & ZERO_RS_NORM) != 0);
         cudaError_t e = cudaEventRecord(s->bucket_event[b], cs);
         if (e == cudaSuccess) e = cudaStreamWaitEvent(s->comm, s->bucket_event[b], 0);
         if (e == cudaSuccess)
             e = zb::launch_reduce_scatter(ctx->R, ctx->dtype, ctx->S, ctx->bucket_lo[b], ctx->bucket_hi[b],
                                           ctx->st, p, s->comm, (flags & ZERO_RS_ACCUMULATE) != 0,
-                                          last_bucket ? 0 : s->comm_sms);
-        if (e != cudaSuccess) return cuda_err(where, e);
+                                          last_bucket ? 0 : s->comm_sms, norm.partials ? &norm : nullptr);
+        if (e != cudaSuccess) {
+            ctx->rs_norm_valid[b] = 0;
+            return cuda_err(where, e);
+        }
         s->buckets_issued += 1;
     }
     return ZERO_OK;
