@@ -39,6 +39,10 @@ def main():
                     c.step_fused_accum(3, 3.0)
                 else:
                     c.step_ex(2, 2.0, 1e-3)
+                    c.compare()
+                    c.step_ex(2, 2.0, 1e-3, rs_norm=True)  # the norm from the reduce-scatters
+                    c.compare()
+                    c.step_ex(1, 1.0, 1e-3, rs_norm=True, whole=True)
                 c.compare()
                 splits = [(o, o + 1) for o in range(R)]
                 if path == "fused_acc":

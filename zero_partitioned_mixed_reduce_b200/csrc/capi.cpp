@@ -246,6 +246,7 @@ zb::RsNorm zb_rs_norm_note(zero_ctx_t* ctx, int64_t bucket, bool norm) {
     n.partials = ctx->rs_norm_partials + slot * static_cast<size_t>(ctx->grid_cap);
     n.done = ctx->rs_norm_done + slot;
     n.out = ctx->rs_norm + slot;
+    n.cap = static_cast<uint32_t>(ctx->grid_cap);
     n.mode = ctx->cfg.mode;
     n.divisor = ctx->grad_divisor;
     return n;

@@ -83,6 +83,7 @@ struct RsNorm {
     double* partials = nullptr;
     uint32_t* done = nullptr;
     double* out = nullptr;
+    uint32_t cap = 0;      // entries of `partials`
     int32_t mode = 0;
     double divisor = 1.0;
 };

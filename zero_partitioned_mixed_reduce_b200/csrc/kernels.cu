@@ -41,7 +41,7 @@ namespace zb {
 // Sites: 1 fused vector, 2 fused accumulator, 3 staged tile issue, 4 staged
 // tile store, 5 two-pass vector, 6 accumulator norm, 7 replica norm,
 // 8 reduce-scatter vector, 9 reduce-scatter element, 10 gather vector,
-// 11 gather element.
+// 11 gather element, 12 reduce-scatter norm partial.
 // ---------------------------------------------------------------------------
 #ifdef ZERO_DEBUG_BOUNDS
 __device__ unsigned long long g_bounds_count = 0;
@@ -717,7 +717,7 @@ __device__ void rs_norm_finish(const RsNorm& n, double nrm) {
     __shared__ int last;
     const double bn = block_sum(nrm, red);
     if (threadIdx.x == 0) {
-        n.partials[blockIdx.x] = bn;
+        if (ZB_IN(blockIdx.x < n.cap, 12, blockIdx.x)) n.partials[blockIdx.x] = bn;
         __threadfence();
         last = (atomicAdd(n.done, 1u) == gridDim.x - 1);
     }
@@ -726,7 +726,7 @@ __device__ void rs_norm_finish(const RsNorm& n, double nrm) {
     __threadfence();
     double x = 0.0;
     for (unsigned i = threadIdx.x; i < gridDim.x; i += kThreads)
-        x += *reinterpret_cast<volatile double*>(&n.partials[i]);
+        if (ZB_IN(i < n.cap, 12, i)) x += *reinterpret_cast<volatile double*>(&n.partials[i]);
     const double total = block_sum(x, red);
     if (threadIdx.x == 0) {
         *n.out = total;
