@@ -65,6 +65,10 @@ def lib():
         L.oracle_step_ex.restype = C.c_int32
         L.oracle_step_ex.argtypes = [C.c_int64, C.c_int32, C.c_int32, C.c_int32, P, P, P, P, P,
                                      C.POINTER(AdamW), C.POINTER(StepOpts), C.POINTER(FSM)]
+        L.oracle_step_ex_sample.restype = C.c_int32
+        L.oracle_step_ex_sample.argtypes = [C.c_int64, C.c_int32, C.c_int32, C.c_int32, P, P, P, P, P,
+                                            C.POINTER(AdamW), C.POINTER(StepOpts), C.POINTER(FSM),
+                                            C.c_double]
         L.oracle_model_state_bytes.restype = C.c_double
         L.oracle_model_state_bytes.argtypes = [C.c_int32, C.c_double, C.c_double]
         L.oracle_fp32_weight_bytes.restype = C.c_double
@@ -187,6 +191,21 @@ def step_ex(state: State, micro_grads: np.ndarray, hp: AdamW, fsm: FSM, grad_div
                               C.byref(opts), C.byref(fsm))
     if rc < 0:
         raise ValueError("oracle_step_ex rejected its arguments")
+    return bool(rc)
+
+
+def step_ex_sample(state: State, micro_grads: np.ndarray, hp: AdamW, fsm: FSM, grad_divisor,
+                   max_grad_norm, norm_sq_all) -> bool:
+    """step_ex on a sample of a model's elements, clipping with the whole
+    model's squared norm norm_sq_all. Returns skipped."""
+    g = np.ascontiguousarray(micro_grads, dtype=np.uint16)
+    n_micro, R, P = g.shape
+    opts = StepOpts(grad_divisor, max_grad_norm)
+    rc = lib().oracle_step_ex_sample(P, R, state.dtype, n_micro, _ptr(g), _ptr(state.master),
+                                     _ptr(state.m), _ptr(state.v), _ptr(state.param), C.byref(hp),
+                                     C.byref(opts), C.byref(fsm), float(norm_sq_all))
+    if rc < 0:
+        raise ValueError("oracle_step_ex_sample rejected its arguments")
     return bool(rc)
 
 

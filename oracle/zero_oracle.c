@@ -360,9 +360,13 @@ int32_t oracle_step(int64_t P, int32_t R, int32_t dtype, const uint16_t* grads,
 /*    clipping.                                                             */
 /* ======================================================================= */
 
-int32_t oracle_step_ex(int64_t P, int32_t R, int32_t dtype, int32_t n_micro, const uint16_t* grads,
-                       float* master, float* m, float* v, uint16_t* param,
-                       const oracle_adamw* hp, const oracle_step_opts* opts, oracle_fsm* st) {
+/* The step of every element given to it. The clipping norm is the one of
+ * these elements, unless norm_sq_all is given: then the elements are a
+ * sample of a larger model and *norm_sq_all is that model's norm (the only
+ * quantity of the step that couples elements besides the overflow flag). */
+static int32_t step_ex_impl(int64_t P, int32_t R, int32_t dtype, int32_t n_micro, const uint16_t* grads,
+                            float* master, float* m, float* v, uint16_t* param, const oracle_adamw* hp,
+                            const oracle_step_opts* opts, oracle_fsm* st, const double* norm_sq_all) {
     if (n_micro < 1 || opts->grad_divisor < 1.0) return -2;
     float* acc = (float*)malloc(sizeof(float) * (size_t)(P > 0 ? P : 1));
     float* part = (float*)malloc(sizeof(float) * (size_t)(P > 0 ? P : 1));
@@ -389,6 +393,7 @@ int32_t oracle_step_ex(int64_t P, int32_t R, int32_t dtype, int32_t n_micro, con
         float g = acc[e] * c.inv;
         nrm += (double)g * (double)g;
     }
+    if (norm_sq_all) nrm = *norm_sq_all;
     float coef = 1.0f;
     if (opts->max_grad_norm > 0.0) {
         double cd = opts->max_grad_norm / (sqrt(nrm) + 1e-6);
@@ -416,6 +421,19 @@ int32_t oracle_step_ex(int64_t P, int32_t R, int32_t dtype, int32_t n_micro, con
     free(acc);
     free(part);
     return skip;
+}
+
+int32_t oracle_step_ex(int64_t P, int32_t R, int32_t dtype, int32_t n_micro, const uint16_t* grads,
+                       float* master, float* m, float* v, uint16_t* param,
+                       const oracle_adamw* hp, const oracle_step_opts* opts, oracle_fsm* st) {
+    return step_ex_impl(P, R, dtype, n_micro, grads, master, m, v, param, hp, opts, st, NULL);
+}
+
+int32_t oracle_step_ex_sample(int64_t P, int32_t R, int32_t dtype, int32_t n_micro, const uint16_t* grads,
+                              float* master, float* m, float* v, uint16_t* param,
+                              const oracle_adamw* hp, const oracle_step_opts* opts, oracle_fsm* st,
+                              double norm_sq_all) {
+    return step_ex_impl(P, R, dtype, n_micro, grads, master, m, v, param, hp, opts, st, &norm_sq_all);
 }
 
 /* ======================================================================= */

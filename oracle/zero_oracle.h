@@ -124,6 +124,17 @@ int32_t oracle_step_ex(int64_t P, int32_t R, int32_t dtype, int32_t n_micro, con
                        float* master, float* m, float* v, uint16_t* param,
                        const oracle_adamw* hp, const oracle_step_opts* opts, oracle_fsm* st);
 
+/* oracle_step_ex on a sample of a model's elements: every argument as for
+ * oracle_step_ex, except that the clipping coefficient comes from
+ * norm_sq_all, the whole model's squared norm (computed elsewhere), which is
+ * also what grad_norm_sq records. The overflow flag covers the sample only,
+ * so the sample must contain any non-finite element of the model. With
+ * norm_sq_all equal to the sample's own norm it is oracle_step_ex. */
+int32_t oracle_step_ex_sample(int64_t P, int32_t R, int32_t dtype, int32_t n_micro, const uint16_t* grads,
+                              float* master, float* m, float* v, uint16_t* param,
+                              const oracle_adamw* hp, const oracle_step_opts* opts, oracle_fsm* st,
+                              double norm_sq_all);
+
 /* ---- per-rank model-state memory (bytes) --------------------------------
  * stage 0 = plain data parallel, 1/2/3 = ZeRO stages; psi parameters, N
  * data-parallel ranks; 2 + 2 + 12 bytes per parameter. */

@@ -55,9 +55,13 @@ def read_flat(shards, S, padded_idx):
 
 
 class Workload:
-    def __init__(self, name, path, sample=1 << 16):
+    """path: "pingpong", "inplace", "twopass", or "twopass_clip" (two-pass,
+    global-norm clipping at `clip` with the norm taken by the reduce-scatters;
+    the oracle steps the sample with the whole model's norm)."""
+
+    def __init__(self, name, path, sample=1 << 16, clip=0.0):
         self.wl = wl = synth.workload(name)
-        self.path = path
+        self.path, self.clip = path, clip
         self.R, self.dtype = wl["R"], wl["dtype"]
         self.lay = O.Layout(wl["numels"], wl["R"], 8, wl["bucket_elems"], wl["layer_ids"])
         self.plan = Z.Plan(wl["numels"], wl["layer_ids"], wl["R"], wl["dtype"], 8,
@@ -65,7 +69,7 @@ class Workload:
         layout_matches(self.plan, self.lay)
         self.S, self.T = self.plan.S, self.plan.T
         sets = 2 if path == "pingpong" else 1
-        self.state = Z.ShardedState(self.plan, sets=sets, with_acc=(path == "twopass"))
+        self.state = Z.ShardedState(self.plan, sets=sets, with_acc=path.startswith("twopass"))
         starts = np.concatenate([[0], np.cumsum(wl["numels"])[:-1]])
         # sample of unpadded indices: random, every tensor's first and last
         # element, the neighbours of every shard boundary, the injection point
@@ -148,10 +152,18 @@ class Workload:
             for b in range(len(self.plan.buckets)):
                 Z.zero_reduce_scatter_bucket(self.ctx, b, self.grads, self.state.acc)
             Z.zero_step(self.ctx, hp, self.state.handle, None)
+        elif self.path == "twopass_clip":
+            for b in range(len(self.plan.buckets)):
+                Z.zero_reduce_scatter_bucket_ex(self.ctx, b, self.grads, self.state.acc, Z.ZERO_RS_NORM)
+            Z.zero_step_ex(self.ctx, hp, self.state.handle, None, 1.0, self.clip,
+                           flags=Z.ZERO_STEP_NORM_FROM_RS)
         else:
             Z.zero_step(self.ctx, hp, self.state.handle, self.grads)
         ref_norm = self.reference_norm(scale_before)
-        O.step(self.ostate, sample_g, self.ohp, self.ofsm)
+        if self.path == "twopass_clip":
+            O.step_ex_sample(self.ostate, sample_g[None], self.ohp, self.ofsm, 1.0, self.clip, ref_norm)
+        else:
+            O.step(self.ostate, sample_g, self.ohp, self.ofsm)
         return ref_norm
 
     def check(self, ref_norm):
@@ -176,8 +188,8 @@ class Workload:
         return f
 
 
-def run(name, path, gather=False, steps=None):
-    w = Workload(name, path)
+def run(name, path, gather=False, steps=None, clip=0.0):
+    w = Workload(name, path, clip=clip)
     try:
         for _ in range(steps or w.wl["steps"]):
             ref = w.step()
@@ -227,6 +239,14 @@ def test_gpt2s_dynamic_with_injected_inf():
 
 def test_gpt2s_two_pass_buckets():
     run("gpt2s", "twopass", steps=4)
+
+
+def test_gpt2s_two_pass_clipped_with_the_norm_from_the_reduce_scatters():
+    # the unscaled gradient's norm is about 0.4 here: a 0.1 threshold clips
+    # every applied step; step 3's injected inf is still skipped
+    fsm = run("gpt2s", "twopass_clip", steps=4, clip=0.1)
+    assert fsm.t == 3 and fsm.scale == 2.0 ** 15
+    assert fsm.grad_norm_sq > 0.1 ** 2
 
 
 def test_d1p3b_with_layer_gathers():

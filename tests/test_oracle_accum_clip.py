@@ -133,3 +133,49 @@ def test_overflow_in_any_micro_batch_skips():
     assert O.step_ex(st, g, HP, fsm, 3.0, 1.0)
     assert fsm.scale == 32.0 and fsm.t == 0
     assert np.array_equal(st.master, before.master)
+
+
+@pytest.mark.parametrize("max_norm", [0.0, 0.05, 1e9])
+@pytest.mark.parametrize("dtype", [O.BF16, O.FP16])
+def test_step_on_a_sample_with_the_whole_norm_equals_the_whole_step(max_norm, dtype):
+    # given the whole model's norm, each element's step depends on its own
+    # inputs only: a sample stepped with that norm has the whole step's bytes
+    rng = np.random.default_rng(40 + dtype)
+    n, R, P = 2, 3, 5000
+    x = rng.normal(0, 0.02, P).astype(np.float32)
+    whole = O.State(x, dtype)
+    fw = O.make_fsm(O.SCALE_STATIC, 4.0)
+    idx = np.sort(rng.choice(P, 300, replace=False))
+    part = O.State(x[idx].copy(), dtype)
+    fp = O.make_fsm(O.SCALE_STATIC, 4.0)
+    for _ in range(3):
+        g = O.float_to_half(rng.normal(0, 1e-2, (n, R, P)).astype(np.float32) * 4.0, dtype)
+        O.step_ex(whole, g, HP, fw, 2.0, max_norm)
+        O.step_ex_sample(part, g[:, :, idx], HP, fp, 2.0, max_norm, fw.grad_norm_sq)
+        for a in ("master", "m", "v"):
+            assert np.array_equal(getattr(whole, a)[idx].view(np.uint32), getattr(part, a).view(np.uint32)), a
+        assert np.array_equal(whole.param[idx], part.param)
+        assert fp.grad_norm_sq == fw.grad_norm_sq and fp.t == fw.t
+    # the sample's own norm instead: clipping with it changes the result
+    if max_norm == 0.05:
+        own = O.State(x[idx].copy(), dtype)
+        fo = O.make_fsm(O.SCALE_STATIC, 4.0)
+        g = O.float_to_half(rng.normal(0, 1e-2, (n, R, P)).astype(np.float32) * 4.0, dtype)
+        O.step_ex(own, g[:, :, idx], HP, fo, 2.0, max_norm)
+        alt = O.State(x[idx].copy(), dtype)
+        fa = O.make_fsm(O.SCALE_STATIC, 4.0)
+        O.step_ex_sample(alt, g[:, :, idx], HP, fa, 2.0, max_norm, fo.grad_norm_sq * 16.0)
+        assert not np.array_equal(own.master, alt.master)
+
+
+def test_step_on_a_sample_with_its_own_norm_is_step_ex():
+    rng = np.random.default_rng(9)
+    R, P = 2, 777
+    x = rng.normal(0, 0.02, P).astype(np.float32)
+    g = O.float_to_half(rng.normal(0, 1e-2, (1, R, P)).astype(np.float32), O.FP16)
+    a, b = O.State(x, O.FP16), O.State(x, O.FP16)
+    fa, fb = O.make_fsm(O.SCALE_DYNAMIC, 2.0), O.make_fsm(O.SCALE_DYNAMIC, 2.0)
+    O.step_ex(a, g, HP, fa, 1.0, 0.01)
+    O.step_ex_sample(b, g, HP, fb, 1.0, 0.01, fa.grad_norm_sq)
+    for k in ("master", "m", "v", "param"):
+        assert np.array_equal(getattr(a, k), getattr(b, k))
