@@ -11,6 +11,12 @@ if ROOT not in sys.path:
 def pytest_configure(config):
     config.addinivalue_line("markers", "gpu: needs a CUDA GPU (B200, sm_100a)")
     config.addinivalue_line("markers", "slow: long-running; opt-in via ZERO_SLOW=1")
+    # a fresh checkout has no built library yet: build it (nvcc cross-compiles
+    # for sm_100a without a GPU) before any test module imports the package
+    lib = os.path.join(ROOT, "zero_partitioned_mixed_reduce_b200", "libzero_b200.so")
+    if not os.path.exists(lib) and not os.environ.get("ZERO_B200_LIB"):
+        import __graft_entry__
+        __graft_entry__.build()
 
 
 def pytest_collection_modifyitems(config, items):
