@@ -31,7 +31,7 @@ STATUS_NAMES = {0: "ZERO_OK", 1: "ZERO_ERR_INVALID_ARG", 2: "ZERO_ERR_ALIGN", 3:
 
 if not os.path.exists(LIB_PATH):
     raise ImportError(
-        f"{LIB_PATH} is missing: build it with `python -m zero_partitioned_mixed_reduce_b200.build` "
+        f"{LIB_PATH} is missing: build it with `python zero_partitioned_mixed_reduce_b200/build.py` "
         "(nvcc, sm_100a). There is no CPU fallback.")
 
 
