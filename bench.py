@@ -594,50 +594,126 @@ def e2e(b, args, stream, world):
 
 # ---- the CPU oracle as a baseline ----------------------------------------------
 
-def oracle_sample(name, target_s=10.0, max_elems=1 << 26):
-    """Time the oracle's step on a prefix sample of the workload, sized for
-    about target_s seconds. Returns (params/s, sample elements, seconds)."""
+def oracle_inputs(name, n):
+    """The oracle's state, replicas, hyper-parameters and loss-scale state
+    for the first n params of the workload."""
     import oracle as O
     from zero_partitioned_mixed_reduce_b200 import synth
     wl = synth.workload(name)
     R, dtype = wl["R"], wl["dtype"]
     scale = wl["init_scale"] if wl["mode"] != synth.NONE else 1.0
-
-    def inputs(n):
-        numels, left = [], n
-        for k in wl["numels"]:
-            if left <= 0:
-                break
-            numels.append(min(k, left))
-            left -= numels[-1]
-        x = torch.cat([synth.tensor_master(c, wl["index"], k, "cpu") for k, c in enumerate(numels)])
-        g = np.stack([torch.cat([synth.tensor_grads(c, wl["dist"], wl["sigma"], scale, dtype,
-                                                    wl["index"], 1, r, k, "cpu")
-                                 for k, c in enumerate(numels)]).view(torch.int16).numpy()
-                      .view(np.uint16) for r in range(R)])
-        return O.State(x.numpy(), dtype), g
-
+    numels, left = [], n
+    for k in wl["numels"]:
+        if left <= 0:
+            break
+        numels.append(min(k, left))
+        left -= numels[-1]
+    x = torch.cat([synth.tensor_master(c, wl["index"], k, "cpu") for k, c in enumerate(numels)])
+    g = np.stack([torch.cat([synth.tensor_grads(c, wl["dist"], wl["sigma"], scale, dtype,
+                                                wl["index"], 1, r, k, "cpu")
+                             for k, c in enumerate(numels)]).view(torch.int16).numpy()
+                  .view(np.uint16) for r in range(R)])
     hp = O.AdamW(**{k: wl["hp"][k] for k in ("lr", "beta1", "beta2", "eps", "weight_decay")})
-    n = 1 << 18
-    st, g = inputs(n)
     fsm = O.make_fsm(wl["mode"], scale=scale, interval=wl["interval"])
+    return O.State(x.numpy(), dtype), g, hp, fsm
+
+
+def oracle_sample(name, target_s=10.0, max_elems=1 << 26):
+    """Time the oracle's step on a prefix sample of the workload, sized for
+    about target_s seconds. Returns (params/s, sample elements, seconds)."""
+    import oracle as O
+    n = 1 << 18
+    st, g, hp, fsm = oracle_inputs(name, n)
     t = time.perf_counter()
     O.step(st, g, hp, fsm)
     rate = n / (time.perf_counter() - t)
     n = int(min(max_elems, max(n, rate * target_s)))
-    st, g = inputs(n)
-    fsm = O.make_fsm(wl["mode"], scale=scale, interval=wl["interval"])
+    st, g, hp, fsm = oracle_inputs(name, n)
     t = time.perf_counter()
     O.step(st, g, hp, fsm)
     dt = time.perf_counter() - t
     return n / dt, n, dt, (st, g, hp, fsm)
 
 
+def _oracle_crew_worker(name, n, barrier, conn):
+    """One single-threaded oracle process of OracleCrew: builds its sample,
+    then on each request runs k steps between a common barrier and reports
+    its start and end time (CLOCK_MONOTONIC, comparable across processes)."""
+    import oracle as O
+    torch.set_num_threads(1)
+    st, g, hp, fsm = oracle_inputs(name, n)
+    conn.send("ready")
+    while True:
+        k = conn.recv()
+        if k is None:
+            break
+        barrier.wait()
+        t0 = time.perf_counter()
+        for _ in range(k):
+            O.step(st, g, hp, fsm)
+        conn.send((t0, time.perf_counter()))
+
+
+class OracleCrew:
+    """The oracle, as it stands, on every host core: one spawned process per
+    hardware thread, each stepping its own copy of the same prefix sample.
+    Throughput = processes x sample x steps / (last end - first start)."""
+
+    def __init__(self, name, n, procs=None):
+        import multiprocessing as mp
+        ctx = mp.get_context("spawn")  # never fork a process that holds CUDA
+        self.n, self.procs = n, procs or (os.cpu_count() or 1)
+        self.barrier = ctx.Barrier(self.procs)
+        self.conns, self.ps = [], []
+        old = {k: os.environ.get(k) for k in ("OMP_NUM_THREADS", "MKL_NUM_THREADS")}
+        os.environ.update(OMP_NUM_THREADS="1", MKL_NUM_THREADS="1")
+        try:
+            for _ in range(self.procs):
+                a, b = ctx.Pipe()
+                p = ctx.Process(target=_oracle_crew_worker, args=(name, n, self.barrier, b), daemon=True)
+                p.start()
+                self.conns.append(a)
+                self.ps.append(p)
+        finally:
+            for k, v in old.items():
+                if v is None:
+                    os.environ.pop(k, None)
+                else:
+                    os.environ[k] = v
+        for c in self.conns:
+            assert c.recv() == "ready"
+
+    def run(self, k):
+        """k steps in every process; returns (params/s, seconds)."""
+        for c in self.conns:
+            c.send(k)
+        spans = [c.recv() for c in self.conns]
+        sec = max(t1 for _, t1 in spans) - min(t0 for t0, _ in spans)
+        return self.procs * self.n * k / sec, sec
+
+    def close(self):
+        for c in self.conns:
+            c.send(None)
+        for p in self.ps:
+            p.join(timeout=30)
+
+
 def cpu_baseline(name):
-    rate, n, dt, _ = oracle_sample(name)
-    return {"value": rate, "unit": "params/s", "cores": 1, "kind": "oracle",
-            "sample": f"one step of the first {n} params of {name} (all R replicas), "
-                      f"{dt:.1f} s single-threaded"}
+    """The oracle on all host cores (one process per hardware thread), plus
+    its single-threaded rate."""
+    rate1, n1, dt1, _ = oracle_sample(name)
+    n = 1 << 22
+    crew = OracleCrew(name, n)
+    try:
+        crew.run(1)  # warm-up
+        rate, sec = crew.run(2)
+    finally:
+        crew.close()
+    return {"value": rate, "unit": "params/s", "cores": crew.procs, "kind": "oracle",
+            "sample": f"{crew.procs} single-threaded processes, each 2 steps of the first {n} params of "
+                      f"{name} (all R replicas), {sec:.1f} s",
+            "single_thread": {"value": rate1, "cores": 1,
+                              "sample": f"one step of the first {n1} params, {dt1:.1f} s"}}
 
 
 def run_overlap(args, world, rank, local):
@@ -1118,16 +1194,14 @@ def run_reference(args, world, rank):
     """The oracle on host cores: each step a bounded prefix sample."""
     if rank != 0:
         return
-    import oracle as O
-    rate, n, dt, (st, g, hp, fsm) = oracle_sample(args.workload, target_s=1.0,
-                                                  max_elems=1 << 22)
-    for _ in range(args.warmup):
-        O.step(st, g, hp, fsm)
-    t = time.perf_counter()
-    for _ in range(args.steps):
-        O.step(st, g, hp, fsm)
-    sec = time.perf_counter() - t
-    value = n * args.steps / sec
+    # every host core runs the oracle on its own copy of a 1M-param prefix
+    n = 1 << 20
+    crew = OracleCrew(args.workload, n)
+    try:
+        crew.run(args.warmup)
+        value, sec = crew.run(args.steps)
+    finally:
+        crew.close()
     from zero_partitioned_mixed_reduce_b200 import synth
     wl = synth.workload(args.workload)
     out = {
@@ -1136,9 +1210,10 @@ def run_reference(args, world, rank):
         "ms_per_step": sec * 1e3 / args.steps, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f32", "data": "synthetic",
         "config": {"workload": workload_label(args.workload, wl), "R": wl["R"],
-                   "P": sum(wl["numels"]), "sample_params_per_step": n},
-        "cpu_baseline": {"value": value, "unit": "params/s", "cores": 1, "kind": "oracle",
-                         "sample": f"each step the first {n} params of {args.workload}"},
+                   "P": sum(wl["numels"]), "sample_params_per_step": n * crew.procs},
+        "cpu_baseline": {"value": value, "unit": "params/s", "cores": crew.procs, "kind": "oracle",
+                         "sample": f"each step, in each of {crew.procs} single-threaded processes, "
+                                   f"the first {n} params of {args.workload}"},
         "e2e": {"value": value, "unit": "params/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }
