@@ -472,7 +472,10 @@ def run_ours(args, world, rank, local):
         kernel_name = "grad_norm+fused_step_kernel (clip)"
     elif b.accum > 1:
         kernel_name = f"reduce_scatter+fused_step_kernel (accum {b.accum}, last micro-batch fused)"
-    traffic = profiled_traffic(kernel_name, args.workload)
+    # the stored counters describe the full workload on the ping-pong fused
+    # path; any other configuration reports no traffic
+    same_config = args.first_tensors == 0 and b.path == "pingpong"
+    traffic = profiled_traffic(kernel_name, args.workload) if same_config else None
     clip_label = ("" if b.clip <= 0 else
                   "global-norm clip from the reduce-scatters' norm shares, " if b.rs_norm else
                   "global-norm clip pass, ")
