@@ -828,7 +828,8 @@ def run_rs_sweep(args, world, rank, local):
     """The bucketed reduce-scatter (one pass over every bucket of the plan)
     against bucket size, on the workload's tensors: for each size a plan is
     built (the flat layout does not depend on it), and the pass is timed
-    issued launch by launch and replayed from a CUDA graph. Reported as the
+    issued launch by launch, replayed from a CUDA graph, and with consecutive
+    buckets grouped into launches of about 25M elements. Reported as the
     kernel's algorithmic (2R + 4) bytes per padded element over the pass."""
     if not torch.cuda.is_available():
         print(json.dumps({"error": "no CUDA device"}))
@@ -871,7 +872,18 @@ def run_rs_sweep(args, world, rank, local):
             for b in range(nb):
                 Z.zero_reduce_scatter_bucket(ctx, b, grads, acc, s)
 
+        # consecutive buckets grouped into launches of about 25M elements
+        # (zero_reduce_scatter_buckets), as a caller reporting a layer at a
+        # time would issue them
+        group = max(1, (25 << 20) // size) if size > 0 else 1
+        runs = [(b, min(group, nb - b)) for b in range(0, nb, group)]
+
+        def grouped_pass(s=stream):
+            for first, count in runs:
+                Z.zero_reduce_scatter_buckets(ctx, first, count, grads, acc, 0, s)
+
         t_eager = timed(one_pass)
+        t_grouped = timed(grouped_pass)
         side = torch.cuda.Stream()
         side.wait_stream(stream)
         g = torch.cuda.CUDAGraph()
@@ -884,6 +896,8 @@ def run_rs_sweep(args, world, rank, local):
         Z.zero_ctx_destroy(ctx)
         rows.append({"bucket_elems": size if size > 0 else "whole model", "buckets": nb,
                      "ms_eager": t_eager, "ms_graph": t_graph,
+                     "grouped_launches": len(runs), "ms_grouped": t_grouped,
+                     "gbs_grouped": nbytes / (t_grouped * 1e-3) / 1e9,
                      "gbs_eager": nbytes / (t_eager * 1e-3) / 1e9,
                      "gbs_graph": nbytes / (t_graph * 1e-3) / 1e9,
                      "frac_graph": nbytes / (t_graph * 1e-3) / 1e9 / peak,

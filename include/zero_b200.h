@@ -297,6 +297,25 @@ zero_status zero_reduce_scatter_bucket_ex(zero_ctx_t* ctx, int64_t bucket, const
                                           float* const* acc, int32_t flags, void* stream);
 
 /*
+ * zero_reduce_scatter_buckets -- zero_reduce_scatter_bucket_ex over the
+ * consecutive buckets [first, first + count) in one launch. Consecutive
+ * buckets are adjacent in the flat layout (bucket b + 1 ends where bucket b
+ * begins), so this is one reduce-scatter of the flat range from the start of
+ * bucket first + count - 1 to the end of bucket first: the same bytes as
+ * count separate calls, with one launch instead of count. For small buckets
+ * the launches, not the bytes, bound the separate calls. first = -1 with
+ * count = 1 is the whole range. With ZERO_RS_NORM the group's norm share
+ * lands in the slot of bucket `first` and the other buckets' slots hold 0,
+ * so the step's sum over every slot is the same norm.
+ * Defines: [legal] "Bandwidth Optimization" (fusing small parameter groups
+ * into larger transfers) applied to launches.
+ * Errors: as zero_reduce_scatter_bucket_ex; ZERO_ERR_RANGE unless
+ * 0 <= first, 1 <= count and first + count <= n_buckets.
+ */
+zero_status zero_reduce_scatter_buckets(zero_ctx_t* ctx, int64_t first, int64_t count, const void* const* grads,
+                                        float* const* acc, int32_t flags, void* stream);
+
+/*
  * zero_ctx_set_grad_divisor -- the gradient divisor d (>= 1, finite) that
  * later ZERO_RS_NORM reduce-scatters unscale by; the step checks that its
  * own grad_divisor equals the one each slot was taken with. Host state
@@ -626,7 +645,10 @@ zero_status zero_sched_set_comm_sms(zero_ctx_t* ctx, int32_t sms);
  * bucket whose tensors have then all been reported is reduce-scattered at
  * once (as zero_reduce_scatter_bucket_ex with `flags`) on the communication
  * stream, ordered after that work by an event, so the reduction of early
- * buckets overlaps the caller's next work on `stream`.
+ * buckets overlaps the caller's next work on `stream`. Buckets that one call
+ * completes and that are consecutive go in one launch, as
+ * zero_reduce_scatter_buckets (a caller reporting a whole layer at a time
+ * pays one launch per layer, however small the buckets).
  * Defines: [legal] "Communication Overlap" (a layer's gradient reduction
  * starts as soon as its gradients are computed, hidden behind the backward
  * pass) and [genomic] "Reduce-Scatter Overlap".

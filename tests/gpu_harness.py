@@ -142,12 +142,14 @@ class Case:
         return skipped
 
     def step_ex(self, n_micro, grad_divisor=1.0, max_grad_norm=0.0, inject=None, rs_norm=False,
-                whole=False):
+                whole=False, groups=None):
         """Two-pass step over n_micro accumulated micro-batches, optionally
         clipped; inject: (micro, rank, element, bits) tuples. rs_norm: the
         last micro-batch's reduce-scatters record the clipping norm
         (ZERO_RS_NORM) and the step sums their shares; whole: one
-        reduce-scatter over the whole range per micro-batch."""
+        reduce-scatter over the whole range per micro-batch; groups: (first,
+        count) runs of consecutive buckets, one zero_reduce_scatter_buckets
+        call each."""
         assert self.path.startswith("twopass")
         norm_flag = Z.ZERO_RS_NORM if rs_norm else 0
         if rs_norm:
@@ -168,6 +170,10 @@ class Case:
                 gp[self.idx] = g[mu, r]
                 self.grads[r].view(torch.int16).copy_(torch.from_numpy(gp.view(np.int16)))
             flags = (Z.ZERO_RS_ACCUMULATE if mu else 0) | (norm_flag if mu == n_micro - 1 else 0)
+            if groups is not None:
+                for first, count in groups:
+                    Z.zero_reduce_scatter_buckets(self.ctx, first, count, self.grads, self.acc, flags)
+                continue
             for b in ([-1] if whole else range(len(self.plan.buckets))):
                 Z.zero_reduce_scatter_bucket_ex(self.ctx, b, self.grads, self.acc, flags)
         Z.zero_step_ex(self.ctx, self.hp, self.handle, None, grad_divisor, max_grad_norm,
@@ -197,12 +203,15 @@ class Case:
         self.g.check()
         return skipped
 
-    def step_overlap(self, n_micro=1, grad_divisor=1.0, max_grad_norm=0.0, busy=None, rs_norm=False):
+    def step_overlap(self, n_micro=1, grad_divisor=1.0, max_grad_norm=0.0, busy=None, rs_norm=False,
+                     per_call=1):
         """Two-pass step whose reduce-scatters are issued by the overlap
         scheduler: each tensor's gradients are written on the caller's stream
         (after `busy` work, standing in for backward) in reverse tensor order,
         then reported ready; join; step. rs_norm: the last micro-batch's
-        reduce-scatters record the clipping norm."""
+        reduce-scatters record the clipping norm. per_call: tensors reported
+        per zero_grads_ready call (a call that completes consecutive buckets
+        reduces them in one launch)."""
         assert self.path.startswith("twopass")
         if rs_norm:
             Z.zero_ctx_set_grad_divisor(self.ctx, grad_divisor)
@@ -219,16 +228,19 @@ class Case:
         torch.cuda.synchronize()
         for r in range(self.R):
             self.grads[r].zero_()
+        nt = len(self.lay.numels)
         for mu in range(n_micro):
-            for k in reversed(range(len(self.lay.numels))):
+            for hi in range(nt, 0, -per_call):
+                lo = max(0, hi - per_call)
                 if busy is not None:
                     busy()
-                off, n, st = int(self.lay.offsets[k]), int(self.lay.numels[k]), int(starts[k])
-                for r in range(self.R):
-                    self.grads[r].view(torch.int16)[off:off + n].copy_(dev[mu][r, st:st + n])
+                for k in range(lo, hi):
+                    off, n, st = int(self.lay.offsets[k]), int(self.lay.numels[k]), int(starts[k])
+                    for r in range(self.R):
+                        self.grads[r].view(torch.int16)[off:off + n].copy_(dev[mu][r, st:st + n])
                 flags = (Z.ZERO_RS_ACCUMULATE if mu else 0) | \
                     (Z.ZERO_RS_NORM if rs_norm and mu == n_micro - 1 else 0)
-                Z.zero_grads_ready(self.ctx, k, 1, self.grads, self.acc, flags,
+                Z.zero_grads_ready(self.ctx, lo, hi - lo, self.grads, self.acc, flags,
                                    torch.cuda.current_stream())
             Z.zero_grads_join(self.ctx, torch.cuda.current_stream())
         Z.zero_step_ex(self.ctx, self.hp, self.handle, None, grad_divisor, max_grad_norm,

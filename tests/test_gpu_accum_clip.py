@@ -245,3 +245,36 @@ def test_norm_from_reduce_scatter_refusals():
         assert e.value.status == Z.ZERO_ERR_STATE
     finally:
         c.close()
+
+
+@pytest.mark.parametrize("R,dtype", [(3, O.FP16), (8, O.BF16)])
+@pytest.mark.parametrize("rs_norm", [False, True])
+def test_grouped_reduce_scatters_match_oracle(R, dtype, rs_norm):
+    # consecutive buckets in one launch each (zero_reduce_scatter_buckets):
+    # the oracle's bytes, with accumulation, clipping and the norm shares
+    mode = O.SCALE_DYNAMIC if dtype == O.FP16 else O.SCALE_NONE
+    c = Case([70_001, 13, 4096, 7, 999, 20_000, 3, 5000], R, dtype, 8 if R != 3 else 1, mode,
+             init_scale=256.0, interval=2, path="twopass_pp", bucket_elems=3000)
+    nb = len(c.plan.buckets)
+    assert nb >= 5
+    try:
+        for groups in ([(0, nb)], [(0, 2), (2, 1), (3, nb - 3)], [(b, 1) for b in range(nb)]):
+            c.step_ex(2, 2.0, 1e-3, rs_norm=rs_norm, groups=groups)
+            c.compare()
+    finally:
+        c.close()
+
+
+def test_grouped_reduce_scatter_range_errors():
+    c = Case([3000, 17, 2048], 2, O.BF16, 8, O.SCALE_NONE, path="twopass", bucket_elems=1000)
+    nb = len(c.plan.buckets)
+    try:
+        for first, count in ((0, 0), (-2, 1), (-1, 2), (1, nb), (nb, 1)):
+            with pytest.raises(Z.ZeroError) as e:
+                Z.zero_reduce_scatter_buckets(c.ctx, first, count, c.grads, c.acc)
+            assert e.value.status == Z.ZERO_ERR_RANGE, (first, count)
+        with pytest.raises(Z.ZeroError) as e:
+            Z.zero_reduce_scatter_buckets(c.ctx, 0, 1, c.grads, c.acc, 8)
+        assert e.value.status == Z.ZERO_ERR_INVALID_ARG
+    finally:
+        c.close()

@@ -68,6 +68,24 @@ def test_overlapped_reduce_scatter_with_norm_matches_oracle(R, dtype, n_micro, c
         c.close()
 
 
+@pytest.mark.parametrize("per_call", [3, 8])
+@pytest.mark.parametrize("rs_norm", [False, True])
+def test_reports_of_several_tensors_coalesce_and_match_oracle(per_call, rs_norm):
+    # a call that completes several consecutive buckets reduces them in one
+    # launch; the result is the oracle's either way
+    numels = [70_001, 13, 4096, 7, 999, 30_000, 5, 12_000, 800]
+    c = Case(numels, 8, O.FP16, 8, O.SCALE_DYNAMIC, init_scale=256.0, interval=3, path="twopass",
+             bucket_elems=5_000)
+    busy = make_busy()
+    try:
+        for n_micro in (1, 2):
+            c.step_overlap(n_micro, float(n_micro), 1e-3 if rs_norm else 0.0, busy, rs_norm=rs_norm,
+                           per_call=per_call)
+            c.compare()
+    finally:
+        c.close()
+
+
 def test_grads_join_refuses_missing_and_repeated_reports():
     c = Case([100, 200, 300], 2, O.BF16, 8, O.SCALE_NONE, path="twopass", bucket_elems=250)
     try:

@@ -117,6 +117,7 @@ _sig("zero_test_drop_tile", _S, [_P, C.c_int64])
 _sig("zero_reduce_scatter_bucket", _S, [_P, C.c_int64, _PP, _PP, _P])
 _sig("zero_step", _S, [_P, C.POINTER(zero_adamw), C.POINTER(zero_state), _PP, _P])
 _sig("zero_reduce_scatter_bucket_ex", _S, [_P, C.c_int64, _PP, _PP, C.c_int32, _P])
+_sig("zero_reduce_scatter_buckets", _S, [_P, C.c_int64, C.c_int64, _PP, _PP, C.c_int32, _P])
 _sig("zero_step_ex", _S, [_P, C.POINTER(zero_adamw), C.POINTER(zero_state), _PP,
                           C.POINTER(zero_step_opts), _P])
 _sig("zero_gather_layer", _S, [_P, C.c_int64, C.POINTER(zero_state), _P, _P])
@@ -286,6 +287,13 @@ def zero_reduce_scatter_bucket(ctx, bucket, grads, acc, stream=None):
     g, ga = _ptr_array(grads)
     a, aa = _ptr_array(acc)
     _check(_lib.zero_reduce_scatter_bucket(ctx, bucket, g, a, _stream(stream)))
+
+
+def zero_reduce_scatter_buckets(ctx, first, count, grads, acc, flags=0, stream=None):
+    """Buckets first .. first+count-1 (a contiguous flat range) in one launch."""
+    g, ga = _ptr_array(grads)
+    a, aa = _ptr_array(acc)
+    _check(_lib.zero_reduce_scatter_buckets(ctx, first, count, g, a, flags, _stream(stream)))
 
 
 def zero_ctx_set_grad_divisor(ctx, grad_divisor):

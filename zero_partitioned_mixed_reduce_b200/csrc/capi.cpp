@@ -230,19 +230,23 @@ extern "C" zero_status zero_ctx_set_grad_divisor(zero_ctx_t* ctx, double grad_di
     return ZERO_OK;
 }
 
-zb::RsNorm zb_rs_norm_note(zero_ctx_t* ctx, int64_t bucket, bool norm) {
+zb::RsNorm zb_rs_norm_note(zero_ctx_t* ctx, int64_t first, int64_t count, bool norm) {
     const size_t whole = ctx->bucket_lo.size();
-    const size_t slot = bucket < 0 ? whole : static_cast<size_t>(bucket);
-    if (bucket < 0) {
+    const size_t slot = first < 0 ? whole : static_cast<size_t>(first);
+    if (first < 0) {
         // the whole range is rewritten: every per-bucket share is stale
         std::fill(ctx->rs_norm_valid.begin(), ctx->rs_norm_valid.end(), 0);
+        ctx->rs_norm_valid[whole] = norm ? 1 : 0;
+        ctx->rs_norm_div[whole] = ctx->grad_divisor;
     } else {
         ctx->rs_norm_valid[whole] = 0;
+        for (int64_t b = first; b < first + count; ++b) {
+            ctx->rs_norm_valid[static_cast<size_t>(b)] = norm ? 1 : 0;
+            ctx->rs_norm_div[static_cast<size_t>(b)] = ctx->grad_divisor;
+        }
     }
-    ctx->rs_norm_valid[slot] = norm ? 1 : 0;
     zb::RsNorm n;
     if (!norm) return n;
-    ctx->rs_norm_div[slot] = ctx->grad_divisor;
     n.partials = ctx->rs_norm_partials + slot * static_cast<size_t>(ctx->grid_cap);
     n.done = ctx->rs_norm_done + slot;
     n.out = ctx->rs_norm + slot;
@@ -250,6 +254,31 @@ zb::RsNorm zb_rs_norm_note(zero_ctx_t* ctx, int64_t bucket, bool norm) {
     n.mode = ctx->cfg.mode;
     n.divisor = ctx->grad_divisor;
     return n;
+}
+
+cudaError_t zb_rs_launch(zero_ctx_t* ctx, int64_t first, int64_t count, const zb::RankPtrs& p,
+                         cudaStream_t s, int32_t flags, int max_sms) {
+    int64_t lo = 0, hi = ctx->T;
+    if (first >= 0) {
+        lo = ctx->bucket_lo[static_cast<size_t>(first + count - 1)];
+        hi = ctx->bucket_hi[static_cast<size_t>(first)];
+    }
+    const bool with_norm = (flags & ZERO_RS_NORM) != 0;
+    const zb::RsNorm norm = zb_rs_norm_note(ctx, first, count, with_norm);
+    cudaError_t e = cudaSuccess;
+    // a group's share lands in its first bucket's slot; the others hold 0
+    if (with_norm && first >= 0 && count > 1)
+        e = cudaMemsetAsync(ctx->rs_norm + first + 1, 0, sizeof(double) * static_cast<size_t>(count - 1), s);
+    if (e == cudaSuccess)
+        e = zb::launch_reduce_scatter(ctx->R, ctx->dtype, ctx->S, lo, hi, ctx->st, p, s,
+                                      (flags & ZERO_RS_ACCUMULATE) != 0, max_sms,
+                                      with_norm ? &norm : nullptr);
+    if (e != cudaSuccess) {
+        const size_t whole = ctx->bucket_lo.size();
+        if (first < 0) ctx->rs_norm_valid[whole] = 0;
+        for (int64_t b = first; first >= 0 && b < first + count; ++b) ctx->rs_norm_valid[static_cast<size_t>(b)] = 0;
+    }
+    return e;
 }
 
 extern "C" zero_status zero_ctx_destroy(zero_ctx_t* ctx) {
@@ -299,22 +328,25 @@ extern "C" zero_status zero_reduce_scatter_bucket(zero_ctx_t* ctx, int64_t bucke
 extern "C" zero_status zero_reduce_scatter_bucket_ex(zero_ctx_t* ctx, int64_t bucket,
                                                      const void* const* grads, float* const* acc,
                                                      int32_t flags, void* stream) {
+    if (bucket == -1) return zero_reduce_scatter_buckets(ctx, -1, 1, grads, acc, flags, stream);
+    if (ctx && (bucket < 0 || bucket >= static_cast<int64_t>(ctx->bucket_lo.size())))
+        return zb_fail(ZERO_ERR_RANGE, "zero_reduce_scatter_bucket: bucket index out of range");
+    return zero_reduce_scatter_buckets(ctx, bucket, 1, grads, acc, flags, stream);
+}
+
+extern "C" zero_status zero_reduce_scatter_buckets(zero_ctx_t* ctx, int64_t first, int64_t count,
+                                                   const void* const* grads, float* const* acc,
+                                                   int32_t flags, void* stream) {
     const char* where = "zero_reduce_scatter_bucket";
     if (flags & ~(ZERO_RS_ACCUMULATE | ZERO_RS_NORM))
         return zb_fail(ZERO_ERR_INVALID_ARG, "zero_reduce_scatter_bucket_ex: unknown flags");
     if (!ctx) return zb_fail(ZERO_ERR_INVALID_ARG, "zero_reduce_scatter_bucket: ctx is NULL");
     zero_status s = check_device(ctx, where);
     if (s != ZERO_OK) return s;
-    int64_t lo, hi;
-    if (bucket == -1) {
-        lo = 0;
-        hi = ctx->T;
-    } else if (bucket < 0 || bucket >= static_cast<int64_t>(ctx->bucket_lo.size())) {
-        return zb_fail(ZERO_ERR_RANGE, "zero_reduce_scatter_bucket: bucket index out of range");
-    } else {
-        lo = ctx->bucket_lo[bucket];
-        hi = ctx->bucket_hi[bucket];
-    }
+    const int64_t nb = static_cast<int64_t>(ctx->bucket_lo.size());
+    if (!(first == -1 && count == 1) && (first < 0 || count < 1 || first > nb - count))
+        return zb_fail(ZERO_ERR_RANGE, "zero_reduce_scatter_buckets: need 0 <= first, 1 <= count and "
+                                       "first + count <= n_buckets (or first = -1, count = 1)");
     if ((s = check_ranks(grads, ctx->R, 16, where, "grads")) != ZERO_OK) return s;
     if ((s = check_ranks(acc, ctx->R, 32, where, "acc")) != ZERO_OK) return s;
     zb::RankPtrs p;
@@ -322,15 +354,8 @@ extern "C" zero_status zero_reduce_scatter_bucket_ex(zero_ctx_t* ctx, int64_t bu
         p.g[r] = grads[r];
         p.acc[r] = acc[r];
     }
-    const zb::RsNorm norm = zb_rs_norm_note(ctx, bucket, (flags & ZERO_RS_NORM) != 0);
-    cudaError_t e = zb::launch_reduce_scatter(ctx->R, ctx->dtype, ctx->S, lo, hi, ctx->st, p,
-                                              static_cast<cudaStream_t>(stream),
-                                              (flags & ZERO_RS_ACCUMULATE) != 0, 0,
-                                              norm.partials ? &norm : nullptr);
-    if (e != cudaSuccess) {
-        ctx->rs_norm_valid[bucket < 0 ? ctx->bucket_lo.size() : static_cast<size_t>(bucket)] = 0;
-        return cuda_fail(where, e);
-    }
+    cudaError_t e = zb_rs_launch(ctx, first, count, p, static_cast<cudaStream_t>(stream), flags, 0);
+    if (e != cudaSuccess) return cuda_fail(where, e);
     return ZERO_OK;
 }
 
@@ -575,7 +600,7 @@ extern "C" zero_status zero_reduce_scatter_shard(zero_ctx_t* ctx, int64_t bucket
     // the bucket's part inside the owners' flat range [owner_lo * S, owner_hi * S)
     lo = std::max<int64_t>(lo, static_cast<int64_t>(owner_lo) * ctx->S);
     hi = std::min<int64_t>(hi, static_cast<int64_t>(owner_hi) * ctx->S);
-    zb_rs_norm_note(ctx, bucket, false);  // the bucket's norm share (if any) is stale now
+    zb_rs_norm_note(ctx, bucket, 1, false);  // the bucket's norm share (if any) is stale now
     if (lo >= hi) return ZERO_OK;  // no element of this bucket is owned here
     zb::RankPtrs p{};
     for (int r = 0; r < ctx->R; ++r) {

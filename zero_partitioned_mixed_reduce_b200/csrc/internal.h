@@ -156,9 +156,15 @@ struct zero_ctx_s {
     double grad_divisor = 1.0;    // the divisor ZERO_RS_NORM unscales by
 };
 
-// Bookkeeping of a reduce-scatter of `bucket` (-1: whole range), with or
-// without its norm share; returns the launch's norm arguments (capi.cpp).
-zb::RsNorm zb_rs_norm_note(zero_ctx_t* ctx, int64_t bucket, bool norm);
+// Bookkeeping of a reduce-scatter of buckets [first, first + count) (first
+// -1: the whole range), with or without its norm share; returns the launch's
+// norm arguments for the first bucket's slot (capi.cpp).
+zb::RsNorm zb_rs_norm_note(zero_ctx_t* ctx, int64_t first, int64_t count, bool norm);
+// One reduce-scatter launch over buckets [first, first + count), a
+// contiguous flat range (first -1, count 1: every element), flags as for
+// zero_reduce_scatter_bucket_ex, grid capped at max_sms SMs (0: all).
+cudaError_t zb_rs_launch(zero_ctx_t* ctx, int64_t first, int64_t count, const zb::RankPtrs& p,
+                         cudaStream_t s, int32_t flags, int max_sms);
 
 void zb_sched_destroy(zero_ctx_t* ctx);
 

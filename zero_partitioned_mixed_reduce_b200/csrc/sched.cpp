@@ -130,25 +130,29 @@ extern "C" zero_status zero_grads_ready(zero_ctx_t* ctx, int64_t first, int64_t 
         p.acc[r] = acc[r];
     }
     cudaStream_t cs = static_cast<cudaStream_t>(stream);
+    // the buckets this call completes, in ascending order
+    std::vector<int64_t> done;
     for (int64_t k = first; k < first + count; ++k) {
         s->tensor_ready[k] = 1;
         const int64_t b = ctx->tensor_bucket[k];
-        if (++s->bucket_ready[b] != ctx->bucket_ntensors[b]) continue;
-        // the step's last bucket has no compute left to hide behind: whole GPU
-        const bool last_bucket = s->buckets_issued + 1 == static_cast<int64_t>(ctx->bucket_lo.size());
-        // the whole bucket is ready: reduce-scatter it behind the caller's work
-        const zb::RsNorm norm = zb_rs_norm_note(ctx, b, (flags & ZERO_RS_NORM) != 0);
-        cudaError_t e = cudaEventRecord(s->bucket_event[b], cs);
-        if (e == cudaSuccess) e = cudaStreamWaitEvent(s->comm, s->bucket_event[b], 0);
-        if (e == cudaSuccess)
-            e = zb::launch_reduce_scatter(ctx->R, ctx->dtype, ctx->S, ctx->bucket_lo[b], ctx->bucket_hi[b],
-                                          ctx->st, p, s->comm, (flags & ZERO_RS_ACCUMULATE) != 0,
-                                          last_bucket ? 0 : s->comm_sms, norm.partials ? &norm : nullptr);
-        if (e != cudaSuccess) {
-            ctx->rs_norm_valid[b] = 0;
-            return cuda_err(where, e);
-        }
-        s->buckets_issued += 1;
+        if (++s->bucket_ready[b] == ctx->bucket_ntensors[b]) done.push_back(b);
+    }
+    std::sort(done.begin(), done.end());
+    const int64_t nb = static_cast<int64_t>(ctx->bucket_lo.size());
+    // each run of consecutive buckets is one contiguous flat range: one
+    // launch behind the caller's work so far
+    for (size_t i = 0; i < done.size();) {
+        size_t j = i + 1;
+        while (j < done.size() && done[j] == done[j - 1] + 1) ++j;
+        const int64_t b0 = done[i], cnt = static_cast<int64_t>(j - i);
+        // the step's last buckets have no compute left to hide behind: whole GPU
+        const bool last = s->buckets_issued + cnt == nb;
+        cudaError_t e = cudaEventRecord(s->bucket_event[b0], cs);
+        if (e == cudaSuccess) e = cudaStreamWaitEvent(s->comm, s->bucket_event[b0], 0);
+        if (e == cudaSuccess) e = zb_rs_launch(ctx, b0, cnt, p, s->comm, flags, last ? 0 : s->comm_sms);
+        if (e != cudaSuccess) return cuda_err(where, e);
+        s->buckets_issued += cnt;
+        i = j;
     }
     return ZERO_OK;
 }
