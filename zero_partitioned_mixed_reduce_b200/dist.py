@@ -157,19 +157,34 @@ class DistributedZero:
             self.bucket_seen = [0] * len(self.plan.buckets)
             self.comm_token = torch.zeros(1, dtype=torch.float32, device=self.token.device)
         compute = torch.cuda.current_stream()
+        done = []
         for k in range(first, first + count):
             b = self.plan.tensor_bucket[k]
             self.bucket_seen[b] += 1
-            if self.bucket_seen[b] != self.bucket_size[b]:
-                continue
-            ready = torch.cuda.Event()
-            ready.record(compute)
-            with torch.cuda.stream(self.comm):
-                self.comm.wait_event(ready)
-                dist.all_reduce(self.comm_token, group=self.group)  # every rank wrote bucket b
-                Z.zero_reduce_scatter_shard(self.ctx, b, self.grad_ptrs, self.acc_list, self.rank,
-                                            self.rank + 1, Z.ZERO_RS_ACCUMULATE if self.micro else 0,
-                                            self.comm)
+            if self.bucket_seen[b] == self.bucket_size[b]:
+                done.append(b)
+        if not done:
+            return
+        ready = torch.cuda.Event()
+        ready.record(compute)
+        # one token all-reduce per run of consecutive buckets this call
+        # completes (every rank reports alike, so the runs match across ranks)
+        done.sort()
+        runs, i = [], 0
+        while i < len(done):
+            j = i + 1
+            while j < len(done) and done[j] == done[j - 1] + 1:
+                j += 1
+            runs.append(done[i:j])
+            i = j
+        with torch.cuda.stream(self.comm):
+            self.comm.wait_event(ready)
+            for run in runs:
+                dist.all_reduce(self.comm_token, group=self.group)  # every rank wrote these buckets
+                for b in run:
+                    Z.zero_reduce_scatter_shard(self.ctx, b, self.grad_ptrs, self.acc_list, self.rank,
+                                                self.rank + 1, Z.ZERO_RS_ACCUMULATE if self.micro else 0,
+                                                self.comm)
 
     def join(self):
         """End of a micro-batch's backward: every bucket must have been
