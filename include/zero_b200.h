@@ -789,6 +789,47 @@ zero_status zero_cpu_update(const zero_plan_t* plan, const zero_loss_scale_state
 zero_status zero_cpu_commit(const zero_loss_scale_config* cfg, zero_loss_scale_state* inout,
                             const zero_cpu_decision* decision);
 
+/*
+ * Per-call tracing. zero_trace_start makes every later call of the context
+ * that queues GPU work bracket that work with two timing events on its
+ * stream, up to `capacity` calls (1 .. 2^20; later ones are counted as
+ * dropped); it replaces a trace already started. zero_trace_read waits for
+ * the recorded events and copies the records, in call order, into out
+ * (host, room for max), sets *count (and *dropped, if not NULL), and empties
+ * the trace; zero_trace_stop ends tracing and frees its events. Traced
+ * calls: the reduce-scatters (ZERO_TRACE_REDUCE_SCATTER, arg = first bucket
+ * or -1), including those the scheduler issues on its stream; zero_step /
+ * zero_step_ex (ZERO_TRACE_STEP, the norm pass included) and
+ * zero_step_shard(_ex) (ZERO_TRACE_STEP, arg = owner_lo); zero_grad_norm_shard
+ * (ZERO_TRACE_NORM); zero_step_commit (ZERO_TRACE_COMMIT); zero_gather_layer
+ * and zero_gather_layers (ZERO_TRACE_GATHER, arg = first layer), including
+ * the scheduler's prefetches. A call made while its stream is being
+ * captured into a CUDA graph is not traced. ms is the device time between
+ * the two events: the call's own kernels plus anything the stream ran in
+ * between. A record whose end event could not be placed has call 0 and
+ * ms -1. Host state: calls on one context must not overlap (as for every
+ * call on a context).
+ * Errors: ZERO_ERR_INVALID_ARG; zero_trace_read: ZERO_ERR_STATE (not
+ * started), ZERO_ERR_RANGE (max smaller than the record count; nothing is
+ * consumed), ZERO_ERR_CUDA.
+ */
+#define ZERO_TRACE_REDUCE_SCATTER 1
+#define ZERO_TRACE_STEP 2
+#define ZERO_TRACE_GATHER 3
+#define ZERO_TRACE_NORM 4
+#define ZERO_TRACE_COMMIT 5
+typedef struct {
+    int32_t call;     /* ZERO_TRACE_* */
+    int32_t reserved;
+    int64_t arg;      /* bucket, layer or owner index; -1 for the whole range */
+    float ms;         /* device time between the call's two events */
+    float reserved2;
+} zero_trace_record;
+zero_status zero_trace_start(zero_ctx_t* ctx, int32_t capacity);
+zero_status zero_trace_read(zero_ctx_t* ctx, zero_trace_record* out, int32_t max, int32_t* count,
+                            int64_t* dropped);
+zero_status zero_trace_stop(zero_ctx_t* ctx);
+
 /* zero_sync -- synchronize `stream` and report any pending CUDA error. */
 zero_status zero_sync(zero_ctx_t* ctx, void* stream);
 

@@ -25,6 +25,13 @@ ZERO_RS_ACCUMULATE = 1
 ZERO_RS_NORM = 2
 ZERO_STEP_ADD_ACC = 1
 ZERO_STEP_NORM_FROM_RS = 2
+ZERO_TRACE_REDUCE_SCATTER, ZERO_TRACE_STEP, ZERO_TRACE_GATHER, ZERO_TRACE_NORM, ZERO_TRACE_COMMIT = 1, 2, 3, 4, 5
+TRACE_NAMES = {0: "untimed", 1: "reduce_scatter", 2: "step", 3: "gather", 4: "norm", 5: "commit"}
+
+
+class zero_trace_record(C.Structure):
+    _fields_ = [("call", C.c_int32), ("reserved", C.c_int32), ("arg", C.c_int64), ("ms", C.c_float),
+                ("reserved2", C.c_float)]
 
 STATUS_NAMES = {0: "ZERO_OK", 1: "ZERO_ERR_INVALID_ARG", 2: "ZERO_ERR_ALIGN", 3: "ZERO_ERR_CUDA",
                 4: "ZERO_ERR_OOM", 5: "ZERO_ERR_RANGE", 6: "ZERO_ERR_TIMEOUT", 7: "ZERO_ERR_STATE"}
@@ -118,6 +125,10 @@ _sig("zero_reduce_scatter_bucket", _S, [_P, C.c_int64, _PP, _PP, _P])
 _sig("zero_step", _S, [_P, C.POINTER(zero_adamw), C.POINTER(zero_state), _PP, _P])
 _sig("zero_reduce_scatter_bucket_ex", _S, [_P, C.c_int64, _PP, _PP, C.c_int32, _P])
 _sig("zero_reduce_scatter_buckets", _S, [_P, C.c_int64, C.c_int64, _PP, _PP, C.c_int32, _P])
+_sig("zero_trace_start", _S, [_P, C.c_int32])
+_sig("zero_trace_read", _S, [_P, C.POINTER(zero_trace_record), C.c_int32, C.POINTER(C.c_int32),
+                             C.POINTER(C.c_int64)])
+_sig("zero_trace_stop", _S, [_P])
 _sig("zero_step_ex", _S, [_P, C.POINTER(zero_adamw), C.POINTER(zero_state), _PP,
                           C.POINTER(zero_step_opts), _P])
 _sig("zero_gather_layer", _S, [_P, C.c_int64, C.POINTER(zero_state), _P, _P])
@@ -294,6 +305,23 @@ def zero_reduce_scatter_buckets(ctx, first, count, grads, acc, flags=0, stream=N
     g, ga = _ptr_array(grads)
     a, aa = _ptr_array(acc)
     _check(_lib.zero_reduce_scatter_buckets(ctx, first, count, g, a, flags, _stream(stream)))
+
+
+def zero_trace_start(ctx, capacity=4096):
+    _check(_lib.zero_trace_start(ctx, capacity))
+
+
+def zero_trace_read(ctx, max_records=4096):
+    """The traced calls since the last read: (list of (name, arg, ms), dropped)."""
+    buf = (zero_trace_record * max_records)()
+    n, dropped = C.c_int32(0), C.c_int64(0)
+    _check(_lib.zero_trace_read(ctx, buf, max_records, C.byref(n), C.byref(dropped)))
+    return [(TRACE_NAMES.get(buf[i].call, str(buf[i].call)), int(buf[i].arg), float(buf[i].ms))
+            for i in range(n.value)], int(dropped.value)
+
+
+def zero_trace_stop(ctx):
+    _check(_lib.zero_trace_stop(ctx))
 
 
 def zero_ctx_set_grad_divisor(ctx, grad_divisor):

@@ -265,6 +265,7 @@ cudaError_t zb_rs_launch(zero_ctx_t* ctx, int64_t first, int64_t count, const zb
     }
     const bool with_norm = (flags & ZERO_RS_NORM) != 0;
     const zb::RsNorm norm = zb_rs_norm_note(ctx, first, count, with_norm);
+    ZbTraceScope trace(ctx, ZERO_TRACE_REDUCE_SCATTER, s, first);
     cudaError_t e = cudaSuccess;
     // a group's share lands in its first bucket's slot; the others hold 0
     if (with_norm && first >= 0 && count > 1)
@@ -288,6 +289,7 @@ extern "C" zero_status zero_ctx_destroy(zero_ctx_t* ctx) {
     cudaSetDevice(ctx->device);
     cudaError_t e = cudaDeviceSynchronize();
     zb_sched_destroy(ctx);
+    zb_trace_destroy(ctx);
     cudaFree(ctx->st);
     cudaFree(ctx->partials);
     cudaFree(ctx->rs_norm_partials);
@@ -524,6 +526,7 @@ extern "C" zero_status zero_step_ex(zero_ctx_t* ctx, const zero_adamw* hp, const
                            "not record a current norm share of every bucket with this grad_divisor");
         }
     }
+    ZbTraceScope trace(ctx, ZERO_TRACE_STEP, cs, -1);
     cudaError_t e = cudaSuccess;
     // clipping needs the global norm before any element is updated: the
     // reduce-scatters' shares, or one read-only pass over the accumulators,
@@ -607,6 +610,7 @@ extern "C" zero_status zero_reduce_scatter_shard(zero_ctx_t* ctx, int64_t bucket
         p.g[r] = grads[r];
         p.acc[r] = (r >= owner_lo && r < owner_hi) ? acc[r] : nullptr;
     }
+    ZbTraceScope trace(ctx, ZERO_TRACE_REDUCE_SCATTER, static_cast<cudaStream_t>(stream), bucket);
     cudaError_t e = zb::launch_reduce_scatter(ctx->R, ctx->dtype, ctx->S, lo, hi, ctx->st, p,
                                               static_cast<cudaStream_t>(stream), (flags & ZERO_RS_ACCUMULATE) != 0);
     if (e != cudaSuccess) return cuda_fail(where, e);
@@ -635,6 +639,7 @@ extern "C" zero_status zero_grad_norm_shard(zero_ctx_t* ctx, const void* const* 
         p.acc[r] = (acc && r >= owner_lo && r < owner_hi) ? acc[r] : nullptr;
     }
     cudaStream_t cs = static_cast<cudaStream_t>(stream);
+    ZbTraceScope trace(ctx, ZERO_TRACE_NORM, cs, owner_lo);
     cudaError_t e = grads ? zb::launch_grad_norm(sp, p, cs) : zb::launch_clip_norm(sp, p, cs);
     if (e != cudaSuccess) return cuda_fail(where, e);
     return ZERO_OK;
@@ -689,6 +694,7 @@ extern "C" zero_status zero_step_shard_ex(zero_ctx_t* ctx, const zero_adamw* hp,
             p.param[k][r] = owned ? state->param[from][r] : nullptr;
         }
     }
+    ZbTraceScope trace(ctx, ZERO_TRACE_STEP, cs, owner_lo);
     cudaError_t e = cudaSuccess;
     if (clip) e = zb::launch_clip_from_norm(sp, global_norm_sq, cs);
     if (e == cudaSuccess) e = fused ? zb::launch_fused_step(sp, p, cs) : zb::launch_step_from_acc(sp, p, cs);
@@ -722,6 +728,7 @@ extern "C" zero_status zero_step_commit(zero_ctx_t* ctx, const double* reduced, 
     sp.backoff = ctx->cfg.backoff_factor;
     sp.min_scale = ctx->cfg.min_scale;
     sp.st = ctx->st;
+    ZbTraceScope trace(ctx, ZERO_TRACE_COMMIT, static_cast<cudaStream_t>(stream), -1);
     cudaError_t e = zb::launch_fsm_commit(sp, reduced, static_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return cuda_fail(where, e);
     return ZERO_OK;
@@ -747,6 +754,7 @@ extern "C" zero_status zero_gather_layer(zero_ctx_t* ctx, int64_t layer, const z
         p.param[0][r] = state->param[0][r];
         p.param[1][r] = sets == 2 ? state->param[1][r] : state->param[0][r];
     }
+    ZbTraceScope trace(ctx, ZERO_TRACE_GATHER, static_cast<cudaStream_t>(stream), layer);
     cudaError_t e = zb::launch_gather(ctx->R, ctx->S, ctx->layer_lo[layer], ctx->layer_hi[layer],
                                       ctx->st, p, out, static_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return cuda_fail(where, e);
@@ -782,6 +790,7 @@ extern "C" zero_status zero_gather_layers(zero_ctx_t* ctx, int64_t first, int64_
         p.param[0][r] = state->param[0][r];
         p.param[1][r] = sets == 2 ? state->param[1][r] : state->param[0][r];
     }
+    ZbTraceScope trace(ctx, ZERO_TRACE_GATHER, static_cast<cudaStream_t>(stream), first);
     cudaError_t e = zb::launch_gather_many(ctx->R, ctx->S, static_cast<int>(count),
                                            ctx->layer_lo.data() + first, ctx->layer_hi.data() + first,
                                            ctx->st, p, outs, static_cast<cudaStream_t>(stream));

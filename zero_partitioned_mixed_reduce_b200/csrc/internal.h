@@ -122,6 +122,7 @@ int step_grid_cap(int device);
 // Context: the plan's layout, the loss-scale config, the device scratch, and
 // the overlap / prefetch scheduler (sched.cpp).
 struct zero_sched;  // scheduler state, sched.cpp
+struct zero_trace;  // per-call trace, trace.cpp
 
 struct zero_ctx_s {
     int device = 0;
@@ -154,6 +155,24 @@ struct zero_ctx_s {
     std::vector<uint8_t> rs_norm_valid;
     std::vector<double> rs_norm_div;
     double grad_divisor = 1.0;    // the divisor ZERO_RS_NORM unscales by
+    zero_trace* trace = nullptr;  // per-call trace while started
+};
+
+void zb_trace_destroy(zero_ctx_t* ctx);
+
+// Brackets the work a traced call queues on `s` with the trace's two events
+// (nothing while the trace is off, the ring is full or `s` is capturing).
+class ZbTraceScope {
+public:
+    ZbTraceScope(zero_ctx_t* ctx, int32_t call, cudaStream_t s, int64_t arg);
+    ~ZbTraceScope();
+    ZbTraceScope(const ZbTraceScope&) = delete;
+    ZbTraceScope& operator=(const ZbTraceScope&) = delete;
+
+private:
+    zero_trace* t_;
+    cudaStream_t s_;
+    int32_t slot_;
 };
 
 // Bookkeeping of a reduce-scatter of buckets [first, first + count) (first

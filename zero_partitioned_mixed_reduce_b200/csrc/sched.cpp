@@ -244,10 +244,12 @@ zero_status issue_upto(zero_ctx_t* ctx, int64_t upto) {
         if (s->slot_pos[slot] >= 0) e = cudaStreamWaitEvent(s->comm, s->slot_free[slot], 0);
         const int64_t layer = s->dir > 0 ? pos : nl - 1 - pos;
         void* out = s->bufs[slot];
-        if (e == cudaSuccess)
+        if (e == cudaSuccess) {
+            ZbTraceScope trace(ctx, ZERO_TRACE_GATHER, s->comm, layer);
             // the pass's first gather has nothing before it to hide behind: whole GPU
             e = zb::launch_gather_many(ctx->R, ctx->S, 1, &ctx->layer_lo[layer], &ctx->layer_hi[layer], ctx->st,
                                        s->params, &out, s->comm, pos == 0 ? 0 : s->comm_sms);
+        }
         if (e == cudaSuccess) e = cudaEventRecord(s->slot_ready[slot], s->comm);
         if (e != cudaSuccess) return cuda_err("zero_layer_acquire", e);
         s->slot_pos[slot] = pos;
