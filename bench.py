@@ -461,6 +461,20 @@ def run_ours(args, world, rank, local):
     assert f1["last_overflow"] == 0 and f1["t"] == f0["t"] + K
     ms, units = aggregate(ms_local, float(b.P) * K, world)
 
+    # one more step, untimed, through the library's per-call trace: the
+    # device time of each call kind
+    Z = b.Z
+    Z.zero_trace_start(b.ctx, 4096)
+    b.step_main(stream)
+    b.gather(stream)
+    recs, _ = Z.zero_trace_read(b.ctx)
+    Z.zero_trace_stop(b.ctx)
+    per_call = {}
+    for name, _, t_ms in recs:
+        e = per_call.setdefault(name, {"calls": 0, "ms": 0.0})
+        e["calls"] += 1
+        e["ms"] += t_ms
+
     step_bytes, main_bytes = b.step_bytes()
     peak, peak_src = hbm_peak()
     kavg = statistics.mean(kern_ms)
@@ -527,6 +541,8 @@ def run_ours(args, world, rank, local):
                    "launches_per_step": len(b.gather_buckets) or len(b.plan.layers)},
         "clocks": clk,
         "gpu_launches": K * b.launches_per_step(),
+        "trace_one_step": {"source": "zero_trace_read, one untimed step after the timed region",
+                           "calls": per_call},
     }
     if not args.no_e2e:
         out["e2e"] = e2e(b, args, stream, world)
