@@ -16,8 +16,10 @@ than the 126 MB L2.
 
 With N > 1 (under torch.distributed.run) every rank runs its own independent
 replica of the workload (weak scaling, no collective on the data path); the
-time is the maximum over ranks. `--impl reference` times the CPU oracle on
-host cores on a bounded sample of the same workload.
+time is the maximum over ranks. The step and the gathers are captured once
+into CUDA graphs through the C ABI and replayed (`--eager` issues every
+launch instead). `--impl reference` times the CPU oracle on host cores on a
+bounded sample of the same workload.
 """
 import argparse
 import datetime
@@ -83,8 +85,11 @@ def parse_args(argv=None):
                     help="bucket sizes (elements; 0: one bucket for the whole model) for --rs-sweep")
     ap.add_argument("--dist", action="store_true",
                     help="the real multi-GPU ZeRO step over the job's GPUs (DistributedZero) instead")
-    ap.add_argument("--graph", action="store_true",
-                    help="capture the step and the gathers once into CUDA graphs and replay them")
+    ap.add_argument("--graph", dest="graph", action="store_true", default=True,
+                    help="(default) capture the step and the gathers once into CUDA graphs, "
+                         "through the C ABI, and replay them")
+    ap.add_argument("--eager", dest="graph", action="store_false",
+                    help="issue every launch through the C ABI instead of replaying CUDA graphs")
     ap.add_argument("--first-tensors", type=int, default=0,
                     help="use only the first N tensors of the workload (small profiling cases)")
     return ap.parse_args(argv)
@@ -387,32 +392,42 @@ class Bench:
                 Z.zero_gather_layer(self.ctx, l, self.state.handle, self.layer_buf, stream)
 
     def capture(self, stream, steps):
-        """Capture the step and the gathers into two CUDA graphs (the event
+        """Capture the step and the gathers into CUDA graphs (the event
         between them stays outside) after reserving `steps` bias corrections."""
         hp = self.wl["hp"]
         self.Z.zero_ctx_reserve_steps(self.ctx, steps, hp["beta1"], hp["beta2"], stream)
+        self.step_graphs = {}
+        self.capture_step(stream, self.grads)
         side = torch.cuda.Stream()
         side.wait_stream(stream)
-        self.graphs = (torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph())
-        with torch.cuda.graph(self.graphs[0], stream=side):
-            self.step_main(torch.cuda.current_stream())
-        with torch.cuda.graph(self.graphs[1], stream=side):
+        self.gather_graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(self.gather_graph, stream=side):
             self.gather(torch.cuda.current_stream())
         stream.wait_stream(side)
+        self.graphs = True
+
+    def capture_step(self, stream, grads):
+        """One step graph per set of replica buffers (the e2e leg double-buffers)."""
+        side = torch.cuda.Stream()
+        side.wait_stream(stream)
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=side):
+            self.step_main(torch.cuda.current_stream(), grads)
+        stream.wait_stream(side)
+        self.step_graphs[id(grads)] = (g, grads)
 
     def step(self, stream, ev=None, grads=None):
         graphs = getattr(self, "graphs", None)
         if ev is not None:
             ev[0].record(stream)
         if graphs:
-            assert grads is None or grads is self.grads
-            graphs[0].replay()
+            self.step_graphs[id(self.grads if grads is None else grads)][0].replay()
         else:
             self.step_main(stream, grads)
         if ev is not None:
             ev[1].record(stream)
         if graphs:
-            graphs[1].replay()
+            self.gather_graph.replay()
         else:
             self.gather(stream)
         if ev is not None and len(ev) > 2:
@@ -529,8 +544,8 @@ def run_ours(args, world, rank, local):
             "bytes_per_step": step_bytes,
             "l2": f"inputs larger than L2 ({step_bytes / 1e9:.1f} GB touched per step, L2 126 MB)",
             "parallelism": "1 GPU" if world == 1 else f"{world} independent replicas",
-            "launch": "CUDA graph replay (step graph, event, gather graph)" if args.graph
-                      else "eager launches through the C ABI",
+            "launch": "CUDA graph replay (step graph, event, gather graph), captured through the C ABI"
+                      if args.graph else "eager launches through the C ABI",
         },
         "roofline": {"bound": "hbm", "kernel": kernel_name, "achieved": achieved, "peak": peak,
                      "peak_source": f"{peak_src} hbm_gbs", "unit": "GB/s", "frac": achieved / peak,
@@ -547,6 +562,7 @@ def run_ours(args, world, rank, local):
     if not args.no_e2e:
         out["e2e"] = e2e(b, args, stream, world)
     b.graphs = None
+    b.step_graphs, b.gather_graph = {}, None
     b.close()
     del b
     torch.cuda.empty_cache()
@@ -560,15 +576,17 @@ def e2e(b, args, stream, world):
     """The same metric through the C ABI with host buffers: every step copies
     its R gradient replicas from pinned host memory and reads the step's
     result (the loss-scale state: overflow, skip, scale, grad norm) back.
-    Without --graph the replicas are double-buffered: step s+1's upload runs
-    on a copy stream while step s computes; every copy is inside the timed
-    region."""
+    The replicas are double-buffered where a second set fits: step s+1's
+    upload runs on a copy stream while step s computes (with graphs, one step
+    graph per buffer set); every copy is inside the timed region."""
     host = [g.cpu().pin_memory() for g in b.grads]
     K = max(3, min(args.steps, 10))
     nbytes = sum(h.numel() * h.element_size() for h in host)
     graphs = getattr(b, "graphs", None)
     room = torch.cuda.mem_get_info()[0] > 1.25 * nbytes
-    bufs = [b.grads] if (graphs or not room) else [b.grads, [torch.empty_like(g) for g in b.grads]]
+    bufs = [b.grads] if not room else [b.grads, [torch.empty_like(g) for g in b.grads]]
+    if graphs and len(bufs) == 2:
+        b.capture_step(stream, bufs[1])
     copy = torch.cuda.Stream()
     copied = [torch.cuda.Event() for _ in bufs]
     consumed = [torch.cuda.Event() for _ in bufs]
@@ -607,8 +625,7 @@ def e2e(b, args, stream, world):
     return {"value": units / (ms * 1e-3), "unit": "params/s", "h2d_bytes_per_step": nbytes,
             "d2h_bytes_per_step": 40, "steps": K,
             "pipelining": "double-buffered replicas: step s+1 uploads during step s"
-                          if len(bufs) == 2 else
-                          "none (graph replay reads fixed buffers, or no room for a second set)"}
+                          if len(bufs) == 2 else "none (no room for a second set of replicas)"}
 
 
 # ---- the CPU oracle as a baseline ----------------------------------------------
