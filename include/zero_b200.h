@@ -480,7 +480,11 @@ zero_status zero_step_shard_ex(zero_ctx_t* ctx, const zero_adamw* hp, const zero
  * This is rank o's part of a multi-GPU bucketed reduce-scatter: grads[r] is
  * rank r's gradient buffer (peer-mapped; plain loads, no multicast) and only
  * acc[o] for the owned ranks is touched (other entries may be NULL). A
- * bucket with no owned element launches nothing.
+ * bucket with no owned element launches nothing. ZERO_RS_NORM takes the
+ * owned part's norm share as zero_reduce_scatter_bucket_ex does (0 for a
+ * bucket with no owned element), recorded for this owner range; a context
+ * that several owner ranges share keeps only the last range's shares, so
+ * use one context per rank for it.
  * Defines: [legal] "Reduce-Scatter" and [instr] ZeRO-2 "Communication".
  * Errors: ZERO_ERR_RANGE (bucket, owner range), ZERO_ERR_INVALID_ARG,
  * ZERO_ERR_ALIGN, ZERO_ERR_CUDA.
@@ -496,10 +500,16 @@ zero_status zero_reduce_scatter_shard(zero_ctx_t* ctx, int64_t bucket, const voi
  * scale)), where x is the element's reduced gradient read either from the
  * R replicas (grads != NULL, summed in rank order as the fused step sums
  * them) or from the owners' accumulators (acc != NULL); partial[1] = 0.
- * Exactly one of grads and acc is given. The ranks all-reduce partial[0]
- * (sum) and pass it to zero_step_shard_ex as global_norm_sq.
+ * With grads and acc both NULL, partial[0] is instead the sum, in slot
+ * order, of the norm shares that this owner range's ZERO_RS_NORM
+ * reduce-scatters (zero_reduce_scatter_shard) took with this grad_divisor
+ * (the context's, zero_ctx_set_grad_divisor): no accumulator is read.
+ * The ranks all-reduce partial[0] (sum) and pass it to zero_step_shard_ex
+ * as global_norm_sq.
  * partial: device, 2 doubles, 8-byte aligned.
- * Errors: ZERO_ERR_RANGE, ZERO_ERR_INVALID_ARG, ZERO_ERR_ALIGN, ZERO_ERR_CUDA.
+ * Errors: ZERO_ERR_RANGE, ZERO_ERR_INVALID_ARG (both grads and acc given),
+ * ZERO_ERR_ALIGN, ZERO_ERR_CUDA; ZERO_ERR_STATE when the shares are stale,
+ * missing, or were taken with another owner range or divisor.
  */
 zero_status zero_grad_norm_shard(zero_ctx_t* ctx, const void* const* grads, float* const* acc,
                                  double grad_divisor, int32_t owner_lo, int32_t owner_hi,

@@ -79,17 +79,21 @@ def main():
         dz.layer_release(l)
     dz.close()
     check_accumulate_and_clip(rank, world)
+    # the same with the clipping norm taken by the reduce-scatters (divisor 2:
+    # the two-micro-batch steps use the shares, the others the accumulator)
+    check_accumulate_and_clip(rank, world, norm_divisor=2.0)
     dist.barrier()
     dist.destroy_process_group()
     if rank == 0:
         print("ok")
 
 
-def check_accumulate_and_clip(rank, world):
+def check_accumulate_and_clip(rank, world, norm_divisor=None):
     """Two-pass steps over accumulated micro-batches and fused steps, with
     global-norm clipping, against the oracle's step_ex."""
     numels = [50_001, 77, 3000]
-    dz = DistributedZero(numels, None, Z.ZERO_BF16, Z.ZERO_SCALE_NONE, bucket_elems=20_000, accumulate=True)
+    dz = DistributedZero(numels, None, Z.ZERO_BF16, Z.ZERO_SCALE_NONE, bucket_elems=20_000, accumulate=True,
+                         norm_divisor=norm_divisor)
     wl = synth.custom_workload(numels, world, Z.ZERO_BF16, Z.ZERO_SCALE_NONE, 1.0, 1000, sigma=1e-2,
                                index=56)
     lay = O.Layout(numels, world, 8)

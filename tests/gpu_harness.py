@@ -303,14 +303,18 @@ class Case:
         self.g.check()
         return skipped
 
-    def step_sharded_ex(self, splits, n_micro=1, grad_divisor=1.0, max_grad_norm=0.0, inject=None):
+    def step_sharded_ex(self, splits, n_micro=1, grad_divisor=1.0, max_grad_norm=0.0, inject=None,
+                        rs_norm=False):
         """The multi-rank step emulated shard range by shard range, with the
         cross-rank sums done here: fused (path "pingpong"/"inplace") or
         two-pass (paths "twopass*": per micro-batch and bucket,
         zero_reduce_scatter_shard for each range), optional global-norm
         clipping (zero_grad_norm_shard per range, summed), then
         zero_step_shard_ex per range and one zero_step_commit.
-        inject: (micro, rank, element, bits)."""
+        inject: (micro, rank, element, bits). rs_norm (two-pass, clipped): each
+        range's last reduce-scatters take its norm share (ZERO_RS_NORM), summed
+        by zero_grad_norm_shard from the shares before the next range's
+        reduce-scatters reuse the context's slots."""
         self.step_no += 1
         scale = self.ofsm.scale if self.mode != O.SCALE_NONE else 1.0
         g = np.stack([np.stack([u16(synth.flat_grads(self.wl, self.step_no * 100 + mu, r, scale, "cpu"))
@@ -321,19 +325,30 @@ class Case:
         add_acc = self.path == "fused_acc" and n_micro > 1  # last micro-batch fused into the step
         assert twopass or add_acc or n_micro == 1
         dev = lambda: torch.zeros(2, dtype=torch.float64, device="cuda")
+        rs_norm = rs_norm and twopass and max_grad_norm > 0
+        if rs_norm:
+            Z.zero_ctx_set_grad_divisor(self.ctx, grad_divisor)
+        shares = []
         for mu in range(n_micro):
             for r in range(self.R):
                 gp = np.zeros(self.plan.T, np.uint16)
                 gp[self.idx] = g[mu, r]
                 self.grads[r].view(torch.int16).copy_(torch.from_numpy(gp.view(np.int16)))
             if twopass or (add_acc and mu < n_micro - 1):
+                last = rs_norm and mu == n_micro - 1
                 for lo, hi in splits:
                     acc = [self.acc[o] if lo <= o < hi else None for o in range(self.R)]
+                    flags = (Z.ZERO_RS_ACCUMULATE if mu else 0) | (Z.ZERO_RS_NORM if last else 0)
                     for b in range(len(self.plan.buckets)):
-                        Z.zero_reduce_scatter_shard(self.ctx, b, self.grads, acc, lo, hi,
-                                                    Z.ZERO_RS_ACCUMULATE if mu else 0)
+                        Z.zero_reduce_scatter_shard(self.ctx, b, self.grads, acc, lo, hi, flags)
+                    if last:
+                        part = dev()
+                        Z.zero_grad_norm_shard(self.ctx, None, None, lo, hi, part, grad_divisor)
+                        shares.append(part)
         norm = None
-        if max_grad_norm > 0:
+        if rs_norm:
+            norm = torch.stack(shares).sum(0)[:1].contiguous()  # the cross-rank all-reduce
+        elif max_grad_norm > 0:
             parts = []
             for lo, hi in splits:
                 part = dev()

@@ -103,6 +103,56 @@ def test_sharded_two_pass_matches_oracle(R, path, mode, dtype, n_micro, divisor,
         c.close()
 
 
+@pytest.mark.parametrize("R", [1, 2, 3, 4, 8])
+@pytest.mark.parametrize("path,mode,dtype", [("twopass_pp", O.SCALE_DYNAMIC, O.FP16),
+                                             ("twopass", O.SCALE_NONE, O.BF16)])
+@pytest.mark.parametrize("n_micro,divisor,clip", [(1, 1.0, 1e-3), (3, 3.0, 1e-3), (2, 2.0, 1e9)])
+def test_sharded_norm_from_the_reduce_scatters_matches_oracle(R, path, mode, dtype, n_micro, divisor, clip):
+    # each range's last reduce-scatters take its norm share (ZERO_RS_NORM);
+    # zero_grad_norm_shard sums the shares instead of reading the accumulator
+    c = Case([70_001, 13, 4096, 7, 999], R, dtype, 8, mode, init_scale=256.0, interval=2, path=path,
+             bucket_elems=9000, seed=R * 7 + n_micro)
+    try:
+        for step in range(3):
+            c.step_sharded_ex(SPLITS[R][step % len(SPLITS[R])], n_micro, divisor, clip, rs_norm=True)
+            c.compare()
+    finally:
+        c.close()
+
+
+def test_sharded_norm_shares_refusals():
+    c = Case([3000, 17, 2048], 2, O.BF16, 8, O.SCALE_NONE, path="twopass", bucket_elems=1000)
+    nb = len(c.plan.buckets)
+    part = torch.zeros(2, dtype=torch.float64, device="cuda")
+    acc0 = [c.acc[0], None]
+    try:
+        # no shares yet
+        with pytest.raises(Z.ZeroError) as e:
+            Z.zero_grad_norm_shard(c.ctx, None, None, 0, 1, part)
+        assert e.value.status == Z.ZERO_ERR_STATE
+        for b in range(nb):
+            Z.zero_reduce_scatter_shard(c.ctx, b, c.grads, acc0, 0, 1, Z.ZERO_RS_NORM)
+        Z.zero_grad_norm_shard(c.ctx, None, None, 0, 1, part)  # current: accepted
+        # another owner range, or another divisor: refused
+        with pytest.raises(Z.ZeroError) as e:
+            Z.zero_grad_norm_shard(c.ctx, None, None, 1, 2, part)
+        assert e.value.status == Z.ZERO_ERR_STATE
+        with pytest.raises(Z.ZeroError) as e:
+            Z.zero_grad_norm_shard(c.ctx, None, None, 0, 1, part, 2.0)
+        assert e.value.status == Z.ZERO_ERR_STATE
+        # a range's shares never feed the whole-model step
+        with pytest.raises(Z.ZeroError) as e:
+            Z.zero_step_ex(c.ctx, c.hp, c.handle, None, 1.0, 1.0, flags=Z.ZERO_STEP_NORM_FROM_RS)
+        assert e.value.status == Z.ZERO_ERR_STATE
+        # a later reduce-scatter of a bucket without the flag makes it stale
+        Z.zero_reduce_scatter_shard(c.ctx, 0, c.grads, acc0, 0, 1, 0)
+        with pytest.raises(Z.ZeroError) as e:
+            Z.zero_grad_norm_shard(c.ctx, None, None, 0, 1, part)
+        assert e.value.status == Z.ZERO_ERR_STATE
+    finally:
+        c.close()
+
+
 @pytest.mark.parametrize("R", [1, 2, 4, 8])
 @pytest.mark.parametrize("path,mode", [("pingpong", O.SCALE_DYNAMIC), ("inplace", O.SCALE_NONE)])
 @pytest.mark.parametrize("clip", [1e-3, 1e9])

@@ -538,7 +538,8 @@ def zero_reduce_scatter_shard(ctx, bucket, grads, acc, owner_lo, owner_hi, flags
 
 
 def zero_grad_norm_shard(ctx, grads, acc, owner_lo, owner_hi, partial, grad_divisor=1.0, stream=None):
-    """Owners [lo, hi)'s sum of unscaled g^2 into partial[0] (from grads or from acc)."""
+    """Owners [lo, hi)'s sum of unscaled g^2 into partial[0] (from grads, from
+    acc, or with both None from the reduce-scatters' ZERO_RS_NORM shares)."""
     g = _ptr_array(grads)
     a = _ptr_array(acc)
     _check(_lib.zero_grad_norm_shard(ctx, g[0] if g else None, a[0] if a else None, grad_divisor,

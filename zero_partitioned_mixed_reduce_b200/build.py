@@ -35,7 +35,7 @@ CXX_FLAGS = ["-O2", "-std=c++17", "-fPIC", "-Wall", "-Wextra", "-ffp-contract=of
 # does not change any result (sqrt is correctly rounded either way)
 CXX_EXTRA = {"cpu_adam.cpp": ["-O3", "-pthread", "-fno-math-errno"]}
 
-CU_SOURCES = ["kernels.cu", "noalloc.cu"]
+CU_SOURCES = ["kernels.cu", "noalloc.cu", "norm_slots.cu"]
 CPP_SOURCES = ["plan.cpp", "capi.cpp", "sched.cpp", "cpu_adam.cpp", "trace.cpp"]
 
 

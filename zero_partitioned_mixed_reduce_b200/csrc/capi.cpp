@@ -189,6 +189,7 @@ extern "C" zero_status zero_ctx_create(const zero_plan_t* plan, const zero_loss_
     const size_t slots = ctx->bucket_lo.size() + 1;
     ctx->rs_norm_valid.assign(slots, 0);
     ctx->rs_norm_div.assign(slots, 1.0);
+    ctx->rs_norm_owner.assign(slots, 0);
     auto free_scratch = [ctx] {
         cudaFree(ctx->st);
         cudaFree(ctx->partials);
@@ -230,19 +231,24 @@ extern "C" zero_status zero_ctx_set_grad_divisor(zero_ctx_t* ctx, double grad_di
     return ZERO_OK;
 }
 
-zb::RsNorm zb_rs_norm_note(zero_ctx_t* ctx, int64_t first, int64_t count, bool norm) {
+zb::RsNorm zb_rs_norm_note(zero_ctx_t* ctx, int64_t first, int64_t count, bool norm, int32_t owner_lo,
+                           int32_t owner_hi) {
     const size_t whole = ctx->bucket_lo.size();
     const size_t slot = first < 0 ? whole : static_cast<size_t>(first);
+    if (owner_hi < 0) owner_hi = ctx->R;
+    const int64_t owner = (static_cast<int64_t>(owner_lo) << 32) | static_cast<int64_t>(owner_hi);
     if (first < 0) {
         // the whole range is rewritten: every per-bucket share is stale
         std::fill(ctx->rs_norm_valid.begin(), ctx->rs_norm_valid.end(), 0);
         ctx->rs_norm_valid[whole] = norm ? 1 : 0;
         ctx->rs_norm_div[whole] = ctx->grad_divisor;
+        ctx->rs_norm_owner[whole] = owner;
     } else {
         ctx->rs_norm_valid[whole] = 0;
         for (int64_t b = first; b < first + count; ++b) {
             ctx->rs_norm_valid[static_cast<size_t>(b)] = norm ? 1 : 0;
             ctx->rs_norm_div[static_cast<size_t>(b)] = ctx->grad_divisor;
+            ctx->rs_norm_owner[static_cast<size_t>(b)] = owner;
         }
     }
     zb::RsNorm n;
@@ -512,7 +518,11 @@ extern "C" zero_status zero_step_ex(zero_ctx_t* ctx, const zero_adamw* hp, const
     const size_t nb = ctx->bucket_lo.size();
     int64_t slot_first = 0, slot_count = 0;
     if (o.flags & ZERO_STEP_NORM_FROM_RS) {
-        auto ok = [&](size_t k) { return ctx->rs_norm_valid[k] && ctx->rs_norm_div[k] == o.grad_divisor; };
+        const int64_t all_owners = static_cast<int64_t>(ctx->R);  // owner range [0, R)
+        auto ok = [&](size_t k) {
+            return ctx->rs_norm_valid[k] && ctx->rs_norm_div[k] == o.grad_divisor &&
+                   ctx->rs_norm_owner[k] == all_owners;
+        };
         bool all = true;
         for (size_t b = 0; b < nb && all; ++b) all = ok(b);
         if (ok(nb)) {
@@ -584,7 +594,8 @@ extern "C" zero_status zero_reduce_scatter_shard(zero_ctx_t* ctx, int64_t bucket
                                                  int32_t flags, void* stream) {
     const char* where = "zero_reduce_scatter_shard";
     if (!ctx || !grads) return zb_fail(ZERO_ERR_INVALID_ARG, "zero_reduce_scatter_shard: NULL ctx or grads");
-    if (flags & ~ZERO_RS_ACCUMULATE) return zb_fail(ZERO_ERR_INVALID_ARG, "zero_reduce_scatter_shard: unknown flags");
+    if (flags & ~(ZERO_RS_ACCUMULATE | ZERO_RS_NORM))
+        return zb_fail(ZERO_ERR_INVALID_ARG, "zero_reduce_scatter_shard: unknown flags");
     zero_status s = check_device(ctx, where);
     if (s != ZERO_OK) return s;
     if ((s = check_owner_range(ctx, owner_lo, owner_hi, where)) != ZERO_OK) return s;
@@ -603,17 +614,33 @@ extern "C" zero_status zero_reduce_scatter_shard(zero_ctx_t* ctx, int64_t bucket
     // the bucket's part inside the owners' flat range [owner_lo * S, owner_hi * S)
     lo = std::max<int64_t>(lo, static_cast<int64_t>(owner_lo) * ctx->S);
     hi = std::min<int64_t>(hi, static_cast<int64_t>(owner_hi) * ctx->S);
-    zb_rs_norm_note(ctx, bucket, 1, false);  // the bucket's norm share (if any) is stale now
-    if (lo >= hi) return ZERO_OK;  // no element of this bucket is owned here
+    const bool with_norm = (flags & ZERO_RS_NORM) != 0;
+    const zb::RsNorm norm = zb_rs_norm_note(ctx, bucket, 1, with_norm, owner_lo, owner_hi);
+    cudaStream_t cs = static_cast<cudaStream_t>(stream);
+    const size_t slot = bucket < 0 ? ctx->bucket_lo.size() : static_cast<size_t>(bucket);
+    if (lo >= hi) {
+        // no element of this bucket is owned here: its share is 0
+        if (!with_norm) return ZERO_OK;
+        cudaError_t e = cudaMemsetAsync(norm.out, 0, sizeof(double), cs);
+        if (e != cudaSuccess) {
+            ctx->rs_norm_valid[slot] = 0;
+            return cuda_fail(where, e);
+        }
+        return ZERO_OK;
+    }
     zb::RankPtrs p{};
     for (int r = 0; r < ctx->R; ++r) {
         p.g[r] = grads[r];
         p.acc[r] = (r >= owner_lo && r < owner_hi) ? acc[r] : nullptr;
     }
-    ZbTraceScope trace(ctx, ZERO_TRACE_REDUCE_SCATTER, static_cast<cudaStream_t>(stream), bucket);
-    cudaError_t e = zb::launch_reduce_scatter(ctx->R, ctx->dtype, ctx->S, lo, hi, ctx->st, p,
-                                              static_cast<cudaStream_t>(stream), (flags & ZERO_RS_ACCUMULATE) != 0);
-    if (e != cudaSuccess) return cuda_fail(where, e);
+    ZbTraceScope trace(ctx, ZERO_TRACE_REDUCE_SCATTER, cs, bucket);
+    cudaError_t e = zb::launch_reduce_scatter(ctx->R, ctx->dtype, ctx->S, lo, hi, ctx->st, p, cs,
+                                              (flags & ZERO_RS_ACCUMULATE) != 0, 0,
+                                              with_norm ? &norm : nullptr);
+    if (e != cudaSuccess) {
+        ctx->rs_norm_valid[slot] = 0;
+        return cuda_fail(where, e);
+    }
     return ZERO_OK;
 }
 
@@ -622,14 +649,39 @@ extern "C" zero_status zero_grad_norm_shard(zero_ctx_t* ctx, const void* const* 
                                             double* partial, void* stream) {
     const char* where = "zero_grad_norm_shard";
     if (!ctx || !partial) return zb_fail(ZERO_ERR_INVALID_ARG, "zero_grad_norm_shard: NULL ctx or partial");
-    if ((grads == nullptr) == (acc == nullptr))
-        return zb_fail(ZERO_ERR_INVALID_ARG, "zero_grad_norm_shard: give exactly one of grads and acc");
+    if (grads && acc) return zb_fail(ZERO_ERR_INVALID_ARG, "zero_grad_norm_shard: give at most one of grads and acc");
     if (!(grad_divisor >= 1.0) || !std::isfinite(grad_divisor))
         return zb_fail(ZERO_ERR_INVALID_ARG, "zero_grad_norm_shard: need a finite grad_divisor >= 1");
     zero_status s = check_device(ctx, where);
     if (s != ZERO_OK) return s;
     if ((s = check_owner_range(ctx, owner_lo, owner_hi, where)) != ZERO_OK) return s;
     if (!aligned(partial, 8)) return zb_fail(ZERO_ERR_ALIGN, "zero_grad_norm_shard: partial not 8-byte aligned");
+    if (!grads && !acc) {
+        // the sum of the shares this owner range's ZERO_RS_NORM reduce-scatters took
+        const size_t nb = ctx->bucket_lo.size();
+        const int64_t owner = (static_cast<int64_t>(owner_lo) << 32) | static_cast<int64_t>(owner_hi);
+        auto ok = [&](size_t k) {
+            return ctx->rs_norm_valid[k] && ctx->rs_norm_div[k] == grad_divisor && ctx->rs_norm_owner[k] == owner;
+        };
+        bool all = true;
+        for (size_t b = 0; b < nb && all; ++b) all = ok(b);
+        int64_t first = 0, count = 0;
+        if (ok(nb)) {
+            first = static_cast<int64_t>(nb);
+            count = 1;
+        } else if (all) {
+            count = static_cast<int64_t>(nb);
+        } else {
+            return zb_fail(ZERO_ERR_STATE,
+                           "zero_grad_norm_shard: no current ZERO_RS_NORM share of every bucket for this owner "
+                           "range and grad_divisor");
+        }
+        cudaStream_t cs = static_cast<cudaStream_t>(stream);
+        ZbTraceScope trace(ctx, ZERO_TRACE_NORM, cs, owner_lo);
+        cudaError_t e = zb::launch_sum_norm_slots(ctx->rs_norm, first, count, partial, cs);
+        if (e != cudaSuccess) return cuda_fail(where, e);
+        return ZERO_OK;
+    }
     if (grads && (s = check_all_grads(ctx, grads, where)) != ZERO_OK) return s;
     if (acc && (s = check_owned_acc(ctx, acc, owner_lo, owner_hi, where)) != ZERO_OK) return s;
     zb::StepParams sp = shard_params(ctx, owner_lo, owner_hi, grad_divisor, partial);

@@ -97,6 +97,10 @@ cudaError_t launch_step_from_acc(const StepParams& sp, const RankPtrs& p, cudaSt
 cudaError_t launch_reduce_scatter(int32_t R, int32_t dtype, int64_t S, int64_t lo, int64_t hi,
                                   DevState* st, const RankPtrs& p, cudaStream_t s,
                                   bool accumulate = false, int max_sms = 0, const RsNorm* norm = nullptr);
+// A sharded rank's norm part from norm slots [first, first + count) into
+// out[0] (out[1] = 0) (norm_slots.cu).
+cudaError_t launch_sum_norm_slots(const double* slots, int64_t first, int64_t count, double* out,
+                                  cudaStream_t s);
 // The clipping coefficient from norm slots [first, first + count).
 cudaError_t launch_clip_from_rs_norm(const StepParams& sp, const double* slots, int64_t first, int64_t count,
                                      cudaStream_t s);
@@ -154,6 +158,7 @@ struct zero_ctx_s {
     double* rs_norm = nullptr;
     std::vector<uint8_t> rs_norm_valid;
     std::vector<double> rs_norm_div;
+    std::vector<int64_t> rs_norm_owner;  // owner range of each share: lo << 32 | hi
     double grad_divisor = 1.0;    // the divisor ZERO_RS_NORM unscales by
     zero_trace* trace = nullptr;  // per-call trace while started
 };
@@ -178,7 +183,8 @@ private:
 // Bookkeeping of a reduce-scatter of buckets [first, first + count) (first
 // -1: the whole range), with or without its norm share; returns the launch's
 // norm arguments for the first bucket's slot (capi.cpp).
-zb::RsNorm zb_rs_norm_note(zero_ctx_t* ctx, int64_t first, int64_t count, bool norm);
+zb::RsNorm zb_rs_norm_note(zero_ctx_t* ctx, int64_t first, int64_t count, bool norm, int32_t owner_lo = 0,
+                           int32_t owner_hi = -1);
 // One reduce-scatter launch over buckets [first, first + count), a
 // contiguous flat range (first -1, count 1: every element), flags as for
 // zero_reduce_scatter_bucket_ex, grid capped at max_sms SMs (0: all).

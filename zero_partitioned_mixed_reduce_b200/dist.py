@@ -47,7 +47,7 @@ from .state import HALF, Plan
 class DistributedZero:
     def __init__(self, numels, layer_ids=None, dtype=Z.ZERO_BF16, mode=Z.ZERO_SCALE_NONE,
                  init_scale=1.0, growth_interval=1000, tensor_align=8, bucket_elems=0, group=None,
-                 accumulate=False):
+                 accumulate=False, norm_divisor=None):
         import torch.distributed._symmetric_memory as symm
         self.group = group or dist.group.WORLD
         self.world = dist.get_world_size(self.group)
@@ -91,6 +91,12 @@ class DistributedZero:
         self.gather_handle = Z.StateHandle([dict(master=[None] * R, m=[None] * R, v=[None] * R,
                                                  param=self.param_ptrs[k]) for k in range(sets)])
         self.ctx = Z.zero_ctx_create(self.plan.handle, mode, init_scale, growth_interval)
+        # norm_divisor: the reduce-scatters also take this rank's share of the
+        # clipping norm, unscaled by this gradient divisor, so that a clipped
+        # step_accumulated with the same divisor reads no accumulator first
+        self.norm_divisor = norm_divisor
+        if norm_divisor is not None:
+            Z.zero_ctx_set_grad_divisor(self.ctx, float(norm_divisor))
         self.partial = torch.zeros(2, dtype=torch.float64, device=dev)
         self.norm = torch.zeros(2, dtype=torch.float64, device=dev)
         self.token = torch.zeros(1, dtype=torch.float32, device=dev)
@@ -134,6 +140,12 @@ class DistributedZero:
         Z.zero_step_commit(self.ctx, self.partial, stream)
         self.micro = 0
 
+    def _rs_flags(self):
+        # every micro-batch takes its norm share: the last one leaves the share
+        # of the final accumulator
+        return ((Z.ZERO_RS_ACCUMULATE if self.micro else 0) |
+                (Z.ZERO_RS_NORM if self.norm_divisor is not None else 0))
+
     def reduce_scatter(self, stream=None):
         """After a micro-batch's backward wrote self.grads on every rank: add
         this rank's shard of the reduced gradients to its accumulator (the
@@ -141,7 +153,7 @@ class DistributedZero:
         assert self.acc is not None, "construct with accumulate=True"
         dist.all_reduce(self.token, group=self.group)  # every replica is written
         Z.zero_reduce_scatter_shard(self.ctx, -1, self.grad_ptrs, self.acc_list, self.rank, self.rank + 1,
-                                    Z.ZERO_RS_ACCUMULATE if self.micro else 0, stream)
+                                    self._rs_flags(), stream)
         dist.all_reduce(self.token, group=self.group)  # every peer has read this rank's replica
         self.micro += 1
 
@@ -183,8 +195,7 @@ class DistributedZero:
                 dist.all_reduce(self.comm_token, group=self.group)  # every rank wrote these buckets
                 for b in run:
                     Z.zero_reduce_scatter_shard(self.ctx, b, self.grad_ptrs, self.acc_list, self.rank,
-                                                self.rank + 1, Z.ZERO_RS_ACCUMULATE if self.micro else 0,
-                                                self.comm)
+                                                self.rank + 1, self._rs_flags(), self.comm)
 
     def join(self):
         """End of a micro-batch's backward: every bucket must have been
@@ -202,7 +213,11 @@ class DistributedZero:
         to their count (the mean)."""
         assert self.micro > 0, "no micro-batch was reduce-scattered"
         k = float(self.micro) if grad_divisor is None else grad_divisor
-        if max_grad_norm > 0:
+        if max_grad_norm > 0 and self.norm_divisor is not None and float(self.norm_divisor) == k:
+            # the reduce-scatters' shares: nothing to read again
+            Z.zero_grad_norm_shard(self.ctx, None, None, self.rank, self.rank + 1, self.norm, k, stream)
+            dist.all_reduce(self.norm, group=self.group)
+        elif max_grad_norm > 0:
             self._global_norm(None, self.acc_list, k, stream)
         Z.zero_step_shard_ex(self.ctx, hp, self.handle, None, self.rank, self.rank + 1, self.partial, k,
                              max_grad_norm, self.norm, stream)
