@@ -27,6 +27,8 @@
  *    work surfaces as ZERO_ERR_CUDA on a later call or on zero_sync.
  *  - A context is bound to the CUDA device that was current when it was
  *    created; calls with another device current return ZERO_ERR_INVALID_ARG.
+ *  - No C++ exception crosses this interface: a call that runs out of host
+ *    memory or threads returns ZERO_ERR_OOM.
  *  - Threads: a plan is read-only after zero_plan and may be shared. A
  *    context holds host-side state (the step count bound, the scheduler's
  *    readiness counters, the prefetch ring), so calls on one context must
@@ -734,7 +736,8 @@ zero_status zero_layer_release(zero_ctx_t* ctx, int64_t layer, void* stream);
  * forward pass (it releases no lock and touches no GPU state).
  * All pointers are HOST memory: R pointers each, S elements per shard
  * (pinned memory makes the surrounding copies asynchronous). nthreads <= 0
- * uses every hardware thread (the calling thread is one of them); the result
+ * uses every hardware thread (the calling thread is one of them), and more
+ * than 1024 count as 1024; the result
  * does not depend on nthreads except for the summation order of
  * grad_norm_sq. Work under 65,536 elements runs on the calling thread.
  * Errors: ZERO_ERR_INVALID_ARG.

@@ -330,9 +330,13 @@ zero_status check_cfg(const zero_loss_scale_config* cfg, const char* where) {
     return ZERO_OK;
 }
 
+// at most kMaxThreads: a request for more would only start threads that
+// compete for the same memory bandwidth
+constexpr int kMaxThreads = 1024;
+
 int thread_count(int32_t nthreads) {
     int n = nthreads >= 1 ? nthreads : static_cast<int>(std::thread::hardware_concurrency());
-    return n >= 1 ? n : 1;
+    return n < 1 ? 1 : (n > kMaxThreads ? kMaxThreads : n);
 }
 
 }  // namespace
@@ -340,56 +344,58 @@ int thread_count(int32_t nthreads) {
 extern "C" zero_status zero_cpu_scan(const zero_plan_t* plan, const zero_loss_scale_config* cfg,
                                      const zero_loss_scale_state* in, const zero_step_opts* opts,
                                      const float* const* acc, int32_t nthreads, zero_cpu_decision* out) {
-    if (!plan || !cfg || !in || !acc || !out) return zb_fail(ZERO_ERR_INVALID_ARG, "zero_cpu_scan: NULL argument");
-    zero_step_opts o{1.0, 0.0, 0, 0};
-    if (opts) o = *opts;
-    if (!(o.grad_divisor >= 1.0) || !std::isfinite(o.grad_divisor) || !(o.max_grad_norm >= 0.0) ||
-        !std::isfinite(o.max_grad_norm) || o.flags != 0 || o.reserved != 0)
-        return zb_fail(ZERO_ERR_INVALID_ARG,
-                       "zero_cpu_step: need grad_divisor >= 1, finite max_grad_norm >= 0, no flags");
-    zero_status st = check_cfg(cfg, "zero_cpu_step");
-    if (st != ZERO_OK) return st;
-    const float scale = cfg->mode == ZERO_SCALE_NONE ? 1.0f : in->scale;
-    if (!(scale > 0.0f) || !std::isfinite(scale) || in->t < 0)
-        return zb_fail(ZERO_ERR_INVALID_ARG, "zero_cpu_step: need a finite scale > 0 and t >= 0");
-    const int R = plan->R;
-    for (int r = 0; r < R; ++r)
-        if (!acc[r]) return zb_fail(ZERO_ERR_INVALID_ARG, "zero_cpu_step: NULL rank pointer");
-    const int nt = thread_count(nthreads);
-    const int64_t S = plan->S;
-    const float inv =
-        static_cast<float>(1.0 / ((static_cast<double>(R) * o.grad_divisor) * static_cast<double>(scale)));
-    // overflow and squared norm; each thread sums its pieces in order, and
-    // the per-thread partials are summed in thread order
-    std::vector<double> part(static_cast<size_t>(nt), 0.0);
-    std::vector<int> bad(static_cast<size_t>(nt), 0);
-    parallel_shards(R, 0, S, nt, [&](int t, int r, int64_t a, int64_t b) {
-        double pn = 0.0;
-        int pb = 0;
-        scan_range(acc[r] + a, inv, b - a, &pn, &pb);
-        part[t] += pn;
-        bad[t] |= pb;
+    return zb_guarded("zero_cpu_scan", [&]() -> zero_status {
+        if (!plan || !cfg || !in || !acc || !out) return zb_fail(ZERO_ERR_INVALID_ARG, "zero_cpu_scan: NULL argument");
+        zero_step_opts o{1.0, 0.0, 0, 0};
+        if (opts) o = *opts;
+        if (!(o.grad_divisor >= 1.0) || !std::isfinite(o.grad_divisor) || !(o.max_grad_norm >= 0.0) ||
+            !std::isfinite(o.max_grad_norm) || o.flags != 0 || o.reserved != 0)
+            return zb_fail(ZERO_ERR_INVALID_ARG,
+                           "zero_cpu_step: need grad_divisor >= 1, finite max_grad_norm >= 0, no flags");
+        zero_status st = check_cfg(cfg, "zero_cpu_step");
+        if (st != ZERO_OK) return st;
+        const float scale = cfg->mode == ZERO_SCALE_NONE ? 1.0f : in->scale;
+        if (!(scale > 0.0f) || !std::isfinite(scale) || in->t < 0)
+            return zb_fail(ZERO_ERR_INVALID_ARG, "zero_cpu_step: need a finite scale > 0 and t >= 0");
+        const int R = plan->R;
+        for (int r = 0; r < R; ++r)
+            if (!acc[r]) return zb_fail(ZERO_ERR_INVALID_ARG, "zero_cpu_step: NULL rank pointer");
+        const int nt = thread_count(nthreads);
+        const int64_t S = plan->S;
+        const float inv =
+            static_cast<float>(1.0 / ((static_cast<double>(R) * o.grad_divisor) * static_cast<double>(scale)));
+        // overflow and squared norm; each thread sums its pieces in order, and
+        // the per-thread partials are summed in thread order
+        std::vector<double> part(static_cast<size_t>(nt), 0.0);
+        std::vector<int> bad(static_cast<size_t>(nt), 0);
+        parallel_shards(R, 0, S, nt, [&](int t, int r, int64_t a, int64_t b) {
+            double pn = 0.0;
+            int pb = 0;
+            scan_range(acc[r] + a, inv, b - a, &pn, &pb);
+            part[t] += pn;
+            bad[t] |= pb;
+        });
+        double nrm = 0.0;
+        int overflow = 0;
+        for (size_t i = 0; i < part.size(); ++i) {
+            nrm += part[i];
+            overflow |= bad[i];
+        }
+        zero_cpu_decision d;
+        d.grad_norm_sq = nrm;
+        d.inv = inv;
+        d.clip = 1.0f;
+        if (o.max_grad_norm > 0.0) {
+            const double cd = o.max_grad_norm / (std::sqrt(nrm) + 1e-6);
+            d.clip = static_cast<float>(cd < 1.0 ? cd : 1.0);
+        }
+        d.overflow = overflow;
+        d.skip = (cfg->mode == ZERO_SCALE_DYNAMIC && overflow) ? 1 : 0;
+        d.clipping = o.max_grad_norm > 0.0 ? 1 : 0;
+        d.reserved = 0;
+        *out = d;
+        return ZERO_OK;
     });
-    double nrm = 0.0;
-    int overflow = 0;
-    for (size_t i = 0; i < part.size(); ++i) {
-        nrm += part[i];
-        overflow |= bad[i];
-    }
-    zero_cpu_decision d;
-    d.grad_norm_sq = nrm;
-    d.inv = inv;
-    d.clip = 1.0f;
-    if (o.max_grad_norm > 0.0) {
-        const double cd = o.max_grad_norm / (std::sqrt(nrm) + 1e-6);
-        d.clip = static_cast<float>(cd < 1.0 ? cd : 1.0);
-    }
-    d.overflow = overflow;
-    d.skip = (cfg->mode == ZERO_SCALE_DYNAMIC && overflow) ? 1 : 0;
-    d.clipping = o.max_grad_norm > 0.0 ? 1 : 0;
-    d.reserved = 0;
-    *out = d;
-    return ZERO_OK;
 }
 
 extern "C" zero_status zero_cpu_update(const zero_plan_t* plan, const zero_loss_scale_state* in,
@@ -397,85 +403,91 @@ extern "C" zero_status zero_cpu_update(const zero_plan_t* plan, const zero_loss_
                                        const float* const* acc, float* const* master, float* const* m,
                                        float* const* v, void* const* param, int64_t lo, int64_t hi,
                                        int32_t nthreads) {
-    if (!plan || !in || !hp || !d || !acc || !master || !m || !v || !param)
-        return zb_fail(ZERO_ERR_INVALID_ARG, "zero_cpu_update: NULL argument");
-    if (!(hp->lr >= 0.0) || !(hp->beta1 >= 0.0 && hp->beta1 < 1.0) || !(hp->beta2 >= 0.0 && hp->beta2 < 1.0) ||
-        !(hp->eps > 0.0) || !(hp->weight_decay >= 0.0))
-        return zb_fail(ZERO_ERR_INVALID_ARG, "zero_cpu_step: bad hyper-parameters");
-    const int64_t S = plan->S;
-    if (lo < 0 || lo > hi || hi > S)
-        return zb_fail(ZERO_ERR_RANGE, "zero_cpu_update: need 0 <= lo <= hi <= S");
-    if (in->t < 0) return zb_fail(ZERO_ERR_INVALID_ARG, "zero_cpu_update: need t >= 0");
-    const int R = plan->R;
-    for (int r = 0; r < R; ++r)
-        if (!acc[r] || !master[r] || !m[r] || !v[r] || !param[r])
-            return zb_fail(ZERO_ERR_INVALID_ARG, "zero_cpu_step: NULL rank pointer");
-    if (d->skip || lo == hi) return ZERO_OK;  // a skipped step writes nothing
-    const int nt = thread_count(nthreads);
-    Coeffs c;
-    const double t1 = static_cast<double>(in->t + 1);
-    c.inv = d->inv;
-    c.dec = static_cast<float>(1.0 - hp->lr * hp->weight_decay);
-    c.b1f = static_cast<float>(hp->beta1);
-    c.omb1 = static_cast<float>(1.0 - hp->beta1);
-    c.b2f = static_cast<float>(hp->beta2);
-    c.omb2 = static_cast<float>(1.0 - hp->beta2);
-    c.epsf = static_cast<float>(hp->eps);
-    c.ss = static_cast<float>(hp->lr / (1.0 - std::pow(hp->beta1, t1)));
-    c.bc2s = static_cast<float>(std::sqrt(1.0 - std::pow(hp->beta2, t1)));
-    c.clip = d->clip;
-    const bool fp16 = plan->dtype == ZERO_FP16, clip = d->clipping != 0;
-    parallel_shards(R, lo, hi, nt, [&](int, int r, int64_t a, int64_t b) {
-        const int64_t n = b - a;
-        uint16_t* out = static_cast<uint16_t*>(param[r]) + a;
-        if (fp16 && clip) update_range<true, true>(c, acc[r] + a, master[r] + a, m[r] + a, v[r] + a, out, n);
-        else if (fp16) update_range<true, false>(c, acc[r] + a, master[r] + a, m[r] + a, v[r] + a, out, n);
-        else if (clip) update_range<false, true>(c, acc[r] + a, master[r] + a, m[r] + a, v[r] + a, out, n);
-        else update_range<false, false>(c, acc[r] + a, master[r] + a, m[r] + a, v[r] + a, out, n);
+    return zb_guarded("zero_cpu_update", [&]() -> zero_status {
+        if (!plan || !in || !hp || !d || !acc || !master || !m || !v || !param)
+            return zb_fail(ZERO_ERR_INVALID_ARG, "zero_cpu_update: NULL argument");
+        if (!(hp->lr >= 0.0) || !(hp->beta1 >= 0.0 && hp->beta1 < 1.0) || !(hp->beta2 >= 0.0 && hp->beta2 < 1.0) ||
+            !(hp->eps > 0.0) || !(hp->weight_decay >= 0.0))
+            return zb_fail(ZERO_ERR_INVALID_ARG, "zero_cpu_step: bad hyper-parameters");
+        const int64_t S = plan->S;
+        if (lo < 0 || lo > hi || hi > S)
+            return zb_fail(ZERO_ERR_RANGE, "zero_cpu_update: need 0 <= lo <= hi <= S");
+        if (in->t < 0) return zb_fail(ZERO_ERR_INVALID_ARG, "zero_cpu_update: need t >= 0");
+        const int R = plan->R;
+        for (int r = 0; r < R; ++r)
+            if (!acc[r] || !master[r] || !m[r] || !v[r] || !param[r])
+                return zb_fail(ZERO_ERR_INVALID_ARG, "zero_cpu_step: NULL rank pointer");
+        if (d->skip || lo == hi) return ZERO_OK;  // a skipped step writes nothing
+        const int nt = thread_count(nthreads);
+        Coeffs c;
+        const double t1 = static_cast<double>(in->t + 1);
+        c.inv = d->inv;
+        c.dec = static_cast<float>(1.0 - hp->lr * hp->weight_decay);
+        c.b1f = static_cast<float>(hp->beta1);
+        c.omb1 = static_cast<float>(1.0 - hp->beta1);
+        c.b2f = static_cast<float>(hp->beta2);
+        c.omb2 = static_cast<float>(1.0 - hp->beta2);
+        c.epsf = static_cast<float>(hp->eps);
+        c.ss = static_cast<float>(hp->lr / (1.0 - std::pow(hp->beta1, t1)));
+        c.bc2s = static_cast<float>(std::sqrt(1.0 - std::pow(hp->beta2, t1)));
+        c.clip = d->clip;
+        const bool fp16 = plan->dtype == ZERO_FP16, clip = d->clipping != 0;
+        parallel_shards(R, lo, hi, nt, [&](int, int r, int64_t a, int64_t b) {
+            const int64_t n = b - a;
+            uint16_t* out = static_cast<uint16_t*>(param[r]) + a;
+            if (fp16 && clip) update_range<true, true>(c, acc[r] + a, master[r] + a, m[r] + a, v[r] + a, out, n);
+            else if (fp16) update_range<true, false>(c, acc[r] + a, master[r] + a, m[r] + a, v[r] + a, out, n);
+            else if (clip) update_range<false, true>(c, acc[r] + a, master[r] + a, m[r] + a, v[r] + a, out, n);
+            else update_range<false, false>(c, acc[r] + a, master[r] + a, m[r] + a, v[r] + a, out, n);
+        });
+        return ZERO_OK;
     });
-    return ZERO_OK;
 }
 
 extern "C" zero_status zero_cpu_commit(const zero_loss_scale_config* cfg, zero_loss_scale_state* inout,
                                        const zero_cpu_decision* d) {
-    if (!cfg || !inout || !d) return zb_fail(ZERO_ERR_INVALID_ARG, "zero_cpu_commit: NULL argument");
-    zero_status st = check_cfg(cfg, "zero_cpu_commit");
-    if (st != ZERO_OK) return st;
-    // the loss-scale state machine, the same rules as the device step
-    int skipped = 0;
-    if (cfg->mode == ZERO_SCALE_DYNAMIC) {
-        if (d->overflow) {
-            const float s = inout->scale * cfg->backoff_factor;
-            inout->scale = (s < cfg->min_scale) ? cfg->min_scale : s;
-            inout->good = 0;
-            skipped = 1;
+    return zb_guarded("zero_cpu_commit", [&]() -> zero_status {
+        if (!cfg || !inout || !d) return zb_fail(ZERO_ERR_INVALID_ARG, "zero_cpu_commit: NULL argument");
+        zero_status st = check_cfg(cfg, "zero_cpu_commit");
+        if (st != ZERO_OK) return st;
+        // the loss-scale state machine, the same rules as the device step
+        int skipped = 0;
+        if (cfg->mode == ZERO_SCALE_DYNAMIC) {
+            if (d->overflow) {
+                const float s = inout->scale * cfg->backoff_factor;
+                inout->scale = (s < cfg->min_scale) ? cfg->min_scale : s;
+                inout->good = 0;
+                skipped = 1;
+            } else {
+                inout->t += 1;
+                inout->good += 1;
+                if (inout->good >= cfg->growth_interval) {
+                    inout->scale = inout->scale * cfg->growth_factor;
+                    inout->good = 0;
+                }
+            }
         } else {
             inout->t += 1;
-            inout->good += 1;
-            if (inout->good >= cfg->growth_interval) {
-                inout->scale = inout->scale * cfg->growth_factor;
-                inout->good = 0;
-            }
         }
-    } else {
-        inout->t += 1;
-    }
-    inout->last_overflow = d->overflow;
-    inout->last_skipped = skipped;
-    inout->grad_norm_sq = d->grad_norm_sq;
-    return ZERO_OK;
+        inout->last_overflow = d->overflow;
+        inout->last_skipped = skipped;
+        inout->grad_norm_sq = d->grad_norm_sq;
+        return ZERO_OK;
+    });
 }
 
 extern "C" zero_status zero_cpu_step(const zero_plan_t* plan, const zero_loss_scale_config* cfg,
                                      zero_loss_scale_state* inout, const zero_adamw* hp,
                                      const zero_step_opts* opts, const float* const* acc, float* const* master,
                                      float* const* m, float* const* v, void* const* param, int32_t nthreads) {
-    if (!plan || !cfg || !inout || !hp || !acc || !master || !m || !v || !param)
-        return zb_fail(ZERO_ERR_INVALID_ARG, "zero_cpu_step: NULL argument");
-    zero_cpu_decision d;
-    zero_status st = zero_cpu_scan(plan, cfg, inout, opts, acc, nthreads, &d);
-    if (st == ZERO_OK)
-        st = zero_cpu_update(plan, inout, hp, &d, acc, master, m, v, param, 0, plan->S, nthreads);
-    if (st == ZERO_OK) st = zero_cpu_commit(cfg, inout, &d);
-    return st;
+    return zb_guarded("zero_cpu_step", [&]() -> zero_status {
+        if (!plan || !cfg || !inout || !hp || !acc || !master || !m || !v || !param)
+            return zb_fail(ZERO_ERR_INVALID_ARG, "zero_cpu_step: NULL argument");
+        zero_cpu_decision d;
+        zero_status st = zero_cpu_scan(plan, cfg, inout, opts, acc, nthreads, &d);
+        if (st == ZERO_OK)
+            st = zero_cpu_update(plan, inout, hp, &d, acc, master, m, v, param, 0, plan->S, nthreads);
+        if (st == ZERO_OK) st = zero_cpu_commit(cfg, inout, &d);
+        return st;
+    });
 }

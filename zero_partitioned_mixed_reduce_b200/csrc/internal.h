@@ -194,4 +194,17 @@ cudaError_t zb_rs_launch(zero_ctx_t* ctx, int64_t first, int64_t count, const zb
 void zb_sched_destroy(zero_ctx_t* ctx);
 
 // Set the calling thread's last error message; returns `code`.
-zero_status zb_fail(zero_status code, const std::string& msg);
+zero_status zb_fail(zero_status code, const std::string& msg) noexcept;
+
+// No exception crosses the C ABI: every entry point runs its body through
+// zb_guarded, which turns an exception in flight (host memory or threads
+// exhausted) into ZERO_ERR_OOM with the exception's message.
+zero_status zb_exception(const char* where) noexcept;
+template <typename F>
+zero_status zb_guarded(const char* where, F&& body) noexcept {
+    try {
+        return body();
+    } catch (...) {
+        return zb_exception(where);
+    }
+}

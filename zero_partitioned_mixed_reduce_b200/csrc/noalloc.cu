@@ -161,125 +161,127 @@ extern "C" zero_status zero_step_noalloc(const zero_plan_t* plan, const zero_los
                                          const void* const* grads, float* const* master,
                                          float* const* m, float* const* v, void* const* param,
                                          void* stream) {
-    using namespace zb;
-    if (!plan || !cfg || !inout || !hp)
-        return zb_fail(ZERO_ERR_INVALID_ARG, "zero_step_noalloc: NULL plan, cfg, state or hp");
-    if (plan->T > kNoallocMaxElems)
-        return zb_fail(ZERO_ERR_RANGE,
-                       "zero_step_noalloc: the padded model has " + std::to_string(plan->T) +
-                           " elements, more than the static scratch holds (" +
-                           std::to_string(kNoallocMaxElems) + "); use zero_step with a context");
-    if (cfg->mode < ZERO_SCALE_NONE || cfg->mode > ZERO_SCALE_DYNAMIC ||
-        (cfg->mode == ZERO_SCALE_DYNAMIC &&
-         (cfg->growth_interval < 1 || !(cfg->growth_factor > 1.0f) ||
-          !(cfg->backoff_factor > 0.0f && cfg->backoff_factor < 1.0f) || !(cfg->min_scale > 0.0f))))
-        return zb_fail(ZERO_ERR_INVALID_ARG, "zero_step_noalloc: bad loss-scale config");
-    const float scale = cfg->mode == ZERO_SCALE_NONE ? 1.0f : inout->scale;
-    if (!(scale > 0.0f) || !std::isfinite(scale) || inout->t < 0 || inout->good < 0 || inout->cur != 0)
-        return zb_fail(ZERO_ERR_INVALID_ARG,
-                       "zero_step_noalloc: need finite scale > 0, t >= 0, good >= 0 and cur == 0");
-    if (!(hp->lr >= 0.0) || !(hp->beta1 >= 0.0 && hp->beta1 < 1.0) ||
-        !(hp->beta2 >= 0.0 && hp->beta2 < 1.0) || !(hp->eps > 0.0) || !(hp->weight_decay >= 0.0) ||
-        !std::isfinite(hp->lr) || !std::isfinite(hp->weight_decay))
-        return zb_fail(ZERO_ERR_INVALID_ARG,
-                       "zero_step_noalloc: need lr >= 0, 0 <= beta < 1, eps > 0, weight_decay >= 0");
-    const int R = plan->R;
-    zero_status s;
-    if ((s = check_list(grads, R, 16, "grads")) != ZERO_OK) return s;
-    if ((s = check_list(master, R, 32, "master")) != ZERO_OK) return s;
-    if ((s = check_list(m, R, 32, "m")) != ZERO_OK) return s;
-    if ((s = check_list(v, R, 32, "v")) != ZERO_OK) return s;
-    if ((s = check_list(param, R, 16, "param")) != ZERO_OK) return s;
+    return zb_guarded("zero_step_noalloc", [&]() -> zero_status {
+        using namespace zb;
+        if (!plan || !cfg || !inout || !hp)
+            return zb_fail(ZERO_ERR_INVALID_ARG, "zero_step_noalloc: NULL plan, cfg, state or hp");
+        if (plan->T > kNoallocMaxElems)
+            return zb_fail(ZERO_ERR_RANGE,
+                           "zero_step_noalloc: the padded model has " + std::to_string(plan->T) +
+                               " elements, more than the static scratch holds (" +
+                               std::to_string(kNoallocMaxElems) + "); use zero_step with a context");
+        if (cfg->mode < ZERO_SCALE_NONE || cfg->mode > ZERO_SCALE_DYNAMIC ||
+            (cfg->mode == ZERO_SCALE_DYNAMIC &&
+             (cfg->growth_interval < 1 || !(cfg->growth_factor > 1.0f) ||
+              !(cfg->backoff_factor > 0.0f && cfg->backoff_factor < 1.0f) || !(cfg->min_scale > 0.0f))))
+            return zb_fail(ZERO_ERR_INVALID_ARG, "zero_step_noalloc: bad loss-scale config");
+        const float scale = cfg->mode == ZERO_SCALE_NONE ? 1.0f : inout->scale;
+        if (!(scale > 0.0f) || !std::isfinite(scale) || inout->t < 0 || inout->good < 0 || inout->cur != 0)
+            return zb_fail(ZERO_ERR_INVALID_ARG,
+                           "zero_step_noalloc: need finite scale > 0, t >= 0, good >= 0 and cur == 0");
+        if (!(hp->lr >= 0.0) || !(hp->beta1 >= 0.0 && hp->beta1 < 1.0) ||
+            !(hp->beta2 >= 0.0 && hp->beta2 < 1.0) || !(hp->eps > 0.0) || !(hp->weight_decay >= 0.0) ||
+            !std::isfinite(hp->lr) || !std::isfinite(hp->weight_decay))
+            return zb_fail(ZERO_ERR_INVALID_ARG,
+                           "zero_step_noalloc: need lr >= 0, 0 <= beta < 1, eps > 0, weight_decay >= 0");
+        const int R = plan->R;
+        zero_status s;
+        if ((s = check_list(grads, R, 16, "grads")) != ZERO_OK) return s;
+        if ((s = check_list(master, R, 32, "master")) != ZERO_OK) return s;
+        if ((s = check_list(m, R, 32, "m")) != ZERO_OK) return s;
+        if ((s = check_list(v, R, 32, "v")) != ZERO_OK) return s;
+        if ((s = check_list(param, R, 16, "param")) != ZERO_OK) return s;
 
-    unsigned char* base = nullptr;
-    if ((s = scratch_for_current_device(&base)) != ZERO_OK) return s;
-    float* acc = reinterpret_cast<float*>(base);
-    double* partials = reinterpret_cast<double*>(base + kAccBytes);
-    DevState* ctrl = reinterpret_cast<DevState*>(base + kAccBytes + kPartialBytes);
-    cudaStream_t cs = static_cast<cudaStream_t>(stream);
+        unsigned char* base = nullptr;
+        if ((s = scratch_for_current_device(&base)) != ZERO_OK) return s;
+        float* acc = reinterpret_cast<float*>(base);
+        double* partials = reinterpret_cast<double*>(base + kAccBytes);
+        DevState* ctrl = reinterpret_cast<DevState*>(base + kAccBytes + kPartialBytes);
+        cudaStream_t cs = static_cast<cudaStream_t>(stream);
 
-    // the control word must start at zero: no overflow, no finished blocks
-    cudaError_t e = cudaMemsetAsync(ctrl, 0, sizeof(DevState), cs);
-    if (e != cudaSuccess) return zb_fail(ZERO_ERR_CUDA, std::string("zero_step_noalloc: ") + cudaGetErrorString(e));
+        // the control word must start at zero: no overflow, no finished blocks
+        cudaError_t e = cudaMemsetAsync(ctrl, 0, sizeof(DevState), cs);
+        if (e != cudaSuccess) return zb_fail(ZERO_ERR_CUDA, std::string("zero_step_noalloc: ") + cudaGetErrorString(e));
 
-    RankPtrs p;
-    for (int r = 0; r < R; ++r) {
-        p.g[r] = grads[r];
-        p.acc[r] = acc + static_cast<size_t>(r) * plan->S;
-    }
-    e = launch_reduce_scatter(R, plan->dtype, plan->S, 0, plan->T, ctrl, p, cs);
-    if (e != cudaSuccess) return zb_fail(ZERO_ERR_CUDA, std::string("zero_step_noalloc: ") + cudaGetErrorString(e));
+        RankPtrs p;
+        for (int r = 0; r < R; ++r) {
+            p.g[r] = grads[r];
+            p.acc[r] = acc + static_cast<size_t>(r) * plan->S;
+        }
+        e = launch_reduce_scatter(R, plan->dtype, plan->S, 0, plan->T, ctrl, p, cs);
+        if (e != cudaSuccess) return zb_fail(ZERO_ERR_CUDA, std::string("zero_step_noalloc: ") + cudaGetErrorString(e));
 
-    // coefficients of step t+1, formed on the host in double, rounded once
-    NoallocArgs a;
-    const double t1 = static_cast<double>(inout->t + 1);
-    a.c.inv = static_cast<float>(1.0 / (static_cast<double>(R) * static_cast<double>(scale)));
-    a.c.dec = static_cast<float>(1.0 - hp->lr * hp->weight_decay);
-    a.c.b1f = static_cast<float>(hp->beta1);
-    a.c.omb1 = static_cast<float>(1.0 - hp->beta1);
-    a.c.b2f = static_cast<float>(hp->beta2);
-    a.c.omb2 = static_cast<float>(1.0 - hp->beta2);
-    a.c.epsf = static_cast<float>(hp->eps);
-    a.c.ss = static_cast<float>(hp->lr / (1.0 - std::pow(hp->beta1, t1)));
-    a.c.bc2s = static_cast<float>(std::sqrt(1.0 - std::pow(hp->beta2, t1)));
-    a.c.clip = 1.0f;
-    a.dynamic = cfg->mode == ZERO_SCALE_DYNAMIC;
-    a.S8 = static_cast<uint32_t>(plan->S / 8);
-    a.T8 = static_cast<uint32_t>(plan->T / 8);
-    a.ctrl = ctrl;
-    a.partials = partials;
-    for (int r = 0; r < R; ++r) {
-        a.acc[r] = p.acc[r];
-        a.master[r] = master[r];
-        a.m[r] = m[r];
-        a.v[r] = v[r];
-        a.param[r] = static_cast<uint4*>(param[r]);
-    }
-    int sms = 0, dev = 0, per_sm = 0;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    if (plan->dtype == ZERO_FP16)
-        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, noalloc_step_kernel<Fp16>, kThreads, 0);
-    else
-        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, noalloc_step_kernel<Bf16>, kThreads, 0);
-    int64_t grid = static_cast<int64_t>(sms) * (per_sm > 0 ? per_sm : 1);
-    const int64_t need = (static_cast<int64_t>(a.T8) + kThreads - 1) / kThreads;
-    if (grid > need) grid = need;
-    if (grid > kNoallocMaxBlocks) grid = kNoallocMaxBlocks;
-    if (grid < 1) grid = 1;
-    if (plan->dtype == ZERO_FP16)
-        noalloc_step_kernel<Fp16><<<static_cast<unsigned>(grid), kThreads, 0, cs>>>(a);
-    else
-        noalloc_step_kernel<Bf16><<<static_cast<unsigned>(grid), kThreads, 0, cs>>>(a);
-    e = cudaGetLastError();
-    if (e != cudaSuccess) return zb_fail(ZERO_ERR_CUDA, std::string("zero_step_noalloc: ") + cudaGetErrorString(e));
+        // coefficients of step t+1, formed on the host in double, rounded once
+        NoallocArgs a;
+        const double t1 = static_cast<double>(inout->t + 1);
+        a.c.inv = static_cast<float>(1.0 / (static_cast<double>(R) * static_cast<double>(scale)));
+        a.c.dec = static_cast<float>(1.0 - hp->lr * hp->weight_decay);
+        a.c.b1f = static_cast<float>(hp->beta1);
+        a.c.omb1 = static_cast<float>(1.0 - hp->beta1);
+        a.c.b2f = static_cast<float>(hp->beta2);
+        a.c.omb2 = static_cast<float>(1.0 - hp->beta2);
+        a.c.epsf = static_cast<float>(hp->eps);
+        a.c.ss = static_cast<float>(hp->lr / (1.0 - std::pow(hp->beta1, t1)));
+        a.c.bc2s = static_cast<float>(std::sqrt(1.0 - std::pow(hp->beta2, t1)));
+        a.c.clip = 1.0f;
+        a.dynamic = cfg->mode == ZERO_SCALE_DYNAMIC;
+        a.S8 = static_cast<uint32_t>(plan->S / 8);
+        a.T8 = static_cast<uint32_t>(plan->T / 8);
+        a.ctrl = ctrl;
+        a.partials = partials;
+        for (int r = 0; r < R; ++r) {
+            a.acc[r] = p.acc[r];
+            a.master[r] = master[r];
+            a.m[r] = m[r];
+            a.v[r] = v[r];
+            a.param[r] = static_cast<uint4*>(param[r]);
+        }
+        int sms = 0, dev = 0, per_sm = 0;
+        cudaGetDevice(&dev);
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+        if (plan->dtype == ZERO_FP16)
+            cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, noalloc_step_kernel<Fp16>, kThreads, 0);
+        else
+            cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, noalloc_step_kernel<Bf16>, kThreads, 0);
+        int64_t grid = static_cast<int64_t>(sms) * (per_sm > 0 ? per_sm : 1);
+        const int64_t need = (static_cast<int64_t>(a.T8) + kThreads - 1) / kThreads;
+        if (grid > need) grid = need;
+        if (grid > kNoallocMaxBlocks) grid = kNoallocMaxBlocks;
+        if (grid < 1) grid = 1;
+        if (plan->dtype == ZERO_FP16)
+            noalloc_step_kernel<Fp16><<<static_cast<unsigned>(grid), kThreads, 0, cs>>>(a);
+        else
+            noalloc_step_kernel<Bf16><<<static_cast<unsigned>(grid), kThreads, 0, cs>>>(a);
+        e = cudaGetLastError();
+        if (e != cudaSuccess) return zb_fail(ZERO_ERR_CUDA, std::string("zero_step_noalloc: ") + cudaGetErrorString(e));
 
-    // bring the step's result back and run the loss-scale update on the host
-    DevState out{};
-    e = cudaMemcpyAsync(&out, ctrl, sizeof(DevState), cudaMemcpyDeviceToHost, cs);
-    if (e == cudaSuccess) e = cudaStreamSynchronize(cs);
-    if (e != cudaSuccess) return zb_fail(ZERO_ERR_CUDA, std::string("zero_step_noalloc: ") + cudaGetErrorString(e));
-    const int overflow = out.last_overflow != 0;
-    int skipped = 0;
-    if (cfg->mode == ZERO_SCALE_DYNAMIC) {
-        if (overflow) {
-            const float sc = inout->scale * cfg->backoff_factor;
-            inout->scale = (sc < cfg->min_scale) ? cfg->min_scale : sc;
-            inout->good = 0;
-            skipped = 1;
+        // bring the step's result back and run the loss-scale update on the host
+        DevState out{};
+        e = cudaMemcpyAsync(&out, ctrl, sizeof(DevState), cudaMemcpyDeviceToHost, cs);
+        if (e == cudaSuccess) e = cudaStreamSynchronize(cs);
+        if (e != cudaSuccess) return zb_fail(ZERO_ERR_CUDA, std::string("zero_step_noalloc: ") + cudaGetErrorString(e));
+        const int overflow = out.last_overflow != 0;
+        int skipped = 0;
+        if (cfg->mode == ZERO_SCALE_DYNAMIC) {
+            if (overflow) {
+                const float sc = inout->scale * cfg->backoff_factor;
+                inout->scale = (sc < cfg->min_scale) ? cfg->min_scale : sc;
+                inout->good = 0;
+                skipped = 1;
+            } else {
+                inout->t += 1;
+                inout->good += 1;
+                if (inout->good >= cfg->growth_interval) {
+                    inout->scale = inout->scale * cfg->growth_factor;
+                    inout->good = 0;
+                }
+            }
         } else {
             inout->t += 1;
-            inout->good += 1;
-            if (inout->good >= cfg->growth_interval) {
-                inout->scale = inout->scale * cfg->growth_factor;
-                inout->good = 0;
-            }
         }
-    } else {
-        inout->t += 1;
-    }
-    inout->last_overflow = overflow;
-    inout->last_skipped = skipped;
-    inout->grad_norm_sq = out.grad_norm_sq;
-    return ZERO_OK;
+        inout->last_overflow = overflow;
+        inout->last_skipped = skipped;
+        inout->grad_norm_sq = out.grad_norm_sq;
+        return ZERO_OK;
+    });
 }

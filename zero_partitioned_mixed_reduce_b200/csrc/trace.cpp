@@ -5,6 +5,7 @@
 // test. Calls made while their stream is being captured into a CUDA graph are
 // not traced (a graph replays without the host, so there is nothing to pair
 // the events with).
+#include <memory>
 #include <string>
 #include <vector>
 
@@ -72,69 +73,74 @@ ZbTraceScope::~ZbTraceScope() {
 }
 
 extern "C" zero_status zero_trace_start(zero_ctx_t* ctx, int32_t capacity) {
-    if (!ctx) return zb_fail(ZERO_ERR_INVALID_ARG, "zero_trace_start: ctx is NULL");
-    if (capacity < 1 || capacity > (1 << 20))
-        return zb_fail(ZERO_ERR_INVALID_ARG, "zero_trace_start: need 1 <= capacity <= 2^20");
-    int dev = -1;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev != ctx->device) {
-        cudaGetLastError();
-        return zb_fail(ZERO_ERR_INVALID_ARG, "zero_trace_start: context belongs to another device");
-    }
-    zb_trace_destroy(ctx);
-    zero_trace* t = new zero_trace();
-    t->capacity = capacity;
-    t->ev.assign(2 * static_cast<size_t>(capacity), nullptr);
-    t->rec.reserve(capacity);
-    for (cudaEvent_t& e : t->ev) {
-        cudaError_t err = cudaEventCreate(&e);
-        if (err != cudaSuccess) {
+    return zb_guarded("zero_trace_start", [&]() -> zero_status {
+        if (!ctx) return zb_fail(ZERO_ERR_INVALID_ARG, "zero_trace_start: ctx is NULL");
+        if (capacity < 1 || capacity > (1 << 20))
+            return zb_fail(ZERO_ERR_INVALID_ARG, "zero_trace_start: need 1 <= capacity <= 2^20");
+        int dev = -1;
+        if (cudaGetDevice(&dev) != cudaSuccess || dev != ctx->device) {
             cudaGetLastError();
-            free_trace(t);
-            return zb_fail(ZERO_ERR_CUDA, std::string("zero_trace_start: ") + cudaGetErrorString(err));
+            return zb_fail(ZERO_ERR_INVALID_ARG, "zero_trace_start: context belongs to another device");
         }
-    }
-    ctx->trace = t;
-    return ZERO_OK;
+        zb_trace_destroy(ctx);
+        std::unique_ptr<zero_trace, void (*)(zero_trace*)> t(new zero_trace(), free_trace);
+        t->capacity = capacity;
+        t->ev.assign(2 * static_cast<size_t>(capacity), nullptr);
+        t->rec.reserve(capacity);
+        for (cudaEvent_t& e : t->ev) {
+            cudaError_t err = cudaEventCreate(&e);
+            if (err != cudaSuccess) {
+                cudaGetLastError();
+                return zb_fail(ZERO_ERR_CUDA, std::string("zero_trace_start: ") + cudaGetErrorString(err));
+            }
+        }
+        ctx->trace = t.release();
+        return ZERO_OK;
+    });
 }
 
 extern "C" zero_status zero_trace_read(zero_ctx_t* ctx, zero_trace_record* out, int32_t max, int32_t* count,
                                        int64_t* dropped) {
-    if (!ctx || !count || (max > 0 && !out))
-        return zb_fail(ZERO_ERR_INVALID_ARG, "zero_trace_read: NULL argument");
-    zero_trace* t = ctx->trace;
-    if (!t) return zb_fail(ZERO_ERR_STATE, "zero_trace_read: tracing is not started");
-    const int32_t n = static_cast<int32_t>(t->rec.size());
-    if (max < n)
-        return zb_fail(ZERO_ERR_RANGE, "zero_trace_read: " + std::to_string(n) + " records, room for " +
-                                           std::to_string(max));
-    for (int32_t i = 0; i < n; ++i) {
-        zero_trace_record r = t->rec[i];
-        if (r.call != 0) {
-            cudaError_t e = cudaEventSynchronize(t->ev[2 * i + 1]);
-            float ms = -1.0f;
-            if (e == cudaSuccess) e = cudaEventElapsedTime(&ms, t->ev[2 * i], t->ev[2 * i + 1]);
-            if (e != cudaSuccess) {
-                cudaGetLastError();
-                return zb_fail(ZERO_ERR_CUDA, std::string("zero_trace_read: ") + cudaGetErrorString(e));
+    return zb_guarded("zero_trace_read", [&]() -> zero_status {
+        if (!ctx || !count || (max > 0 && !out))
+            return zb_fail(ZERO_ERR_INVALID_ARG, "zero_trace_read: NULL argument");
+        zero_trace* t = ctx->trace;
+        if (!t) return zb_fail(ZERO_ERR_STATE, "zero_trace_read: tracing is not started");
+        const int32_t n = static_cast<int32_t>(t->rec.size());
+        if (max < n)
+            return zb_fail(ZERO_ERR_RANGE, "zero_trace_read: " + std::to_string(n) + " records, room for " +
+                                               std::to_string(max));
+        for (int32_t i = 0; i < n; ++i) {
+            zero_trace_record r = t->rec[i];
+            if (r.call != 0) {
+                cudaError_t e = cudaEventSynchronize(t->ev[2 * i + 1]);
+                float ms = -1.0f;
+                if (e == cudaSuccess) e = cudaEventElapsedTime(&ms, t->ev[2 * i], t->ev[2 * i + 1]);
+                if (e != cudaSuccess) {
+                    cudaGetLastError();
+                    return zb_fail(ZERO_ERR_CUDA, std::string("zero_trace_read: ") + cudaGetErrorString(e));
+                }
+                r.ms = ms;
             }
-            r.ms = ms;
+            out[i] = r;
         }
-        out[i] = r;
-    }
-    *count = n;
-    if (dropped) *dropped = t->dropped;
-    t->rec.clear();
-    t->dropped = 0;
-    return ZERO_OK;
+        *count = n;
+        if (dropped) *dropped = t->dropped;
+        t->rec.clear();
+        t->dropped = 0;
+        return ZERO_OK;
+    });
 }
 
 extern "C" zero_status zero_trace_stop(zero_ctx_t* ctx) {
-    if (!ctx) return zb_fail(ZERO_ERR_INVALID_ARG, "zero_trace_stop: ctx is NULL");
-    if (ctx->trace) {
-        // events still queued must complete before they are destroyed
-        for (size_t i = 0; i < ctx->trace->rec.size(); ++i) cudaEventSynchronize(ctx->trace->ev[2 * i + 1]);
-        cudaGetLastError();
-    }
-    zb_trace_destroy(ctx);
-    return ZERO_OK;
+    return zb_guarded("zero_trace_stop", [&]() -> zero_status {
+        if (!ctx) return zb_fail(ZERO_ERR_INVALID_ARG, "zero_trace_stop: ctx is NULL");
+        if (ctx->trace) {
+            // events still queued must complete before they are destroyed
+            for (size_t i = 0; i < ctx->trace->rec.size(); ++i) cudaEventSynchronize(ctx->trace->ev[2 * i + 1]);
+            cudaGetLastError();
+        }
+        zb_trace_destroy(ctx);
+        return ZERO_OK;
+    });
 }
