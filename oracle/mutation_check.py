@@ -73,6 +73,7 @@ MUTANTS = [
     ("sharded_flag_one_owner", "overflow |= flag_o;", "overflow = flag_o;"),
     ("sharded_rank_stride", "s = s + oracle_half_to_float(grads[(int64_t)r * T + i], dtype);",
      "s = s + oracle_half_to_float(grads[(int64_t)r * S + i], dtype);"),
+    ("sample_norm_ignored", "if (norm_sq_all) nrm = *norm_sq_all;", "(void)norm_sq_all;"),
 ]
 
 
