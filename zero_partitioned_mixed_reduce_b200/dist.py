@@ -15,7 +15,11 @@ read every other rank's buffers with plain loads over NVLink. A step is:
   4. zero_step_commit, the same skip / loss-scale decision on every rank.
 
 With global-norm clipping, a norm pass over the rank's shard (again through
-the peer pointers) and a one-double all-reduce come before step 2.
+the peer pointers) and a one-double all-reduce come before step 2. Built
+with norm_divisor=k, the reduce-scatters of the two-pass form also take the
+rank's share of that norm (unscaled by the divisor k), and a clipped
+step_accumulated with divisor k sums the shares instead of reading the
+accumulator again.
 
 Gradient accumulation uses the two-pass form: after each micro-batch,
 reduce_scatter() sums the rank's shard of every replica into its local fp32
