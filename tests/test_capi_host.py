@@ -148,3 +148,25 @@ def test_release_build_carries_no_bounds_checks():
     if os.environ.get("ZERO_B200_LIB"):
         pytest.skip("another build is loaded")
     assert Z.zero_debug_bounds() == (-1, 0, 0)
+
+
+@pytest.mark.parametrize("seed", range(6))
+def test_pack_places_tensors_at_the_oracle_offsets(seed):
+    # the host marshalling (Plan.pack / unpack) against the oracle's own layout
+    import torch
+    rng = np.random.default_rng(300 + seed)
+    n = int(rng.integers(1, 12))
+    numels = rng.integers(1, 300, n).tolist()
+    R = int(rng.integers(1, 9))
+    align = int(rng.choice([1, 8]))
+    plan = Z.Plan(numels, None, R, Z.ZERO_BF16, align, 0)
+    lay = O.Layout(numels, R, align)
+    x = torch.from_numpy(rng.normal(0, 1, sum(numels)).astype(np.float32))
+    packed = plan.pack(x, fill=-7.0)
+    assert packed.numel() == lay.T
+    idx = lay.flat_index()
+    assert np.array_equal(packed.numpy()[idx], x.numpy())
+    pad = np.ones(lay.T, bool)
+    pad[idx] = False
+    assert np.all(packed.numpy()[pad] == -7.0)
+    assert torch.equal(plan.unpack(packed), x)
