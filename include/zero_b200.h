@@ -740,6 +740,10 @@ zero_status zero_layer_release(zero_ctx_t* ctx, int64_t layer, void* stream);
  * than 1024 count as 1024; the result
  * does not depend on nthreads except for the summation order of
  * grad_norm_sq. Work under 65,536 elements runs on the calling thread.
+ * Without a skip to decide (NONE or STATIC mode) and without clipping, the
+ * accumulators are scanned block by block right before each block's update,
+ * in one pass (30 bytes per element instead of 34); otherwise every
+ * accumulator is scanned first, as zero_cpu_scan does.
  * Errors: ZERO_ERR_INVALID_ARG.
  */
 zero_status zero_cpu_step(const zero_plan_t* plan, const zero_loss_scale_config* cfg,

@@ -205,6 +205,25 @@ __attribute__((target_clones("avx512f", "avx2", "default"))) void scan_range(
     *bad = b;
 }
 
+// Scan and update together, block by block: each 2048-element block is
+// scanned (overflow, squared norm) right before it is updated, so the
+// accumulator block is read from memory once. Only for steps whose update
+// needs nothing from the scan: no skip (NONE or STATIC mode) and no clipping.
+template <bool FP16>
+void scan_update_range(const Coeffs c, const float* __restrict acc, float* __restrict p, float* __restrict m,
+                       float* __restrict v, uint16_t* __restrict out, int64_t n, double* nrm, int* bad) {
+    constexpr int64_t kBlock = 2048;
+    for (int64_t b = 0; b < n; b += kBlock) {
+        const int64_t k = n - b < kBlock ? n - b : kBlock;
+        double bn = 0.0;
+        int bb = 0;
+        scan_range(acc + b, c.inv, k, &bn, &bb);
+        *nrm += bn;
+        *bad |= bb;
+        update_range<FP16, false>(c, acc + b, p + b, m + b, v + b, out + b, k);
+    }
+}
+
 // Worker threads kept between calls: a step on a small model, or an update
 // issued in several ranges, would otherwise spend a noticeable part of its
 // time starting threads. The caller's thread runs job 0 itself. One job runs
@@ -339,6 +358,49 @@ int thread_count(int32_t nthreads) {
     return n < 1 ? 1 : (n > kMaxThreads ? kMaxThreads : n);
 }
 
+// The AdamW coefficients of step t + 1, formed in double and rounded once,
+// exactly as the device step forms them.
+Coeffs make_coeffs(float inv, float clip, const zero_adamw& hp, int64_t t) {
+    Coeffs c;
+    const double t1 = static_cast<double>(t + 1);
+    c.inv = inv;
+    c.dec = static_cast<float>(1.0 - hp.lr * hp.weight_decay);
+    c.b1f = static_cast<float>(hp.beta1);
+    c.omb1 = static_cast<float>(1.0 - hp.beta1);
+    c.b2f = static_cast<float>(hp.beta2);
+    c.omb2 = static_cast<float>(1.0 - hp.beta2);
+    c.epsf = static_cast<float>(hp.eps);
+    c.ss = static_cast<float>(hp.lr / (1.0 - std::pow(hp.beta1, t1)));
+    c.bc2s = static_cast<float>(std::sqrt(1.0 - std::pow(hp.beta2, t1)));
+    c.clip = clip;
+    return c;
+}
+
+bool hp_ok(const zero_adamw* hp) {
+    return hp->lr >= 0.0 && hp->beta1 >= 0.0 && hp->beta1 < 1.0 && hp->beta2 >= 0.0 && hp->beta2 < 1.0 &&
+           hp->eps > 0.0 && hp->weight_decay >= 0.0;
+}
+
+// Everything zero_cpu_scan and zero_cpu_update check, for the one-pass step.
+zero_status check_step_args(const zero_plan_t* plan, const zero_loss_scale_config* cfg,
+                            const zero_loss_scale_state* in, const zero_adamw* hp, const zero_step_opts& o,
+                            const float* const* acc, float* const* master, float* const* m, float* const* v,
+                            void* const* param) {
+    if (!(o.grad_divisor >= 1.0) || !std::isfinite(o.grad_divisor))
+        return zb_fail(ZERO_ERR_INVALID_ARG, "zero_cpu_step: need grad_divisor >= 1, finite max_grad_norm >= 0, "
+                                             "no flags");
+    zero_status st = check_cfg(cfg, "zero_cpu_step");
+    if (st != ZERO_OK) return st;
+    const float scale = cfg->mode == ZERO_SCALE_NONE ? 1.0f : in->scale;
+    if (!(scale > 0.0f) || !std::isfinite(scale) || in->t < 0)
+        return zb_fail(ZERO_ERR_INVALID_ARG, "zero_cpu_step: need a finite scale > 0 and t >= 0");
+    if (!hp_ok(hp)) return zb_fail(ZERO_ERR_INVALID_ARG, "zero_cpu_step: bad hyper-parameters");
+    for (int r = 0; r < plan->R; ++r)
+        if (!acc[r] || !master[r] || !m[r] || !v[r] || !param[r])
+            return zb_fail(ZERO_ERR_INVALID_ARG, "zero_cpu_step: NULL rank pointer");
+    return ZERO_OK;
+}
+
 }  // namespace
 
 extern "C" zero_status zero_cpu_scan(const zero_plan_t* plan, const zero_loss_scale_config* cfg,
@@ -406,9 +468,7 @@ extern "C" zero_status zero_cpu_update(const zero_plan_t* plan, const zero_loss_
     return zb_guarded("zero_cpu_update", [&]() -> zero_status {
         if (!plan || !in || !hp || !d || !acc || !master || !m || !v || !param)
             return zb_fail(ZERO_ERR_INVALID_ARG, "zero_cpu_update: NULL argument");
-        if (!(hp->lr >= 0.0) || !(hp->beta1 >= 0.0 && hp->beta1 < 1.0) || !(hp->beta2 >= 0.0 && hp->beta2 < 1.0) ||
-            !(hp->eps > 0.0) || !(hp->weight_decay >= 0.0))
-            return zb_fail(ZERO_ERR_INVALID_ARG, "zero_cpu_step: bad hyper-parameters");
+        if (!hp_ok(hp)) return zb_fail(ZERO_ERR_INVALID_ARG, "zero_cpu_step: bad hyper-parameters");
         const int64_t S = plan->S;
         if (lo < 0 || lo > hi || hi > S)
             return zb_fail(ZERO_ERR_RANGE, "zero_cpu_update: need 0 <= lo <= hi <= S");
@@ -419,18 +479,7 @@ extern "C" zero_status zero_cpu_update(const zero_plan_t* plan, const zero_loss_
                 return zb_fail(ZERO_ERR_INVALID_ARG, "zero_cpu_step: NULL rank pointer");
         if (d->skip || lo == hi) return ZERO_OK;  // a skipped step writes nothing
         const int nt = thread_count(nthreads);
-        Coeffs c;
-        const double t1 = static_cast<double>(in->t + 1);
-        c.inv = d->inv;
-        c.dec = static_cast<float>(1.0 - hp->lr * hp->weight_decay);
-        c.b1f = static_cast<float>(hp->beta1);
-        c.omb1 = static_cast<float>(1.0 - hp->beta1);
-        c.b2f = static_cast<float>(hp->beta2);
-        c.omb2 = static_cast<float>(1.0 - hp->beta2);
-        c.epsf = static_cast<float>(hp->eps);
-        c.ss = static_cast<float>(hp->lr / (1.0 - std::pow(hp->beta1, t1)));
-        c.bc2s = static_cast<float>(std::sqrt(1.0 - std::pow(hp->beta2, t1)));
-        c.clip = d->clip;
+        const Coeffs c = make_coeffs(d->inv, d->clip, *hp, in->t);
         const bool fp16 = plan->dtype == ZERO_FP16, clip = d->clipping != 0;
         parallel_shards(R, lo, hi, nt, [&](int, int r, int64_t a, int64_t b) {
             const int64_t n = b - a;
@@ -483,11 +532,55 @@ extern "C" zero_status zero_cpu_step(const zero_plan_t* plan, const zero_loss_sc
     return zb_guarded("zero_cpu_step", [&]() -> zero_status {
         if (!plan || !cfg || !inout || !hp || !acc || !master || !m || !v || !param)
             return zb_fail(ZERO_ERR_INVALID_ARG, "zero_cpu_step: NULL argument");
+        zero_step_opts o{1.0, 0.0, 0, 0};
+        if (opts) o = *opts;
+        const bool one_pass = cfg->mode != ZERO_SCALE_DYNAMIC && o.max_grad_norm == 0.0 && o.flags == 0 &&
+                              o.reserved == 0;
+        if (!one_pass) {
+            // the update depends on the whole scan (a skip, or the clipping
+            // coefficient): scan every accumulator first
+            zero_cpu_decision d;
+            zero_status st = zero_cpu_scan(plan, cfg, inout, opts, acc, nthreads, &d);
+            if (st == ZERO_OK)
+                st = zero_cpu_update(plan, inout, hp, &d, acc, master, m, v, param, 0, plan->S, nthreads);
+            if (st == ZERO_OK) st = zero_cpu_commit(cfg, inout, &d);
+            return st;
+        }
+        // NONE / STATIC without clipping: one pass (scan and update per block)
         zero_cpu_decision d;
-        zero_status st = zero_cpu_scan(plan, cfg, inout, opts, acc, nthreads, &d);
-        if (st == ZERO_OK)
-            st = zero_cpu_update(plan, inout, hp, &d, acc, master, m, v, param, 0, plan->S, nthreads);
-        if (st == ZERO_OK) st = zero_cpu_commit(cfg, inout, &d);
-        return st;
+        zero_status st = check_step_args(plan, cfg, inout, hp, o, acc, master, m, v, param);
+        if (st != ZERO_OK) return st;
+        const int R = plan->R;
+        const int nt = thread_count(nthreads);
+        const float scale = cfg->mode == ZERO_SCALE_NONE ? 1.0f : inout->scale;
+        const float inv =
+            static_cast<float>(1.0 / ((static_cast<double>(R) * o.grad_divisor) * static_cast<double>(scale)));
+        const Coeffs c = make_coeffs(inv, 1.0f, *hp, inout->t);
+        const bool fp16 = plan->dtype == ZERO_FP16;
+        std::vector<double> part(static_cast<size_t>(nt), 0.0);
+        std::vector<int> bad(static_cast<size_t>(nt), 0);
+        parallel_shards(R, 0, plan->S, nt, [&](int t, int r, int64_t a, int64_t b) {
+            uint16_t* out = static_cast<uint16_t*>(param[r]) + a;
+            if (fp16)
+                scan_update_range<true>(c, acc[r] + a, master[r] + a, m[r] + a, v[r] + a, out, b - a, &part[t],
+                                        &bad[t]);
+            else
+                scan_update_range<false>(c, acc[r] + a, master[r] + a, m[r] + a, v[r] + a, out, b - a, &part[t],
+                                         &bad[t]);
+        });
+        double nrm = 0.0;
+        int overflow = 0;
+        for (size_t i = 0; i < part.size(); ++i) {
+            nrm += part[i];
+            overflow |= bad[i];
+        }
+        d.grad_norm_sq = nrm;
+        d.inv = inv;
+        d.clip = 1.0f;
+        d.overflow = overflow;
+        d.skip = 0;
+        d.clipping = 0;
+        d.reserved = 0;
+        return zero_cpu_commit(cfg, inout, &d);
     });
 }
