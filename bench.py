@@ -1222,15 +1222,19 @@ def run_offload(args, world, rank, local):
     host_triad = best_rate(lambda: torch.add(a, b, alpha=2.0, out=c), 3 * 4 * a.numel())
     torch.set_num_threads(nthr)
     del a, b, c
+    # host bytes per element: acc, master, m, v read and master, m, v, param
+    # written (30); DYNAMIC mode and clipping scan the accumulators first (+4)
+    cpu_bpp = 34.0 if wl["mode"] == synth.DYNAMIC else 30.0
     out = {"mode": "offload", "workload": args.workload, "P": P, "R": R, "tokens": args.tokens,
            "host_threads": os.cpu_count(), "gemm_flops_per_step": 2.0 * args.tokens * d * 8192 * n_gemm,
            "ms_serialized": t_ser * 1e3, "ms_delayed_update": t_dpu * 1e3,
            "ms_serialized_pipelined_upload": t_ser_pipe * 1e3,
            "ms_delayed_update_pipelined_upload": t_dpu_pipe * 1e3,
            "ms_gpu_part": t_gpu * 1e3, "ms_cpu_adamw": t_cpu * 1e3, "ms_param_upload": t_up * 1e3,
-           "cpu_adamw_params_per_s": T / t_cpu, "cpu_adamw_host_GBps": 30.0 * T / t_cpu / 1e9,
+           "cpu_adamw_params_per_s": T / t_cpu, "cpu_adamw_bytes_per_param": cpu_bpp,
+           "cpu_adamw_host_GBps": cpu_bpp * T / t_cpu / 1e9,
            "host_copy_GBps": host_copy, "host_triad_GBps": host_triad,
-           "cpu_adamw_frac_of_host_stream": 30.0 * T / t_cpu / 1e9 / max(host_copy, host_triad),
+           "cpu_adamw_frac_of_host_stream": cpu_bpp * T / t_cpu / 1e9 / max(host_copy, host_triad),
            "cpu_threads_overlapped": max(1, ncpu - 1),
            "speedup_from_delayed_update": t_ser / t_dpu, "steps": K,
            "timing": "host wall clock around synchronized loops (the CPU step is host work), "
