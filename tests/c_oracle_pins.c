@@ -4,7 +4,7 @@
  * golden fixtures, with no Python in between. Built and run by
  * tests/test_oracle_c_pins.py.
  *
- *   c_oracle_pins adamw_one_param.txt memory_pages.txt fsm_sequences.txt
+ *   c_oracle_pins adamw_one_param.txt memory_pages.txt fsm_sequences.txt layout_worked.txt
  *
  * - adamw_one_param.txt: two AdamW steps of one parameter, computed by hand
  *   in exact decimal arithmetic; the oracle's fp32 state must agree to a
@@ -13,6 +13,7 @@
  *   figures (~ within 1 %, "over" and "under" as stated).
  * - fsm_sequences.txt: loss-scale state machine sequences written by hand;
  *   every listed step's overflow, skip, scale, clean count and t.
+ * - layout_worked.txt: flat layouts worked by hand (offsets, P, L, S, T).
  * Prints one line per failed check and exits non-zero if any failed.
  */
 #include <math.h>
@@ -122,6 +123,55 @@ static void check_memory(const char* path) {
     if (rows < 5) fail("memory", "fewer than five rows");
 }
 
+static int parse_list(char* s, int64_t* out, int cap) {
+    int n = 0;
+    for (char* tok = strtok(s, ","); tok && n < cap; tok = strtok(NULL, ",")) out[n++] = strtoll(tok, NULL, 10);
+    return n;
+}
+
+static void check_layout(const char* path) {
+    FILE* f = fopen(path, "r");
+    if (!f) {
+        fail("layout", "cannot open the fixture");
+        return;
+    }
+    char line[1024];
+    int rows = 0;
+    while (fgets(line, sizeof line, f)) {
+        if (is_comment_or_blank(line)) continue;
+        char name[64], sizes_s[512], offs_s[512];
+        int R, align;
+        long long P, L, S, T;
+        if (sscanf(line, "%63s %d %d %511s %511s %lld %lld %lld %lld", name, &R, &align, sizes_s, offs_s, &P, &L,
+                   &S, &T) != 9) {
+            fail("layout", "unreadable row");
+            continue;
+        }
+        int64_t sizes[64], want_off[64], off[64], out[6], tb[64], blo[64], bhi[64], llo[64], lhi[64];
+        const int n = parse_list(sizes_s, sizes, 64);
+        const int no = parse_list(offs_s, want_off, 64);
+        if (n < 1 || no != n) {
+            fail("layout", "bad size or offset list");
+            continue;
+        }
+        if (oracle_layout(sizes, n, R, align, 0, NULL, off, out, tb, blo, bhi, llo, lhi) != 0) {
+            fail("layout", "oracle_layout rejected a worked example");
+            continue;
+        }
+        int ok = out[0] == P && out[1] == L && out[2] == S && out[3] == T;
+        for (int k = 0; k < n; k++) ok = ok && off[k] == want_off[k];
+        if (!ok) {
+            char msg[256];
+            snprintf(msg, sizeof msg, "%s: P %lld L %lld S %lld T %lld", name, (long long)out[0], (long long)out[1],
+                     (long long)out[2], (long long)out[3]);
+            fail("layout", msg);
+        }
+        rows += 1;
+    }
+    fclose(f);
+    if (rows < 4) fail("layout", "fewer than four rows");
+}
+
 static int mode_of(const char* s) {
     if (strcmp(s, "DYNAMIC") == 0) return ORACLE_SCALE_DYNAMIC;
     if (strcmp(s, "STATIC") == 0) return ORACLE_SCALE_STATIC;
@@ -204,13 +254,15 @@ static void check_fsm(const char* path) {
 }
 
 int main(int argc, char** argv) {
-    if (argc != 4) {
-        fprintf(stderr, "usage: %s adamw_one_param.txt memory_pages.txt fsm_sequences.txt\n", argv[0]);
+    if (argc != 5) {
+        fprintf(stderr, "usage: %s adamw_one_param.txt memory_pages.txt fsm_sequences.txt layout_worked.txt\n",
+                argv[0]);
         return 2;
     }
     check_adamw(argv[1]);
     check_memory(argv[2]);
     check_fsm(argv[3]);
+    check_layout(argv[4]);
     if (failures) return 1;
     printf("oracle pins ok\n");
     return 0;

@@ -1,17 +1,20 @@
 """The oracle's pins from C (tests/c_oracle_pins.c): a strict C99 program,
 linked to the oracle alone, checks it against the golden fixtures (the
 hand-computed AdamW steps, the pages' memory figures, the hand-written
-loss-scale sequences), and a planted mistake in the oracle makes it fail."""
+loss-scale sequences, the worked layouts), and a planted mistake in the
+oracle makes it fail."""
 import os
 import subprocess
 import tempfile
+
+import pytest
 
 import oracle as O
 
 HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 GOLDEN = [os.path.join(HERE, "golden", f)
-          for f in ("adamw_one_param.txt", "memory_pages.txt", "fsm_sequences.txt")]
+          for f in ("adamw_one_param.txt", "memory_pages.txt", "fsm_sequences.txt", "layout_worked.txt")]
 
 
 def _build(tmp, lib):
@@ -30,11 +33,16 @@ def test_c_program_passes_on_the_oracle():
     assert "oracle pins ok" in r.stdout
 
 
-def test_c_program_catches_a_planted_mistake():
-    # the same program against an oracle whose growth factor is wrong
+@pytest.mark.parametrize("old,new,where", [
+    ("st->scale = st->scale * st->growth_factor;", "st->scale = st->scale * 4.0f;", "fsm"),
+    ("int64_t S = round_up((L + R - 1) / R, 8);", "int64_t S = round_up(L / R, 8);", "layout"),
+    ("float pp = *p * c->dec;", "float pp = *p;", "adamw"),
+])
+def test_c_program_catches_a_planted_mistake(old, new, where):
+    # the same program against an oracle with one planted mistake
     src = open(os.path.join(ROOT, "oracle", "zero_oracle.c")).read()
-    bad = src.replace("st->scale = st->scale * st->growth_factor;", "st->scale = st->scale * 4.0f;")
-    assert bad != src
+    assert src.count(old) == 1
+    bad = src.replace(old, new)
     with tempfile.TemporaryDirectory() as tmp:
         c = os.path.join(tmp, "zero_oracle.c")
         open(c, "w").write(bad)
@@ -42,4 +50,4 @@ def test_c_program_catches_a_planted_mistake():
         subprocess.run(["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-ffp-contract=off",
                         "-I", os.path.join(ROOT, "oracle"), c, "-o", lib, "-lm"], check=True)
         r = subprocess.run([_build(tmp, lib), *GOLDEN], capture_output=True, text=True)
-    assert r.returncode == 1 and "FAIL fsm" in r.stderr
+    assert r.returncode == 1 and ("FAIL " + where) in r.stderr
