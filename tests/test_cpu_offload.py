@@ -235,3 +235,25 @@ def test_concurrent_cpu_steps_from_two_host_threads():
         for x, y in zip(param, lone[0][3]):
             assert np.array_equal(x, y)
         assert ls == lone[0][4]
+
+
+def test_random_configurations_match_oracle():
+    # property check over random configurations: tensor lists, R, dtype,
+    # alignment, loss-scale mode, micro-batches with their divisor, clipping,
+    # thread count; every step bit for bit against the oracle. Sizes straddle
+    # the one-thread threshold (65,536 elements) and the 2,048-element blocks.
+    from hypothesis import HealthCheck, given, settings, strategies as st
+
+    @settings(max_examples=25, deadline=None, suppress_health_check=list(HealthCheck))
+    @given(numels=st.lists(st.integers(1, 40_000), min_size=1, max_size=5),
+           R=st.integers(1, 6), dtype=st.sampled_from([O.BF16, O.FP16]), align=st.sampled_from([1, 8]),
+           mode=st.sampled_from([O.SCALE_NONE, O.SCALE_STATIC, O.SCALE_DYNAMIC]),
+           n_micro=st.integers(1, 3), clip=st.sampled_from([0.0, 1e-3, 1e9]),
+           nthreads=st.sampled_from([0, 1, 3]), seed=st.integers(0, 2**16))
+    def check(numels, R, dtype, align, mode, n_micro, clip, nthreads, seed):
+        o = Offload(numels, R, dtype, align, mode, seed=seed)
+        for _ in range(2):
+            o.step(n_micro, float(n_micro), clip, None, nthreads)
+            o.compare()
+
+    check()
