@@ -807,6 +807,42 @@ zero_status zero_cpu_commit(const zero_loss_scale_config* cfg, zero_loss_scale_s
                             const zero_cpu_decision* decision);
 
 /*
+ * The CPU step across processes (ZeRO-Offload with one process per rank,
+ * each holding only its own shards in host memory):
+ *
+ * zero_cpu_scan_shard -- zero_cpu_scan restricted to the owners
+ * [owner_lo, owner_hi): partial[0] = their sum of (double)((float)(acc *
+ * inv))^2, partial[1] = 1 if one of their accumulators is inf or NaN, else
+ * 0. Only acc[o] of the owners is read (other entries may be NULL).
+ * partial: host, 2 doubles. The ranks all-reduce partial (sum).
+ *
+ * zero_cpu_decide -- the step's decision from the all-reduced totals
+ * (reduced[0] = the squared norm, reduced[1] = the overflow count): the
+ * same decision zero_cpu_scan forms from all accumulators in one process.
+ *
+ * zero_cpu_update_shard -- zero_cpu_update of every element of the owners'
+ * shards; only the owners' pointers are read.
+ *
+ * Every rank then applies zero_cpu_commit with the same decision, so every
+ * rank's loss-scale state stays the same. The norm's summation grouping
+ * differs from one process's by rounding only.
+ * Defines: [legal] "CPU Offload"; [instr] ZeRO-2 "Mechanism" (each process
+ * updates its own partition).
+ * Errors: ZERO_ERR_INVALID_ARG, ZERO_ERR_RANGE (owner range).
+ */
+zero_status zero_cpu_scan_shard(const zero_plan_t* plan, const zero_loss_scale_config* cfg,
+                                const zero_loss_scale_state* in, const zero_step_opts* opts,
+                                const float* const* acc, int32_t owner_lo, int32_t owner_hi, int32_t nthreads,
+                                double* partial);
+zero_status zero_cpu_decide(const zero_plan_t* plan, const zero_loss_scale_config* cfg,
+                            const zero_loss_scale_state* in, const zero_step_opts* opts, const double* reduced,
+                            zero_cpu_decision* out);
+zero_status zero_cpu_update_shard(const zero_plan_t* plan, const zero_loss_scale_state* in, const zero_adamw* hp,
+                                  const zero_cpu_decision* decision, const float* const* acc,
+                                  float* const* master, float* const* m, float* const* v, void* const* param,
+                                  int32_t owner_lo, int32_t owner_hi, int32_t nthreads);
+
+/*
  * Per-call tracing. zero_trace_start makes every later call of the context
  * that queues GPU work bracket that work with two timing events on its
  * stream, up to `capacity` calls (1 .. 2^20; later ones are counted as

@@ -151,6 +151,14 @@ _sig("zero_cpu_scan", _S, [_P, C.POINTER(zero_loss_scale_config), C.POINTER(zero
 _sig("zero_cpu_update", _S, [_P, C.POINTER(zero_loss_scale_state), C.POINTER(zero_adamw),
                              C.POINTER(zero_cpu_decision), _PP, _PP, _PP, _PP, _PP, C.c_int64, C.c_int64,
                              C.c_int32])
+_sig("zero_cpu_scan_shard", _S, [_P, C.POINTER(zero_loss_scale_config), C.POINTER(zero_loss_scale_state),
+                                 C.POINTER(zero_step_opts), _PP, C.c_int32, C.c_int32, C.c_int32,
+                                 C.POINTER(C.c_double)])
+_sig("zero_cpu_decide", _S, [_P, C.POINTER(zero_loss_scale_config), C.POINTER(zero_loss_scale_state),
+                             C.POINTER(zero_step_opts), C.POINTER(C.c_double), C.POINTER(zero_cpu_decision)])
+_sig("zero_cpu_update_shard", _S, [_P, C.POINTER(zero_loss_scale_state), C.POINTER(zero_adamw),
+                                   C.POINTER(zero_cpu_decision), _PP, _PP, _PP, _PP, _PP, C.c_int32, C.c_int32,
+                                   C.c_int32])
 _sig("zero_cpu_commit", _S, [C.POINTER(zero_loss_scale_config), C.POINTER(zero_loss_scale_state),
                              C.POINTER(zero_cpu_decision)])
 _sig("zero_step_shard", _S, [_P, C.POINTER(zero_adamw), C.POINTER(zero_state), _PP, C.c_int32,
@@ -492,6 +500,36 @@ def zero_cpu_update(plan, state, hp, decision, acc, master, m, v, param, lo, hi,
                                 *[a[0] for a in arrays], lo, hi, nthreads))
 
 
+def zero_cpu_scan_shard(plan, cfg, state, acc, owner_lo, owner_hi, grad_divisor=1.0, max_grad_norm=0.0,
+                        nthreads=0):
+    """Owners [lo, hi)'s part of the CPU scan: (sum of unscaled g^2, overflow 0/1)."""
+    c, st = _cpu_cfg(cfg), _cpu_state(state)
+    opts = zero_step_opts(grad_divisor, max_grad_norm)
+    a = _ptr_array([_host_addr(x) for x in acc])
+    part = (C.c_double * 2)()
+    _check(_lib.zero_cpu_scan_shard(plan, C.byref(c), C.byref(st), C.byref(opts), a[0], owner_lo, owner_hi,
+                                    nthreads, part))
+    return float(part[0]), float(part[1])
+
+
+def zero_cpu_decide(plan, cfg, state, reduced, grad_divisor=1.0, max_grad_norm=0.0):
+    """The decision from all-reduced (norm sum, overflow count)."""
+    c, st = _cpu_cfg(cfg), _cpu_state(state)
+    opts = zero_step_opts(grad_divisor, max_grad_norm)
+    red = (C.c_double * 2)(float(reduced[0]), float(reduced[1]))
+    d = zero_cpu_decision()
+    _check(_lib.zero_cpu_decide(plan, C.byref(c), C.byref(st), C.byref(opts), red, C.byref(d)))
+    return d
+
+
+def zero_cpu_update_shard(plan, state, hp, decision, acc, master, m, v, param, owner_lo, owner_hi, nthreads=0):
+    """Update every element of shards [owner_lo, owner_hi) (the others' pointers may be None)."""
+    st, hp = _cpu_state(state), _cpu_hp(hp)
+    arrays = [_ptr_array([_host_addr(x) for x in xs]) for xs in (acc, master, m, v, param)]
+    _check(_lib.zero_cpu_update_shard(plan, C.byref(st), C.byref(hp), C.byref(decision),
+                                      *[a[0] for a in arrays], owner_lo, owner_hi, nthreads))
+
+
 def zero_cpu_commit(cfg, state, decision):
     """The loss-scale state after the step (a dict)."""
     c, st = _cpu_cfg(cfg), _cpu_state(state)
@@ -500,6 +538,8 @@ def zero_cpu_commit(cfg, state, decision):
 
 
 def _host_addr(x):
+    if x is None:
+        return 0
     if isinstance(x, int):
         return x
     if hasattr(x, "ctypes"):  # numpy

@@ -403,59 +403,155 @@ zero_status check_step_args(const zero_plan_t* plan, const zero_loss_scale_confi
 
 }  // namespace
 
+namespace {
+
+// Options of the CPU step, validated; the fp32 unscale factor into *inv.
+zero_status scan_args(const zero_plan_t* plan, const zero_loss_scale_config* cfg, const zero_loss_scale_state* in,
+                      const zero_step_opts* opts, zero_step_opts* o, float* inv) {
+    *o = zero_step_opts{1.0, 0.0, 0, 0};
+    if (opts) *o = *opts;
+    if (!(o->grad_divisor >= 1.0) || !std::isfinite(o->grad_divisor) || !(o->max_grad_norm >= 0.0) ||
+        !std::isfinite(o->max_grad_norm) || o->flags != 0 || o->reserved != 0)
+        return zb_fail(ZERO_ERR_INVALID_ARG, "zero_cpu_step: need grad_divisor >= 1, finite max_grad_norm >= 0, no flags");
+    zero_status st = check_cfg(cfg, "zero_cpu_step");
+    if (st != ZERO_OK) return st;
+    const float scale = cfg->mode == ZERO_SCALE_NONE ? 1.0f : in->scale;
+    if (!(scale > 0.0f) || !std::isfinite(scale) || in->t < 0)
+        return zb_fail(ZERO_ERR_INVALID_ARG, "zero_cpu_step: need a finite scale > 0 and t >= 0");
+    *inv = static_cast<float>(1.0 / ((static_cast<double>(plan->R) * o->grad_divisor) * static_cast<double>(scale)));
+    return ZERO_OK;
+}
+
+zero_status check_owners(const zero_plan_t* plan, int32_t owner_lo, int32_t owner_hi, const char* where) {
+    if (owner_lo < 0 || owner_lo >= owner_hi || owner_hi > plan->R)
+        return zb_fail(ZERO_ERR_RANGE, std::string(where) + ": need 0 <= owner_lo < owner_hi <= R");
+    return ZERO_OK;
+}
+
+// Overflow and squared norm over shards [r0, r1): each thread sums its
+// pieces in order, and the per-thread partials are summed in thread order.
+void scan_shards(const zero_plan_t* plan, const float* const* acc, float inv, int32_t r0, int32_t r1, int nt,
+                 double* nrm, int* overflow) {
+    std::vector<double> part(static_cast<size_t>(nt), 0.0);
+    std::vector<int> bad(static_cast<size_t>(nt), 0);
+    parallel_shards(r1 - r0, 0, plan->S, nt, [&](int t, int i, int64_t a, int64_t b) {
+        double pn = 0.0;
+        int pb = 0;
+        scan_range(acc[r0 + i] + a, inv, b - a, &pn, &pb);
+        part[t] += pn;
+        bad[t] |= pb;
+    });
+    double s = 0.0;
+    int o = 0;
+    for (size_t k = 0; k < part.size(); ++k) {
+        s += part[k];
+        o |= bad[k];
+    }
+    *nrm = s;
+    *overflow = o;
+}
+
+// The step's decision from the (global) squared norm and overflow.
+zero_cpu_decision decide(const zero_loss_scale_config* cfg, const zero_step_opts& o, float inv, double nrm,
+                         int overflow) {
+    zero_cpu_decision d;
+    d.grad_norm_sq = nrm;
+    d.inv = inv;
+    d.clip = 1.0f;
+    if (o.max_grad_norm > 0.0) {
+        const double cd = o.max_grad_norm / (std::sqrt(nrm) + 1e-6);
+        d.clip = static_cast<float>(cd < 1.0 ? cd : 1.0);
+    }
+    d.overflow = overflow ? 1 : 0;
+    d.skip = (cfg->mode == ZERO_SCALE_DYNAMIC && overflow) ? 1 : 0;
+    d.clipping = o.max_grad_norm > 0.0 ? 1 : 0;
+    d.reserved = 0;
+    return d;
+}
+
+// Elements [lo, hi) of shards [r0, r1) from a decision.
+zero_status update_shards(const zero_plan_t* plan, const zero_loss_scale_state* in, const zero_adamw* hp,
+                          const zero_cpu_decision* d, const float* const* acc, float* const* master, float* const* m,
+                          float* const* v, void* const* param, int32_t r0, int32_t r1, int64_t lo, int64_t hi,
+                          int32_t nthreads) {
+    if (!hp_ok(hp)) return zb_fail(ZERO_ERR_INVALID_ARG, "zero_cpu_step: bad hyper-parameters");
+    if (in->t < 0) return zb_fail(ZERO_ERR_INVALID_ARG, "zero_cpu_update: need t >= 0");
+    for (int r = r0; r < r1; ++r)
+        if (!acc[r] || !master[r] || !m[r] || !v[r] || !param[r])
+            return zb_fail(ZERO_ERR_INVALID_ARG, "zero_cpu_step: NULL rank pointer");
+    if (d->skip || lo == hi) return ZERO_OK;  // a skipped step writes nothing
+    const int nt = thread_count(nthreads);
+    const Coeffs c = make_coeffs(d->inv, d->clip, *hp, in->t);
+    const bool fp16 = plan->dtype == ZERO_FP16, clip = d->clipping != 0;
+    parallel_shards(r1 - r0, lo, hi, nt, [&](int, int i, int64_t a, int64_t b) {
+        const int r = r0 + i;
+        const int64_t n = b - a;
+        uint16_t* out = static_cast<uint16_t*>(param[r]) + a;
+        if (fp16 && clip) update_range<true, true>(c, acc[r] + a, master[r] + a, m[r] + a, v[r] + a, out, n);
+        else if (fp16) update_range<true, false>(c, acc[r] + a, master[r] + a, m[r] + a, v[r] + a, out, n);
+        else if (clip) update_range<false, true>(c, acc[r] + a, master[r] + a, m[r] + a, v[r] + a, out, n);
+        else update_range<false, false>(c, acc[r] + a, master[r] + a, m[r] + a, v[r] + a, out, n);
+    });
+    return ZERO_OK;
+}
+
+}  // namespace
+
 extern "C" zero_status zero_cpu_scan(const zero_plan_t* plan, const zero_loss_scale_config* cfg,
                                      const zero_loss_scale_state* in, const zero_step_opts* opts,
                                      const float* const* acc, int32_t nthreads, zero_cpu_decision* out) {
     return zb_guarded("zero_cpu_scan", [&]() -> zero_status {
         if (!plan || !cfg || !in || !acc || !out) return zb_fail(ZERO_ERR_INVALID_ARG, "zero_cpu_scan: NULL argument");
-        zero_step_opts o{1.0, 0.0, 0, 0};
-        if (opts) o = *opts;
-        if (!(o.grad_divisor >= 1.0) || !std::isfinite(o.grad_divisor) || !(o.max_grad_norm >= 0.0) ||
-            !std::isfinite(o.max_grad_norm) || o.flags != 0 || o.reserved != 0)
-            return zb_fail(ZERO_ERR_INVALID_ARG,
-                           "zero_cpu_step: need grad_divisor >= 1, finite max_grad_norm >= 0, no flags");
-        zero_status st = check_cfg(cfg, "zero_cpu_step");
+        zero_step_opts o;
+        float inv = 0.0f;
+        zero_status st = scan_args(plan, cfg, in, opts, &o, &inv);
         if (st != ZERO_OK) return st;
-        const float scale = cfg->mode == ZERO_SCALE_NONE ? 1.0f : in->scale;
-        if (!(scale > 0.0f) || !std::isfinite(scale) || in->t < 0)
-            return zb_fail(ZERO_ERR_INVALID_ARG, "zero_cpu_step: need a finite scale > 0 and t >= 0");
-        const int R = plan->R;
-        for (int r = 0; r < R; ++r)
+        for (int r = 0; r < plan->R; ++r)
             if (!acc[r]) return zb_fail(ZERO_ERR_INVALID_ARG, "zero_cpu_step: NULL rank pointer");
-        const int nt = thread_count(nthreads);
-        const int64_t S = plan->S;
-        const float inv =
-            static_cast<float>(1.0 / ((static_cast<double>(R) * o.grad_divisor) * static_cast<double>(scale)));
-        // overflow and squared norm; each thread sums its pieces in order, and
-        // the per-thread partials are summed in thread order
-        std::vector<double> part(static_cast<size_t>(nt), 0.0);
-        std::vector<int> bad(static_cast<size_t>(nt), 0);
-        parallel_shards(R, 0, S, nt, [&](int t, int r, int64_t a, int64_t b) {
-            double pn = 0.0;
-            int pb = 0;
-            scan_range(acc[r] + a, inv, b - a, &pn, &pb);
-            part[t] += pn;
-            bad[t] |= pb;
-        });
         double nrm = 0.0;
         int overflow = 0;
-        for (size_t i = 0; i < part.size(); ++i) {
-            nrm += part[i];
-            overflow |= bad[i];
-        }
-        zero_cpu_decision d;
-        d.grad_norm_sq = nrm;
-        d.inv = inv;
-        d.clip = 1.0f;
-        if (o.max_grad_norm > 0.0) {
-            const double cd = o.max_grad_norm / (std::sqrt(nrm) + 1e-6);
-            d.clip = static_cast<float>(cd < 1.0 ? cd : 1.0);
-        }
-        d.overflow = overflow;
-        d.skip = (cfg->mode == ZERO_SCALE_DYNAMIC && overflow) ? 1 : 0;
-        d.clipping = o.max_grad_norm > 0.0 ? 1 : 0;
-        d.reserved = 0;
-        *out = d;
+        scan_shards(plan, acc, inv, 0, plan->R, thread_count(nthreads), &nrm, &overflow);
+        *out = decide(cfg, o, inv, nrm, overflow);
+        return ZERO_OK;
+    });
+}
+
+extern "C" zero_status zero_cpu_scan_shard(const zero_plan_t* plan, const zero_loss_scale_config* cfg,
+                                           const zero_loss_scale_state* in, const zero_step_opts* opts,
+                                           const float* const* acc, int32_t owner_lo, int32_t owner_hi,
+                                           int32_t nthreads, double* partial) {
+    return zb_guarded("zero_cpu_scan_shard", [&]() -> zero_status {
+        if (!plan || !cfg || !in || !acc || !partial)
+            return zb_fail(ZERO_ERR_INVALID_ARG, "zero_cpu_scan_shard: NULL argument");
+        zero_status st = check_owners(plan, owner_lo, owner_hi, "zero_cpu_scan_shard");
+        if (st != ZERO_OK) return st;
+        zero_step_opts o;
+        float inv = 0.0f;
+        if ((st = scan_args(plan, cfg, in, opts, &o, &inv)) != ZERO_OK) return st;
+        for (int r = owner_lo; r < owner_hi; ++r)
+            if (!acc[r]) return zb_fail(ZERO_ERR_INVALID_ARG, "zero_cpu_scan_shard: NULL owned accumulator");
+        double nrm = 0.0;
+        int overflow = 0;
+        scan_shards(plan, acc, inv, owner_lo, owner_hi, thread_count(nthreads), &nrm, &overflow);
+        partial[0] = nrm;
+        partial[1] = overflow ? 1.0 : 0.0;
+        return ZERO_OK;
+    });
+}
+
+extern "C" zero_status zero_cpu_decide(const zero_plan_t* plan, const zero_loss_scale_config* cfg,
+                                       const zero_loss_scale_state* in, const zero_step_opts* opts,
+                                       const double* reduced, zero_cpu_decision* out) {
+    return zb_guarded("zero_cpu_decide", [&]() -> zero_status {
+        if (!plan || !cfg || !in || !reduced || !out)
+            return zb_fail(ZERO_ERR_INVALID_ARG, "zero_cpu_decide: NULL argument");
+        zero_step_opts o;
+        float inv = 0.0f;
+        zero_status st = scan_args(plan, cfg, in, opts, &o, &inv);
+        if (st != ZERO_OK) return st;
+        if (!(reduced[1] >= 0.0) || !(reduced[0] >= 0.0 || std::isnan(reduced[0])))
+            return zb_fail(ZERO_ERR_INVALID_ARG, "zero_cpu_decide: need a norm sum and an overflow count >= 0");
+        *out = decide(cfg, o, inv, reduced[0], reduced[1] > 0.0 ? 1 : 0);
         return ZERO_OK;
     });
 }
@@ -468,28 +564,23 @@ extern "C" zero_status zero_cpu_update(const zero_plan_t* plan, const zero_loss_
     return zb_guarded("zero_cpu_update", [&]() -> zero_status {
         if (!plan || !in || !hp || !d || !acc || !master || !m || !v || !param)
             return zb_fail(ZERO_ERR_INVALID_ARG, "zero_cpu_update: NULL argument");
-        if (!hp_ok(hp)) return zb_fail(ZERO_ERR_INVALID_ARG, "zero_cpu_step: bad hyper-parameters");
-        const int64_t S = plan->S;
-        if (lo < 0 || lo > hi || hi > S)
+        if (lo < 0 || lo > hi || hi > plan->S)
             return zb_fail(ZERO_ERR_RANGE, "zero_cpu_update: need 0 <= lo <= hi <= S");
-        if (in->t < 0) return zb_fail(ZERO_ERR_INVALID_ARG, "zero_cpu_update: need t >= 0");
-        const int R = plan->R;
-        for (int r = 0; r < R; ++r)
-            if (!acc[r] || !master[r] || !m[r] || !v[r] || !param[r])
-                return zb_fail(ZERO_ERR_INVALID_ARG, "zero_cpu_step: NULL rank pointer");
-        if (d->skip || lo == hi) return ZERO_OK;  // a skipped step writes nothing
-        const int nt = thread_count(nthreads);
-        const Coeffs c = make_coeffs(d->inv, d->clip, *hp, in->t);
-        const bool fp16 = plan->dtype == ZERO_FP16, clip = d->clipping != 0;
-        parallel_shards(R, lo, hi, nt, [&](int, int r, int64_t a, int64_t b) {
-            const int64_t n = b - a;
-            uint16_t* out = static_cast<uint16_t*>(param[r]) + a;
-            if (fp16 && clip) update_range<true, true>(c, acc[r] + a, master[r] + a, m[r] + a, v[r] + a, out, n);
-            else if (fp16) update_range<true, false>(c, acc[r] + a, master[r] + a, m[r] + a, v[r] + a, out, n);
-            else if (clip) update_range<false, true>(c, acc[r] + a, master[r] + a, m[r] + a, v[r] + a, out, n);
-            else update_range<false, false>(c, acc[r] + a, master[r] + a, m[r] + a, v[r] + a, out, n);
-        });
-        return ZERO_OK;
+        return update_shards(plan, in, hp, d, acc, master, m, v, param, 0, plan->R, lo, hi, nthreads);
+    });
+}
+
+extern "C" zero_status zero_cpu_update_shard(const zero_plan_t* plan, const zero_loss_scale_state* in,
+                                             const zero_adamw* hp, const zero_cpu_decision* d,
+                                             const float* const* acc, float* const* master, float* const* m,
+                                             float* const* v, void* const* param, int32_t owner_lo,
+                                             int32_t owner_hi, int32_t nthreads) {
+    return zb_guarded("zero_cpu_update_shard", [&]() -> zero_status {
+        if (!plan || !in || !hp || !d || !acc || !master || !m || !v || !param)
+            return zb_fail(ZERO_ERR_INVALID_ARG, "zero_cpu_update_shard: NULL argument");
+        zero_status st = check_owners(plan, owner_lo, owner_hi, "zero_cpu_update_shard");
+        if (st != ZERO_OK) return st;
+        return update_shards(plan, in, hp, d, acc, master, m, v, param, owner_lo, owner_hi, 0, plan->S, nthreads);
     });
 }
 
