@@ -170,3 +170,11 @@ def test_pack_places_tensors_at_the_oracle_offsets(seed):
     pad[idx] = False
     assert np.all(packed.numpy()[pad] == -7.0)
     assert torch.equal(plan.unpack(packed), x)
+
+
+def test_every_declared_function_has_a_binding_of_the_same_name():
+    hdr = open(os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include",
+                            "zero_b200.h")).read()
+    names = sorted(set(re.findall(r"^\w[\w\s\*]*?\b(zero_\w+)\s*\(", hdr, re.M)))
+    assert len(names) >= 40
+    assert [n for n in names if not callable(getattr(Z, n, None))] == []
