@@ -10,6 +10,9 @@
  *       one zero_cpu_step (NONE mode, fixed hyper-parameters) on host shards
  *       read from in_file (acc, master, m, v: R*S fp32 each, rank after rank)
  *       writing out_file (master, m, v as fp32, then param as uint16)
+ *   c_abi_client cpu_step_shard ...
+ *       the same step one owner at a time (zero_cpu_scan_shard, the summed
+ *       totals, zero_cpu_decide, zero_cpu_update_shard, zero_cpu_commit)
  *   c_abi_client errors
  *       error statuses and messages of a few invalid calls
  */
@@ -89,7 +92,7 @@ static int cmd_plan(int argc, char** argv) {
 
 static int read_all(FILE* f, void* p, size_t bytes) { return fread(p, 1, bytes, f) == bytes ? 0 : 1; }
 
-static int cmd_cpu_step(int argc, char** argv) {
+static int cmd_cpu_step(int argc, char** argv, int sharded) {
     if (argc < 5) return 2;
     int32_t R = atoi(argv[2]), dtype = atoi(argv[3]);
     zero_plan_t* plan = NULL;
@@ -126,8 +129,31 @@ static int cmd_cpu_step(int argc, char** argv) {
     memset(&st, 0, sizeof st);
     st.scale = 1.0f;
     zero_adamw hp = {1e-3, 0.9, 0.999, 1e-8, 0.01};
-    zero_status s = zero_cpu_step(plan, &cfg, &st, &hp, NULL, acc, master, m, v, par, 2);
-    if (s != ZERO_OK) return fail("zero_cpu_step", s);
+    zero_status s = ZERO_OK;
+    if (!sharded) {
+        s = zero_cpu_step(plan, &cfg, &st, &hp, NULL, acc, master, m, v, par, 2);
+        if (s != ZERO_OK) return fail("zero_cpu_step", s);
+    } else {
+        /* one owner at a time, as separate processes would: its totals, the
+           summed totals, one decision, its own update, one commit */
+        double total[2] = {0.0, 0.0};
+        for (int32_t o = 0; o < R; o++) {
+            double part[2];
+            s = zero_cpu_scan_shard(plan, &cfg, &st, NULL, acc, o, o + 1, 2, part);
+            if (s != ZERO_OK) return fail("zero_cpu_scan_shard", s);
+            total[0] += part[0];
+            total[1] += part[1];
+        }
+        zero_cpu_decision d;
+        s = zero_cpu_decide(plan, &cfg, &st, NULL, total, &d);
+        if (s != ZERO_OK) return fail("zero_cpu_decide", s);
+        for (int32_t o = 0; o < R; o++) {
+            s = zero_cpu_update_shard(plan, &st, &hp, &d, acc, master, m, v, par, o, o + 1, 2);
+            if (s != ZERO_OK) return fail("zero_cpu_update_shard", s);
+        }
+        s = zero_cpu_commit(&cfg, &st, &d);
+        if (s != ZERO_OK) return fail("zero_cpu_commit", s);
+    }
     printf("state %lld %d %d %.17g\n", (long long)st.t, (int)st.last_overflow, (int)st.last_skipped,
            st.grad_norm_sq);
     FILE* out = fopen(argv[next + 1], "wb");
@@ -181,7 +207,8 @@ static int cmd_errors(void) {
 int main(int argc, char** argv) {
     if (argc < 2) return 2;
     if (strcmp(argv[1], "plan") == 0) return cmd_plan(argc, argv);
-    if (strcmp(argv[1], "cpu_step") == 0) return cmd_cpu_step(argc, argv);
+    if (strcmp(argv[1], "cpu_step") == 0) return cmd_cpu_step(argc, argv, 0);
+    if (strcmp(argv[1], "cpu_step_shard") == 0) return cmd_cpu_step(argc, argv, 1);
     if (strcmp(argv[1], "errors") == 0) return cmd_errors();
     return 2;
 }

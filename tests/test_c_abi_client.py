@@ -62,8 +62,10 @@ def test_plan_from_c_matches_oracle_layout(client, seed):
         assert memory[stage] == O.model_state_bytes(stage, lay.T, R)
 
 
+@pytest.mark.parametrize("mode", ["cpu_step", "cpu_step_shard"])
 @pytest.mark.parametrize("R,dtype", [(1, O.BF16), (4, O.FP16), (3, O.BF16)])
-def test_cpu_step_from_c_matches_oracle(client, tmp_path, R, dtype):
+def test_cpu_step_from_c_matches_oracle(client, tmp_path, R, dtype, mode):
+    # the whole CPU step, or the per-owner calls of a multi-process offload
     rng = np.random.default_rng(R * 7 + dtype)
     numels = [3001, 17, 4096]
     lay = O.Layout(numels, R, 8)
@@ -82,7 +84,7 @@ def test_cpu_step_from_c_matches_oracle(client, tmp_path, R, dtype):
                            np.zeros(lay.T, np.float32)])
     fin, fout = tmp_path / "in.bin", tmp_path / "out.bin"
     blob.tofile(fin)
-    out = run(client, "cpu_step", R, dtype, len(numels), *numels, fin, fout)
+    out = run(client, mode, R, dtype, len(numels), *numels, fin, fout)
     fsm = O.make_fsm(O.SCALE_NONE)
     O.step(st, g, O.AdamW(1e-3, 0.9, 0.999, 1e-8, 0.01), fsm)
     state = out[0]
