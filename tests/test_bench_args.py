@@ -20,3 +20,14 @@ def test_workload_label_names_the_sizes():
     wl = synth.workload("gpt2s")
     label = bench.workload_label("gpt2s", wl)
     assert "P=124439808" in label and "R=8" in label and "fp16" in label
+
+
+def test_oracle_crew_runs_the_oracle_on_several_processes():
+    # the all-core CPU baseline: spawned single-threaded oracle processes,
+    # timed between a common barrier and the last end
+    crew = bench.OracleCrew("tiny", 4096, procs=2)
+    try:
+        rate, sec = crew.run(1)
+    finally:
+        crew.close()
+    assert rate > 0 and sec > 0 and crew.procs == 2
