@@ -243,7 +243,7 @@ class Bench:
     def __init__(self, name, path, first_tensors=0, gather_bucket=32 << 20, accum=1, clip=0.0,
                  bucket_elems=None, clip_norm="rs"):
         import zero_partitioned_mixed_reduce_b200 as Z
-        from zero_partitioned_mixed_reduce_b200 import synth
+        import synth
         self.Z, self.synth = Z, synth
         self.wl = wl = synth.workload(name)
         if bucket_elems is not None:
@@ -634,7 +634,7 @@ def oracle_inputs(name, n):
     """The oracle's state, replicas, hyper-parameters and loss-scale state
     for the first n params of the workload."""
     import oracle as O
-    from zero_partitioned_mixed_reduce_b200 import synth
+    import synth
     wl = synth.workload(name)
     R, dtype = wl["R"], wl["dtype"]
     scale = wl["init_scale"] if wl["mode"] != synth.NONE else 1.0
@@ -868,7 +868,7 @@ def run_rs_sweep(args, world, rank, local):
         print(json.dumps({"error": "no CUDA device"}))
         sys.exit(1)
     import zero_partitioned_mixed_reduce_b200 as Z
-    from zero_partitioned_mixed_reduce_b200 import synth
+    import synth
     wl = synth.workload(args.workload)
     R, dtype = wl["R"], wl["dtype"]
     sizes = [int(x) for x in args.rs_sizes.split(",")]
@@ -951,7 +951,7 @@ def run_dist(args, world, rank, local):
     the model is fixed, N ranks share it. Each rank writes its own replica."""
     import socket
     import torch.distributed as dist
-    from zero_partitioned_mixed_reduce_b200 import synth
+    import synth
     from zero_partitioned_mixed_reduce_b200.dist import DistributedZero
     if not torch.cuda.is_available():
         print(json.dumps({"error": "no CUDA device"}))
@@ -1064,7 +1064,7 @@ def run_offload(args, world, rank, local):
         print(json.dumps({"error": "no CUDA device"}))
         sys.exit(1)
     import zero_partitioned_mixed_reduce_b200 as Z
-    from zero_partitioned_mixed_reduce_b200 import synth
+    import synth
     wl = synth.workload(args.workload)
     if args.first_tensors:
         wl["numels"] = wl["numels"][:args.first_tensors]
@@ -1256,7 +1256,7 @@ def run_reference(args, world, rank):
         value, sec = crew.run(args.steps)
     finally:
         crew.close()
-    from zero_partitioned_mixed_reduce_b200 import synth
+    import synth
     wl = synth.workload(args.workload)
     out = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "params/s",

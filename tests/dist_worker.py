@@ -13,7 +13,7 @@ sys.path.insert(0, ROOT)
 
 import oracle as O  # noqa: E402
 import zero_partitioned_mixed_reduce_b200 as Z  # noqa: E402
-from zero_partitioned_mixed_reduce_b200 import synth  # noqa: E402
+import synth  # noqa: E402
 from zero_partitioned_mixed_reduce_b200.dist import DistributedZero  # noqa: E402
 
 

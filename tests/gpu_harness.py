@@ -11,7 +11,7 @@ import torch
 
 import oracle as O
 import zero_partitioned_mixed_reduce_b200 as Z
-from zero_partitioned_mixed_reduce_b200 import synth
+import synth
 
 GUARD = 64  # elements; keeps 32-byte alignment for fp32 and 16-byte for half
 CANARY_F32 = 0x7FBADBAD  # a NaN pattern no kernel writes

@@ -16,7 +16,7 @@ def test_eager_and_graph_flags():
 
 
 def test_workload_label_names_the_sizes():
-    from zero_partitioned_mixed_reduce_b200 import synth
+    import synth
     wl = synth.workload("gpt2s")
     label = bench.workload_label("gpt2s", wl)
     assert "P=124439808" in label and "R=8" in label and "fp16" in label

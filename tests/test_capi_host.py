@@ -13,7 +13,8 @@ import torch
 
 import oracle as O
 import zero_partitioned_mixed_reduce_b200 as Z
-from zero_partitioned_mixed_reduce_b200 import _capi, synth
+from zero_partitioned_mixed_reduce_b200 import _capi
+import synth
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 

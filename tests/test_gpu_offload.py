@@ -16,7 +16,7 @@ pytestmark = pytest.mark.gpu
 
 if torch.cuda.is_available():
     import zero_partitioned_mixed_reduce_b200 as Z
-    from zero_partitioned_mixed_reduce_b200 import synth
+    import synth
     from gpu_harness import u16
 
 HALF = {0: torch.bfloat16, 1: torch.float16}

@@ -41,7 +41,7 @@ def _bits(ts):
 @pytest.mark.parametrize("dtype,mode", [(1, 2), (0, 1), (0, 0)])
 def test_noalloc_matches_context_two_pass(dtype, mode):
     import zero_partitioned_mixed_reduce_b200 as Z
-    from zero_partitioned_mixed_reduce_b200 import synth
+    import synth
 
     numels, R = [70_001, 13, 4096, 777, 5], 4
     plan = Z.Plan(numels, None, R, dtype, 8, 0)
