@@ -3,23 +3,27 @@
 
 One step = one pass of the whole path over one batch of synthetic
 gradients: the fused reduce-scatter + unscale + overflow check + AdamW +
-cast kernel over every shard (ping-pong state under dynamic loss scaling),
-the device-side loss-scale update, and the ZeRO-3 gather of every layer into
-a contiguous buffer. The partition plan is built once, before timing.
+cast kernel over every shard (ping-pong state), the device-side loss-scale
+update, and the ZeRO-3 gather of every layer into a contiguous buffer. The
+partition plan is built once, before timing.
 
-Default workload: GPT-2-small-shaped parameter list (124,439,808 params,
-148 tensors), R=8 simulated ranks, fp16 gradients, dynamic loss scaling from
-2^16. Inputs (about 5.7 GB touched per step) are resident in HBM and larger
-than the 126 MB L2.
+Default workload: the Llama-style 3B-shaped parameter list (3,606,752,256
+params, 255 tensors, 28 layers, d=3072, SwiGLU 8192, GQA 24/8 heads, vocab
+128256, untied embeddings), R=4 simulated ranks, bf16 gradients
+1e-4 * Student-t(3), no loss scaling. The step touches about 137 GB of HBM,
+far more than the 126 MB L2. `--workload gpt2s|d1p3b|irr_r2|irr_r16|tiny`
+selects the other configurations.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
-With N > 1 (under torch.distributed.run) every rank runs its own independent
-replica of the workload (weak scaling, no collective on the data path); the
-time is the maximum over ranks. The step and the gathers are captured once
-into CUDA graphs through the C ABI and replayed (`--eager` issues every
-launch instead). `--impl reference` times the CPU oracle on host cores on a
-bounded sample of the same workload.
+With N > 1 (under torch.distributed.run) the job runs the real multi-GPU
+ZeRO step (DistributedZero): rank o owns shard o of the workload, its fused
+step reads the other ranks' gradient replicas over NVLink, and the ZeRO-3
+gathers read every rank's parameter shard; the time is the maximum over
+ranks. `--replicas` runs N independent single-GPU copies instead. The step
+and the gathers are captured once into CUDA graphs through the C ABI and
+replayed (`--eager` issues every launch instead). `--impl reference` times
+the CPU oracle on host cores on a bounded sample of the same workload.
 """
 import argparse
 import datetime
@@ -47,7 +51,7 @@ def parse_args(argv=None):
     ap.add_argument("--steps", type=int, default=100)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", default="gpt2s")
+    ap.add_argument("--workload", default="llama3b")
     ap.add_argument("--path", choices=["auto", "pingpong", "inplace", "twopass", "twopass_pingpong"],
                     default="auto",
                     help="fused step (ping-pong or in-place state) or the two-pass path "
@@ -84,7 +88,14 @@ def parse_args(argv=None):
     ap.add_argument("--rs-sizes", default="0,1000000,5000000,25000000,50000000,100000000,200000000",
                     help="bucket sizes (elements; 0: one bucket for the whole model) for --rs-sweep")
     ap.add_argument("--dist", action="store_true",
-                    help="the real multi-GPU ZeRO step over the job's GPUs (DistributedZero) instead")
+                    help="the real multi-GPU ZeRO step over the job's GPUs (DistributedZero), also at "
+                         "N = 1 (the default whenever N > 1)")
+    ap.add_argument("--replicas", action="store_true",
+                    help="with N > 1: N independent single-GPU copies of the workload (no collective on "
+                         "the data path) instead of the sharded multi-GPU step")
+    ap.add_argument("--rs-group", type=int, default=25 << 20,
+                    help="two-pass path: consecutive buckets reduce-scattered in one launch up to this "
+                         "many elements (0: one launch per bucket)")
     ap.add_argument("--graph", dest="graph", action="store_true", default=True,
                     help="(default) capture the step and the gathers once into CUDA graphs, "
                          "through the C ABI, and replay them")
@@ -239,9 +250,25 @@ def workload_label(name, wl, first_tensors=0):
             f"loss scale mode {wl['mode']}")
 
 
+def bucket_runs(buckets, group):
+    """Consecutive buckets, as (first, count), in launches of up to `group`
+    elements (a larger bucket alone); group 0: one launch per bucket.
+    Consecutive buckets are one contiguous flat range."""
+    runs, first, size = [], 0, 0
+    for b, (lo, hi) in enumerate(buckets):
+        n = hi - lo
+        if b > first and (group <= 0 or size + n > group):
+            runs.append((first, b - first))
+            first, size = b, 0
+        size += n
+    if buckets:
+        runs.append((first, len(buckets) - first))
+    return runs
+
+
 class Bench:
     def __init__(self, name, path, first_tensors=0, gather_bucket=32 << 20, accum=1, clip=0.0,
-                 bucket_elems=None, clip_norm="rs"):
+                 bucket_elems=None, clip_norm="rs", rs_group=25 << 20):
         import zero_partitioned_mixed_reduce_b200 as Z
         import synth
         self.Z, self.synth = Z, synth
@@ -272,6 +299,9 @@ class Bench:
         self.plan = Z.Plan(wl["numels"], wl["layer_ids"], wl["R"], wl["dtype"], 8,
                            wl["bucket_elems"])
         self.P, self.T, self.S, self.L = self.plan.P, self.plan.T, self.plan.S, self.plan.L
+        # reduce-scatters of consecutive buckets grouped into launches, as a
+        # caller whose backward has written them issues them
+        self.rs_runs = bucket_runs(self.plan.buckets, rs_group)
         # the two-pass step measured the same in place as ping-pong, so it
         # keeps one state set
         sets = 2 if path in ("pingpong", "twopass_pingpong") else 1
@@ -330,9 +360,9 @@ class Bench:
     def launches_per_step(self):
         n = 1 + (len(self.gather_buckets) if self.gather_buckets else len(self.plan.layers))
         if self.twopass:
-            n += self.accum * len(self.plan.buckets)
+            n += self.accum * len(self.rs_runs)
         else:
-            n += (self.accum - 1) * len(self.plan.buckets)
+            n += (self.accum - 1) * len(self.rs_runs)
         if self.clip > 0:
             n += 1  # the norm pass
         return n
@@ -365,16 +395,17 @@ class Bench:
                 flags = Z.ZERO_RS_ACCUMULATE if mu else 0
                 if self.rs_norm and mu == self.accum - 1:
                     flags |= Z.ZERO_RS_NORM
-                for b in range(len(self.plan.buckets)):
-                    Z.zero_reduce_scatter_bucket_ex(self.ctx, b, grads, self.state.acc, flags,
-                                                    stream)
+                for first, count in self.rs_runs:
+                    Z.zero_reduce_scatter_buckets(self.ctx, first, count, grads, self.state.acc, flags,
+                                                  stream)
             Z.zero_step_ex(self.ctx, hp, self.state.handle, None, float(self.accum), self.clip,
                            stream, flags=Z.ZERO_STEP_NORM_FROM_RS if self.rs_norm else 0)
         elif self.accum > 1:
             for mu in range(self.accum - 1):
                 flags = Z.ZERO_RS_ACCUMULATE if mu else 0
-                for b in range(len(self.plan.buckets)):
-                    Z.zero_reduce_scatter_bucket_ex(self.ctx, b, grads, self.state.acc, flags, stream)
+                for first, count in self.rs_runs:
+                    Z.zero_reduce_scatter_buckets(self.ctx, first, count, grads, self.state.acc, flags,
+                                                  stream)
             Z.zero_step_ex(self.ctx, hp, self.state.handle, grads, float(self.accum), 0.0, stream,
                            flags=Z.ZERO_STEP_ADD_ACC)
         elif self.clip > 0:
@@ -445,7 +476,7 @@ def run_ours(args, world, rank, local):
         print(json.dumps({"error": "no CUDA device: the benchmark has no CPU fallback"}))
         sys.exit(1)
     b = Bench(args.workload, args.path, args.first_tensors, args.gather_bucket, args.accum,
-              args.clip, clip_norm=args.clip_norm)
+              args.clip, clip_norm=args.clip_norm, rs_group=args.rs_group)
     stream = torch.cuda.current_stream()
     if args.graph:
         b.capture(stream, args.warmup + args.steps + 16)  # + the e2e leg's steps
@@ -531,10 +562,12 @@ def run_ours(args, world, rank, local):
                                  "fused reduce-scatter+AdamW, ping-pong state",
                      "inplace": f"{'global-norm clip pass, ' if b.clip > 0 else ''}"
                                 "fused reduce-scatter+AdamW, in place",
-                     "twopass": f"bucketed reduce-scatter ({b.accum} micro-batch(es)), "
+                     "twopass": f"bucketed reduce-scatter ({b.accum} micro-batch(es), "
+                       f"{len(b.plan.buckets)} buckets in {len(b.rs_runs)} grouped launches each), "
                        f"{clip_label}"
                        "then AdamW from fp32 accumulators, in place",
-                     "twopass_pingpong": f"bucketed reduce-scatter ({b.accum} micro-batch(es)), "
+                     "twopass_pingpong": f"bucketed reduce-scatter ({b.accum} micro-batch(es), "
+                       f"{len(b.plan.buckets)} buckets in {len(b.rs_runs)} grouped launches each), "
                        f"{clip_label}"
                        "then AdamW from fp32 accumulators, ping-pong state"}[b.path]
                     + " + device loss-scale update + ZeRO-3 gather of every layer",
@@ -543,7 +576,7 @@ def run_ours(args, world, rank, local):
                        else f"{len(b.plan.layers)} per-layer launches"),
             "bytes_per_step": step_bytes,
             "l2": f"inputs larger than L2 ({step_bytes / 1e9:.1f} GB touched per step, L2 126 MB)",
-            "parallelism": "1 GPU" if world == 1 else f"{world} independent replicas",
+            "parallelism": "1 GPU" if world == 1 else f"{world} independent replicas (--replicas)",
             "launch": "CUDA graph replay (step graph, event, gather graph), captured through the C ABI"
                       if args.graph else "eager launches through the C ABI",
         },
@@ -573,31 +606,42 @@ def run_ours(args, world, rank, local):
 
 
 def e2e(b, args, stream, world):
-    """The same metric through the C ABI with host buffers: every step copies
-    its R gradient replicas from pinned host memory and reads the step's
-    result (the loss-scale state: overflow, skip, scale, grad norm) back.
-    The replicas are double-buffered where a second set fits: step s+1's
-    upload runs on a copy stream while step s computes (with graphs, one step
-    graph per buffer set); every copy is inside the timed region."""
+    """The same metric through the C ABI with host buffers. Every step
+    copies its R gradient replicas from pinned host memory, runs the step and
+    the gathers, and reads the step's products back to pinned host memory:
+    the updated half parameters of every shard (the model the next forward
+    uses) and the loss-scale state (overflow, skip, scale, grad norm; this
+    read synchronizes). The replicas are double-buffered where a second set
+    fits: step s+1's upload runs on one copy stream while step s computes
+    (with graphs, one step graph per buffer set), and step s's parameters go
+    down on a second copy stream while step s+1 computes. Every copy is
+    inside the timed region."""
     host = [g.cpu().pin_memory() for g in b.grads]
+    half = b.grads[0].dtype
+    host_param = [torch.empty(b.S, dtype=half).pin_memory() for _ in range(b.R)]
     K = max(3, min(args.steps, 10))
     nbytes = sum(h.numel() * h.element_size() for h in host)
+    dbytes = sum(h.numel() * h.element_size() for h in host_param) + 40
     graphs = getattr(b, "graphs", None)
     room = torch.cuda.mem_get_info()[0] > 1.25 * nbytes
     bufs = [b.grads] if not room else [b.grads, [torch.empty_like(g) for g in b.grads]]
     if graphs and len(bufs) == 2:
         b.capture_step(stream, bufs[1])
-    copy = torch.cuda.Stream()
+    up, down = torch.cuda.Stream(), torch.cuda.Stream()
     copied = [torch.cuda.Event() for _ in bufs]
     consumed = [torch.cuda.Event() for _ in bufs]
+    downloaded = [torch.cuda.Event() for _ in range(2)]
+    # a step writes set 1-cur (two sets) or set cur (one): the download that
+    # reads those parameters, step s-2's or step s-1's, must be done first
+    lag = 2 if b.state.sets == 2 else 1
 
     def upload(i):
         k = i % len(bufs)
-        copy.wait_event(consumed[k])  # the step that last read this buffer is done
-        with torch.cuda.stream(copy):
+        up.wait_event(consumed[k])  # the step that last read this buffer is done
+        with torch.cuda.stream(up):
             for r in range(b.R):
                 bufs[k][r].copy_(host[r], non_blocking=True)
-        copied[k].record(copy)
+        copied[k].record(up)
 
     def run(n):
         for i in range(min(len(bufs), n)):
@@ -605,11 +649,19 @@ def e2e(b, args, stream, world):
         for i in range(n):
             k = i % len(bufs)
             stream.wait_event(copied[k])
+            if i >= lag:
+                stream.wait_event(downloaded[(i - lag) % 2])
             b.step(stream, grads=bufs[k])
             consumed[k].record(stream)
-            b.loss_scale(stream)  # synchronizes the stream: the result is on the host
+            cur = b.loss_scale(stream)["cur"]  # synchronizes: the state is on the host
+            down.wait_stream(stream)
+            with torch.cuda.stream(down):
+                for r in range(b.R):
+                    host_param[r].copy_(b.state.param[cur][r], non_blocking=True)
+            downloaded[i % 2].record(down)
             if i + len(bufs) < n:
                 upload(i + len(bufs))
+        stream.wait_stream(down)  # the last parameters are on the host
 
     for e in consumed:
         e.record(stream)
@@ -622,10 +674,12 @@ def e2e(b, args, stream, world):
     end.record(stream)
     torch.cuda.synchronize()
     ms, units = aggregate(start.elapsed_time(end), float(b.P) * K, world)
-    return {"value": units / (ms * 1e-3), "unit": "params/s", "h2d_bytes_per_step": nbytes,
-            "d2h_bytes_per_step": 40, "steps": K,
-            "pipelining": "double-buffered replicas: step s+1 uploads during step s"
-                          if len(bufs) == 2 else "none (no room for a second set of replicas)"}
+    return {"value": units / (ms * 1e-3), "unit": "params/s", "h2d_bytes_per_step": nbytes * world,
+            "d2h_bytes_per_step": dbytes * world, "steps": K,
+            "d2h": "updated half parameters of every shard (2 B x T) + loss-scale state (40 B)",
+            "pipelining": ("double-buffered replicas: step s+1 uploads during step s; step s's "
+                           "parameters download during step s+1") if len(bufs) == 2
+                          else "parameters download during the next step; one set of replicas"}
 
 
 # ---- the CPU oracle as a baseline ----------------------------------------------
@@ -943,6 +997,56 @@ def run_rs_sweep(args, world, rank, local):
         print(json.dumps(out), flush=True)
 
 
+def dist_layer_buckets(layers, cap):
+    """Consecutive layers gathered in one launch, up to `cap` elements (a
+    larger layer alone) and 64 layers; each layer lands in its own
+    16-byte-aligned slice of one bucket buffer. Returns [(first, offsets, size)]."""
+    buckets, first, size, offs = [], 0, 0, []
+    for l, (lo, hi) in enumerate(layers):
+        n = hi - lo
+        if offs and (size + n > cap or len(offs) == 64):
+            buckets.append((first, offs, size))
+            first, size, offs = l, 0, []
+        offs.append(size)
+        size += (n + 7) // 8 * 8
+    buckets.append((first, offs, size))
+    return buckets
+
+
+def dist_step_bytes(T, S, N):
+    """Algorithmic bytes of one rank's share of the sharded step.
+    hbm: the fused launch reads the rank's own replica slice and serves its
+    N - 1 peers theirs (2N S), reads and writes its state (26 S); the gathers
+    read every rank's parameter slice (2T across all ranks, each rank
+    serving its own 2S to N readers: 2N S) and write the whole model (2T).
+    nvlink: the bytes the rank reads from its peers (per direction, the same
+    amount it serves them): 2(N - 1) S in the step, 2(N - 1) S in the gathers."""
+    step_hbm = (2 * N + 26) * S
+    gather_hbm = 2 * N * S + 2 * T
+    nvlink_step = 2 * (N - 1) * S
+    nvlink_gather = 2 * (N - 1) * S
+    return {"step_hbm": step_hbm, "gather_hbm": gather_hbm, "nvlink_step": nvlink_step,
+            "nvlink_gather": nvlink_gather}
+
+
+NVLINK_PEER_GBS = 770.0  # measured peer copy per direction on this part (900 nominal)
+
+
+def dist_roofline(nbytes, ms, peak_hbm):
+    """The slower of the HBM stream and the NVLink reads bounds a sharded
+    launch; achieved is that resource's bytes over the measured time."""
+    t_hbm = nbytes["hbm"] / (peak_hbm * 1e9)
+    t_nvl = nbytes["nvlink"] / (NVLINK_PEER_GBS * 1e9)
+    if nbytes["nvlink"] > 0 and t_nvl > t_hbm:
+        achieved = nbytes["nvlink"] / (ms * 1e-3) / 1e9
+        return {"bound": "nvlink", "achieved": achieved, "peak": NVLINK_PEER_GBS,
+                "peak_source": "measured peer copy per direction", "unit": "GB/s",
+                "frac": achieved / NVLINK_PEER_GBS, "target_ms": 1e3 * t_nvl}
+    achieved = nbytes["hbm"] / (ms * 1e-3) / 1e9
+    return {"bound": "hbm", "achieved": achieved, "peak": peak_hbm, "unit": "GB/s",
+            "frac": achieved / peak_hbm, "target_ms": 1e3 * t_hbm}
+
+
 def run_dist(args, world, rank, local):
     """The real multi-GPU ZeRO step (DistributedZero): the workload's tensors
     sharded over the N GPUs of the job, each rank owning one shard and reading
@@ -954,7 +1058,7 @@ def run_dist(args, world, rank, local):
     import synth
     from zero_partitioned_mixed_reduce_b200.dist import DistributedZero
     if not torch.cuda.is_available():
-        print(json.dumps({"error": "no CUDA device"}))
+        print(json.dumps({"error": "no CUDA device: the benchmark has no CPU fallback"}))
         sys.exit(1)
     if not dist.is_initialized():  # one process: a group of one
         with socket.socket() as sk:
@@ -965,9 +1069,13 @@ def run_dist(args, world, rank, local):
         dist.init_process_group("nccl", rank=0, world_size=1, timeout=datetime.timedelta(seconds=300))
     N = dist.get_world_size()
     wl = synth.workload(args.workload)
+    if args.first_tensors:
+        wl["numels"] = wl["numels"][:args.first_tensors]
+        wl["layer_ids"] = wl["layer_ids"][:args.first_tensors] if wl["layer_ids"] else None
     dz = DistributedZero(wl["numels"], wl["layer_ids"], wl["dtype"], wl["mode"], wl["init_scale"],
                          wl["interval"], 8, wl["bucket_elems"])
     plan = dz.plan
+    T, S = plan.T, plan.S
     half = {0: torch.bfloat16, 1: torch.float16}[wl["dtype"]]
     x = torch.cat([synth.tensor_master(n, wl["index"], k, "cuda") for k, n in enumerate(wl["numels"])])
     dz.load(plan.pack(x), plan.pack(x.to(half)))
@@ -978,15 +1086,7 @@ def run_dist(args, world, rank, local):
                                                    1, dz.rank, k, "cuda")
     torch.cuda.synchronize()
     # ZeRO-3 gathers of every layer, bucketed as in the single-GPU step
-    buckets, first, size, offs = [], 0, 0, []
-    for l, (lo, hi) in enumerate(plan.layers):
-        n = hi - lo
-        if offs and (size + n > args.gather_bucket or len(offs) == 64):
-            buckets.append((first, offs, size))
-            first, size, offs = l, 0, []
-        offs.append(size)
-        size += (n + 7) // 8 * 8
-    buckets.append((first, offs, size))
+    buckets = dist_layer_buckets(plan.layers, args.gather_bucket if args.gather_bucket > 0 else 1)
     layer_buf = torch.empty(max(b[2] for b in buckets), dtype=half, device="cuda")
     outs = [[layer_buf.data_ptr() + 2 * o for o in offs] for _, offs, _ in buckets]
     hp = wl["hp"]
@@ -1000,13 +1100,15 @@ def run_dist(args, world, rank, local):
             ev[1].record(stream)
         for (f, _, _), o in zip(buckets, outs):
             dz.gather_layers(f, o)
+        if ev is not None:
+            ev[2].record(stream)
 
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize()
     f0 = dz.loss_scale()
     K = args.steps
-    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    evs = [tuple(torch.cuda.Event(enable_timing=True) for _ in range(3)) for _ in range(K)]
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     clocks = ClockSampler(local)
     clocks.start()
@@ -1020,36 +1122,82 @@ def run_dist(args, world, rank, local):
     dist.barrier()
     clk = clocks.stop()
     f1 = dz.loss_scale()
-    assert f1["last_overflow"] == 0 and f1["t"] == f0["t"] + K
+    ok = f1["last_overflow"] == 0 and f1["t"] == f0["t"] + K
     ms, units = aggregate(start.elapsed_time(end), float(plan.P) * K / N, N)
-    step_ms, _ = aggregate(statistics.mean(e0.elapsed_time(e1) for e0, e1 in evs), 0.0, N)
-    S = plan.S
-    kbytes = (2 * N + 26) * S  # one rank's fused launch: N replica slices, its own state
+    step_ms, _ = aggregate(statistics.mean(e0.elapsed_time(e1) for e0, e1, _ in evs), 0.0, N)
+    gather_ms, _ = aggregate(statistics.mean(e1.elapsed_time(e2) for _, e1, e2 in evs), 0.0, N)
+    nb = dist_step_bytes(T, S, N)
     peak, peak_src = hbm_peak()
+    roof = dist_roofline({"hbm": nb["step_hbm"], "nvlink": nb["nvlink_step"]}, step_ms, peak)
+    roof.update({"kernel": "fused_step_kernel (sharded: one owner per rank) + loss-scale commit",
+                 "traffic": None, "algorithmic_bytes_per_launch": nb["step_hbm"], "avg_launch_ms": step_ms})
+    roof.setdefault("peak_source", f"{peak_src} hbm_gbs")
+    e2e_out = None if args.no_e2e else dist_e2e(dz, step, args, stream, N)
     out = {
-        "mode": "distributed", "metric": METRIC, "value": units / (ms * 1e-3), "unit": "params/s",
+        "metric": METRIC, "value": units / (ms * 1e-3), "unit": "params/s",
         "n_gpus": N, "steps": K, "warmup": args.warmup, "ms_per_step": ms / K, "higher_is_better": True,
-        "scaling": "strong", "dtype": "f32", "data": "synthetic",
-        "config": {"workload": f"{args.workload}: {len(wl['numels'])} tensors, P={plan.P}, sharded over "
-                               f"{N} rank(s), one per GPU, {'fp16' if wl['dtype'] else 'bf16'} grads, "
-                               f"loss scale mode {wl['mode']}",
-                   "R": N, "P": plan.P, "S": S,
-                   "parallelism": f"{N} GPU(s), one shard each (DistributedZero: fused step reading the "
-                                  "peers' replicas over NVLink, NCCL for 4-16 byte all-reduces)",
-                   "gather": f"{len(buckets)} bucketed launches per step over every rank's shard"},
-        "step_ms_max_over_ranks": step_ms,
-        "per_rank_step_bytes": kbytes, "per_rank_nvlink_bytes": 2 * (N - 1) * S,
-        "per_rank_step_gbs": kbytes / (step_ms * 1e-3) / 1e9, "peak": peak,
-        "peak_source": f"{peak_src} hbm_gbs", "clocks": clk,
-        # the slower of the HBM stream and the NVLink reads (770 GB/s per direction,
-        # the machine's measured peer copy) bounds the step
-        "roofline": {"bound": "nvlink" if 2 * (N - 1) * S / 770e9 > kbytes / (peak * 1e9) else "hbm",
-                     "target_ms": 1e3 * max(kbytes / (peak * 1e9), 2 * (N - 1) * S / 770e9),
-                     "frac": 1e3 * max(kbytes / (peak * 1e9), 2 * (N - 1) * S / 770e9) / step_ms},
+        "scaling": "strong", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "config": {"workload": workload_label(args.workload, wl, args.first_tensors).split(", R=")[0]
+                               + f", sharded over {N} rank(s), one per GPU",
+                   "R": N, "P": plan.P, "T": T, "S": S, "n_layers": len(plan.layers),
+                   "path": "DistributedZero: 4-byte NCCL all-reduce (every replica written), fused "
+                           "reduce-scatter+AdamW over the rank's shard reading the peers' replicas over "
+                           "NVLink (plain or 1-D bulk loads, no multicast), 16-byte NCCL all-reduce of "
+                           "{norm, overflow}, loss-scale commit, ZeRO-3 gather of every layer from every "
+                           "rank's shard",
+                   "l2": f"inputs larger than L2 ({(nb['step_hbm'] + nb['gather_hbm']) / 1e9:.1f} GB "
+                         "of HBM per rank per step, L2 126 MB)",
+                   "parallelism": f"dp{N}: {N} GPU(s), one shard each",
+                   "gather": f"{len(buckets)} bucketed launches per step over every rank's shard",
+                   "launch": "eager (the step issues NCCL all-reduces between its launches)"},
+        "roofline": roof,
+        "gather": {"avg_ms_per_step": gather_ms, "elements": plan.L, "launches_per_step": len(buckets),
+                   "roofline": dist_roofline({"hbm": nb["gather_hbm"], "nvlink": nb["nvlink_gather"]},
+                                             gather_ms, peak)},
+        "per_rank_bytes": nb,
+        "nccl": {"backend": dist.get_backend(), "world_size": N,
+                 "version": ".".join(str(v) for v in torch.cuda.nccl.version())},
+        "clocks": clk,
+        "gpu_launches": K * (2 + len(buckets)),
+        "state_check": "ok" if ok else f"t {f0['t']} -> {f1['t']}, overflow {f1['last_overflow']}",
     }
+    if e2e_out is not None:
+        out["e2e"] = e2e_out
     dz.close()
     if rank == 0:
         print(json.dumps(out), flush=True)
+
+
+def dist_e2e(dz, step, args, stream, N):
+    """The sharded step through the public API with host buffers: every rank
+    uploads its gradient replica from pinned host memory, runs the step and
+    the gathers, and reads back its updated parameter shard and the loss-scale
+    state (which synchronizes). Time: max over ranks."""
+    import torch.distributed as dist
+    host_g = dz.grads.cpu().pin_memory()
+    host_p = torch.empty(dz.plan.S, dtype=dz.grads.dtype).pin_memory()
+    K = max(3, min(args.steps, 10))
+
+    def one():
+        dz.grads.copy_(host_g, non_blocking=True)
+        step()
+        host_p.copy_(dz.current("param"), non_blocking=True)
+        dz.loss_scale()
+
+    one()
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    dist.barrier()
+    torch.cuda.synchronize()
+    start.record(stream)
+    for _ in range(K):
+        one()
+    end.record(stream)
+    torch.cuda.synchronize()
+    ms, units = aggregate(start.elapsed_time(end), float(dz.plan.P) * K / N, N)
+    return {"value": units / (ms * 1e-3), "unit": "params/s",
+            "h2d_bytes_per_step": host_g.numel() * host_g.element_size() * N,
+            "d2h_bytes_per_step": (host_p.numel() * host_p.element_size() + 40) * N, "steps": K,
+            "pipelining": "none: each rank uploads, steps, gathers and reads back in turn"}
 
 
 def run_offload(args, world, rank, local):
@@ -1274,19 +1422,42 @@ def run_reference(args, world, rank):
     print(json.dumps(out), flush=True)
 
 
+def choose_mode(args, world):
+    """The measurement a command line asks for. With N > 1 GPUs the default
+    is the real sharded step over the job (DistributedZero); `--replicas`
+    keeps N independent single-GPU copies instead."""
+    if args.impl == "reference":
+        return "reference"
+    if args.overlap:
+        return "overlap"
+    if args.offload:
+        return "offload"
+    if args.rs_sweep:
+        return "rs_sweep"
+    if args.dist or (world > 1 and not args.replicas):
+        return "dist"
+    return "single"
+
+
 def main(argv=None):
     args = parse_args(argv)
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    mode = choose_mode(args, world)
+    if mode == "dist" and world > 1 and "NCCL_DEBUG" not in os.environ:
+        # the communicators' set-up lines (ranks, devices, transports) on stderr,
+        # so that a log shows how many ranks the step ran over
+        os.environ.update(NCCL_DEBUG="INFO", NCCL_DEBUG_SUBSYS="INIT", NCCL_DEBUG_FILE="/dev/stderr")
     world, rank, local = dist_init()
     try:
-        if args.impl == "reference":
+        if mode == "reference":
             run_reference(args, world, rank)
-        elif args.overlap:
+        elif mode == "overlap":
             run_overlap(args, world, rank, local)
-        elif args.offload:
+        elif mode == "offload":
             run_offload(args, world, rank, local)
-        elif args.rs_sweep:
+        elif mode == "rs_sweep":
             run_rs_sweep(args, world, rank, local)
-        elif args.dist:
+        elif mode == "dist":
             run_dist(args, world, rank, local)
         else:
             run_ours(args, world, rank, local)

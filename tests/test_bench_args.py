@@ -4,7 +4,8 @@ import bench
 
 def test_defaults():
     a = bench.parse_args([])
-    assert a.gpus == 1 and a.impl == "ours" and a.workload == "gpt2s"
+    # the largest configuration that fits one GPU: the Llama-style 3B list, R = 4
+    assert a.gpus == 1 and a.impl == "ours" and a.workload == "llama3b"
     assert a.warmup >= 3 and a.steps >= 1
     assert a.graph is True  # CUDA-graph replay of the captured step by default
     assert a.clip_norm == "rs"
@@ -31,3 +32,44 @@ def test_oracle_crew_runs_the_oracle_on_several_processes():
     finally:
         crew.close()
     assert rate > 0 and sec > 0 and crew.procs == 2
+
+
+def test_mode_routing():
+    # one GPU: the single-GPU step; N > 1: the sharded step over the job's
+    # GPUs unless --replicas asks for independent copies
+    p = bench.parse_args
+    assert bench.choose_mode(p([]), 1) == "single"
+    assert bench.choose_mode(p(["--gpus", "8"]), 8) == "dist"
+    assert bench.choose_mode(p(["--gpus", "8", "--replicas"]), 8) == "single"
+    assert bench.choose_mode(p(["--dist"]), 1) == "dist"
+    assert bench.choose_mode(p(["--impl", "reference", "--gpus", "4"]), 4) == "reference"
+    assert bench.choose_mode(p(["--rs-sweep"]), 1) == "rs_sweep"
+
+
+def test_bucket_runs_cover_every_bucket_once_in_order():
+    buckets = [(90, 100), (60, 90), (59, 60), (10, 59), (0, 10)]  # reverse flat order
+    for group in (0, 1, 10, 31, 40, 1000):
+        runs = bench.bucket_runs(buckets, group)
+        covered = [b for first, count in runs for b in range(first, first + count)]
+        assert covered == list(range(len(buckets)))
+        for first, count in runs:
+            n = sum(hi - lo for lo, hi in buckets[first:first + count])
+            assert count == 1 or n <= group
+    assert bench.bucket_runs(buckets, 0) == [(b, 1) for b in range(5)]
+    assert bench.bucket_runs(buckets, 1000) == [(0, 5)]
+    assert bench.bucket_runs(buckets, 40) == [(0, 2), (2, 1), (3, 1), (4, 1)]
+    assert bench.bucket_runs(buckets, 60) == [(0, 3), (3, 2)]
+
+
+def test_dist_bytes_and_roofline():
+    T, N = 8 * 1000, 4
+    S = T // N
+    nb = bench.dist_step_bytes(T, S, N)
+    assert nb["step_hbm"] == (2 * N + 26) * S and nb["nvlink_step"] == 2 * (N - 1) * S
+    assert nb["gather_hbm"] == 2 * N * S + 2 * T and nb["nvlink_gather"] == 2 * (N - 1) * S
+    # NVLink-bound when its bytes take longer at 770 GB/s than the HBM bytes at peak
+    r = bench.dist_roofline({"hbm": 1e9, "nvlink": 1e9}, 2.0, 6000.0)
+    assert r["bound"] == "nvlink" and abs(r["achieved"] - 500.0) < 1e-9
+    assert abs(r["frac"] - 500.0 / bench.NVLINK_PEER_GBS) < 1e-12
+    r = bench.dist_roofline({"hbm": 6e9, "nvlink": 0}, 1.0, 6000.0)
+    assert r["bound"] == "hbm" and abs(r["frac"] - 1.0) < 1e-12

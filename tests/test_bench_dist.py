@@ -1,5 +1,6 @@
 """The benchmark's multi-rank path on CPU with gloo, world size 2: the
-whole-job aggregation (max of the per-rank times, sum of the units) and the
+routing (N > 1 runs the sharded step), the whole-job aggregation (max of the
+per-rank times, sum of the units) as the sharded step reports it, and the
 reference arm under torch.distributed.run (rank 0 alone works and prints)."""
 import datetime
 import json
@@ -30,7 +31,13 @@ def _worker(rank, world, port, q):
     try:
         ms, units = bench.aggregate(10.0 + rank, 100.0 * (rank + 1), world)
         bench.barrier(world)
-        q.put((rank, ms, units))
+        # the sharded step: every rank counts its P / N share of each of K
+        # steps; the job's rate is P * K over the slowest rank's time
+        args = bench.parse_args(["--gpus", str(world), "--steps", "7"])
+        mode = bench.choose_mode(args, world)
+        P, K = 1000, args.steps
+        dms, dunits = bench.aggregate(5.0 * (rank + 1), float(P) * K / world, world)
+        q.put((rank, ms, units, mode, dms, dunits))
     finally:
         dist.destroy_process_group()
 
@@ -46,8 +53,9 @@ def test_aggregate_max_time_sum_units_gloo():
         p.join(120)
         assert p.exitcode == 0
     got = sorted(q.get(timeout=10) for _ in range(2))
-    for rank, ms, units in got:
+    for rank, ms, units, mode, dms, dunits in got:
         assert ms == 11.0 and units == 300.0
+        assert mode == "dist" and dms == 10.0 and dunits == 7000.0
 
 
 def test_reference_arm_under_torchrun_two_ranks():
