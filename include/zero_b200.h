@@ -158,6 +158,22 @@ zero_status zero_plan_layer(const zero_plan_t* plan, int64_t l, int64_t* lo, int
  */
 zero_status zero_plan_memory(const zero_plan_t* plan, int32_t stage, int64_t* bytes_per_rank);
 
+/*
+ * zero_plan_step_tiles -- how the staged fused step (the kernel zero_step
+ * runs for R <= 2, whose reads are bulk copies into shared memory) cuts this
+ * plan's shards: each shard of S elements into *tiles_per_shard tiles of
+ * *tile_elems elements, the last tile of a shard holding the rest,
+ * S - (tiles_per_shard - 1) * tile_elems (a multiple of 8, at least 8); the
+ * step's work is *tiles_total = R * tiles_per_shard tiles. Host arithmetic
+ * in 64 bits, the same the launch uses, so a shard longer than 2^32
+ * elements is tiled completely. Any output may be NULL.
+ * Defines: [instr] ZeRO-1/2 "Mechanism" bullets (each owner updates every
+ * element of its partition).
+ * Errors: ZERO_ERR_INVALID_ARG for a NULL plan.
+ */
+zero_status zero_plan_step_tiles(const zero_plan_t* plan, int64_t* tile_elems, int64_t* tiles_per_shard,
+                                 int64_t* tiles_total);
+
 /* ------------------------------------------------------------------------ */
 /* Context: device scratch and the loss-scale state.                        */
 /* ------------------------------------------------------------------------ */
@@ -600,10 +616,15 @@ zero_status zero_loss_scale(zero_ctx_t* ctx, zero_loss_scale_state* inout, int32
  * synchronize the device or can fail mid-run. This call allocates nothing
  * and needs no context: its scratch (the accumulators, the per-block norm
  * partials and a control word) lives in one static device array of
- * 16 MiB + 32 KiB + 256 B that every GPU loading this library holds until
- * the process exits. The pages have no counterpart to this entry point; it
- * is a deployment variant of zero_reduce_scatter_bucket(-1) + zero_step
- * (grads == NULL) and gives the same results.
+ * 16 MiB + 32 KiB + 256 B. A device reserves the array when the library's
+ * code module that holds it is loaded there; under CUDA's default lazy
+ * module loading that is the first zero_step_noalloc call on the device
+ * (its set-up, below), and the device then holds the array until the
+ * process exits. So make the first call on each device before another
+ * allocator has taken all of its memory; later calls reserve nothing. The
+ * pages have no counterpart to this entry point; it is a deployment variant
+ * of zero_reduce_scatter_bucket(-1) + zero_step (grads == NULL) and gives
+ * the same results.
  *
  * plan: the layout (host only); its padded length T must be at most
  * ZERO_NOALLOC_MAX_ELEMS, else ZERO_ERR_RANGE. cfg: loss-scale mode and
@@ -614,8 +635,9 @@ zero_status zero_loss_scale(zero_ctx_t* ctx, zero_loss_scale_state* inout, int32
  * pointers to the shards of S elements, updated in place.
  *
  * Set-up: the first call on each device (with that device current) looks up
- * the device address of the static scratch; make that first call before any
- * stream capture begins. Every call shares the same scratch and leaves the
+ * the device address of the static scratch, again after the device's
+ * context has been replaced (a device reset); make that first call before
+ * any stream capture begins. Every call shares the same scratch and leaves the
  * last call's contents in it (the control word is cleared at the start of
  * each call). Calls whose work overlaps on the GPU -- two streams, two host
  * threads, or two devices' calls racing on one device -- race on the

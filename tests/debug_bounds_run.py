@@ -56,6 +56,18 @@ def main():
                 runs += 1
             finally:
                 c.close()
+    # the static-scratch step (zero_step_noalloc): R = 3 with packed tensors
+    # and a skipped step, and R = 16
+    for R, align, mode, dtype in ((3, 1, O.SCALE_DYNAMIC, O.FP16), (16, 8, O.SCALE_STATIC, O.BF16)):
+        c = Case(numels, R, dtype, align, mode, init_scale=256.0, interval=2, path="inplace",
+                 layer_ids=layers, seed=R + 100)
+        try:
+            for s in range(3):
+                c.step_noalloc(inject=[(1, 5, 0x7C00)] if (s == 1 and mode == O.SCALE_DYNAMIC) else None)
+                c.compare(fsm=c.noalloc_ls)
+            runs += 1
+        finally:
+            c.close()
     count, site, index = Z.zero_debug_bounds()
     print(json.dumps({"cases": runs, "count": count, "first_site": site, "first_index": index}))
 

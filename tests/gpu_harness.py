@@ -70,6 +70,7 @@ class Case:
         self.wl = synth.custom_workload(numels, R, dtype, mode, init_scale, interval, sigma,
                                         layer_ids=layer_ids, bucket_elems=bucket_elems, index=seed)
         self.R, self.dtype, self.mode, self.path = R, dtype, mode, path
+        self.init_scale, self.interval = init_scale, interval
         self.hp = hp or self.wl["hp"]
         self.lay = O.Layout(numels, R, align, bucket_elems, layer_ids)
         self.plan = Z.Plan(numels, layer_ids, R, dtype, align, bucket_elems)
@@ -135,6 +136,30 @@ class Case:
             Z.zero_step(self.ctx, self.hp, self.handle, None)
         else:
             Z.zero_step(self.ctx, self.hp, self.handle, self.grads)
+        skipped = O.step(self.ostate, g, O.AdamW(**{k: self.hp[k] for k in
+                                                    ("lr", "beta1", "beta2", "eps",
+                                                     "weight_decay")}), self.ofsm)
+        self.g.check()
+        return skipped
+
+    def step_noalloc(self, inject=None):
+        """The two-pass step through zero_step_noalloc (all scratch in the
+        library's static array, no context; the loss-scale state lives on
+        the host in self.noalloc_ls) on set 0, against the oracle."""
+        assert self.path == "inplace"
+        self.step_no += 1
+        g = self.make_grads(inject)
+        for r in range(self.R):
+            gp = np.zeros(self.plan.T, np.uint16)
+            gp[self.idx] = g[r]
+            self.grads[r].view(torch.int16).copy_(torch.from_numpy(gp.view(np.int16)))
+        if not hasattr(self, "noalloc_ls"):
+            self.noalloc_ls = dict(scale=self.init_scale if self.mode != O.SCALE_NONE else 1.0,
+                                   cur=0, good=0, t=0)
+        cfg = dict(mode=self.mode, growth_interval=self.interval, growth_factor=2.0,
+                   backoff_factor=0.5, min_scale=1.0)
+        self.noalloc_ls = Z.zero_step_noalloc(self.plan.handle, cfg, self.noalloc_ls, self.hp, self.grads,
+                                              self.master[0], self.m[0], self.v[0], self.param[0])
         skipped = O.step(self.ostate, g, O.AdamW(**{k: self.hp[k] for k in
                                                     ("lr", "beta1", "beta2", "eps",
                                                      "weight_decay")}), self.ofsm)
@@ -377,8 +402,8 @@ class Case:
     def gpu_fsm(self):
         return Z.zero_loss_scale(self.ctx)
 
-    def gpu_state(self):
-        cur = self.gpu_fsm()["cur"]
+    def gpu_state(self, cur=None):
+        cur = self.gpu_fsm()["cur"] if cur is None else cur
         k = cur if self.sets == 2 else 0
         idx = self.idx
         cat = lambda bufs: torch.cat([b for b in bufs]).cpu()
@@ -392,9 +417,10 @@ class Case:
                     pad_master=cat(self.master[k]).numpy()[pads],
                     pad_param=u16(torch.cat(self.param[k]))[pads])
 
-    def compare(self, exact=True):
-        """Assert parity with the oracle after the last step."""
-        f = self.gpu_fsm()
+    def compare(self, exact=True, fsm=None):
+        """Assert parity with the oracle after the last step; fsm: the
+        loss-scale state to check (default: the context's)."""
+        f = self.gpu_fsm() if fsm is None else fsm
         o = self.ofsm
         assert (f["t"], f["good"], f["last_overflow"], f["last_skipped"]) == \
                (o.t, o.good, o.last_overflow, o.last_skipped), (f, o.t, o.good)
@@ -403,7 +429,7 @@ class Case:
             assert abs(f["grad_norm_sq"] - o.grad_norm_sq) <= 1e-9 * abs(o.grad_norm_sq) + 1e-300
         else:
             assert not np.isfinite(f["grad_norm_sq"])
-        s = self.gpu_state()
+        s = self.gpu_state(f["cur"])
         st = self.ostate
         for name in ("master", "m", "v"):
             a, b = s[name], getattr(st, name)

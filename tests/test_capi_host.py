@@ -179,3 +179,18 @@ def test_every_declared_function_has_a_binding_of_the_same_name():
     names = sorted(set(re.findall(r"^\w[\w\s\*]*?\b(zero_\w+)\s*\(", hdr, re.M)))
     assert len(names) >= 40
     assert [n for n in names if not callable(getattr(Z, n, None))] == []
+
+
+@pytest.mark.parametrize("R,P", [(1, (1 << 32) + 8), (2, (1 << 33) + 24), (1, 5), (2, 4097)])
+def test_staged_step_tiles_cover_long_shards(R, P):
+    # shards of 2^32 + 8 and more elements (R = 1 at 34 GB of half gradients,
+    # R = 2 at 8.6 G params): the staged step's tiles, in 64-bit arithmetic,
+    # cover every element of every shard; host only, nothing is allocated
+    p = Z.Plan([P], None, R, 0, 8, 0)
+    tile, tps, total = Z.zero_plan_step_tiles(p.handle)
+    assert tile == 2048 and total == R * tps
+    assert (tps - 1) * tile < p.S <= tps * tile
+    last = p.S - (tps - 1) * tile
+    assert 8 <= last <= tile and last % 8 == 0
+    if P == (1 << 32) + 8:
+        assert p.S == (1 << 32) + 8 and tps == (1 << 21) + 1 and last == 8

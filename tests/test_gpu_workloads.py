@@ -257,6 +257,12 @@ def test_llama3b_two_pass_50M_buckets():
     run("llama3b", "twopass")
 
 
+def test_llama3b_fused_pingpong_with_layer_gathers():
+    # the benchmark's default configuration: 3,606,752,256 params, R = 4, bf16,
+    # the fused step on ping-pong state (130 GB resident), and every layer gathered
+    run("llama3b", "pingpong", gather=True)
+
+
 def test_irregular_r16():
     run("irr_r16", "pingpong", gather=True)
 

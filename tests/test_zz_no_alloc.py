@@ -6,10 +6,14 @@ training loop that must not allocate or free once it runs (cudaFree
 synchronizes the whole device, and an allocation can fail mid-run). For them
 zero_step_noalloc runs the two-pass step with all of its scratch in a static
 device array inside the library and no context. These tests check, through
-the C ABI, that two calls in a row give the same model state and loss-scale
-state as the context-based two-pass path (zero_reduce_scatter_bucket over the
-whole range + zero_step from the accumulators), bit for bit on the model
-state and within the parity tests' bound on the gradient norm.
+the C ABI, on two and more calls in a row:
+  - the model state and loss-scale state equal the context-based two-pass
+    path (zero_reduce_scatter_bucket over the whole range + zero_step from
+    the accumulators) bit for bit, and the gradient norm within the parity
+    tests' bound, including a model whose padded length is exactly the
+    static scratch's limit and an overflow under static and dynamic scaling;
+  - the same state equals the oracle's step on the same bytes;
+  - the calls after the first allocate no device memory.
 
 The file is named so that pytest collects it last.
 """
@@ -17,9 +21,15 @@ import numpy as np
 import pytest
 import torch
 
+import oracle as O
+
 pytestmark = pytest.mark.gpu
 
 HALF = {0: torch.bfloat16, 1: torch.float16}
+MAX = 4194304  # ZERO_NOALLOC_MAX_ELEMS
+# a two-tensor list whose padded length at R = 16 is exactly MAX: L = 4,194,298
+# (the second tensor starts at the 8-aligned 4,194,208), S = 262,144
+AT_LIMIT = [MAX - 100, 90]
 
 
 def _state(plan, master0, param0, device="cuda"):
@@ -38,14 +48,24 @@ def _bits(ts):
                       for t in ts]).cpu().numpy()
 
 
-@pytest.mark.parametrize("dtype,mode", [(1, 2), (0, 1), (0, 0)])
-def test_noalloc_matches_context_two_pass(dtype, mode):
+# (numels, R, dtype, mode, the call whose replica 1 carries an inf)
+CASES = [
+    ([70_001, 13, 4096, 777, 5], 4, 1, 2, 2),  # fp16, dynamic: call 2 is skipped and backs off
+    ([70_001, 13, 4096, 777, 5], 4, 0, 1, None),  # bf16, static scale
+    ([70_001, 13, 4096, 777, 5], 4, 0, 0, None),  # bf16, no scaling
+    (AT_LIMIT, 16, 0, 1, 2),  # at the size limit; static mode applies the non-finite step
+]
+
+
+@pytest.mark.parametrize("numels,R,dtype,mode,inf_call", CASES)
+def test_noalloc_matches_context_two_pass(numels, R, dtype, mode, inf_call):
     import zero_partitioned_mixed_reduce_b200 as Z
     import synth
 
-    numels, R = [70_001, 13, 4096, 777, 5], 4
     plan = Z.Plan(numels, None, R, dtype, 8, 0)
-    assert plan.T <= Z.ZERO_NOALLOC_MAX_ELEMS
+    assert plan.T <= Z.ZERO_NOALLOC_MAX_ELEMS == MAX
+    if numels is AT_LIMIT:
+        assert plan.T == MAX
     wl = synth.custom_workload(numels, R, dtype, mode, 256.0, 3, sigma=1e-2, index=77)
     x = plan.pack(synth.flat_master(wl, "cuda"))
     p0 = x.to(HALF[dtype])
@@ -57,17 +77,28 @@ def test_noalloc_matches_context_two_pass(dtype, mode):
     ctx = Z.zero_ctx_create(plan.handle, mode, init, 3)
     cfg = dict(mode=mode, growth_interval=3, growth_factor=2.0, backoff_factor=0.5, min_scale=1.0)
     ls = dict(scale=init, cur=0, good=0, t=0)
+    calls = (1, 2, 3)
+    # every input of every call exists before the first call, so that nothing
+    # else allocates device memory between the calls; the replicas are drawn
+    # at the initial scale (the skipped call's backoff does not change them)
+    grads = {c: [plan.pack(synth.flat_grads(wl, c, r, init, "cuda")) for r in range(R)] for c in calls}
+    if inf_call:
+        grads[inf_call][1][plan.offsets[-1] + 3] = float("inf")
+    free = {}
     try:
-        for call in (1, 2):
-            grads = [plan.pack(synth.flat_grads(wl, call, r, ls["scale"] if mode else 1.0, "cuda"))
-                     for r in range(R)]
-            if call == 2 and mode == 2:  # the second call overflows and must be skipped
-                grads[1][plan.offsets[2] + 9] = float("inf")
-            Z.zero_reduce_scatter_bucket(ctx, -1, grads, acc)
+        for call in calls:
+            Z.zero_reduce_scatter_bucket(ctx, -1, grads[call], acc)
             Z.zero_step(ctx, wl["hp"], handle, None)
             want = Z.zero_loss_scale(ctx)
-            ls = Z.zero_step_noalloc(plan.handle, cfg, ls, wl["hp"], grads, new["master"],
+            torch.cuda.synchronize()
+            free[call] = torch.cuda.mem_get_info()[0]
+            ls = Z.zero_step_noalloc(plan.handle, cfg, ls, wl["hp"], grads[call], new["master"],
                                      new["m"], new["v"], new["param"])
+            torch.cuda.synchronize()
+            if call > 1:
+                # the second and later calls take no device memory: the static
+                # array was reserved by the first call's set-up, if not before
+                assert torch.cuda.mem_get_info()[0] == free[call], (call, free[call])
             for f in ("master", "m", "v", "param"):
                 assert np.array_equal(_bits(ref[f]), _bits(new[f])), (call, f)
             for k in ("t", "good", "last_overflow", "last_skipped", "cur"):
@@ -80,9 +111,31 @@ def test_noalloc_matches_context_two_pass(dtype, mode):
             else:
                 assert not np.isfinite(a)
         if mode == 2:
-            assert ls["last_skipped"] == 1 and ls["scale"] == 128.0 and ls["t"] == 1
+            assert ls["last_overflow"] == 0 and ls["t"] == 2 and ls["scale"] == 128.0
+        if mode == 1 and inf_call:
+            assert want["last_overflow"] == 0 and want["t"] == 3  # static mode never skips
     finally:
         Z.zero_ctx_destroy(ctx)
+
+
+@pytest.mark.parametrize("numels,R,dtype,align,mode", [
+    ([70_001, 13, 4096, 777, 5], 3, 1, 1, 2),  # R = 3, packed tensors, dynamic scaling with a skip
+    (AT_LIMIT, 16, 0, 8, 1),  # at the size limit, static scaling with an overflow
+])
+def test_noalloc_matches_the_oracle(numels, R, dtype, align, mode):
+    from gpu_harness import Case
+    c = Case(numels, R, dtype, align, mode, init_scale=256.0, interval=2, path="inplace", seed=R + 40)
+    inf = 0x7C00 if dtype == O.FP16 else 0x7F80
+    try:
+        for call in (1, 2, 3):
+            c.step_noalloc(inject=[(1, 17, inf)] if call == 2 else None)
+            c.compare(fsm=c.noalloc_ls)
+        if mode == O.SCALE_DYNAMIC:
+            assert c.noalloc_ls["t"] == 2 and c.noalloc_ls["scale"] == 128.0
+        else:
+            assert c.noalloc_ls["t"] == 3 and c.noalloc_ls["last_skipped"] == 0
+    finally:
+        c.close()
 
 
 def test_noalloc_rejects_models_beyond_its_scratch():

@@ -13,7 +13,7 @@ from ._capi import (  # noqa: F401
     zero_adamw, zero_ctx_create, zero_ctx_destroy, zero_gather_layer, zero_gather_layers,
     ZERO_GATHER_MAX_LAYERS, zero_last_error,
     zero_loss_scale, zero_plan, zero_plan_bucket, zero_plan_destroy, zero_plan_get_info,
-    zero_plan_layer, zero_plan_memory, zero_plan_tensor, zero_reduce_scatter_bucket, zero_step,
+    zero_plan_layer, zero_plan_memory, zero_plan_step_tiles, zero_plan_tensor, zero_reduce_scatter_bucket, zero_step,
     zero_reduce_scatter_bucket_ex, zero_step_ex, ZERO_RS_ACCUMULATE, ZERO_STEP_ADD_ACC,
     zero_step_noalloc, ZERO_NOALLOC_MAX_ELEMS, zero_sync, zero_version, zero_grads_ready,
     zero_grads_join, zero_prefetch_begin, zero_layer_acquire, zero_layer_release, zero_cpu_step,

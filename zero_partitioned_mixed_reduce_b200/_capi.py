@@ -116,6 +116,7 @@ _sig("zero_plan_tensor", _S, [_P, C.c_int64, C.POINTER(C.c_int64), C.POINTER(C.c
 _sig("zero_plan_bucket", _S, [_P, C.c_int64, C.POINTER(C.c_int64), C.POINTER(C.c_int64)])
 _sig("zero_plan_layer", _S, [_P, C.c_int64, C.POINTER(C.c_int64), C.POINTER(C.c_int64)])
 _sig("zero_plan_memory", _S, [_P, C.c_int32, C.POINTER(C.c_int64)])
+_sig("zero_plan_step_tiles", _S, [_P, C.POINTER(C.c_int64), C.POINTER(C.c_int64), C.POINTER(C.c_int64)])
 _sig("zero_ctx_create", _S, [_P, C.POINTER(zero_loss_scale_config), C.POINTER(_P)])
 _sig("zero_ctx_destroy", _S, [_P])
 _sig("zero_ctx_reserve_steps", _S, [_P, C.c_int64, C.c_double, C.c_double, _P])
@@ -253,6 +254,13 @@ def zero_plan_memory(plan, stage):
     b = C.c_int64()
     _check(_lib.zero_plan_memory(plan, stage, C.byref(b)))
     return b.value
+
+
+def zero_plan_step_tiles(plan):
+    """(tile_elems, tiles_per_shard, tiles_total) of the staged fused step."""
+    e, t, n = C.c_int64(), C.c_int64(), C.c_int64()
+    _check(_lib.zero_plan_step_tiles(plan, C.byref(e), C.byref(t), C.byref(n)))
+    return e.value, t.value, n.value
 
 
 # ---- context ---------------------------------------------------------------

@@ -40,7 +40,7 @@ CPP_SOURCES = ["plan.cpp", "capi.cpp", "sched.cpp", "cpu_adam.cpp", "trace.cpp"]
 
 
 def _sources():
-    return ([os.path.join(CSRC, s) for s in CU_SOURCES + CPP_SOURCES + ["internal.h", "device_common.cuh"]]
+    return ([os.path.join(CSRC, s) for s in CU_SOURCES + CPP_SOURCES + ["internal.h", "device_common.cuh", "debug_bounds.cuh"]]
             + [os.path.join(INCLUDE, "zero_b200.h")])
 
 

@@ -22,6 +22,11 @@ struct zero_plan_s {
 
 namespace zb {
 
+// The staged fused step's tile: each shard is cut into tiles of this many
+// elements (the last tile of a shard shorter), in 64-bit arithmetic.
+constexpr int64_t kStagedTile = 2048;
+inline int64_t staged_tiles_per_shard(int64_t S) { return (S + kStagedTile - 1) / kStagedTile; }
+
 // Device-resident loss-scale / step state. One per context, in the
 // context's device scratch. Written by the last block of every step kernel.
 struct alignas(64) DevState {
@@ -120,6 +125,12 @@ cudaError_t launch_gather_many(int32_t R, int64_t S, int nl, const int64_t* lo, 
 
 // Grid the step kernels use for a given problem (for sizing `partials`).
 int step_grid_cap(int device);
+
+#ifdef ZERO_DEBUG_BOUNDS
+// The bounds record of the static-scratch step's module (noalloc.cu), zero
+// when that step never ran in this process; optionally cleared.
+cudaError_t noalloc_bounds_record(unsigned long long* count, unsigned long long* first, bool reset);
+#endif
 
 }  // namespace zb
 

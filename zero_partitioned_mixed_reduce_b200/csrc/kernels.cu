@@ -28,33 +28,11 @@
 #include <mutex>
 #include <string>
 
+#include "debug_bounds.cuh"
 #include "device_common.cuh"
 #include "internal.h"
 
 namespace zb {
-
-// ---------------------------------------------------------------------------
-// Bounds checks of the debug build (ZERO_DEBUG_BOUNDS). ZB_IN(cond, site,
-// index) guards an access: in the debug build a false cond is counted, the
-// first failing site and index are kept, and the caller skips the access; in
-// the release build it is the constant true and cond is not evaluated.
-// Sites: 1 fused vector, 2 fused accumulator, 3 staged tile issue, 4 staged
-// tile store, 5 two-pass vector, 6 accumulator norm, 7 replica norm,
-// 8 reduce-scatter vector, 9 reduce-scatter element, 10 gather vector,
-// 11 gather element, 12 reduce-scatter norm partial.
-// ---------------------------------------------------------------------------
-#ifdef ZERO_DEBUG_BOUNDS
-__device__ unsigned long long g_bounds_count = 0;
-__device__ unsigned long long g_bounds_first = 0;
-__device__ __noinline__ bool bounds_fail(unsigned site, unsigned long long index) {
-    atomicAdd(&g_bounds_count, 1ull);
-    atomicCAS(&g_bounds_first, 0ull, (static_cast<unsigned long long>(site) << 48) | (index & 0xffffffffffffull));
-    return false;
-}
-#define ZB_IN(cond, site, index) ((cond) ? true : ::zb::bounds_fail((site), (index)))
-#else
-#define ZB_IN(cond, site, index) true
-#endif
 
 template <typename T, int CAP>
 __device__ __forceinline__ bool ptrs_ok(T* const (&p)[CAP], int n) {
@@ -1226,19 +1204,15 @@ extern "C" zero_status zero_debug_bounds(int64_t* count, int64_t* first_site, in
     if (!count || !first_site || !first_index)
         return zb_fail(ZERO_ERR_INVALID_ARG, "zero_debug_bounds: NULL output");
 #ifdef ZERO_DEBUG_BOUNDS
-    unsigned long long c = 0, f = 0;
-    cudaError_t e = cudaDeviceSynchronize();
-    if (e == cudaSuccess) e = cudaMemcpyFromSymbol(&c, zb::g_bounds_count, sizeof c);
-    if (e == cudaSuccess) e = cudaMemcpyFromSymbol(&f, zb::g_bounds_first, sizeof f);
-    if (e == cudaSuccess && reset) {
-        const unsigned long long zero = 0;
-        e = cudaMemcpyToSymbol(zb::g_bounds_count, &zero, sizeof zero);
-        if (e == cudaSuccess) e = cudaMemcpyToSymbol(zb::g_bounds_first, &zero, sizeof zero);
-    }
+    unsigned long long c = 0, f = 0, c2 = 0, f2 = 0;
+    cudaError_t e = zb::bounds_record(&c, &f, reset != 0);
+    if (e == cudaSuccess) e = zb::noalloc_bounds_record(&c2, &f2, reset != 0);
     if (e != cudaSuccess) {
         cudaGetLastError();
         return zb_fail(ZERO_ERR_CUDA, std::string("zero_debug_bounds: ") + cudaGetErrorString(e));
     }
+    c += c2;
+    if (f == 0) f = f2;
     *count = static_cast<int64_t>(c);
     *first_site = static_cast<int64_t>(f >> 48);
     *first_index = static_cast<int64_t>(f & 0xffffffffffffull);

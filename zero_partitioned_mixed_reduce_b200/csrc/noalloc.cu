@@ -4,10 +4,14 @@
 // per-block norm partials and a small control word -- lives in one static
 // device array in this file, so the call makes no cudaMalloc / cudaFree and
 // needs no context. See include/zero_b200.h for the contract.
+#include <cuda.h>
+
+#include <atomic>
 #include <cmath>
 #include <mutex>
 #include <string>
 
+#include "debug_bounds.cuh"
 #include "device_common.cuh"
 #include "internal.h"
 
@@ -32,6 +36,7 @@ namespace {
 
 struct NoallocArgs {
     Coef c;
+    int32_t R;
     int32_t dynamic;
     uint32_t S8, T8;
     DevState* ctrl;
@@ -64,6 +69,10 @@ __global__ void __launch_bounds__(kThreads) noalloc_step_kernel(const __grid_con
         oc.seek(vi);
         const uint32_t o = oc.o;
         const size_t j8 = static_cast<size_t>(vi - oc.base) * 8;
+        if (!ZB_IN(o < static_cast<uint32_t>(a.R) && vi - oc.base < a.S8 && a.acc[o] && a.master[o] && a.m[o] &&
+                       a.v[o] && a.param[o],
+                   13, vi))
+            continue;
         const F8 acc = ld_f8(a.acc[o] + j8);
         if (skip) {
 #pragma unroll
@@ -109,11 +118,38 @@ __global__ void __launch_bounds__(kThreads) noalloc_step_kernel(const __grid_con
     }
 }
 
-// Device address of g_noalloc_scratch, looked up once per device with that
-// device current. In host code the array's name only stands in for the
-// symbol; it is not a device address.
+// Device address of g_noalloc_scratch, looked up once per device and CUDA
+// context with that device current (a reset device gets a new context, and
+// its array a new address). In host code the array's name only stands in for
+// the symbol; it is not a device address.
+struct ScratchSlot {
+    CUcontext ctx = nullptr;
+    unsigned char* addr = nullptr;
+};
 std::mutex g_scratch_mu;
-unsigned char* g_scratch_addr[64] = {};
+ScratchSlot g_scratch_slot[64];
+std::atomic<bool> g_noalloc_used{false};
+
+using CtxGetCurrent = CUresult (*)(CUcontext*);
+
+// The calling thread's current context through the driver's entry point
+// (the library links no driver library); NULL when none is current yet or
+// the entry point is unavailable.
+CUcontext current_context() {
+    static const CtxGetCurrent fn = [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q = cudaDriverEntryPointSymbolNotFound;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) != cudaSuccess ||
+            q != cudaDriverEntryPointSuccess) {
+            cudaGetLastError();
+            p = nullptr;
+        }
+        return reinterpret_cast<CtxGetCurrent>(p);
+    }();
+    CUcontext c = nullptr;
+    if (fn && fn(&c) != CUDA_SUCCESS) c = nullptr;
+    return c;
+}
 
 zero_status scratch_for_current_device(unsigned char** out) {
     int dev = -1;
@@ -122,7 +158,11 @@ zero_status scratch_for_current_device(unsigned char** out) {
         return zb_fail(ZERO_ERR_CUDA, std::string("zero_step_noalloc: ") + cudaGetErrorString(e));
     if (dev < 0 || dev >= 64) return zb_fail(ZERO_ERR_RANGE, "zero_step_noalloc: device index >= 64");
     std::lock_guard<std::mutex> lock(g_scratch_mu);
-    if (!g_scratch_addr[dev]) {
+    ScratchSlot& slot = g_scratch_slot[dev];
+    const CUcontext ctx = current_context();
+    if (ctx == nullptr || slot.ctx != ctx || slot.addr == nullptr) {
+        // set-up: under CUDA's lazy module loading this also loads this
+        // file's module on the device, which reserves the static array
         void* p = nullptr;
         e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
         if (e != cudaSuccess || p == nullptr) {
@@ -131,9 +171,11 @@ zero_status scratch_for_current_device(unsigned char** out) {
                            std::string("zero_step_noalloc: cannot resolve the static scratch: ") +
                                cudaGetErrorString(e));
         }
-        g_scratch_addr[dev] = static_cast<unsigned char*>(p);
+        slot.addr = static_cast<unsigned char*>(p);
+        slot.ctx = current_context();  // the look-up made the device's context current
     }
-    *out = g_scratch_addr[dev];
+    g_noalloc_used.store(true);
+    *out = slot.addr;
     return ZERO_OK;
 }
 
@@ -154,6 +196,18 @@ zero_status check_list(Ptr const* arr, int R, uintptr_t align, const char* what)
 }
 
 }  // namespace
+
+#ifdef ZERO_DEBUG_BOUNDS
+cudaError_t noalloc_bounds_record(unsigned long long* count, unsigned long long* first, bool reset) {
+    *count = 0;
+    *first = 0;
+    // reading the record would load this module, and reserve its array, in a
+    // process that never used it
+    if (!g_noalloc_used.load()) return cudaSuccess;
+    return bounds_record(count, first, reset);
+}
+#endif
+
 }  // namespace zb
 
 extern "C" zero_status zero_step_noalloc(const zero_plan_t* plan, const zero_loss_scale_config* cfg,
@@ -224,6 +278,7 @@ extern "C" zero_status zero_step_noalloc(const zero_plan_t* plan, const zero_los
         a.c.ss = static_cast<float>(hp->lr / (1.0 - std::pow(hp->beta1, t1)));
         a.c.bc2s = static_cast<float>(std::sqrt(1.0 - std::pow(hp->beta2, t1)));
         a.c.clip = 1.0f;
+        a.R = R;
         a.dynamic = cfg->mode == ZERO_SCALE_DYNAMIC;
         a.S8 = static_cast<uint32_t>(plan->S / 8);
         a.T8 = static_cast<uint32_t>(plan->T / 8);

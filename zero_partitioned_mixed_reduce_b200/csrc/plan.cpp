@@ -204,3 +204,15 @@ extern "C" zero_status zero_plan_memory(const zero_plan_t* plan, int32_t stage, 
         return ZERO_OK;
     });
 }
+
+extern "C" zero_status zero_plan_step_tiles(const zero_plan_t* plan, int64_t* tile_elems, int64_t* tiles_per_shard,
+                                            int64_t* tiles_total) {
+    return zb_guarded("zero_plan_step_tiles", [&]() -> zero_status {
+        if (!plan) return zb_fail(ZERO_ERR_INVALID_ARG, "zero_plan_step_tiles: plan is NULL");
+        const int64_t tps = zb::staged_tiles_per_shard(plan->S);
+        if (tile_elems) *tile_elems = zb::kStagedTile;
+        if (tiles_per_shard) *tiles_per_shard = tps;
+        if (tiles_total) *tiles_total = tps * plan->R;
+        return ZERO_OK;
+    });
+}
