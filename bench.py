@@ -103,7 +103,33 @@ def parse_args(argv=None):
                     help="issue every launch through the C ABI instead of replaying CUDA graphs")
     ap.add_argument("--first-tensors", type=int, default=0,
                     help="use only the first N tensors of the workload (small profiling cases)")
-    return ap.parse_args(argv)
+    ap.add_argument("--tensors", default="",
+                    help="use only tensors LO:HI of the workload's list (small profiling cases)")
+    args = ap.parse_args(argv)
+    args.tensor_range = None
+    if args.tensors:
+        lo, hi = (int(x) for x in args.tensors.split(":"))
+        args.tensor_range = (lo, hi)
+    elif args.first_tensors:
+        args.tensor_range = (0, args.first_tensors)
+    return args
+
+
+def restrict(wl, rng):
+    """The workload cut to tensors [lo, hi) of its list (layer ids renumbered
+    from 0); rng None keeps it whole."""
+    if rng is None:
+        return wl
+    lo, hi = rng
+    wl["numels"] = wl["numels"][lo:hi]
+    if wl["layer_ids"]:
+        ids = wl["layer_ids"][lo:hi]
+        wl["layer_ids"] = [i - ids[0] for i in ids]
+    if wl.get("inject") and not (lo <= wl["inject"]["tensor"] < hi):
+        wl["inject"] = None
+    elif wl.get("inject"):
+        wl["inject"] = dict(wl["inject"], tensor=wl["inject"]["tensor"] - lo)
+    return wl
 
 
 # ---- distributed plumbing ---------------------------------------------------
@@ -242,9 +268,9 @@ def profiled_traffic(kernel, workload):
 
 # ---- the workload -------------------------------------------------------------
 
-def workload_label(name, wl, first_tensors=0):
+def workload_label(name, wl, tensor_range=None):
     """The workload as both arms name it in their `config`."""
-    part = f" (first {first_tensors} tensors)" if first_tensors else ""
+    part = f" (tensors {tensor_range[0]}:{tensor_range[1]})" if tensor_range else ""
     return (f"{name}{part}: {len(wl['numels'])} tensors, P={sum(wl['numels'])}, R={wl['R']} "
             f"simulated ranks, {'fp16' if wl['dtype'] else 'bf16'} grads, "
             f"loss scale mode {wl['mode']}")
@@ -267,7 +293,7 @@ def bucket_runs(buckets, group):
 
 
 class Bench:
-    def __init__(self, name, path, first_tensors=0, gather_bucket=32 << 20, accum=1, clip=0.0,
+    def __init__(self, name, path, tensor_range=None, gather_bucket=32 << 20, accum=1, clip=0.0,
                  bucket_elems=None, clip_norm="rs", rs_group=25 << 20):
         import zero_partitioned_mixed_reduce_b200 as Z
         import synth
@@ -275,9 +301,7 @@ class Bench:
         self.wl = wl = synth.workload(name)
         if bucket_elems is not None:
             wl["bucket_elems"] = bucket_elems
-        if first_tensors:
-            wl["numels"] = wl["numels"][:first_tensors]
-            wl["layer_ids"] = wl["layer_ids"][:first_tensors] if wl["layer_ids"] else None
+        restrict(wl, tensor_range)
         self.R, self.dtype = wl["R"], wl["dtype"]
         self.accum, self.clip = accum, clip
         if path == "auto":
@@ -475,7 +499,7 @@ def run_ours(args, world, rank, local):
     if not torch.cuda.is_available():
         print(json.dumps({"error": "no CUDA device: the benchmark has no CPU fallback"}))
         sys.exit(1)
-    b = Bench(args.workload, args.path, args.first_tensors, args.gather_bucket, args.accum,
+    b = Bench(args.workload, args.path, args.tensor_range, args.gather_bucket, args.accum,
               args.clip, clip_norm=args.clip_norm, rs_group=args.rs_group)
     stream = torch.cuda.current_stream()
     if args.graph:
@@ -534,7 +558,7 @@ def run_ours(args, world, rank, local):
         kernel_name = f"reduce_scatter+fused_step_kernel (accum {b.accum}, last micro-batch fused)"
     # the stored counters describe the full workload on the ping-pong fused
     # path; any other configuration reports no traffic
-    same_config = args.first_tensors == 0 and b.path == "pingpong"
+    same_config = args.tensor_range is None and b.path == "pingpong"
     traffic = profiled_traffic(kernel_name, args.workload) if same_config else None
     clip_label = ("" if b.clip <= 0 else
                   "global-norm clip from the reduce-scatters' norm shares, " if b.rs_norm else
@@ -555,7 +579,7 @@ def run_ours(args, world, rank, local):
         "hbm_gbs": step_bytes * K * world / (ms * 1e-3) / 1e9,
         "hbm_frac_of_peak": step_bytes * K / (ms * 1e-3) / 1e9 / peak,
         "config": {
-            "workload": workload_label(args.workload, b.wl, args.first_tensors),
+            "workload": workload_label(args.workload, b.wl, args.tensor_range),
             "R": b.R, "P": b.P, "T": b.T, "S": b.S, "n_layers": len(b.plan.layers),
             "path": {"pingpong": f"{'global-norm clip pass, ' if b.clip > 0 else ''}"
                                  f"{f'{b.accum - 1} micro-batch(es) reduce-scattered, last ' if b.accum > 1 else ''}"
@@ -816,7 +840,7 @@ def run_overlap(args, world, rank, local):
     if not torch.cuda.is_available():
         print(json.dumps({"error": "no CUDA device"}))
         sys.exit(1)
-    b = Bench(args.workload, "twopass", args.first_tensors, 0, bucket_elems=args.bucket_elems)
+    b = Bench(args.workload, "twopass", args.tensor_range, 0, bucket_elems=args.bucket_elems)
     Z = b.Z
     stream = torch.cuda.current_stream()
     wl, plan = b.wl, b.plan
@@ -1069,9 +1093,7 @@ def run_dist(args, world, rank, local):
         dist.init_process_group("nccl", rank=0, world_size=1, timeout=datetime.timedelta(seconds=300))
     N = dist.get_world_size()
     wl = synth.workload(args.workload)
-    if args.first_tensors:
-        wl["numels"] = wl["numels"][:args.first_tensors]
-        wl["layer_ids"] = wl["layer_ids"][:args.first_tensors] if wl["layer_ids"] else None
+    restrict(wl, args.tensor_range)
     dz = DistributedZero(wl["numels"], wl["layer_ids"], wl["dtype"], wl["mode"], wl["init_scale"],
                          wl["interval"], 8, wl["bucket_elems"])
     plan = dz.plan
@@ -1137,7 +1159,7 @@ def run_dist(args, world, rank, local):
         "metric": METRIC, "value": units / (ms * 1e-3), "unit": "params/s",
         "n_gpus": N, "steps": K, "warmup": args.warmup, "ms_per_step": ms / K, "higher_is_better": True,
         "scaling": "strong", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
-        "config": {"workload": workload_label(args.workload, wl, args.first_tensors).split(", R=")[0]
+        "config": {"workload": workload_label(args.workload, wl, args.tensor_range).split(", R=")[0]
                                + f", sharded over {N} rank(s), one per GPU",
                    "R": N, "P": plan.P, "T": T, "S": S, "n_layers": len(plan.layers),
                    "path": "DistributedZero: 4-byte NCCL all-reduce (every replica written), fused "
@@ -1214,9 +1236,7 @@ def run_offload(args, world, rank, local):
     import zero_partitioned_mixed_reduce_b200 as Z
     import synth
     wl = synth.workload(args.workload)
-    if args.first_tensors:
-        wl["numels"] = wl["numels"][:args.first_tensors]
-        wl["layer_ids"] = wl["layer_ids"][:args.first_tensors]
+    restrict(wl, args.tensor_range)
     plan = Z.Plan(wl["numels"], wl["layer_ids"], wl["R"], wl["dtype"], 8, wl["bucket_elems"])
     R, S, T, P = plan.R, plan.S, plan.T, plan.P
     half = Z.state.HALF[wl["dtype"]]

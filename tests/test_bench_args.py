@@ -73,3 +73,15 @@ def test_dist_bytes_and_roofline():
     assert abs(r["frac"] - 500.0 / bench.NVLINK_PEER_GBS) < 1e-12
     r = bench.dist_roofline({"hbm": 6e9, "nvlink": 0}, 1.0, 6000.0)
     assert r["bound"] == "hbm" and abs(r["frac"] - 1.0) < 1e-12
+
+
+def test_tensor_range_selection():
+    import synth
+    a = bench.parse_args(["--tensors", "1:10"])
+    assert a.tensor_range == (1, 10)
+    assert bench.parse_args(["--first-tensors", "6"]).tensor_range == (0, 6)
+    assert bench.parse_args([]).tensor_range is None
+    wl = bench.restrict(synth.workload("llama3b"), (1, 10))
+    # one decoder layer of the Llama-style list: norms, q/k/v/o, gate/up/down
+    assert len(wl["numels"]) == 9 and sum(wl["numels"]) == 100_669_440
+    assert wl["layer_ids"] == [0] * 9

@@ -42,5 +42,7 @@ def test_bench_distributed_mode():
     assert r.returncode == 0, (r.stdout[-3000:], r.stderr[-3000:])
     line = [ln for ln in r.stdout.splitlines() if ln.startswith("{")][-1]
     out = json.loads(line)
-    assert out["mode"] == "distributed" and out["n_gpus"] == 1 and out["scaling"] == "strong"
-    assert out["value"] > 0 and out["config"]["R"] == 1
+    assert out["n_gpus"] == 1 and out["scaling"] == "strong" and out["config"]["parallelism"].startswith("dp1")
+    assert out["value"] > 0 and out["config"]["R"] == 1 and out["state_check"] == "ok"
+    assert out["roofline"]["bound"] in ("hbm", "nvlink") and out["roofline"]["achieved"] > 0
+    assert out["gpu_launches"] > 0 and out["e2e"]["value"] > 0 and out["nccl"]["world_size"] == 1

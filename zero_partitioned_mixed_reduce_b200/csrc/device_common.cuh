@@ -162,8 +162,11 @@ __device__ __forceinline__ double warp_sum(double x) {
     return x;
 }
 
-// Deterministic for a fixed grid: fixed per-thread order, fixed tree.
+// Deterministic for a fixed grid: fixed per-thread order, fixed tree. NW is
+// the block's warp count (smem holds NW entries); every thread calls it.
+template <int NW = kWarps>
 __device__ __forceinline__ double block_sum(double x, double* smem) {
+    static_assert(NW >= 1 && NW <= 32, "one warp sums the warps' partials");
     x = warp_sum(x);
     const int w = threadIdx.x >> 5, l = threadIdx.x & 31;
     __syncthreads();
@@ -171,7 +174,7 @@ __device__ __forceinline__ double block_sum(double x, double* smem) {
     __syncthreads();
     double r = 0.0;
     if (w == 0) {
-        r = l < kWarps ? smem[l] : 0.0;
+        r = l < NW ? smem[l] : 0.0;
         r = warp_sum(r);
     }
     return r;  // valid in thread 0

@@ -129,11 +129,12 @@ __device__ void fsm_update(const StepParams& sp, DevState* st, double norm) {
 // Every block publishes its norm partial and flag; the last block to finish
 // sums the partials in block order and runs the state machine -- or, for a
 // sharded step, hands its local totals to the caller for a cross-rank
-// reduction and a later commit.
+// reduction and a later commit. NW: the block's warps.
+template <int NW = kWarps>
 __device__ void step_epilogue(const StepParams& sp, double nrm, bool bad) {
-    __shared__ double red[kWarps];
+    __shared__ double red[NW];
     __shared__ int last;
-    const double bn = block_sum(nrm, red);
+    const double bn = block_sum<NW>(nrm, red);
     const int any_bad = __syncthreads_or(bad ? 1 : 0);
     if (threadIdx.x == 0) {
         sp.partials[blockIdx.x] = bn;
@@ -146,9 +147,9 @@ __device__ void step_epilogue(const StepParams& sp, double nrm, bool bad) {
     if (!last) return;
     __threadfence();
     double x = 0.0;
-    for (unsigned i = threadIdx.x; i < gridDim.x; i += kThreads)
+    for (unsigned i = threadIdx.x; i < gridDim.x; i += NW * 32)
         x += *reinterpret_cast<volatile double*>(&sp.partials[i]);
-    const double total = block_sum(x, red);
+    const double total = block_sum<NW>(x, red);
     if (threadIdx.x == 0) {
         if (sp.partial_out) {
             sp.partial_out[0] = total;
@@ -254,22 +255,34 @@ __global__ void __launch_bounds__(kThreads)
 
 // ---------------------------------------------------------------------------
 // The same fused step with the read streams staged through shared memory by
-// the Tensor Memory Accelerator: one thread issues 1-D bulk copies
-// (cp.async.bulk, no multicast) of a whole tile -- R gradient segments and
-// the master/m/v segments of one shard -- into a 2-stage ring completed by
-// mbarrier transaction counts, while the block computes the previous tile
-// from shared memory. Loads in flight then cost no registers. Used when R is
-// small: the per-element read (2R + 12 bytes) leaves room for 3 blocks of 256
-// threads per SM, and the register path keeps too few bytes in flight. Tiles
-// are shard-local (2048 elements, the last one of a shard shorter). Every
-// mbarrier wait gives up after 2 s of %globaltimer: the block then records
-// ZERO_ERR_TIMEOUT in the device state, waits (bounded) for its copies in
-// flight, and finishes without updating further tiles.
+// the Tensor Memory Accelerator, for small R: the per-element read (2R + 12
+// bytes) then leaves too few bytes in flight per thread on the register
+// path. A block is 8 consumer warps and one producer warp. The producer's
+// elected lane issues, per 2048-element shard-local tile, 1-D bulk copies
+// (cp.async.bulk, no multicast) of the R gradient segments and the
+// master/m/v segments into a 2-stage shared-memory ring; each stage has a
+// "full" mbarrier (completed by the copies' transaction bytes) and an
+// "empty" mbarrier (completed when all 256 consumer threads have read the
+// stage into registers). Consumers release a stage before doing the
+// arithmetic, so the next tile's copies overlap the current tile's math and
+// no block-wide barrier sits in the loop. Tile indices, shard offsets and
+// lengths are 64-bit: a shard may hold more than 2^32 elements. Every
+// mbarrier wait gives up after 2 s of %globaltimer: the waiting thread
+// records ZERO_ERR_TIMEOUT in the device state and leaves its loop, and the
+// producer waits (bounded) for its copies still in flight before the block
+// finishes; the last block then abandons the step.
 // ---------------------------------------------------------------------------
 
 constexpr int kTmaTile = kThreads * 8;
+static_assert(kTmaTile == kStagedTile, "the host tiling and the kernel's tile agree");
 constexpr int kTmaStages = 2;
+constexpr int kTmaThreads = kThreads + 32;  // consumers + one producer warp
+constexpr int kTmaWarps = kTmaThreads / 32;
 constexpr int kErrTimeout = 2;
+// Two resident blocks per SM measured faster than three (R = 2 at 1.37 G
+// elements per shard: 6024 against 5926 GB/s, same process): the grid is
+// capped there.
+constexpr int kTmaBlocksPerSm = 2;
 
 template <int RC>
 struct TmaStage {
@@ -286,6 +299,9 @@ __device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
 }
 __device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
     asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+    asm volatile("{ .reg .b64 st; mbarrier.arrive.shared::cta.b64 st, [%0]; }" ::"r"(bar) : "memory");
 }
 __device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
     asm volatile(
@@ -321,80 +337,103 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
 __device__ __forceinline__ uint4 lds16(const void* p) { return *reinterpret_cast<const uint4*>(p); }
 
 template <typename H, int RC, bool CLIP>
-__global__ void __launch_bounds__(kThreads)
-    fused_step_tma_kernel(const __grid_constant__ FusedArgs<RC> a, uint32_t tiles_per_shard) {
+__global__ void __launch_bounds__(kTmaThreads, kTmaBlocksPerSm)
+    fused_step_tma_kernel(const __grid_constant__ FusedArgs<RC> a, uint64_t tiles_per_shard) {
     using L = TmaStage<RC>;
     extern __shared__ __align__(128) unsigned char smem[];
-    __shared__ __align__(8) uint64_t bars[kTmaStages];
+    __shared__ __align__(8) uint64_t full[kTmaStages], empty[kTmaStages];
     const StepParams& sp = a.sp;
     __shared__ Prologue pro;
     read_prologue(sp, RC, &pro, false);
     const Coef c = pro.c;
     const int src = pro.src, dst = pro.dst;
-    const uint32_t S = sp.S8 * 8;
-    const uint32_t tbeg = static_cast<uint32_t>(sp.obeg) * tiles_per_shard;
-    const uint32_t ntiles = static_cast<uint32_t>(sp.oend) * tiles_per_shard;  // one past the last tile
+    const uint64_t S = static_cast<uint64_t>(sp.S8) * 8;
+    const uint64_t tps = tiles_per_shard;
+    const uint64_t t0 = static_cast<uint64_t>(sp.obeg) * tps, t1 = static_cast<uint64_t>(sp.oend) * tps;
+    // this block's tiles: t0 + blockIdx.x + k * gridDim.x, k < count
+    const uint64_t G = gridDim.x, first = t0 + blockIdx.x;
+    const uint64_t count = first < t1 ? (t1 - first + G - 1) / G : 0;
     if (threadIdx.x == 0) {
-        for (int s = 0; s < kTmaStages; ++s) mbar_init(smem_u32(&bars[s]), 1);
+        for (int s = 0; s < kTmaStages; ++s) {
+            mbar_init(smem_u32(&full[s]), 1);
+            mbar_init(smem_u32(&empty[s]), kThreads);
+        }
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
     __syncthreads();
-    // one thread queues tile `tile` into stage s
-    auto issue = [&](uint32_t tile, int s) {
-        const uint32_t o = tile / tiles_per_shard;
-        const uint32_t j0 = (tile - o * tiles_per_shard) * kTmaTile;
-        const uint32_t len = min(static_cast<uint32_t>(kTmaTile), S - j0);
-        unsigned char* base = smem + s * L::kBytes;
-        const uint32_t bar = smem_u32(&bars[s]);
-        if (tile == sp.drop_tile) return;  // test support: this tile's wait must run out
-        if (!ZB_IN(o >= static_cast<uint32_t>(sp.obeg) && o < static_cast<uint32_t>(sp.oend) && j0 < S &&
-                       len % 8 == 0 && j0 + len <= S && ptrs_ok(a.g, RC) && a.master[src][o] && a.m[src][o] &&
-                       a.v[src][o],
-                   3, tile))
-            return;  // skipped: the wait for this tile runs out and the step is abandoned
-        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-        mbar_expect_tx(bar, len * (RC * 2 + 12));
-#pragma unroll
-        for (int r = 0; r < RC; ++r)
-            bulk_g2s(smem_u32(base + r * kTmaTile * 2),
-                     reinterpret_cast<const uint16_t*>(a.g[r]) + static_cast<size_t>(o) * S + j0, len * 2,
-                     bar);
-        bulk_g2s(smem_u32(base + L::kGradBytes), a.master[src][o] + j0, len * 4, bar);
-        bulk_g2s(smem_u32(base + L::kGradBytes + kTmaTile * 4), a.m[src][o] + j0, len * 4, bar);
-        bulk_g2s(smem_u32(base + L::kGradBytes + 2 * kTmaTile * 4), a.v[src][o] + j0, len * 4, bar);
-    };
-    if (threadIdx.x == 0)
-        for (int s = 0; s < kTmaStages; ++s) {
-            const uint32_t tile = tbeg + blockIdx.x + s * gridDim.x;
-            if (tile < ntiles) issue(tile, s);
-        }
     double nrm = 0.0;
-    bool bad = false, failed = false;
-    int j = 0;
-    for (uint32_t tile = tbeg + blockIdx.x; tile < ntiles; tile += gridDim.x, ++j) {
-        const int s = j % kTmaStages;
-        const bool ok = mbar_wait(smem_u32(&bars[s]), (j / kTmaStages) & 1);
-        if (__syncthreads_or(!ok)) {
-            failed = true;
-            break;
-        }
-        const uint32_t o = tile / tiles_per_shard;
-        const uint32_t j0 = (tile - o * tiles_per_shard) * kTmaTile;
-        const uint32_t len = min(static_cast<uint32_t>(kTmaTile), S - j0);
-        const uint32_t e0 = threadIdx.x * 8;
-        if (e0 < len) {
-            const unsigned char* base = smem + s * L::kBytes;
-            uint4 gv[RC];
+    bool bad = false;
+    if (threadIdx.x >= kThreads) {
+        // producer warp: one lane issues every copy
+        if (threadIdx.x == kThreads) {
+            uint64_t k = 0, dropped = ~0ull;
+            for (; k < count; ++k) {
+                const int s = static_cast<int>(k % kTmaStages);
+                if (k >= kTmaStages &&
+                    !mbar_wait(smem_u32(&empty[s]), static_cast<uint32_t>((k / kTmaStages - 1) & 1))) {
+                    sp.st->err = kErrTimeout;
+                    break;
+                }
+                const uint64_t tile = first + k * G;
+                const uint64_t o = tile / tps;
+                const uint64_t j0 = (tile - o * tps) * kTmaTile;
+                const uint32_t len = static_cast<uint32_t>(S - j0 < kTmaTile ? S - j0 : kTmaTile);
+                // test support (a tile whose copies never come), or a failed
+                // check of the debug build: the consumers' wait runs out
+                if (tile == sp.drop_tile ||
+                    !ZB_IN(o >= static_cast<uint64_t>(sp.obeg) && o < static_cast<uint64_t>(sp.oend) && j0 < S &&
+                               len % 8 == 0 && j0 + len <= S && ptrs_ok(a.g, RC) && a.master[src][o] &&
+                               a.m[src][o] && a.v[src][o],
+                           3, tile)) {
+                    dropped = k;
+                    continue;
+                }
+                unsigned char* base = smem + s * L::kBytes;
+                const uint32_t bar = smem_u32(&full[s]);
+                asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+                mbar_expect_tx(bar, len * (RC * 2 + 12));
 #pragma unroll
-            for (int r = 0; r < RC; ++r) gv[r] = lds16(base + r * kTmaTile * 2 + e0 * 2);
-            const float* ps = reinterpret_cast<const float*>(base + L::kGradBytes);
+                for (int r = 0; r < RC; ++r)
+                    bulk_g2s(smem_u32(base + r * kTmaTile * 2),
+                             reinterpret_cast<const uint16_t*>(a.g[r]) + o * S + j0, len * 2, bar);
+                bulk_g2s(smem_u32(base + L::kGradBytes), a.master[src][o] + j0, len * 4, bar);
+                bulk_g2s(smem_u32(base + L::kGradBytes + kTmaTile * 4), a.m[src][o] + j0, len * 4, bar);
+                bulk_g2s(smem_u32(base + L::kGradBytes + 2 * kTmaTile * 4), a.v[src][o] + j0, len * 4, bar);
+            }
+            // copies still in flight land before the block's shared memory is released
+            for (uint64_t q = k > kTmaStages ? k - kTmaStages : 0; q < k; ++q)
+                if (q != dropped)
+                    mbar_wait(smem_u32(&full[q % kTmaStages]), static_cast<uint32_t>((q / kTmaStages) & 1));
+        }
+    } else {
+        for (uint64_t k = 0; k < count; ++k) {
+            const int s = static_cast<int>(k % kTmaStages);
+            if (!mbar_wait(smem_u32(&full[s]), static_cast<uint32_t>((k / kTmaStages) & 1))) {
+                sp.st->err = kErrTimeout;
+                break;
+            }
+            const uint64_t tile = first + k * G;
+            const uint64_t o = tile / tps;
+            const uint64_t j0 = (tile - o * tps) * kTmaTile;
+            const uint32_t len = static_cast<uint32_t>(S - j0 < kTmaTile ? S - j0 : kTmaTile);
+            const uint32_t e0 = threadIdx.x * 8;
+            const bool act = e0 < len;
+            uint4 gv[RC];
             F8 p, m, v;
-            *reinterpret_cast<uint4*>(&p.x[0]) = lds16(ps + e0);
-            *reinterpret_cast<uint4*>(&p.x[4]) = lds16(ps + e0 + 4);
-            *reinterpret_cast<uint4*>(&m.x[0]) = lds16(ps + kTmaTile + e0);
-            *reinterpret_cast<uint4*>(&m.x[4]) = lds16(ps + kTmaTile + e0 + 4);
-            *reinterpret_cast<uint4*>(&v.x[0]) = lds16(ps + 2 * kTmaTile + e0);
-            *reinterpret_cast<uint4*>(&v.x[4]) = lds16(ps + 2 * kTmaTile + e0 + 4);
+            if (act) {
+                const unsigned char* base = smem + s * L::kBytes;
+#pragma unroll
+                for (int r = 0; r < RC; ++r) gv[r] = lds16(base + r * kTmaTile * 2 + e0 * 2);
+                const float* ps = reinterpret_cast<const float*>(base + L::kGradBytes);
+                *reinterpret_cast<uint4*>(&p.x[0]) = lds16(ps + e0);
+                *reinterpret_cast<uint4*>(&p.x[4]) = lds16(ps + e0 + 4);
+                *reinterpret_cast<uint4*>(&m.x[0]) = lds16(ps + kTmaTile + e0);
+                *reinterpret_cast<uint4*>(&m.x[4]) = lds16(ps + kTmaTile + e0 + 4);
+                *reinterpret_cast<uint4*>(&v.x[0]) = lds16(ps + 2 * kTmaTile + e0);
+                *reinterpret_cast<uint4*>(&v.x[4]) = lds16(ps + 2 * kTmaTile + e0 + 4);
+            }
+            mbar_arrive(smem_u32(&empty[s]));  // this thread is done with stage s
+            if (!act) continue;
             float acc[8];
             unpack8<H>(gv[0], acc);
 #pragma unroll
@@ -407,8 +446,7 @@ __global__ void __launch_bounds__(kThreads)
                 nrm = fma(gd, gd, nrm);
                 out[e] = p.x[e];
             }
-            const size_t jj = static_cast<size_t>(j0) + e0;
-            // a guarded block, not a continue: every thread must reach the barrier below
+            const uint64_t jj = j0 + e0;
             if (ZB_IN(jj + 8 <= S && a.master[dst][o] && a.m[dst][o] && a.v[dst][o] && a.param[dst][o], 4, jj)) {
                 st_f8(a.master[dst][o] + jj, p);
                 st_f8(a.m[dst][o] + jj, m);
@@ -416,16 +454,8 @@ __global__ void __launch_bounds__(kThreads)
                 st_u4(a.param[dst][o] + (jj >> 3), pack8<H>(out));
             }
         }
-        __syncthreads();  // every thread is done with stage s
-        const uint32_t next = tile + kTmaStages * gridDim.x;
-        if (threadIdx.x == 0 && next < ntiles) issue(next, s);
     }
-    if (failed) {
-        if (threadIdx.x == 0) sp.st->err = kErrTimeout;
-        for (int k = 0; k < kTmaStages; ++k)  // let copies in flight land (bounded)
-            mbar_wait(smem_u32(&bars[(j + k) % kTmaStages]), ((j + k) / kTmaStages) & 1);
-    }
-    step_epilogue(sp, nrm, bad);
+    step_epilogue<kTmaWarps>(sp, nrm, bad);
 }
 
 // ---------------------------------------------------------------------------
@@ -958,14 +988,13 @@ cudaError_t fused_tma_t(const StepParams& sp, const RankPtrs& p, cudaStream_t s)
         cudaFuncSetAttribute(fused_step_tma_kernel<H, RC, CLIP>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              smem);
         int n = 0;
-        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, fused_step_tma_kernel<H, RC, CLIP>, kThreads, smem);
-        return n > 0 ? n : 1;
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, fused_step_tma_kernel<H, RC, CLIP>, kTmaThreads, smem);
+        return n > kTmaBlocksPerSm ? kTmaBlocksPerSm : (n > 0 ? n : 1);
     }();
-    const uint32_t S = sp.S8 * 8;
-    const uint32_t tiles_per_shard = (S + kTmaTile - 1) / kTmaTile;
-    const uint32_t grid = grid_for(static_cast<uint64_t>(tiles_per_shard) * (sp.oend - sp.obeg) * kThreads, per_sm,
-                                   sp.grid_cap);
-    fused_step_tma_kernel<H, RC, CLIP><<<grid, kThreads, smem, s>>>(a, tiles_per_shard);
+    const int64_t tiles_per_shard = staged_tiles_per_shard(static_cast<int64_t>(sp.S8) * 8);
+    const uint64_t tiles = static_cast<uint64_t>(tiles_per_shard) * static_cast<uint64_t>(sp.oend - sp.obeg);
+    const uint32_t grid = grid_for(tiles * kThreads, per_sm, sp.grid_cap);
+    fused_step_tma_kernel<H, RC, CLIP><<<grid, kTmaThreads, smem, s>>>(a, static_cast<uint64_t>(tiles_per_shard));
     return cudaGetLastError();
 }
 
