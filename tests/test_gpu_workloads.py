@@ -59,8 +59,8 @@ class Workload:
     global-norm clipping at `clip` with the norm taken by the reduce-scatters;
     the oracle steps the sample with the whole model's norm)."""
 
-    def __init__(self, name, path, sample=1 << 16, clip=0.0):
-        self.wl = wl = synth.workload(name)
+    def __init__(self, name, path, sample=1 << 16, clip=0.0, extra=None):
+        self.wl = wl = synth.workload(name) if isinstance(name, str) else name
         self.path, self.clip = path, clip
         self.R, self.dtype = wl["R"], wl["dtype"]
         self.lay = O.Layout(wl["numels"], wl["R"], 8, wl["bucket_elems"], wl["layer_ids"])
@@ -85,6 +85,8 @@ class Workload:
         inj = wl["inject"]
         if inj:
             s.append(np.array([starts[inj["tensor"]] + inj["element"]]))
+        if extra is not None:
+            s.append(np.asarray(extra))
         self.u = np.unique(np.concatenate(s).astype(np.int64))
         kk = np.searchsorted(starts, self.u, side="right") - 1
         self.p = (self.lay.offsets[kk] + (self.u - starts[kk])).astype(np.int64)
@@ -188,8 +190,8 @@ class Workload:
         return f
 
 
-def run(name, path, gather=False, steps=None, clip=0.0):
-    w = Workload(name, path, clip=clip)
+def run(name, path, gather=False, steps=None, clip=0.0, extra=None):
+    w = Workload(name, path, clip=clip, extra=extra)
     try:
         for _ in range(steps or w.wl["steps"]):
             ref = w.step()
@@ -269,3 +271,19 @@ def test_irregular_r16():
 
 def test_irregular_r2():
     run("irr_r2", "pingpong")
+
+
+def test_shard_longer_than_2_to_the_32_staged_step():
+    # R = 1 with a shard of 2^32 + 8 elements (69 GB in place): the staged
+    # kernel's tile index, shard offset and tile length pass 2^32, so every
+    # element past it must be updated; the sample covers the last 4104 elements
+    # (the last tile holds 8) besides random ones across the whole shard, and
+    # both layers (the second ends past 2^32) are gathered and compared whole
+    n = 1 << 31
+    wl = synth.custom_workload([n, n + 8], 1, 0, synth.NONE, 1.0, 1000, sigma=1e-4, index=31)
+    wl["steps"] = 2
+    p = Z.Plan(wl["numels"], None, 1, 0, 8, 0)
+    tile, tps, _ = Z.zero_plan_step_tiles(p.handle)
+    assert p.S == (1 << 32) + 8 and (tps - 1) * tile == 1 << 32
+    del p
+    run(wl, "inplace", gather=True, extra=np.arange((1 << 32) - 4096, (1 << 32) + 8))
