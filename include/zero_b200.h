@@ -654,6 +654,59 @@ zero_status zero_step_noalloc(const zero_plan_t* plan, const zero_loss_scale_con
                               float* const* v, void* const* param, void* stream);
 
 /* ------------------------------------------------------------------------ */
+/* Buffers shared across the processes of a multi-GPU job (CUDA IPC).       */
+/* ------------------------------------------------------------------------ */
+
+/*
+ * One rank's device buffer as its peers need it to map it: the IPC handle of
+ * the cudaMalloc allocation that holds the buffer, the buffer's byte offset
+ * in that allocation and the allocation's size. Plain bytes: a job passes it
+ * between its processes with any collective.
+ */
+typedef struct {
+    uint8_t handle[64];
+    int64_t offset;
+    int64_t alloc_bytes;
+} zero_ipc_handle;
+
+/*
+ * zero_ipc_export -- describe the device buffer at `ptr` for the other
+ * processes of the job. With one process per GPU, rank o's fused step and
+ * gathers read every peer's gradient replica and parameter shard; the peers
+ * reach those buffers through zero_ipc_open.
+ * Defines: the exchanges of [legal] "Reduce-Scatter" and "All-Gather on
+ * Demand" (each rank reads its partition of every peer's gradients, and
+ * every layer's parameters from their owners) as peer reads over NVLink.
+ * ptr: any address inside a device allocation made with cudaMalloc (for
+ * example a PyTorch tensor from its default allocator); an allocation from
+ * a virtual-memory pool cannot be exported and returns ZERO_ERR_CUDA. The
+ * caller keeps the allocation alive until every peer has closed its handle.
+ * Errors: ZERO_ERR_INVALID_ARG (NULL, or host memory), ZERO_ERR_CUDA.
+ */
+zero_status zero_ipc_export(const void* ptr, zero_ipc_handle* out);
+
+/*
+ * zero_ipc_open -- map a buffer that another process exported (on another
+ * GPU of this node) into this process: *out is its device address here,
+ * which the entry points above accept as a peer's buffer (plain loads and
+ * 1-D bulk copies; never a multicast load). The allocation is mapped once
+ * per process however many of its buffers are opened; peer access to the
+ * exporting GPU is enabled for this mapping. Call with the device that will
+ * read the buffer current.
+ * Errors: ZERO_ERR_INVALID_ARG, ZERO_ERR_RANGE (an offset outside the
+ * allocation), ZERO_ERR_CUDA (for instance a handle from this process).
+ */
+zero_status zero_ipc_open(const zero_ipc_handle* h, void** out);
+
+/*
+ * zero_ipc_close -- end one zero_ipc_open of this handle; the allocation is
+ * unmapped when its last open buffer is closed. Nothing may still read the
+ * buffer (synchronize first). Errors: ZERO_ERR_INVALID_ARG, ZERO_ERR_STATE
+ * (the handle is not open here), ZERO_ERR_CUDA.
+ */
+zero_status zero_ipc_close(const zero_ipc_handle* h);
+
+/* ------------------------------------------------------------------------ */
 /* Overlap and prefetch scheduling (a communication stream owned by the     */
 /* context, created on first use with the highest stream priority).         */
 /* ------------------------------------------------------------------------ */

@@ -194,3 +194,18 @@ def test_staged_step_tiles_cover_long_shards(R, P):
     assert 8 <= last <= tile and last % 8 == 0
     if P == (1 << 32) + 8:
         assert p.S == (1 << 32) + 8 and tps == (1 << 21) + 1 and last == 8
+
+
+def test_ipc_argument_errors_without_a_device():
+    # the checks that need no GPU: a NULL buffer, an offset outside the
+    # exported allocation, closing a handle that was never opened
+    with pytest.raises(Z.ZeroError) as e:
+        Z.zero_ipc_export(0)
+    assert e.value.status == Z.ZERO_ERR_INVALID_ARG
+    blob = bytes(64) + (4096).to_bytes(8, "little") + (4096).to_bytes(8, "little")
+    with pytest.raises(Z.ZeroError) as e:
+        Z.zero_ipc_open(blob)
+    assert e.value.status == Z.ZERO_ERR_RANGE
+    with pytest.raises(Z.ZeroError) as e:
+        Z.zero_ipc_close(bytes(80))
+    assert e.value.status == Z.ZERO_ERR_STATE

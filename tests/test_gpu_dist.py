@@ -1,4 +1,4 @@
-"""DistributedZero (the multi-GPU ZeRO step over symmetric memory) launched
+"""DistributedZero (the multi-GPU ZeRO step over CUDA-IPC peer mappings) launched
 under torch.distributed.run on the GPUs this machine offers, compared with
 the oracle in the worker (tests/dist_worker.py)."""
 import os

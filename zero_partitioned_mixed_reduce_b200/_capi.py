@@ -117,6 +117,15 @@ _sig("zero_plan_bucket", _S, [_P, C.c_int64, C.POINTER(C.c_int64), C.POINTER(C.c
 _sig("zero_plan_layer", _S, [_P, C.c_int64, C.POINTER(C.c_int64), C.POINTER(C.c_int64)])
 _sig("zero_plan_memory", _S, [_P, C.c_int32, C.POINTER(C.c_int64)])
 _sig("zero_plan_step_tiles", _S, [_P, C.POINTER(C.c_int64), C.POINTER(C.c_int64), C.POINTER(C.c_int64)])
+
+
+class zero_ipc_handle(C.Structure):
+    _fields_ = [("handle", C.c_uint8 * 64), ("offset", C.c_int64), ("alloc_bytes", C.c_int64)]
+
+
+_sig("zero_ipc_export", _S, [_P, C.POINTER(zero_ipc_handle)])
+_sig("zero_ipc_open", _S, [C.POINTER(zero_ipc_handle), C.POINTER(C.c_void_p)])
+_sig("zero_ipc_close", _S, [C.POINTER(zero_ipc_handle)])
 _sig("zero_ctx_create", _S, [_P, C.POINTER(zero_loss_scale_config), C.POINTER(_P)])
 _sig("zero_ctx_destroy", _S, [_P])
 _sig("zero_ctx_reserve_steps", _S, [_P, C.c_int64, C.c_double, C.c_double, _P])
@@ -254,6 +263,27 @@ def zero_plan_memory(plan, stage):
     b = C.c_int64()
     _check(_lib.zero_plan_memory(plan, stage, C.byref(b)))
     return b.value
+
+
+def zero_ipc_export(ptr):
+    """The IPC description (bytes) of the device buffer at ptr, for the job's
+    other processes."""
+    h = zero_ipc_handle()
+    _check(_lib.zero_ipc_export(_addr(ptr), C.byref(h)))
+    return C.string_at(C.addressof(h), C.sizeof(h))
+
+
+def zero_ipc_open(blob):
+    """Map a buffer another process exported; returns its device address here."""
+    h = zero_ipc_handle.from_buffer_copy(blob)
+    p = C.c_void_p()
+    _check(_lib.zero_ipc_open(C.byref(h), C.byref(p)))
+    return p.value
+
+
+def zero_ipc_close(blob):
+    h = zero_ipc_handle.from_buffer_copy(blob)
+    _check(_lib.zero_ipc_close(C.byref(h)))
 
 
 def zero_plan_step_tiles(plan):

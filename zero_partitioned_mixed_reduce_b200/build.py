@@ -36,7 +36,7 @@ CXX_FLAGS = ["-O2", "-std=c++17", "-fPIC", "-Wall", "-Wextra", "-ffp-contract=of
 CXX_EXTRA = {"cpu_adam.cpp": ["-O3", "-pthread", "-fno-math-errno"]}
 
 CU_SOURCES = ["kernels.cu", "noalloc.cu", "norm_slots.cu"]
-CPP_SOURCES = ["plan.cpp", "capi.cpp", "sched.cpp", "cpu_adam.cpp", "trace.cpp"]
+CPP_SOURCES = ["plan.cpp", "capi.cpp", "sched.cpp", "cpu_adam.cpp", "trace.cpp", "ipc.cpp"]
 
 
 def _sources():

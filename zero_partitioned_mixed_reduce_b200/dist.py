@@ -1,8 +1,10 @@
 """ZeRO across GPUs: one process per GPU, rank o owns shard o.
 
-Each rank keeps its full gradient buffer and its half parameter shard in
-symmetric memory (torch.distributed._symmetric_memory), so every rank can
-read every other rank's buffers with plain loads over NVLink. A step is:
+Each rank's full gradient buffer and half parameter shards are shared with
+its peers through CUDA IPC (zero_ipc_export / zero_ipc_open: the handles
+travel in one all_gather_object), so every rank reads every other rank's
+buffers with plain loads over NVLink: a plain peer mapping, with no NVLink
+multicast object and no allocator of its own. A step is:
 
   1. a one-element all-reduce on the compute stream, so that every rank's
      gradients are written before any rank reads them;
@@ -52,8 +54,8 @@ class DistributedZero:
     def __init__(self, numels, layer_ids=None, dtype=Z.ZERO_BF16, mode=Z.ZERO_SCALE_NONE,
                  init_scale=1.0, growth_interval=1000, tensor_align=8, bucket_elems=0, group=None,
                  accumulate=False, norm_divisor=None):
-        import torch.distributed._symmetric_memory as symm
         self.group = group or dist.group.WORLD
+        self._opened = []  # peers' IPC handles this rank has mapped
         self.world = dist.get_world_size(self.group)
         self.rank = dist.get_rank(self.group)
         self.plan = Plan(numels, layer_ids, self.world, dtype, tensor_align, bucket_elems)
@@ -62,25 +64,15 @@ class DistributedZero:
         half = HALF[dtype]
         self.dtype, self.mode = dtype, mode
         # this rank's full gradient buffer, readable by every rank
-        self.grads = symm.empty(T, dtype=half, device=dev)
-        self.grads.zero_()
-        h = symm.rendezvous(self.grads, self.group.group_name)
-        self.grad_ptrs = [int(h.buffer_ptrs[r]) for r in range(R)]
-        self._handles = [h]
+        self.grads = torch.zeros(T, dtype=half, device=dev)
+        self.grad_ptrs = self._share(self.grads)
         sets = 2 if mode == Z.ZERO_SCALE_DYNAMIC else 1
         self.sets = sets
         self.master = [torch.zeros(S, dtype=torch.float32, device=dev) for _ in range(sets)]
         self.m = [torch.zeros(S, dtype=torch.float32, device=dev) for _ in range(sets)]
         self.v = [torch.zeros(S, dtype=torch.float32, device=dev) for _ in range(sets)]
-        self.param = []
-        self.param_ptrs = []
-        for _ in range(sets):
-            p = symm.empty(S, dtype=half, device=dev)
-            p.zero_()
-            hp = symm.rendezvous(p, self.group.group_name)
-            self.param.append(p)
-            self.param_ptrs.append([int(hp.buffer_ptrs[r]) for r in range(R)])
-            self._handles.append(hp)
+        self.param = [torch.zeros(S, dtype=half, device=dev) for _ in range(sets)]
+        self.param_ptrs = [self._share(p) for p in self.param]
 
         def own(x):  # pointer list with only this rank's shard filled in
             return [x.data_ptr() if r == self.rank else None for r in range(R)]
@@ -104,6 +96,24 @@ class DistributedZero:
         self.partial = torch.zeros(2, dtype=torch.float64, device=dev)
         self.norm = torch.zeros(2, dtype=torch.float64, device=dev)
         self.token = torch.zeros(1, dtype=torch.float32, device=dev)
+
+    def _share(self, t):
+        """Every rank's device address of its own tensor `t` (one per rank, the
+        same shape everywhere): this rank's pointer, and the peers' buffers
+        mapped through CUDA IPC. The tensors stay alive until close()."""
+        torch.cuda.synchronize()  # t is allocated and initialized before a peer maps it
+        if self.world == 1:
+            return [t.data_ptr()]
+        blobs = [None] * self.world
+        dist.all_gather_object(blobs, Z.zero_ipc_export(t), group=self.group)
+        ptrs = []
+        for r in range(self.world):
+            if r == self.rank:
+                ptrs.append(t.data_ptr())
+            else:
+                ptrs.append(Z.zero_ipc_open(blobs[r]))
+                self._opened.append(blobs[r])
+        return ptrs
 
     def load(self, master_padded, param_padded):
         """Initialize this rank's shard from padded flat master (fp32) and param
@@ -260,7 +270,16 @@ class DistributedZero:
         return getattr(self, field)[k]
 
     def close(self):
+        """Release the context and unmap the peers' buffers. Every rank calls
+        it; no rank frees its own shared buffers before all have unmapped them
+        (the barrier at the end)."""
         if self.ctx:
             torch.cuda.synchronize()
             Z.zero_ctx_destroy(self.ctx)
             self.ctx = None
+        if self._opened:
+            for blob in self._opened:
+                Z.zero_ipc_close(blob)
+            self._opened = []
+        if self.world > 1:
+            dist.barrier(self.group)
