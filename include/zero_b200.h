@@ -679,8 +679,9 @@ typedef struct {
  * every layer's parameters from their owners) as peer reads over NVLink.
  * ptr: any address inside a device allocation made with cudaMalloc (for
  * example a PyTorch tensor from its default allocator); an allocation from
- * a virtual-memory pool cannot be exported and returns ZERO_ERR_CUDA. The
- * caller keeps the allocation alive until every peer has closed its handle.
+ * a virtual-memory pool cannot be exported and returns ZERO_ERR_CUDA. Call
+ * with the device that owns `ptr` current. The caller keeps the allocation
+ * alive until every peer has closed its handle.
  * Errors: ZERO_ERR_INVALID_ARG (NULL, or host memory), ZERO_ERR_CUDA.
  */
 zero_status zero_ipc_export(const void* ptr, zero_ipc_handle* out);
