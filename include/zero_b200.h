@@ -418,16 +418,31 @@ zero_status zero_step(zero_ctx_t* ctx, const zero_adamw* hp, const zero_state* s
  *    (ZERO_ERR_STATE) unless every slot it needs is current and was taken
  *    with this call's grad_divisor. Every zero_step_ex marks the slots
  *    used up.
+ *  flags & ZERO_STEP_PUSH_PARAMS: the step also writes every updated half
+ *    parameter vector into the full-model parameter buffers registered with
+ *    zero_ctx_set_param_push, one per rank (the ZeRO-1/2 all-gather of the
+ *    updated parameters, done by the step itself): buffer [dst][r] for every
+ *    rank r, where dst is the state set the step writes (1-cur with
+ *    ping-pong, else cur), at the element's flat index. After the step (and,
+ *    for a sharded step, the commit), each rank's buffer of set cur holds
+ *    the whole updated model, padding zero. 2 more bytes per element per
+ *    rank are written; with one process per GPU the peers' buffers are
+ *    peer-mapped (zero_ipc_open) and written with plain stores, so the
+ *    all-gather's NVLink traffic leaves while the step streams HBM.
  * Defines: not on the pages (clipping and accumulation are common practice
- * around ZeRO training loops, not part of the method the pages describe).
+ * around ZeRO training loops, not part of the method the pages describe);
+ * the parameter push follows [instr] ZeRO-1 "Mechanism" (the updated
+ * partitions are all-gathered so that every process holds the full model).
  * Errors: as zero_step, plus ZERO_ERR_INVALID_ARG for a divisor < 1, a
  * negative or non-finite max norm, unknown flags, ZERO_STEP_ADD_ACC
  * without grads, without state->acc or with clipping, or
  * ZERO_STEP_NORM_FROM_RS with grads or without clipping; ZERO_ERR_STATE for
- * ZERO_STEP_NORM_FROM_RS without current norm slots.
+ * ZERO_STEP_NORM_FROM_RS without current norm slots, or for
+ * ZERO_STEP_PUSH_PARAMS without registered buffers for the set written.
  */
 #define ZERO_STEP_ADD_ACC 1
 #define ZERO_STEP_NORM_FROM_RS 2
+#define ZERO_STEP_PUSH_PARAMS 4
 typedef struct {
     double grad_divisor;
     double max_grad_norm;
@@ -436,6 +451,20 @@ typedef struct {
 } zero_step_opts;
 zero_status zero_step_ex(zero_ctx_t* ctx, const zero_adamw* hp, const zero_state* state,
                          const void* const* grads, const zero_step_opts* opts, void* stream);
+
+/*
+ * zero_ctx_set_param_push -- register the full-model parameter buffers that
+ * steps with ZERO_STEP_PUSH_PARAMS write: full0[r] (state set 0) and
+ * full1[r] (set 1, needed once ping-pong state is used), for r in [0, R),
+ * each T half elements, 16-byte aligned, caller-owned; with one process per
+ * GPU, rank r's buffers as this process maps them (its own, or a peer's
+ * through zero_ipc_open). full0 == NULL clears the registration. The
+ * pointers are copied; the buffers must outlive the steps that write them.
+ * Defines: [instr] ZeRO-1 "Mechanism" (every process ends the step with the
+ * full updated parameters).
+ * Errors: ZERO_ERR_INVALID_ARG (a NULL entry), ZERO_ERR_ALIGN.
+ */
+zero_status zero_ctx_set_param_push(zero_ctx_t* ctx, void* const* full0, void* const* full1);
 
 /*
  * zero_step_shard -- the fused step (grads != NULL path of zero_step) on
@@ -476,7 +505,10 @@ zero_status zero_step_shard(zero_ctx_t* ctx, const zero_adamw* hp, const zero_st
  *    min(1, max_norm / (sqrt(global_norm_sq) + 1e-6)) is formed from it on
  *    the device. global_norm_sq may be NULL without clipping.
  *  - opts->flags may hold ZERO_STEP_ADD_ACC (fused path, as for
- *    zero_step_ex): only the owners' accumulators are read.
+ *    zero_step_ex): only the owners' accumulators are read; and
+ *    ZERO_STEP_PUSH_PARAMS: the owners' updated parameters are written into
+ *    every rank's registered full-model buffer of the set the step writes,
+ *    so that after the commit each rank holds the whole model in set cur.
  * partial and the commit are as for zero_step_shard. Running every owner
  * range in one process, with the partials summed, gives exactly zero_step_ex.
  * Defines: [instr] ZeRO-2 "Mechanism"; clipping and accumulation are not on

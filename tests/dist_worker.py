@@ -26,7 +26,7 @@ def main():
     dist.init_process_group("nccl")
     rank, world = dist.get_rank(), dist.get_world_size()
     numels, layer_ids = [70_001, 13, 4096, 999], [0, 0, 1, 1]
-    dz = DistributedZero(numels, layer_ids, Z.ZERO_FP16, Z.ZERO_SCALE_DYNAMIC, 256.0, 3)
+    dz = DistributedZero(numels, layer_ids, Z.ZERO_FP16, Z.ZERO_SCALE_DYNAMIC, 256.0, 3, push_params=True)
     wl = synth.custom_workload(numels, world, Z.ZERO_FP16, Z.ZERO_SCALE_DYNAMIC, 256.0, 3, sigma=1e-2,
                                layer_ids=layer_ids, index=55)
     lay = O.Layout(numels, world, 8, 0, layer_ids)
@@ -54,6 +54,10 @@ def main():
         flat[idx] = ost.master
         mine = dz.current("master").cpu().numpy()
         assert np.array_equal(mine.view(np.uint32), flat[rank * S:(rank + 1) * S].view(np.uint32)), step
+        # the parameters every rank's step pushed: the whole model on every rank
+        pfull = np.zeros(dz.plan.T, np.uint16)
+        pfull[idx] = ost.param
+        assert np.array_equal(u16(dz.full_params()), pfull), step
     # ZeRO-3 gather from every rank's shard
     pflat = np.zeros(dz.plan.T, np.uint16)
     pflat[idx] = ost.param

@@ -25,6 +25,7 @@ ZERO_RS_ACCUMULATE = 1
 ZERO_RS_NORM = 2
 ZERO_STEP_ADD_ACC = 1
 ZERO_STEP_NORM_FROM_RS = 2
+ZERO_STEP_PUSH_PARAMS = 4
 ZERO_TRACE_REDUCE_SCATTER, ZERO_TRACE_STEP, ZERO_TRACE_GATHER, ZERO_TRACE_NORM, ZERO_TRACE_COMMIT = 1, 2, 3, 4, 5
 TRACE_NAMES = {0: "untimed", 1: "reduce_scatter", 2: "step", 3: "gather", 4: "norm", 5: "commit"}
 
@@ -130,6 +131,7 @@ _sig("zero_ctx_create", _S, [_P, C.POINTER(zero_loss_scale_config), C.POINTER(_P
 _sig("zero_ctx_destroy", _S, [_P])
 _sig("zero_ctx_reserve_steps", _S, [_P, C.c_int64, C.c_double, C.c_double, _P])
 _sig("zero_ctx_set_grad_divisor", _S, [_P, C.c_double])
+_sig("zero_ctx_set_param_push", _S, [_P, _PP, _PP])
 _sig("zero_test_drop_tile", _S, [_P, C.c_int64])
 _sig("zero_reduce_scatter_bucket", _S, [_P, C.c_int64, _PP, _PP, _P])
 _sig("zero_step", _S, [_P, C.POINTER(zero_adamw), C.POINTER(zero_state), _PP, _P])
@@ -375,6 +377,15 @@ def zero_ctx_set_grad_divisor(ctx, grad_divisor):
     _check(_lib.zero_ctx_set_grad_divisor(ctx, float(grad_divisor)))
 
 
+def zero_ctx_set_param_push(ctx, full0, full1=None):
+    """Register every rank's full-model parameter buffer of state set 0
+    (full0) and set 1 (full1) for steps with ZERO_STEP_PUSH_PARAMS; full0 None
+    clears the registration."""
+    a = _ptr_array(full0)
+    b = _ptr_array(full1)
+    _check(_lib.zero_ctx_set_param_push(ctx, a[0] if a else None, b[0] if b else None))
+
+
 def zero_reduce_scatter_bucket_ex(ctx, bucket, grads, acc, flags=0, stream=None):
     """flags: ZERO_RS_ACCUMULATE adds to the accumulators; ZERO_RS_NORM also
     records the bucket's share of the clipping norm."""
@@ -397,7 +408,9 @@ def zero_step_ex(ctx, hp, state: StateHandle, grads=None, grad_divisor=1.0, max_
                  stream=None, flags=0):
     """zero_step with a grad divisor, global-norm clipping and flags
     (ZERO_STEP_ADD_ACC: the fused step adds state's accumulators;
-    ZERO_STEP_NORM_FROM_RS: the clipping norm from the reduce-scatters' shares)."""
+    ZERO_STEP_NORM_FROM_RS: the clipping norm from the reduce-scatters' shares;
+    ZERO_STEP_PUSH_PARAMS: the step also writes every rank's registered
+    full-model parameter buffer)."""
     if isinstance(hp, dict):
         hp = zero_adamw(hp["lr"], hp["beta1"], hp["beta2"], hp["eps"], hp["weight_decay"])
     g = None

@@ -469,7 +469,7 @@ zero_status check_step_opts(const zero_step_opts* opts, bool fused, const char* 
         !std::isfinite(o.max_grad_norm) || o.reserved != 0)
         return zb_fail(ZERO_ERR_INVALID_ARG,
                        std::string(where) + ": need grad_divisor >= 1, finite max_grad_norm >= 0, reserved 0");
-    if (o.flags & ~static_cast<int64_t>(ZERO_STEP_ADD_ACC | ZERO_STEP_NORM_FROM_RS))
+    if (o.flags & ~static_cast<int64_t>(ZERO_STEP_ADD_ACC | ZERO_STEP_NORM_FROM_RS | ZERO_STEP_PUSH_PARAMS))
         return zb_fail(ZERO_ERR_INVALID_ARG, std::string(where) + ": unknown flags");
     if ((o.flags & ZERO_STEP_ADD_ACC) && (!fused || o.max_grad_norm > 0.0))
         return zb_fail(ZERO_ERR_INVALID_ARG,
@@ -491,6 +491,26 @@ zero_status check_hp(const zero_adamw* hp, const char* where) {
     return ZERO_OK;
 }
 
+// ZERO_STEP_PUSH_PARAMS: the registered full-model buffers of every set the
+// step may write (both with ping-pong state) into p->full; none without it.
+zero_status fill_push_ptrs(const zero_ctx_t* ctx, const zero_step_opts& o, int sets, const char* where,
+                           zb::RankPtrs* p) {
+    const bool push = (o.flags & ZERO_STEP_PUSH_PARAMS) != 0;
+    for (int k = 0; k < 2; ++k)
+        for (int r = 0; r < ctx->R; ++r) p->full[k][r] = nullptr;
+    if (!push) return ZERO_OK;
+    for (int k = 0; k < sets; ++k)
+        if (ctx->push_full[k].size() != static_cast<size_t>(ctx->R))
+            return zb_fail(ZERO_ERR_STATE, std::string(where) + ": ZERO_STEP_PUSH_PARAMS, but no full-model buffers of "
+                                                                 "state set " + std::to_string(k) +
+                                                                 " are registered (zero_ctx_set_param_push)");
+    for (int k = 0; k < 2; ++k) {
+        const int from = k < sets ? k : 0;  // one set: both slots alias set 0
+        for (int r = 0; r < ctx->R; ++r) p->full[k][r] = ctx->push_full[from][static_cast<size_t>(r)];
+    }
+    return ZERO_OK;
+}
+
 // Everything a step launch needs, for owners [owner_lo, owner_hi).
 zb::StepParams step_params(const zero_ctx_t* ctx, const zero_adamw* hp, const zero_step_opts& o, int sets,
                            int32_t owner_lo, int32_t owner_hi, double* partial) {
@@ -506,6 +526,7 @@ zb::StepParams step_params(const zero_ctx_t* ctx, const zero_adamw* hp, const ze
     sp.max_norm = o.max_grad_norm;
     sp.clip = o.max_grad_norm > 0.0 ? 1 : 0;
     sp.add_acc = (o.flags & ZERO_STEP_ADD_ACC) ? 1 : 0;
+    sp.push = (o.flags & ZERO_STEP_PUSH_PARAMS) ? 1 : 0;
     return sp;
 }
 
@@ -552,6 +573,7 @@ extern "C" zero_status zero_step_ex(zero_ctx_t* ctx, const zero_adamw* hp, const
             p.g[r] = fused ? grads[r] : nullptr;
             p.acc[r] = (!fused || add_acc) ? state->acc[r] : nullptr;
         }
+        if ((s = fill_push_ptrs(ctx, o, sets, "zero_step", &p)) != ZERO_OK) return s;
         // with ZERO_STEP_NORM_FROM_RS: the current norm slots, whole range or
         // every bucket, each taken with this step's divisor
         const size_t nb = ctx->bucket_lo.size();
@@ -791,6 +813,7 @@ extern "C" zero_status zero_step_shard_ex(zero_ctx_t* ctx, const zero_adamw* hp,
                 p.param[k][r] = owned ? state->param[from][r] : nullptr;
             }
         }
+        if ((s = fill_push_ptrs(ctx, o, sets, where, &p)) != ZERO_OK) return s;
         ZbTraceScope trace(ctx, ZERO_TRACE_STEP, cs, owner_lo);
         cudaError_t e = cudaSuccess;
         if (clip) e = zb::launch_clip_from_norm(sp, global_norm_sq, cs);
@@ -800,6 +823,33 @@ extern "C" zero_status zero_step_shard_ex(zero_ctx_t* ctx, const zero_adamw* hp,
         if (fused) ctx->drop_tile = 0xffffffffu;
         ctx->shard_pingpong = sp.pingpong;
         if (sp.pingpong) ctx->two_sets = true;
+        return ZERO_OK;
+    });
+}
+
+extern "C" zero_status zero_ctx_set_param_push(zero_ctx_t* ctx, void* const* full0, void* const* full1) {
+    return zb_guarded("zero_ctx_set_param_push", [&]() -> zero_status {
+        if (!ctx) return zb_fail(ZERO_ERR_INVALID_ARG, "zero_ctx_set_param_push: ctx is NULL");
+        if (!full0) {
+            ctx->push_full[0].clear();
+            ctx->push_full[1].clear();
+            return ZERO_OK;
+        }
+        void* const* sets[2] = {full0, full1};
+        std::vector<void*> got[2];
+        for (int k = 0; k < 2; ++k) {
+            if (!sets[k]) continue;
+            for (int r = 0; r < ctx->R; ++r) {
+                if (!sets[k][r])
+                    return zb_fail(ZERO_ERR_INVALID_ARG, "zero_ctx_set_param_push: full" + std::to_string(k) + "[" +
+                                                             std::to_string(r) + "] is NULL");
+                if (!aligned(sets[k][r], 16))
+                    return zb_fail(ZERO_ERR_ALIGN, "zero_ctx_set_param_push: a buffer is not 16-byte aligned");
+                got[k].push_back(sets[k][r]);
+            }
+        }
+        ctx->push_full[0] = std::move(got[0]);
+        ctx->push_full[1] = std::move(got[1]);
         return ZERO_OK;
     });
 }

@@ -68,6 +68,9 @@ struct StepParams {
     // test support (zero_test_drop_tile): the staged kernel issues no copy
     // for this tile, so the block waiting for it gives up after its limit
     uint32_t drop_tile = 0xffffffffu;
+    // the step also writes each updated parameter vector into every rank's
+    // full-model buffer RankPtrs::full[dst][r] (ZERO_STEP_PUSH_PARAMS)
+    int32_t push = 0;
 };
 
 // Rank pointer tables, sized for the largest R.
@@ -78,6 +81,7 @@ struct RankPtrs {
     float* m[2][ZERO_MAX_RANKS];
     float* v[2][ZERO_MAX_RANKS];
     void* param[2][ZERO_MAX_RANKS];
+    void* full[2][ZERO_MAX_RANKS];  // full-model parameter buffers of the push
 };
 
 // A reduce-scatter's share of the clipping norm (ZERO_RS_NORM): the launch
@@ -171,6 +175,7 @@ struct zero_ctx_s {
     std::vector<double> rs_norm_div;
     std::vector<int64_t> rs_norm_owner;  // owner range of each share: lo << 32 | hi
     double grad_divisor = 1.0;    // the divisor ZERO_RS_NORM unscales by
+    std::vector<void*> push_full[2];  // zero_ctx_set_param_push: R buffers per state set (empty: none)
     zero_trace* trace = nullptr;  // per-call trace while started
 };
 

@@ -181,9 +181,14 @@ struct FusedArgs {
     float* m[2][CAP];
     float* v[2][CAP];
     uint4* param[2][CAP];
+    uint4* full[2][CAP];    // PUSH variant: every rank's full-model parameter buffer
 };
 
-template <typename H, int RC, bool CLIP, bool ACC = false>
+// PUSH: each updated parameter vector is also stored into every rank's
+// full-model buffer of the set written (the ZeRO-1/2 all-gather of the
+// parameters, done by the step); with one process per GPU those stores go
+// to peer-mapped memory over NVLink while the step streams HBM.
+template <typename H, int RC, bool CLIP, bool ACC = false, bool PUSH = false>
 __global__ void __launch_bounds__(kThreads)
     fused_step_kernel(const __grid_constant__ FusedArgs<RC == 0 ? ZERO_MAX_RANKS : RC> a) {
     const StepParams& sp = a.sp;
@@ -205,7 +210,8 @@ __global__ void __launch_bounds__(kThreads)
         const size_t j8 = static_cast<size_t>(vi - oc.base) * 8;
         if (!ZB_IN(vi < sp.T8 && o >= static_cast<uint32_t>(sp.obeg) && o < static_cast<uint32_t>(sp.oend) &&
                        vi - oc.base < sp.S8 && ptrs_ok(a.g, R) && a.master[src][o] && a.m[src][o] &&
-                       a.v[src][o] && a.master[dst][o] && a.m[dst][o] && a.v[dst][o] && a.param[dst][o],
+                       a.v[src][o] && a.master[dst][o] && a.m[dst][o] && a.v[dst][o] && a.param[dst][o] &&
+                       (!PUSH || ptrs_ok(a.full[dst], R)),
                    1, vi))
             continue;
         float acc[8];
@@ -248,7 +254,11 @@ __global__ void __launch_bounds__(kThreads)
         st_f8(a.master[dst][o] + j8, p);
         st_f8(a.m[dst][o] + j8, m);
         st_f8(a.v[dst][o] + j8, v);
-        st_u4(a.param[dst][o] + (j8 >> 3), pack8<H>(out));
+        const uint4 pk = pack8<H>(out);
+        st_u4(a.param[dst][o] + (j8 >> 3), pk);
+        if constexpr (PUSH) {
+            for (int r = 0; r < R; ++r) st_u4(a.full[dst][r] + vi, pk);
+        }
     }
     step_epilogue(sp, nrm, bad);
 }
@@ -473,9 +483,10 @@ struct AccArgs {
     float* m[2][ZERO_MAX_RANKS];
     float* v[2][ZERO_MAX_RANKS];
     uint4* param[2][ZERO_MAX_RANKS];
+    uint4* full[2][ZERO_MAX_RANKS];  // PUSH variant, as for the fused step
 };
 
-template <typename H, bool CLIP>
+template <typename H, bool CLIP, bool PUSH = false>
 __global__ void __launch_bounds__(kThreads) step_from_acc_kernel(const __grid_constant__ AccArgs a) {
     const StepParams& sp = a.sp;
     __shared__ Prologue pro;
@@ -497,7 +508,8 @@ __global__ void __launch_bounds__(kThreads) step_from_acc_kernel(const __grid_co
         const size_t j8 = static_cast<size_t>(vi - oc.base) * 8;
         if (!ZB_IN(o >= static_cast<uint32_t>(sp.obeg) && o < static_cast<uint32_t>(sp.oend) && vi - oc.base < sp.S8 &&
                        a.acc[o] && (skip || (a.master[src][o] && a.m[src][o] && a.v[src][o] &&
-                                             a.master[dst][o] && a.m[dst][o] && a.v[dst][o] && a.param[dst][o])),
+                                             a.master[dst][o] && a.m[dst][o] && a.v[dst][o] && a.param[dst][o] &&
+                                             (!PUSH || ptrs_ok(a.full[dst], sp.R)))),
                    5, vi))
             continue;
         const F8 acc = ld_f8(a.acc[o] + j8);
@@ -523,7 +535,11 @@ __global__ void __launch_bounds__(kThreads) step_from_acc_kernel(const __grid_co
         st_f8(a.master[dst][o] + j8, p);
         st_f8(a.m[dst][o] + j8, m);
         st_f8(a.v[dst][o] + j8, v);
-        st_u4(a.param[dst][o] + (j8 >> 3), pack8<H>(out));
+        const uint4 pk = pack8<H>(out);
+        st_u4(a.param[dst][o] + (j8 >> 3), pk);
+        if constexpr (PUSH) {
+            for (int r = 0; r < sp.R; ++r) st_u4(a.full[dst][r] + vi, pk);
+        }
     }
     step_epilogue(sp, nrm, false);
 }
@@ -949,7 +965,7 @@ uint32_t grid_for(uint64_t work_items, int per_sm, int cap) {
     return static_cast<uint32_t>(g > 0 ? g : 1);
 }
 
-template <typename H, int RC, bool CLIP, bool ACC = false>
+template <typename H, int RC, bool CLIP, bool ACC = false, bool PUSH = false>
 cudaError_t fused_t(const StepParams& sp, const RankPtrs& p, cudaStream_t s) {
     constexpr int CAP = RC == 0 ? ZERO_MAX_RANKS : RC;
     FusedArgs<CAP> a;
@@ -962,11 +978,12 @@ cudaError_t fused_t(const StepParams& sp, const RankPtrs& p, cudaStream_t s) {
             a.m[k][r] = p.m[k][r];
             a.v[k][r] = p.v[k][r];
             a.param[k][r] = static_cast<uint4*>(p.param[k][r]);
+            a.full[k][r] = static_cast<uint4*>(p.full[k][r]);
         }
     }
-    static const int per_sm = blocks_per_sm(fused_step_kernel<H, RC, CLIP, ACC>);
+    static const int per_sm = blocks_per_sm(fused_step_kernel<H, RC, CLIP, ACC, PUSH>);
     const uint32_t grid = grid_for(static_cast<uint64_t>(sp.oend - sp.obeg) * sp.S8, per_sm, sp.grid_cap);
-    fused_step_kernel<H, RC, CLIP, ACC><<<grid, kThreads, 0, s>>>(a);
+    fused_step_kernel<H, RC, CLIP, ACC, PUSH><<<grid, kThreads, 0, s>>>(a);
     return cudaGetLastError();
 }
 
@@ -1071,7 +1088,7 @@ cudaError_t rs_dispatch(int32_t R, int64_t S, int64_t lo, int64_t hi, DevState* 
     }
 }
 
-template <typename H, bool CLIP>
+template <typename H, bool CLIP, bool PUSH = false>
 cudaError_t acc_t(const StepParams& sp, const RankPtrs& p, cudaStream_t s) {
     AccArgs a;
     a.sp = sp;
@@ -1082,17 +1099,28 @@ cudaError_t acc_t(const StepParams& sp, const RankPtrs& p, cudaStream_t s) {
             a.m[k][r] = p.m[k][r];
             a.v[k][r] = p.v[k][r];
             a.param[k][r] = static_cast<uint4*>(p.param[k][r]);
+            a.full[k][r] = static_cast<uint4*>(p.full[k][r]);
         }
     }
-    static const int per_sm = blocks_per_sm(step_from_acc_kernel<H, CLIP>);
+    static const int per_sm = blocks_per_sm(step_from_acc_kernel<H, CLIP, PUSH>);
     const uint32_t grid = grid_for(static_cast<uint64_t>(sp.oend - sp.obeg) * sp.S8, per_sm, sp.grid_cap);
-    step_from_acc_kernel<H, CLIP><<<grid, kThreads, 0, s>>>(a);
+    step_from_acc_kernel<H, CLIP, PUSH><<<grid, kThreads, 0, s>>>(a);
     return cudaGetLastError();
+}
+
+// The step with the parameter push: the runtime-R register kernel, whatever R.
+template <typename H>
+cudaError_t fused_push_dispatch(const StepParams& sp, const RankPtrs& p, cudaStream_t s) {
+    if (sp.add_acc) return fused_t<H, 0, false, true, true>(sp, p, s);
+    if (sp.clip) return fused_t<H, 0, true, false, true>(sp, p, s);
+    return fused_t<H, 0, false, false, true>(sp, p, s);
 }
 
 }  // namespace
 
 cudaError_t launch_fused_step(const StepParams& sp, const RankPtrs& p, cudaStream_t s) {
+    if (sp.push)
+        return sp.dtype == ZERO_FP16 ? fused_push_dispatch<Fp16>(sp, p, s) : fused_push_dispatch<Bf16>(sp, p, s);
     if (sp.add_acc)
         return sp.dtype == ZERO_FP16 ? fused_acc_dispatch<Fp16>(sp, p, s) : fused_acc_dispatch<Bf16>(sp, p, s);
     if (sp.clip)
@@ -1106,6 +1134,11 @@ cudaError_t launch_fsm_commit(const StepParams& sp, const double* reduced, cudaS
 }
 
 cudaError_t launch_step_from_acc(const StepParams& sp, const RankPtrs& p, cudaStream_t s) {
+    if (sp.push) {
+        if (sp.clip)
+            return sp.dtype == ZERO_FP16 ? acc_t<Fp16, true, true>(sp, p, s) : acc_t<Bf16, true, true>(sp, p, s);
+        return sp.dtype == ZERO_FP16 ? acc_t<Fp16, false, true>(sp, p, s) : acc_t<Bf16, false, true>(sp, p, s);
+    }
     if (sp.clip) return sp.dtype == ZERO_FP16 ? acc_t<Fp16, true>(sp, p, s) : acc_t<Bf16, true>(sp, p, s);
     return sp.dtype == ZERO_FP16 ? acc_t<Fp16, false>(sp, p, s) : acc_t<Bf16, false>(sp, p, s);
 }

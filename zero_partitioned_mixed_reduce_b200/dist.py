@@ -39,7 +39,12 @@ no peer still reads this rank's gradients, and makes the compute stream wait
 for the communication stream. Every rank reports the same tensors in the
 same order, so the ranks issue the same collectives in the same order.
 
-ZeRO-3 layer gathers read the peers' parameter shards the same way.
+ZeRO-3 layer gathers read the peers' parameter shards the same way. Built
+with push_params=True (ZeRO-1/2: every rank keeps the whole model), each
+rank's step also stores its updated parameters into every rank's full-model
+buffer over the same peer mappings (ZERO_STEP_PUSH_PARAMS): the all-gather
+of the parameters leaves with the step's own stores, and after the commit
+full_params() holds the whole updated model on every rank.
 Argument marshalling only; the arithmetic runs in libzero_b200.so. The
 loads from peer memory are plain loads or bulk copies without multicast.
 """
@@ -53,7 +58,7 @@ from .state import HALF, Plan
 class DistributedZero:
     def __init__(self, numels, layer_ids=None, dtype=Z.ZERO_BF16, mode=Z.ZERO_SCALE_NONE,
                  init_scale=1.0, growth_interval=1000, tensor_align=8, bucket_elems=0, group=None,
-                 accumulate=False, norm_divisor=None):
+                 accumulate=False, norm_divisor=None, push_params=False):
         self.group = group or dist.group.WORLD
         self._opened = []  # peers' IPC handles this rank has mapped
         self.world = dist.get_world_size(self.group)
@@ -93,6 +98,13 @@ class DistributedZero:
         self.norm_divisor = norm_divisor
         if norm_divisor is not None:
             Z.zero_ctx_set_grad_divisor(self.ctx, float(norm_divisor))
+        # push_params: every rank's full-model parameter buffer, one per state
+        # set, written by every rank's step
+        self.push = bool(push_params)
+        if self.push:
+            self.full = [torch.zeros(T, dtype=half, device=dev) for _ in range(sets)]
+            self.full_ptrs = [self._share(f) for f in self.full]
+            Z.zero_ctx_set_param_push(self.ctx, self.full_ptrs[0], self.full_ptrs[1] if sets == 2 else None)
         self.partial = torch.zeros(2, dtype=torch.float64, device=dev)
         self.norm = torch.zeros(2, dtype=torch.float64, device=dev)
         self.token = torch.zeros(1, dtype=torch.float32, device=dev)
@@ -144,7 +156,7 @@ class DistributedZero:
             self.step_accumulated(hp, grad_divisor, max_grad_norm, stream)
             return
         k = float(self.micro + 1) if grad_divisor is None else grad_divisor
-        flags = Z.ZERO_STEP_ADD_ACC if self.micro > 0 else 0
+        flags = (Z.ZERO_STEP_ADD_ACC if self.micro > 0 else 0) | self._push_flag()
         dist.all_reduce(self.token, group=self.group)
         if max_grad_norm > 0:
             self._global_norm(self.grad_ptrs, None, k, stream)
@@ -153,6 +165,16 @@ class DistributedZero:
         dist.all_reduce(self.partial, group=self.group)
         Z.zero_step_commit(self.ctx, self.partial, stream)
         self.micro = 0
+
+    def _push_flag(self):
+        return Z.ZERO_STEP_PUSH_PARAMS if self.push else 0
+
+    def full_params(self):
+        """With push_params: this rank's copy of the whole updated model (the
+        current set), in the plan's flat layout."""
+        assert self.push, "construct with push_params=True"
+        k = self.loss_scale()["cur"] if self.sets == 2 else 0
+        return self.full[k]
 
     def _rs_flags(self):
         # every micro-batch takes its norm share: the last one leaves the share
@@ -234,7 +256,7 @@ class DistributedZero:
         elif max_grad_norm > 0:
             self._global_norm(None, self.acc_list, k, stream)
         Z.zero_step_shard_ex(self.ctx, hp, self.handle, None, self.rank, self.rank + 1, self.partial, k,
-                             max_grad_norm, self.norm, stream)
+                             max_grad_norm, self.norm, stream, flags=self._push_flag())
         dist.all_reduce(self.partial, group=self.group)
         Z.zero_step_commit(self.ctx, self.partial, stream)
         self.micro = 0
