@@ -90,6 +90,9 @@ def parse_args(argv=None):
     ap.add_argument("--dist", action="store_true",
                     help="the real multi-GPU ZeRO step over the job's GPUs (DistributedZero), also at "
                          "N = 1 (the default whenever N > 1)")
+    ap.add_argument("--zero2", action="store_true",
+                    help="sharded step: ZeRO-1/2 parameters (every rank keeps the whole model, which each "
+                         "rank's step pushes to every rank) instead of the ZeRO-3 layer gathers")
     ap.add_argument("--replicas", action="store_true",
                     help="with N > 1: N independent single-GPU copies of the workload (no collective on "
                          "the data path) instead of the sharded multi-GPU step")
@@ -1037,18 +1040,22 @@ def dist_layer_buckets(layers, cap):
     return buckets
 
 
-def dist_step_bytes(T, S, N):
+def dist_step_bytes(T, S, N, push=False):
     """Algorithmic bytes of one rank's share of the sharded step.
     hbm: the fused launch reads the rank's own replica slice and serves its
     N - 1 peers theirs (2N S), reads and writes its state (26 S); the gathers
     read every rank's parameter slice (2T across all ranks, each rank
     serving its own 2S to N readers: 2N S) and write the whole model (2T).
     nvlink: the bytes the rank reads from its peers (per direction, the same
-    amount it serves them): 2(N - 1) S in the step, 2(N - 1) S in the gathers."""
-    step_hbm = (2 * N + 26) * S
-    gather_hbm = 2 * N * S + 2 * T
-    nvlink_step = 2 * (N - 1) * S
-    nvlink_gather = 2 * (N - 1) * S
+    amount it serves them): 2(N - 1) S in the step, 2(N - 1) S in the gathers.
+    push (ZeRO-1/2): no gathers; the step also writes the whole model into the
+    rank's full buffer (its own 2S, and 2(N - 1) S its peers push: 2T of HBM
+    writes) and pushes its 2S to each of its N - 1 peers, the same 2(N - 1) S
+    per direction that the gathers would have moved, now during the step."""
+    step_hbm = (2 * N + 26) * S + (2 * T if push else 0)
+    gather_hbm = 0 if push else 2 * N * S + 2 * T
+    nvlink_step = 2 * (N - 1) * S + (2 * (N - 1) * S if push else 0)
+    nvlink_gather = 0 if push else 2 * (N - 1) * S
     return {"step_hbm": step_hbm, "gather_hbm": gather_hbm, "nvlink_step": nvlink_step,
             "nvlink_gather": nvlink_gather}
 
@@ -1095,7 +1102,7 @@ def run_dist(args, world, rank, local):
     wl = synth.workload(args.workload)
     restrict(wl, args.tensor_range)
     dz = DistributedZero(wl["numels"], wl["layer_ids"], wl["dtype"], wl["mode"], wl["init_scale"],
-                         wl["interval"], 8, wl["bucket_elems"])
+                         wl["interval"], 8, wl["bucket_elems"], push_params=args.zero2)
     plan = dz.plan
     T, S = plan.T, plan.S
     half = {0: torch.bfloat16, 1: torch.float16}[wl["dtype"]]
@@ -1120,8 +1127,9 @@ def run_dist(args, world, rank, local):
         dz.step(hp)
         if ev is not None:
             ev[1].record(stream)
-        for (f, _, _), o in zip(buckets, outs):
-            dz.gather_layers(f, o)
+        if not args.zero2:  # ZeRO-2 pushed the parameters within the step
+            for (f, _, _), o in zip(buckets, outs):
+                dz.gather_layers(f, o)
         if ev is not None:
             ev[2].record(stream)
 
@@ -1148,7 +1156,7 @@ def run_dist(args, world, rank, local):
     ms, units = aggregate(start.elapsed_time(end), float(plan.P) * K / N, N)
     step_ms, _ = aggregate(statistics.mean(e0.elapsed_time(e1) for e0, e1, _ in evs), 0.0, N)
     gather_ms, _ = aggregate(statistics.mean(e1.elapsed_time(e2) for _, e1, e2 in evs), 0.0, N)
-    nb = dist_step_bytes(T, S, N)
+    nb = dist_step_bytes(T, S, N, push=args.zero2)
     peak, peak_src = hbm_peak()
     roof = dist_roofline({"hbm": nb["step_hbm"], "nvlink": nb["nvlink_step"]}, step_ms, peak)
     roof.update({"kernel": "fused_step_kernel (sharded: one owner per rank) + loss-scale commit",
@@ -1164,23 +1172,26 @@ def run_dist(args, world, rank, local):
                    "R": N, "P": plan.P, "T": T, "S": S, "n_layers": len(plan.layers),
                    "path": "DistributedZero: 4-byte NCCL all-reduce (every replica written), fused "
                            "reduce-scatter+AdamW over the rank's shard reading the peers' replicas over "
-                           "NVLink (plain or 1-D bulk loads, no multicast), 16-byte NCCL all-reduce of "
-                           "{norm, overflow}, loss-scale commit, ZeRO-3 gather of every layer from every "
-                           "rank's shard",
+                           "NVLink (plain or 1-D bulk loads, no multicast)"
+                           + (", the updated parameters pushed into every rank's full-model buffer by the "
+                              "same kernel (ZeRO-1/2)" if args.zero2 else "")
+                           + ", 16-byte NCCL all-reduce of {norm, overflow}, loss-scale commit"
+                           + ("" if args.zero2 else ", ZeRO-3 gather of every layer from every rank's shard"),
                    "l2": f"inputs larger than L2 ({(nb['step_hbm'] + nb['gather_hbm']) / 1e9:.1f} GB "
                          "of HBM per rank per step, L2 126 MB)",
                    "parallelism": f"dp{N}: {N} GPU(s), one shard each",
-                   "gather": f"{len(buckets)} bucketed launches per step over every rank's shard",
+                   "gather": ("none: the step pushes the parameters (ZeRO-1/2)" if args.zero2 else
+                              f"{len(buckets)} bucketed launches per step over every rank's shard"),
                    "launch": "eager (the step issues NCCL all-reduces between its launches)"},
         "roofline": roof,
-        "gather": {"avg_ms_per_step": gather_ms, "elements": plan.L, "launches_per_step": len(buckets),
-                   "roofline": dist_roofline({"hbm": nb["gather_hbm"], "nvlink": nb["nvlink_gather"]},
-                                             gather_ms, peak)},
+        "gather": None if args.zero2 else {
+            "avg_ms_per_step": gather_ms, "elements": plan.L, "launches_per_step": len(buckets),
+            "roofline": dist_roofline({"hbm": nb["gather_hbm"], "nvlink": nb["nvlink_gather"]}, gather_ms, peak)},
         "per_rank_bytes": nb,
         "nccl": {"backend": dist.get_backend(), "world_size": N,
                  "version": ".".join(str(v) for v in torch.cuda.nccl.version())},
         "clocks": clk,
-        "gpu_launches": K * (2 + len(buckets)),
+        "gpu_launches": K * (2 + (0 if args.zero2 else len(buckets))),
         "state_check": "ok" if ok else f"t {f0['t']} -> {f1['t']}, overflow {f1['last_overflow']}",
     }
     if e2e_out is not None:

@@ -85,3 +85,13 @@ def test_tensor_range_selection():
     # one decoder layer of the Llama-style list: norms, q/k/v/o, gate/up/down
     assert len(wl["numels"]) == 9 and sum(wl["numels"]) == 100_669_440
     assert wl["layer_ids"] == [0] * 9
+
+
+def test_dist_bytes_with_the_parameter_push():
+    T, N = 8 * 1000, 4
+    S = T // N
+    nb = bench.dist_step_bytes(T, S, N, push=True)
+    assert nb["gather_hbm"] == 0 and nb["nvlink_gather"] == 0
+    assert nb["step_hbm"] == (2 * N + 26) * S + 2 * T
+    assert nb["nvlink_step"] == 4 * (N - 1) * S
+    assert bench.parse_args(["--zero2"]).zero2 and not bench.parse_args([]).zero2

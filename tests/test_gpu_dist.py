@@ -46,3 +46,18 @@ def test_bench_distributed_mode():
     assert out["value"] > 0 and out["config"]["R"] == 1 and out["state_check"] == "ok"
     assert out["roofline"]["bound"] in ("hbm", "nvlink") and out["roofline"]["achieved"] > 0
     assert out["gpu_launches"] > 0 and out["e2e"]["value"] > 0 and out["nccl"]["world_size"] == 1
+
+
+def test_bench_distributed_zero2_mode():
+    # bench.py --dist --zero2: the step pushes the parameters, no layer gathers
+    import json
+    env = dict(os.environ, NCCL_NVLS_ENABLE="0")
+    cmd = ["timeout", "-k", "30", "600", sys.executable, "-m", "torch.distributed.run", "--nnodes=1",
+           "--nproc-per-node=1", "--master-addr", "127.0.0.1", "--master-port", str(free_port()),
+           os.path.join(ROOT, "bench.py"), "--dist", "--zero2", "--workload", "gpt2s", "--steps", "3",
+           "--warmup", "3"]
+    r = subprocess.run(cmd, capture_output=True, text=True, env=env, cwd=ROOT)
+    assert r.returncode == 0, (r.stdout[-3000:], r.stderr[-3000:])
+    out = json.loads([ln for ln in r.stdout.splitlines() if ln.startswith("{")][-1])
+    assert out["gather"] is None and out["state_check"] == "ok" and "pushed" in out["config"]["path"]
+    assert out["per_rank_bytes"]["gather_hbm"] == 0 and out["value"] > 0
