@@ -68,6 +68,35 @@ def main():
             runs += 1
         finally:
             c.close()
+    # the parameter push (fused ping-pong and two-pass), R = 3 with packed tensors
+    for path in ("pingpong", "twopass"):
+        c = Case(numels, 3, O.FP16, 1, O.SCALE_STATIC, init_scale=64.0, path=path, layer_ids=layers, seed=300)
+        try:
+            full = [[c.g.half(c.plan.T, c.dtype) for _ in range(c.R)] for _ in range(c.sets)]
+            Z.zero_ctx_set_param_push(c.ctx, full[0], full[1] if c.sets == 2 else None)
+            for _ in range(2):
+                c.step_no += 1
+                g = c.make_grads()
+                for r in range(c.R):
+                    gp = np.zeros(c.plan.T, np.uint16)
+                    gp[c.idx] = g[r]
+                    c.grads[r].view(torch.int16).copy_(torch.from_numpy(gp.view(np.int16)))
+                if path == "twopass":
+                    Z.zero_reduce_scatter_bucket(c.ctx, -1, c.grads, c.acc)
+                Z.zero_step_ex(c.ctx, c.hp, c.handle, c.grads if path == "pingpong" else None,
+                               flags=Z.ZERO_STEP_PUSH_PARAMS)
+                O.step(c.ostate, g, O.AdamW(**{k: c.hp[k] for k in ("lr", "beta1", "beta2", "eps",
+                                                                    "weight_decay")}), c.ofsm)
+                c.g.check()
+                c.compare()
+            cur = c.gpu_fsm()["cur"] if c.sets == 2 else 0
+            want = np.zeros(c.plan.T, np.uint16)
+            want[c.idx] = c.ostate.param
+            from gpu_harness import u16
+            assert all(np.array_equal(u16(full[cur][r]), want) for r in range(c.R))
+            runs += 1
+        finally:
+            c.close()
     count, site, index = Z.zero_debug_bounds()
     print(json.dumps({"cases": runs, "count": count, "first_site": site, "first_index": index}))
 

@@ -24,5 +24,5 @@ def test_debug_build_records_no_out_of_range_access():
                        capture_output=True, text=True, env=env, cwd=ROOT, timeout=900)
     assert r.returncode == 0, (r.stdout[-3000:], r.stderr[-3000:])
     rec = json.loads(r.stdout.strip().splitlines()[-1])
-    assert rec["cases"] == 32
+    assert rec["cases"] == 34
     assert rec["count"] == 0, rec
