@@ -723,7 +723,7 @@ zero_status zero_ipc_export(const void* ptr, zero_ipc_handle* out);
  * GPU of this node) into this process: *out is its device address here,
  * which the entry points above accept as a peer's buffer (plain loads and
  * 1-D bulk copies; never a multicast load). The allocation is mapped once
- * per process however many of its buffers are opened; peer access to the
+ * per process and device however many of its buffers are opened; peer access to the
  * exporting GPU is enabled for this mapping. Call with the device that will
  * read the buffer current.
  * Errors: ZERO_ERR_INVALID_ARG, ZERO_ERR_RANGE (an offset outside the
@@ -732,9 +732,9 @@ zero_status zero_ipc_export(const void* ptr, zero_ipc_handle* out);
 zero_status zero_ipc_open(const zero_ipc_handle* h, void** out);
 
 /*
- * zero_ipc_close -- end one zero_ipc_open of this handle; the allocation is
- * unmapped when its last open buffer is closed. Nothing may still read the
- * buffer (synchronize first). Errors: ZERO_ERR_INVALID_ARG, ZERO_ERR_STATE
+ * zero_ipc_close -- end one zero_ipc_open of this handle (with the same
+ * device current); the allocation is unmapped when its last open buffer is
+ * closed. Nothing may still read the buffer (synchronize first). Errors: ZERO_ERR_INVALID_ARG, ZERO_ERR_STATE
  * (the handle is not open here), ZERO_ERR_CUDA.
  */
 zero_status zero_ipc_close(const zero_ipc_handle* h);

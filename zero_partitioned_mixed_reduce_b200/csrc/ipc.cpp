@@ -36,8 +36,9 @@ GetAddressRange address_range() {
     return fn;
 }
 
-// Allocations of other processes mapped into this one, by handle: the same
-// allocation may carry several exported buffers, and is mapped once.
+// Allocations of other processes mapped into this one, by reading device and
+// handle: the same allocation may carry several exported buffers, and is
+// mapped once per device that reads it.
 struct Mapping {
     void* base = nullptr;
     int refs = 0;
@@ -45,8 +46,9 @@ struct Mapping {
 std::mutex g_mu;
 std::map<std::string, Mapping> g_mapped;
 
-std::string key_of(const zero_ipc_handle* h) {
-    return std::string(reinterpret_cast<const char*>(h->handle), sizeof h->handle);
+std::string key_of(const zero_ipc_handle* h, int device) {
+    return std::to_string(device) + ":" +
+           std::string(reinterpret_cast<const char*>(h->handle), sizeof h->handle);
 }
 
 zero_status ipc_fail(const char* where, cudaError_t e, const char* hint = "") {
@@ -89,15 +91,19 @@ extern "C" zero_status zero_ipc_open(const zero_ipc_handle* h, void** out) {
         if (!h || !out) return zb_fail(ZERO_ERR_INVALID_ARG, "zero_ipc_open: NULL handle or output");
         if (h->offset < 0 || h->offset >= h->alloc_bytes)
             return zb_fail(ZERO_ERR_RANGE, "zero_ipc_open: offset outside the exported allocation");
+        int dev = 0;
+        cudaError_t de = cudaGetDevice(&dev);
+        if (de != cudaSuccess) return ipc_fail("zero_ipc_open", de);
+        const std::string key = key_of(h, dev);
         std::lock_guard<std::mutex> lock(g_mu);
-        Mapping& m = g_mapped[key_of(h)];
+        Mapping& m = g_mapped[key];
         if (m.refs == 0) {
             cudaIpcMemHandle_t ch;
             std::memcpy(&ch, h->handle, sizeof ch);
             void* base = nullptr;
             const cudaError_t e = cudaIpcOpenMemHandle(&base, ch, cudaIpcMemLazyEnablePeerAccess);
             if (e != cudaSuccess) {
-                g_mapped.erase(key_of(h));
+                g_mapped.erase(key);
                 return ipc_fail("zero_ipc_open", e);
             }
             m.base = base;
@@ -111,8 +117,14 @@ extern "C" zero_status zero_ipc_open(const zero_ipc_handle* h, void** out) {
 extern "C" zero_status zero_ipc_close(const zero_ipc_handle* h) {
     return zb_guarded("zero_ipc_close", [&]() -> zero_status {
         if (!h) return zb_fail(ZERO_ERR_INVALID_ARG, "zero_ipc_close: NULL handle");
+        int dev = 0;
+        cudaError_t de = cudaGetDevice(&dev);
+        if (de != cudaSuccess) {
+            cudaGetLastError();
+            dev = -1;  // no device: nothing can be open
+        }
         std::lock_guard<std::mutex> lock(g_mu);
-        auto it = g_mapped.find(key_of(h));
+        auto it = g_mapped.find(key_of(h, dev));
         if (it == g_mapped.end() || it->second.refs <= 0)
             return zb_fail(ZERO_ERR_STATE, "zero_ipc_close: the handle is not open in this process");
         if (--it->second.refs > 0) return ZERO_OK;
