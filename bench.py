@@ -1267,6 +1267,10 @@ def run_offload(args, world, rank, local):
     v = [pin(torch.zeros(S)) for _ in range(R)]
     param_host = [pin(torch.zeros(S, dtype=half)) for _ in range(R)]
     acc_host = [[pin(torch.zeros(S)) for _ in range(R)] for _ in range(2)]
+    # the reduce-scatters' overflow flag, taken on the GPU and copied down with
+    # the accumulators: a clean DYNAMIC step then runs in one pass on the CPU
+    flag_gpu = torch.zeros(1, dtype=torch.int32, device="cuda")
+    flag_host = [pin(torch.zeros(1, dtype=torch.int32)) for _ in range(2)]
     param_gpu = [torch.zeros(S, dtype=half, device="cuda") for _ in range(R)]
     copy = torch.cuda.Stream()
     d = 768 if args.workload == "gpt2s" else 2048
@@ -1281,12 +1285,14 @@ def run_offload(args, world, rank, local):
         for _ in range(n_gemm):
             x @ w
         Z.zero_reduce_scatter_bucket(ctx, -1, grads, acc_gpu)
+        Z.zero_take_overflow(ctx, flag_gpu)
         ev = torch.cuda.Event()
         ev.record()
         copy.wait_event(ev)
         with torch.cuda.stream(copy):
             for r in range(R):
                 acc_host[slot][r].copy_(acc_gpu[r], non_blocking=True)
+            flag_host[slot].copy_(flag_gpu, non_blocking=True)
         done = torch.cuda.Event()
         done.record(copy)
         torch.cuda.current_stream().wait_event(done)
@@ -1301,8 +1307,9 @@ def run_offload(args, world, rank, local):
         done.synchronize()
         if ls["up"] is not None:
             ls["up"].synchronize()  # the last upload has finished reading param_host
+        clean = Z.ZERO_STEP_CLEAN if int(flag_host[slot][0]) == 0 else 0
         ls["state"] = Z.zero_cpu_step(plan.handle, cfg, ls["state"], hp, acc_host[slot], master, m, v,
-                                      param_host, nthreads=nt["n"])
+                                      param_host, nthreads=nt["n"], flags=clean)
 
     chunks = [(S * i // 8, S * (i + 1) // 8) for i in range(8)]
 
@@ -1402,8 +1409,10 @@ def run_offload(args, world, rank, local):
     torch.set_num_threads(nthr)
     del a, b, c
     # host bytes per element: acc, master, m, v read and master, m, v, param
-    # written (30); DYNAMIC mode and clipping scan the accumulators first (+4)
-    cpu_bpp = 34.0 if wl["mode"] == synth.DYNAMIC else 30.0
+    # written (30); a DYNAMIC step runs in one pass when the GPU's overflow flag
+    # said clean (the serialized zero_cpu_step here), else it scans the
+    # accumulators first (+4; the pipelined variant always scans)
+    cpu_bpp = 30.0
     out = {"mode": "offload", "workload": args.workload, "P": P, "R": R, "tokens": args.tokens,
            "host_threads": os.cpu_count(), "gemm_flops_per_step": 2.0 * args.tokens * d * 8192 * n_gemm,
            "ms_serialized": t_ser * 1e3, "ms_delayed_update": t_dpu * 1e3,

@@ -852,12 +852,34 @@ zero_status zero_layer_release(zero_ctx_t* ctx, int64_t layer, void* stream);
  * accumulators are scanned block by block right before each block's update,
  * in one pass (30 bytes per element instead of 34); otherwise every
  * accumulator is scanned first, as zero_cpu_scan does.
- * Errors: ZERO_ERR_INVALID_ARG.
+ * opts->flags may hold ZERO_STEP_CLEAN (no other flag): the caller vouches
+ * that no accumulator element is inf or NaN, for instance because
+ * zero_take_overflow read 0 after the reduce-scatters that wrote them. A
+ * DYNAMIC-mode step without clipping then has no skip to decide first and
+ * runs in one pass too. Should the pass meet an inf or NaN all the same,
+ * the update has been applied: the call returns ZERO_ERR_STATE and leaves
+ * *inout as it was.
+ * Errors: ZERO_ERR_INVALID_ARG, ZERO_ERR_STATE (ZERO_STEP_CLEAN contradicted).
  */
+#define ZERO_STEP_CLEAN 8
 zero_status zero_cpu_step(const zero_plan_t* plan, const zero_loss_scale_config* cfg,
                           zero_loss_scale_state* inout, const zero_adamw* hp, const zero_step_opts* opts,
                           const float* const* acc, float* const* master, float* const* m, float* const* v,
                           void* const* param, int32_t nthreads);
+
+/*
+ * zero_take_overflow -- the overflow flag that this context's reduce-scatters
+ * OR-ed since the last step (1 if some value they wrote is inf or NaN, else
+ * 0) into *flag, and the flag cleared: for a step taken outside the GPU,
+ * such as zero_cpu_step of ZeRO-Offload, which can then skip its scan
+ * (ZERO_STEP_CLEAN). A GPU step consumes and clears the flag by itself.
+ * Asynchronous on `stream`, after the reduce-scatters queued there.
+ * Defines: [legal] "Dynamic Loss Scaling" (the overflow decides the skip)
+ * and [legal] "CPU Offload" (the optimizer step runs on the CPU).
+ * flag: device memory, one int32, caller-owned, 4-byte aligned.
+ * Errors: ZERO_ERR_INVALID_ARG, ZERO_ERR_ALIGN, ZERO_ERR_CUDA.
+ */
+zero_status zero_take_overflow(zero_ctx_t* ctx, int32_t* flag, void* stream);
 
 /*
  * zero_debug_bounds -- what the bounds-checking debug build recorded. That

@@ -35,7 +35,7 @@ class Offload:
         self.cfg = dict(mode=mode, growth_interval=interval)
         self.ls = dict(scale=scale if mode else 1.0, cur=0, good=0, t=0)
 
-    def step(self, n_micro=1, divisor=1.0, clip=0.0, inject=None, nthreads=0):
+    def step(self, n_micro=1, divisor=1.0, clip=0.0, inject=None, nthreads=0, flags=0):
         P, S = self.lay.P, self.lay.S
         g = O.float_to_half(
             (self.rng.normal(0, 1e-2, (n_micro, self.R, P)) * self.fsm.scale).astype(np.float32),
@@ -51,7 +51,7 @@ class Offload:
         for r in range(self.R):
             self.acc[r][:] = flat[r * S:(r + 1) * S]
         self.ls = Z.zero_cpu_step(self.plan.handle, self.cfg, self.ls, HP, self.acc, self.master,
-                                  self.m, self.v, self.param, divisor, clip, nthreads)
+                                  self.m, self.v, self.param, divisor, clip, nthreads, flags)
         O.step_ex(self.ost, g, OHP, self.fsm, divisor, clip)
 
     def compare(self):
@@ -257,3 +257,31 @@ def test_random_configurations_match_oracle():
             o.compare()
 
     check()
+
+
+@pytest.mark.parametrize("R,dtype", [(1, O.FP16), (3, O.BF16), (8, O.FP16)])
+def test_dynamic_step_known_clean_runs_in_one_pass(R, dtype):
+    # ZERO_STEP_CLEAN: the caller knows no accumulator overflowed (the GPU's
+    # flag), so a DYNAMIC step needs no scan first; the result is the oracle's
+    o = Offload([40_000, 17, 9999], R, dtype, 8, O.SCALE_DYNAMIC, interval=2, seed=R + 90)
+    for s in range(4):
+        o.step(divisor=2.0 if s == 2 else 1.0, flags=Z.ZERO_STEP_CLEAN)
+        o.compare()
+    assert o.fsm.t == 4 and o.fsm.scale == 1024.0  # grew twice at interval 2
+
+
+def test_clean_claim_contradicted_is_refused():
+    o = Offload([30_000, 5], 2, O.FP16, 8, O.SCALE_DYNAMIC, seed=95)
+    o.step()
+    before = dict(o.ls)
+    with pytest.raises(Z.ZeroError) as e:
+        o.step(inject=(0, 1, 7), flags=Z.ZERO_STEP_CLEAN)
+    assert e.value.status == Z.ZERO_ERR_STATE
+    assert o.ls == before  # the loss-scale state did not advance
+
+
+def test_cpu_step_rejects_gpu_step_flags():
+    o = Offload([1000], 1, O.BF16, 8, O.SCALE_NONE, seed=96)
+    with pytest.raises(Z.ZeroError) as e:
+        o.step(flags=Z.ZERO_STEP_PUSH_PARAMS)
+    assert e.value.status == Z.ZERO_ERR_INVALID_ARG

@@ -164,3 +164,40 @@ def test_offload_pipeline_matches_oracle(delayed, pipelined, R, dtype, mode):
         o.compare()
     finally:
         o.close()
+
+
+def test_take_overflow_hands_the_flag_to_the_cpu_step():
+    # the reduce-scatters' overflow flag, taken and cleared, lets a DYNAMIC
+    # CPU step run in one pass (ZERO_STEP_CLEAN) when it reads 0; an inf sets
+    # it, and the scan-first step then skips as the oracle does
+    run = OffloadRun([30_000, 13, 4099], 2, O.FP16, O.SCALE_DYNAMIC, interval=2)
+    flag = torch.zeros(1, dtype=torch.int32, device="cuda")
+    try:
+        for step in range(1, 5):
+            run.step_no += 1
+            g = np.stack([u16(synth.flat_grads(run.wl, run.step_no, r, run.fsm.scale, "cpu"))
+                          for r in range(run.R)])
+            if step == 2:
+                g[1, 5] = 0x7C00
+            for r in range(run.R):
+                gp = np.zeros(run.plan.T, np.uint16)
+                gp[run.idx] = g[r]
+                run.grads[r].view(torch.int16).copy_(torch.from_numpy(gp.view(np.int16)))
+            Z.zero_reduce_scatter_bucket(run.ctx, -1, run.grads, run.acc_gpu)
+            Z.zero_take_overflow(run.ctx, flag)
+            for r in range(run.R):
+                run.acc_host[0][r].copy_(run.acc_gpu[r])
+            f = int(flag.item())
+            assert f == (1 if step == 2 else 0), step
+            Z.zero_take_overflow(run.ctx, flag)
+            assert int(flag.item()) == 0  # taken: cleared
+            run.ls = Z.zero_cpu_step(run.plan.handle, run.cfg, run.ls, run.hp, run.acc_host[0], run.master,
+                                     run.m, run.v, run.param_host, flags=0 if f else Z.ZERO_STEP_CLEAN)
+            O.step(run.ost, g, run.ohp, run.fsm)
+            cat = lambda xs: torch.cat(xs).numpy()[run.idx]
+            assert np.array_equal(cat(run.master).view(np.uint32), run.ost.master.view(np.uint32)), step
+            assert np.array_equal(u16(torch.cat(run.param_host))[run.idx], run.ost.param), step
+            assert (run.ls["t"], run.ls["last_skipped"], run.ls["scale"]) == \
+                (run.fsm.t, run.fsm.last_skipped, run.fsm.scale), step
+    finally:
+        Z.zero_ctx_destroy(run.ctx)

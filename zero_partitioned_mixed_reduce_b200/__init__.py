@@ -22,5 +22,6 @@ from ._capi import (  # noqa: F401
     zero_debug_bounds, zero_cpu_scan, zero_cpu_update, zero_cpu_commit, zero_ctx_set_grad_divisor,
     ZERO_RS_NORM, ZERO_STEP_NORM_FROM_RS, zero_reduce_scatter_buckets, zero_trace_start, zero_trace_read,
     zero_trace_stop, TRACE_NAMES, zero_cpu_scan_shard, zero_cpu_decide, zero_cpu_update_shard,
-    zero_ipc_export, zero_ipc_open, zero_ipc_close, zero_ctx_set_param_push, ZERO_STEP_PUSH_PARAMS)
+    zero_ipc_export, zero_ipc_open, zero_ipc_close, zero_ctx_set_param_push, ZERO_STEP_PUSH_PARAMS,
+    zero_take_overflow, ZERO_STEP_CLEAN)
 from .state import Plan, ShardedState  # noqa: F401

@@ -26,6 +26,7 @@ ZERO_RS_NORM = 2
 ZERO_STEP_ADD_ACC = 1
 ZERO_STEP_NORM_FROM_RS = 2
 ZERO_STEP_PUSH_PARAMS = 4
+ZERO_STEP_CLEAN = 8
 ZERO_TRACE_REDUCE_SCATTER, ZERO_TRACE_STEP, ZERO_TRACE_GATHER, ZERO_TRACE_NORM, ZERO_TRACE_COMMIT = 1, 2, 3, 4, 5
 TRACE_NAMES = {0: "untimed", 1: "reduce_scatter", 2: "step", 3: "gather", 4: "norm", 5: "commit"}
 
@@ -132,6 +133,7 @@ _sig("zero_ctx_destroy", _S, [_P])
 _sig("zero_ctx_reserve_steps", _S, [_P, C.c_int64, C.c_double, C.c_double, _P])
 _sig("zero_ctx_set_grad_divisor", _S, [_P, C.c_double])
 _sig("zero_ctx_set_param_push", _S, [_P, _PP, _PP])
+_sig("zero_take_overflow", _S, [_P, _P, _P])
 _sig("zero_test_drop_tile", _S, [_P, C.c_int64])
 _sig("zero_reduce_scatter_bucket", _S, [_P, C.c_int64, _PP, _PP, _P])
 _sig("zero_step", _S, [_P, C.POINTER(zero_adamw), C.POINTER(zero_state), _PP, _P])
@@ -377,6 +379,12 @@ def zero_ctx_set_grad_divisor(ctx, grad_divisor):
     _check(_lib.zero_ctx_set_grad_divisor(ctx, float(grad_divisor)))
 
 
+def zero_take_overflow(ctx, flag, stream=None):
+    """The reduce-scatters' overflow flag (0/1) into the device int32 `flag`,
+    and the flag cleared (asynchronous on the stream)."""
+    _check(_lib.zero_take_overflow(ctx, _addr(flag), _stream(stream)))
+
+
 def zero_ctx_set_param_push(ctx, full0, full1=None):
     """Register every rank's full-model parameter buffer of state set 0
     (full0) and set 1 (full1) for steps with ZERO_STEP_PUSH_PARAMS; full0 None
@@ -521,12 +529,13 @@ def _cpu_hp(hp):
 
 
 def zero_cpu_step(plan, cfg, state, hp, acc, master, m, v, param, grad_divisor=1.0,
-                  max_grad_norm=0.0, nthreads=0):
+                  max_grad_norm=0.0, nthreads=0, flags=0):
     """The optimizer step on host memory (all buffers host pointers, numpy
     arrays or CPU tensors). cfg / state as for zero_step_noalloc; returns the
-    loss-scale state after the step."""
+    loss-scale state after the step. flags: ZERO_STEP_CLEAN (no accumulator is
+    inf or NaN, as zero_take_overflow reported) lets a DYNAMIC step run in one pass."""
     c, st, hp = _cpu_cfg(cfg), _cpu_state(state), _cpu_hp(hp)
-    opts = zero_step_opts(grad_divisor, max_grad_norm)
+    opts = zero_step_opts(grad_divisor, max_grad_norm, flags)
     arrays = [_ptr_array([_host_addr(x) for x in xs]) for xs in (acc, master, m, v, param)]
     _check(_lib.zero_cpu_step(plan, C.byref(c), C.byref(st), C.byref(hp), C.byref(opts),
                               *[a[0] for a in arrays], nthreads))

@@ -827,6 +827,19 @@ extern "C" zero_status zero_step_shard_ex(zero_ctx_t* ctx, const zero_adamw* hp,
     });
 }
 
+extern "C" zero_status zero_take_overflow(zero_ctx_t* ctx, int32_t* flag, void* stream) {
+    return zb_guarded("zero_take_overflow", [&]() -> zero_status {
+        const char* where = "zero_take_overflow";
+        if (!ctx || !flag) return zb_fail(ZERO_ERR_INVALID_ARG, "zero_take_overflow: NULL ctx or flag");
+        zero_status s = check_device(ctx, where);
+        if (s != ZERO_OK) return s;
+        if (!aligned(flag, 4)) return zb_fail(ZERO_ERR_ALIGN, "zero_take_overflow: flag not 4-byte aligned");
+        cudaError_t e = zb::launch_take_overflow(ctx->st, flag, static_cast<cudaStream_t>(stream));
+        if (e != cudaSuccess) return cuda_fail(where, e);
+        return ZERO_OK;
+    });
+}
+
 extern "C" zero_status zero_ctx_set_param_push(zero_ctx_t* ctx, void* const* full0, void* const* full1) {
     return zb_guarded("zero_ctx_set_param_push", [&]() -> zero_status {
         if (!ctx) return zb_fail(ZERO_ERR_INVALID_ARG, "zero_ctx_set_param_push: ctx is NULL");

@@ -625,19 +625,24 @@ extern "C" zero_status zero_cpu_step(const zero_plan_t* plan, const zero_loss_sc
             return zb_fail(ZERO_ERR_INVALID_ARG, "zero_cpu_step: NULL argument");
         zero_step_opts o{1.0, 0.0, 0, 0};
         if (opts) o = *opts;
-        const bool one_pass = cfg->mode != ZERO_SCALE_DYNAMIC && o.max_grad_norm == 0.0 && o.flags == 0 &&
+        if (o.flags & ~static_cast<int64_t>(ZERO_STEP_CLEAN))
+            return zb_fail(ZERO_ERR_INVALID_ARG, "zero_cpu_step: the only flag is ZERO_STEP_CLEAN");
+        const bool clean = (o.flags & ZERO_STEP_CLEAN) != 0;
+        o.flags = 0;  // the scan and update below take no flags
+        const bool one_pass = (cfg->mode != ZERO_SCALE_DYNAMIC || clean) && o.max_grad_norm == 0.0 &&
                               o.reserved == 0;
         if (!one_pass) {
             // the update depends on the whole scan (a skip, or the clipping
             // coefficient): scan every accumulator first
             zero_cpu_decision d;
-            zero_status st = zero_cpu_scan(plan, cfg, inout, opts, acc, nthreads, &d);
+            zero_status st = zero_cpu_scan(plan, cfg, inout, &o, acc, nthreads, &d);
             if (st == ZERO_OK)
                 st = zero_cpu_update(plan, inout, hp, &d, acc, master, m, v, param, 0, plan->S, nthreads);
             if (st == ZERO_OK) st = zero_cpu_commit(cfg, inout, &d);
             return st;
         }
-        // NONE / STATIC without clipping: one pass (scan and update per block)
+        // NONE / STATIC, or DYNAMIC known clean, without clipping: one pass
+        // (scan and update per block)
         zero_cpu_decision d;
         zero_status st = check_step_args(plan, cfg, inout, hp, o, acc, master, m, v, param);
         if (st != ZERO_OK) return st;
@@ -665,6 +670,10 @@ extern "C" zero_status zero_cpu_step(const zero_plan_t* plan, const zero_loss_sc
             nrm += part[i];
             overflow |= bad[i];
         }
+        if (overflow && clean && cfg->mode == ZERO_SCALE_DYNAMIC)
+            return zb_fail(ZERO_ERR_STATE,
+                           "zero_cpu_step: ZERO_STEP_CLEAN, but an accumulator is inf or NaN; the update was "
+                           "applied and the loss-scale state left as it was");
         d.grad_norm_sq = nrm;
         d.inv = inv;
         d.clip = 1.0f;

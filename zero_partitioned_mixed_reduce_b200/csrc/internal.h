@@ -110,6 +110,8 @@ cudaError_t launch_reduce_scatter(int32_t R, int32_t dtype, int64_t S, int64_t l
 // out[0] (out[1] = 0) (norm_slots.cu).
 cudaError_t launch_sum_norm_slots(const double* slots, int64_t first, int64_t count, double* out,
                                   cudaStream_t s);
+// *out = the reduce-scatters' overflow flag (0/1), which is cleared (norm_slots.cu).
+cudaError_t launch_take_overflow(DevState* st, int32_t* out, cudaStream_t s);
 // The clipping coefficient from norm slots [first, first + count).
 cudaError_t launch_clip_from_rs_norm(const StepParams& sp, const double* slots, int64_t first, int64_t count,
                                      cudaStream_t s);
