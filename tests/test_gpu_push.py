@@ -143,3 +143,20 @@ def test_push_needs_registered_buffers():
         Z.zero_ctx_set_param_push(c.ctx, None)
     finally:
         c.close()
+
+
+def test_push_registration_errors():
+    c = Case([1_000], 2, O.BF16, 8, O.SCALE_NONE, path="inplace", seed=215)
+    try:
+        full = [c.g.half(c.plan.T, c.dtype) for _ in range(c.R)]
+        with pytest.raises(Z.ZeroError) as e:
+            Z.zero_ctx_set_param_push(c.ctx, [full[0], None])
+        assert e.value.status == Z.ZERO_ERR_INVALID_ARG
+        with pytest.raises(Z.ZeroError) as e:
+            Z.zero_ctx_set_param_push(c.ctx, [full[0].data_ptr() + 2, full[1]])
+        assert e.value.status == Z.ZERO_ERR_ALIGN
+        with pytest.raises(Z.ZeroError) as e:  # the push is not a CPU-step flag, nor CLEAN a GPU one
+            Z.zero_step_ex(c.ctx, c.hp, c.handle, c.grads, flags=Z.ZERO_STEP_CLEAN)
+        assert e.value.status == Z.ZERO_ERR_INVALID_ARG
+    finally:
+        c.close()
