@@ -1,5 +1,5 @@
 """Worker for tests/test_gpu_dist.py, launched with torch.distributed.run:
-DistributedZero (one process per GPU, NCCL, symmetric memory) against the
+DistributedZero (one process per GPU, NCCL, CUDA IPC peer mappings) against the
 oracle. Prints "ok" on rank 0 when every step matched."""
 import os
 import sys
@@ -39,6 +39,7 @@ def main():
     hp = wl["hp"]
     ohp = O.AdamW(*(hp[k] for k in ("lr", "beta1", "beta2", "eps", "weight_decay")))
     S = dz.plan.S
+    side = torch.cuda.Stream()
     for step in range(1, 6):
         g = np.stack([u16(synth.flat_grads(wl, step, r, fsm.scale, "cpu")) for r in range(world)])
         if step == 3:
@@ -46,7 +47,17 @@ def main():
         gp = np.zeros(dz.plan.T, np.uint16)
         gp[idx] = g[rank]
         dz.grads.view(torch.int16).copy_(torch.from_numpy(gp.view(np.int16)))
-        dz.step(hp)
+        if step == 2:  # a side stream made current: kernels and collectives follow it
+            side.wait_stream(torch.cuda.current_stream())
+            with torch.cuda.stream(side):
+                dz.step(hp)
+            torch.cuda.current_stream().wait_stream(side)
+        elif step == 4:  # a side stream passed in
+            side.wait_stream(torch.cuda.current_stream())
+            dz.step(hp, stream=side)
+            torch.cuda.current_stream().wait_stream(side)
+        else:
+            dz.step(hp)
         O.step(ost, g, ohp, fsm)
         f = dz.loss_scale()
         assert (f["t"], f["last_skipped"], f["scale"]) == (fsm.t, fsm.last_skipped, fsm.scale), (step, f)

@@ -45,6 +45,10 @@ rank's step also stores its updated parameters into every rank's full-model
 buffer over the same peer mappings (ZERO_STEP_PUSH_PARAMS): the all-gather
 of the parameters leaves with the step's own stores, and after the commit
 full_params() holds the whole updated model on every rank.
+Every method takes an optional stream (a torch.cuda.Stream or a raw
+handle; default the current stream). Its kernels and its collectives run in
+that stream's order: the collectives are issued with it as the current
+stream, so a launch never overtakes the all-reduce that orders it.
 Argument marshalling only; the arithmetic runs in libzero_b200.so. The
 loads from peer memory are plain loads or bulk copies without multicast.
 """
@@ -53,6 +57,16 @@ import torch.distributed as dist
 
 from . import _capi as Z
 from .state import HALF, Plan
+
+
+def _resolve(stream):
+    """The torch stream a call runs on: the given one (a raw handle is
+    wrapped), else the current stream."""
+    if stream is None:
+        return torch.cuda.current_stream()
+    if isinstance(stream, int):
+        return torch.cuda.ExternalStream(stream)
+    return stream
 
 
 class DistributedZero:
@@ -140,6 +154,7 @@ class DistributedZero:
         dist.barrier(self.group)
 
     def _global_norm(self, grads, acc, divisor, stream):
+        # stream is the current stream here (the callers' context)
         Z.zero_grad_norm_shard(self.ctx, grads, acc, self.rank, self.rank + 1, self.norm, divisor,
                                stream)
         dist.all_reduce(self.norm, group=self.group)
@@ -151,19 +166,21 @@ class DistributedZero:
         one: it is added to the accumulator inside the fused step
         (ZERO_STEP_ADD_ACC), or, with clipping, reduce-scattered first.
         grad_divisor defaults to the number of micro-batches."""
+        stream = _resolve(stream)
         if self.micro > 0 and max_grad_norm > 0:
             self.reduce_scatter(stream)
             self.step_accumulated(hp, grad_divisor, max_grad_norm, stream)
             return
         k = float(self.micro + 1) if grad_divisor is None else grad_divisor
         flags = (Z.ZERO_STEP_ADD_ACC if self.micro > 0 else 0) | self._push_flag()
-        dist.all_reduce(self.token, group=self.group)
-        if max_grad_norm > 0:
-            self._global_norm(self.grad_ptrs, None, k, stream)
-        Z.zero_step_shard_ex(self.ctx, hp, self.handle, self.grad_ptrs, self.rank, self.rank + 1,
-                             self.partial, k, max_grad_norm, self.norm, stream, flags=flags)
-        dist.all_reduce(self.partial, group=self.group)
-        Z.zero_step_commit(self.ctx, self.partial, stream)
+        with torch.cuda.stream(stream):
+            dist.all_reduce(self.token, group=self.group)
+            if max_grad_norm > 0:
+                self._global_norm(self.grad_ptrs, None, k, stream)
+            Z.zero_step_shard_ex(self.ctx, hp, self.handle, self.grad_ptrs, self.rank, self.rank + 1,
+                                 self.partial, k, max_grad_norm, self.norm, stream, flags=flags)
+            dist.all_reduce(self.partial, group=self.group)
+            Z.zero_step_commit(self.ctx, self.partial, stream)
         self.micro = 0
 
     def _push_flag(self):
@@ -187,10 +204,12 @@ class DistributedZero:
         this rank's shard of the reduced gradients to its accumulator (the
         first micro-batch of a step overwrites it)."""
         assert self.acc is not None, "construct with accumulate=True"
-        dist.all_reduce(self.token, group=self.group)  # every replica is written
-        Z.zero_reduce_scatter_shard(self.ctx, -1, self.grad_ptrs, self.acc_list, self.rank, self.rank + 1,
-                                    self._rs_flags(), stream)
-        dist.all_reduce(self.token, group=self.group)  # every peer has read this rank's replica
+        stream = _resolve(stream)
+        with torch.cuda.stream(stream):
+            dist.all_reduce(self.token, group=self.group)  # every replica is written
+            Z.zero_reduce_scatter_shard(self.ctx, -1, self.grad_ptrs, self.acc_list, self.rank, self.rank + 1,
+                                        self._rs_flags(), stream)
+            dist.all_reduce(self.token, group=self.group)  # every peer has read this rank's replica
         self.micro += 1
 
     def grads_ready(self, first, count=1):
@@ -249,25 +268,27 @@ class DistributedZero:
         to their count (the mean)."""
         assert self.micro > 0, "no micro-batch was reduce-scattered"
         k = float(self.micro) if grad_divisor is None else grad_divisor
-        if max_grad_norm > 0 and self.norm_divisor is not None and float(self.norm_divisor) == k:
-            # the reduce-scatters' shares: nothing to read again
-            Z.zero_grad_norm_shard(self.ctx, None, None, self.rank, self.rank + 1, self.norm, k, stream)
-            dist.all_reduce(self.norm, group=self.group)
-        elif max_grad_norm > 0:
-            self._global_norm(None, self.acc_list, k, stream)
-        Z.zero_step_shard_ex(self.ctx, hp, self.handle, None, self.rank, self.rank + 1, self.partial, k,
-                             max_grad_norm, self.norm, stream, flags=self._push_flag())
-        dist.all_reduce(self.partial, group=self.group)
-        Z.zero_step_commit(self.ctx, self.partial, stream)
+        stream = _resolve(stream)
+        with torch.cuda.stream(stream):
+            if max_grad_norm > 0 and self.norm_divisor is not None and float(self.norm_divisor) == k:
+                # the reduce-scatters' shares: nothing to read again
+                Z.zero_grad_norm_shard(self.ctx, None, None, self.rank, self.rank + 1, self.norm, k, stream)
+                dist.all_reduce(self.norm, group=self.group)
+            elif max_grad_norm > 0:
+                self._global_norm(None, self.acc_list, k, stream)
+            Z.zero_step_shard_ex(self.ctx, hp, self.handle, None, self.rank, self.rank + 1, self.partial, k,
+                                 max_grad_norm, self.norm, stream, flags=self._push_flag())
+            dist.all_reduce(self.partial, group=self.group)
+            Z.zero_step_commit(self.ctx, self.partial, stream)
         self.micro = 0
 
     def gather_layer(self, layer, out, stream=None):
         """ZeRO-3 all-gather of one layer from every rank's parameter shard."""
-        Z.zero_gather_layer(self.ctx, layer, self.gather_handle, out, stream)
+        Z.zero_gather_layer(self.ctx, layer, self.gather_handle, out, _resolve(stream))
 
     def gather_layers(self, first, outs, stream=None):
         """ZeRO-3 all-gather of consecutive layers first, first+1, ... in one launch."""
-        Z.zero_gather_layers(self.ctx, first, outs, self.gather_handle, stream)
+        Z.zero_gather_layers(self.ctx, first, outs, self.gather_handle, _resolve(stream))
 
     def prefetch_begin(self, bufs, depth, direction=1, stream=None):
         """Start a pass of look-ahead ZeRO-3 gathers into the ring `bufs`
@@ -275,13 +296,13 @@ class DistributedZero:
         then acquire / release each layer in order. The step that produced
         the parameters has been committed on every rank, so their shards
         are final."""
-        Z.zero_prefetch_begin(self.ctx, self.gather_handle, bufs, depth, direction, stream)
+        Z.zero_prefetch_begin(self.ctx, self.gather_handle, bufs, depth, direction, _resolve(stream))
 
     def layer_acquire(self, layer, stream=None):
-        return Z.zero_layer_acquire(self.ctx, layer, stream)
+        return Z.zero_layer_acquire(self.ctx, layer, _resolve(stream))
 
     def layer_release(self, layer, stream=None):
-        Z.zero_layer_release(self.ctx, layer, stream)
+        Z.zero_layer_release(self.ctx, layer, _resolve(stream))
 
     def loss_scale(self):
         return Z.zero_loss_scale(self.ctx)
