@@ -223,7 +223,7 @@ zero_status zero_ctx_reserve_steps(zero_ctx_t* ctx, int64_t steps, double beta1,
 /*
  * zero_test_drop_tile -- test support for the error path of the staged
  * fused step (R <= 2): the next zero_step / zero_step_shard with gradients
- * issues no copy for tile `tile` (tiles are 2048-element pieces of the
+ * issues no copy for tile `tile` (tiles are 4096-element pieces of the
  * shards, numbered shard after shard), so the block that waits for it gives
  * up after its 2 s limit, as it would if a copy never arrived. The step is
  * then abandoned and reported as ZERO_ERR_TIMEOUT (see zero_loss_scale);

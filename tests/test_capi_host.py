@@ -188,12 +188,12 @@ def test_staged_step_tiles_cover_long_shards(R, P):
     # cover every element of every shard; host only, nothing is allocated
     p = Z.Plan([P], None, R, 0, 8, 0)
     tile, tps, total = Z.zero_plan_step_tiles(p.handle)
-    assert tile == 2048 and total == R * tps
+    assert tile == 4096 and total == R * tps
     assert (tps - 1) * tile < p.S <= tps * tile
     last = p.S - (tps - 1) * tile
     assert 8 <= last <= tile and last % 8 == 0
     if P == (1 << 32) + 8:
-        assert p.S == (1 << 32) + 8 and tps == (1 << 21) + 1 and last == 8
+        assert p.S == (1 << 32) + 8 and tps == (1 << 20) + 1 and last == 8
 
 
 def test_ipc_argument_errors_without_a_device():

@@ -23,7 +23,7 @@ def tensor_list(seed, big=False):
     sizes = rng.integers(1, 3000, n)
     sizes[0] = int(rng.choice([1, 7, 8, 9]))
     if big:
-        sizes[-1] = 70_001  # many 2048-element block tiles and a ragged tail
+        sizes[-1] = 70_001  # many block passes and staged tiles, and a ragged tail
     return sizes.tolist()
 
 

@@ -24,7 +24,7 @@ namespace zb {
 
 // The staged fused step's tile: each shard is cut into tiles of this many
 // elements (the last tile of a shard shorter), in 64-bit arithmetic.
-constexpr int64_t kStagedTile = 2048;
+constexpr int64_t kStagedTile = 4096;
 inline int64_t staged_tiles_per_shard(int64_t S) { return (S + kStagedTile - 1) / kStagedTile; }
 
 // Device-resident loss-scale / step state. One per context, in the

@@ -267,12 +267,12 @@ __global__ void __launch_bounds__(kThreads)
 // The same fused step with the read streams staged through shared memory by
 // the Tensor Memory Accelerator, for small R: the per-element read (2R + 12
 // bytes) then leaves too few bytes in flight per thread on the register
-// path. A block is 8 consumer warps and one producer warp. The producer's
-// elected lane issues, per 2048-element shard-local tile, 1-D bulk copies
-// (cp.async.bulk, no multicast) of the R gradient segments and the
-// master/m/v segments into a 2-stage shared-memory ring; each stage has a
-// "full" mbarrier (completed by the copies' transaction bytes) and an
-// "empty" mbarrier (completed when all 256 consumer threads have read the
+// path. A block is 16 consumer warps and one producer warp, one block per
+// SM. The producer's elected lane issues, per 4096-element shard-local tile,
+// 1-D bulk copies (cp.async.bulk, no multicast) of the R gradient segments
+// and the master/m/v segments into a 2-stage shared-memory ring; each stage
+// has a "full" mbarrier (completed by the copies' transaction bytes) and an
+// "empty" mbarrier (completed when all 512 consumer threads have read the
 // stage into registers). Consumers release a stage before doing the
 // arithmetic, so the next tile's copies overlap the current tile's math and
 // no block-wide barrier sits in the loop. Tile indices, shard offsets and
@@ -283,16 +283,20 @@ __global__ void __launch_bounds__(kThreads)
 // finishes; the last block then abandons the step.
 // ---------------------------------------------------------------------------
 
-constexpr int kTmaTile = kThreads * 8;
+constexpr int kTmaTile = 4096;
 static_assert(kTmaTile == kStagedTile, "the host tiling and the kernel's tile agree");
 constexpr int kTmaStages = 2;
-constexpr int kTmaThreads = kThreads + 32;  // consumers + one producer warp
+constexpr int kTmaConsumers = kTmaTile / 8;        // 8 elements per consumer thread
+constexpr int kTmaThreads = kTmaConsumers + 32;    // consumers + one producer warp
 constexpr int kTmaWarps = kTmaThreads / 32;
 constexpr int kErrTimeout = 2;
-// Two resident blocks per SM measured faster than three (R = 2 at 1.37 G
-// elements per shard: 6024 against 5926 GB/s, same process): the grid is
-// capped there.
-constexpr int kTmaBlocksPerSm = 2;
+// One block per SM: the ring takes 2 x (R x 8 KB + 48 KB) of shared memory.
+// At R = 2 and 1.37 G elements per shard, measured in the benchmark step:
+// 4096-element tiles at one block per SM ran 2-3 % faster than 2048-element
+// tiles at two blocks of 288 threads per SM; 5120- and 6144-element tiles,
+// a third stage, and 1024-element tiles with 3-4 stages at 3-4 blocks per SM
+// were all slower.
+constexpr int kTmaBlocksPerSm = 1;
 
 template <int RC>
 struct TmaStage {
@@ -366,16 +370,16 @@ __global__ void __launch_bounds__(kTmaThreads, kTmaBlocksPerSm)
     if (threadIdx.x == 0) {
         for (int s = 0; s < kTmaStages; ++s) {
             mbar_init(smem_u32(&full[s]), 1);
-            mbar_init(smem_u32(&empty[s]), kThreads);
+            mbar_init(smem_u32(&empty[s]), kTmaConsumers);
         }
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
     __syncthreads();
     double nrm = 0.0;
     bool bad = false;
-    if (threadIdx.x >= kThreads) {
+    if (threadIdx.x >= kTmaConsumers) {
         // producer warp: one lane issues every copy
-        if (threadIdx.x == kThreads) {
+        if (threadIdx.x == kTmaConsumers) {
             uint64_t k = 0, dropped = ~0ull;
             for (; k < count; ++k) {
                 const int s = static_cast<int>(k % kTmaStages);
