@@ -279,6 +279,27 @@ def workload_label(name, wl, tensor_range=None):
             f"loss scale mode {wl['mode']}")
 
 
+def job_config(args, world, wl, R, T, S, n_layers, sharded):
+    """The workload a command line measures, as every arm of that command
+    line reports it in `config` (the GPU arms take T, S and the layer count
+    from the library's plan, the reference arm from the oracle's layout; they
+    agree bit for bit). How an arm runs it goes elsewhere in its line.
+    sharded: the DistributedZero job (one shard per rank), else one GPU or
+    independent replicas."""
+    label = workload_label(args.workload, wl, args.tensor_range)
+    if sharded:
+        label = label.split(", R=")[0] + f", sharded over {world} rank(s), one per GPU"
+        par = f"dp{world}: {world} GPU(s), one shard each"
+        moved, per = (2 * R + 26) * S, "per rank"
+    else:
+        par = "1 GPU" if world == 1 else f"{world} independent replicas (--replicas)"
+        moved, per = (2 * R + 26) * T, "per GPU"
+    return {"workload": label, "R": R, "P": sum(wl["numels"]), "T": T, "S": S, "n_layers": n_layers,
+            "l2": f"inputs larger than L2: every step reads and writes at least (2R + 26) x "
+                  f"{'S' if sharded else 'T'} = {moved / 1e9:.1f} GB {per} (L2 126 MB)",
+            "parallelism": par}
+
+
 def bucket_runs(buckets, group):
     """Consecutive buckets, as (first, count), in launches of up to `group`
     elements (a larger bucket alone); group 0: one launch per bucket.
@@ -581,9 +602,8 @@ def run_ours(args, world, rank, local):
         "data": "synthetic",
         "hbm_gbs": step_bytes * K * world / (ms * 1e-3) / 1e9,
         "hbm_frac_of_peak": step_bytes * K / (ms * 1e-3) / 1e9 / peak,
-        "config": {
-            "workload": workload_label(args.workload, b.wl, args.tensor_range),
-            "R": b.R, "P": b.P, "T": b.T, "S": b.S, "n_layers": len(b.plan.layers),
+        "config": job_config(args, world, b.wl, b.R, b.T, b.S, len(b.plan.layers), False),
+        "step": {
             "path": {"pingpong": f"{'global-norm clip pass, ' if b.clip > 0 else ''}"
                                  f"{f'{b.accum - 1} micro-batch(es) reduce-scattered, last ' if b.accum > 1 else ''}"
                                  "fused reduce-scatter+AdamW, ping-pong state",
@@ -602,8 +622,6 @@ def run_ours(args, world, rank, local):
                        f"(<= {args.gather_bucket} elements each)" if b.gather_buckets
                        else f"{len(b.plan.layers)} per-layer launches"),
             "bytes_per_step": step_bytes,
-            "l2": f"inputs larger than L2 ({step_bytes / 1e9:.1f} GB touched per step, L2 126 MB)",
-            "parallelism": "1 GPU" if world == 1 else f"{world} independent replicas (--replicas)",
             "launch": "CUDA graph replay (step graph, event, gather graph), captured through the C ABI"
                       if args.graph else "eager launches through the C ABI",
         },
@@ -711,13 +729,14 @@ def e2e(b, args, stream, world):
 
 # ---- the CPU oracle as a baseline ----------------------------------------------
 
-def oracle_inputs(name, n):
+def oracle_inputs(name, n, R=None):
     """The oracle's state, replicas, hyper-parameters and loss-scale state
-    for the first n params of the workload."""
+    for the first n params of the workload (R replicas: the workload's own
+    count unless given)."""
     import oracle as O
     import synth
     wl = synth.workload(name)
-    R, dtype = wl["R"], wl["dtype"]
+    R, dtype = R or wl["R"], wl["dtype"]
     scale = wl["init_scale"] if wl["mode"] != synth.NONE else 1.0
     numels, left = [], n
     for k in wl["numels"]:
@@ -752,13 +771,13 @@ def oracle_sample(name, target_s=10.0, max_elems=1 << 26):
     return n / dt, n, dt, (st, g, hp, fsm)
 
 
-def _oracle_crew_worker(name, n, barrier, conn):
+def _oracle_crew_worker(name, n, R, barrier, conn):
     """One single-threaded oracle process of OracleCrew: builds its sample,
     then on each request runs k steps between a common barrier and reports
     its start and end time (CLOCK_MONOTONIC, comparable across processes)."""
     import oracle as O
     torch.set_num_threads(1)
-    st, g, hp, fsm = oracle_inputs(name, n)
+    st, g, hp, fsm = oracle_inputs(name, n, R)
     conn.send("ready")
     while True:
         k = conn.recv()
@@ -776,7 +795,7 @@ class OracleCrew:
     hardware thread, each stepping its own copy of the same prefix sample.
     Throughput = processes x sample x steps / (last end - first start)."""
 
-    def __init__(self, name, n, procs=None):
+    def __init__(self, name, n, procs=None, R=None):
         import multiprocessing as mp
         ctx = mp.get_context("spawn")  # never fork a process that holds CUDA
         self.n, self.procs = n, procs or (os.cpu_count() or 1)
@@ -787,7 +806,7 @@ class OracleCrew:
         try:
             for _ in range(self.procs):
                 a, b = ctx.Pipe()
-                p = ctx.Process(target=_oracle_crew_worker, args=(name, n, self.barrier, b), daemon=True)
+                p = ctx.Process(target=_oracle_crew_worker, args=(name, n, R, self.barrier, b), daemon=True)
                 p.start()
                 self.conns.append(a)
                 self.ps.append(p)
@@ -1167,22 +1186,18 @@ def run_dist(args, world, rank, local):
         "metric": METRIC, "value": units / (ms * 1e-3), "unit": "params/s",
         "n_gpus": N, "steps": K, "warmup": args.warmup, "ms_per_step": ms / K, "higher_is_better": True,
         "scaling": "strong", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
-        "config": {"workload": workload_label(args.workload, wl, args.tensor_range).split(", R=")[0]
-                               + f", sharded over {N} rank(s), one per GPU",
-                   "R": N, "P": plan.P, "T": T, "S": S, "n_layers": len(plan.layers),
-                   "path": "DistributedZero: 4-byte NCCL all-reduce (every replica written), fused "
+        "config": job_config(args, N, wl, N, T, S, len(plan.layers), True),
+        "step": {"path": "DistributedZero: 4-byte NCCL all-reduce (every replica written), fused "
                            "reduce-scatter+AdamW over the rank's shard reading the peers' replicas over "
                            "NVLink (plain or 1-D bulk loads, no multicast)"
                            + (", the updated parameters pushed into every rank's full-model buffer by the "
                               "same kernel (ZeRO-1/2)" if args.zero2 else "")
                            + ", 16-byte NCCL all-reduce of {norm, overflow}, loss-scale commit"
                            + ("" if args.zero2 else ", ZeRO-3 gather of every layer from every rank's shard"),
-                   "l2": f"inputs larger than L2 ({(nb['step_hbm'] + nb['gather_hbm']) / 1e9:.1f} GB "
-                         "of HBM per rank per step, L2 126 MB)",
-                   "parallelism": f"dp{N}: {N} GPU(s), one shard each",
-                   "gather": ("none: the step pushes the parameters (ZeRO-1/2)" if args.zero2 else
+                 "bytes_per_rank_per_step": nb["step_hbm"] + nb["gather_hbm"],
+                 "gather": ("none: the step pushes the parameters (ZeRO-1/2)" if args.zero2 else
                               f"{len(buckets)} bucketed launches per step over every rank's shard"),
-                   "launch": "eager (the step issues NCCL all-reduces between its launches)"},
+                 "launch": "eager (the step issues NCCL all-reduces between its launches)"},
         "roofline": roof,
         "gather": None if args.zero2 else {
             "avg_ms_per_step": gather_ms, "elements": plan.L, "launches_per_step": len(buckets),
@@ -1436,26 +1451,36 @@ def run_reference(args, world, rank):
     """The oracle on host cores: each step a bounded prefix sample."""
     if rank != 0:
         return
+    import oracle as O
+    import synth
+    # the same `config` as the GPU arm of this command line: the sharded job
+    # over the ranks, else the workload's own simulated ranks
+    sharded = args.dist or (world > 1 and not args.replicas)
+    wl = synth.workload(args.workload)
+    restrict(wl, args.tensor_range)
+    R = world if sharded else wl["R"]
+    lay = O.Layout(wl["numels"], R, 8, 0, wl["layer_ids"])
+    config = job_config(args, world, wl, R, lay.T, lay.S, len(lay.layers), sharded)
     # every host core runs the oracle on its own copy of a 1M-param prefix
+    # (all R replicas)
     n = 1 << 20
-    crew = OracleCrew(args.workload, n)
+    crew = OracleCrew(args.workload, n, R=R)
     try:
         crew.run(args.warmup)
         value, sec = crew.run(args.steps)
     finally:
         crew.close()
-    import synth
-    wl = synth.workload(args.workload)
     out = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "params/s",
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
-        "ms_per_step": sec * 1e3 / args.steps, "higher_is_better": True, "scaling": "weak",
+        "ms_per_step": sec * 1e3 / args.steps, "higher_is_better": True,
+        "scaling": "strong" if sharded else "weak",
         "vs_baseline": None, "dtype": "f32", "data": "synthetic",
-        "config": {"workload": workload_label(args.workload, wl), "R": wl["R"],
-                   "P": sum(wl["numels"]), "sample_params_per_step": n * crew.procs},
+        "config": config,
         "cpu_baseline": {"value": value, "unit": "params/s", "cores": crew.procs, "kind": "oracle",
                          "sample": f"each step, in each of {crew.procs} single-threaded processes, "
-                                   f"the first {n} params of {args.workload}"},
+                                   f"the first {n} params of {args.workload} ({R} replicas); "
+                                   f"{n * crew.procs} params per step"},
         "e2e": {"value": value, "unit": "params/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }

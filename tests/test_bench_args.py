@@ -95,3 +95,26 @@ def test_dist_bytes_with_the_parameter_push():
     assert nb["step_hbm"] == (2 * N + 26) * S + 2 * T
     assert nb["nvlink_step"] == 4 * (N - 1) * S
     assert bench.parse_args(["--zero2"]).zero2 and not bench.parse_args([]).zero2
+
+
+def test_reference_arm_reports_the_gpu_arms_config():
+    # one GPU: the reference arm's `config` (from the oracle's layout) equals
+    # the one the GPU arm builds from the library's plan
+    import json
+    import os
+    import subprocess
+    import sys
+    import synth
+    import zero_partitioned_mixed_reduce_b200 as Z
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    env = dict(os.environ, CUDA_VISIBLE_DEVICES="")
+    r = subprocess.run([sys.executable, os.path.join(root, "bench.py"), "--impl", "reference", "--workload", "tiny",
+                        "--steps", "1", "--warmup", "0"], capture_output=True, text=True, timeout=600, env=env,
+                       cwd=root)
+    assert r.returncode == 0, r.stderr[-2000:]
+    out = json.loads([ln for ln in r.stdout.splitlines() if ln.startswith("{")][-1])
+    args = bench.parse_args(["--workload", "tiny"])
+    wl = synth.workload("tiny")
+    plan = Z.Plan(wl["numels"], wl["layer_ids"], wl["R"], wl["dtype"], 8, wl["bucket_elems"])
+    assert out["config"] == bench.job_config(args, 1, wl, wl["R"], plan.T, plan.S, len(plan.layers), False)
+    assert out["config"]["parallelism"] == "1 GPU" and out["scaling"] == "weak"

@@ -71,3 +71,13 @@ def test_reference_arm_under_torchrun_two_ranks():
     out = json.loads(lines[0])
     assert out["impl"] == "reference" and out["n_gpus"] == 2 and out["value"] > 0
     assert out["e2e"]["h2d_bytes_per_step"] == 0 and out["cpu_baseline"]["kind"] == "oracle"
+    # the same `config` as the GPU arm of the same command line: the sharded
+    # job over two ranks, its layout from the library's plan
+    import bench
+    import synth
+    import zero_partitioned_mixed_reduce_b200 as Z
+    args = bench.parse_args(["--gpus", "2"])
+    wl = synth.workload(args.workload)
+    plan = Z.Plan(wl["numels"], wl["layer_ids"], 2, wl["dtype"], 8, 0)
+    assert out["config"] == bench.job_config(args, 2, wl, 2, plan.T, plan.S, len(plan.layers), True)
+    assert out["config"]["parallelism"].startswith("dp2") and out["scaling"] == "strong"

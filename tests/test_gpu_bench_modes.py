@@ -20,7 +20,7 @@ def test_two_pass_clip_bench(clip_norm, accum):
     r = subprocess.run(cmd, capture_output=True, text=True, cwd=ROOT)
     assert r.returncode == 0, (r.stdout[-3000:], r.stderr[-3000:])
     out = json.loads([ln for ln in r.stdout.splitlines() if ln.startswith("{")][-1])
-    path = out["config"]["path"]
+    path = out["step"]["path"]
     if clip_norm == "rs":
         assert "norm shares" in path
     else:

@@ -59,5 +59,5 @@ def test_bench_distributed_zero2_mode():
     r = subprocess.run(cmd, capture_output=True, text=True, env=env, cwd=ROOT)
     assert r.returncode == 0, (r.stdout[-3000:], r.stderr[-3000:])
     out = json.loads([ln for ln in r.stdout.splitlines() if ln.startswith("{")][-1])
-    assert out["gather"] is None and out["state_check"] == "ok" and "pushed" in out["config"]["path"]
+    assert out["gather"] is None and out["state_check"] == "ok" and "pushed" in out["step"]["path"]
     assert out["per_rank_bytes"]["gather_hbm"] == 0 and out["value"] > 0
