@@ -477,7 +477,8 @@ __global__ void __launch_bounds__(kTmaThreads, kTmaBlocksPerSm)
 // reduce-scatter kernel. In place on set cur, or from set cur into set 1-cur
 // when both sets are given (ping-pong); skipped (no state written) in
 // DYNAMIC mode when the reduce-scatter raised the overflow flag. The norm is
-// always formed from the accumulators.
+// always formed from the accumulators. This register kernel runs the push
+// variant; without the push the staged kernel below runs.
 // ---------------------------------------------------------------------------
 
 struct AccArgs {
@@ -546,6 +547,142 @@ __global__ void __launch_bounds__(kThreads) step_from_acc_kernel(const __grid_co
         }
     }
     step_epilogue(sp, nrm, false);
+}
+
+// ---------------------------------------------------------------------------
+// The two-pass step from the fp32 accumulators, staged like the fused step
+// at R <= 2: whatever R, it reads one fp32 accumulator and master/m/v (16
+// bytes) and writes 14, the R = 2 fused step's mix, where staging wins. Per
+// 4096-element shard-local tile the producer warp's elected lane bulk-copies
+// the accumulator segment and, unless the step is skipped, the master/m/v
+// segments into the 2-stage ring; 16 consumer warps release a stage once read
+// and then do the arithmetic. A skipped step (DYNAMIC, the reduce-scatter
+// raised the overflow flag) loads only the accumulators and forms the norm.
+// Same bounded waits as the fused staged kernel. The push variant runs on the
+// register kernel above.
+// ---------------------------------------------------------------------------
+
+struct TmaAccStage {
+    static constexpr int kBytes = 4 * kTmaTile * 4;  // acc, master, m, v
+    static constexpr int kSmem = kTmaStages * kBytes;
+};
+
+template <typename H, bool CLIP>
+__global__ void __launch_bounds__(kTmaThreads, kTmaBlocksPerSm)
+    step_from_acc_tma_kernel(const __grid_constant__ AccArgs a, uint64_t tiles_per_shard) {
+    using L = TmaAccStage;
+    extern __shared__ __align__(128) unsigned char smem[];
+    __shared__ __align__(8) uint64_t full[kTmaStages], empty[kTmaStages];
+    const StepParams& sp = a.sp;
+    __shared__ Prologue pro;
+    read_prologue(sp, sp.R, &pro, sp.partial_out == nullptr);
+    const Coef c = pro.c;
+    const int src = pro.src, dst = pro.dst;
+    const bool skip = pro.skip != 0;
+    const uint64_t S = static_cast<uint64_t>(sp.S8) * 8;
+    const uint64_t tps = tiles_per_shard;
+    const uint64_t t0 = static_cast<uint64_t>(sp.obeg) * tps, t1 = static_cast<uint64_t>(sp.oend) * tps;
+    const uint64_t G = gridDim.x, first = t0 + blockIdx.x;
+    const uint64_t count = first < t1 ? (t1 - first + G - 1) / G : 0;
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kTmaStages; ++s) {
+            mbar_init(smem_u32(&full[s]), 1);
+            mbar_init(smem_u32(&empty[s]), kTmaConsumers);
+        }
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    __syncthreads();
+    double nrm = 0.0;
+    if (threadIdx.x >= kTmaConsumers) {
+        if (threadIdx.x == kTmaConsumers) {
+            uint64_t k = 0, dropped = ~0ull;
+            for (; k < count; ++k) {
+                const int s = static_cast<int>(k % kTmaStages);
+                if (k >= kTmaStages &&
+                    !mbar_wait(smem_u32(&empty[s]), static_cast<uint32_t>((k / kTmaStages - 1) & 1))) {
+                    sp.st->err = kErrTimeout;
+                    break;
+                }
+                const uint64_t tile = first + k * G;
+                const uint64_t o = tile / tps;
+                const uint64_t j0 = (tile - o * tps) * kTmaTile;
+                const uint32_t len = static_cast<uint32_t>(S - j0 < kTmaTile ? S - j0 : kTmaTile);
+                if (!ZB_IN(o >= static_cast<uint64_t>(sp.obeg) && o < static_cast<uint64_t>(sp.oend) && j0 < S &&
+                               len % 8 == 0 && j0 + len <= S && a.acc[o] &&
+                               (skip || (a.master[src][o] && a.m[src][o] && a.v[src][o])),
+                           14, tile)) {
+                    dropped = k;
+                    continue;
+                }
+                unsigned char* base = smem + s * L::kBytes;
+                const uint32_t bar = smem_u32(&full[s]);
+                asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+                mbar_expect_tx(bar, len * (skip ? 4 : 16));
+                bulk_g2s(smem_u32(base), a.acc[o] + j0, len * 4, bar);
+                if (!skip) {
+                    bulk_g2s(smem_u32(base + kTmaTile * 4), a.master[src][o] + j0, len * 4, bar);
+                    bulk_g2s(smem_u32(base + 2 * kTmaTile * 4), a.m[src][o] + j0, len * 4, bar);
+                    bulk_g2s(smem_u32(base + 3 * kTmaTile * 4), a.v[src][o] + j0, len * 4, bar);
+                }
+            }
+            for (uint64_t q = k > kTmaStages ? k - kTmaStages : 0; q < k; ++q)
+                if (q != dropped)
+                    mbar_wait(smem_u32(&full[q % kTmaStages]), static_cast<uint32_t>((q / kTmaStages) & 1));
+        }
+    } else {
+        for (uint64_t k = 0; k < count; ++k) {
+            const int s = static_cast<int>(k % kTmaStages);
+            if (!mbar_wait(smem_u32(&full[s]), static_cast<uint32_t>((k / kTmaStages) & 1))) {
+                sp.st->err = kErrTimeout;
+                break;
+            }
+            const uint64_t tile = first + k * G;
+            const uint64_t o = tile / tps;
+            const uint64_t j0 = (tile - o * tps) * kTmaTile;
+            const uint32_t len = static_cast<uint32_t>(S - j0 < kTmaTile ? S - j0 : kTmaTile);
+            const uint32_t e0 = threadIdx.x * 8;
+            const bool act = e0 < len;
+            F8 g, p, m, v;
+            if (act) {
+                const float* ps = reinterpret_cast<const float*>(smem + s * L::kBytes);
+                *reinterpret_cast<uint4*>(&g.x[0]) = lds16(ps + e0);
+                *reinterpret_cast<uint4*>(&g.x[4]) = lds16(ps + e0 + 4);
+                if (!skip) {
+                    *reinterpret_cast<uint4*>(&p.x[0]) = lds16(ps + kTmaTile + e0);
+                    *reinterpret_cast<uint4*>(&p.x[4]) = lds16(ps + kTmaTile + e0 + 4);
+                    *reinterpret_cast<uint4*>(&m.x[0]) = lds16(ps + 2 * kTmaTile + e0);
+                    *reinterpret_cast<uint4*>(&m.x[4]) = lds16(ps + 2 * kTmaTile + e0 + 4);
+                    *reinterpret_cast<uint4*>(&v.x[0]) = lds16(ps + 3 * kTmaTile + e0);
+                    *reinterpret_cast<uint4*>(&v.x[4]) = lds16(ps + 3 * kTmaTile + e0 + 4);
+                }
+            }
+            mbar_arrive(smem_u32(&empty[s]));  // this thread is done with stage s
+            if (!act) continue;
+            if (skip) {
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    const double gd = static_cast<double>(__fmul_rn(g.x[e], c.inv));
+                    nrm = fma(gd, gd, nrm);
+                }
+                continue;
+            }
+            float out[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                const double gd = static_cast<double>(adamw1<CLIP>(c, g.x[e], p.x[e], m.x[e], v.x[e]));
+                nrm = fma(gd, gd, nrm);
+                out[e] = p.x[e];
+            }
+            const uint64_t jj = j0 + e0;
+            if (ZB_IN(jj + 8 <= S && a.master[dst][o] && a.m[dst][o] && a.v[dst][o] && a.param[dst][o], 15, jj)) {
+                st_f8(a.master[dst][o] + jj, p);
+                st_f8(a.m[dst][o] + jj, m);
+                st_f8(a.v[dst][o] + jj, v);
+                st_u4(a.param[dst][o] + (jj >> 3), pack8<H>(out));
+            }
+        }
+    }
+    step_epilogue<kTmaWarps>(sp, nrm, false);
 }
 
 // ---------------------------------------------------------------------------
@@ -1112,9 +1249,24 @@ cudaError_t acc_t(const StepParams& sp, const RankPtrs& p, cudaStream_t s) {
             a.full[k][r] = static_cast<uint4*>(p.full[k][r]);
         }
     }
-    static const int per_sm = blocks_per_sm(step_from_acc_kernel<H, CLIP, PUSH>);
-    const uint32_t grid = grid_for(static_cast<uint64_t>(sp.oend - sp.obeg) * sp.S8, per_sm, sp.grid_cap);
-    step_from_acc_kernel<H, CLIP, PUSH><<<grid, kThreads, 0, s>>>(a);
+    if constexpr (!PUSH) {
+        constexpr int smem = TmaAccStage::kSmem;
+        static const int per_sm = [] {
+            cudaFuncSetAttribute(step_from_acc_tma_kernel<H, CLIP>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 smem);
+            int n = 0;
+            cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, step_from_acc_tma_kernel<H, CLIP>, kTmaThreads, smem);
+            return n > kTmaBlocksPerSm ? kTmaBlocksPerSm : (n > 0 ? n : 1);
+        }();
+        const int64_t tiles_per_shard = staged_tiles_per_shard(static_cast<int64_t>(sp.S8) * 8);
+        const uint64_t tiles = static_cast<uint64_t>(tiles_per_shard) * static_cast<uint64_t>(sp.oend - sp.obeg);
+        const uint32_t grid = grid_for(tiles * kThreads, per_sm, sp.grid_cap);
+        step_from_acc_tma_kernel<H, CLIP><<<grid, kTmaThreads, smem, s>>>(a, static_cast<uint64_t>(tiles_per_shard));
+    } else {
+        static const int per_sm = blocks_per_sm(step_from_acc_kernel<H, CLIP, PUSH>);
+        const uint32_t grid = grid_for(static_cast<uint64_t>(sp.oend - sp.obeg) * sp.S8, per_sm, sp.grid_cap);
+        step_from_acc_kernel<H, CLIP, PUSH><<<grid, kThreads, 0, s>>>(a);
+    }
     return cudaGetLastError();
 }
 
