@@ -159,10 +159,11 @@ zero_status zero_plan_layer(const zero_plan_t* plan, int64_t l, int64_t* lo, int
 zero_status zero_plan_memory(const zero_plan_t* plan, int32_t stage, int64_t* bytes_per_rank);
 
 /*
- * zero_plan_step_tiles -- how the staged fused step (the kernel zero_step
- * runs for R <= 2, whose reads are bulk copies into shared memory) cuts this
- * plan's shards: each shard of S elements into *tiles_per_shard tiles of
- * *tile_elems elements, the last tile of a shard holding the rest,
+ * zero_plan_step_tiles -- how the staged steps (the fused step zero_step
+ * runs for R <= 2, and the step from the accumulators at every R; their reads
+ * are bulk copies into shared memory) cut this plan's shards: each shard
+ * of S elements into *tiles_per_shard tiles of *tile_elems elements, the
+ * last tile of a shard holding the rest,
  * S - (tiles_per_shard - 1) * tile_elems (a multiple of 8, at least 8); the
  * step's work is *tiles_total = R * tiles_per_shard tiles. Host arithmetic
  * in 64 bits, the same the launch uses, so a shard longer than 2^32
