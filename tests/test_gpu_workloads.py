@@ -287,3 +287,14 @@ def test_shard_longer_than_2_to_the_32_staged_step():
     assert p.S == (1 << 32) + 8 and (tps - 1) * tile == 1 << 32
     del p
     run(wl, "inplace", gather=True, extra=np.arange((1 << 32) - 4096, (1 << 32) + 8))
+
+
+def test_shard_longer_than_2_to_the_32_two_pass_step():
+    # the same shard of 2^32 + 8 elements on the two-pass path: one
+    # reduce-scatter into the fp32 accumulator, then the staged step from the
+    # accumulator, whose tiles pass 2^32 like the fused step's (86 GB on the
+    # device); the sample covers the last 4104 elements again
+    n = 1 << 31
+    wl = synth.custom_workload([n, n + 8], 1, 0, synth.NONE, 1.0, 1000, sigma=1e-4, index=32)
+    wl["steps"] = 2
+    run(wl, "twopass", extra=np.arange((1 << 32) - 4096, (1 << 32) + 8))
