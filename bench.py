@@ -138,14 +138,18 @@ def restrict(wl, rng):
 # ---- distributed plumbing ---------------------------------------------------
 
 def dist_init():
+    """One process per GPU: NCCL when there are GPUs, gloo otherwise.
+    ZB_BENCH_BACKEND=gloo keeps gloo with GPUs, so that several ranks can
+    share one GPU in a functional test of the multi-rank path (rank r on GPU
+    r mod the GPU count); such a run measures nothing."""
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
     if world > 1:
         import torch.distributed as dist
-        backend = "nccl" if torch.cuda.is_available() else "gloo"
-        if backend == "nccl":
-            torch.cuda.set_device(local)
+        backend = os.environ.get("ZB_BENCH_BACKEND") or ("nccl" if torch.cuda.is_available() else "gloo")
+        if torch.cuda.is_available():
+            torch.cuda.set_device(local % torch.cuda.device_count())
         dist.init_process_group(backend, timeout=datetime.timedelta(seconds=300))
     elif torch.cuda.is_available():
         torch.cuda.set_device(local)

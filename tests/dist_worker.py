@@ -1,6 +1,7 @@
 """Worker for tests/test_gpu_dist.py, launched with torch.distributed.run:
 DistributedZero (one process per GPU, NCCL, CUDA IPC peer mappings) against the
 oracle. Prints "ok" on rank 0 when every step matched."""
+import datetime
 import os
 import sys
 
@@ -22,8 +23,13 @@ def u16(t):
 
 
 def main():
-    torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", "0")))
-    dist.init_process_group("nccl")
+    # ZB_DIST_BACKEND=gloo runs the ranks as processes sharing this machine's
+    # GPUs (several ranks on one GPU): their buffers are still shared through
+    # CUDA IPC, and the ordering all-reduces go through gloo, which blocks on
+    # the host; no kernel ever waits for another rank's
+    backend = os.environ.get("ZB_DIST_BACKEND", "nccl")
+    torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", "0")) % torch.cuda.device_count())
+    dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
     rank, world = dist.get_rank(), dist.get_world_size()
     numels, layer_ids = [70_001, 13, 4096, 999], [0, 0, 1, 1]
     dz = DistributedZero(numels, layer_ids, Z.ZERO_FP16, Z.ZERO_SCALE_DYNAMIC, 256.0, 3, push_params=True)
