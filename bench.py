@@ -23,7 +23,10 @@ gathers read every rank's parameter shard; the time is the maximum over
 ranks. `--replicas` runs N independent single-GPU copies instead. The step
 and the gathers are captured once into CUDA graphs through the C ABI and
 replayed (`--eager` issues every launch instead). `--impl reference` times
-the CPU oracle on host cores on a bounded sample of the same workload.
+the CPU oracle on host cores on a bounded sample of the same workload, and
+reports the same `config`. ZB_BENCH_BACKEND=gloo runs a multi-rank job with
+several ranks sharing a GPU (a functional test of that path, not a
+measurement).
 """
 import argparse
 import datetime
