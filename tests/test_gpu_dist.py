@@ -31,7 +31,7 @@ def test_distributed_zero_matches_oracle():
     assert "ok" in r.stdout
 
 
-@pytest.mark.parametrize("nproc", [2, 4])
+@pytest.mark.parametrize("nproc", [2, 4, 8])
 def test_ranks_sharing_one_gpu_over_gloo(nproc):
     # the multi-rank path on the GPU this suite has: nproc processes, each
     # mapping the others' gradient buffers, parameter shards and full-model
