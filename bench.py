@@ -1415,6 +1415,33 @@ def run_offload(args, world, rank, local):
     nt["n"] = 0
     t_cpu = med(lambda: [cpu_half(0, done) for _ in range(K)])
     t_up = med(lambda: [upload() for _ in range(K)])
+    # the clipped CPU step alone: the host scans every accumulator for the
+    # norm first (zero_cpu_step with clipping), against the decision from the
+    # norm and flag the GPU took while reducing (ZERO_RS_NORM shares with the
+    # host's loss scale on the device, zero_take_overflow), after which the
+    # update reads each host accumulator once
+    clip = 1.0
+    Z.zero_loss_scale(ctx, Z.ZERO_LOSS_SCALE_SET, ls["state"])
+    Z.zero_reduce_scatter_shard(ctx, -1, grads, acc_gpu, 0, R, Z.ZERO_RS_NORM)
+    norm_dev = torch.zeros(2, dtype=torch.float64, device="cuda")
+    Z.zero_grad_norm_shard(ctx, None, None, 0, R, norm_dev, 1.0)
+    Z.zero_take_overflow(ctx, flag_gpu)
+    for r in range(R):
+        acc_host[0][r].copy_(acc_gpu[r])
+    reduced = (float(norm_dev[0].item()), float(flag_gpu.item()))
+
+    def clip_scan():
+        ls["state"] = Z.zero_cpu_step(plan.handle, cfg, ls["state"], hp, acc_host[0], master, m, v, param_host,
+                                      max_grad_norm=clip)
+
+    def clip_device_norm():
+        st = ls["state"]
+        dec = Z.zero_cpu_decide(plan.handle, cfg, st, reduced, 1.0, clip)
+        Z.zero_cpu_update(plan.handle, st, hp, dec, acc_host[0], master, m, v, param_host, 0, S)
+        ls["state"] = Z.zero_cpu_commit(cfg, st, dec)
+
+    t_clip_scan = med(lambda: [clip_scan() for _ in range(K)])
+    t_clip_dev = med(lambda: [clip_device_norm() for _ in range(K)])
     # the host's streaming rates, measured now on all hardware threads: a copy
     # (1 read + 1 write) and a triad (2 reads + 1 write) over 1 GiB fp32 buffers
     nthr = torch.get_num_threads()
@@ -1450,7 +1477,13 @@ def run_offload(args, world, rank, local):
            "host_copy_GBps": host_copy, "host_triad_GBps": host_triad,
            "cpu_adamw_frac_of_host_stream": cpu_bpp * T / t_cpu / 1e9 / max(host_copy, host_triad),
            "cpu_threads_overlapped": max(1, ncpu - 1),
-           "speedup_from_delayed_update": t_ser / t_dpu, "steps": K,
+           "speedup_from_delayed_update": t_ser / t_dpu,
+           "clipped_cpu_step": {"max_grad_norm": clip, "ms_host_scan_first": t_clip_scan * 1e3,
+                                "ms_norm_from_device": t_clip_dev * 1e3,
+                                "speedup": t_clip_scan / t_clip_dev,
+                                "host_bytes_per_param": {"host_scan_first": cpu_bpp + 4.0,
+                                                         "norm_from_device": cpu_bpp}},
+           "steps": K,
            "timing": "host wall clock around synchronized loops (the CPU step is host work), "
                      "median of 3 loops"}
     Z.zero_ctx_destroy(ctx)

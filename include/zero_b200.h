@@ -957,6 +957,14 @@ zero_status zero_cpu_commit(const zero_loss_scale_config* cfg, zero_loss_scale_s
  * Every rank then applies zero_cpu_commit with the same decision, so every
  * rank's loss-scale state stays the same. The norm's summation grouping
  * differs from one process's by rounding only.
+ * In one process, the totals may come from the GPU that reduced the
+ * gradients: with the context holding the host's loss scale
+ * (zero_loss_scale SET) and the step's divisor (zero_ctx_set_grad_divisor),
+ * ZERO_RS_NORM reduce-scatters leave the squared norm for
+ * zero_grad_norm_shard (NULL grads and acc, every owner) and
+ * zero_take_overflow gives the flag; zero_cpu_decide then decides a clipped
+ * step without a host scan, and zero_cpu_update reads each host accumulator
+ * once.
  * Defines: [legal] "CPU Offload"; [instr] ZeRO-2 "Mechanism" (each process
  * updates its own partition).
  * Errors: ZERO_ERR_INVALID_ARG, ZERO_ERR_RANGE (owner range).

@@ -201,3 +201,55 @@ def test_take_overflow_hands_the_flag_to_the_cpu_step():
                 (run.fsm.t, run.fsm.last_skipped, run.fsm.scale), step
     finally:
         Z.zero_ctx_destroy(run.ctx)
+
+
+@pytest.mark.parametrize("divisor", [1.0, 2.0])
+def test_clipped_offload_step_reads_the_host_accumulators_once(divisor):
+    # with clipping the CPU step needs the global norm before its first
+    # update; the reduce-scatters take it on the device as they write the
+    # accumulators (ZERO_RS_NORM, the context holding the host's loss scale
+    # and the step's divisor), zero_take_overflow hands over the flag, and
+    # zero_cpu_decide turns the two into the decision: zero_cpu_update then
+    # reads every host accumulator once, with no scan first
+    run = OffloadRun([30_000, 13, 4099], 4, O.FP16, O.SCALE_DYNAMIC, interval=2)
+    flag = torch.zeros(1, dtype=torch.int32, device="cuda")
+    part = torch.zeros(2, dtype=torch.float64, device="cuda")
+    acc_list = list(run.acc_gpu)
+    S, R = run.plan.S, run.R
+    clip = 1e-3  # below the gradients' norm: every applied step clips
+    Z.zero_ctx_set_grad_divisor(run.ctx, divisor)
+    try:
+        for step in range(1, 6):
+            run.step_no += 1
+            g = np.stack([u16(synth.flat_grads(run.wl, run.step_no, r, run.fsm.scale, "cpu")) for r in range(R)])
+            if step == 3:
+                g[2, 17] = 0x7C00
+            for r in range(R):
+                gp = np.zeros(run.plan.T, np.uint16)
+                gp[run.idx] = g[r]
+                run.grads[r].view(torch.int16).copy_(torch.from_numpy(gp.view(np.int16)))
+            Z.zero_loss_scale(run.ctx, Z.ZERO_LOSS_SCALE_SET, run.ls)  # the host's scale on the device
+            Z.zero_reduce_scatter_shard(run.ctx, -1, run.grads, acc_list, 0, R, Z.ZERO_RS_NORM)
+            Z.zero_grad_norm_shard(run.ctx, None, None, 0, R, part, divisor)
+            Z.zero_take_overflow(run.ctx, flag)
+            for r in range(R):
+                run.acc_host[0][r].copy_(run.acc_gpu[r])
+            reduced = (float(part[0].item()), float(flag.item()))
+            dec = Z.zero_cpu_decide(run.plan.handle, run.cfg, run.ls, reduced, divisor, clip)
+            Z.zero_cpu_update(run.plan.handle, run.ls, run.hp, dec, run.acc_host[0], run.master, run.m, run.v,
+                              run.param_host, 0, S)
+            run.ls = Z.zero_cpu_commit(run.cfg, run.ls, dec)
+            O.step_ex(run.ost, g[None], run.ohp, run.fsm, divisor, clip)
+            assert bool(dec.skip) == (step == 3)
+            if step != 3:
+                assert dec.clip < 1.0
+                assert abs(dec.grad_norm_sq - run.fsm.grad_norm_sq) <= 1e-9 * run.fsm.grad_norm_sq
+            cat = lambda xs: torch.cat(xs).numpy()[run.idx]
+            for name, a, b in (("master", cat(run.master), run.ost.master), ("m", cat(run.m), run.ost.m),
+                               ("v", cat(run.v), run.ost.v)):
+                assert np.array_equal(a.view(np.uint32), b.view(np.uint32)), (name, step)
+            assert np.array_equal(u16(torch.cat(run.param_host))[run.idx], run.ost.param), step
+            assert (run.ls["t"], run.ls["last_skipped"], run.ls["scale"]) == \
+                (run.fsm.t, run.fsm.last_skipped, run.fsm.scale), step
+    finally:
+        Z.zero_ctx_destroy(run.ctx)
