@@ -1297,6 +1297,13 @@ def run_offload(args, world, rank, local):
     # the accumulators: a clean DYNAMIC step then runs in one pass on the CPU
     flag_gpu = torch.zeros(1, dtype=torch.int32, device="cuda")
     flag_host = [pin(torch.zeros(1, dtype=torch.int32)) for _ in range(2)]
+    # the reduce-scatters also take the squared norm (ZERO_RS_NORM, with the
+    # host's loss scale on the device), copied down with the flag: the split
+    # CPU step (and the clipped one under --clip) decides from the two without
+    # scanning the host accumulators
+    clip_on = args.clip > 0
+    norm_gpu = torch.zeros(2, dtype=torch.float64, device="cuda")
+    norm_host = [pin(torch.zeros(2, dtype=torch.float64)) for _ in range(2)]
     param_gpu = [torch.zeros(S, dtype=half, device="cuda") for _ in range(R)]
     copy = torch.cuda.Stream()
     d = 768 if args.workload == "gpt2s" else 2048
@@ -1310,7 +1317,11 @@ def run_offload(args, world, rank, local):
     def gpu_half(slot):
         for _ in range(n_gemm):
             x @ w
-        Z.zero_reduce_scatter_bucket(ctx, -1, grads, acc_gpu)
+        if ls.get("scale_on_device") != ls["state"]["scale"]:  # the host's loss scale moved
+            Z.zero_loss_scale(ctx, Z.ZERO_LOSS_SCALE_SET, ls["state"])
+            ls["scale_on_device"] = ls["state"]["scale"]
+        Z.zero_reduce_scatter_shard(ctx, -1, grads, acc_gpu, 0, R, Z.ZERO_RS_NORM)
+        Z.zero_grad_norm_shard(ctx, None, None, 0, R, norm_gpu, 1.0)
         Z.zero_take_overflow(ctx, flag_gpu)
         ev = torch.cuda.Event()
         ev.record()
@@ -1319,6 +1330,7 @@ def run_offload(args, world, rank, local):
             for r in range(R):
                 acc_host[slot][r].copy_(acc_gpu[r], non_blocking=True)
             flag_host[slot].copy_(flag_gpu, non_blocking=True)
+            norm_host[slot].copy_(norm_gpu, non_blocking=True)
         done = torch.cuda.Event()
         done.record(copy)
         torch.cuda.current_stream().wait_event(done)
@@ -1333,9 +1345,21 @@ def run_offload(args, world, rank, local):
         done.synchronize()
         if ls["up"] is not None:
             ls["up"].synchronize()  # the last upload has finished reading param_host
+        if clip_on:
+            st = ls["state"]
+            dec = decide(slot, st)
+            Z.zero_cpu_update(plan.handle, st, hp, dec, acc_host[slot], master, m, v, param_host, 0, S,
+                              nthreads=nt["n"])
+            ls["state"] = Z.zero_cpu_commit(cfg, st, dec)
+            return
         clean = Z.ZERO_STEP_CLEAN if int(flag_host[slot][0]) == 0 else 0
         ls["state"] = Z.zero_cpu_step(plan.handle, cfg, ls["state"], hp, acc_host[slot], master, m, v,
                                       param_host, nthreads=nt["n"], flags=clean)
+
+    def decide(slot, st):
+        """The step's decision from the device's norm and flag."""
+        reduced = (float(norm_host[slot][0]), float(flag_host[slot][0]))
+        return Z.zero_cpu_decide(plan.handle, cfg, st, reduced, 1.0, args.clip if clip_on else 0.0)
 
     chunks = [(S * i // 8, S * (i + 1) // 8) for i in range(8)]
 
@@ -1346,7 +1370,7 @@ def run_offload(args, world, rank, local):
         if ls["up"] is not None:
             ls["up"].synchronize()
         st = ls["state"]
-        dec = Z.zero_cpu_scan(plan.handle, cfg, st, acc_host[slot])
+        dec = decide(slot, st)
         for lo, hi in chunks:
             Z.zero_cpu_update(plan.handle, st, hp, dec, acc_host[slot], master, m, v, param_host, lo, hi,
                               nthreads=nt["n"])
@@ -1420,7 +1444,7 @@ def run_offload(args, world, rank, local):
     # norm and flag the GPU took while reducing (ZERO_RS_NORM shares with the
     # host's loss scale on the device, zero_take_overflow), after which the
     # update reads each host accumulator once
-    clip = 1.0
+    clip = args.clip if clip_on else 1.0
     Z.zero_loss_scale(ctx, Z.ZERO_LOSS_SCALE_SET, ls["state"])
     Z.zero_reduce_scatter_shard(ctx, -1, grads, acc_gpu, 0, R, Z.ZERO_RS_NORM)
     norm_dev = torch.zeros(2, dtype=torch.float64, device="cuda")
@@ -1464,9 +1488,11 @@ def run_offload(args, world, rank, local):
     # host bytes per element: acc, master, m, v read and master, m, v, param
     # written (30); a DYNAMIC step runs in one pass when the GPU's overflow flag
     # said clean (the serialized zero_cpu_step here), else it scans the
-    # accumulators first (+4; the pipelined variant always scans)
+    # accumulators first (+4); the split steps (pipelined upload, --clip)
+    # decide from the device's norm and flag and read them once
     cpu_bpp = 30.0
     out = {"mode": "offload", "workload": args.workload, "P": P, "R": R, "tokens": args.tokens,
+           "clip": args.clip if clip_on else None,
            "host_threads": os.cpu_count(), "gemm_flops_per_step": 2.0 * args.tokens * d * 8192 * n_gemm,
            "ms_serialized": t_ser * 1e3, "ms_delayed_update": t_dpu * 1e3,
            "ms_serialized_pipelined_upload": t_ser_pipe * 1e3,
