@@ -34,6 +34,7 @@ def test_bench_line_has_the_contract_keys():
         assert k in roof, k
     assert roof["bound"] == "hbm" and roof["unit"] == "GB/s" and roof["achieved"] > 0
     assert abs(roof["frac"] - roof["achieved"] / roof["peak"]) <= 1e-12
+    assert abs(roof["frac_of_nominal"] - roof["achieved"] / 8000.0) <= 1e-12  # the 8 TB/s spec figure
     assert roof["traffic"] is None  # no stored counters for this workload
     cb = out["cpu_baseline"]
     assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["value"] > 0 and cb["sample"]
